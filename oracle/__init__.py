@@ -1,0 +1,186 @@
+"""fp64 CPU oracle for the selective scan (S6): Python side.
+
+TEST INFRASTRUCTURE ONLY.  Only the tests, ``__graft_entry__.smoke()`` and the
+CPU-baseline / reference leg of ``bench.py`` may import this package.  The
+product path (the ``selective_state_space_mss_b200`` package and its CUDA
+library) never imports it, and it never imports the product path: the two
+share no code.  The only module both sides use is the seeded input generator,
+which holds none of the method's arithmetic.
+
+``mss_oracle.c`` holds the definition of the forward pass and of the decode
+step (citations are in its header); this module builds it with gcc, loads it
+with ctypes and converts numpy arrays.  ``scans.py`` holds the alternative
+scan orders and matrix views used to pin the sequential definition.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import subprocess
+import threading
+
+import numpy as np
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+_SRC = os.path.join(_HERE, "mss_oracle.c")
+_LIB_PATH = os.path.join(_HERE, "liboracle.so")
+_lock = threading.Lock()
+_lib = None
+
+
+def build(force: bool = False) -> str:
+    """Compile ``mss_oracle.c`` into ``liboracle.so`` next to it (gcc, -O2).
+
+    Plain C99 with libm and pthreads; no fast-math, so every operation is an
+    IEEE fp64 operation in program order.
+    """
+    if force or not os.path.exists(_LIB_PATH) or (
+        os.path.getmtime(_LIB_PATH) < os.path.getmtime(_SRC)
+    ):
+        tmp = _LIB_PATH + f".tmp{os.getpid()}"
+        subprocess.check_call(
+            ["gcc", "-std=c99", "-O2", "-fno-fast-math", "-ffp-contract=off",
+             "-Wall", "-Wextra", "-fPIC", "-shared", "-o", tmp, _SRC,
+             "-lm", "-lpthread"]
+        )
+        os.replace(tmp, _LIB_PATH)
+    return _LIB_PATH
+
+
+def _load():
+    global _lib
+    with _lock:
+        if _lib is None:
+            # MSS_ORACLE_LIB points the pins at another build of this same
+            # source (the mutation test plants mistakes in copies of it).
+            path = os.environ.get("MSS_ORACLE_LIB") or build()
+            lib = ctypes.CDLL(path)
+            f, d, i64, i = (ctypes.POINTER(ctypes.c_float), ctypes.POINTER(ctypes.c_double),
+                            ctypes.c_int64, ctypes.c_int)
+            lib.mss_oracle_scan_fwd.argtypes = [f, f, f, f, f, f, f, f, i, d, d,
+                                                i64, i64, i64, i64, i]
+            lib.mss_oracle_scan_fwd.restype = i
+            lib.mss_oracle_state_update.argtypes = [d, f, f, f, f, f, f, f, f, i, d,
+                                                    i64, i64, i64, i]
+            lib.mss_oracle_state_update.restype = i
+            lib.mss_oracle_recurrence.argtypes = [d, d, d, i64, i64, d, d]
+            lib.mss_oracle_recurrence.restype = i
+            lib.mss_oracle_softplus.argtypes = [ctypes.c_double]
+            lib.mss_oracle_softplus.restype = ctypes.c_double
+            lib.mss_oracle_silu.argtypes = [ctypes.c_double]
+            lib.mss_oracle_silu.restype = ctypes.c_double
+            _lib = lib
+    return _lib
+
+
+def default_threads() -> int:
+    return max(1, len(os.sched_getaffinity(0)))
+
+
+def _f32(x, shape=None, name="array"):
+    if x is None:
+        return None, None
+    a = np.ascontiguousarray(np.asarray(x, dtype=np.float32))
+    if shape is not None and a.shape != tuple(shape):
+        raise ValueError(f"{name}: expected shape {tuple(shape)}, got {a.shape}")
+    return a, a.ctypes.data_as(ctypes.POINTER(ctypes.c_float))
+
+
+def _dptr(a):
+    return a.ctypes.data_as(ctypes.POINTER(ctypes.c_double))
+
+
+def softplus(s: float) -> float:
+    """ln(1 + e^s) in fp64."""
+    return _load().mss_oracle_softplus(float(s))
+
+
+def silu(z: float) -> float:
+    """z / (1 + e^-z) in fp64."""
+    return _load().mss_oracle_silu(float(z))
+
+
+def scan_fwd(u, delta, A, B, C, D=None, z=None, delta_bias=None, softplus_flag=True,
+             nthreads=None):
+    """Selective-scan forward pass in fp64.
+
+    u, delta, z: [batch, dim, L]; A: [dim, N]; B, C: [batch, N, L];
+    D, delta_bias: [dim].  Values are taken as fp32 (bf16 inputs must already
+    be widened, which is exact).  Returns (y [batch, dim, L] fp64,
+    last_state [batch, dim, N] fp64).
+    """
+    u_a, u_p = _f32(u, name="u")
+    if u_a.ndim != 3:
+        raise ValueError("u must be [batch, dim, L]")
+    batch, dim, L = u_a.shape
+    A_a, A_p = _f32(A, name="A")
+    if A_a.ndim != 2 or A_a.shape[0] != dim:
+        raise ValueError("A must be [dim, N]")
+    N = A_a.shape[1]
+    d_a, d_p = _f32(delta, (batch, dim, L), "delta")
+    B_a, B_p = _f32(B, (batch, N, L), "B")
+    C_a, C_p = _f32(C, (batch, N, L), "C")
+    D_a, D_p = _f32(D, (dim,), "D")
+    z_a, z_p = _f32(z, (batch, dim, L), "z")
+    b_a, b_p = _f32(delta_bias, (dim,), "delta_bias")
+    y = np.empty((batch, dim, L), dtype=np.float64)
+    last = np.empty((batch, dim, N), dtype=np.float64)
+    rc = _load().mss_oracle_scan_fwd(
+        u_p, d_p, A_p, B_p, C_p, D_p, z_p, b_p, int(bool(softplus_flag)),
+        _dptr(y), _dptr(last), batch, dim, N, L,
+        default_threads() if nthreads is None else int(nthreads))
+    if rc != 0:
+        raise RuntimeError(f"mss_oracle_scan_fwd failed with code {rc}")
+    del u_a, d_a, B_a, C_a, D_a, z_a, b_a, A_a  # keep buffers alive until here
+    return y, last
+
+
+def state_update(state, u, delta, A, B, C, D=None, z=None, delta_bias=None,
+                 softplus_flag=True, nthreads=None):
+    """One decode step in fp64.
+
+    state: [batch, dim, N] (fp64, updated in place and returned);
+    u, delta, z: [batch, dim]; A: [dim, N]; B, C: [batch, N]; D, delta_bias: [dim].
+    Returns (y [batch, dim] fp64, state).
+    """
+    if not (isinstance(state, np.ndarray) and state.dtype == np.float64
+            and state.flags.c_contiguous):
+        raise ValueError("state must be a C-contiguous float64 numpy array")
+    batch, dim, N = state.shape
+    u_a, u_p = _f32(u, (batch, dim), "u")
+    d_a, d_p = _f32(delta, (batch, dim), "delta")
+    A_a, A_p = _f32(A, (dim, N), "A")
+    B_a, B_p = _f32(B, (batch, N), "B")
+    C_a, C_p = _f32(C, (batch, N), "C")
+    D_a, D_p = _f32(D, (dim,), "D")
+    z_a, z_p = _f32(z, (batch, dim), "z")
+    b_a, b_p = _f32(delta_bias, (dim,), "delta_bias")
+    y = np.empty((batch, dim), dtype=np.float64)
+    rc = _load().mss_oracle_state_update(
+        _dptr(state), u_p, d_p, A_p, B_p, C_p, D_p, z_p, b_p, int(bool(softplus_flag)),
+        _dptr(y), batch, dim, N,
+        default_threads() if nthreads is None else int(nthreads))
+    if rc != 0:
+        raise RuntimeError(f"mss_oracle_state_update failed with code {rc}")
+    del u_a, d_a, A_a, B_a, C_a, D_a, z_a, b_a
+    return y, state
+
+
+def recurrence(abar, bbar_x, c):
+    """Discrete recurrence with given coefficients (rows are tokens).
+
+    abar, bbar_x, c: [L, N] fp64.  Returns (h [L, N], y [L]) with h starting at 0.
+    """
+    abar = np.ascontiguousarray(abar, dtype=np.float64)
+    bbar_x = np.ascontiguousarray(bbar_x, dtype=np.float64)
+    c = np.ascontiguousarray(c, dtype=np.float64)
+    L, N = abar.shape
+    if bbar_x.shape != (L, N) or c.shape != (L, N):
+        raise ValueError("abar, bbar_x, c must share the shape [L, N]")
+    h = np.empty((L, N), dtype=np.float64)
+    y = np.empty((L,), dtype=np.float64)
+    rc = _load().mss_oracle_recurrence(_dptr(abar), _dptr(bbar_x), _dptr(c), L, N,
+                                       _dptr(h), _dptr(y))
+    if rc != 0:
+        raise RuntimeError(f"mss_oracle_recurrence failed with code {rc}")
+    return h, y

@@ -1,0 +1,350 @@
+/*
+ * mss_oracle.c -- plain, slow, fp64 CPU oracle for the selective scan (S6)
+ * forward pass and its single-token decode update.
+ *
+ * TEST INFRASTRUCTURE ONLY.  Nothing on the product path may call, link or
+ * load this file or the library built from it: only the tests, the smoke
+ * check of __graft_entry__ and the CPU-baseline leg of bench.py use it.  It
+ * shares no source, header, table or helper with the CUDA library.
+ *
+ * What it computes, and where each step comes from:
+ *
+ *   - Continuous diagonal SSM h'(t) = A h(t) + B x(t), y = C h(t), one
+ *     real SISO system per channel with diagonal A
+ *     ["Mamba" paper review, section "SSM": the ODE and the diagonal/SISO
+ *      shapes A in R^{NxN} diag, B in R^{Nx1}, C in R^{1xN}].
+ *   - Step size Delta = softplus(Delta_raw + bias), softplus(x) = ln(1+e^x)
+ *     ["Exercises -- State-space models (Mamba, S4)", the softplus exercise:
+ *      Delta must be strictly positive, softplus maps R onto (0, inf)].
+ *     softplus can be switched off (then Delta = Delta_raw + bias).
+ *   - Zero-order hold for the transition: Abar = exp(Delta*A), per state for
+ *     a diagonal A ["Mamba" paper review, section "SSM", discretisation
+ *     formula; "Paper: Mamba" course page, Objectives, zero-order hold].
+ *   - Input matrix by the Euler rule Bbar = Delta*B (the course page lists
+ *     Euler as the alternative to the exact ZOH input matrix); so the input
+ *     term is Bbar x = Delta * B_t * u_t.
+ *   - Selective recurrence, state zero before the first token, update then
+ *     read out:  h_t = Abar_t (.) h_{t-1} + Bbar_t x_t ,  y_t = C_t . h_t
+ *     ["Mamba" paper review, section "SSM", discrete recurrence; "Exercises",
+ *      recurrent view h_k = Abar h_{k-1} + Bbar x_k, then y_k = C h_k, worked
+ *      impulse response starting from h = 0].  B_t and C_t depend on the
+ *     token ("Mamba" paper review, section "Selection Mechanism").
+ *   - Skip term and gate: y_t = (C_t . h_t + D u_t) * silu(z_t), with
+ *     silu(z) = z / (1 + e^{-z}); z absent means no gate, D absent means 0.
+ *     The pages name a gating mechanism that mixes in the residual
+ *     ("Mamba" paper review, section "SSM", block description) but print no
+ *     formula for it: this part has no printed value to pin against
+ *     (parity unpinned beyond its closed-form definition).
+ *   - Final state: the state after the last token.  Decode: one step of the
+ *     same recurrence starting from a caller-supplied state, which the
+ *     "Exercises" page describes as the generation-time view (constant-size
+ *     state, O(1) work per token).
+ *
+ * The sequential loop below is the plain definition.  A parallel scan
+ * reaches the same numbers up to rounding order because the composition of
+ * affine steps is associative ("NN Lab: Mamba", section "The Associative
+ * Property of Linear Recurrence").
+ *
+ * Precision: every operation is fp64.  Inputs arrive as fp32 arrays: bf16
+ * inputs are widened exactly by the caller, so no information is lost.
+ */
+#include <math.h>
+#include <pthread.h>
+#include <stdint.h>
+#include <stdlib.h>
+
+#define ORACLE_OK 0
+#define ORACLE_EINVAL (-1)
+#define ORACLE_ENOMEM (-2)
+
+/* softplus(s) = ln(1 + e^s).  For s > 0 the identity
+ * ln(1 + e^s) = s + ln(1 + e^{-s}) keeps exp from overflowing; it is exact
+ * algebra, not an approximation. */
+double mss_oracle_softplus(double s)
+{
+    if (s > 0.0)
+        return s + log1p(exp(-s));
+    return log1p(exp(s));
+}
+
+/* silu(z) = z * sigmoid(z) = z / (1 + e^{-z}). */
+double mss_oracle_silu(double z)
+{
+    return z / (1.0 + exp(-z));
+}
+
+/* One step of the discrete recurrence of one channel:
+ *   h[n] <- abar[n] * h[n] + bx[n]    for every state n,
+ * and the read-out sum_n c[n] * h[n] of the updated state. */
+static double recurrence_step(double *h, const double *abar, const double *bx,
+                              const double *c, int64_t N)
+{
+    double acc = 0.0;
+    for (int64_t n = 0; n < N; ++n) {
+        h[n] = abar[n] * h[n] + bx[n];
+        acc += c[n] * h[n];
+    }
+    return acc;
+}
+
+/* The discrete recurrence fed with already-discretised coefficients, for one
+ * channel:  abar, bbar_x, c are [L][N] (row t holds Abar_t, Bbar_t x_t, C_t);
+ * h starts at zero.  Writes y_out[L] and, if h_out is not NULL, the state
+ * after every token into h_out[L][N].  Used to check the recurrence on the
+ * worked example of the "Exercises" page, where Abar and Bbar are given. */
+int mss_oracle_recurrence(const double *abar, const double *bbar_x, const double *c,
+                          int64_t L, int64_t N, double *h_out, double *y_out)
+{
+    if (!abar || !bbar_x || !c || !y_out || L < 0 || N <= 0)
+        return ORACLE_EINVAL;
+    double *h = (double *)calloc((size_t)N, sizeof(double));
+    if (!h)
+        return ORACLE_ENOMEM;
+    for (int64_t t = 0; t < L; ++t) {
+        y_out[t] = recurrence_step(h, abar + t * N, bbar_x + t * N, c + t * N, N);
+        if (h_out)
+            for (int64_t n = 0; n < N; ++n)
+                h_out[t * N + n] = h[n];
+    }
+    free(h);
+    return ORACLE_OK;
+}
+
+/* ------------------------------------------------------------------------ */
+/* Selective scan forward pass.                                              */
+
+typedef struct {
+    /* inputs, layouts as documented at mss_oracle_scan_fwd */
+    const float *u, *delta, *A, *B, *C, *D, *z, *bias;
+    int softplus_flag;
+    double *y, *last_state;
+    int64_t batch, dim, N, L;
+    /* rows [row_begin, row_end) of the flattened (batch, dim) index */
+    int64_t row_begin, row_end;
+    int status;
+} scan_job;
+
+/* Discretise one token of one channel: Delta from the raw value, then
+ * Abar[n] = exp(Delta*A[n]) and Bbar x[n] = Delta * B[n] * u. */
+static double discretise(double delta_raw, double bias, int softplus_flag,
+                         const float *A_row, const float *B_bt, const float *C_bt,
+                         int64_t L, int64_t N, double u,
+                         double *abar, double *bx, double *c)
+{
+    double s = delta_raw + bias;
+    double dt = softplus_flag ? mss_oracle_softplus(s) : s;
+    for (int64_t n = 0; n < N; ++n) {
+        abar[n] = exp(dt * (double)A_row[n]);
+        bx[n] = dt * (double)B_bt[n * L] * u;
+        c[n] = (double)C_bt[n * L];
+    }
+    return dt;
+}
+
+static void *scan_rows(void *arg)
+{
+    scan_job *j = (scan_job *)arg;
+    const int64_t N = j->N, L = j->L;
+    double *work = (double *)malloc((size_t)(4 * N) * sizeof(double));
+    if (!work) {
+        j->status = ORACLE_ENOMEM;
+        return NULL;
+    }
+    double *h = work, *abar = work + N, *bx = work + 2 * N, *c = work + 3 * N;
+    for (int64_t row = j->row_begin; row < j->row_end; ++row) {
+        const int64_t b = row / j->dim, d = row % j->dim;
+        const float *u = j->u + row * L;
+        const float *dr = j->delta + row * L;
+        const float *z = j->z ? j->z + row * L : NULL;
+        const float *A_row = j->A + d * N;
+        const float *B_b = j->B + b * N * L; /* B[b][n][t] = B_b[n*L + t] */
+        const float *C_b = j->C + b * N * L;
+        const double Dd = j->D ? (double)j->D[d] : 0.0;
+        const double bias = j->bias ? (double)j->bias[d] : 0.0;
+        double *y = j->y + row * L;
+        for (int64_t n = 0; n < N; ++n)
+            h[n] = 0.0;
+        for (int64_t t = 0; t < L; ++t) {
+            const double ut = (double)u[t];
+            discretise((double)dr[t], bias, j->softplus_flag, A_row, B_b + t, C_b + t,
+                       L, N, ut, abar, bx, c);
+            double out = recurrence_step(h, abar, bx, c, N) + Dd * ut;
+            if (z)
+                out *= mss_oracle_silu((double)z[t]);
+            y[t] = out;
+        }
+        if (j->last_state)
+            for (int64_t n = 0; n < N; ++n)
+                j->last_state[row * N + n] = h[n];
+    }
+    free(work);
+    j->status = ORACLE_OK;
+    return NULL;
+}
+
+/* Run `fn` over rows [0, rows) split into `nthreads` contiguous ranges. */
+static int run_threaded(scan_job *proto, int64_t rows, int nthreads, void *(*fn)(void *))
+{
+    if (nthreads < 1)
+        nthreads = 1;
+    if ((int64_t)nthreads > rows)
+        nthreads = rows > 0 ? (int)rows : 1;
+    scan_job *jobs = (scan_job *)calloc((size_t)nthreads, sizeof(scan_job));
+    pthread_t *tids = (pthread_t *)calloc((size_t)nthreads, sizeof(pthread_t));
+    if (!jobs || !tids) {
+        free(jobs);
+        free(tids);
+        return ORACLE_ENOMEM;
+    }
+    for (int i = 0; i < nthreads; ++i) {
+        jobs[i] = *proto;
+        jobs[i].row_begin = rows * i / nthreads;
+        jobs[i].row_end = rows * (i + 1) / nthreads;
+        jobs[i].status = ORACLE_EINVAL;
+        /* one range runs here; so does a range whose thread could not start */
+        if (nthreads == 1 || pthread_create(&tids[i], NULL, fn, &jobs[i]) != 0) {
+            fn(&jobs[i]);
+            tids[i] = 0;
+        }
+    }
+    int rc = ORACLE_OK;
+    for (int i = 0; i < nthreads; ++i) {
+        if (tids[i])
+            pthread_join(tids[i], NULL);
+        if (jobs[i].status != ORACLE_OK)
+            rc = jobs[i].status;
+    }
+    free(jobs);
+    free(tids);
+    return rc;
+}
+
+/*
+ * Forward pass.  Layouts (all contiguous, C order):
+ *   u, delta, z : [batch][dim][L]   (token index fastest)
+ *   A           : [dim][N]          (negative reals for a stable system)
+ *   B, C        : [batch][N][L]     (shared by all channels of a batch row)
+ *   D, bias     : [dim]             (D, z, bias may be NULL)
+ *   y           : [batch][dim][L]   fp64 output
+ *   last_state  : [batch][dim][N]   fp64 output, may be NULL
+ * Returns 0, or a negative code for bad arguments / no memory.
+ */
+int mss_oracle_scan_fwd(const float *u, const float *delta, const float *A,
+                        const float *B, const float *C, const float *D,
+                        const float *z, const float *delta_bias, int softplus_flag,
+                        double *y, double *last_state,
+                        int64_t batch, int64_t dim, int64_t dstate, int64_t seqlen,
+                        int nthreads)
+{
+    if (!u || !delta || !A || !B || !C || !y)
+        return ORACLE_EINVAL;
+    if (batch < 0 || dim < 0 || dstate <= 0 || seqlen < 0)
+        return ORACLE_EINVAL;
+    scan_job proto = {u, delta, A, B, C, D, z, delta_bias, softplus_flag, y, last_state,
+                      batch, dim, dstate, seqlen, 0, 0, ORACLE_OK};
+    if (batch * dim == 0)
+        return ORACLE_OK;
+    return run_threaded(&proto, batch * dim, nthreads, scan_rows);
+}
+
+/* ------------------------------------------------------------------------ */
+/* Single-token decode update.                                               */
+
+typedef struct {
+    double *state;
+    const float *u, *delta, *A, *B, *C, *D, *z, *bias;
+    int softplus_flag;
+    double *y;
+    int64_t dim, N;
+    int64_t row_begin, row_end;
+    int status;
+} step_job;
+
+static void *step_rows(void *arg)
+{
+    step_job *j = (step_job *)arg;
+    const int64_t N = j->N;
+    double *work = (double *)malloc((size_t)(3 * N) * sizeof(double));
+    if (!work) {
+        j->status = ORACLE_ENOMEM;
+        return NULL;
+    }
+    double *abar = work, *bx = work + N, *c = work + 2 * N;
+    for (int64_t row = j->row_begin; row < j->row_end; ++row) {
+        const int64_t b = row / j->dim, d = row % j->dim;
+        const double ut = (double)j->u[row];
+        const double bias = j->bias ? (double)j->bias[d] : 0.0;
+        /* B, C of a decode step are [batch][N]: stride 1 between states. */
+        discretise((double)j->delta[row], bias, j->softplus_flag, j->A + d * N,
+                   j->B + b * N, j->C + b * N, 1, N, ut, abar, bx, c);
+        double out = recurrence_step(j->state + row * N, abar, bx, c, N);
+        out += (j->D ? (double)j->D[d] : 0.0) * ut;
+        if (j->z)
+            out *= mss_oracle_silu((double)j->z[row]);
+        j->y[row] = out;
+    }
+    free(work);
+    j->status = ORACLE_OK;
+    return NULL;
+}
+
+static int run_steps(step_job *proto, int64_t rows, int nthreads)
+{
+    if (nthreads < 1)
+        nthreads = 1;
+    if ((int64_t)nthreads > rows)
+        nthreads = rows > 0 ? (int)rows : 1;
+    step_job *jobs = (step_job *)calloc((size_t)nthreads, sizeof(step_job));
+    pthread_t *tids = (pthread_t *)calloc((size_t)nthreads, sizeof(pthread_t));
+    if (!jobs || !tids) {
+        free(jobs);
+        free(tids);
+        return ORACLE_ENOMEM;
+    }
+    for (int i = 0; i < nthreads; ++i) {
+        jobs[i] = *proto;
+        jobs[i].row_begin = rows * i / nthreads;
+        jobs[i].row_end = rows * (i + 1) / nthreads;
+        jobs[i].status = ORACLE_EINVAL;
+        if (nthreads == 1 || pthread_create(&tids[i], NULL, step_rows, &jobs[i]) != 0) {
+            step_rows(&jobs[i]);
+            tids[i] = 0;
+        }
+    }
+    int rc = ORACLE_OK;
+    for (int i = 0; i < nthreads; ++i) {
+        if (tids[i])
+            pthread_join(tids[i], NULL);
+        if (jobs[i].status != ORACLE_OK)
+            rc = jobs[i].status;
+    }
+    free(jobs);
+    free(tids);
+    return rc;
+}
+
+/*
+ * One decode step for every (batch, channel):
+ *   state      : [batch][dim][N] fp64, read and overwritten in place
+ *   u, delta, z: [batch][dim]
+ *   A          : [dim][N]
+ *   B, C       : [batch][N]
+ *   D, bias    : [dim]  (D, z, bias may be NULL)
+ *   y          : [batch][dim] fp64 output
+ */
+int mss_oracle_state_update(double *state, const float *u, const float *delta,
+                            const float *A, const float *B, const float *C,
+                            const float *D, const float *z, const float *delta_bias,
+                            int softplus_flag, double *y,
+                            int64_t batch, int64_t dim, int64_t dstate, int nthreads)
+{
+    if (!state || !u || !delta || !A || !B || !C || !y)
+        return ORACLE_EINVAL;
+    if (batch < 0 || dim < 0 || dstate <= 0)
+        return ORACLE_EINVAL;
+    step_job proto = {state, u, delta, A, B, C, D, z, delta_bias, softplus_flag, y,
+                      dim, dstate, 0, 0, ORACLE_OK};
+    if (batch * dim == 0)
+        return ORACLE_OK;
+    return run_steps(&proto, batch * dim, nthreads);
+}

@@ -1,0 +1,162 @@
+"""Seeded synthetic inputs for the selective scan, shared by the CUDA path's
+tests/bench and by the fp64 oracle.
+
+This module holds none of the method's arithmetic: it only draws random
+numbers, rounds them to the storage type (bf16 round-to-nearest-even, done
+here on the host so that both sides see the very same values) and widens
+bf16 back to fp32 (exact).  The step-size bias is chosen with the inverse of
+softplus so that the step sizes land in the stated range; that inverse is
+input construction only, never part of either computation.
+
+Recipe (the same for every workload; the seed is fixed per workload):
+
+* u, z, B, C ~ N(0, 1)
+* delta_raw = 0.1 * N(0, 1)
+* bias[d] = softplus^-1(dt_d) = log(expm1(dt_d)),  dt_d = exp(U(ln 1e-3, ln 1e-1)),
+  so that softplus(delta_raw + bias) is log-uniform on about [1e-3, 1e-1]
+* A[d, n] = -(n + 1)  (the S4D-Real initialisation with negative real poles)
+* D = 1, or D ~ N(1, 0.1) where the workload says so
+* everything is drawn in fp32, then rounded to bf16 for bf16 workloads;
+  A, D and bias stay fp32.
+"""
+from __future__ import annotations
+
+import dataclasses
+from typing import Optional
+
+import numpy as np
+
+
+@dataclasses.dataclass(frozen=True)
+class Workload:
+    name: str
+    batch: int
+    dim: int
+    dstate: int
+    seqlen: int          # 0 for a decode workload
+    dtype: str           # "f32" or "bf16"
+    d_skip: str          # "one" or "normal"
+    seed: int
+    decode_steps: int = 0
+
+    @property
+    def channel_tokens(self) -> int:
+        return self.batch * self.dim * max(self.seqlen, 1)
+
+
+# Named by what they are, with their sizes.  Seeds are 1000 + the workload's
+# position in the list.
+WORKLOADS = {
+    w.name: w
+    for w in [
+        Workload("s6-fwd-fp32-b1-d16-n4-l256", 1, 16, 4, 256, "f32", "one", 1001),
+        Workload("mamba130m-layer-bf16-b8-d1536-n16-l2048", 8, 1536, 16, 2048, "bf16", "one", 1002),
+        Workload("mamba1.4b-layer-bf16-b4-d4096-n16-l4096", 4, 4096, 16, 4096, "bf16", "normal", 1003),
+        Workload("long-seq-bf16-b1-d2048-n16-l131072", 1, 2048, 16, 131072, "bf16", "one", 1004),
+        Workload("decode-bf16-b256-d5120-n16-x1024", 256, 5120, 16, 0, "bf16", "normal", 1005,
+                 decode_steps=1024),
+    ]
+}
+
+FWD_WORKLOADS = [n for n, w in WORKLOADS.items() if w.seqlen > 0]
+BENCH_WORKLOAD = "mamba1.4b-layer-bf16-b4-d4096-n16-l4096"
+DECODE_WORKLOAD = "decode-bf16-b256-d5120-n16-x1024"
+
+
+def to_bf16_bits(x: np.ndarray) -> np.ndarray:
+    """Round fp32 values to bf16 (round to nearest, ties to even); returns the
+    16-bit patterns as uint16.  Inputs here are finite."""
+    b = np.ascontiguousarray(x, dtype=np.float32).view(np.uint32)
+    rounded = b + (np.uint32(0x7FFF) + ((b >> np.uint32(16)) & np.uint32(1)))
+    return (rounded >> np.uint32(16)).astype(np.uint16)
+
+
+def bf16_bits_to_f32(bits: np.ndarray) -> np.ndarray:
+    """Widen bf16 bit patterns to fp32 (exact)."""
+    return (np.ascontiguousarray(bits, dtype=np.uint16).astype(np.uint32)
+            << np.uint32(16)).view(np.float32)
+
+
+@dataclasses.dataclass
+class Tensor:
+    """One input tensor: the values both sides compute on (fp32, exact) and the
+    bytes the device receives (fp32 values, or bf16 bit patterns)."""
+    values: np.ndarray       # float32
+    stored: np.ndarray       # float32 or uint16 (bf16 bits)
+    dtype: str               # "f32" or "bf16"
+
+
+def _store(x32: np.ndarray, dtype: str) -> Tensor:
+    x32 = np.ascontiguousarray(x32, dtype=np.float32)
+    if dtype == "f32":
+        return Tensor(x32, x32, "f32")
+    if dtype == "bf16":
+        bits = to_bf16_bits(x32)
+        return Tensor(bf16_bits_to_f32(bits), bits, "bf16")
+    raise ValueError(f"unknown dtype {dtype!r}")
+
+
+def _rng(seed, *stream):
+    return np.random.Generator(np.random.PCG64(np.random.SeedSequence([int(seed), *map(int, stream)])))
+
+
+def channel_params(dim: int, dstate: int, d_skip: str, seed: int):
+    """A [dim, N], D [dim], bias [dim] -- fp32."""
+    rng = _rng(seed, 0)
+    A = -np.broadcast_to(np.arange(1, dstate + 1, dtype=np.float32), (dim, dstate)).copy()
+    log_dt = rng.uniform(np.log(1e-3), np.log(1e-1), size=dim)
+    dt = np.exp(log_dt)
+    bias = np.log(np.expm1(dt)).astype(np.float32)
+    if d_skip == "one":
+        D = np.ones(dim, dtype=np.float32)
+    elif d_skip == "normal":
+        D = (1.0 + 0.1 * rng.standard_normal(dim)).astype(np.float32)
+    else:
+        raise ValueError(f"unknown D recipe {d_skip!r}")
+    return A, D, bias
+
+
+def scan_inputs(batch: int, dim: int, dstate: int, seqlen: int, dtype: str,
+                seed: int, d_skip: str = "one") -> dict:
+    """Inputs of one forward pass.  u, delta, z: [batch, dim, L]; B, C:
+    [batch, N, L]; A: [dim, N]; D, delta_bias: [dim]."""
+    A, D, bias = channel_params(dim, dstate, d_skip, seed)
+    rng = _rng(seed, 1)
+    shape = (batch, dim, seqlen)
+    u = _store(rng.standard_normal(shape, dtype=np.float32), dtype)
+    delta = _store(np.float32(0.1) * rng.standard_normal(shape, dtype=np.float32), dtype)
+    z = _store(rng.standard_normal(shape, dtype=np.float32), dtype)
+    B = _store(rng.standard_normal((batch, dstate, seqlen), dtype=np.float32), dtype)
+    C = _store(rng.standard_normal((batch, dstate, seqlen), dtype=np.float32), dtype)
+    return dict(u=u, delta=delta, z=z, B=B, C=C, A=A, D=D, delta_bias=bias,
+                batch=batch, dim=dim, dstate=dstate, seqlen=seqlen, dtype=dtype)
+
+
+def workload_inputs(name: str, seqlen: Optional[int] = None) -> dict:
+    w = WORKLOADS[name]
+    if w.seqlen == 0:
+        raise ValueError(f"{name} is a decode workload; use decode_step_inputs")
+    return scan_inputs(w.batch, w.dim, w.dstate, w.seqlen if seqlen is None else seqlen,
+                       w.dtype, w.seed, w.d_skip)
+
+
+def decode_step_inputs(batch: int, dim: int, dstate: int, dtype: str, seed: int,
+                       step: int) -> dict:
+    """Per-token inputs of decode step `step`: u, delta, z [batch, dim];
+    B, C [batch, N].  Each step draws from its own seeded stream."""
+    rng = _rng(seed, 2, step)
+    u = _store(rng.standard_normal((batch, dim), dtype=np.float32), dtype)
+    delta = _store(np.float32(0.1) * rng.standard_normal((batch, dim), dtype=np.float32), dtype)
+    z = _store(rng.standard_normal((batch, dim), dtype=np.float32), dtype)
+    B = _store(rng.standard_normal((batch, dstate), dtype=np.float32), dtype)
+    C = _store(rng.standard_normal((batch, dstate), dtype=np.float32), dtype)
+    return dict(u=u, delta=delta, z=z, B=B, C=C)
+
+
+def initial_state(batch: int, dim: int, dstate: int, seed: int, kind: str = "zero") -> np.ndarray:
+    """fp32 starting state [batch, dim, N]: zeros, or N(0, 1) draws."""
+    if kind == "zero":
+        return np.zeros((batch, dim, dstate), dtype=np.float32)
+    if kind == "normal":
+        return _rng(seed, 3).standard_normal((batch, dim, dstate), dtype=np.float32)
+    raise ValueError(f"unknown initial state {kind!r}")

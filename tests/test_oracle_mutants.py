@@ -1,0 +1,70 @@
+"""The pins must catch plausible mistakes in the oracle.
+
+Each case copies oracle/mss_oracle.c, plants one mistake (a dropped term, a
+wrong sign, a swapped operand, a wrong index or order), builds the copy and
+runs the pin tests against it in a subprocess.  The pins must fail for every
+mutant and pass for the unmodified source.  CPU only; nothing here touches
+the CUDA path.
+"""
+import os
+import subprocess
+import sys
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+SRC = os.path.join(ROOT, "oracle", "mss_oracle.c")
+
+MUTANTS = {
+    "drop_input_term": ("h[n] = abar[n] * h[n] + bx[n];", "h[n] = abar[n] * h[n];"),
+    "exponent_sign": ("abar[n] = exp(dt * (double)A_row[n]);", "abar[n] = exp(-dt * (double)A_row[n]);"),
+    "readout_before_update": (
+        "h[n] = abar[n] * h[n] + bx[n];\n        acc += c[n] * h[n];",
+        "acc += c[n] * h[n];\n        h[n] = abar[n] * h[n] + bx[n];"),
+    "B_and_C_swapped": ("bx[n] = dt * (double)B_bt[n * L] * u;", "bx[n] = dt * (double)C_bt[n * L] * u;"),
+    "input_rule_without_step": ("bx[n] = dt * (double)B_bt[n * L] * u;", "bx[n] = (double)B_bt[n * L] * u;"),
+    "softplus_drops_one": ("return log1p(exp(s));", "return log(exp(s));"),
+    "softplus_positive_branch": ("return s + log1p(exp(-s));", "return log1p(exp(-s));"),
+    "bias_dropped": ("double s = delta_raw + bias;", "double s = delta_raw;"),
+    "skip_dropped": ("double out = recurrence_step(h, abar, bx, c, N) + Dd * ut;",
+                     "double out = recurrence_step(h, abar, bx, c, N);"),
+    "gate_is_sigmoid": ("return z / (1.0 + exp(-z));", "return 1.0 / (1.0 + exp(-z));"),
+    "state_not_reset_per_row": ("        for (int64_t n = 0; n < N; ++n)\n            h[n] = 0.0;\n        for (int64_t t = 0; t < L; ++t) {",
+                                "        for (int64_t t = 0; t < L; ++t) {"),
+    "decode_B_token_stride": ("j->B + b * N, j->C + b * N, 1, N,", "j->B + b * N, j->C + b * N, N, N,"),
+    "B_batch_index": ("const float *B_b = j->B + b * N * L;", "const float *B_b = j->B;"),
+}
+
+
+def _run_pins(lib_path):
+    env = dict(os.environ, MSS_ORACLE_LIB=lib_path)
+    return subprocess.run(
+        [sys.executable, "-m", "pytest", "-q", "-x", "-p", "no:cacheprovider",
+         os.path.join(ROOT, "tests", "test_oracle_pins.py")],
+        cwd=ROOT, env=env, capture_output=True, text=True, timeout=600)
+
+
+def _build(src_text, tmp_path, name):
+    c = tmp_path / f"{name}.c"
+    so = tmp_path / f"{name}.so"
+    c.write_text(src_text)
+    subprocess.check_call(["gcc", "-std=c99", "-O2", "-fno-fast-math", "-ffp-contract=off",
+                           "-fPIC", "-shared", "-o", str(so), str(c), "-lm", "-lpthread"])
+    return str(so)
+
+
+def test_unmodified_source_passes(tmp_path):
+    with open(SRC) as f:
+        text = f.read()
+    r = _run_pins(_build(text, tmp_path, "original"))
+    assert r.returncode == 0, r.stdout[-2000:]
+
+
+@pytest.mark.parametrize("name", sorted(MUTANTS))
+def test_pins_catch_mutant(name, tmp_path):
+    old, new = MUTANTS[name]
+    with open(SRC) as f:
+        text = f.read()
+    assert text.count(old) == 1, f"mutation site for {name} not found exactly once"
+    r = _run_pins(_build(text.replace(old, new), tmp_path, name))
+    assert r.returncode != 0, f"pins did not catch mutant {name}"

@@ -1,0 +1,421 @@
+"""Pins of the fp64 oracle against what the pages and the mathematics fix.
+
+CPU only.  Each test checks the oracle against something other than itself:
+values the pages print (tests/golden/, each file names its page and
+exercise), closed forms, alternative scan orders and matrix views written
+independently in oracle/scans.py, and exact invariants (causality, zero step
+size, linearity, contraction).  The citations name the page and section.
+"""
+import json
+import math
+import os
+
+import numpy as np
+import pytest
+
+import oracle
+from oracle import scans
+
+GOLDEN = os.path.join(os.path.dirname(__file__), "golden")
+
+
+def _golden(name):
+    with open(os.path.join(GOLDEN, name)) as f:
+        return json.load(f)
+
+
+def _impulse_inputs(A_vals, B_vals, C_vals, delta_raw, L, u=None):
+    """One channel (batch 1, dim 1) with per-token-constant B, C and step."""
+    N = len(A_vals)
+    if u is None:
+        u = np.zeros(L, dtype=np.float32)
+        u[0] = 1.0
+    return dict(
+        u=np.asarray(u, dtype=np.float32).reshape(1, 1, L),
+        delta=np.full((1, 1, L), delta_raw, dtype=np.float32),
+        A=np.asarray(A_vals, dtype=np.float32).reshape(1, N),
+        B=np.repeat(np.asarray(B_vals, dtype=np.float32).reshape(1, N, 1), L, axis=2),
+        C=np.repeat(np.asarray(C_vals, dtype=np.float32).reshape(1, N, 1), L, axis=2),
+    )
+
+
+# --------------------------------------------------------------------------
+# Worked example: 2-state impulse response
+# ("Exercises -- State-space models (Mamba, S4)", recurrent view, steps 1-3)
+
+def test_worked_example_recurrence_states_and_outputs():
+    g = _golden("impulse_response_2state.json")
+    L = len(g["x"])
+    abar = np.tile(g["Abar_diag"], (L, 1))
+    bx = np.outer(g["x"], g["Bbar"])
+    c = np.tile(g["C"], (L, 1))
+    h, y = oracle.recurrence(abar, bx, c)
+    np.testing.assert_allclose(h, g["h"], rtol=0, atol=1e-15)
+    np.testing.assert_allclose(y, g["y"], rtol=0, atol=1e-15)
+
+
+def test_worked_example_kernel_is_impulse_response():
+    # convolution-kernel exercise: K = (C Bbar, C Abar Bbar, C Abar^2 Bbar)
+    g = _golden("impulse_response_2state.json")
+    K = scans.conv_kernel(g["Abar_diag"], g["Bbar"], g["C"], len(g["kernel"]))
+    np.testing.assert_allclose(K, g["kernel"], rtol=0, atol=1e-15)
+    # any input convolved with K equals the recurrence (same page)
+    rng = np.random.default_rng(7)
+    x = rng.standard_normal(12)
+    L = len(x)
+    K12 = scans.conv_kernel(g["Abar_diag"], g["Bbar"], g["C"], L)
+    _, y = oracle.recurrence(np.tile(g["Abar_diag"], (L, 1)), np.outer(x, g["Bbar"]),
+                             np.tile(g["C"], (L, 1)))
+    np.testing.assert_allclose(y, scans.causal_conv(K12, x), rtol=1e-13, atol=1e-14)
+
+
+@pytest.mark.parametrize("step", [1.0, 0.5, 0.125])
+def test_worked_example_through_full_forward(step):
+    """The same example through the forward entry point: softplus off, no
+    bias, A = ln(Abar)/step, B = Bbar/step.  With the Euler input rule
+    (Bbar = step*B) and Abar = exp(step*A) this must reproduce the page's
+    outputs for every step size; an input rule that ignored the step, or an
+    exponent without it, would only match at step = 1."""
+    g = _golden("impulse_response_2state.json")
+    A = [math.log(a) / step for a in g["Abar_diag"]]
+    Bv = [b / step for b in g["Bbar"]]
+    inp = _impulse_inputs(A, Bv, g["C"], step, 3)
+    y, last = oracle.scan_fwd(**inp, softplus_flag=False)
+    # A and B are rounded to fp32 on the way in: allow that rounding only
+    np.testing.assert_allclose(y[0, 0], g["y"], rtol=0, atol=2e-7)
+    np.testing.assert_allclose(last[0, 0], g["h"][-1], rtol=0, atol=2e-7)
+
+
+# --------------------------------------------------------------------------
+# Closed forms of the discretisation and of softplus
+# ("Exercises -- State-space models (Mamba, S4)": stability exercise (b),
+#  softplus exercise, decay-time exercise, the A = -0.02 follow-up)
+
+def _half_unit(digits):
+    return 0.5 * 10.0 ** (-digits)
+
+
+def _abar_via_impulse(A, delta_raw, softplus_flag):
+    """N=1, B=C=1, impulse input: y_0 = step, y_1 = Abar * step."""
+    inp = _impulse_inputs([A], [1.0], [1.0], delta_raw, 2)
+    y, _ = oracle.scan_fwd(**inp, softplus_flag=softplus_flag)
+    return y[0, 0, 0], y[0, 0, 1] / y[0, 0, 0]
+
+
+def test_abar_closed_forms():
+    for case in _golden("discretisation_closed_forms.json")["abar"]:
+        step, abar = _abar_via_impulse(case["A"], case["delta"], False)
+        assert step == case["delta"]
+        assert abs(abar - case["value"]) <= _half_unit(case["digits"]), case
+
+
+def test_softplus_values():
+    for case in _golden("discretisation_closed_forms.json")["softplus"]:
+        assert abs(oracle.softplus(case["x"]) - case["value"]) <= _half_unit(case["digits"])
+        # the same value is the step size the forward pass uses
+        step, _ = _abar_via_impulse(-1.0, case["x"], True)
+        assert abs(step - case["value"]) <= _half_unit(case["digits"]), case
+
+
+def test_abar_after_softplus():
+    for case in _golden("discretisation_closed_forms.json")["abar_after_softplus"]:
+        _, abar = _abar_via_impulse(case["A"], case["delta_raw"], True)
+        assert abs(abar - case["value"]) <= _half_unit(case["digits"]), case
+
+
+def test_decay_time_to_one_over_e():
+    """n = -1/ln(Abar) steps to fall to 1/e; the impulse response of one
+    state is step * Abar^k, so its envelope crosses step/e between k = floor(n)
+    and k = ceil(n)."""
+    for case in _golden("discretisation_closed_forms.json")["decay_to_1_over_e"]:
+        L = 40
+        inp = _impulse_inputs([case["A"]], [1.0], [1.0], case["delta_raw"], L)
+        y, _ = oracle.scan_fwd(**inp, softplus_flag=True)
+        r = y[0, 0] / y[0, 0, 0]
+        n = -1.0 / math.log(r[1])
+        assert abs(n - case["steps"]) <= _half_unit(case["digits"]), case
+        below = np.nonzero(r < math.exp(-1.0))[0]
+        assert below[0] == math.ceil(case["steps"])
+
+
+# --------------------------------------------------------------------------
+# Scan orders and associativity
+# ("Paper: Mamba" course page, section "Code": sequential and
+#  Blelloch / Hillis-Steele / chunked scans tested equal;
+#  "NN Lab: Mamba", "The Associative Property of Linear Recurrence")
+
+def _random_pairs(rng, L, N):
+    return [(rng.uniform(0.05, 0.999, N), rng.standard_normal(N)) for _ in range(L)]
+
+
+@pytest.mark.parametrize("L", [1, 2, 3, 5, 8, 13, 31, 64])
+def test_scan_orders_agree_with_oracle(L):
+    rng = np.random.default_rng(100 + L)
+    N = 3
+    pairs = _random_pairs(rng, L, N)
+    a = np.array([p[0] for p in pairs])
+    b = np.array([p[1] for p in pairs])
+    h_oracle, _ = oracle.recurrence(a, b, np.ones((L, N)))
+    for name, prefixes in [
+        ("sequential", scans.scan_sequential(pairs)),
+        ("blelloch", scans.scan_blelloch(pairs)),
+        ("hillis_steele", scans.scan_hillis_steele(pairs)),
+    ] + [(f"chunked{c}", scans.scan_chunked(pairs, c)) for c in sorted({1, 2, 3, 7, L})]:
+        h = np.array(scans.states_from_scan(prefixes))
+        np.testing.assert_allclose(h, h_oracle, rtol=1e-12, atol=1e-14, err_msg=name)
+
+
+def test_composition_is_associative_bitwise():
+    # dyadic rationals with small denominators: every product and sum below
+    # is exact in fp64, so associativity must hold to the last bit
+    rng = np.random.default_rng(3)
+    for _ in range(2000):
+        p, q, r = [(rng.integers(1, 64) / 64.0, rng.integers(-64, 65) / 64.0) for _ in range(3)]
+        left = scans.compose(scans.compose(p, q), r)
+        right = scans.compose(p, scans.compose(q, r))
+        assert left == right
+
+
+def test_composition_order_matters():
+    # the composition is not commutative: (a,b) then (a',b') differs from the reverse
+    p, q = (0.5, 1.0), (0.25, -2.0)
+    assert scans.compose(p, q) != scans.compose(q, p)
+    # "p then q" applied to h: q(p(h))
+    a, b = scans.compose(p, q)
+    h = 3.0
+    assert a * h + b == q[0] * (p[0] * h + p[1]) + q[1]
+
+
+def _discretised(inp, softplus_flag):
+    """Abar, Bbar*u and C as [batch, dim, L, N] arrays, for the matrix and scan
+    views below (the step size comes from the oracle's own softplus)."""
+    u, dr, A, B, C = (np.asarray(inp[k], dtype=np.float64) for k in ("u", "delta", "A", "B", "C"))
+    bias = np.asarray(inp.get("delta_bias"), dtype=np.float64) if inp.get("delta_bias") is not None else 0.0
+    s = dr + (bias[None, :, None] if np.ndim(bias) else 0.0)
+    step = np.vectorize(oracle.softplus)(s) if softplus_flag else s
+    abar = np.exp(step[..., None] * A[None, :, None, :])
+    bx = (step * u)[..., None] * np.transpose(B, (0, 2, 1))[:, None, :, :]
+    c = np.broadcast_to(np.transpose(C, (0, 2, 1))[:, None, :, :], abar.shape)
+    return abar, bx, c
+
+
+def test_forward_equals_blelloch_scan_of_the_same_steps():
+    rng = np.random.default_rng(11)
+    batch, dim, N, L = 2, 3, 4, 37
+    inp = dict(
+        u=rng.standard_normal((batch, dim, L)).astype(np.float32),
+        delta=(0.1 * rng.standard_normal((batch, dim, L))).astype(np.float32),
+        A=-np.tile(np.arange(1, N + 1, dtype=np.float32), (dim, 1)),
+        B=rng.standard_normal((batch, N, L)).astype(np.float32),
+        C=rng.standard_normal((batch, N, L)).astype(np.float32),
+        delta_bias=np.log(np.expm1(np.array([1e-3, 1e-2, 1e-1]))).astype(np.float32),
+    )
+    y, last = oracle.scan_fwd(**inp, softplus_flag=True)
+    abar, bx, c = _discretised(inp, True)
+    for b in range(batch):
+        for d in range(dim):
+            pairs = [(abar[b, d, t], bx[b, d, t]) for t in range(L)]
+            h = np.array(scans.states_from_scan(scans.scan_blelloch(pairs)))
+            np.testing.assert_allclose(np.sum(c[b, d] * h, axis=1), y[b, d], rtol=1e-12, atol=1e-13)
+            np.testing.assert_allclose(h[-1], last[b, d], rtol=1e-12, atol=1e-13)
+
+
+# --------------------------------------------------------------------------
+# Semiseparable matrix form and the scalar case
+# ("Mamba" paper review, section "Mamba 2")
+
+def test_semiseparable_matrix_form():
+    rng = np.random.default_rng(5)
+    L, N = 9, 3
+    inp = dict(
+        u=rng.standard_normal((1, 1, L)).astype(np.float32),
+        delta=rng.uniform(0.01, 0.5, (1, 1, L)).astype(np.float32),
+        A=-rng.uniform(0.5, 3.0, (1, N)).astype(np.float32),
+        B=rng.standard_normal((1, N, L)).astype(np.float32),
+        C=rng.standard_normal((1, N, L)).astype(np.float32),
+    )
+    y, _ = oracle.scan_fwd(**inp, softplus_flag=False)
+    step = inp["delta"][0, 0].astype(np.float64)
+    abar = np.exp(step[:, None] * inp["A"][0].astype(np.float64)[None, :])
+    bbar = step[:, None] * inp["B"][0].T.astype(np.float64)        # Euler input matrix
+    M = scans.sss_matrix(abar, bbar, inp["C"][0].T)
+    np.testing.assert_allclose(M @ inp["u"][0, 0].astype(np.float64), y[0, 0], rtol=1e-12, atol=1e-13)
+    assert np.all(np.triu(M, 1) == 0.0)
+
+
+def test_scalar_case_is_first_order_recurrence():
+    # N = 1, B = C = 1, no skip, no gate: y_t = a_t y_{t-1} + step_t u_t
+    rng = np.random.default_rng(6)
+    L = 50
+    inp = _impulse_inputs([-0.7], [1.0], [1.0], 0.0, L, u=rng.standard_normal(L))
+    inp["delta"] = rng.uniform(0.01, 1.0, (1, 1, L)).astype(np.float32)
+    y, _ = oracle.scan_fwd(**inp, softplus_flag=False)
+    step = inp["delta"][0, 0].astype(np.float64)
+    a = np.exp(step * np.float64(np.float32(-0.7)))
+    prev = 0.0
+    for t in range(L):
+        prev = a[t] * prev + step[t] * np.float64(inp["u"][0, 0, t])
+        assert abs(y[0, 0, t] - prev) <= 1e-13 * max(1.0, abs(prev))
+
+
+# --------------------------------------------------------------------------
+# The time-invariant special case is a convolution
+# ("Exercises -- State-space models (Mamba, S4)", convolutional view)
+
+def test_time_invariant_forward_is_causal_convolution():
+    rng = np.random.default_rng(8)
+    N, L = 4, 40
+    A = -rng.uniform(0.1, 2.0, N)
+    Bv, Cv = rng.standard_normal(N), rng.standard_normal(N)
+    step = 0.3
+    u = rng.standard_normal(L)
+    inp = _impulse_inputs(A, Bv, Cv, step, L, u=u)
+    y, _ = oracle.scan_fwd(**inp, softplus_flag=False)
+    A32 = inp["A"][0].astype(np.float64)
+    abar = np.exp(np.float64(np.float32(step)) * A32)
+    bbar = np.float64(np.float32(step)) * inp["B"][0, :, 0].astype(np.float64)
+    K = scans.conv_kernel(abar, bbar, inp["C"][0, :, 0], L)
+    np.testing.assert_allclose(y[0, 0], scans.causal_conv(K, inp["u"][0, 0]), rtol=1e-11, atol=1e-12)
+
+
+# --------------------------------------------------------------------------
+# Invariants
+
+def _random_forward_inputs(seed, batch=2, dim=5, N=4, L=64):
+    rng = np.random.default_rng(seed)
+    return dict(
+        u=rng.standard_normal((batch, dim, L)).astype(np.float32),
+        delta=(0.1 * rng.standard_normal((batch, dim, L))).astype(np.float32),
+        A=-np.tile(np.arange(1, N + 1, dtype=np.float32), (dim, 1)),
+        B=rng.standard_normal((batch, N, L)).astype(np.float32),
+        C=rng.standard_normal((batch, N, L)).astype(np.float32),
+        D=rng.standard_normal(dim).astype(np.float32),
+        z=rng.standard_normal((batch, dim, L)).astype(np.float32),
+        delta_bias=np.log(np.expm1(rng.uniform(1e-3, 1e-1, dim))).astype(np.float32),
+    )
+
+
+def test_zero_step_ignores_the_input():
+    """A zero step leaves the state unchanged ("Mamba" paper review, section
+    "Selection Mechanism": with Delta = 0 the input is ignored)."""
+    inp = _random_forward_inputs(21)
+    inp.pop("delta_bias")
+    t0 = 30
+    inp["delta"] = np.abs(inp["delta"]) + np.float32(0.01)
+    inp["delta"][:, :, t0] = 0.0
+    _, before = oracle.scan_fwd(**{k: (v[..., :t0] if k in ("u", "delta", "z", "B", "C") else v)
+                                   for k, v in inp.items()}, softplus_flag=False)
+    _, after = oracle.scan_fwd(**{k: (v[..., :t0 + 1] if k in ("u", "delta", "z", "B", "C") else v)
+                                  for k, v in inp.items()}, softplus_flag=False)
+    assert np.array_equal(before, after)
+
+
+def test_causality():
+    inp = _random_forward_inputs(22)
+    y0, _ = oracle.scan_fwd(**inp)
+    t0 = 40
+    inp["u"][:, :, t0] += 1.0
+    inp["delta"][:, :, t0] -= 0.5
+    inp["B"][:, :, t0] *= -3.0
+    y1, _ = oracle.scan_fwd(**inp)
+    assert np.array_equal(y0[..., :t0], y1[..., :t0])
+    assert not np.array_equal(y0[..., t0:], y1[..., t0:])
+
+
+def test_linearity_in_u_without_gate():
+    inp = _random_forward_inputs(23)
+    inp.pop("z")
+    rng = np.random.default_rng(24)
+    # multiples of 1/256 in [-4, 4]: the combination below is exact in fp32
+    u1 = (rng.integers(-1024, 1025, inp["u"].shape) / 256.0).astype(np.float32)
+    u2 = (rng.integers(-1024, 1025, inp["u"].shape) / 256.0).astype(np.float32)
+    u3 = (np.float32(2.0) * u1 - np.float32(0.5) * u2).astype(np.float32)
+    assert np.array_equal(u3.astype(np.float64), 2.0 * u1.astype(np.float64) - 0.5 * u2.astype(np.float64))
+    y1, _ = oracle.scan_fwd(**{**inp, "u": u1})
+    y2, _ = oracle.scan_fwd(**{**inp, "u": u2})
+    y3, _ = oracle.scan_fwd(**{**inp, "u": u3})
+    np.testing.assert_allclose(y3, 2.0 * y1 - 0.5 * y2, rtol=1e-12, atol=1e-12)
+
+
+def test_contraction_and_state_bound():
+    """For A < 0 and a positive step, 0 < Abar < 1 ("NN Lab: Mamba", "Proof of
+    Spectral Stability & Contraction Mapping"; "Exercises", stability
+    exercise (a)), so |h_t| <= max|x| / (1 - max Abar) per state."""
+    for A, step in [(-1.0, 1e-3), (-16.0, 1e-3), (-1.0, 5.0), (-0.02, 0.0486)]:
+        _, abar = _abar_via_impulse(A, step, False)
+        assert 0.0 < abar < 1.0
+    inp = _random_forward_inputs(25, L=512)
+    _, last = oracle.scan_fwd(**inp)
+    abar, bx, _ = _discretised(inp, True)
+    assert np.all((abar > 0) & (abar < 1))
+    bound = np.max(np.abs(bx), axis=2) / (1.0 - np.max(abar, axis=2))
+    assert np.all(np.abs(last) <= bound)
+    # A = 0 is marginal (never forgets) and A > 0 grows ("Exercises", stability (a))
+    _, abar0 = _abar_via_impulse(0.0, 0.5, False)
+    _, abar_pos = _abar_via_impulse(0.5, 0.5, False)
+    assert abar0 == 1.0 and abar_pos > 1.0
+
+
+def test_silu_closed_forms():
+    # silu(z) = z * sigmoid(z): silu(0) = 0; sigmoid(0) = 1/2 so the slope at 0
+    # is 1/2; silu(z) -> z for large z and -> 0 for very negative z
+    assert oracle.silu(0.0) == 0.0
+    assert abs(oracle.silu(1e-8) / 1e-8 - 0.5) < 1e-8
+    assert abs(oracle.silu(40.0) - 40.0) < 1e-12
+    assert abs(oracle.silu(-40.0)) < 1e-15
+    assert abs(oracle.silu(1.0) - 1.0 / (1.0 + math.e ** -1)) < 1e-16
+
+
+# --------------------------------------------------------------------------
+# Decode step and chaining
+# ("Exercises", generation view: one token at a time with a constant-size state)
+
+def _slice_t(inp, t0, t1):
+    return {k: (v[..., t0:t1] if k in ("u", "delta", "z", "B", "C") else v) for k, v in inp.items()}
+
+
+def test_decode_steps_equal_forward():
+    inp = _random_forward_inputs(31, L=20)
+    y, last = oracle.scan_fwd(**inp)
+    batch, dim, N = last.shape
+    state = np.zeros((batch, dim, N))
+    for t in range(20):
+        step = {k: np.ascontiguousarray(v[..., t]) for k, v in inp.items() if k in ("u", "delta", "z", "B", "C")}
+        yt, state = oracle.state_update(state, A=inp["A"], D=inp["D"], delta_bias=inp["delta_bias"], **step)
+        np.testing.assert_allclose(yt, y[..., t], rtol=1e-13, atol=1e-14)
+    np.testing.assert_allclose(state, last, rtol=1e-13, atol=1e-14)
+
+
+def test_forward_then_decode_equals_longer_forward():
+    inp = _random_forward_inputs(32, L=48)
+    y_full, last_full = oracle.scan_fwd(**inp)
+    L0 = 40
+    _, state = oracle.scan_fwd(**_slice_t(inp, 0, L0))
+    for t in range(L0, 48):
+        step = {k: np.ascontiguousarray(v[..., t]) for k, v in inp.items() if k in ("u", "delta", "z", "B", "C")}
+        yt, state = oracle.state_update(state, A=inp["A"], D=inp["D"], delta_bias=inp["delta_bias"], **step)
+        np.testing.assert_allclose(yt, y_full[..., t], rtol=1e-13, atol=1e-14)
+    np.testing.assert_allclose(state, last_full, rtol=1e-13, atol=1e-14)
+
+
+def test_empty_sizes():
+    inp = _random_forward_inputs(33, L=0)
+    y, last = oracle.scan_fwd(**inp)
+    assert y.shape == (2, 5, 0)
+    assert np.all(last == 0.0)
+    inp = _random_forward_inputs(34, batch=0)
+    y, last = oracle.scan_fwd(**inp)
+    assert y.shape[0] == 0 and last.shape[0] == 0
+
+
+def test_skip_term_alone():
+    """With B = 0 nothing enters the state, so y = D*u (no gate) and
+    y = D*u*silu(z) (gate): the skip term and the gate in isolation."""
+    inp = _random_forward_inputs(35)
+    inp["B"][:] = 0.0
+    y, last = oracle.scan_fwd(**{k: v for k, v in inp.items() if k != "z"})
+    Du = inp["D"][None, :, None].astype(np.float64) * inp["u"].astype(np.float64)
+    assert np.array_equal(y, Du) and np.all(last == 0.0)
+    yg, _ = oracle.scan_fwd(**inp)
+    gate = np.vectorize(oracle.silu)(inp["z"].astype(np.float64))
+    assert np.array_equal(yg, Du * gate)
