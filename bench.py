@@ -1,0 +1,467 @@
+#!/usr/bin/env python3
+"""Throughput of the selective scan (S6) on B200: one JSON line on stdout.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl mss|reference]
+
+A step is one pass of the whole hot path over one batch of the
+Mamba-1.4B-shaped layer workload (batch 4, d_inner 4096, N 16, L 4096, bf16
+inputs, fp32 state and arithmetic): the forward scan over the full sequences
+(load, step size, discretisation, scan, gated read-out, final state) followed
+by one decode token for the same channels, continuing from the final state.
+Inputs are synthetic and seeded (selective_state_space_mss_b200.inputs).
+
+`value` is whole-job channel-tokens per second with inputs resident in HBM.
+With N > 1 (torchrun, one process per GPU, NCCL) every rank runs its own
+replica of the workload -- the channels are independent, so the path shards
+with no data-path collective -- and the time is the max over ranks.
+
+`--impl reference` times the fp64 CPU oracle on a bounded sample of the same
+workload (rank 0 only) and prints the same line with "impl": "reference".
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+from selective_state_space_mss_b200 import inputs as gen  # noqa: E402
+
+METRIC = "selective-scan fwd: achieved HBM GB/s (% of B200 peak) and channel-tokens/s"
+UNIT = "channel-tokens/s"
+WORKLOAD = gen.BENCH_WORKLOAD
+FALLBACK_HBM_GBS = 6650.0
+KERNEL_SOURCES = ["selective_state_space_mss_b200/csrc"]
+
+
+def log(*a):
+    print(*a, file=sys.stderr, flush=True)
+
+
+# ---------------------------------------------------------------------------
+# Algorithmic bytes: every element read or written once.
+
+def fwd_bytes(batch, dim, N, L, esz=2, z=True):
+    seq = batch * dim * L * esz
+    return (seq * (3 if z else 2)            # u, delta, z read
+            + seq                             # y written
+            + 2 * batch * N * L * esz         # B, C read once per (batch, token)
+            + dim * N * 4 + 2 * dim * 4       # A, D, bias
+            + batch * dim * N * 4)            # last_state written
+
+
+def decode_bytes(batch, dim, N, esz=2, z=True):
+    return (2 * batch * dim * N * 4           # state read + written
+            + batch * dim * esz * (4 if z else 3)  # u, delta, z read, y written
+            + 2 * batch * N * esz + dim * N * 4 + 2 * dim * 4)
+
+
+def measured_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(p) as f:
+            d = json.load(f)
+        return float(d["hbm_gbs"]), "measured"
+    except Exception:
+        return FALLBACK_HBM_GBS, "fallback"
+
+
+def kernel_source_hash():
+    h = hashlib.sha256()
+    for rel in KERNEL_SOURCES:
+        base = os.path.join(ROOT, rel)
+        for name in sorted(os.listdir(base)):
+            with open(os.path.join(base, name), "rb") as f:
+                h.update(name.encode() + b"\0" + f.read())
+    return h.hexdigest()[:16]
+
+
+def recorded_traffic():
+    """DRAM bytes per launch of the forward kernel from the committed ncu
+    summary, if it was taken on the kernel as it is now; else None."""
+    p = os.path.join(ROOT, "profiles", "scan_fwd_dram_traffic.json")
+    try:
+        with open(p) as f:
+            d = json.load(f)
+        if d.get("kernel_source_sha") == kernel_source_hash() and d.get("workload") == WORKLOAD:
+            return float(d["dram_bytes_per_launch"])
+    except Exception:
+        pass
+    return None
+
+
+# ---------------------------------------------------------------------------
+# Clocks during the timed region (nvidia-smi sampled every 200 ms).
+
+class ClockSampler:
+    QUERY = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+             "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+             "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index):
+        self.gpu = gpu_index
+        self.proc = None
+
+    def __enter__(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--id={self.gpu}", f"--query-gpu={self.QUERY}",
+                 "--format=csv,noheader,nounits", "-lms", "200"],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except Exception:
+            self.proc = None
+        return self
+
+    def __exit__(self, *exc):
+        self.out = ""
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                self.out, _ = self.proc.communicate(timeout=5)
+            except Exception:
+                self.proc.kill()
+        return False
+
+    def summary(self):
+        rows = []
+        for line in (self.out or "").splitlines():
+            parts = [p.strip() for p in line.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                rows.append(dict(sm=float(parts[1]), max=float(parts[2]), power=float(parts[3]),
+                                 hw=parts[5], hw_thermal=parts[6], sw_thermal=parts[7],
+                                 power_cap=parts[8]))
+            except ValueError:
+                continue
+        if not rows:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unsampled"], "samples": 0}
+        reasons = []
+        for key, name in [("hw", "hw_slowdown"), ("hw_thermal", "hw_thermal_slowdown"),
+                          ("sw_thermal", "sw_thermal_slowdown"), ("power_cap", "sw_power_cap")]:
+            if any(r[key].lower().startswith("active") for r in rows):
+                reasons.append(name)
+        return {"sm_mhz": statistics.median(r["sm"] for r in rows),
+                "sm_max_mhz": max(r["max"] for r in rows),
+                "power_w_max": max(r["power"] for r in rows),
+                "reasons": reasons, "samples": len(rows)}
+
+
+def physical_gpu_index(local_rank):
+    vis = os.environ.get("CUDA_VISIBLE_DEVICES")
+    if vis:
+        ids = [v.strip() for v in vis.split(",") if v.strip()]
+        if local_rank < len(ids):
+            return ids[local_rank]
+    return str(local_rank)
+
+
+# ---------------------------------------------------------------------------
+# The CPU oracle, timed (cpu_baseline and the reference arm).
+
+def oracle_sample_rate(inp, rows, nthreads):
+    """Run the oracle on the first `rows` channels of batch row 0; returns
+    (channel-tokens, seconds)."""
+    import oracle
+
+    L = inp["seqlen"]
+    t0 = time.perf_counter()
+    oracle.scan_fwd(inp["u"].values[:1, :rows], inp["delta"].values[:1, :rows], inp["A"][:rows],
+                    inp["B"].values[:1], inp["C"].values[:1], D=inp["D"][:rows],
+                    z=inp["z"].values[:1, :rows], delta_bias=inp["delta_bias"][:rows],
+                    nthreads=nthreads)
+    return rows * L, time.perf_counter() - t0
+
+
+def calibrate_rows(inp, nthreads, target_s):
+    rows = max(nthreads, 8)
+    ct, sec = oracle_sample_rate(inp, rows, nthreads)
+    per_row = sec / rows
+    return int(min(inp["dim"], max(nthreads, target_s / max(per_row, 1e-9))))
+
+
+def cpu_baseline(inp, target_s=12.0):
+    import oracle
+
+    nthreads = oracle.default_threads()
+    rows = calibrate_rows(inp, nthreads, target_s)
+    ct, sec = oracle_sample_rate(inp, rows, nthreads)
+    return {"value": ct / sec, "unit": UNIT, "cores": nthreads, "kind": "oracle",
+            "sample": f"{rows} channels x {inp['seqlen']} tokens of batch row 0 of {WORKLOAD} "
+                      f"(fp64, {nthreads} threads, {sec:.1f} s)"}
+
+
+def run_reference(args, rank):
+    if rank != 0:
+        return 0
+    import oracle
+
+    inp = gen.workload_inputs(WORKLOAD)
+    nthreads = oracle.default_threads()
+    rows = calibrate_rows(inp, nthreads, target_s=min(8.0, 150.0 / max(1, args.steps + args.warmup)))
+    for _ in range(args.warmup):
+        oracle_sample_rate(inp, rows, nthreads)
+    times = []
+    for _ in range(args.steps):
+        ct, sec = oracle_sample_rate(inp, rows, nthreads)
+        times.append(sec)
+    total = sum(times)
+    value = rows * inp["seqlen"] * args.steps / total
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": UNIT,
+        "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": 1e3 * total / args.steps, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {"workload": WORKLOAD, "sample_rows": rows, "seqlen": inp["seqlen"]},
+        "cpu_baseline": {"value": value, "unit": UNIT, "cores": nthreads, "kind": "oracle",
+                         "sample": f"{rows} channels x {inp['seqlen']} tokens per step, fp64"},
+        "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+# ---------------------------------------------------------------------------
+# The CUDA path.
+
+def run_mss(args, rank, world, local_rank):
+    import torch
+    import torch.distributed as dist
+
+    import selective_state_space_mss_b200 as mss
+    from selective_state_space_mss_b200 import build as mss_build
+
+    if not os.path.exists(mss.library_path()):
+        mss_build.build()
+    dev = torch.device("cuda", local_rank)
+    torch.cuda.set_device(dev)
+    stream = torch.cuda.current_stream(dev)
+
+    w = gen.WORKLOADS[WORKLOAD]
+    if args.seqlen:
+        import dataclasses
+
+        w = dataclasses.replace(w, seqlen=args.seqlen)
+    inp = gen.scan_inputs(w.batch, w.dim, w.dstate, w.seqlen, w.dtype, w.seed + 100 * rank, w.d_skip)
+    nxt = gen.decode_step_inputs(w.batch, w.dim, w.dstate, w.dtype, w.seed + 100 * rank, 0)
+
+    def to_dev(t):
+        return torch.from_numpy(np.ascontiguousarray(t.stored).view(np.int16)).view(torch.bfloat16).to(dev)
+
+    d = dict(u=to_dev(inp["u"]), delta=to_dev(inp["delta"]), z=to_dev(inp["z"]),
+             B=to_dev(inp["B"]), C=to_dev(inp["C"]), A=torch.from_numpy(inp["A"]).to(dev),
+             D=torch.from_numpy(inp["D"]).to(dev), delta_bias=torch.from_numpy(inp["delta_bias"]).to(dev))
+    s1 = {k: to_dev(nxt[k]) for k in ("u", "delta", "z", "B", "C")}
+    y = torch.empty_like(d["u"])
+    state = torch.empty(w.batch, w.dim, w.dstate, dtype=torch.float32, device=dev)
+    y1 = torch.empty_like(s1["u"])
+
+    def step(flags=0, ev=None):
+        if ev is not None:
+            ev[0].record(stream)
+        mss.scan_fwd(**d, y=y, last_state=state, flags=flags)
+        if ev is not None:
+            ev[1].record(stream)
+        mss.state_update(state, A=d["A"], D=d["D"], delta_bias=d["delta_bias"], y=y1, **s1)
+
+    launches_per_step = 2
+    ct_per_step = w.batch * w.dim * w.seqlen + w.batch * w.dim
+    bytes_fwd = fwd_bytes(w.batch, w.dim, w.dstate, w.seqlen)
+    bytes_step = bytes_fwd + decode_bytes(w.batch, w.dim, w.dstate)
+
+    def timed(flags, k, warm, with_clocks=False):
+        for _ in range(warm):
+            step(flags)
+        if world > 1:
+            dist.barrier()
+        torch.cuda.synchronize(dev)
+        evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(k)]
+        start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        sampler = ClockSampler(physical_gpu_index(local_rank))
+        if with_clocks:
+            sampler.__enter__()
+            time.sleep(0.3)
+        start.record(stream)
+        for i in range(k):
+            step(flags, evs[i])
+        end.record(stream)
+        torch.cuda.synchronize(dev)
+        if with_clocks:
+            sampler.__exit__(None, None, None)
+        if world > 1:
+            dist.barrier()
+        ms = start.elapsed_time(end)
+        fwd_ms = [a.elapsed_time(b) for a, b in evs]
+        if world > 1:
+            t = torch.tensor([ms], device=dev)
+            dist.all_reduce(t, op=dist.ReduceOp.MAX)
+            ms = float(t.item())
+        return ms, fwd_ms, (sampler.summary() if with_clocks else None)
+
+    assert mss.get_device_error() == 0
+    if args.kernel_only:
+        # forward launches only (used for profiling captures): no JSON line
+        for _ in range(args.warmup + args.steps):
+            mss.scan_fwd(**d, y=y, last_state=state)
+        torch.cuda.synchronize(dev)
+        assert mss.get_device_error() == 0
+        log(f"kernel-only: {args.warmup + args.steps} forward launches on {w.batch}x{w.dim}x{w.dstate}x{w.seqlen}")
+        return 0
+    # the timed run keeps the clock sampler busy for at least ~2 s
+    k_clock = args.steps
+    ms, fwd_ms, clocks = timed(0, k_clock, args.warmup, with_clocks=True)
+    assert mss.get_device_error() == 0
+    ms_gen, fwd_ms_gen, _ = timed(mss.FLAG_GENERAL_A, args.steps, args.warmup)
+
+    # end to end through the public call with host buffers: pinned host inputs,
+    # copies in, forward + decode token, results copied out, every step
+    host = {k: v.cpu().pin_memory() for k, v in d.items()}
+    host1 = {k: v.cpu().pin_memory() for k, v in s1.items()}
+    y_host = torch.empty(y.shape, dtype=y.dtype, pin_memory=True)
+    st_host = torch.empty(state.shape, dtype=state.dtype, pin_memory=True)
+    y1_host = torch.empty(y1.shape, dtype=y1.dtype, pin_memory=True)
+    h2d = sum(v.numel() * v.element_size() for v in list(host.values()) + list(host1.values()))
+    d2h = y_host.numel() * 2 + st_host.numel() * 4 + y1_host.numel() * 2
+
+    def e2e_step():
+        for k_, v in host.items():
+            d[k_].copy_(v, non_blocking=True)
+        for k_, v in host1.items():
+            s1[k_].copy_(v, non_blocking=True)
+        step(0)
+        y_host.copy_(y, non_blocking=True)
+        st_host.copy_(state, non_blocking=True)
+        y1_host.copy_(y1, non_blocking=True)
+
+    for _ in range(max(1, args.warmup)):
+        e2e_step()
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize(dev)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(args.steps):
+        e2e_step()
+    e1.record(stream)
+    torch.cuda.synchronize(dev)
+    e2e_ms = e0.elapsed_time(e1)
+    if world > 1:
+        t = torch.tensor([e2e_ms], device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        e2e_ms = float(t.item())
+    assert mss.get_device_error() == 0
+
+    # decode workload (256 x 5120 x 16 state): per-token time with L2 flushed
+    # before every timed token, since the 84 MB state would otherwise stay in L2
+    dw = gen.WORKLOADS[gen.DECODE_WORKLOAD]
+    A5, D5, b5 = (torch.from_numpy(x).to(dev) for x in gen.channel_params(dw.dim, dw.dstate, dw.d_skip, dw.seed))
+    st5 = torch.zeros(dw.batch, dw.dim, dw.dstate, device=dev)
+    steps5 = [{k: to_dev(v) for k, v in gen.decode_step_inputs(dw.batch, dw.dim, dw.dstate, dw.dtype,
+                                                              dw.seed, t).items()} for t in range(4)]
+    y5 = torch.empty(dw.batch, dw.dim, dtype=torch.bfloat16, device=dev)
+    flush = torch.empty(512 * 2 ** 20, dtype=torch.uint8, device=dev)
+    dec_ms = []
+    for t in range(args.warmup + 20):
+        flush.fill_(t & 0xff)
+        a_, b_ = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a_.record(stream)
+        mss.state_update(st5, A=A5, D=D5, delta_bias=b5, y=y5, **steps5[t % 4])
+        b_.record(stream)
+        torch.cuda.synchronize(dev)
+        if t >= args.warmup:
+            dec_ms.append(a_.elapsed_time(b_))
+    dec_med = statistics.median(dec_ms)
+    dec_bytes = decode_bytes(dw.batch, dw.dim, dw.dstate)
+
+    peak, peak_kind = measured_peaks()
+    fwd_avg = sum(fwd_ms) / len(fwd_ms)
+    fwd_avg_gen = sum(fwd_ms_gen) / len(fwd_ms_gen)
+    achieved = bytes_fwd / (fwd_avg * 1e-3) / 1e9
+    achieved_gen = bytes_fwd / (fwd_avg_gen * 1e-3) / 1e9
+    value = world * ct_per_step * args.steps / (ms * 1e-3)
+    line = {
+        "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": ms / args.steps, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f32",
+        "data": "synthetic: seeded N(0,1) u/z/B/C, delta_raw 0.1*N(0,1), log-uniform steps "
+                "[1e-3,1e-1], A=-(n+1), D~N(1,0.1); bf16 storage",
+        "config": {"workload": WORKLOAD, "batch": w.batch, "d_inner": w.dim, "dstate": w.dstate,
+                   "seqlen": w.seqlen, "io_dtype": "bf16",
+                   "step": "forward scan over all tokens + one decode token (all hot-path rows)",
+                   "l2": f"inputs larger than L2: {bytes_step / 1e6:.0f} MB of algorithmic traffic per step",
+                   "parallelism": f"replicas x{world} (channels shard with no collective)"},
+        "achieved_hbm_gbs": world * bytes_step * args.steps / (ms * 1e-3) / 1e9,
+        "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
+                     "frac": achieved / peak, "traffic": recorded_traffic(),
+                     "kernel": "scan_fwd (forward scan)", "peak_kind": peak_kind,
+                     "algorithmic_bytes_per_launch": bytes_fwd, "launch_ms_avg": fwd_avg},
+        "general_A_path": {"fwd_ms_avg": fwd_avg_gen, "achieved_gbs": achieved_gen,
+                           "frac": achieved_gen / peak,
+                           "channel_tokens_per_s": w.batch * w.dim * w.seqlen / (fwd_avg_gen * 1e-3)},
+        "decode": {"workload": gen.DECODE_WORKLOAD, "ms_per_token_median": dec_med,
+                   "achieved_gbs": dec_bytes / (dec_med * 1e-3) / 1e9,
+                   "frac": dec_bytes / (dec_med * 1e-3) / 1e9 / peak, "l2": "flushed before each token"},
+        "e2e": {"value": world * ct_per_step * args.steps / (e2e_ms * 1e-3), "unit": UNIT,
+                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
+        "gpu_launches": launches_per_step * args.steps,
+        "clocks": clocks,
+        "kernel_source_sha": kernel_source_hash(),
+    }
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        line["cpu_baseline"] = cpu_baseline(inp)
+    elif rank == 0:
+        line["cpu_baseline"] = None
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    return 0
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", choices=["mss", "reference"], default="mss")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--kernel-only", action="store_true",
+                    help="only launch the forward kernel (warmup + steps times); for profiler captures")
+    ap.add_argument("--seqlen", type=int, default=0, help="override the workload's sequence length")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        ap.error("--warmup must be at least 3")
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+    if args.impl == "reference":
+        return run_reference(args, rank)
+
+    if world > 1:
+        import datetime
+
+        import torch
+        import torch.distributed as dist
+
+        torch.cuda.set_device(local_rank)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=torch.device("cuda", local_rank))
+    try:
+        return run_mss(args, rank, world, local_rank)
+    finally:
+        if world > 1:
+            import torch.distributed as dist
+
+            dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    sys.exit(main())

@@ -1,0 +1,156 @@
+/*
+ * mss.h -- C ABI of libmss.so, the B200 (sm_100a) selective scan (S6).
+ *
+ * The library computes, per channel d of batch row b and token t, a diagonal
+ * real state-space model discretised per token:
+ *
+ *   Delta_t  = softplus(delta[b,d,t] + delta_bias[d])   (or without softplus)
+ *   Abar_t,n = exp(Delta_t * A[d,n])                     zero-order hold
+ *   h_t,n    = Abar_t,n * h_{t-1},n + Delta_t * B[b,n,t] * u[b,d,t]
+ *   y[b,d,t] = (sum_n C[b,n,t] * h_t,n + D[d] * u[b,d,t]) * silu(z[b,d,t])
+ *
+ * with h_{-1} = 0 and silu(z) = z / (1 + e^{-z}).  Sources: the continuous
+ * SSM, the zero-order-hold transition exp(Delta A) and the discrete
+ * recurrence ("Mamba" paper review, section "SSM"); token-dependent B, C and
+ * step ("Mamba" paper review, section "Selection Mechanism"); softplus for the
+ * step ("Exercises -- State-space models (Mamba, S4)", softplus exercise);
+ * the Euler input rule Bbar = Delta B, listed beside zero-order hold on the
+ * "Paper: Mamba" course page (Objectives, Math & data structures); the gate
+ * and skip term of the block ("Mamba" paper review, section "SSM", block
+ * description; the pages print no formula for them, the form above is the
+ * library's definition).
+ *
+ * Conventions shared by every entry point:
+ *   - Every tensor pointer is a DEVICE pointer owned by the caller, C-contiguous
+ *     in the layout given below.  The library never allocates memory on the
+ *     forward or decode path and never frees caller memory.
+ *   - Work is enqueued on `stream` (a cudaStream_t passed as void*; NULL means
+ *     the legacy default stream) and is asynchronous: a return of MSS_OK means
+ *     the launch was accepted, not that it has finished.
+ *   - Argument errors are detected on the host before any launch; the outputs
+ *     are then left untouched.
+ *   - Optional pointers: z == NULL means no gate, D == NULL means D = 0,
+ *     delta_bias == NULL means bias 0, last_state == NULL means not written.
+ *   - `dtype` selects the element type of u, delta, z, B, C and y:
+ *     MSS_DTYPE_F32 (float) or MSS_DTYPE_BF16 (bfloat16, round-to-nearest-even
+ *     on store).  A, D, delta_bias, last_state and the decode state are always
+ *     float.  All arithmetic is fp32.
+ *   - dstate (N) must be 1, 2, 4, 8 or 16.
+ *   - Outputs must not overlap inputs (the decode state is in/out by design).
+ *   - Thread safety: the library keeps no host state besides a per-device,
+ *     lazily resolved driver entry point; calls from several host threads are
+ *     safe.
+ */
+#ifndef MSS_H
+#define MSS_H
+
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define MSS_API __attribute__((visibility("default")))
+#else
+#define MSS_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#define MSS_VERSION 10000 /* major*10000 + minor*100 + patch: 1.0.0 */
+
+enum mss_dtype {
+    MSS_DTYPE_F32 = 0,
+    MSS_DTYPE_BF16 = 1
+};
+
+enum mss_status {
+    MSS_OK = 0,
+    MSS_ERR_NULL = -1,           /* a required pointer is NULL */
+    MSS_ERR_SHAPE = -2,          /* a size is negative, or a size product overflows int64 */
+    MSS_ERR_UNSUPPORTED_N = -3,  /* dstate is not 1, 2, 4, 8 or 16 */
+    MSS_ERR_DTYPE = -4,          /* dtype is not an mss_dtype */
+    MSS_ERR_ALIGN = -5,          /* a pointer is not aligned to its element size */
+    MSS_ERR_CUDA = -6,           /* a CUDA call failed (launch or device query) */
+    MSS_ERR_DEVICE_TIMEOUT = -7, /* a bounded wait inside a kernel gave up */
+    MSS_ERR_FLAGS = -8,          /* unknown bits in `flags` */
+    MSS_ERR_ALIAS = -9           /* an output overlaps an input */
+};
+
+/* Flags of mss_scan_fwd_ex. */
+#define MSS_FLAG_GENERAL_A 0x1u /* never use the fast path for A[d,n] = (n+1)*A[d,0] */
+#define MSS_FLAG_SIMPLE 0x2u    /* run the one-thread-per-channel reference kernel */
+
+/*
+ * mss_scan_fwd -- selective-scan forward pass over whole sequences.
+ *
+ *   u, delta, z : [batch][dim][seqlen]  dtype     (z may be NULL)
+ *   A           : [dim][dstate]         float     (negative for a stable system)
+ *   B, C        : [batch][dstate][seqlen] dtype   (shared by all channels of a row)
+ *   D, delta_bias: [dim]                float     (each may be NULL)
+ *   softplus_flag: nonzero -> Delta = softplus(delta + bias), else delta + bias
+ *   y           : [batch][dim][seqlen]  dtype     output
+ *   last_state  : [batch][dim][dstate]  float     output h_{seqlen-1} (may be NULL)
+ *
+ * Any seqlen >= 0 works (a ragged tail is masked); seqlen == 0 writes
+ * last_state = 0 and then u, delta, z, B, C and y may be NULL.  batch * dim == 0 launches nothing.  The fp32 state stays
+ * on chip; only last_state is written.  Any pointer alignment that matches
+ * the element size is accepted: 16-byte aligned rows take the vectorised
+ * kernel, others a scalar one.
+ *
+ * Returns MSS_OK or a negative mss_status.
+ */
+MSS_API int mss_scan_fwd(const void *u, const void *delta, const float *A, const void *B,
+                 const void *C, const float *D, const void *z, const float *delta_bias,
+                 int softplus_flag, void *y, float *last_state,
+                 int64_t batch, int64_t dim, int64_t dstate, int64_t seqlen,
+                 int dtype, void *stream);
+
+/* mss_scan_fwd with `flags` (MSS_FLAG_*): the same computation, with a choice
+ * of kernel for testing and measurement.  flags == 0 is mss_scan_fwd. */
+MSS_API int mss_scan_fwd_ex(const void *u, const void *delta, const float *A, const void *B,
+                    const void *C, const float *D, const void *z, const float *delta_bias,
+                    int softplus_flag, void *y, float *last_state,
+                    int64_t batch, int64_t dim, int64_t dstate, int64_t seqlen,
+                    int dtype, unsigned flags, void *stream);
+
+/*
+ * mss_state_update -- one decode token for every (batch, channel):
+ * the recurrence above applied once to a caller-held state
+ * (the generation-time view of "Exercises -- State-space models (Mamba, S4)":
+ * O(1) work and O(N) memory per token).
+ *
+ *   state       : [batch][dim][dstate] float, read and overwritten in place
+ *   u, delta, z : [batch][dim]         dtype (z may be NULL)
+ *   A           : [dim][dstate]        float
+ *   B, C        : [batch][dstate]      dtype
+ *   D, delta_bias: [dim]               float (each may be NULL)
+ *   y           : [batch][dim]         dtype output
+ *
+ * Returns MSS_OK or a negative mss_status.
+ */
+MSS_API int mss_state_update(float *state, const void *u, const void *delta, const float *A,
+                     const void *B, const void *C, const float *D, const void *z,
+                     const float *delta_bias, int softplus_flag, void *y,
+                     int64_t batch, int64_t dim, int64_t dstate, int dtype, void *stream);
+
+/*
+ * mss_get_device_error -- synchronises `stream`, then reports and clears the
+ * device error word that kernels set when a bounded wait gives up
+ * (MSS_ERR_DEVICE_TIMEOUT), or MSS_ERR_CUDA if the stream itself reports an
+ * error.  Returns MSS_OK when neither happened.  The error word is one
+ * word of device memory per device, defined in the library image; nothing
+ * is allocated.
+ */
+MSS_API int mss_get_device_error(void *stream);
+
+/* Human-readable text for a status code (static storage, never NULL). */
+MSS_API const char *mss_strerror(int code);
+
+/* MSS_VERSION of the library that was loaded. */
+MSS_API int mss_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* MSS_H */

@@ -1,1 +1,192 @@
-"""B200-native selective scan (S6): CUDA library + thin Python binding."""
+"""B200-native selective scan (S6): thin Python binding over libmss.so.
+
+Argument marshalling only.  Every step of the forward pass and of the decode
+update runs in the CUDA kernels of libmss.so; PyTorch supplies device memory
+and streams.  There is no fallback: if the library is missing or a tensor is
+not on a CUDA device, the call raises.
+
+    y, last_state = scan_fwd(u, delta, A, B, C, D=D, z=z, delta_bias=bias)
+    y = state_update(state, u, delta, A, B, C, D=D, z=z, delta_bias=bias)
+
+Layouts (C-contiguous): u, delta, z, y [batch, dim, L]; B, C [batch, N, L];
+A [dim, N] float32; D, delta_bias [dim] float32; last_state [batch, dim, N]
+float32.  Decode: state [batch, dim, N] float32 (updated in place); u, delta,
+z, y [batch, dim]; B, C [batch, N].  u, delta, z, B, C share one dtype,
+float32 or bfloat16, which is also the dtype of y.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import threading
+
+import torch
+
+__all__ = ["scan_fwd", "state_update", "get_device_error", "library_path",
+           "FLAG_GENERAL_A", "FLAG_SIMPLE", "MssError", "load_library"]
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+_LIB_PATH = os.path.join(_HERE, "libmss.so")
+
+DTYPE_F32 = 0
+DTYPE_BF16 = 1
+FLAG_GENERAL_A = 0x1
+FLAG_SIMPLE = 0x2
+
+_lib = None
+_lock = threading.Lock()
+
+
+class MssError(RuntimeError):
+    def __init__(self, code: int, what: str):
+        self.code = code
+        super().__init__(f"{what} failed: {_strerror(code)} (code {code})")
+
+
+def library_path() -> str:
+    return _LIB_PATH
+
+
+def load_library():
+    """Load libmss.so (built in-tree by __graft_entry__.build() or
+    ``python -m selective_state_space_mss_b200.build``)."""
+    global _lib
+    with _lock:
+        if _lib is None:
+            if not os.path.exists(_LIB_PATH):
+                raise RuntimeError(
+                    f"{_LIB_PATH} is not built; run `python -m selective_state_space_mss_b200.build`")
+            lib = ctypes.CDLL(_LIB_PATH)
+            vp, fp, i64, i, u32 = (ctypes.c_void_p, ctypes.c_void_p, ctypes.c_int64,
+                                   ctypes.c_int, ctypes.c_uint)
+            lib.mss_scan_fwd_ex.argtypes = [vp, vp, fp, vp, vp, fp, vp, fp, i, vp, fp,
+                                            i64, i64, i64, i64, i, u32, vp]
+            lib.mss_scan_fwd_ex.restype = i
+            lib.mss_scan_fwd.argtypes = [vp, vp, fp, vp, vp, fp, vp, fp, i, vp, fp,
+                                         i64, i64, i64, i64, i, vp]
+            lib.mss_scan_fwd.restype = i
+            lib.mss_state_update.argtypes = [fp, vp, vp, fp, vp, vp, fp, vp, fp, i, vp,
+                                             i64, i64, i64, i, vp]
+            lib.mss_state_update.restype = i
+            lib.mss_get_device_error.argtypes = [vp]
+            lib.mss_get_device_error.restype = i
+            lib.mss_strerror.argtypes = [i]
+            lib.mss_strerror.restype = ctypes.c_char_p
+            lib.mss_version.argtypes = []
+            lib.mss_version.restype = i
+            _lib = lib
+    return _lib
+
+
+def _strerror(code: int) -> str:
+    return load_library().mss_strerror(int(code)).decode()
+
+
+def _ptr(t):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _check(t, name, shape, dtype, device, optional=False):
+    if t is None:
+        if optional:
+            return
+        raise ValueError(f"{name} is required")
+    if not isinstance(t, torch.Tensor):
+        raise TypeError(f"{name} must be a torch.Tensor")
+    if t.device != device:
+        raise ValueError(f"{name} is on {t.device}, expected {device}")
+    if t.dtype != dtype:
+        raise TypeError(f"{name} has dtype {t.dtype}, expected {dtype}")
+    if tuple(t.shape) != tuple(shape):
+        raise ValueError(f"{name} has shape {tuple(t.shape)}, expected {tuple(shape)}")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+
+
+def _io_dtype(t):
+    if t.dtype == torch.float32:
+        return DTYPE_F32
+    if t.dtype == torch.bfloat16:
+        return DTYPE_BF16
+    raise TypeError(f"unsupported dtype {t.dtype}: use torch.float32 or torch.bfloat16")
+
+
+def _stream_handle(stream, device):
+    s = torch.cuda.current_stream(device) if stream is None else stream
+    return ctypes.c_void_p(s.cuda_stream)
+
+
+def scan_fwd(u, delta, A, B, C, D=None, z=None, delta_bias=None, softplus=True,
+             y=None, last_state=None, want_last_state=True, flags=0, stream=None):
+    """Selective-scan forward pass (mss_scan_fwd_ex).  Returns (y, last_state);
+    last_state is None when want_last_state is False and none was given."""
+    if not isinstance(u, torch.Tensor) or u.device.type != "cuda":
+        raise ValueError("u must be a CUDA tensor (there is no CPU path)")
+    if u.dim() != 3:
+        raise ValueError("u must be [batch, dim, L]")
+    batch, dim, L = u.shape
+    dev, dt = u.device, u.dtype
+    code = _io_dtype(u)
+    if A.dim() != 2:
+        raise ValueError("A must be [dim, N]")
+    N = A.shape[1]
+    _check(u, "u", (batch, dim, L), dt, dev)
+    _check(delta, "delta", (batch, dim, L), dt, dev)
+    _check(A, "A", (dim, N), torch.float32, dev)
+    _check(B, "B", (batch, N, L), dt, dev)
+    _check(C, "C", (batch, N, L), dt, dev)
+    _check(D, "D", (dim,), torch.float32, dev, optional=True)
+    _check(z, "z", (batch, dim, L), dt, dev, optional=True)
+    _check(delta_bias, "delta_bias", (dim,), torch.float32, dev, optional=True)
+    if y is None:
+        y = torch.empty((batch, dim, L), dtype=dt, device=dev)
+    _check(y, "y", (batch, dim, L), dt, dev)
+    if last_state is None and want_last_state:
+        last_state = torch.empty((batch, dim, N), dtype=torch.float32, device=dev)
+    _check(last_state, "last_state", (batch, dim, N), torch.float32, dev, optional=True)
+    rc = load_library().mss_scan_fwd_ex(
+        _ptr(u), _ptr(delta), _ptr(A), _ptr(B), _ptr(C), _ptr(D), _ptr(z), _ptr(delta_bias),
+        int(bool(softplus)), _ptr(y), _ptr(last_state), batch, dim, N, L, code,
+        int(flags), _stream_handle(stream, dev))
+    if rc != 0:
+        raise MssError(rc, "mss_scan_fwd")
+    return y, last_state
+
+
+def state_update(state, u, delta, A, B, C, D=None, z=None, delta_bias=None, softplus=True,
+                 y=None, stream=None):
+    """One decode token (mss_state_update); `state` is updated in place.
+    Returns y [batch, dim]."""
+    if not isinstance(state, torch.Tensor) or state.device.type != "cuda":
+        raise ValueError("state must be a CUDA tensor (there is no CPU path)")
+    if state.dim() != 3:
+        raise ValueError("state must be [batch, dim, N]")
+    batch, dim, N = state.shape
+    dev, dt = state.device, u.dtype
+    code = _io_dtype(u)
+    _check(state, "state", (batch, dim, N), torch.float32, dev)
+    _check(u, "u", (batch, dim), dt, dev)
+    _check(delta, "delta", (batch, dim), dt, dev)
+    _check(A, "A", (dim, N), torch.float32, dev)
+    _check(B, "B", (batch, N), dt, dev)
+    _check(C, "C", (batch, N), dt, dev)
+    _check(D, "D", (dim,), torch.float32, dev, optional=True)
+    _check(z, "z", (batch, dim), dt, dev, optional=True)
+    _check(delta_bias, "delta_bias", (dim,), torch.float32, dev, optional=True)
+    if y is None:
+        y = torch.empty((batch, dim), dtype=dt, device=dev)
+    _check(y, "y", (batch, dim), dt, dev)
+    rc = load_library().mss_state_update(
+        _ptr(state), _ptr(u), _ptr(delta), _ptr(A), _ptr(B), _ptr(C), _ptr(D), _ptr(z),
+        _ptr(delta_bias), int(bool(softplus)), _ptr(y), batch, dim, N, code,
+        _stream_handle(stream, dev))
+    if rc != 0:
+        raise MssError(rc, "mss_state_update")
+    return y
+
+
+def get_device_error(stream=None, device=None) -> int:
+    """Synchronise the stream and return (and clear) the library's device
+    error status: 0, or a negative mss_status code."""
+    dev = torch.device("cuda", torch.cuda.current_device()) if device is None else device
+    return int(load_library().mss_get_device_error(_stream_handle(stream, dev)))

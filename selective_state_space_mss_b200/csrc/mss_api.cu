@@ -1,0 +1,316 @@
+// mss_api.cu -- the C ABI of libmss.so (declared in include/mss.h): argument
+// checks on the host, kernel choice, launches.  No allocation, no host
+// synchronisation on the forward and decode paths.
+#include <cstdint>
+#include <cstring>
+#include <mutex>
+#include <type_traits>
+
+#include <cuda.h>
+#include <cudaTypedefs.h>
+#include <cuda_runtime.h>
+
+#include "../../include/mss.h"
+#include "mss_device.cuh"
+#include "mss_params.h"
+#include "scan_seq.cuh"
+#include "scan_simple.cuh"
+#include "state_update.cuh"
+
+namespace {
+
+using mss::bf16_t;
+
+inline bool mul_ok(int64_t a, int64_t b, int64_t* out) { return !__builtin_mul_overflow(a, b, out); }
+
+inline bool aligned(const void* p, size_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
+
+inline bool valid_n(int64_t n) { return n == 1 || n == 2 || n == 4 || n == 8 || n == 16; }
+
+// [p, p + bytes) and [q, q + qbytes) overlap (null or empty ranges never do)
+inline bool overlaps(const void* p, int64_t bytes, const void* q, int64_t qbytes) {
+    if (!p || !q || bytes <= 0 || qbytes <= 0) return false;
+    const uintptr_t a = reinterpret_cast<uintptr_t>(p), b = reinterpret_cast<uintptr_t>(q);
+    return a < b + uint64_t(qbytes) && b < a + uint64_t(bytes);
+}
+
+// Dispatch on N: calls f(std::integral_constant<int, N>).
+template <typename F>
+int with_n(int64_t n, F&& f) {
+    switch (n) {
+        case 1: return f(std::integral_constant<int, 1>{});
+        case 2: return f(std::integral_constant<int, 2>{});
+        case 4: return f(std::integral_constant<int, 4>{});
+        case 8: return f(std::integral_constant<int, 8>{});
+        case 16: return f(std::integral_constant<int, 16>{});
+        default: return MSS_ERR_UNSUPPORTED_N;
+    }
+}
+
+inline int launch_status() { return cudaGetLastError() == cudaSuccess ? MSS_OK : MSS_ERR_CUDA; }
+
+// cuTensorMapEncodeTiled, resolved once through the runtime so that the
+// library does not link the driver library itself.
+PFN_cuTensorMapEncodeTiled_v12000 encode_tiled_fn() {
+    static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+    static std::once_flag once;
+    std::call_once(once, [] {
+        void* f = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &f, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(f);
+    });
+    return fn;
+}
+
+// [rows, L] row-major view, box = 32 rows x 128 bytes, 128-byte swizzle.
+bool encode_rows(CUtensorMap* m, const void* base, int64_t rows, int64_t L, int esz) {
+    auto enc = encode_tiled_fn();
+    if (!enc) return false;
+    const cuuint64_t dims[2] = {cuuint64_t(L), cuuint64_t(rows)};
+    const cuuint64_t strides[1] = {cuuint64_t(L * esz)};
+    const cuuint32_t box[2] = {cuuint32_t(128 / esz), 32u};
+    const cuuint32_t estr[2] = {1u, 1u};
+    return enc(m, esz == 2 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 2,
+               const_cast<void*>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+               CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+// [batch, N, L] view, box = 1 x N x 128 bytes, no swizzle.
+bool encode_bc(CUtensorMap* m, const void* base, int64_t batch, int64_t N, int64_t L, int esz) {
+    auto enc = encode_tiled_fn();
+    if (!enc) return false;
+    const cuuint64_t dims[3] = {cuuint64_t(L), cuuint64_t(N), cuuint64_t(batch)};
+    const cuuint64_t strides[2] = {cuuint64_t(L * esz), cuuint64_t(N * L * esz)};
+    const cuuint32_t box[3] = {cuuint32_t(128 / esz), cuuint32_t(N), 1u};
+    const cuuint32_t estr[3] = {1u, 1u, 1u};
+    return enc(m, esz == 2 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 3,
+               const_cast<void*>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+               CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+template <typename T, int N>
+int launch_simple(const mss::ScanParams& p, cudaStream_t stream) {
+    const int64_t rows = p.batch * p.dim;
+    const int threads = 128;
+    const int64_t blocks = (rows + threads - 1) / threads;
+    if (blocks > 0x7fffffffLL) return MSS_ERR_SHAPE;
+    mss::scan_fwd_simple_kernel<T, N><<<dim3(unsigned(blocks)), threads, 0, stream>>>(p);
+    return launch_status();
+}
+
+// The throughput kernel's requirements; otherwise the scalar kernel runs.
+bool seq_eligible(const mss::ScanParams& p, int64_t N, int esz, unsigned flags) {
+    if (flags & MSS_FLAG_SIMPLE) return false;
+    if (N != 4 && N != 8 && N != 16) return false;
+    if ((p.seqlen * esz) % 16 != 0) return false;
+    if (p.batch * p.dim >= (int64_t(1) << 31) || p.seqlen >= (int64_t(1) << 31)) return false;
+    if ((p.dim + 31) / 32 > 0x7fffffffLL || p.batch > 65535) return false;
+    const void* v[] = {p.u, p.delta, p.z, p.B, p.C, p.y, p.last_state};
+    for (const void* q : v)
+        if (q && !aligned(q, 16)) return false;
+    return true;
+}
+
+template <typename T, int N, bool kGate, bool kSoftplus>
+int launch_seq_variant(const mss::SeqMaps& maps, const mss::ScanParams& p, unsigned flags, cudaStream_t stream) {
+    auto kern = mss::scan_fwd_seq_kernel<T, N, kGate, kSoftplus>;
+    const int smem = mss::SeqLayout<T, N>::kSmemBytes;
+    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess)
+        return MSS_ERR_CUDA;
+    const dim3 grid(unsigned((p.dim + 31) / 32), unsigned(p.batch));
+    kern<<<grid, 32, smem, stream>>>(maps, p, (flags & MSS_FLAG_GENERAL_A) ? 0 : 1);
+    return launch_status();
+}
+
+template <typename T, int N>
+int launch_seq(const mss::ScanParams& p, unsigned flags, cudaStream_t stream) {
+    constexpr int esz = int(sizeof(T));
+    mss::SeqMaps maps;
+    std::memset(&maps, 0, sizeof(maps));
+    const int64_t rows = p.batch * p.dim;
+    if (!encode_rows(&maps.u, p.u, rows, p.seqlen, esz) || !encode_rows(&maps.delta, p.delta, rows, p.seqlen, esz) ||
+        (p.z && !encode_rows(&maps.z, p.z, rows, p.seqlen, esz)) ||
+        !encode_bc(&maps.B, p.B, p.batch, N, p.seqlen, esz) || !encode_bc(&maps.C, p.C, p.batch, N, p.seqlen, esz))
+        return MSS_ERR_CUDA;
+    if (p.z)
+        return p.softplus ? launch_seq_variant<T, N, true, true>(maps, p, flags, stream)
+                          : launch_seq_variant<T, N, true, false>(maps, p, flags, stream);
+    return p.softplus ? launch_seq_variant<T, N, false, true>(maps, p, flags, stream)
+                      : launch_seq_variant<T, N, false, false>(maps, p, flags, stream);
+}
+
+template <typename T, int N>
+int launch_scan(const mss::ScanParams& p, unsigned flags, cudaStream_t stream) {
+    if constexpr (N == 4 || N == 8 || N == 16) {
+        if (seq_eligible(p, N, int(sizeof(T)), flags)) return launch_seq<T, N>(p, flags, stream);
+    }
+    return launch_simple<T, N>(p, stream);
+}
+
+}  // namespace
+
+extern "C" {
+
+int mss_version(void) { return MSS_VERSION; }
+
+const char* mss_strerror(int code) {
+    switch (code) {
+        case MSS_OK: return "success";
+        case MSS_ERR_NULL: return "a required pointer is NULL";
+        case MSS_ERR_SHAPE: return "a size is negative or a size product overflows";
+        case MSS_ERR_UNSUPPORTED_N: return "dstate must be 1, 2, 4, 8 or 16";
+        case MSS_ERR_DTYPE: return "dtype must be MSS_DTYPE_F32 or MSS_DTYPE_BF16";
+        case MSS_ERR_ALIGN: return "a pointer is not aligned to its element size";
+        case MSS_ERR_CUDA: return "a CUDA call failed";
+        case MSS_ERR_DEVICE_TIMEOUT: return "a bounded wait inside a kernel gave up";
+        case MSS_ERR_FLAGS: return "unknown bits in flags";
+        case MSS_ERR_ALIAS: return "an output overlaps an input";
+        default: return "unknown status code";
+    }
+}
+
+int mss_scan_fwd_ex(const void* u, const void* delta, const float* A, const void* B,
+                    const void* C, const float* D, const void* z, const float* delta_bias,
+                    int softplus_flag, void* y, float* last_state,
+                    int64_t batch, int64_t dim, int64_t dstate, int64_t seqlen,
+                    int dtype, unsigned flags, void* stream) {
+    if (dtype != MSS_DTYPE_F32 && dtype != MSS_DTYPE_BF16) return MSS_ERR_DTYPE;
+    if (flags & ~(MSS_FLAG_GENERAL_A | MSS_FLAG_SIMPLE)) return MSS_ERR_FLAGS;
+    if (batch < 0 || dim < 0 || seqlen < 0) return MSS_ERR_SHAPE;
+    if (!valid_n(dstate)) return MSS_ERR_UNSUPPORTED_N;
+    const int64_t esz = dtype == MSS_DTYPE_BF16 ? 2 : 4;
+    int64_t rows, seq_elems, seq_bytes, bc_elems, bc_bytes, st_elems, st_bytes;
+    if (!mul_ok(batch, dim, &rows) || !mul_ok(rows, seqlen, &seq_elems) ||
+        !mul_ok(seq_elems, esz, &seq_bytes) || !mul_ok(batch * dstate, seqlen, &bc_elems) ||
+        !mul_ok(bc_elems, esz, &bc_bytes) || !mul_ok(rows, dstate, &st_elems) ||
+        !mul_ok(st_elems, 4, &st_bytes) || rows > (int64_t(1) << 40))
+        return MSS_ERR_SHAPE;
+    if (rows == 0) return MSS_OK;
+    // with no tokens the sequence tensors are empty and may be NULL
+    if (!A || (seqlen > 0 && (!u || !delta || !B || !C || !y))) return MSS_ERR_NULL;
+    const void* io[] = {u, delta, B, C, z, y};
+    for (const void* p : io)
+        if (p && !aligned(p, size_t(esz))) return MSS_ERR_ALIGN;
+    const void* fp[] = {A, D, delta_bias, last_state};
+    for (const void* p : fp)
+        if (p && !aligned(p, 4)) return MSS_ERR_ALIGN;
+    // outputs must not overlap inputs
+    const void* in_seq[] = {u, delta, z};
+    for (const void* p : in_seq)
+        if (overlaps(y, seq_bytes, p, seq_bytes) || overlaps(last_state, st_bytes, p, seq_bytes))
+            return MSS_ERR_ALIAS;
+    const void* in_bc[] = {B, C};
+    for (const void* p : in_bc)
+        if (overlaps(y, seq_bytes, p, bc_bytes) || overlaps(last_state, st_bytes, p, bc_bytes))
+            return MSS_ERR_ALIAS;
+    const int64_t n_param_bytes = dim * 4;
+    const void* params[] = {D, delta_bias};
+    for (const void* p : params)
+        if (overlaps(y, seq_bytes, p, n_param_bytes) || overlaps(last_state, st_bytes, p, n_param_bytes))
+            return MSS_ERR_ALIAS;
+    if (overlaps(y, seq_bytes, A, dim * dstate * 4) || overlaps(last_state, st_bytes, A, dim * dstate * 4) ||
+        overlaps(y, seq_bytes, last_state, st_bytes))
+        return MSS_ERR_ALIAS;
+
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    if (seqlen == 0) {
+        if (last_state && cudaMemsetAsync(last_state, 0, size_t(st_bytes), s) != cudaSuccess)
+            return MSS_ERR_CUDA;
+        return MSS_OK;
+    }
+    mss::ScanParams p{u, delta, A, B, C, D, z, delta_bias, y, last_state,
+                      batch, dim, seqlen, softplus_flag ? 1 : 0};
+    return with_n(dstate, [&](auto nc) {
+        constexpr int N = decltype(nc)::value;
+        return dtype == MSS_DTYPE_BF16 ? launch_scan<bf16_t, N>(p, flags, s)
+                                       : launch_scan<float, N>(p, flags, s);
+    });
+}
+
+int mss_scan_fwd(const void* u, const void* delta, const float* A, const void* B,
+                 const void* C, const float* D, const void* z, const float* delta_bias,
+                 int softplus_flag, void* y, float* last_state,
+                 int64_t batch, int64_t dim, int64_t dstate, int64_t seqlen,
+                 int dtype, void* stream) {
+    return mss_scan_fwd_ex(u, delta, A, B, C, D, z, delta_bias, softplus_flag, y, last_state,
+                           batch, dim, dstate, seqlen, dtype, 0u, stream);
+}
+
+int mss_state_update(float* state, const void* u, const void* delta, const float* A,
+                     const void* B, const void* C, const float* D, const void* z,
+                     const float* delta_bias, int softplus_flag, void* y,
+                     int64_t batch, int64_t dim, int64_t dstate, int dtype, void* stream) {
+    if (dtype != MSS_DTYPE_F32 && dtype != MSS_DTYPE_BF16) return MSS_ERR_DTYPE;
+    if (batch < 0 || dim < 0) return MSS_ERR_SHAPE;
+    if (!valid_n(dstate)) return MSS_ERR_UNSUPPORTED_N;
+    const int64_t esz = dtype == MSS_DTYPE_BF16 ? 2 : 4;
+    int64_t rows, st_elems, st_bytes;
+    if (!mul_ok(batch, dim, &rows) || !mul_ok(rows, dstate, &st_elems) ||
+        !mul_ok(st_elems, 4, &st_bytes) || rows > (int64_t(1) << 40))
+        return MSS_ERR_SHAPE;
+    if (rows == 0) return MSS_OK;
+    if (!state || !u || !delta || !A || !B || !C || !y) return MSS_ERR_NULL;
+    const void* io[] = {u, delta, B, C, z, y};
+    for (const void* p : io)
+        if (p && !aligned(p, size_t(esz))) return MSS_ERR_ALIGN;
+    const void* fp[] = {state, A, D, delta_bias};
+    for (const void* p : fp)
+        if (p && !aligned(p, 4)) return MSS_ERR_ALIGN;
+    const int64_t io_bytes = rows * esz, bc_bytes = batch * dstate * esz;
+    const void* in_io[] = {u, delta, z};
+    for (const void* p : in_io)
+        if (overlaps(y, io_bytes, p, io_bytes) || overlaps(state, st_bytes, p, io_bytes)) return MSS_ERR_ALIAS;
+    const void* in_bc[] = {B, C};
+    for (const void* p : in_bc)
+        if (overlaps(y, io_bytes, p, bc_bytes) || overlaps(state, st_bytes, p, bc_bytes)) return MSS_ERR_ALIAS;
+    const void* params[] = {D, delta_bias};
+    for (const void* p : params)
+        if (overlaps(y, io_bytes, p, dim * 4) || overlaps(state, st_bytes, p, dim * 4)) return MSS_ERR_ALIAS;
+    if (overlaps(y, io_bytes, A, dim * dstate * 4) || overlaps(state, st_bytes, A, dim * dstate * 4) ||
+        overlaps(y, io_bytes, state, st_bytes))
+        return MSS_ERR_ALIAS;
+
+    mss::StepParams p{state, u, delta, A, B, C, D, z, delta_bias, y, batch, dim, softplus_flag ? 1 : 0};
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    const bool vec = aligned(state, 16) && aligned(A, 16);
+    return with_n(dstate, [&](auto nc) {
+        constexpr int N = decltype(nc)::value;
+        constexpr int TPC = N < 4 ? 1 : N / 4;
+        const int threads = 256;
+        const int64_t blocks = (rows * TPC + threads - 1) / threads;
+        if (blocks > 0x7fffffffLL) return int(MSS_ERR_SHAPE);
+        auto go = [&](auto kern) {
+            kern<<<dim3(unsigned(blocks)), threads, 0, s>>>(p);
+            return launch_status();
+        };
+        if (dtype == MSS_DTYPE_BF16)
+            return vec ? go(mss::state_update_kernel<bf16_t, N, true>)
+                       : go(mss::state_update_kernel<bf16_t, N, false>);
+        return vec ? go(mss::state_update_kernel<float, N, true>)
+                   : go(mss::state_update_kernel<float, N, false>);
+    });
+}
+
+int mss_get_device_error(void* stream) {
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    if (cudaStreamSynchronize(s) != cudaSuccess) return MSS_ERR_CUDA;
+    unsigned int word = 0, zero = 0;
+    if (cudaMemcpyFromSymbolAsync(&word, mss::g_mss_device_error, sizeof(word), 0,
+                                  cudaMemcpyDeviceToHost, s) != cudaSuccess)
+        return MSS_ERR_CUDA;
+    if (cudaStreamSynchronize(s) != cudaSuccess) return MSS_ERR_CUDA;
+    if (word != 0) {
+        if (cudaMemcpyToSymbolAsync(mss::g_mss_device_error, &zero, sizeof(zero), 0,
+                                    cudaMemcpyHostToDevice, s) != cudaSuccess ||
+            cudaStreamSynchronize(s) != cudaSuccess)
+            return MSS_ERR_CUDA;
+        return MSS_ERR_DEVICE_TIMEOUT;
+    }
+    return MSS_OK;
+}
+
+}  // extern "C"

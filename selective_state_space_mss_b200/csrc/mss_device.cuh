@@ -1,0 +1,118 @@
+// mss_device.cuh -- device-side helpers shared by the selective-scan kernels:
+// element loads/stores for float and bf16, the step-size and gate functions,
+// and thin wrappers over single sm_100a instructions.
+#pragma once
+
+#include <cstdint>
+#include <cuda_runtime.h>
+
+namespace mss {
+
+// ---------------------------------------------------------------------------
+// Element types.  bf16 travels as its 16-bit pattern; widening is exact
+// (the pattern is the top half of an fp32), narrowing rounds to nearest even
+// with the hardware conversion instruction.
+
+struct bf16_t {
+    uint16_t bits;
+};
+
+__device__ __forceinline__ float to_f32(float x) { return x; }
+__device__ __forceinline__ float to_f32(bf16_t x) { return __uint_as_float(uint32_t(x.bits) << 16); }
+
+template <typename T> __device__ __forceinline__ T from_f32(float x);
+template <> __device__ __forceinline__ float from_f32<float>(float x) { return x; }
+template <> __device__ __forceinline__ bf16_t from_f32<bf16_t>(float x) {
+    uint16_t r;
+    asm("cvt.rn.bf16.f32 %0, %1;" : "=h"(r) : "f"(x));
+    return bf16_t{r};
+}
+
+// Two fp32 values -> one 32-bit word of two bf16 (lo in the low half).
+__device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
+    uint32_t r;
+    asm("cvt.rn.bf16x2.f32 %0, %1, %2;" : "=r"(r) : "f"(hi), "f"(lo));
+    return r;
+}
+__device__ __forceinline__ float bf16_lo(uint32_t w) { return __uint_as_float(w << 16); }
+__device__ __forceinline__ float bf16_hi(uint32_t w) { return __uint_as_float(w & 0xffff0000u); }
+
+template <typename T> __device__ __forceinline__ float ld(const T* p) { return to_f32(*p); }
+
+// ---------------------------------------------------------------------------
+// Single-instruction approximations (MUFU).  Their accuracy is the PTX ISA's
+// documented bound for each instruction; callers that need the full-precision
+// library function use expf / log1pf instead.
+
+__device__ __forceinline__ float ex2_approx(float x) {
+    float r;
+    asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(r) : "f"(x));
+    return r;
+}
+__device__ __forceinline__ float rcp_approx(float x) {
+    float r;
+    asm("rcp.approx.ftz.f32 %0, %1;" : "=f"(r) : "f"(x));
+    return r;
+}
+
+constexpr float kLog2e = 1.4426950408889634f;  // 1 / ln 2
+
+// ---------------------------------------------------------------------------
+// Step size and gate.
+//
+// softplus(s) = ln(1 + e^s) ("Exercises -- State-space models (Mamba, S4)",
+// softplus exercise).  Above s = 20 the correction ln(1 + e^{-s}) < 2.1e-9 is
+// below half an ulp of s in fp32, so s itself is the correctly rounded result.
+
+// Full precision: the CUDA math library's expf and log1pf.
+__device__ __forceinline__ float softplus_precise(float s) {
+    return s > 20.f ? s : log1pf(expf(s));
+}
+
+// Fast form for the throughput kernels.  softplus(s) = max(s,0) + ln(1+e),
+// e = e^{-|s|} in (0, 1].  ln(1+e) = 2 atanh(v) with v = e / (2 + e) in
+// (0, 1/3], summed as the odd power series 2 (v + v^3/3 + v^5/5 + ...)
+// -- the classical atanh series for the logarithm, with coefficients
+// 2/(2k+1) -- truncated after v^15: the first dropped term is
+// 2 v^17 / 17 <= 1.5e-9 relative to 2v at v = 1/3, below fp32 rounding.
+// Unlike ln(1 + e) evaluated directly, it keeps full relative accuracy when
+// e is tiny (steps of 1e-3 and below).
+__device__ __forceinline__ float log1p_unit(float e) {  // e in [0, 1]
+    const float v = e * rcp_approx(2.f + e);
+    const float w = v * v;
+    float p = 2.f / 15.f;
+    p = fmaf(p, w, 2.f / 13.f);
+    p = fmaf(p, w, 2.f / 11.f);
+    p = fmaf(p, w, 2.f / 9.f);
+    p = fmaf(p, w, 2.f / 7.f);
+    p = fmaf(p, w, 2.f / 5.f);
+    p = fmaf(p, w, 2.f / 3.f);
+    p = fmaf(p, w, 2.f);
+    return v * p;
+}
+__device__ __forceinline__ float softplus_fast(float s) {
+    const float e = ex2_approx(-fabsf(s) * kLog2e);
+    const float r = fmaxf(s, 0.f) + log1p_unit(e);
+    return s > 20.f ? s : r;
+}
+
+// silu(z) = z * sigmoid(z) = z / (1 + e^{-z}).
+__device__ __forceinline__ float silu_precise(float z) { return z / (1.f + expf(-z)); }
+__device__ __forceinline__ float silu_fast(float z) {
+    // e^{-z} overflows to +inf for z < -88: rcp(inf) = 0 gives the right limit
+    return z * rcp_approx(1.f + ex2_approx(-z * kLog2e));
+}
+
+// ---------------------------------------------------------------------------
+// Device error word: set by kernels whose bounded waits give up, read and
+// cleared by mss_get_device_error.  The library is built as a single
+// translation unit (mss_api.cu includes every kernel), so this is its only
+// definition.
+__device__ unsigned int g_mss_device_error = 0u;
+constexpr unsigned int kDeviceErrTimeout = 1u;
+
+__device__ __forceinline__ void raise_device_error(unsigned int code) {
+    atomicOr(&g_mss_device_error, code);
+}
+
+}  // namespace mss

@@ -1,0 +1,38 @@
+// mss_params.h -- kernel argument blocks (passed by value to every launch).
+#pragma once
+
+#include <cstdint>
+
+namespace mss {
+
+struct ScanParams {
+    const void* u;
+    const void* delta;
+    const float* A;
+    const void* B;
+    const void* C;
+    const float* D;           // may be null
+    const void* z;            // may be null
+    const float* delta_bias;  // may be null
+    void* y;
+    float* last_state;        // may be null
+    int64_t batch, dim, seqlen;
+    int softplus;
+};
+
+struct StepParams {
+    float* state;
+    const void* u;
+    const void* delta;
+    const float* A;
+    const void* B;
+    const void* C;
+    const float* D;
+    const void* z;
+    const float* delta_bias;
+    void* y;
+    int64_t batch, dim;
+    int softplus;
+};
+
+}  // namespace mss

@@ -1,0 +1,63 @@
+// scan_simple.cuh -- reference forward kernel: one thread per (batch, channel),
+// the recurrence run token by token in registers with full-precision math.
+//
+// It accepts any element-aligned pointers and any shape, and it is the
+// parity anchor for the throughput kernel (scan_chunked.cuh): both must agree
+// with the oracle, and with each other within the same tolerance.  It is not
+// meant to be fast -- its u/delta/z loads are one element per thread at a row
+// stride -- and it is only chosen by MSS_FLAG_SIMPLE or for rows that are not
+// 16-byte aligned.
+#pragma once
+
+#include "mss_device.cuh"
+#include "mss_params.h"
+
+namespace mss {
+
+template <typename T, int N>
+__global__ void __launch_bounds__(128) scan_fwd_simple_kernel(ScanParams p) {
+    const int64_t rows = p.batch * p.dim;
+    const int64_t row = int64_t(blockIdx.x) * blockDim.x + threadIdx.x;
+    if (row >= rows) return;
+    const int64_t b = row / p.dim, d = row % p.dim;
+    const int64_t L = p.seqlen;
+
+    const T* u = static_cast<const T*>(p.u) + row * L;
+    const T* dr = static_cast<const T*>(p.delta) + row * L;
+    const T* z = p.z ? static_cast<const T*>(p.z) + row * L : nullptr;
+    const T* Bb = static_cast<const T*>(p.B) + b * N * L;  // B[b][n][t]
+    const T* Cb = static_cast<const T*>(p.C) + b * N * L;
+    T* y = static_cast<T*>(p.y) + row * L;
+
+    float a[N], h[N];
+#pragma unroll
+    for (int n = 0; n < N; ++n) {
+        a[n] = p.A[d * N + n];
+        h[n] = 0.f;
+    }
+    const float bias = p.delta_bias ? p.delta_bias[d] : 0.f;
+    const float Dd = p.D ? p.D[d] : 0.f;
+
+    for (int64_t t = 0; t < L; ++t) {
+        const float ut = ld(u + t);
+        const float s = ld(dr + t) + bias;
+        const float dt = p.softplus ? softplus_precise(s) : s;
+        const float du = dt * ut;
+        float acc = 0.f;
+#pragma unroll
+        for (int n = 0; n < N; ++n) {
+            const float dA = expf(dt * a[n]);
+            h[n] = fmaf(dA, h[n], du * ld(Bb + n * L + t));
+            acc = fmaf(ld(Cb + n * L + t), h[n], acc);
+        }
+        float out = fmaf(Dd, ut, acc);
+        if (z) out *= silu_precise(ld(z + t));
+        y[t] = from_f32<T>(out);
+    }
+    if (p.last_state) {
+#pragma unroll
+        for (int n = 0; n < N; ++n) p.last_state[row * N + n] = h[n];
+    }
+}
+
+}  // namespace mss

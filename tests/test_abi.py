@@ -1,0 +1,122 @@
+"""The C ABI: the library loads and exports what include/mss.h declares, and
+argument errors are reported before any launch (so these run without a GPU:
+every call below fails a host-side check and touches no device)."""
+import ctypes
+import os
+import re
+
+import pytest
+
+import selective_state_space_mss_b200 as mss
+from selective_state_space_mss_b200 import build as mss_build
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "mss.h")
+
+
+@pytest.fixture(scope="module")
+def lib():
+    mss_build.build()
+    return mss.load_library()
+
+
+def _header():
+    with open(HEADER) as f:
+        return f.read()
+
+
+def _declared_functions():
+    return re.findall(r"^MSS_API\s+[\w\s\*]+?\b(mss_\w+)\s*\(", _header(), flags=re.M)
+
+
+def _enum(name):
+    body = re.search(r"enum %s \{(.*?)\};" % name, _header(), flags=re.S).group(1)
+    return {k: int(v) for k, v in re.findall(r"(MSS_\w+)\s*=\s*(-?\d+)", body)}
+
+
+def test_exports_every_declared_symbol(lib):
+    declared = _declared_functions()
+    assert set(declared) >= {"mss_scan_fwd", "mss_scan_fwd_ex", "mss_state_update",
+                             "mss_get_device_error", "mss_strerror", "mss_version"}
+    for name in declared:
+        assert hasattr(lib, name), f"{name} declared in mss.h but not exported"
+
+
+def test_exports_nothing_else(lib):
+    out = os.popen(f"nm -D --defined-only {mss.library_path()}").read()
+    exported = {l.split()[-1] for l in out.splitlines() if " T " in l}
+    assert exported == set(_declared_functions())
+
+
+def test_version_and_strerror(lib):
+    ver = int(re.search(r"#define MSS_VERSION (\d+)", _header()).group(1))
+    assert lib.mss_version() == ver
+    codes = _enum("mss_status")
+    texts = {lib.mss_strerror(c).decode() for c in codes.values()}
+    assert len(texts) == len(codes) and all(texts)
+    assert lib.mss_strerror(12345).decode() == "unknown status code"
+
+
+P = 0x10000  # a fake, 256-byte aligned address: never dereferenced below
+
+
+def _fwd(lib, **kw):
+    a = dict(u=P, delta=P + 0x1000000, A=P + 0x2000000, B=P + 0x3000000, C=P + 0x4000000,
+             D=None, z=None, bias=None, softplus=1, y=P + 0x5000000, last=None,
+             batch=2, dim=8, N=16, L=32, dtype=1, flags=0)
+    a.update(kw)
+    v = lambda x: ctypes.c_void_p(x) if x is not None else None
+    return lib.mss_scan_fwd_ex(v(a["u"]), v(a["delta"]), v(a["A"]), v(a["B"]), v(a["C"]),
+                               v(a["D"]), v(a["z"]), v(a["bias"]), a["softplus"], v(a["y"]),
+                               v(a["last"]), a["batch"], a["dim"], a["N"], a["L"], a["dtype"],
+                               a["flags"], None)
+
+
+def test_forward_argument_errors(lib):
+    codes = _enum("mss_status")
+    assert _fwd(lib, dtype=7) == codes["MSS_ERR_DTYPE"]
+    assert _fwd(lib, flags=0x100) == codes["MSS_ERR_FLAGS"]
+    assert _fwd(lib, batch=-1) == codes["MSS_ERR_SHAPE"]
+    assert _fwd(lib, L=-5) == codes["MSS_ERR_SHAPE"]
+    assert _fwd(lib, batch=2 ** 40, dim=2 ** 30) == codes["MSS_ERR_SHAPE"]
+    for n in (0, 3, 32, -16):
+        assert _fwd(lib, N=n) == codes["MSS_ERR_UNSUPPORTED_N"]
+    for k in ("u", "delta", "A", "B", "C", "y"):
+        assert _fwd(lib, **{k: None}) == codes["MSS_ERR_NULL"], k
+    assert _fwd(lib, u=P + 1) == codes["MSS_ERR_ALIGN"]
+    assert _fwd(lib, A=P + 2) == codes["MSS_ERR_ALIGN"]
+    assert _fwd(lib, dtype=0, z=P + 0x6000002) == codes["MSS_ERR_ALIGN"]
+    assert _fwd(lib, y=P + 64) == codes["MSS_ERR_ALIAS"]          # y inside u
+    assert _fwd(lib, last=P + 0x3000000) == codes["MSS_ERR_ALIAS"]  # last_state on B
+    # nothing to do: accepted without a launch
+    assert _fwd(lib, batch=0) == 0 and _fwd(lib, dim=0, u=None) == 0
+
+
+def test_decode_argument_errors(lib):
+    codes = _enum("mss_status")
+    v = ctypes.c_void_p
+
+    def step(**kw):
+        a = dict(state=P, u=P + 0x1000000, delta=P + 0x2000000, A=P + 0x3000000,
+                 B=P + 0x4000000, C=P + 0x5000000, y=P + 0x6000000, batch=4, dim=8, N=16, dtype=1)
+        a.update(kw)
+        w = lambda x: v(x) if x is not None else None
+        return lib.mss_state_update(w(a["state"]), w(a["u"]), w(a["delta"]), w(a["A"]), w(a["B"]),
+                                    w(a["C"]), None, None, None, 1, w(a["y"]), a["batch"],
+                                    a["dim"], a["N"], a["dtype"], None)
+
+    assert step(dtype=2) == codes["MSS_ERR_DTYPE"]
+    assert step(N=5) == codes["MSS_ERR_UNSUPPORTED_N"]
+    assert step(dim=-1) == codes["MSS_ERR_SHAPE"]
+    assert step(state=None) == codes["MSS_ERR_NULL"]
+    assert step(state=P + 2) == codes["MSS_ERR_ALIGN"]
+    assert step(y=P + 8) == codes["MSS_ERR_ALIAS"]  # y on the state
+    assert step(batch=0) == 0
+
+
+def test_binding_refuses_cpu_tensors():
+    import torch
+
+    x = torch.zeros(1, 2, 3)
+    with pytest.raises(ValueError, match="CUDA"):
+        mss.scan_fwd(x, x, torch.zeros(2, 4), x, x)
