@@ -64,13 +64,13 @@ PFN_cuTensorMapEncodeTiled_v12000 encode_tiled_fn() {
     return fn;
 }
 
-// [rows, L] row-major view, box = 32 rows x 128 bytes, 128-byte swizzle.
-bool encode_rows(CUtensorMap* m, const void* base, int64_t rows, int64_t L, int esz) {
+// [rows, L] row-major view, box = box_rows rows x 128 bytes, 128-byte swizzle.
+bool encode_rows(CUtensorMap* m, const void* base, int64_t rows, int64_t L, int esz, int box_rows) {
     auto enc = encode_tiled_fn();
     if (!enc) return false;
     const cuuint64_t dims[2] = {cuuint64_t(L), cuuint64_t(rows)};
     const cuuint64_t strides[1] = {cuuint64_t(L * esz)};
-    const cuuint32_t box[2] = {cuuint32_t(128 / esz), 32u};
+    const cuuint32_t box[2] = {cuuint32_t(128 / esz), cuuint32_t(box_rows)};
     const cuuint32_t estr[2] = {1u, 1u};
     return enc(m, esz == 2 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 2,
                const_cast<void*>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
@@ -108,8 +108,8 @@ bool seq_eligible(const mss::ScanParams& p, int64_t N, int esz, unsigned flags) 
     if (N != 4 && N != 8 && N != 16) return false;
     if ((p.seqlen * esz) % 16 != 0) return false;
     if (p.batch * p.dim >= (int64_t(1) << 31) || p.seqlen >= (int64_t(1) << 31)) return false;
-    if ((p.dim + 31) / 32 > 0x7fffffffLL || p.batch > 65535) return false;
-    const void* v[] = {p.u, p.delta, p.z, p.B, p.C, p.y, p.last_state};
+    if ((p.dim + 15) / 16 > 0x7fffffffLL || p.batch > 65535) return false;
+    const void* v[] = {p.u, p.delta, p.z, p.B, p.C, p.y};
     for (const void* q : v)
         if (q && !aligned(q, 16)) return false;
     return true;
@@ -121,7 +121,8 @@ int launch_seq_variant(const mss::SeqMaps& maps, const mss::ScanParams& p, unsig
     const int smem = mss::SeqLayout<T, N>::kSmemBytes;
     if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess)
         return MSS_ERR_CUDA;
-    const dim3 grid(unsigned((p.dim + 31) / 32), unsigned(p.batch));
+    constexpr int rows = mss::SeqLayout<T, N>::kRows;
+    const dim3 grid(unsigned((p.dim + rows - 1) / rows), unsigned(p.batch));
     kern<<<grid, 32, smem, stream>>>(maps, p, (flags & MSS_FLAG_GENERAL_A) ? 0 : 1);
     return launch_status();
 }
@@ -132,8 +133,10 @@ int launch_seq(const mss::ScanParams& p, unsigned flags, cudaStream_t stream) {
     mss::SeqMaps maps;
     std::memset(&maps, 0, sizeof(maps));
     const int64_t rows = p.batch * p.dim;
-    if (!encode_rows(&maps.u, p.u, rows, p.seqlen, esz) || !encode_rows(&maps.delta, p.delta, rows, p.seqlen, esz) ||
-        (p.z && !encode_rows(&maps.z, p.z, rows, p.seqlen, esz)) ||
+    constexpr int br = mss::SeqLayout<T, N>::kRows;
+    if (!encode_rows(&maps.u, p.u, rows, p.seqlen, esz, br) ||
+        !encode_rows(&maps.delta, p.delta, rows, p.seqlen, esz, br) ||
+        (p.z && !encode_rows(&maps.z, p.z, rows, p.seqlen, esz, br)) ||
         !encode_bc(&maps.B, p.B, p.batch, N, p.seqlen, esz) || !encode_bc(&maps.C, p.C, p.batch, N, p.seqlen, esz))
         return MSS_ERR_CUDA;
     if (p.z)
