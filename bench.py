@@ -65,14 +65,30 @@ def decode_bytes(batch, dim, N, esz=2, z=True):
             + 2 * batch * N * esz + dim * N * 4 + 2 * dim * 4)
 
 
+def fwd_alu_ops(batch, dim, N, L):
+    """Algorithmic fp32 lane operations of one forward launch: per token and
+    state the definition's four (transition via the S4D-Real identity, input
+    term, update, read-out), per token ten more (bias add, softplus, Delta*u,
+    Delta*A_0, skip, read-out sum, gate)."""
+    return batch * dim * L * (4 * N + 10)
+
+
+# B200: 148 SMs x 128 fp32 lanes per SM and clock, at the maximum SM clock.
+SMS, FP32_LANES_PER_SM = 148, 128
+
+
+def alu_peak_ops(sm_max_mhz):
+    return SMS * FP32_LANES_PER_SM * sm_max_mhz * 1e6
+
+
 def measured_peaks():
     p = os.path.join(ROOT, "MEASURED_PEAKS.json")
     try:
         with open(p) as f:
             d = json.load(f)
-        return float(d["hbm_gbs"]), "measured"
+        return float(d["hbm_gbs"]), "measured", float(d.get("sm_max_mhz", 1965.0))
     except Exception:
-        return FALLBACK_HBM_GBS, "fallback"
+        return FALLBACK_HBM_GBS, "fallback", 1965.0
 
 
 def kernel_source_hash():
@@ -156,6 +172,33 @@ class ClockSampler:
                 "reasons": reasons, "samples": len(rows)}
 
 
+# ---------------------------------------------------------------------------
+# Multi-rank plumbing: every rank runs its own replica of the workload (the
+# channels are independent, so there is no data-path collective); the only
+# collectives are barriers and the max-over-ranks of the measured time.
+
+def rank_seed(base_seed, rank):
+    """Seed of rank `rank`'s replica (distinct inputs per rank)."""
+    return base_seed + 100 * rank
+
+
+def max_over_ranks(ms, world, device):
+    """The slowest rank's time (collective: every rank must call it)."""
+    if world <= 1:
+        return float(ms)
+    import torch
+    import torch.distributed as dist
+
+    t = torch.tensor([float(ms)], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def whole_job_rate(units_per_rank, world, steps, ms_max):
+    """Units of all ranks per second over the slowest rank's time."""
+    return world * units_per_rank * steps / (ms_max * 1e-3)
+
+
 def physical_gpu_index(local_rank):
     vis = os.environ.get("CUDA_VISIBLE_DEVICES")
     if vis:
@@ -169,35 +212,42 @@ def physical_gpu_index(local_rank):
 # The CPU oracle, timed (cpu_baseline and the reference arm).
 
 def oracle_sample_rate(inp, rows, nthreads):
-    """Run the oracle on the first `rows` channels of batch row 0; returns
-    (channel-tokens, seconds)."""
+    """Run the oracle on the first `rows` channels of every batch row;
+    returns (channel-tokens, seconds)."""
     import oracle
 
     L = inp["seqlen"]
     t0 = time.perf_counter()
-    oracle.scan_fwd(inp["u"].values[:1, :rows], inp["delta"].values[:1, :rows], inp["A"][:rows],
-                    inp["B"].values[:1], inp["C"].values[:1], D=inp["D"][:rows],
-                    z=inp["z"].values[:1, :rows], delta_bias=inp["delta_bias"][:rows],
+    oracle.scan_fwd(inp["u"].values[:, :rows], inp["delta"].values[:, :rows], inp["A"][:rows],
+                    inp["B"].values, inp["C"].values, D=inp["D"][:rows],
+                    z=inp["z"].values[:, :rows], delta_bias=inp["delta_bias"][:rows],
                     nthreads=nthreads)
-    return rows * L, time.perf_counter() - t0
+    return inp["batch"] * rows * L, time.perf_counter() - t0
 
 
 def calibrate_rows(inp, nthreads, target_s):
-    rows = max(nthreads, 8)
-    ct, sec = oracle_sample_rate(inp, rows, nthreads)
+    """Channels per batch row for one oracle pass of about target_s seconds
+    (at most the whole workload)."""
+    rows = min(inp["dim"], max(nthreads, 16))
+    _, sec = oracle_sample_rate(inp, rows, nthreads)
     per_row = sec / rows
     return int(min(inp["dim"], max(nthreads, target_s / max(per_row, 1e-9))))
 
 
-def cpu_baseline(inp, target_s=12.0):
+def cpu_baseline(inp, target_s=10.0):
+    """The oracle on the host cores over the same workload, repeated until
+    about target_s seconds of work."""
     import oracle
 
     nthreads = oracle.default_threads()
     rows = calibrate_rows(inp, nthreads, target_s)
-    ct, sec = oracle_sample_rate(inp, rows, nthreads)
-    return {"value": ct / sec, "unit": UNIT, "cores": nthreads, "kind": "oracle",
-            "sample": f"{rows} channels x {inp['seqlen']} tokens of batch row 0 of {WORKLOAD} "
-                      f"(fp64, {nthreads} threads, {sec:.1f} s)"}
+    total_ct, total_s, passes = 0, 0.0, 0
+    while total_s < target_s or passes == 0:
+        ct, sec = oracle_sample_rate(inp, rows, nthreads)
+        total_ct, total_s, passes = total_ct + ct, total_s + sec, passes + 1
+    return {"value": total_ct / total_s, "unit": UNIT, "cores": nthreads, "kind": "oracle",
+            "sample": f"{passes} pass(es) of {inp['batch']}x{rows} channels x {inp['seqlen']} tokens "
+                      f"of {WORKLOAD} (fp64, {nthreads} threads, {total_s:.1f} s)"}
 
 
 def run_reference(args, rank):
@@ -207,23 +257,25 @@ def run_reference(args, rank):
 
     inp = gen.workload_inputs(WORKLOAD)
     nthreads = oracle.default_threads()
+    # each step: one oracle pass over as much of the workload as fits ~8 s
     rows = calibrate_rows(inp, nthreads, target_s=min(8.0, 150.0 / max(1, args.steps + args.warmup)))
     for _ in range(args.warmup):
         oracle_sample_rate(inp, rows, nthreads)
     times = []
     for _ in range(args.steps):
-        ct, sec = oracle_sample_rate(inp, rows, nthreads)
+        _, sec = oracle_sample_rate(inp, rows, nthreads)
         times.append(sec)
     total = sum(times)
-    value = rows * inp["seqlen"] * args.steps / total
+    ct_step = inp["batch"] * rows * inp["seqlen"]
+    value = ct_step * args.steps / total
     line = {
         "impl": "reference", "metric": METRIC, "value": value, "unit": UNIT,
         "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
         "ms_per_step": 1e3 * total / args.steps, "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-        "config": {"workload": WORKLOAD, "sample_rows": rows, "seqlen": inp["seqlen"]},
+        "config": {"workload": WORKLOAD, "sample_channels_per_batch_row": rows, "seqlen": inp["seqlen"]},
         "cpu_baseline": {"value": value, "unit": UNIT, "cores": nthreads, "kind": "oracle",
-                         "sample": f"{rows} channels x {inp['seqlen']} tokens per step, fp64"},
+                         "sample": f"{inp['batch']}x{rows} channels x {inp['seqlen']} tokens per step, fp64"},
         "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
     }
     print(json.dumps(line), flush=True)
@@ -251,8 +303,8 @@ def run_mss(args, rank, world, local_rank):
         import dataclasses
 
         w = dataclasses.replace(w, seqlen=args.seqlen)
-    inp = gen.scan_inputs(w.batch, w.dim, w.dstate, w.seqlen, w.dtype, w.seed + 100 * rank, w.d_skip)
-    nxt = gen.decode_step_inputs(w.batch, w.dim, w.dstate, w.dtype, w.seed + 100 * rank, 0)
+    inp = gen.scan_inputs(w.batch, w.dim, w.dstate, w.seqlen, w.dtype, rank_seed(w.seed, rank), w.d_skip)
+    nxt = gen.decode_step_inputs(w.batch, w.dim, w.dstate, w.dtype, rank_seed(w.seed, rank), 0)
 
     def to_dev(t):
         return torch.from_numpy(np.ascontiguousarray(t.stored).view(np.int16)).view(torch.bfloat16).to(dev)
@@ -299,12 +351,8 @@ def run_mss(args, rank, world, local_rank):
             sampler.__exit__(None, None, None)
         if world > 1:
             dist.barrier()
-        ms = start.elapsed_time(end)
+        ms = max_over_ranks(start.elapsed_time(end), world, dev)
         fwd_ms = [a.elapsed_time(b) for a, b in evs]
-        if world > 1:
-            t = torch.tensor([ms], device=dev)
-            dist.all_reduce(t, op=dist.ReduceOp.MAX)
-            ms = float(t.item())
         return ms, fwd_ms, (sampler.summary() if with_clocks else None)
 
     assert mss.get_device_error() == 0
@@ -353,11 +401,7 @@ def run_mss(args, rank, world, local_rank):
         e2e_step()
     e1.record(stream)
     torch.cuda.synchronize(dev)
-    e2e_ms = e0.elapsed_time(e1)
-    if world > 1:
-        t = torch.tensor([e2e_ms], device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        e2e_ms = float(t.item())
+    e2e_ms = max_over_ranks(e0.elapsed_time(e1), world, dev)
     assert mss.get_device_error() == 0
 
     # decode workload (256 x 5120 x 16 state): per-token time with L2 flushed
@@ -382,12 +426,14 @@ def run_mss(args, rank, world, local_rank):
     dec_med = statistics.median(dec_ms)
     dec_bytes = decode_bytes(dw.batch, dw.dim, dw.dstate)
 
-    peak, peak_kind = measured_peaks()
+    peak, peak_kind, sm_max_mhz = measured_peaks()
+    alu_ops = fwd_alu_ops(w.batch, w.dim, w.dstate, w.seqlen)
+    alu_peak = alu_peak_ops(sm_max_mhz)
     fwd_avg = sum(fwd_ms) / len(fwd_ms)
     fwd_avg_gen = sum(fwd_ms_gen) / len(fwd_ms_gen)
     achieved = bytes_fwd / (fwd_avg * 1e-3) / 1e9
     achieved_gen = bytes_fwd / (fwd_avg_gen * 1e-3) / 1e9
-    value = world * ct_per_step * args.steps / (ms * 1e-3)
+    value = whole_job_rate(ct_per_step, world, args.steps, ms)
     line = {
         "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": ms / args.steps, "higher_is_better": True,
@@ -400,17 +446,23 @@ def run_mss(args, rank, world, local_rank):
                    "l2": f"inputs larger than L2: {bytes_step / 1e6:.0f} MB of algorithmic traffic per step",
                    "parallelism": f"replicas x{world} (channels shard with no collective)"},
         "achieved_hbm_gbs": world * bytes_step * args.steps / (ms * 1e-3) / 1e9,
-        "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
-                     "frac": achieved / peak, "traffic": recorded_traffic(),
-                     "kernel": "scan_fwd (forward scan)", "peak_kind": peak_kind,
-                     "algorithmic_bytes_per_launch": bytes_fwd, "launch_ms_avg": fwd_avg},
+        "roofline": {"bound": "alu", "achieved": alu_ops / (fwd_avg * 1e-3) / 1e12,
+                     "peak": alu_peak / 1e12, "unit": "Tops/s (fp32 lane ops)",
+                     "frac": alu_ops / (fwd_avg * 1e-3) / alu_peak, "traffic": recorded_traffic(),
+                     "kernel": "scan_fwd_seq (forward scan)",
+                     "peak_kind": f"derived: {SMS} SMs x {FP32_LANES_PER_SM} fp32 lanes x {sm_max_mhz:.0f} MHz",
+                     "algorithmic_ops_per_launch": alu_ops, "algorithmic_bytes_per_launch": bytes_fwd,
+                     "launch_ms_avg": fwd_avg},
+        "roofline_hbm": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
+                         "frac": achieved / peak, "traffic": recorded_traffic(),
+                         "peak_kind": peak_kind, "algorithmic_bytes_per_launch": bytes_fwd},
         "general_A_path": {"fwd_ms_avg": fwd_avg_gen, "achieved_gbs": achieved_gen,
                            "frac": achieved_gen / peak,
                            "channel_tokens_per_s": w.batch * w.dim * w.seqlen / (fwd_avg_gen * 1e-3)},
         "decode": {"workload": gen.DECODE_WORKLOAD, "ms_per_token_median": dec_med,
                    "achieved_gbs": dec_bytes / (dec_med * 1e-3) / 1e9,
                    "frac": dec_bytes / (dec_med * 1e-3) / 1e9 / peak, "l2": "flushed before each token"},
-        "e2e": {"value": world * ct_per_step * args.steps / (e2e_ms * 1e-3), "unit": UNIT,
+        "e2e": {"value": whole_job_rate(ct_per_step, world, args.steps, e2e_ms), "unit": UNIT,
                 "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
         "gpu_launches": launches_per_step * args.steps,
         "clocks": clocks,
