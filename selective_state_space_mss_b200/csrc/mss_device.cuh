@@ -69,30 +69,21 @@ __device__ __forceinline__ float softplus_precise(float s) {
     return s > 20.f ? s : log1pf(expf(s));
 }
 
-// Fast form for the throughput kernels.  softplus(s) = max(s,0) + ln(1+e),
-// e = e^{-|s|} in (0, 1].  ln(1+e) = 2 atanh(v) with v = e / (2 + e) in
-// (0, 1/3], summed as the odd power series 2 (v + v^3/3 + v^5/5 + ...)
-// -- the classical atanh series for the logarithm, with coefficients
-// 2/(2k+1) -- truncated after v^15: the first dropped term is
-// 2 v^17 / 17 <= 1.5e-9 relative to 2v at v = 1/3, below fp32 rounding.
-// Unlike ln(1 + e) evaluated directly, it keeps full relative accuracy when
-// e is tiny (steps of 1e-3 and below).
-__device__ __forceinline__ float log1p_unit(float e) {  // e in [0, 1]
-    const float v = e * rcp_approx(2.f + e);
-    const float w = v * v;
-    float p = 2.f / 15.f;
-    p = fmaf(p, w, 2.f / 13.f);
-    p = fmaf(p, w, 2.f / 11.f);
-    p = fmaf(p, w, 2.f / 9.f);
-    p = fmaf(p, w, 2.f / 7.f);
-    p = fmaf(p, w, 2.f / 5.f);
-    p = fmaf(p, w, 2.f / 3.f);
-    p = fmaf(p, w, 2.f);
-    return v * p;
+__device__ __forceinline__ float lg2_approx(float x) {
+    float r;
+    asm("lg2.approx.ftz.f32 %0, %1;" : "=f"(r) : "f"(x));
+    return r;
 }
+
+// Fast form for bf16 io: softplus(s) = max(s, 0) + ln 2 * log2(1 + e^{-|s|}),
+// two MUFU instructions and three fp32 operations.  The single-instruction
+// log2 has an absolute error near 2^-22 on (1, 2], so Delta carries an
+// absolute error of about 2e-7 (relative 2e-4 at Delta = 1e-3, less for
+// larger steps): ten times below the rounding of a bf16 output.  fp32 io uses
+// softplus_precise.
 __device__ __forceinline__ float softplus_fast(float s) {
     const float e = ex2_approx(-fabsf(s) * kLog2e);
-    const float r = fmaxf(s, 0.f) + log1p_unit(e);
+    const float r = fmaf(0.69314718f, lg2_approx(1.f + e), fmaxf(s, 0.f));
     return s > 20.f ? s : r;
 }
 

@@ -279,45 +279,48 @@ __device__ __forceinline__ void scan_seq_body(const SeqMaps& maps, const ScanPar
 #pragma unroll
     for (int i = 0; i < P; ++i) h[i] = make_float2(0.f, 0.f);
     T* yrow = static_cast<T*>(p.y) + row * L + HV * half;
+    const float4* my_bcf = reinterpret_cast<const float4*>(bcf) + half * P;  // this lane's chunks of a row
+    constexpr int kRowF4 = Ly::kBCfRow / 4;
 
     if (!wait_chunk(0)) return;
     convert_bc<T, N>(smem + 3 * Ly::kTile, smem + 3 * Ly::kTile + Ly::kBCTile, bcf, lane);
     __syncwarp();
-    TokenPre nxt[HV];
+
+    // Software pipeline across groups.  Carried into iteration g:
+    //   own[]        this lane's scalars of group g's tokens [half*HV, half*HV + HV)
+    //   pdu[], prd[] the partner's Delta*u and r (or Delta) of group g
+    //   nrow[]       group g's first B/C row
+    //   the previous group's transpose-reduce (finished after token 1 of g)
+    TokenPre own[HV];
+    float pdu[HV], prd[HV];
     {
         float uv[HV], dv[HV], zv[HV];
         load_half(0, uv, dv, zv);
 #pragma unroll
-        for (int k = 0; k < HV; ++k)
-            nxt[k] = token_pre<kFast, kGeo, kGate, kSoftplus>(uv[k], dv[k], kGate ? zv[k] : 0.f, cc);
+        for (int k = 0; k < HV; ++k) {
+            own[k] = token_pre<kFast, kGeo, kGate, kSoftplus>(uv[k], dv[k], kGate ? zv[k] : 0.f, cc);
+            pdu[k] = __shfl_xor_sync(0xffffffffu, own[k].du, 1);
+            prd[k] = __shfl_xor_sync(0xffffffffu, own[k].r, 1);
+        }
     }
-    const float4* my_bcf = reinterpret_cast<const float4*>(bcf) + half * P;  // this lane's chunks of a row
-    constexpr int kRowF4 = Ly::kBCfRow / 4;
+    float4 nrow[P];
+#pragma unroll
+    for (int i = 0; i < P; ++i) nrow[i] = my_bcf[i];
+    float pkeep[HV], precv[HV], pskip[HV], pgate[HV];  // previous group's pending outputs
+    int64_t pend_at = -1;                               // its token offset, -1: none
 
 #pragma unroll 1
     for (int g = 0; g < n_groups; ++g) {
         const int c = g / GPC, j = g % GPC;
-        // this group's scalars: own tokens from the previous iteration, the
-        // partner's by shuffle
-        TokenPre own[HV];
-        float odu[HV], ordt[HV];
-#pragma unroll
-        for (int k = 0; k < HV; ++k) {
-            own[k] = nxt[k];
-            odu[k] = __shfl_xor_sync(0xffffffffu, own[k].du, 1);
-            ordt[k] = __shfl_xor_sync(0xffffffffu, own[k].r, 1);
-        }
-        // the next group's inputs: its u/delta/z must have landed when it opens a new chunk
         const bool has_next = g + 1 < n_groups;
+        // the next group's u/delta/z, first: its stage must have landed when it opens a new chunk
         if (has_next && j == GPC - 1 && !wait_chunk(c + 1)) return;
         float uv[HV], dv[HV], zv[HV];
         load_half(has_next ? g + 1 : g, uv, dv, zv);
 
+        TokenPre nxt[HV];
         float acc[V];
         const float4* base = my_bcf + (j * V) * kRowF4;
-        float4 nrow[P];
-#pragma unroll
-        for (int i = 0; i < P; ++i) nrow[i] = base[i];
 #pragma unroll
         for (int t = 0; t < V; ++t) {
             float4 rowv[P];
@@ -326,24 +329,47 @@ __device__ __forceinline__ void scan_seq_body(const SeqMaps& maps, const ScanPar
             if (t + 1 < V) {
 #pragma unroll
                 for (int i = 0; i < P; ++i) nrow[i] = base[(t + 1) * kRowF4 + i];
+            } else if (j + 1 < GPC) {
+                // the next group's first row (same chunk: already converted)
+#pragma unroll
+                for (int i = 0; i < P; ++i) nrow[i] = base[V * kRowF4 + i];
             }
             // token t belongs to lane half t / HV of the pair
             const bool mine = (t / HV) == half;
-            const float du = mine ? own[t % HV].du : odu[t % HV];
-            const float rdt = mine ? own[t % HV].r : ordt[t % HV];
+            const float du = mine ? own[t % HV].du : pdu[t % HV];
+            const float rdt = mine ? own[t % HV].r : prd[t % HV];
             acc[t] = token_states<N, kFast, kGeo>(h, rowv, du, rdt, half, cc);
-            if (t < HV) nxt[t] = token_pre<kFast, kGeo, kGate, kSoftplus>(uv[t], dv[t], kGate ? zv[t] : 0.f, cc);
+            // the previous group's outputs, once their shuffles have had time
+            if (t == 1 && pend_at >= 0) {
+                float yv[HV];
+#pragma unroll
+                for (int k = 0; k < HV; ++k) yv[k] = (pkeep[k] + precv[k] + pskip[k]) * pgate[k];
+                if (valid) *reinterpret_cast<uint2*>(yrow + pend_at) = pack8<T>(yv);
+            }
+            // the next group's scalars, spread over the middle tokens
+            constexpr int kPre0 = V >= 8 ? 2 : 0;
+            if (t >= kPre0 && t < kPre0 + HV)
+                nxt[t - kPre0] = token_pre<kFast, kGeo, kGate, kSoftplus>(uv[t - kPre0], dv[t - kPre0],
+                                                                            kGate ? zv[t - kPre0] : 0.f, cc);
         }
-        // transpose-reduce: lane half h finishes tokens [h*HV, h*HV + HV)
-        float yv[HV];
+        // this group's read-out: transpose-reduce (lane half h finishes tokens
+        // [h*HV, h*HV + HV)); finished after token 1 of the next group
 #pragma unroll
         for (int k = 0; k < HV; ++k) {
             const float send = half ? acc[k] : acc[HV + k];
-            const float keep = half ? acc[HV + k] : acc[k];
-            const float tot = keep + __shfl_xor_sync(0xffffffffu, send, 1);
-            yv[k] = (tot + own[k].skip) * own[k].gate;
+            pkeep[k] = half ? acc[HV + k] : acc[k];
+            precv[k] = __shfl_xor_sync(0xffffffffu, send, 1);
+            pskip[k] = own[k].skip;
+            pgate[k] = own[k].gate;
         }
-        if (valid) *reinterpret_cast<uint2*>(yrow + int64_t(g) * V) = pack8<T>(yv);
+        pend_at = int64_t(g) * V;
+        // hand over the next group's scalars
+#pragma unroll
+        for (int k = 0; k < HV; ++k) {
+            own[k] = nxt[k];
+            pdu[k] = __shfl_xor_sync(0xffffffffu, nxt[k].du, 1);
+            prd[k] = __shfl_xor_sync(0xffffffffu, nxt[k].r, 1);
+        }
 
         if (j == GPC - 1 || !has_next) {
             // chunk c is consumed: convert the next chunk's B/C (its stage was
@@ -358,7 +384,17 @@ __device__ __forceinline__ void scan_seq_body(const SeqMaps& maps, const ScanPar
                 fence_proxy_async_smem();
                 issue(c + S);
             }
+            // the next group's first row, now that its chunk is converted
+#pragma unroll
+            for (int i = 0; i < P; ++i) nrow[i] = my_bcf[i];
         }
+    }
+    // the last group's outputs
+    if (pend_at >= 0) {
+        float yv[HV];
+#pragma unroll
+        for (int k = 0; k < HV; ++k) yv[k] = (pkeep[k] + precv[k] + pskip[k]) * pgate[k];
+        if (valid) *reinterpret_cast<uint2*>(yrow + pend_at) = pack8<T>(yv);
     }
     if (valid && p.last_state) {
         float* ls = p.last_state + row * N + half;
