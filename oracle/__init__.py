@@ -57,7 +57,7 @@ def _load():
             lib = ctypes.CDLL(path)
             f, d, i64, i = (ctypes.POINTER(ctypes.c_float), ctypes.POINTER(ctypes.c_double),
                             ctypes.c_int64, ctypes.c_int)
-            lib.mss_oracle_scan_fwd.argtypes = [f, f, f, f, f, f, f, f, i, d, d,
+            lib.mss_oracle_scan_fwd.argtypes = [f, f, f, f, f, f, f, f, i, d, d, d,
                                                 i64, i64, i64, i64, i]
             lib.mss_oracle_scan_fwd.restype = i
             lib.mss_oracle_state_update.argtypes = [d, f, f, f, f, f, f, f, f, i, d,
@@ -101,13 +101,14 @@ def silu(z: float) -> float:
 
 
 def scan_fwd(u, delta, A, B, C, D=None, z=None, delta_bias=None, softplus_flag=True,
-             nthreads=None):
+             initial_state=None, nthreads=None):
     """Selective-scan forward pass in fp64.
 
     u, delta, z: [batch, dim, L]; A: [dim, N]; B, C: [batch, N, L];
-    D, delta_bias: [dim].  Values are taken as fp32 (bf16 inputs must already
-    be widened, which is exact).  Returns (y [batch, dim, L] fp64,
-    last_state [batch, dim, N] fp64).
+    D, delta_bias: [dim]; initial_state: [batch, dim, N] (the state before
+    the first token; None for zero).  Values are taken as fp32 (bf16 inputs
+    must already be widened, which is exact); initial_state as fp64.
+    Returns (y [batch, dim, L] fp64, last_state [batch, dim, N] fp64).
     """
     u_a, u_p = _f32(u, name="u")
     if u_a.ndim != 3:
@@ -123,11 +124,16 @@ def scan_fwd(u, delta, A, B, C, D=None, z=None, delta_bias=None, softplus_flag=T
     D_a, D_p = _f32(D, (dim,), "D")
     z_a, z_p = _f32(z, (batch, dim, L), "z")
     b_a, b_p = _f32(delta_bias, (dim,), "delta_bias")
+    h0 = None
+    if initial_state is not None:
+        h0 = np.ascontiguousarray(np.asarray(initial_state, dtype=np.float64))
+        if h0.shape != (batch, dim, N):
+            raise ValueError(f"initial_state: expected shape {(batch, dim, N)}, got {h0.shape}")
     y = np.empty((batch, dim, L), dtype=np.float64)
     last = np.empty((batch, dim, N), dtype=np.float64)
     rc = _load().mss_oracle_scan_fwd(
         u_p, d_p, A_p, B_p, C_p, D_p, z_p, b_p, int(bool(softplus_flag)),
-        _dptr(y), _dptr(last), batch, dim, N, L,
+        _dptr(h0) if h0 is not None else None, _dptr(y), _dptr(last), batch, dim, N, L,
         default_threads() if nthreads is None else int(nthreads))
     if rc != 0:
         raise RuntimeError(f"mss_oracle_scan_fwd failed with code {rc}")

@@ -116,6 +116,7 @@ int mss_oracle_recurrence(const double *abar, const double *bbar_x, const double
 typedef struct {
     /* inputs, layouts as documented at mss_oracle_scan_fwd */
     const float *u, *delta, *A, *B, *C, *D, *z, *bias;
+    const double *initial_state;
     int softplus_flag;
     double *y, *last_state;
     int64_t batch, dim, N, L;
@@ -163,7 +164,7 @@ static void *scan_rows(void *arg)
         const double bias = j->bias ? (double)j->bias[d] : 0.0;
         double *y = j->y + row * L;
         for (int64_t n = 0; n < N; ++n)
-            h[n] = 0.0;
+            h[n] = j->initial_state ? j->initial_state[row * N + n] : 0.0;
         for (int64_t t = 0; t < L; ++t) {
             const double ut = (double)u[t];
             discretise((double)dr[t], bias, j->softplus_flag, A_row, B_b + t, C_b + t,
@@ -225,6 +226,8 @@ static int run_threaded(scan_job *proto, int64_t rows, int nthreads, void *(*fn)
  *   A           : [dim][N]          (negative reals for a stable system)
  *   B, C        : [batch][N][L]     (shared by all channels of a batch row)
  *   D, bias     : [dim]             (D, z, bias may be NULL)
+ *   initial_state: [batch][dim][N]  fp64 state before the first token, or
+ *                                   NULL for the zero state of the pages
  *   y           : [batch][dim][L]   fp64 output
  *   last_state  : [batch][dim][N]   fp64 output, may be NULL
  * Returns 0, or a negative code for bad arguments / no memory.
@@ -232,7 +235,7 @@ static int run_threaded(scan_job *proto, int64_t rows, int nthreads, void *(*fn)
 int mss_oracle_scan_fwd(const float *u, const float *delta, const float *A,
                         const float *B, const float *C, const float *D,
                         const float *z, const float *delta_bias, int softplus_flag,
-                        double *y, double *last_state,
+                        const double *initial_state, double *y, double *last_state,
                         int64_t batch, int64_t dim, int64_t dstate, int64_t seqlen,
                         int nthreads)
 {
@@ -240,8 +243,8 @@ int mss_oracle_scan_fwd(const float *u, const float *delta, const float *A,
         return ORACLE_EINVAL;
     if (batch < 0 || dim < 0 || dstate <= 0 || seqlen < 0)
         return ORACLE_EINVAL;
-    scan_job proto = {u, delta, A, B, C, D, z, delta_bias, softplus_flag, y, last_state,
-                      batch, dim, dstate, seqlen, 0, 0, ORACLE_OK};
+    scan_job proto = {u, delta, A, B, C, D, z, delta_bias, initial_state, softplus_flag,
+                      y, last_state, batch, dim, dstate, seqlen, 0, 0, ORACLE_OK};
     if (batch * dim == 0)
         return ORACLE_OK;
     return run_threaded(&proto, batch * dim, nthreads, scan_rows);

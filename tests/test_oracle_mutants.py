@@ -29,8 +29,9 @@ MUTANTS = {
     "skip_dropped": ("double out = recurrence_step(h, abar, bx, c, N) + Dd * ut;",
                      "double out = recurrence_step(h, abar, bx, c, N);"),
     "gate_is_sigmoid": ("return z / (1.0 + exp(-z));", "return 1.0 / (1.0 + exp(-z));"),
-    "state_not_reset_per_row": ("        for (int64_t n = 0; n < N; ++n)\n            h[n] = 0.0;\n        for (int64_t t = 0; t < L; ++t) {",
+    "state_not_reset_per_row": ("        for (int64_t n = 0; n < N; ++n)\n            h[n] = j->initial_state ? j->initial_state[row * N + n] : 0.0;\n        for (int64_t t = 0; t < L; ++t) {",
                                 "        for (int64_t t = 0; t < L; ++t) {"),
+    "initial_state_ignored": ("h[n] = j->initial_state ? j->initial_state[row * N + n] : 0.0;", "h[n] = 0.0;"),
     "decode_B_token_stride": ("j->B + b * N, j->C + b * N, 1, N,", "j->B + b * N, j->C + b * N, N, N,"),
     "B_batch_index": ("const float *B_b = j->B + b * N * L;", "const float *B_b = j->B;"),
 }

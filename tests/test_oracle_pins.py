@@ -419,3 +419,23 @@ def test_skip_term_alone():
     yg, _ = oracle.scan_fwd(**inp)
     gate = np.vectorize(oracle.silu)(inp["z"].astype(np.float64))
     assert np.array_equal(yg, Du * gate)
+
+
+def test_initial_state_chains_forward_passes():
+    """Starting from the state a prefix ends in continues the prefix exactly:
+    forward(prefix) then forward(rest, initial_state = prefix's last state)
+    equals forward(all), bitwise in fp64 (the same operations in the same
+    order; the generation view of "Exercises" carries the state the same way)."""
+    inp = _random_forward_inputs(36, L=60)
+    y_all, last_all = oracle.scan_fwd(**inp)
+    for L0 in (1, 17, 59):
+        y0, last0 = oracle.scan_fwd(**_slice_t(inp, 0, L0))
+        y1, last1 = oracle.scan_fwd(**_slice_t(inp, L0, 60), initial_state=last0)
+        assert np.array_equal(np.concatenate([y0, y1], axis=2), y_all)
+        assert np.array_equal(last1, last_all)
+    # a nonzero start: one token by hand
+    inp1 = _slice_t(inp, 0, 1)
+    h0 = np.random.default_rng(37).standard_normal(last_all.shape)
+    _, last = oracle.scan_fwd(**inp1, initial_state=h0)
+    abar, bx, _ = _discretised(inp1, True)
+    np.testing.assert_allclose(last, abar[:, :, 0] * h0 + bx[:, :, 0], rtol=1e-14, atol=1e-15)
