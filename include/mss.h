@@ -76,9 +76,10 @@ enum mss_status {
     MSS_ERR_ALIAS = -9           /* an output overlaps an input */
 };
 
-/* Flags of mss_scan_fwd_ex. */
+/* Flags of mss_scan_fwd_ex / mss_scan_fwd_ex2. */
 #define MSS_FLAG_GENERAL_A 0x1u /* never use the fast path for A[d,n] = (n+1)*A[d,0] */
 #define MSS_FLAG_SIMPLE 0x2u    /* run the one-thread-per-channel reference kernel */
+#define MSS_FLAG_NO_SPLIT 0x4u  /* never split the sequence, even with a workspace */
 
 /*
  * mss_scan_fwd -- selective-scan forward pass over whole sequences.
@@ -112,6 +113,48 @@ MSS_API int mss_scan_fwd_ex(const void *u, const void *delta, const float *A, co
                     int softplus_flag, void *y, float *last_state,
                     int64_t batch, int64_t dim, int64_t dstate, int64_t seqlen,
                     int dtype, unsigned flags, void *stream);
+
+/*
+ * mss_scan_fwd_ex2 -- the forward pass with a starting state and an optional
+ * caller-owned workspace.
+ *
+ *   initial_state : [batch][dim][dstate] float, the state before the first
+ *                   token (NULL: zero, the pages' convention).  With it, a
+ *                   sequence can be run in pieces: passing one call's
+ *                   last_state as the next call's initial_state gives the
+ *                   same outputs as one call over the whole sequence.  It
+ *                   must not overlap last_state.
+ *   workspace, workspace_bytes : device memory the call may use for a
+ *                   sequence split (NULL / 0: none).  When the batch has too
+ *                   few channels to occupy the GPU (long sequences), the
+ *                   sequence is cut into segments that run in parallel: a
+ *                   first kernel reduces every segment but the last to its
+ *                   aggregate (the product of its transitions and its final
+ *                   state from zero, 2 * dstate floats per channel), a second
+ *                   runs all segments from their carried-in states.  The
+ *                   size the call would use is mss_scan_fwd_workspace_size;
+ *                   a smaller or NULL workspace disables the split.  The
+ *                   library never allocates; the contents of the workspace
+ *                   on return are unspecified.  Calls that share a workspace
+ *                   must not overlap in time.
+ *
+ * Every other argument, flag and rule is that of mss_scan_fwd_ex.
+ * seqlen == 0 copies initial_state (or zero) to last_state.
+ */
+MSS_API int mss_scan_fwd_ex2(const void *u, const void *delta, const float *A, const void *B,
+                             const void *C, const float *D, const void *z, const float *delta_bias,
+                             int softplus_flag, const float *initial_state, void *y, float *last_state,
+                             int64_t batch, int64_t dim, int64_t dstate, int64_t seqlen,
+                             int dtype, unsigned flags, void *workspace, int64_t workspace_bytes,
+                             void *stream);
+
+/*
+ * mss_scan_fwd_workspace_size -- bytes of workspace mss_scan_fwd_ex2 would use
+ * for these sizes on the current device (0: the sequence is not split), or a
+ * negative mss_status for invalid arguments.  Assumes 16-byte aligned rows.
+ */
+MSS_API int64_t mss_scan_fwd_workspace_size(int64_t batch, int64_t dim, int64_t dstate, int64_t seqlen,
+                                            int dtype, unsigned flags);
 
 /*
  * mss_state_update -- one decode token for every (batch, channel):

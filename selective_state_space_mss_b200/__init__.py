@@ -22,8 +22,8 @@ import threading
 
 import torch
 
-__all__ = ["scan_fwd", "state_update", "get_device_error", "library_path",
-           "FLAG_GENERAL_A", "FLAG_SIMPLE", "MssError", "load_library"]
+__all__ = ["scan_fwd", "state_update", "get_device_error", "library_path", "workspace_size",
+           "FLAG_GENERAL_A", "FLAG_SIMPLE", "FLAG_NO_SPLIT", "MssError", "load_library"]
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
 _LIB_PATH = os.path.join(_HERE, "libmss.so")
@@ -32,6 +32,7 @@ DTYPE_F32 = 0
 DTYPE_BF16 = 1
 FLAG_GENERAL_A = 0x1
 FLAG_SIMPLE = 0x2
+FLAG_NO_SPLIT = 0x4
 
 _lib = None
 _lock = threading.Lock()
@@ -65,6 +66,11 @@ def load_library():
             lib.mss_scan_fwd.argtypes = [vp, vp, fp, vp, vp, fp, vp, fp, i, vp, fp,
                                          i64, i64, i64, i64, i, vp]
             lib.mss_scan_fwd.restype = i
+            lib.mss_scan_fwd_ex2.argtypes = [vp, vp, fp, vp, vp, fp, vp, fp, i, fp, vp, fp,
+                                             i64, i64, i64, i64, i, u32, vp, i64, vp]
+            lib.mss_scan_fwd_ex2.restype = i
+            lib.mss_scan_fwd_workspace_size.argtypes = [i64, i64, i64, i64, i, u32]
+            lib.mss_scan_fwd_workspace_size.restype = i64
             lib.mss_state_update.argtypes = [fp, vp, vp, fp, vp, vp, fp, vp, fp, i, vp,
                                              i64, i64, i64, i, vp]
             lib.mss_state_update.restype = i
@@ -116,10 +122,28 @@ def _stream_handle(stream, device):
     return ctypes.c_void_p(s.cuda_stream)
 
 
+def workspace_size(batch, dim, dstate, seqlen, dtype=torch.bfloat16, flags=0, device=None) -> int:
+    """Bytes of workspace the forward pass would use to split the sequence
+    on `device` (0: no split)."""
+    code = DTYPE_BF16 if dtype == torch.bfloat16 else DTYPE_F32
+    dev = torch.device("cuda", torch.cuda.current_device()) if device is None else torch.device(device)
+    with torch.cuda.device(dev):
+        n = int(load_library().mss_scan_fwd_workspace_size(batch, dim, dstate, seqlen, code, int(flags)))
+    if n < 0:
+        raise MssError(n, "mss_scan_fwd_workspace_size")
+    return n
+
+
 def scan_fwd(u, delta, A, B, C, D=None, z=None, delta_bias=None, softplus=True,
-             y=None, last_state=None, want_last_state=True, flags=0, stream=None):
-    """Selective-scan forward pass (mss_scan_fwd_ex).  Returns (y, last_state);
-    last_state is None when want_last_state is False and none was given."""
+             y=None, last_state=None, want_last_state=True, initial_state=None,
+             workspace="auto", flags=0, stream=None):
+    """Selective-scan forward pass (mss_scan_fwd_ex2).  Returns (y, last_state);
+    last_state is None when want_last_state is False and none was given.
+
+    initial_state: [batch, dim, N] float32 state before the first token (None:
+    zero).  workspace: "auto" (the size the library asks for, allocated from
+    PyTorch's caching allocator), None (no sequence split), or a uint8 CUDA
+    tensor the call may use."""
     if not isinstance(u, torch.Tensor) or u.device.type != "cuda":
         raise ValueError("u must be a CUDA tensor (there is no CPU path)")
     if u.dim() != 3:
@@ -138,16 +162,25 @@ def scan_fwd(u, delta, A, B, C, D=None, z=None, delta_bias=None, softplus=True,
     _check(D, "D", (dim,), torch.float32, dev, optional=True)
     _check(z, "z", (batch, dim, L), dt, dev, optional=True)
     _check(delta_bias, "delta_bias", (dim,), torch.float32, dev, optional=True)
+    _check(initial_state, "initial_state", (batch, dim, N), torch.float32, dev, optional=True)
     if y is None:
         y = torch.empty((batch, dim, L), dtype=dt, device=dev)
     _check(y, "y", (batch, dim, L), dt, dev)
     if last_state is None and want_last_state:
         last_state = torch.empty((batch, dim, N), dtype=torch.float32, device=dev)
     _check(last_state, "last_state", (batch, dim, N), torch.float32, dev, optional=True)
-    rc = load_library().mss_scan_fwd_ex(
+    if isinstance(workspace, str):
+        if workspace != "auto":
+            raise ValueError("workspace must be 'auto', None or a uint8 CUDA tensor")
+        nbytes = workspace_size(batch, dim, N, L, dt, flags, dev)
+        workspace = torch.empty(nbytes, dtype=torch.uint8, device=dev) if nbytes > 0 else None
+    if workspace is not None:
+        _check(workspace, "workspace", (workspace.numel(),), torch.uint8, dev)
+    rc = load_library().mss_scan_fwd_ex2(
         _ptr(u), _ptr(delta), _ptr(A), _ptr(B), _ptr(C), _ptr(D), _ptr(z), _ptr(delta_bias),
-        int(bool(softplus)), _ptr(y), _ptr(last_state), batch, dim, N, L, code,
-        int(flags), _stream_handle(stream, dev))
+        int(bool(softplus)), _ptr(initial_state), _ptr(y), _ptr(last_state), batch, dim, N, L, code,
+        int(flags), _ptr(workspace), 0 if workspace is None else workspace.numel(),
+        _stream_handle(stream, dev))
     if rc != 0:
         raise MssError(rc, "mss_scan_fwd")
     return y, last_state

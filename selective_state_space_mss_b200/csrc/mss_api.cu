@@ -1,6 +1,7 @@
 // mss_api.cu -- the C ABI of libmss.so (declared in include/mss.h): argument
 // checks on the host, kernel choice, launches.  No allocation, no host
 // synchronisation on the forward and decode paths.
+#include <algorithm>
 #include <cstdint>
 #include <cstring>
 #include <mutex>
@@ -115,20 +116,56 @@ bool seq_eligible(const mss::ScanParams& p, int64_t N, int esz, unsigned flags) 
     return true;
 }
 
-template <typename T, int N, bool kGate, bool kSoftplus>
-int launch_seq_variant(const mss::SeqMaps& maps, const mss::ScanParams& p, unsigned flags, cudaStream_t stream) {
-    auto kern = mss::scan_fwd_seq_kernel<T, N, kGate, kSoftplus>;
+template <typename T, int N, bool kGate, bool kSoftplus, bool kFold>
+int launch_seq_variant(const mss::SeqMaps& maps, const mss::ScanParams& p, unsigned flags, int segs,
+                       cudaStream_t stream) {
+    auto kern = mss::scan_fwd_seq_kernel<T, N, kGate, kSoftplus, kFold>;
     const int smem = mss::SeqLayout<T, N>::kSmemBytes;
     if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess)
         return MSS_ERR_CUDA;
     constexpr int rows = mss::SeqLayout<T, N>::kRows;
-    const dim3 grid(unsigned((p.dim + rows - 1) / rows), unsigned(p.batch));
+    const dim3 grid(unsigned((p.dim + rows - 1) / rows), unsigned(p.batch), unsigned(segs));
     kern<<<grid, 32, smem, stream>>>(maps, p, (flags & MSS_FLAG_GENERAL_A) ? 0 : 1);
     return launch_status();
 }
 
+// Sequence split for workloads with too few channels to occupy the GPU:
+// segments per sequence so that the full pass has about two warps per
+// scheduler without exceeding one wave.  1 = no split.
 template <typename T, int N>
-int launch_seq(const mss::ScanParams& p, unsigned flags, cudaStream_t stream) {
+int choose_segments(int64_t batch, int64_t dim, int64_t seqlen) {
+    using Ly = mss::SeqLayout<T, N>;
+    int dev = 0, sms = 0, occ = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess ||
+        cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
+        return 1;
+    auto kern = mss::scan_fwd_seq_kernel<T, N, true, true, false>;
+    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, Ly::kSmemBytes) != cudaSuccess ||
+        cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, kern, 32, Ly::kSmemBytes) != cudaSuccess || occ < 1)
+        return 1;
+    const int64_t ctas = batch * ((dim + Ly::kRows - 1) / Ly::kRows);
+    const int64_t slots = int64_t(occ) * sms;
+    const int64_t target = 2 * 4 * int64_t(sms);  // two warps per scheduler
+    const int64_t n_chunks = (seqlen + Ly::kChunk - 1) / Ly::kChunk;
+    int64_t n = std::min<int64_t>(slots / ctas, (target + ctas - 1) / ctas);
+    n = std::min<int64_t>(std::min<int64_t>(n, n_chunks), 64);
+    if (n < 2) return 1;
+    // equal segments of whole chunks
+    const int64_t seg_chunks = (n_chunks + n - 1) / n;
+    return int((n_chunks + seg_chunks - 1) / seg_chunks);
+}
+
+template <typename T, int N>
+int64_t seg_len_for(int64_t seqlen, int n_seg) {
+    using Ly = mss::SeqLayout<T, N>;
+    const int64_t n_chunks = (seqlen + Ly::kChunk - 1) / Ly::kChunk;
+    return ((n_chunks + n_seg - 1) / n_seg) * Ly::kChunk;
+}
+
+int64_t agg_bytes(int n_seg, int64_t rows, int64_t N) { return n_seg > 1 ? int64_t(n_seg - 1) * 2 * rows * N * 4 : 0; }
+
+template <typename T, int N>
+int launch_seq(mss::ScanParams p, unsigned flags, void* workspace, int64_t workspace_bytes, cudaStream_t stream) {
     constexpr int esz = int(sizeof(T));
     mss::SeqMaps maps;
     std::memset(&maps, 0, sizeof(maps));
@@ -139,17 +176,35 @@ int launch_seq(const mss::ScanParams& p, unsigned flags, cudaStream_t stream) {
         (p.z && !encode_rows(&maps.z, p.z, rows, p.seqlen, esz, br)) ||
         !encode_bc(&maps.B, p.B, p.batch, N, p.seqlen, esz) || !encode_bc(&maps.C, p.C, p.batch, N, p.seqlen, esz))
         return MSS_ERR_CUDA;
+    p.n_seg = 1;
+    p.seg_len = p.seqlen;
+    p.agg = nullptr;
+    if (!(flags & MSS_FLAG_NO_SPLIT) && workspace) {
+        const int n_seg = choose_segments<T, N>(p.batch, p.dim, p.seqlen);
+        if (n_seg > 1 && agg_bytes(n_seg, rows, N) <= workspace_bytes) {
+            p.n_seg = n_seg;
+            p.seg_len = seg_len_for<T, N>(p.seqlen, n_seg);
+            p.agg = static_cast<float*>(workspace);
+        }
+    }
+    if (p.n_seg > 1) {
+        // first pass: each segment but the last folds to its aggregates
+        const int rc = p.softplus ? launch_seq_variant<T, N, false, true, true>(maps, p, flags, p.n_seg - 1, stream)
+                                  : launch_seq_variant<T, N, false, false, true>(maps, p, flags, p.n_seg - 1, stream);
+        if (rc != MSS_OK) return rc;
+    }
     if (p.z)
-        return p.softplus ? launch_seq_variant<T, N, true, true>(maps, p, flags, stream)
-                          : launch_seq_variant<T, N, true, false>(maps, p, flags, stream);
-    return p.softplus ? launch_seq_variant<T, N, false, true>(maps, p, flags, stream)
-                      : launch_seq_variant<T, N, false, false>(maps, p, flags, stream);
+        return p.softplus ? launch_seq_variant<T, N, true, true, false>(maps, p, flags, p.n_seg, stream)
+                          : launch_seq_variant<T, N, true, false, false>(maps, p, flags, p.n_seg, stream);
+    return p.softplus ? launch_seq_variant<T, N, false, true, false>(maps, p, flags, p.n_seg, stream)
+                      : launch_seq_variant<T, N, false, false, false>(maps, p, flags, p.n_seg, stream);
 }
 
 template <typename T, int N>
-int launch_scan(const mss::ScanParams& p, unsigned flags, cudaStream_t stream) {
+int launch_scan(const mss::ScanParams& p, unsigned flags, void* workspace, int64_t workspace_bytes,
+                cudaStream_t stream) {
     if constexpr (N == 4 || N == 8 || N == 16) {
-        if (seq_eligible(p, N, int(sizeof(T)), flags)) return launch_seq<T, N>(p, flags, stream);
+        if (seq_eligible(p, N, int(sizeof(T)), flags)) return launch_seq<T, N>(p, flags, workspace, workspace_bytes, stream);
     }
     return launch_simple<T, N>(p, stream);
 }
@@ -176,14 +231,14 @@ const char* mss_strerror(int code) {
     }
 }
 
-int mss_scan_fwd_ex(const void* u, const void* delta, const float* A, const void* B,
-                    const void* C, const float* D, const void* z, const float* delta_bias,
-                    int softplus_flag, void* y, float* last_state,
-                    int64_t batch, int64_t dim, int64_t dstate, int64_t seqlen,
-                    int dtype, unsigned flags, void* stream) {
+int mss_scan_fwd_ex2(const void* u, const void* delta, const float* A, const void* B,
+                     const void* C, const float* D, const void* z, const float* delta_bias,
+                     int softplus_flag, const float* initial_state, void* y, float* last_state,
+                     int64_t batch, int64_t dim, int64_t dstate, int64_t seqlen,
+                     int dtype, unsigned flags, void* workspace, int64_t workspace_bytes, void* stream) {
     if (dtype != MSS_DTYPE_F32 && dtype != MSS_DTYPE_BF16) return MSS_ERR_DTYPE;
-    if (flags & ~(MSS_FLAG_GENERAL_A | MSS_FLAG_SIMPLE)) return MSS_ERR_FLAGS;
-    if (batch < 0 || dim < 0 || seqlen < 0) return MSS_ERR_SHAPE;
+    if (flags & ~(MSS_FLAG_GENERAL_A | MSS_FLAG_SIMPLE | MSS_FLAG_NO_SPLIT)) return MSS_ERR_FLAGS;
+    if (batch < 0 || dim < 0 || seqlen < 0 || workspace_bytes < 0) return MSS_ERR_SHAPE;
     if (!valid_n(dstate)) return MSS_ERR_UNSUPPORTED_N;
     const int64_t esz = dtype == MSS_DTYPE_BF16 ? 2 : 4;
     int64_t rows, seq_elems, seq_bytes, bc_elems, bc_bytes, st_elems, st_bytes;
@@ -198,40 +253,76 @@ int mss_scan_fwd_ex(const void* u, const void* delta, const float* A, const void
     const void* io[] = {u, delta, B, C, z, y};
     for (const void* p : io)
         if (p && !aligned(p, size_t(esz))) return MSS_ERR_ALIGN;
-    const void* fp[] = {A, D, delta_bias, last_state};
+    const void* fp[] = {A, D, delta_bias, last_state, initial_state, workspace};
     for (const void* p : fp)
         if (p && !aligned(p, 4)) return MSS_ERR_ALIGN;
-    // outputs must not overlap inputs
-    const void* in_seq[] = {u, delta, z};
-    for (const void* p : in_seq)
-        if (overlaps(y, seq_bytes, p, seq_bytes) || overlaps(last_state, st_bytes, p, seq_bytes))
-            return MSS_ERR_ALIAS;
-    const void* in_bc[] = {B, C};
-    for (const void* p : in_bc)
-        if (overlaps(y, seq_bytes, p, bc_bytes) || overlaps(last_state, st_bytes, p, bc_bytes))
-            return MSS_ERR_ALIAS;
-    const int64_t n_param_bytes = dim * 4;
-    const void* params[] = {D, delta_bias};
-    for (const void* p : params)
-        if (overlaps(y, seq_bytes, p, n_param_bytes) || overlaps(last_state, st_bytes, p, n_param_bytes))
-            return MSS_ERR_ALIAS;
-    if (overlaps(y, seq_bytes, A, dim * dstate * 4) || overlaps(last_state, st_bytes, A, dim * dstate * 4) ||
-        overlaps(y, seq_bytes, last_state, st_bytes))
-        return MSS_ERR_ALIAS;
+    // outputs (y, last_state, workspace) must not overlap inputs or each other
+    const int64_t ws = workspace ? workspace_bytes : 0;
+    struct Range { const void* p; int64_t n; };
+    const Range outs[] = {{y, seq_bytes}, {last_state, st_bytes}, {workspace, ws}};
+    const Range ins[] = {{u, seq_bytes}, {delta, seq_bytes}, {z, seq_bytes}, {B, bc_bytes}, {C, bc_bytes},
+                         {A, dim * dstate * 4}, {D, dim * 4}, {delta_bias, dim * 4},
+                         {initial_state, st_bytes}};
+    for (const Range& o : outs) {
+        for (const Range& i : ins)
+            if (overlaps(o.p, o.n, i.p, i.n)) return MSS_ERR_ALIAS;
+        for (const Range& o2 : outs)
+            if (&o != &o2 && overlaps(o.p, o.n, o2.p, o2.n)) return MSS_ERR_ALIAS;
+    }
 
     cudaStream_t s = static_cast<cudaStream_t>(stream);
     if (seqlen == 0) {
-        if (last_state && cudaMemsetAsync(last_state, 0, size_t(st_bytes), s) != cudaSuccess)
-            return MSS_ERR_CUDA;
+        // no tokens: the final state is the starting state
+        if (last_state) {
+            const cudaError_t e = initial_state
+                ? cudaMemcpyAsync(last_state, initial_state, size_t(st_bytes), cudaMemcpyDeviceToDevice, s)
+                : cudaMemsetAsync(last_state, 0, size_t(st_bytes), s);
+            if (e != cudaSuccess) return MSS_ERR_CUDA;
+        }
         return MSS_OK;
     }
-    mss::ScanParams p{u, delta, A, B, C, D, z, delta_bias, y, last_state,
-                      batch, dim, seqlen, softplus_flag ? 1 : 0};
+    mss::ScanParams p{};
+    p.u = u; p.delta = delta; p.A = A; p.B = B; p.C = C; p.D = D; p.z = z; p.delta_bias = delta_bias;
+    p.y = y; p.last_state = last_state; p.batch = batch; p.dim = dim; p.seqlen = seqlen;
+    p.softplus = softplus_flag ? 1 : 0; p.initial_state = initial_state;
+    p.agg = nullptr; p.seg_len = seqlen; p.n_seg = 1;
     return with_n(dstate, [&](auto nc) {
         constexpr int N = decltype(nc)::value;
-        return dtype == MSS_DTYPE_BF16 ? launch_scan<bf16_t, N>(p, flags, s)
-                                       : launch_scan<float, N>(p, flags, s);
+        return dtype == MSS_DTYPE_BF16 ? launch_scan<bf16_t, N>(p, flags, workspace, ws, s)
+                                       : launch_scan<float, N>(p, flags, workspace, ws, s);
     });
+}
+
+int64_t mss_scan_fwd_workspace_size(int64_t batch, int64_t dim, int64_t dstate, int64_t seqlen, int dtype,
+                                    unsigned flags) {
+    if (dtype != MSS_DTYPE_F32 && dtype != MSS_DTYPE_BF16) return MSS_ERR_DTYPE;
+    if (flags & ~(MSS_FLAG_GENERAL_A | MSS_FLAG_SIMPLE | MSS_FLAG_NO_SPLIT)) return MSS_ERR_FLAGS;
+    if (batch < 0 || dim < 0 || seqlen < 0) return MSS_ERR_SHAPE;
+    if (!valid_n(dstate)) return MSS_ERR_UNSUPPORTED_N;
+    int64_t rows;
+    if (!mul_ok(batch, dim, &rows) || rows > (int64_t(1) << 40)) return MSS_ERR_SHAPE;
+    const int64_t esz = dtype == MSS_DTYPE_BF16 ? 2 : 4;
+    if (rows == 0 || seqlen == 0 || (flags & (MSS_FLAG_SIMPLE | MSS_FLAG_NO_SPLIT)) ||
+        (dstate != 4 && dstate != 8 && dstate != 16) || (seqlen * esz) % 16 != 0)
+        return 0;
+    return with_n(dstate, [&](auto nc) -> int64_t {
+        constexpr int N = decltype(nc)::value;
+        if constexpr (N == 4 || N == 8 || N == 16) {
+            const int n_seg = dtype == MSS_DTYPE_BF16 ? choose_segments<bf16_t, N>(batch, dim, seqlen)
+                                                      : choose_segments<float, N>(batch, dim, seqlen);
+            return agg_bytes(n_seg, rows, N);
+        }
+        return 0;
+    });
+}
+
+int mss_scan_fwd_ex(const void* u, const void* delta, const float* A, const void* B,
+                    const void* C, const float* D, const void* z, const float* delta_bias,
+                    int softplus_flag, void* y, float* last_state,
+                    int64_t batch, int64_t dim, int64_t dstate, int64_t seqlen,
+                    int dtype, unsigned flags, void* stream) {
+    return mss_scan_fwd_ex2(u, delta, A, B, C, D, z, delta_bias, softplus_flag, nullptr, y, last_state,
+                            batch, dim, dstate, seqlen, dtype, flags, nullptr, 0, stream);
 }
 
 int mss_scan_fwd(const void* u, const void* delta, const float* A, const void* B,
@@ -239,8 +330,8 @@ int mss_scan_fwd(const void* u, const void* delta, const float* A, const void* B
                  int softplus_flag, void* y, float* last_state,
                  int64_t batch, int64_t dim, int64_t dstate, int64_t seqlen,
                  int dtype, void* stream) {
-    return mss_scan_fwd_ex(u, delta, A, B, C, D, z, delta_bias, softplus_flag, y, last_state,
-                           batch, dim, dstate, seqlen, dtype, 0u, stream);
+    return mss_scan_fwd_ex2(u, delta, A, B, C, D, z, delta_bias, softplus_flag, nullptr, y, last_state,
+                            batch, dim, dstate, seqlen, dtype, 0u, nullptr, 0, stream);
 }
 
 int mss_state_update(float* state, const void* u, const void* delta, const float* A,

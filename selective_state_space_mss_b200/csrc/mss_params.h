@@ -18,6 +18,13 @@ struct ScanParams {
     float* last_state;        // may be null
     int64_t batch, dim, seqlen;
     int softplus;
+    const float* initial_state;  // [batch, dim, N] state before the first token, or null (zero)
+    // Sequence split: n_seg segments of seg_len tokens (the last may be
+    // shorter); agg holds the per-segment aggregates [n_seg-1][2][batch*dim][N]
+    // (exp(A * sum of steps), then the segment's final state from zero).
+    float* agg;
+    int64_t seg_len;
+    int n_seg;
 };
 
 struct StepParams {

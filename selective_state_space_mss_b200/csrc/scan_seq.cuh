@@ -131,6 +131,7 @@ struct LaneConst {
 
 // Per-token scalars of one channel.
 struct TokenPre {
+    float dt;    // Delta
     float du;    // Delta * u
     float r;     // exp(Delta * A[d,0]) with the fast transition, else Delta
     float skip;  // D * u
@@ -143,6 +144,7 @@ __device__ __forceinline__ TokenPre token_pre(float ut, float dr, float zt, cons
     const float s = dr + cc.bias;
     float dt = s;
     if constexpr (kSoftplus) dt = kFast ? softplus_fast(s) : softplus_precise(s);
+    tp.dt = dt;
     tp.du = dt * ut;
     tp.r = kGeo ? ex2_approx(dt * cc.a0) : dt;
     tp.skip = cc.D * ut;
@@ -150,14 +152,11 @@ __device__ __forceinline__ TokenPre token_pre(float ut, float dr, float zt, cons
     return tp;
 }
 
-// One token for this lane's states: h <- Abar (.) h + Delta*u*B, returns the
-// partial read-out over these states.  `row` holds the lane's
-// (B_n, B_n+2, C_n, C_n+2) chunks; `rdt` is r (fast transition) or Delta.
+// The transition pairs (Abar_n, Abar_n+2) of this lane's states for one
+// token; `rdt` is r = exp(Delta A[d,0]) (fast transition) or Delta.
 template <int N, bool kFast, bool kGeo>
-__device__ __forceinline__ float token_states(float2 (&h)[N / 4], const float4 (&row)[N / 4], float du, float rdt,
-                                              int half, const LaneConst<N>& cc) {
+__device__ __forceinline__ void transition(float2 (&dA)[N / 4], float rdt, int half, const LaneConst<N>& cc) {
     constexpr int P = N / 4;
-    float2 dA[P];
     if constexpr (kGeo) {
         // states n = half + 4i and n + 2: Abar = (r^(n+1), r^(n+3))
         const float r = rdt, r2 = r * r;
@@ -183,19 +182,36 @@ __device__ __forceinline__ float token_states(float2 (&h)[N / 4], const float4 (
             }
         }
     }
+}
+
+// One token for this lane's states: h <- Abar (.) h + Delta*u*B; with the
+// read-out (kReadout) returns the partial C . h over these states.  `row`
+// holds the lane's (B_n, B_n+2, C_n, C_n+2) chunks.
+template <int N, bool kFast, bool kGeo, bool kReadout = true>
+__device__ __forceinline__ float token_states(float2 (&h)[N / 4], const float4 (&row)[N / 4], float du, float rdt,
+                                              int half, const LaneConst<N>& cc) {
+    constexpr int P = N / 4;
+    float2 dA[P];
+    transition<N, kFast, kGeo>(dA, rdt, half, cc);
     const float2 du2 = make_float2(du, du);
     float2 acc0 = make_float2(0.f, 0.f), acc1 = make_float2(0.f, 0.f);
 #pragma unroll
     for (int i = 0; i < P; ++i) {
         const float4 v = row[i];  // (B_n, B_n+2, C_n, C_n+2)
         h[i] = __ffma2_rn(dA[i], h[i], __fmul2_rn(du2, make_float2(v.x, v.y)));
-        if (i & 1)
-            acc1 = __ffma2_rn(make_float2(v.z, v.w), h[i], acc1);
-        else
-            acc0 = __ffma2_rn(make_float2(v.z, v.w), h[i], acc0);
+        if constexpr (kReadout) {
+            if (i & 1)
+                acc1 = __ffma2_rn(make_float2(v.z, v.w), h[i], acc1);
+            else
+                acc0 = __ffma2_rn(make_float2(v.z, v.w), h[i], acc0);
+        }
     }
-    const float2 acc = __fadd2_rn(acc0, acc1);
-    return acc.x + acc.y;
+    if constexpr (kReadout) {
+        const float2 acc = __fadd2_rn(acc0, acc1);
+        return acc.x + acc.y;
+    } else {
+        return 0.f;
+    }
 }
 
 // Unpack the tokens of one 8-byte piece of a row (bf16: 4, fp32: 2).
@@ -221,7 +237,11 @@ __device__ __forceinline__ uint2 pack8(const float (&v)[8 / sizeof(T)]) {
     }
 }
 
-template <typename T, int N, bool kGeo, bool kGate, bool kSoftplus>
+// kFold: the first pass of a split sequence -- run the segment from a zero
+// state without read-out and record its aggregates (exp(A * sum of steps) and
+// the final state); otherwise the full pass, starting from the caller's state
+// carried over the earlier segments' aggregates.
+template <typename T, int N, bool kGeo, bool kGate, bool kSoftplus, bool kFold>
 __device__ __forceinline__ void scan_seq_body(const SeqMaps& maps, const ScanParams& p, uint8_t* smem,
                                               uint64_t* bars, const LaneConst<N>& cc, bool valid, int64_t row) {
     using Ly = SeqLayout<T, N>;
@@ -237,15 +257,19 @@ __device__ __forceinline__ void scan_seq_body(const SeqMaps& maps, const ScanPar
     const int b = blockIdx.y;
     const int row0 = int(int64_t(b) * p.dim + int64_t(blockIdx.x) * Ly::kRows);
     const int64_t L = p.seqlen;
-    const int n_chunks = int((L + Ly::kChunk - 1) / Ly::kChunk);
-    const int n_groups = int(L / V);       // L is a multiple of V
+    const int seg = blockIdx.z;
+    const int64_t t_begin = int64_t(seg) * p.seg_len;  // a multiple of the chunk
+    const int64_t Ls = (L - t_begin < p.seg_len) ? L - t_begin : p.seg_len;
+    const int n_chunks = int((Ls + Ly::kChunk - 1) / Ly::kChunk);
+    const int n_groups = int(Ls / V);      // L and seg_len are multiples of V
+    const size_t rows_total = size_t(p.batch) * size_t(p.dim);
     float* bcf = reinterpret_cast<float*>(smem + S * Ly::kStageBytes);
     const uint32_t stage_tx = uint32_t((kGate ? 3 : 2) * Ly::kTile + 2 * Ly::kBCTile);
 
     auto issue = [&](int chunk) {
         uint8_t* st = smem + (chunk % S) * Ly::kStageBytes;
         uint64_t* bar = bars + chunk % S;
-        const int x = chunk * Ly::kChunk;
+        const int x = int(t_begin) + chunk * Ly::kChunk;
         mbar_arrive_expect_tx(bar, stage_tx);
         tma_load_2d(st, &maps.u, x, row0, bar);
         tma_load_2d(st + Ly::kTile, &maps.delta, x, row0, bar);
@@ -275,10 +299,27 @@ __device__ __forceinline__ void scan_seq_body(const SeqMaps& maps, const ScanPar
     if (lane == 0) {
         for (int c = 0; c < S && c < n_chunks; ++c) issue(c);
     }
+    // starting state: zero for a fold; otherwise the caller's state carried
+    // over the aggregates of the earlier segments
     float2 h[P];
 #pragma unroll
     for (int i = 0; i < P; ++i) h[i] = make_float2(0.f, 0.f);
-    T* yrow = static_cast<T*>(p.y) + row * L + HV * half;
+    if constexpr (!kFold) {
+        if (p.initial_state) {
+            const float* h0 = p.initial_state + row * N + half;
+#pragma unroll
+            for (int i = 0; i < P; ++i) h[i] = make_float2(h0[4 * i], h0[4 * i + 2]);
+        }
+        for (int s2 = 0; s2 < seg; ++s2) {
+            const float* ga = p.agg + ((size_t(s2) * 2) * rows_total + size_t(row)) * N + half;
+            const float* gb = ga + rows_total * N;
+#pragma unroll
+            for (int i = 0; i < P; ++i)
+                h[i] = __ffma2_rn(make_float2(ga[4 * i], ga[4 * i + 2]), h[i], make_float2(gb[4 * i], gb[4 * i + 2]));
+        }
+    }
+    float dsum = 0.f, dcomp = 0.f;  // fold: compensated sum of this lane's steps
+    T* yrow = static_cast<T*>(p.y) + row * L + t_begin + HV * half;
     const float4* my_bcf = reinterpret_cast<const float4*>(bcf) + half * P;  // this lane's chunks of a row
     constexpr int kRowF4 = Ly::kBCfRow / 4;
 
@@ -338,9 +379,9 @@ __device__ __forceinline__ void scan_seq_body(const SeqMaps& maps, const ScanPar
             const bool mine = (t / HV) == half;
             const float du = mine ? own[t % HV].du : pdu[t % HV];
             const float rdt = mine ? own[t % HV].r : prd[t % HV];
-            acc[t] = token_states<N, kFast, kGeo>(h, rowv, du, rdt, half, cc);
+            acc[t] = token_states<N, kFast, kGeo, !kFold>(h, rowv, du, rdt, half, cc);
             // the previous group's outputs, once their shuffles have had time
-            if (t == 1 && pend_at >= 0) {
+            if (!kFold && t == 1 && pend_at >= 0) {
                 float yv[HV];
 #pragma unroll
                 for (int k = 0; k < HV; ++k) yv[k] = (pkeep[k] + precv[k] + pskip[k]) * pgate[k];
@@ -352,17 +393,28 @@ __device__ __forceinline__ void scan_seq_body(const SeqMaps& maps, const ScanPar
                 nxt[t - kPre0] = token_pre<kFast, kGeo, kGate, kSoftplus>(uv[t - kPre0], dv[t - kPre0],
                                                                             kGate ? zv[t - kPre0] : 0.f, cc);
         }
-        // this group's read-out: transpose-reduce (lane half h finishes tokens
-        // [h*HV, h*HV + HV)); finished after token 1 of the next group
+        if constexpr (kFold) {
+            // compensated (Kahan) sum of this lane's steps
 #pragma unroll
-        for (int k = 0; k < HV; ++k) {
-            const float send = half ? acc[k] : acc[HV + k];
-            pkeep[k] = half ? acc[HV + k] : acc[k];
-            precv[k] = __shfl_xor_sync(0xffffffffu, send, 1);
-            pskip[k] = own[k].skip;
-            pgate[k] = own[k].gate;
+            for (int k = 0; k < HV; ++k) {
+                const float yk = own[k].dt - dcomp;
+                const float tk = dsum + yk;
+                dcomp = (tk - dsum) - yk;
+                dsum = tk;
+            }
+        } else {
+            // this group's read-out: transpose-reduce (lane half h finishes
+            // tokens [h*HV, h*HV + HV)); finished after token 1 of the next group
+#pragma unroll
+            for (int k = 0; k < HV; ++k) {
+                const float send = half ? acc[k] : acc[HV + k];
+                pkeep[k] = half ? acc[HV + k] : acc[k];
+                precv[k] = __shfl_xor_sync(0xffffffffu, send, 1);
+                pskip[k] = own[k].skip;
+                pgate[k] = own[k].gate;
+            }
+            pend_at = int64_t(g) * V;
         }
-        pend_at = int64_t(g) * V;
         // hand over the next group's scalars
 #pragma unroll
         for (int k = 0; k < HV; ++k) {
@@ -389,6 +441,29 @@ __device__ __forceinline__ void scan_seq_body(const SeqMaps& maps, const ScanPar
             for (int i = 0; i < P; ++i) nrow[i] = my_bcf[i];
         }
     }
+    if constexpr (kFold) {
+        // aggregates of this segment: exp(A_n * sum of its steps) and the state
+        // it ends in from zero
+        const float tot = (dsum + __shfl_xor_sync(0xffffffffu, dsum, 1)) -
+                          (dcomp + __shfl_xor_sync(0xffffffffu, dcomp, 1));
+        if (valid) {
+            float* ga = p.agg + ((size_t(seg) * 2) * rows_total + size_t(row)) * N + half;
+            float* gb = ga + rows_total * N;
+#pragma unroll
+            for (int i = 0; i < P; ++i) {
+                float2 a;
+                if constexpr (kFast)
+                    a = make_float2(ex2_approx(cc.a2[i].x * tot), ex2_approx(cc.a2[i].y * tot));
+                else
+                    a = make_float2(expf(cc.a2[i].x * tot), expf(cc.a2[i].y * tot));
+                ga[4 * i] = a.x;
+                ga[4 * i + 2] = a.y;
+                gb[4 * i] = h[i].x;
+                gb[4 * i + 2] = h[i].y;
+            }
+        }
+        return;
+    }
     // the last group's outputs
     if (pend_at >= 0) {
         float yv[HV];
@@ -396,7 +471,7 @@ __device__ __forceinline__ void scan_seq_body(const SeqMaps& maps, const ScanPar
         for (int k = 0; k < HV; ++k) yv[k] = (pkeep[k] + precv[k] + pskip[k]) * pgate[k];
         if (valid) *reinterpret_cast<uint2*>(yrow + pend_at) = pack8<T>(yv);
     }
-    if (valid && p.last_state) {
+    if (valid && p.last_state && seg == p.n_seg - 1) {
         float* ls = p.last_state + row * N + half;
 #pragma unroll
         for (int i = 0; i < P; ++i) {
@@ -406,11 +481,12 @@ __device__ __forceinline__ void scan_seq_body(const SeqMaps& maps, const ScanPar
     }
 }
 
-// grid = (ceil(dim / 16), batch), block = 32 threads, dynamic shared memory
-// SeqLayout<T, N>::kSmemBytes.  Requirements checked by the host: N in
-// {4, 8, 16}; L * sizeof(T) a multiple of 16; u, delta, z, B, C, y 16-byte
-// aligned.
-template <typename T, int N, bool kGate, bool kSoftplus>
+// grid = (ceil(dim / 16), batch, segments), block = 32 threads, dynamic
+// shared memory SeqLayout<T, N>::kSmemBytes.  A fold launch covers segments
+// 0 .. n_seg-2, the full pass all n_seg (after the fold has completed).
+// Requirements checked by the host: N in {4, 8, 16}; L * sizeof(T) a multiple
+// of 16; u, delta, z, B, C, y 16-byte aligned; seg_len a multiple of the chunk.
+template <typename T, int N, bool kGate, bool kSoftplus, bool kFold>
 __global__ void __launch_bounds__(32) scan_fwd_seq_kernel(const __grid_constant__ SeqMaps maps, ScanParams p,
                                                           int allow_geo) {
     using Ly = SeqLayout<T, N>;
@@ -459,11 +535,11 @@ __global__ void __launch_bounds__(32) scan_fwd_seq_kernel(const __grid_constant_
 
     if constexpr (kFast) {
         if (geo) {
-            scan_seq_body<T, N, true, kGate, kSoftplus>(maps, p, smem, bars, cc, valid, row);
+            scan_seq_body<T, N, true, kGate, kSoftplus, kFold>(maps, p, smem, bars, cc, valid, row);
             return;
         }
     }
-    scan_seq_body<T, N, false, kGate, kSoftplus>(maps, p, smem, bars, cc, valid, row);
+    scan_seq_body<T, N, false, kGate, kSoftplus, kFold>(maps, p, smem, bars, cc, valid, row);
 }
 
 }  // namespace mss

@@ -33,7 +33,7 @@ __global__ void __launch_bounds__(128) scan_fwd_simple_kernel(ScanParams p) {
 #pragma unroll
     for (int n = 0; n < N; ++n) {
         a[n] = p.A[d * N + n];
-        h[n] = 0.f;
+        h[n] = p.initial_state ? p.initial_state[row * N + n] : 0.f;
     }
     const float bias = p.delta_bias ? p.delta_bias[d] : 0.f;
     const float Dd = p.D ? p.D[d] : 0.f;

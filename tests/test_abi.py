@@ -120,3 +120,43 @@ def test_binding_refuses_cpu_tensors():
     x = torch.zeros(1, 2, 3)
     with pytest.raises(ValueError, match="CUDA"):
         mss.scan_fwd(x, x, torch.zeros(2, 4), x, x)
+
+
+def test_ex2_and_workspace_argument_errors(lib):
+    codes = _enum("mss_status")
+    v = ctypes.c_void_p
+
+    def ex2(**kw):
+        a = dict(u=P, delta=P + 0x1000000, A=P + 0x2000000, B=P + 0x3000000, C=P + 0x4000000,
+                 h0=None, y=P + 0x5000000, last=None, ws=None, wsb=0, batch=2, dim=8, N=16, L=32,
+                 dtype=1, flags=0)
+        a.update(kw)
+        w = lambda x: v(x) if x is not None else None
+        return lib.mss_scan_fwd_ex2(w(a["u"]), w(a["delta"]), w(a["A"]), w(a["B"]), w(a["C"]), None, None,
+                                    None, 1, w(a["h0"]), w(a["y"]), w(a["last"]), a["batch"], a["dim"],
+                                    a["N"], a["L"], a["dtype"], a["flags"], w(a["ws"]), a["wsb"], None)
+
+    assert ex2(flags=0x40) == codes["MSS_ERR_FLAGS"]
+    assert ex2(wsb=-1) == codes["MSS_ERR_SHAPE"]
+    assert ex2(h0=P + 0x6000002) == codes["MSS_ERR_ALIGN"]
+    assert ex2(ws=P + 0x6000001, wsb=64) == codes["MSS_ERR_ALIGN"]
+    assert ex2(h0=P + 0x7000000, last=P + 0x7000000) == codes["MSS_ERR_ALIAS"]   # h0 on last_state
+    assert ex2(ws=P + 0x5000000, wsb=256) == codes["MSS_ERR_ALIAS"]              # workspace on y
+    assert ex2(ws=P + 0x2000000, wsb=256) == codes["MSS_ERR_ALIAS"]              # workspace on A
+    assert ex2(batch=0) == 0
+
+
+def test_workspace_size_queries(lib):
+    codes = _enum("mss_status")
+    lib.mss_scan_fwd_workspace_size.restype = ctypes.c_int64
+    q = lambda *a: lib.mss_scan_fwd_workspace_size(*a)
+    assert q(1, 16, 16, 4096, 7, 0) == codes["MSS_ERR_DTYPE"]
+    assert q(1, 16, 3, 4096, 1, 0) == codes["MSS_ERR_UNSUPPORTED_N"]
+    assert q(-1, 16, 16, 4096, 1, 0) == codes["MSS_ERR_SHAPE"]
+    assert q(1, 16, 16, 4096, 1, 0x80) == codes["MSS_ERR_FLAGS"]
+    # no split: scalar kernel, split disabled, nothing to do, rows not 16-byte multiples
+    assert q(1, 16, 16, 4096, 1, 0x2) == 0
+    assert q(1, 16, 16, 4096, 1, 0x4) == 0
+    assert q(1, 16, 16, 0, 1, 0) == 0
+    assert q(1, 16, 16, 4097, 1, 0) == 0
+    assert q(1, 16, 2, 4096, 1, 0) == 0

@@ -242,3 +242,69 @@ def test_repeated_calls_are_deterministic():
     yb, lb = mss.scan_fwd(**d)
     torch.cuda.synchronize()
     assert torch.equal(ya, yb) and torch.equal(la, lb)
+
+
+# ---------------------------------------------------------------------------
+# Starting state and the sequence split
+
+def _inputs_dev_and_oracle(batch, dim, N, L, dtype, seed):
+    inp = gen.scan_inputs(batch, dim, N, L, dtype, seed=seed, d_skip="normal")
+    return inp, device_inputs(inp, DEV)
+
+
+@pytest.mark.parametrize("dtype", ["f32", "bf16"])
+def test_initial_state_matches_oracle_and_chains(dtype):
+    batch, dim, N, L = 2, 48, 16, 512
+    inp, d = _inputs_dev_and_oracle(batch, dim, N, L, dtype, 41)
+    h0 = np.random.default_rng(42).standard_normal((batch, dim, N)).astype(np.float32)
+    y, last = mss.scan_fwd(**d, initial_state=torch.from_numpy(h0).to(DEV))
+    y_ref, last_ref = oracle.scan_fwd(inp["u"].values, inp["delta"].values, inp["A"], inp["B"].values,
+                                      inp["C"].values, D=inp["D"], z=inp["z"].values,
+                                      delta_bias=inp["delta_bias"], initial_state=h0.astype(np.float64))
+    assert_close(to_numpy(y), y_ref, dtype, "y from a starting state")
+    assert_close(to_numpy(last), last_ref, dtype, "last_state from a starting state")
+    # two calls chained through last_state equal one call
+    L0 = 192
+    part = lambda t0, t1: {k: (v[..., t0:t1].contiguous() if k in ("u", "delta", "z", "B", "C") else v)
+                           for k, v in d.items()}
+    y_all, last_all = mss.scan_fwd(**d)
+    y0, last0 = mss.scan_fwd(**part(0, L0))
+    y1, last1 = mss.scan_fwd(**part(L0, L), initial_state=last0)
+    torch.cuda.synchronize()
+    assert_close(to_numpy(torch.cat([y0, y1], dim=2)), to_numpy(y_all).astype(np.float64), dtype, "chained y")
+    assert_close(to_numpy(last1), to_numpy(last_all).astype(np.float64), dtype, "chained last_state")
+
+
+SPLIT_SHAPES = [(1, 16, 16, 4096, "bf16"), (2, 40, 16, 4096 + 448, "bf16"), (1, 32, 8, 8192, "bf16"),
+                (1, 16, 4, 2048, "bf16"), (1, 16, 16, 2048, "f32"), (3, 16, 16, 1024 + 8, "bf16")]
+
+
+@pytest.mark.parametrize("shape", SPLIT_SHAPES, ids=lambda s: "x".join(map(str, s)))
+@pytest.mark.parametrize("with_h0", [False, True])
+def test_sequence_split_matches_oracle(shape, with_h0):
+    batch, dim, N, L, dtype = shape
+    assert mss.workspace_size(batch, dim, N, L, torch.bfloat16 if dtype == "bf16" else torch.float32) > 0
+    inp, d = _inputs_dev_and_oracle(batch, dim, N, L, dtype, 50 + L + N)
+    h0 = np.random.default_rng(51).standard_normal((batch, dim, N)).astype(np.float32) if with_h0 else None
+    h0d = torch.from_numpy(h0).to(DEV) if with_h0 else None
+    y, last = mss.scan_fwd(**d, initial_state=h0d)                      # split (auto workspace)
+    y_ns, last_ns = mss.scan_fwd(**d, initial_state=h0d, workspace=None)  # not split
+    torch.cuda.synchronize()
+    assert mss.get_device_error() == 0
+    y_ref, last_ref = oracle.scan_fwd(inp["u"].values, inp["delta"].values, inp["A"], inp["B"].values,
+                                      inp["C"].values, D=inp["D"], z=inp["z"].values,
+                                      delta_bias=inp["delta_bias"],
+                                      initial_state=None if h0 is None else h0.astype(np.float64))
+    assert_close(to_numpy(y), y_ref, dtype, f"{shape} split y")
+    assert_close(to_numpy(last), last_ref, dtype, f"{shape} split last_state")
+    assert_close(to_numpy(y_ns), y_ref, dtype, f"{shape} unsplit y")
+    # outside the split's first segment only rounding differs from the unsplit pass
+    assert_close(to_numpy(y), to_numpy(y_ns).astype(np.float64), dtype, f"{shape} split vs unsplit")
+
+
+def test_zero_length_copies_initial_state():
+    inp, d = _inputs_dev_and_oracle(2, 4, 16, 0, "bf16", 3)
+    h0 = torch.randn(2, 4, 16, device=DEV)
+    _, last = mss.scan_fwd(**d, initial_state=h0)
+    torch.cuda.synchronize()
+    assert torch.equal(last, h0)
