@@ -73,7 +73,8 @@ enum mss_status {
     MSS_ERR_CUDA = -6,           /* a CUDA call failed (launch or device query) */
     MSS_ERR_DEVICE_TIMEOUT = -7, /* a bounded wait inside a kernel gave up */
     MSS_ERR_FLAGS = -8,          /* unknown bits in `flags` */
-    MSS_ERR_ALIAS = -9           /* an output overlaps an input */
+    MSS_ERR_ALIAS = -9,          /* an output overlaps an input */
+    MSS_ERR_SCRATCH = -10        /* mss_scan_fwd_noalloc: the split needs more than its fixed scratch */
 };
 
 /* Flags of mss_scan_fwd_ex / mss_scan_fwd_ex2. */
@@ -155,6 +156,45 @@ MSS_API int mss_scan_fwd_ex2(const void *u, const void *delta, const float *A, c
  */
 MSS_API int64_t mss_scan_fwd_workspace_size(int64_t batch, int64_t dim, int64_t dstate, int64_t seqlen,
                                             int dtype, unsigned flags);
+
+/*
+ * mss_scan_fwd_noalloc -- mss_scan_fwd_ex2 for callers that cannot allocate
+ * device memory.  The pages have no counterpart: this is an interface
+ * convenience.
+ *
+ * Some callers have no way to get device memory of their own -- a C program
+ * that is only handed its input and output buffers, a plug-in whose host
+ * framework owns all device allocations, a serving loop that must not
+ * allocate after start-up -- and so cannot pass mss_scan_fwd_ex2 a
+ * workspace.  This entry point takes no workspace: when the sequence is
+ * split, the aggregates live in a fixed scratch array of
+ * mss_scan_fwd_noalloc_scratch_bytes() bytes (4 MiB) that is part of the
+ * library image; every GPU that loads the library holds it until the process
+ * exits.  Nothing here allocates (no cudaMalloc, no allocating library call).
+ *
+ *   - Sizes whose split would need more scratch than that are rejected with
+ *     MSS_ERR_SCRATCH before anything is launched (mss_scan_fwd_workspace_size
+ *     gives the need; MSS_FLAG_NO_SPLIT avoids it).
+ *   - The first call on a device looks up the scratch's device address
+ *     (cudaGetSymbolAddress, with that device current) and caches it; make
+ *     that first call before any stream capture on that device.
+ *   - Every call on a device shares the one array, which keeps the last
+ *     call's contents.  Nothing in it needs to start at zero: each call's
+ *     first kernel writes every aggregate its second kernel reads.  Calls that
+ *     overlap on the GPU (other streams, other threads) race on it and must be
+ *     serialised by the caller.
+ *
+ * Arguments, flags and results are those of mss_scan_fwd_ex2 without the
+ * workspace pair.
+ */
+MSS_API int mss_scan_fwd_noalloc(const void *u, const void *delta, const float *A, const void *B,
+                                 const void *C, const float *D, const void *z, const float *delta_bias,
+                                 int softplus_flag, const float *initial_state, void *y, float *last_state,
+                                 int64_t batch, int64_t dim, int64_t dstate, int64_t seqlen,
+                                 int dtype, unsigned flags, void *stream);
+
+/* Size in bytes of mss_scan_fwd_noalloc's fixed scratch (per device). */
+MSS_API int64_t mss_scan_fwd_noalloc_scratch_bytes(void);
 
 /*
  * mss_state_update -- one decode token for every (batch, channel):

@@ -227,6 +227,7 @@ const char* mss_strerror(int code) {
         case MSS_ERR_DEVICE_TIMEOUT: return "a bounded wait inside a kernel gave up";
         case MSS_ERR_FLAGS: return "unknown bits in flags";
         case MSS_ERR_ALIAS: return "an output overlaps an input";
+        case MSS_ERR_SCRATCH: return "the sequence split needs more than the library's fixed scratch holds";
         default: return "unknown status code";
     }
 }
@@ -406,5 +407,64 @@ int mss_get_device_error(void* stream) {
     }
     return MSS_OK;
 }
+
+}  // extern "C"
+
+// ---------------------------------------------------------------------------
+// Forward pass for callers that cannot allocate device memory.
+//
+// Some callers have no way to obtain device memory of their own: a plain C
+// program that is only handed the input and output buffers, a plug-in whose
+// host framework owns every device allocation, a serving loop that must not
+// allocate once it has started.  mss_scan_fwd_noalloc gives them the sequence
+// split without a workspace argument: its scratch is the fixed array below,
+// part of the library image, which every GPU that loads the library holds
+// until the process exits.
+
+namespace {
+
+constexpr int64_t kStaticScratchBytes = int64_t(4) << 20;  // 4 MiB per device
+constexpr int kMaxDevices = 64;
+
+// The scratch itself.  In host code this name is only a stand-in for the
+// symbol, never a device address: kernels get the address that
+// cudaGetSymbolAddress returns for the current device.
+static __device__ __align__(256) float g_mss_static_scratch[kStaticScratchBytes / sizeof(float)];
+
+// Device address of the scratch on the current device, looked up once per
+// device (with that device current) and cached; nullptr on failure.
+void* static_scratch_address() {
+    static std::mutex mu;
+    static void* addr[kMaxDevices] = {};
+    int dev = -1;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return nullptr;
+    std::lock_guard<std::mutex> lock(mu);
+    if (!addr[dev]) {
+        void* p = nullptr;
+        if (cudaGetSymbolAddress(&p, g_mss_static_scratch) != cudaSuccess) return nullptr;
+        addr[dev] = p;
+    }
+    return addr[dev];
+}
+
+}  // namespace
+
+extern "C" {
+
+int mss_scan_fwd_noalloc(const void* u, const void* delta, const float* A, const void* B,
+                         const void* C, const float* D, const void* z, const float* delta_bias,
+                         int softplus_flag, const float* initial_state, void* y, float* last_state,
+                         int64_t batch, int64_t dim, int64_t dstate, int64_t seqlen,
+                         int dtype, unsigned flags, void* stream) {
+    const int64_t need = mss_scan_fwd_workspace_size(batch, dim, dstate, seqlen, dtype, flags);
+    if (need < 0) return int(need);
+    if (need > kStaticScratchBytes) return MSS_ERR_SCRATCH;
+    void* scratch = nullptr;
+    if (need > 0 && !(scratch = static_scratch_address())) return MSS_ERR_CUDA;
+    return mss_scan_fwd_ex2(u, delta, A, B, C, D, z, delta_bias, softplus_flag, initial_state, y, last_state,
+                            batch, dim, dstate, seqlen, dtype, flags, scratch, need, stream);
+}
+
+int64_t mss_scan_fwd_noalloc_scratch_bytes(void) { return kStaticScratchBytes; }
 
 }  // extern "C"
