@@ -57,10 +57,10 @@ def _load():
             lib = ctypes.CDLL(path)
             f, d, i64, i = (ctypes.POINTER(ctypes.c_float), ctypes.POINTER(ctypes.c_double),
                             ctypes.c_int64, ctypes.c_int)
-            lib.mss_oracle_scan_fwd.argtypes = [f, f, f, f, f, f, f, f, i, d, d, d,
+            lib.mss_oracle_scan_fwd.argtypes = [f, f, f, f, f, f, f, f, i, i, d, d, d,
                                                 i64, i64, i64, i64, i]
             lib.mss_oracle_scan_fwd.restype = i
-            lib.mss_oracle_state_update.argtypes = [d, f, f, f, f, f, f, f, f, i, d,
+            lib.mss_oracle_state_update.argtypes = [d, f, f, f, f, f, f, f, f, i, i, d,
                                                     i64, i64, i64, i]
             lib.mss_oracle_state_update.restype = i
             lib.mss_oracle_recurrence.argtypes = [d, d, d, i64, i64, d, d]
@@ -101,12 +101,13 @@ def silu(z: float) -> float:
 
 
 def scan_fwd(u, delta, A, B, C, D=None, z=None, delta_bias=None, softplus_flag=True,
-             initial_state=None, nthreads=None):
+             initial_state=None, zoh_input=False, nthreads=None):
     """Selective-scan forward pass in fp64.
 
     u, delta, z: [batch, dim, L]; A: [dim, N]; B, C: [batch, N, L];
     D, delta_bias: [dim]; initial_state: [batch, dim, N] (the state before
-    the first token; None for zero).  Values are taken as fp32 (bf16 inputs
+    the first token; None for zero); zoh_input: exact zero-order-hold input
+    matrix (e^{Delta A} - 1)/A * B instead of the Euler Delta * B.  Values are taken as fp32 (bf16 inputs
     must already be widened, which is exact); initial_state as fp64.
     Returns (y [batch, dim, L] fp64, last_state [batch, dim, N] fp64).
     """
@@ -132,7 +133,7 @@ def scan_fwd(u, delta, A, B, C, D=None, z=None, delta_bias=None, softplus_flag=T
     y = np.empty((batch, dim, L), dtype=np.float64)
     last = np.empty((batch, dim, N), dtype=np.float64)
     rc = _load().mss_oracle_scan_fwd(
-        u_p, d_p, A_p, B_p, C_p, D_p, z_p, b_p, int(bool(softplus_flag)),
+        u_p, d_p, A_p, B_p, C_p, D_p, z_p, b_p, int(bool(softplus_flag)), int(bool(zoh_input)),
         _dptr(h0) if h0 is not None else None, _dptr(y), _dptr(last), batch, dim, N, L,
         default_threads() if nthreads is None else int(nthreads))
     if rc != 0:
@@ -142,7 +143,7 @@ def scan_fwd(u, delta, A, B, C, D=None, z=None, delta_bias=None, softplus_flag=T
 
 
 def state_update(state, u, delta, A, B, C, D=None, z=None, delta_bias=None,
-                 softplus_flag=True, nthreads=None):
+                 softplus_flag=True, zoh_input=False, nthreads=None):
     """One decode step in fp64.
 
     state: [batch, dim, N] (fp64, updated in place and returned);
@@ -164,7 +165,7 @@ def state_update(state, u, delta, A, B, C, D=None, z=None, delta_bias=None,
     y = np.empty((batch, dim), dtype=np.float64)
     rc = _load().mss_oracle_state_update(
         _dptr(state), u_p, d_p, A_p, B_p, C_p, D_p, z_p, b_p, int(bool(softplus_flag)),
-        _dptr(y), batch, dim, N,
+        int(bool(zoh_input)), _dptr(y), batch, dim, N,
         default_threads() if nthreads is None else int(nthreads))
     if rc != 0:
         raise RuntimeError(f"mss_oracle_state_update failed with code {rc}")

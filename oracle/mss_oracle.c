@@ -22,7 +22,11 @@
  *     formula; "Paper: Mamba" course page, Objectives, zero-order hold].
  *   - Input matrix by the Euler rule Bbar = Delta*B (the course page lists
  *     Euler as the alternative to the exact ZOH input matrix); so the input
- *     term is Bbar x = Delta * B_t * u_t.
+ *     term is Bbar x = Delta * B_t * u_t.  On request (zoh_input), the exact
+ *     zero-order-hold input matrix instead:
+ *     Bbar = (Delta A)^{-1} (e^{Delta A} - I) Delta B = (e^{Delta A} - 1)/A * B
+ *     per state ("Mamba" paper review, section "SSM"; "Paper: Mamba",
+ *     Objectives), written with expm1 and with its limit Delta*B at A = 0.
  *   - Selective recurrence, state zero before the first token, update then
  *     read out:  h_t = Abar_t (.) h_{t-1} + Bbar_t x_t ,  y_t = C_t . h_t
  *     ["Mamba" paper review, section "SSM", discrete recurrence; "Exercises",
@@ -117,7 +121,7 @@ typedef struct {
     /* inputs, layouts as documented at mss_oracle_scan_fwd */
     const float *u, *delta, *A, *B, *C, *D, *z, *bias;
     const double *initial_state;
-    int softplus_flag;
+    int softplus_flag, zoh_input;
     double *y, *last_state;
     int64_t batch, dim, N, L;
     /* rows [row_begin, row_end) of the flattened (batch, dim) index */
@@ -126,8 +130,9 @@ typedef struct {
 } scan_job;
 
 /* Discretise one token of one channel: Delta from the raw value, then
- * Abar[n] = exp(Delta*A[n]) and Bbar x[n] = Delta * B[n] * u. */
-static double discretise(double delta_raw, double bias, int softplus_flag,
+ * Abar[n] = exp(Delta*A[n]) and Bbar x[n] = Delta * B[n] * u (Euler input
+ * rule) or ((e^{Delta A[n]} - 1)/A[n]) * B[n] * u (zero-order hold). */
+static double discretise(double delta_raw, double bias, int softplus_flag, int zoh_input,
                          const float *A_row, const float *B_bt, const float *C_bt,
                          int64_t L, int64_t N, double u,
                          double *abar, double *bx, double *c)
@@ -135,8 +140,10 @@ static double discretise(double delta_raw, double bias, int softplus_flag,
     double s = delta_raw + bias;
     double dt = softplus_flag ? mss_oracle_softplus(s) : s;
     for (int64_t n = 0; n < N; ++n) {
-        abar[n] = exp(dt * (double)A_row[n]);
-        bx[n] = dt * (double)B_bt[n * L] * u;
+        const double a = (double)A_row[n];
+        abar[n] = exp(dt * a);
+        const double w = (zoh_input && a != 0.0) ? expm1(dt * a) / a : dt;
+        bx[n] = w * (double)B_bt[n * L] * u;
         c[n] = (double)C_bt[n * L];
     }
     return dt;
@@ -167,7 +174,7 @@ static void *scan_rows(void *arg)
             h[n] = j->initial_state ? j->initial_state[row * N + n] : 0.0;
         for (int64_t t = 0; t < L; ++t) {
             const double ut = (double)u[t];
-            discretise((double)dr[t], bias, j->softplus_flag, A_row, B_b + t, C_b + t,
+            discretise((double)dr[t], bias, j->softplus_flag, j->zoh_input, A_row, B_b + t, C_b + t,
                        L, N, ut, abar, bx, c);
             double out = recurrence_step(h, abar, bx, c, N) + Dd * ut;
             if (z)
@@ -226,6 +233,7 @@ static int run_threaded(scan_job *proto, int64_t rows, int nthreads, void *(*fn)
  *   A           : [dim][N]          (negative reals for a stable system)
  *   B, C        : [batch][N][L]     (shared by all channels of a batch row)
  *   D, bias     : [dim]             (D, z, bias may be NULL)
+ *   zoh_input   : nonzero -> exact zero-order-hold input matrix, else Euler
  *   initial_state: [batch][dim][N]  fp64 state before the first token, or
  *                                   NULL for the zero state of the pages
  *   y           : [batch][dim][L]   fp64 output
@@ -235,16 +243,16 @@ static int run_threaded(scan_job *proto, int64_t rows, int nthreads, void *(*fn)
 int mss_oracle_scan_fwd(const float *u, const float *delta, const float *A,
                         const float *B, const float *C, const float *D,
                         const float *z, const float *delta_bias, int softplus_flag,
-                        const double *initial_state, double *y, double *last_state,
-                        int64_t batch, int64_t dim, int64_t dstate, int64_t seqlen,
-                        int nthreads)
+                        int zoh_input, const double *initial_state, double *y,
+                        double *last_state, int64_t batch, int64_t dim, int64_t dstate,
+                        int64_t seqlen, int nthreads)
 {
     if (!u || !delta || !A || !B || !C || !y)
         return ORACLE_EINVAL;
     if (batch < 0 || dim < 0 || dstate <= 0 || seqlen < 0)
         return ORACLE_EINVAL;
     scan_job proto = {u, delta, A, B, C, D, z, delta_bias, initial_state, softplus_flag,
-                      y, last_state, batch, dim, dstate, seqlen, 0, 0, ORACLE_OK};
+                      zoh_input, y, last_state, batch, dim, dstate, seqlen, 0, 0, ORACLE_OK};
     if (batch * dim == 0)
         return ORACLE_OK;
     return run_threaded(&proto, batch * dim, nthreads, scan_rows);
@@ -256,7 +264,7 @@ int mss_oracle_scan_fwd(const float *u, const float *delta, const float *A,
 typedef struct {
     double *state;
     const float *u, *delta, *A, *B, *C, *D, *z, *bias;
-    int softplus_flag;
+    int softplus_flag, zoh_input;
     double *y;
     int64_t dim, N;
     int64_t row_begin, row_end;
@@ -278,7 +286,7 @@ static void *step_rows(void *arg)
         const double ut = (double)j->u[row];
         const double bias = j->bias ? (double)j->bias[d] : 0.0;
         /* B, C of a decode step are [batch][N]: stride 1 between states. */
-        discretise((double)j->delta[row], bias, j->softplus_flag, j->A + d * N,
+        discretise((double)j->delta[row], bias, j->softplus_flag, j->zoh_input, j->A + d * N,
                    j->B + b * N, j->C + b * N, 1, N, ut, abar, bx, c);
         double out = recurrence_step(j->state + row * N, abar, bx, c, N);
         out += (j->D ? (double)j->D[d] : 0.0) * ut;
@@ -333,19 +341,20 @@ static int run_steps(step_job *proto, int64_t rows, int nthreads)
  *   A          : [dim][N]
  *   B, C       : [batch][N]
  *   D, bias    : [dim]  (D, z, bias may be NULL)
+ *   zoh_input  : nonzero -> exact zero-order-hold input matrix, else Euler
  *   y          : [batch][dim] fp64 output
  */
 int mss_oracle_state_update(double *state, const float *u, const float *delta,
                             const float *A, const float *B, const float *C,
                             const float *D, const float *z, const float *delta_bias,
-                            int softplus_flag, double *y,
+                            int softplus_flag, int zoh_input, double *y,
                             int64_t batch, int64_t dim, int64_t dstate, int nthreads)
 {
     if (!state || !u || !delta || !A || !B || !C || !y)
         return ORACLE_EINVAL;
     if (batch < 0 || dim < 0 || dstate <= 0)
         return ORACLE_EINVAL;
-    step_job proto = {state, u, delta, A, B, C, D, z, delta_bias, softplus_flag, y,
+    step_job proto = {state, u, delta, A, B, C, D, z, delta_bias, softplus_flag, zoh_input, y,
                       dim, dstate, 0, 0, ORACLE_OK};
     if (batch * dim == 0)
         return ORACLE_OK;

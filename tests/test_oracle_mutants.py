@@ -17,12 +17,16 @@ SRC = os.path.join(ROOT, "oracle", "mss_oracle.c")
 
 MUTANTS = {
     "drop_input_term": ("h[n] = abar[n] * h[n] + bx[n];", "h[n] = abar[n] * h[n];"),
-    "exponent_sign": ("abar[n] = exp(dt * (double)A_row[n]);", "abar[n] = exp(-dt * (double)A_row[n]);"),
+    "exponent_sign": ("abar[n] = exp(dt * a);", "abar[n] = exp(-dt * a);"),
     "readout_before_update": (
         "h[n] = abar[n] * h[n] + bx[n];\n        acc += c[n] * h[n];",
         "acc += c[n] * h[n];\n        h[n] = abar[n] * h[n] + bx[n];"),
-    "B_and_C_swapped": ("bx[n] = dt * (double)B_bt[n * L] * u;", "bx[n] = dt * (double)C_bt[n * L] * u;"),
-    "input_rule_without_step": ("bx[n] = dt * (double)B_bt[n * L] * u;", "bx[n] = (double)B_bt[n * L] * u;"),
+    "B_and_C_swapped": ("bx[n] = w * (double)B_bt[n * L] * u;", "bx[n] = w * (double)C_bt[n * L] * u;"),
+    "input_rule_without_step": ("expm1(dt * a) / a : dt;", "expm1(dt * a) / a : 1.0;"),
+    "zoh_ignored": ("? expm1(dt * a) / a : dt;", "? dt : dt;"),
+    "zoh_second_order_sign": ("? expm1(dt * a) / a : dt;", "? -expm1(-dt * a) / a : dt;"),
+    "zoh_zero_A_limit": ("(zoh_input && a != 0.0) ? expm1(dt * a) / a : dt;",
+                         "zoh_input ? (a != 0.0 ? expm1(dt * a) / a : 0.0) : dt;"),
     "softplus_drops_one": ("return log1p(exp(s));", "return log(exp(s));"),
     "softplus_positive_branch": ("return s + log1p(exp(-s));", "return log1p(exp(-s));"),
     "bias_dropped": ("double s = delta_raw + bias;", "double s = delta_raw;"),

@@ -439,3 +439,99 @@ def test_initial_state_chains_forward_passes():
     _, last = oracle.scan_fwd(**inp1, initial_state=h0)
     abar, bx, _ = _discretised(inp1, True)
     np.testing.assert_allclose(last, abar[:, :, 0] * h0 + bx[:, :, 0], rtol=1e-14, atol=1e-15)
+
+
+# --------------------------------------------------------------------------
+# Exact zero-order-hold input matrix ("Mamba" paper review, section "SSM":
+# Bbar = (Delta A)^{-1} (exp(Delta A) - I) Delta B; "Paper: Mamba", Objectives)
+
+def _rk4_hold(h0, A, b_u, dt, substeps):
+    """Integrate h' = A h + b_u (A diagonal, b_u held constant) over a step of
+    length dt with classical fourth-order Runge-Kutta: the continuous system the
+    discretisation samples, solved without its closed form."""
+    h = np.array(h0, dtype=np.float64)
+    k = dt / substeps
+    f = lambda x: A * x + b_u
+    for _ in range(substeps):
+        k1 = f(h)
+        k2 = f(h + 0.5 * k * k1)
+        k3 = f(h + 0.5 * k * k2)
+        k4 = f(h + k * k3)
+        h = h + (k / 6.0) * (k1 + 2 * k2 + 2 * k3 + k4)
+    return h
+
+
+def test_zoh_input_solves_the_held_input_ode():
+    """With the input held over each step, the zero-order-hold discretisation is
+    the exact solution of the continuous system: every state and output of the
+    oracle equals a fine Runge-Kutta integration of h' = A h + B(t) u(t)."""
+    rng = np.random.default_rng(61)
+    L, N = 12, 5
+    A = np.array([[-3.0, -1.0, -0.25, 0.0, 0.5]], dtype=np.float32)
+    inp = dict(
+        u=rng.standard_normal((1, 1, L)).astype(np.float32),
+        delta=rng.uniform(0.05, 0.6, (1, 1, L)).astype(np.float32),
+        A=A,
+        B=rng.standard_normal((1, N, L)).astype(np.float32),
+        C=rng.standard_normal((1, N, L)).astype(np.float32),
+        D=np.array([0.7], dtype=np.float32),
+    )
+    y, last = oracle.scan_fwd(**inp, softplus_flag=False, zoh_input=True)
+    h = np.zeros(N)
+    a = A[0].astype(np.float64)
+    for t in range(L):
+        b_u = inp["B"][0, :, t].astype(np.float64) * float(inp["u"][0, 0, t])
+        h = _rk4_hold(h, a, b_u, float(inp["delta"][0, 0, t]), 400)
+        want = float(inp["C"][0, :, t].astype(np.float64) @ h) + float(inp["D"][0]) * float(inp["u"][0, 0, t])
+        assert abs(y[0, 0, t] - want) <= 1e-11 * (1 + abs(want)), t
+    np.testing.assert_allclose(last[0, 0], h, rtol=1e-11, atol=1e-12)
+    # the Euler rule differs from the exact solution at this step size
+    y_euler, _ = oracle.scan_fwd(**inp, softplus_flag=False)
+    assert np.max(np.abs(y_euler - y)) > 1e-2
+
+
+def test_zoh_input_small_step_limit():
+    """expm1(dt a)/a = dt (1 + dt a / 2 + O(dt^2)): for a small step the ZOH
+    input term exceeds the Euler one by the relative amount dt*a/2 (smaller for
+    a < 0), and at a = 0 the two coincide exactly."""
+    dt = 1e-3
+    A = [-2.0, -0.5, 0.0, 1.5]
+    inp = _impulse_inputs(A, [1.0, 1.0, 1.0, 1.0], [1.0, 1.0, 1.0, 1.0], dt, 1)
+    _, last_zoh = oracle.scan_fwd(**inp, softplus_flag=False, zoh_input=True)
+    _, last_euler = oracle.scan_fwd(**inp, softplus_flag=False)
+    dt32 = float(np.float32(dt))
+    for n, a in enumerate(A):
+        rel = last_zoh[0, 0, n] / last_euler[0, 0, n] - 1.0
+        assert abs(rel - dt32 * a / 2) <= (dt32 * a) ** 2 / 4 + 1e-15, (n, rel)
+    assert last_zoh[0, 0, 2] == last_euler[0, 0, 2] == dt32
+
+
+def test_zoh_input_zero_A_is_pure_integration():
+    """A = 0 (no decay): h' = B u, so after steps dt_1..dt_k of held input the
+    state is the sum of dt_i B_i u_i, under either input rule."""
+    rng = np.random.default_rng(62)
+    L = 9
+    inp = dict(
+        u=rng.standard_normal((1, 1, L)).astype(np.float32),
+        delta=rng.uniform(0.1, 2.0, (1, 1, L)).astype(np.float32),
+        A=np.zeros((1, 3), dtype=np.float32),
+        B=rng.standard_normal((1, 3, L)).astype(np.float32),
+        C=rng.standard_normal((1, 3, L)).astype(np.float32),
+    )
+    _, last = oracle.scan_fwd(**inp, softplus_flag=False, zoh_input=True)
+    want = np.sum(inp["B"][0].astype(np.float64) * inp["delta"][0, 0].astype(np.float64)
+                  * inp["u"][0, 0].astype(np.float64), axis=1)
+    np.testing.assert_allclose(last[0, 0], want, rtol=1e-13, atol=1e-14)
+
+
+def test_zoh_decode_steps_equal_forward():
+    """The decode update takes the same input rule as the forward pass."""
+    inp = _random_forward_inputs(63, L=24)
+    y, last = oracle.scan_fwd(**inp, zoh_input=True)
+    state = np.zeros_like(last)
+    for t in range(24):
+        step = {k: np.ascontiguousarray(inp[k][..., t]) for k in ("u", "delta", "z", "B", "C")}
+        yt, state = oracle.state_update(state, A=inp["A"], D=inp["D"], delta_bias=inp["delta_bias"],
+                                        zoh_input=True, **step)
+        assert np.array_equal(yt, y[..., t])
+    assert np.array_equal(state, last)
