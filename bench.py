@@ -323,7 +323,8 @@ def run_mss(args, rank, world, local_rank):
         mss.scan_fwd(**d, y=y, last_state=state, flags=flags)
         if ev is not None:
             ev[1].record(stream)
-        mss.state_update(state, A=d["A"], D=d["D"], delta_bias=d["delta_bias"], y=y1, **s1)
+        mss.state_update(state, A=d["A"], D=d["D"], delta_bias=d["delta_bias"], y=y1,
+                         flags=flags & mss.FLAG_ZOH_INPUT, **s1)
 
     launches_per_step = 2
     ct_per_step = w.batch * w.dim * w.seqlen + w.batch * w.dim
@@ -369,6 +370,7 @@ def run_mss(args, rank, world, local_rank):
     ms, fwd_ms, clocks = timed(0, k_clock, args.warmup, with_clocks=True)
     assert mss.get_device_error() == 0
     ms_gen, fwd_ms_gen, _ = timed(mss.FLAG_GENERAL_A, args.steps, args.warmup)
+    ms_zoh, fwd_ms_zoh, _ = timed(mss.FLAG_ZOH_INPUT, args.steps, args.warmup)
 
     # end to end through the public call with host buffers: pinned host inputs,
     # copies in, forward + decode token, results copied out, every step
@@ -436,6 +438,7 @@ def run_mss(args, rank, world, local_rank):
     alu_peak = alu_peak_ops(sm_max_mhz)
     fwd_avg = sum(fwd_ms) / len(fwd_ms)
     fwd_avg_gen = sum(fwd_ms_gen) / len(fwd_ms_gen)
+    fwd_avg_zoh = sum(fwd_ms_zoh) / len(fwd_ms_zoh)
     achieved = bytes_fwd / (fwd_avg * 1e-3) / 1e9
     achieved_gen = bytes_fwd / (fwd_avg_gen * 1e-3) / 1e9
     value = whole_job_rate(ct_per_step, world, args.steps, ms)
@@ -464,6 +467,10 @@ def run_mss(args, rank, world, local_rank):
         "general_A_path": {"fwd_ms_avg": fwd_avg_gen, "achieved_gbs": achieved_gen,
                            "frac": achieved_gen / peak,
                            "channel_tokens_per_s": w.batch * w.dim * w.seqlen / (fwd_avg_gen * 1e-3)},
+        "zoh_input_path": {"fwd_ms_avg": fwd_avg_zoh,
+                           "achieved_gbs": bytes_fwd / (fwd_avg_zoh * 1e-3) / 1e9,
+                           "frac": bytes_fwd / (fwd_avg_zoh * 1e-3) / 1e9 / peak,
+                           "channel_tokens_per_s": w.batch * w.dim * w.seqlen / (fwd_avg_zoh * 1e-3)},
         "decode": {"workload": gen.DECODE_WORKLOAD, "ms_per_token_median": dec_med,
                    "achieved_gbs": dec_bytes / (dec_med * 1e-3) / 1e9,
                    "frac": dec_bytes / (dec_med * 1e-3) / 1e9 / peak,

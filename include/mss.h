@@ -56,7 +56,7 @@
 extern "C" {
 #endif
 
-#define MSS_VERSION 10000 /* major*10000 + minor*100 + patch: 1.0.0 */
+#define MSS_VERSION 10100 /* major*10000 + minor*100 + patch: 1.1.0 */
 
 enum mss_dtype {
     MSS_DTYPE_F32 = 0,
@@ -77,10 +77,17 @@ enum mss_status {
     MSS_ERR_SCRATCH = -10        /* mss_scan_fwd_noalloc: the split needs more than its fixed scratch */
 };
 
-/* Flags of mss_scan_fwd_ex / mss_scan_fwd_ex2. */
+/* Flags of mss_scan_fwd_ex / mss_scan_fwd_ex2 / mss_scan_fwd_noalloc
+ * (MSS_FLAG_ZOH_INPUT also of mss_state_update_ex). */
 #define MSS_FLAG_GENERAL_A 0x1u /* never use the fast path for A[d,n] = (n+1)*A[d,0] */
 #define MSS_FLAG_SIMPLE 0x2u    /* run the one-thread-per-channel reference kernel */
 #define MSS_FLAG_NO_SPLIT 0x4u  /* never split the sequence, even with a workspace */
+/* Input matrix by the exact zero-order hold instead of the Euler rule:
+ * Bbar x = (exp(Delta A[d,n]) - 1) / A[d,n] * B[n] * u per state, with its
+ * limit Delta * B[n] * u at A[d,n] = 0 ("Mamba" paper review, section "SSM";
+ * "Paper: Mamba", Objectives).  The transition Abar = exp(Delta A) is the
+ * same under both rules. */
+#define MSS_FLAG_ZOH_INPUT 0x8u
 
 /*
  * mss_scan_fwd -- selective-scan forward pass over whole sequences.
@@ -215,6 +222,15 @@ MSS_API int mss_state_update(float *state, const void *u, const void *delta, con
                      const void *B, const void *C, const float *D, const void *z,
                      const float *delta_bias, int softplus_flag, void *y,
                      int64_t batch, int64_t dim, int64_t dstate, int dtype, void *stream);
+
+/* mss_state_update with `flags`: 0, or MSS_FLAG_ZOH_INPUT for the
+ * zero-order-hold input matrix (the rule the forward pass that produced the
+ * state used).  Other bits: MSS_ERR_FLAGS.  flags == 0 is mss_state_update. */
+MSS_API int mss_state_update_ex(float *state, const void *u, const void *delta, const float *A,
+                        const void *B, const void *C, const float *D, const void *z,
+                        const float *delta_bias, int softplus_flag, void *y,
+                        int64_t batch, int64_t dim, int64_t dstate, int dtype,
+                        unsigned flags, void *stream);
 
 /*
  * mss_get_device_error -- synchronises `stream`, then reports and clears the

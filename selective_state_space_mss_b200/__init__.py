@@ -23,7 +23,7 @@ import threading
 import torch
 
 __all__ = ["scan_fwd", "state_update", "get_device_error", "library_path", "workspace_size",
-           "FLAG_GENERAL_A", "FLAG_SIMPLE", "FLAG_NO_SPLIT", "MssError", "load_library"]
+           "FLAG_GENERAL_A", "FLAG_SIMPLE", "FLAG_NO_SPLIT", "FLAG_ZOH_INPUT", "MssError", "load_library"]
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
 _LIB_PATH = os.path.join(_HERE, "libmss.so")
@@ -33,6 +33,7 @@ DTYPE_BF16 = 1
 FLAG_GENERAL_A = 0x1
 FLAG_SIMPLE = 0x2
 FLAG_NO_SPLIT = 0x4
+FLAG_ZOH_INPUT = 0x8  # zero-order-hold input matrix (e^{Delta A} - 1)/A * B instead of Delta * B
 
 _lib = None
 _lock = threading.Lock()
@@ -74,6 +75,9 @@ def load_library():
             lib.mss_state_update.argtypes = [fp, vp, vp, fp, vp, vp, fp, vp, fp, i, vp,
                                              i64, i64, i64, i, vp]
             lib.mss_state_update.restype = i
+            lib.mss_state_update_ex.argtypes = [fp, vp, vp, fp, vp, vp, fp, vp, fp, i, vp,
+                                                i64, i64, i64, i, u32, vp]
+            lib.mss_state_update_ex.restype = i
             lib.mss_get_device_error.argtypes = [vp]
             lib.mss_get_device_error.restype = i
             lib.mss_strerror.argtypes = [i]
@@ -141,7 +145,8 @@ def scan_fwd(u, delta, A, B, C, D=None, z=None, delta_bias=None, softplus=True,
     last_state is None when want_last_state is False and none was given.
 
     initial_state: [batch, dim, N] float32 state before the first token (None:
-    zero).  workspace: "auto" (the size the library asks for, allocated from
+    zero).  flags: FLAG_* bits; FLAG_ZOH_INPUT selects the zero-order-hold
+    input matrix.  workspace: "auto" (the size the library asks for, allocated from
     PyTorch's caching allocator), None (no sequence split), or a uint8 CUDA
     tensor the call may use."""
     if not isinstance(u, torch.Tensor) or u.device.type != "cuda":
@@ -187,9 +192,9 @@ def scan_fwd(u, delta, A, B, C, D=None, z=None, delta_bias=None, softplus=True,
 
 
 def state_update(state, u, delta, A, B, C, D=None, z=None, delta_bias=None, softplus=True,
-                 y=None, stream=None):
-    """One decode token (mss_state_update); `state` is updated in place.
-    Returns y [batch, dim]."""
+                 y=None, flags=0, stream=None):
+    """One decode token (mss_state_update_ex); `state` is updated in place.
+    Returns y [batch, dim].  flags: 0 or FLAG_ZOH_INPUT."""
     if not isinstance(state, torch.Tensor) or state.device.type != "cuda":
         raise ValueError("state must be a CUDA tensor (there is no CPU path)")
     if state.dim() != 3:
@@ -209,9 +214,9 @@ def state_update(state, u, delta, A, B, C, D=None, z=None, delta_bias=None, soft
     if y is None:
         y = torch.empty((batch, dim), dtype=dt, device=dev)
     _check(y, "y", (batch, dim), dt, dev)
-    rc = load_library().mss_state_update(
+    rc = load_library().mss_state_update_ex(
         _ptr(state), _ptr(u), _ptr(delta), _ptr(A), _ptr(B), _ptr(C), _ptr(D), _ptr(z),
-        _ptr(delta_bias), int(bool(softplus)), _ptr(y), batch, dim, N, code,
+        _ptr(delta_bias), int(bool(softplus)), _ptr(y), batch, dim, N, code, int(flags),
         _stream_handle(stream, dev))
     if rc != 0:
         raise MssError(rc, "mss_state_update")

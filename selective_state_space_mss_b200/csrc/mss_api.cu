@@ -116,10 +116,10 @@ bool seq_eligible(const mss::ScanParams& p, int64_t N, int esz, unsigned flags) 
     return true;
 }
 
-template <typename T, int N, bool kGate, bool kSoftplus, bool kFold>
+template <typename T, int N, bool kGate, bool kSoftplus, bool kFold, bool kZoh>
 int launch_seq_variant(const mss::SeqMaps& maps, const mss::ScanParams& p, unsigned flags, int segs,
                        cudaStream_t stream) {
-    auto kern = mss::scan_fwd_seq_kernel<T, N, kGate, kSoftplus, kFold>;
+    auto kern = mss::scan_fwd_seq_kernel<T, N, kGate, kSoftplus, kFold, kZoh>;
     const int smem = mss::SeqLayout<T, N>::kSmemBytes;
     if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess)
         return MSS_ERR_CUDA;
@@ -139,7 +139,7 @@ int choose_segments(int64_t batch, int64_t dim, int64_t seqlen) {
     if (cudaGetDevice(&dev) != cudaSuccess ||
         cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
         return 1;
-    auto kern = mss::scan_fwd_seq_kernel<T, N, true, true, false>;
+    auto kern = mss::scan_fwd_seq_kernel<T, N, true, true, false, false>;
     if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, Ly::kSmemBytes) != cudaSuccess ||
         cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, kern, 32, Ly::kSmemBytes) != cudaSuccess || occ < 1)
         return 1;
@@ -162,7 +162,26 @@ int64_t seg_len_for(int64_t seqlen, int n_seg) {
     return ((n_chunks + n_seg - 1) / n_seg) * Ly::kChunk;
 }
 
+constexpr unsigned kScanFlags = MSS_FLAG_GENERAL_A | MSS_FLAG_SIMPLE | MSS_FLAG_NO_SPLIT | MSS_FLAG_ZOH_INPUT;
+
 int64_t agg_bytes(int n_seg, int64_t rows, int64_t N) { return n_seg > 1 ? int64_t(n_seg - 1) * 2 * rows * N * 4 : 0; }
+
+// The fold pass (split sequences only), then the full pass.
+template <typename T, int N, bool kZoh>
+int launch_seq_passes(const mss::SeqMaps& maps, const mss::ScanParams& p, unsigned flags, cudaStream_t stream) {
+    if (p.n_seg > 1) {
+        // first pass: each segment but the last folds to its aggregates
+        const int rc = p.softplus
+                           ? launch_seq_variant<T, N, false, true, true, kZoh>(maps, p, flags, p.n_seg - 1, stream)
+                           : launch_seq_variant<T, N, false, false, true, kZoh>(maps, p, flags, p.n_seg - 1, stream);
+        if (rc != MSS_OK) return rc;
+    }
+    if (p.z)
+        return p.softplus ? launch_seq_variant<T, N, true, true, false, kZoh>(maps, p, flags, p.n_seg, stream)
+                          : launch_seq_variant<T, N, true, false, false, kZoh>(maps, p, flags, p.n_seg, stream);
+    return p.softplus ? launch_seq_variant<T, N, false, true, false, kZoh>(maps, p, flags, p.n_seg, stream)
+                      : launch_seq_variant<T, N, false, false, false, kZoh>(maps, p, flags, p.n_seg, stream);
+}
 
 template <typename T, int N>
 int launch_seq(mss::ScanParams p, unsigned flags, void* workspace, int64_t workspace_bytes, cudaStream_t stream) {
@@ -187,17 +206,8 @@ int launch_seq(mss::ScanParams p, unsigned flags, void* workspace, int64_t works
             p.agg = static_cast<float*>(workspace);
         }
     }
-    if (p.n_seg > 1) {
-        // first pass: each segment but the last folds to its aggregates
-        const int rc = p.softplus ? launch_seq_variant<T, N, false, true, true>(maps, p, flags, p.n_seg - 1, stream)
-                                  : launch_seq_variant<T, N, false, false, true>(maps, p, flags, p.n_seg - 1, stream);
-        if (rc != MSS_OK) return rc;
-    }
-    if (p.z)
-        return p.softplus ? launch_seq_variant<T, N, true, true, false>(maps, p, flags, p.n_seg, stream)
-                          : launch_seq_variant<T, N, true, false, false>(maps, p, flags, p.n_seg, stream);
-    return p.softplus ? launch_seq_variant<T, N, false, true, false>(maps, p, flags, p.n_seg, stream)
-                      : launch_seq_variant<T, N, false, false, false>(maps, p, flags, p.n_seg, stream);
+    return p.zoh ? launch_seq_passes<T, N, true>(maps, p, flags, stream)
+                 : launch_seq_passes<T, N, false>(maps, p, flags, stream);
 }
 
 template <typename T, int N>
@@ -238,7 +248,7 @@ int mss_scan_fwd_ex2(const void* u, const void* delta, const float* A, const voi
                      int64_t batch, int64_t dim, int64_t dstate, int64_t seqlen,
                      int dtype, unsigned flags, void* workspace, int64_t workspace_bytes, void* stream) {
     if (dtype != MSS_DTYPE_F32 && dtype != MSS_DTYPE_BF16) return MSS_ERR_DTYPE;
-    if (flags & ~(MSS_FLAG_GENERAL_A | MSS_FLAG_SIMPLE | MSS_FLAG_NO_SPLIT)) return MSS_ERR_FLAGS;
+    if (flags & ~kScanFlags) return MSS_ERR_FLAGS;
     if (batch < 0 || dim < 0 || seqlen < 0 || workspace_bytes < 0) return MSS_ERR_SHAPE;
     if (!valid_n(dstate)) return MSS_ERR_UNSUPPORTED_N;
     const int64_t esz = dtype == MSS_DTYPE_BF16 ? 2 : 4;
@@ -287,6 +297,7 @@ int mss_scan_fwd_ex2(const void* u, const void* delta, const float* A, const voi
     p.y = y; p.last_state = last_state; p.batch = batch; p.dim = dim; p.seqlen = seqlen;
     p.softplus = softplus_flag ? 1 : 0; p.initial_state = initial_state;
     p.agg = nullptr; p.seg_len = seqlen; p.n_seg = 1;
+    p.zoh = (flags & MSS_FLAG_ZOH_INPUT) ? 1 : 0;
     return with_n(dstate, [&](auto nc) {
         constexpr int N = decltype(nc)::value;
         return dtype == MSS_DTYPE_BF16 ? launch_scan<bf16_t, N>(p, flags, workspace, ws, s)
@@ -297,7 +308,7 @@ int mss_scan_fwd_ex2(const void* u, const void* delta, const float* A, const voi
 int64_t mss_scan_fwd_workspace_size(int64_t batch, int64_t dim, int64_t dstate, int64_t seqlen, int dtype,
                                     unsigned flags) {
     if (dtype != MSS_DTYPE_F32 && dtype != MSS_DTYPE_BF16) return MSS_ERR_DTYPE;
-    if (flags & ~(MSS_FLAG_GENERAL_A | MSS_FLAG_SIMPLE | MSS_FLAG_NO_SPLIT)) return MSS_ERR_FLAGS;
+    if (flags & ~kScanFlags) return MSS_ERR_FLAGS;
     if (batch < 0 || dim < 0 || seqlen < 0) return MSS_ERR_SHAPE;
     if (!valid_n(dstate)) return MSS_ERR_UNSUPPORTED_N;
     int64_t rows;
@@ -339,7 +350,16 @@ int mss_state_update(float* state, const void* u, const void* delta, const float
                      const void* B, const void* C, const float* D, const void* z,
                      const float* delta_bias, int softplus_flag, void* y,
                      int64_t batch, int64_t dim, int64_t dstate, int dtype, void* stream) {
+    return mss_state_update_ex(state, u, delta, A, B, C, D, z, delta_bias, softplus_flag, y,
+                               batch, dim, dstate, dtype, 0u, stream);
+}
+
+int mss_state_update_ex(float* state, const void* u, const void* delta, const float* A,
+                        const void* B, const void* C, const float* D, const void* z,
+                        const float* delta_bias, int softplus_flag, void* y,
+                        int64_t batch, int64_t dim, int64_t dstate, int dtype, unsigned flags, void* stream) {
     if (dtype != MSS_DTYPE_F32 && dtype != MSS_DTYPE_BF16) return MSS_ERR_DTYPE;
+    if (flags & ~unsigned(MSS_FLAG_ZOH_INPUT)) return MSS_ERR_FLAGS;
     if (batch < 0 || dim < 0) return MSS_ERR_SHAPE;
     if (!valid_n(dstate)) return MSS_ERR_UNSUPPORTED_N;
     const int64_t esz = dtype == MSS_DTYPE_BF16 ? 2 : 4;
@@ -369,7 +389,8 @@ int mss_state_update(float* state, const void* u, const void* delta, const float
         overlaps(y, io_bytes, state, st_bytes))
         return MSS_ERR_ALIAS;
 
-    mss::StepParams p{state, u, delta, A, B, C, D, z, delta_bias, y, batch, dim, softplus_flag ? 1 : 0};
+    mss::StepParams p{state, u, delta, A, B, C, D, z, delta_bias, y, batch, dim, softplus_flag ? 1 : 0,
+                      (flags & MSS_FLAG_ZOH_INPUT) ? 1 : 0};
     cudaStream_t s = static_cast<cudaStream_t>(stream);
     const bool vec = aligned(state, 16) && aligned(A, 16);
     return with_n(dstate, [&](auto nc) {

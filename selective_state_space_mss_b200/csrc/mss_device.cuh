@@ -95,6 +95,29 @@ __device__ __forceinline__ float silu_fast(float z) {
 }
 
 // ---------------------------------------------------------------------------
+// Zero-order-hold input weight.  The exact discretisation of the input term
+// ("Mamba" paper review, section "SSM") is Bbar = (e^{Delta a} - 1)/a * B per
+// state, i.e. Delta * phi(Delta a) * B with phi(x) = (e^x - 1)/x.  Formed from
+// the already computed e = e^x as (e - 1)/a it loses |x|^-1 ulps to
+// cancellation, so below |x| = 1/8 the kernels use the Taylor series of phi
+// instead, 1 + x/2 + x^2/6 + x^3/24 + x^4/120, whose first omitted term is
+// under 5e-8 there; above it the cancellation costs less than 3 bits.  phi is
+// finite and positive everywhere and phi(0) = 1 gives the Euler weight Delta
+// at a = 0.
+
+constexpr float kZohTaylorMax = 0.125f;
+constexpr float kLn2 = 0.69314718055994531f;
+
+__device__ __forceinline__ float phi_taylor(float x) {
+    return fmaf(fmaf(fmaf(fmaf(x, 1.f / 120.f, 1.f / 24.f), x, 1.f / 6.f), x, 0.5f), x, 1.f);
+}
+
+// Delta * phi(x) with x = Delta * a and e = e^x: the weight of B * u.
+__device__ __forceinline__ float zoh_weight(float dt, float a, float x, float e) {
+    return fabsf(x) < kZohTaylorMax ? dt * phi_taylor(x) : (e - 1.f) / a;
+}
+
+// ---------------------------------------------------------------------------
 // Device error word: set by kernels whose bounded waits give up, read and
 // cleared by mss_get_device_error.  The library is built as a single
 // translation unit (mss_api.cu includes every kernel), so this is its only

@@ -25,6 +25,7 @@ struct ScanParams {
     float* agg;
     int64_t seg_len;
     int n_seg;
+    int zoh;  // input matrix: 0 Euler Delta*B, 1 zero-order hold (e^{Delta A} - 1)/A * B
 };
 
 struct StepParams {
@@ -40,6 +41,7 @@ struct StepParams {
     void* y;
     int64_t batch, dim;
     int softplus;
+    int zoh;  // as in ScanParams
 };
 
 }  // namespace mss

@@ -42,6 +42,16 @@
 // one ex2 per token and about one multiply per state.  fp32 io uses the
 // full-precision expf for every state.
 //
+// Input matrix.  By default the input term is the Euler Delta*u*B.  With
+// the zero-order hold (kZoh) the weight of state n is Delta*phi(Delta A_n),
+// phi(x) = (e^x - 1)/x.  On the general path it is formed per state from the
+// transition's exponential (zoh_weight: Taylor series near x = 0).  On the
+// fast transition A_n = (n+1) A_0 turns it into a geometric sum,
+// phi(Delta A_n) = phi(Delta A_0) * S_n / (n+1) with S_n = 1 + r + ... + r^n
+// (a sum of positive terms, so no cancellation): phi(Delta A_0) goes into the
+// per-token scalar, S_n costs one packed FMA per state pair, and 1/(n+1) is
+// folded into the fp32 C rows, the lanes keeping (n+1) h_n instead of h_n.
+//
 // Waits are bounded: a stage that does not arrive within ~2 s sets the
 // device error word (read by mss_get_device_error) and the CTA returns after
 // giving its other copies a bounded chance to land.
@@ -83,10 +93,13 @@ struct SeqLayout {
 // Rewrite the staged B and C tiles ([N][chunk] in the io type) as fp32 rows,
 // one per token: chunk p*N/4 + i holds (B_n, B_n+2, C_n, C_n+2) with
 // n = p + 4i, for the even (p = 0) and then the odd (p = 1) states.
-template <typename T, int N>
+// kScaleC: C_n is stored as C_n / (n+1) (zero-order hold on the fast
+// transition, where the lanes keep (n+1) h_n).
+template <typename T, int N, bool kScaleC>
 __device__ __forceinline__ void convert_bc(const uint8_t* btile, const uint8_t* ctile, float* bcf, int lane) {
     using Ly = SeqLayout<T, N>;
     constexpr int P = Ly::kPairs;
+    auto cs = [](int n) { return kScaleC ? 1.f / float(n + 1) : 1.f; };
     if constexpr (sizeof(T) == 2) {
         // lane l: tokens 2l and 2l+1 (one 32-bit word of each state row)
         float4* r0 = reinterpret_cast<float4*>(bcf + (2 * lane) * Ly::kBCfRow);
@@ -100,8 +113,9 @@ __device__ __forceinline__ void convert_bc(const uint8_t* btile, const uint8_t* 
                 const uint32_t b2 = *reinterpret_cast<const uint32_t*>(btile + (n + 2) * Ly::kRowBytes + 4 * lane);
                 const uint32_t c0 = *reinterpret_cast<const uint32_t*>(ctile + n * Ly::kRowBytes + 4 * lane);
                 const uint32_t c2 = *reinterpret_cast<const uint32_t*>(ctile + (n + 2) * Ly::kRowBytes + 4 * lane);
-                r0[p * P + i] = make_float4(bf16_lo(b0), bf16_lo(b2), bf16_lo(c0), bf16_lo(c2));
-                r1[p * P + i] = make_float4(bf16_hi(b0), bf16_hi(b2), bf16_hi(c0), bf16_hi(c2));
+                const float s0 = cs(n), s2 = cs(n + 2);
+                r0[p * P + i] = make_float4(bf16_lo(b0), bf16_lo(b2), s0 * bf16_lo(c0), s2 * bf16_lo(c2));
+                r1[p * P + i] = make_float4(bf16_hi(b0), bf16_hi(b2), s0 * bf16_hi(c0), s2 * bf16_hi(c2));
             }
         }
     } else {
@@ -115,7 +129,7 @@ __device__ __forceinline__ void convert_bc(const uint8_t* btile, const uint8_t* 
 #pragma unroll
             for (int i = 0; i < P; ++i) {
                 const int n = p + 4 * i;
-                r[p * P + i] = make_float4(bp[n * rs], bp[(n + 2) * rs], cp[n * rs], cp[(n + 2) * rs]);
+                r[p * P + i] = make_float4(bp[n * rs], bp[(n + 2) * rs], cs(n) * cp[n * rs], cs(n + 2) * cp[(n + 2) * rs]);
             }
         }
     }
@@ -127,18 +141,21 @@ struct LaneConst {
     float bias, D;
     float a0;          // A[d,0] * log2(e)                            (fast transition)
     float2 a2[N / 4];  // this lane's state pairs of A (times log2(e) for bf16 io)
+    float ia0;         // 1 / A[d,0]                  (zero-order hold, fast transition)
+    float2 ia[N / 4];  // 1 / A of this lane's state pairs (zero-order hold, general path)
 };
 
 // Per-token scalars of one channel.
 struct TokenPre {
     float dt;    // Delta
-    float du;    // Delta * u
+    float du;    // Delta * u; zero-order hold on the fast transition: Delta * u * phi(Delta A[d,0])
+    float u;     // u (zero-order hold, general path)
     float r;     // exp(Delta * A[d,0]) with the fast transition, else Delta
     float skip;  // D * u
     float gate;  // silu(z), or 1 without a gate
 };
 
-template <bool kFast, bool kGeo, bool kGate, bool kSoftplus, int N>
+template <bool kFast, bool kGeo, bool kGate, bool kSoftplus, bool kZoh, int N>
 __device__ __forceinline__ TokenPre token_pre(float ut, float dr, float zt, const LaneConst<N>& cc) {
     TokenPre tp;
     const float s = dr + cc.bias;
@@ -146,7 +163,17 @@ __device__ __forceinline__ TokenPre token_pre(float ut, float dr, float zt, cons
     if constexpr (kSoftplus) dt = kFast ? softplus_fast(s) : softplus_precise(s);
     tp.dt = dt;
     tp.du = dt * ut;
-    tp.r = kGeo ? ex2_approx(dt * cc.a0) : dt;
+    tp.u = ut;
+    if constexpr (kGeo) {
+        const float arg = dt * cc.a0;
+        tp.r = ex2_approx(arg);
+        if constexpr (kZoh) {
+            const float x0 = arg * kLn2;
+            tp.du = fabsf(x0) < kZohTaylorMax ? tp.du * phi_taylor(x0) : ut * ((tp.r - 1.f) * cc.ia0);
+        }
+    } else {
+        tp.r = dt;
+    }
     tp.skip = cc.D * ut;
     tp.gate = kGate ? (kFast ? silu_fast(zt) : silu_precise(zt)) : 1.f;
     return tp;
@@ -184,21 +211,66 @@ __device__ __forceinline__ void transition(float2 (&dA)[N / 4], float rdt, int h
     }
 }
 
-// One token for this lane's states: h <- Abar (.) h + Delta*u*B; with the
-// read-out (kReadout) returns the partial C . h over these states.  `row`
-// holds the lane's (B_n, B_n+2, C_n, C_n+2) chunks.
-template <int N, bool kFast, bool kGeo, bool kReadout = true>
+// Zero-order-hold weights of this lane's state pairs, multiplying B.  Fast
+// transition: the geometric sums S_n = 1 + r + ... + r^n (the rest of the
+// weight is in du and in the scaled C rows), from S_{n+4} = S_n + r^{n+1} S_3
+// and S_{n+8} = S_n + r^{n+1} S_7.  General path: Delta*u*phi(Delta A_n) per
+// state (du = Delta*u, uu = u, rdt = Delta).
+template <int N, bool kFast, bool kGeo>
+__device__ __forceinline__ void zoh_weights(float2 (&w)[N / 4], const float2 (&dA)[N / 4], float du, float uu,
+                                            float rdt, int half, const LaneConst<N>& cc) {
+    constexpr int P = N / 4;
+    if constexpr (kGeo) {
+        const float r = rdt, r2 = r * r;
+        const float s3 = (1.f + r) * (1.f + r2);
+        w[0] = half ? make_float2(1.f + r, s3) : make_float2(1.f, fmaf(r, r, 1.f + r));
+        if constexpr (P >= 2) w[1] = __ffma2_rn(dA[0], make_float2(s3, s3), w[0]);
+        if constexpr (P >= 4) {
+            const float s7 = s3 * fmaf(r2, r2, 1.f);
+            w[2] = __ffma2_rn(dA[0], make_float2(s7, s7), w[0]);
+            w[3] = __ffma2_rn(dA[1], make_float2(s7, s7), w[1]);
+        }
+    } else {
+        const float2 dt2 = make_float2(rdt, rdt), du2 = make_float2(du, du), u2 = make_float2(uu, uu);
+#pragma unroll
+        for (int i = 0; i < P; ++i) {
+            float2 x = __fmul2_rn(dt2, cc.a2[i]);
+            if constexpr (kFast) x = __fmul2_rn(x, make_float2(kLn2, kLn2));
+            float2 t = __ffma2_rn(x, make_float2(1.f / 120.f, 1.f / 120.f), make_float2(1.f / 24.f, 1.f / 24.f));
+            t = __ffma2_rn(t, x, make_float2(1.f / 6.f, 1.f / 6.f));
+            t = __ffma2_rn(t, x, make_float2(0.5f, 0.5f));
+            t = __fmul2_rn(du2, __ffma2_rn(t, x, make_float2(1.f, 1.f)));
+            const float2 big = __fmul2_rn(u2, __fmul2_rn(__fadd2_rn(dA[i], make_float2(-1.f, -1.f)), cc.ia[i]));
+            w[i] = make_float2(fabsf(x.x) < kZohTaylorMax ? t.x : big.x, fabsf(x.y) < kZohTaylorMax ? t.y : big.y);
+        }
+    }
+}
+
+// One token for this lane's states: h <- Abar (.) h + Bbar*u, Bbar*u =
+// Delta*u*B (Euler) or the zero-order hold (kZoh); with the read-out
+// (kReadout) returns the partial C . h over these states.  `row` holds the
+// lane's (B_n, B_n+2, C_n, C_n+2) chunks.
+template <int N, bool kFast, bool kGeo, bool kZoh, bool kReadout = true>
 __device__ __forceinline__ float token_states(float2 (&h)[N / 4], const float4 (&row)[N / 4], float du, float rdt,
-                                              int half, const LaneConst<N>& cc) {
+                                              float uu, int half, const LaneConst<N>& cc) {
     constexpr int P = N / 4;
     float2 dA[P];
     transition<N, kFast, kGeo>(dA, rdt, half, cc);
+    float2 w[P];
+    if constexpr (kZoh) zoh_weights<N, kFast, kGeo>(w, dA, du, uu, rdt, half, cc);
     const float2 du2 = make_float2(du, du);
     float2 acc0 = make_float2(0.f, 0.f), acc1 = make_float2(0.f, 0.f);
 #pragma unroll
     for (int i = 0; i < P; ++i) {
         const float4 v = row[i];  // (B_n, B_n+2, C_n, C_n+2)
-        h[i] = __ffma2_rn(dA[i], h[i], __fmul2_rn(du2, make_float2(v.x, v.y)));
+        float2 bu;
+        if constexpr (!kZoh)
+            bu = __fmul2_rn(du2, make_float2(v.x, v.y));
+        else if constexpr (kGeo)
+            bu = __fmul2_rn(w[i], __fmul2_rn(du2, make_float2(v.x, v.y)));
+        else
+            bu = __fmul2_rn(w[i], make_float2(v.x, v.y));
+        h[i] = __ffma2_rn(dA[i], h[i], bu);
         if constexpr (kReadout) {
             if (i & 1)
                 acc1 = __ffma2_rn(make_float2(v.z, v.w), h[i], acc1);
@@ -241,7 +313,7 @@ __device__ __forceinline__ uint2 pack8(const float (&v)[8 / sizeof(T)]) {
 // state without read-out and record its aggregates (exp(A * sum of steps) and
 // the final state); otherwise the full pass, starting from the caller's state
 // carried over the earlier segments' aggregates.
-template <typename T, int N, bool kGeo, bool kGate, bool kSoftplus, bool kFold>
+template <typename T, int N, bool kGeo, bool kGate, bool kSoftplus, bool kFold, bool kZoh>
 __device__ __forceinline__ void scan_seq_body(const SeqMaps& maps, const ScanParams& p, uint8_t* smem,
                                               uint64_t* bars, const LaneConst<N>& cc, bool valid, int64_t row) {
     using Ly = SeqLayout<T, N>;
@@ -251,6 +323,8 @@ __device__ __forceinline__ void scan_seq_body(const SeqMaps& maps, const ScanPar
     constexpr int HV = Ly::kHalf;          // tokens of a group this lane finishes
     constexpr int P = Ly::kPairs;
     constexpr int GPC = Ly::kChunk / V;    // groups per chunk
+    constexpr bool kZG = kZoh && kGeo;     // lanes keep (n+1) h_n, C rows hold C_n / (n+1)
+    constexpr bool kZU = kZoh && !kGeo;    // per-state weights need u of every token
     const int lane = threadIdx.x;
     const int half = lane & 1;
     const int ch = lane >> 1;
@@ -317,14 +391,26 @@ __device__ __forceinline__ void scan_seq_body(const SeqMaps& maps, const ScanPar
             for (int i = 0; i < P; ++i)
                 h[i] = __ffma2_rn(make_float2(ga[4 * i], ga[4 * i + 2]), h[i], make_float2(gb[4 * i], gb[4 * i + 2]));
         }
+        if constexpr (kZG) {
+#pragma unroll
+            for (int i = 0; i < P; ++i)
+                h[i] = __fmul2_rn(h[i], make_float2(float(half + 4 * i + 1), float(half + 4 * i + 3)));
+        }
     }
+    // the state as h_n (undoing the (n+1) scale of the zero-order hold)
+    auto state_out = [&](int i) -> float2 {
+        if constexpr (kZG)
+            return make_float2(h[i].x / float(half + 4 * i + 1), h[i].y / float(half + 4 * i + 3));
+        else
+            return h[i];
+    };
     float dsum = 0.f, dcomp = 0.f;  // fold: compensated sum of this lane's steps
     T* yrow = static_cast<T*>(p.y) + row * L + t_begin + HV * half;
     const float4* my_bcf = reinterpret_cast<const float4*>(bcf) + half * P;  // this lane's chunks of a row
     constexpr int kRowF4 = Ly::kBCfRow / 4;
 
     if (!wait_chunk(0)) return;
-    convert_bc<T, N>(smem + 3 * Ly::kTile, smem + 3 * Ly::kTile + Ly::kBCTile, bcf, lane);
+    convert_bc<T, N, kZG>(smem + 3 * Ly::kTile, smem + 3 * Ly::kTile + Ly::kBCTile, bcf, lane);
     __syncwarp();
 
     // Software pipeline across groups.  Carried into iteration g:
@@ -333,15 +419,16 @@ __device__ __forceinline__ void scan_seq_body(const SeqMaps& maps, const ScanPar
     //   nrow[]       group g's first B/C row
     //   the previous group's transpose-reduce (finished after token 1 of g)
     TokenPre own[HV];
-    float pdu[HV], prd[HV];
+    float pdu[HV], prd[HV], pu[HV];
     {
         float uv[HV], dv[HV], zv[HV];
         load_half(0, uv, dv, zv);
 #pragma unroll
         for (int k = 0; k < HV; ++k) {
-            own[k] = token_pre<kFast, kGeo, kGate, kSoftplus>(uv[k], dv[k], kGate ? zv[k] : 0.f, cc);
+            own[k] = token_pre<kFast, kGeo, kGate, kSoftplus, kZoh>(uv[k], dv[k], kGate ? zv[k] : 0.f, cc);
             pdu[k] = __shfl_xor_sync(0xffffffffu, own[k].du, 1);
             prd[k] = __shfl_xor_sync(0xffffffffu, own[k].r, 1);
+            if constexpr (kZU) pu[k] = __shfl_xor_sync(0xffffffffu, own[k].u, 1);
         }
     }
     float4 nrow[P];
@@ -379,7 +466,8 @@ __device__ __forceinline__ void scan_seq_body(const SeqMaps& maps, const ScanPar
             const bool mine = (t / HV) == half;
             const float du = mine ? own[t % HV].du : pdu[t % HV];
             const float rdt = mine ? own[t % HV].r : prd[t % HV];
-            acc[t] = token_states<N, kFast, kGeo, !kFold>(h, rowv, du, rdt, half, cc);
+            const float uu = kZU ? (mine ? own[t % HV].u : pu[t % HV]) : 0.f;
+            acc[t] = token_states<N, kFast, kGeo, kZoh, !kFold>(h, rowv, du, rdt, uu, half, cc);
             // the previous group's outputs, once their shuffles have had time
             if (!kFold && t == 1 && pend_at >= 0) {
                 float yv[HV];
@@ -390,8 +478,8 @@ __device__ __forceinline__ void scan_seq_body(const SeqMaps& maps, const ScanPar
             // the next group's scalars, spread over the middle tokens
             constexpr int kPre0 = V >= 8 ? 2 : 0;
             if (t >= kPre0 && t < kPre0 + HV)
-                nxt[t - kPre0] = token_pre<kFast, kGeo, kGate, kSoftplus>(uv[t - kPre0], dv[t - kPre0],
-                                                                            kGate ? zv[t - kPre0] : 0.f, cc);
+                nxt[t - kPre0] = token_pre<kFast, kGeo, kGate, kSoftplus, kZoh>(uv[t - kPre0], dv[t - kPre0],
+                                                                                  kGate ? zv[t - kPre0] : 0.f, cc);
         }
         if constexpr (kFold) {
             // compensated (Kahan) sum of this lane's steps
@@ -421,6 +509,7 @@ __device__ __forceinline__ void scan_seq_body(const SeqMaps& maps, const ScanPar
             own[k] = nxt[k];
             pdu[k] = __shfl_xor_sync(0xffffffffu, nxt[k].du, 1);
             prd[k] = __shfl_xor_sync(0xffffffffu, nxt[k].r, 1);
+            if constexpr (kZU) pu[k] = __shfl_xor_sync(0xffffffffu, nxt[k].u, 1);
         }
 
         if (j == GPC - 1 || !has_next) {
@@ -429,7 +518,7 @@ __device__ __forceinline__ void scan_seq_body(const SeqMaps& maps, const ScanPar
             __syncwarp();
             if (has_next) {
                 const uint8_t* st = smem + ((c + 1) % S) * Ly::kStageBytes;
-                convert_bc<T, N>(st + 3 * Ly::kTile, st + 3 * Ly::kTile + Ly::kBCTile, bcf, lane);
+                convert_bc<T, N, kZG>(st + 3 * Ly::kTile, st + 3 * Ly::kTile + Ly::kBCTile, bcf, lane);
             }
             __syncwarp();
             if (lane == 0 && c + S < n_chunks) {
@@ -456,10 +545,11 @@ __device__ __forceinline__ void scan_seq_body(const SeqMaps& maps, const ScanPar
                     a = make_float2(ex2_approx(cc.a2[i].x * tot), ex2_approx(cc.a2[i].y * tot));
                 else
                     a = make_float2(expf(cc.a2[i].x * tot), expf(cc.a2[i].y * tot));
+                const float2 hs = state_out(i);
                 ga[4 * i] = a.x;
                 ga[4 * i + 2] = a.y;
-                gb[4 * i] = h[i].x;
-                gb[4 * i + 2] = h[i].y;
+                gb[4 * i] = hs.x;
+                gb[4 * i + 2] = hs.y;
             }
         }
         return;
@@ -475,8 +565,9 @@ __device__ __forceinline__ void scan_seq_body(const SeqMaps& maps, const ScanPar
         float* ls = p.last_state + row * N + half;
 #pragma unroll
         for (int i = 0; i < P; ++i) {
-            ls[4 * i] = h[i].x;
-            ls[4 * i + 2] = h[i].y;
+            const float2 hs = state_out(i);
+            ls[4 * i] = hs.x;
+            ls[4 * i + 2] = hs.y;
         }
     }
 }
@@ -486,7 +577,7 @@ __device__ __forceinline__ void scan_seq_body(const SeqMaps& maps, const ScanPar
 // 0 .. n_seg-2, the full pass all n_seg (after the fold has completed).
 // Requirements checked by the host: N in {4, 8, 16}; L * sizeof(T) a multiple
 // of 16; u, delta, z, B, C, y 16-byte aligned; seg_len a multiple of the chunk.
-template <typename T, int N, bool kGate, bool kSoftplus, bool kFold>
+template <typename T, int N, bool kGate, bool kSoftplus, bool kFold, bool kZoh>
 __global__ void __launch_bounds__(32) scan_fwd_seq_kernel(const __grid_constant__ SeqMaps maps, ScanParams p,
                                                           int allow_geo) {
     using Ly = SeqLayout<T, N>;
@@ -523,23 +614,25 @@ __global__ void __launch_bounds__(32) scan_fwd_seq_kernel(const __grid_constant_
     const float* Arow = p.A + d * N;
     const float a_first = Arow[0];
     cc.a0 = a_first * kLog2e;
+    if constexpr (kZoh) cc.ia0 = 1.f / a_first;  // inf at A = 0, where only the Taylor branch is taken
     bool geo = kFast && allow_geo;
 #pragma unroll
     for (int i = 0; i < P; ++i) {
         const int n = half + 4 * i;
         const float x0 = Arow[n], x1 = Arow[n + 2];
         cc.a2[i] = kFast ? make_float2(x0 * kLog2e, x1 * kLog2e) : make_float2(x0, x1);
+        if constexpr (kZoh) cc.ia[i] = make_float2(1.f / x0, 1.f / x1);
         geo = geo && x0 == float(n + 1) * a_first && x1 == float(n + 3) * a_first;
     }
     geo = __all_sync(0xffffffffu, geo || !valid);
 
     if constexpr (kFast) {
         if (geo) {
-            scan_seq_body<T, N, true, kGate, kSoftplus, kFold>(maps, p, smem, bars, cc, valid, row);
+            scan_seq_body<T, N, true, kGate, kSoftplus, kFold, kZoh>(maps, p, smem, bars, cc, valid, row);
             return;
         }
     }
-    scan_seq_body<T, N, false, kGate, kSoftplus, kFold>(maps, p, smem, bars, cc, valid, row);
+    scan_seq_body<T, N, false, kGate, kSoftplus, kFold, kZoh>(maps, p, smem, bars, cc, valid, row);
 }
 
 }  // namespace mss

@@ -46,8 +46,11 @@ __global__ void __launch_bounds__(128) scan_fwd_simple_kernel(ScanParams p) {
         float acc = 0.f;
 #pragma unroll
         for (int n = 0; n < N; ++n) {
-            const float dA = expf(dt * a[n]);
-            h[n] = fmaf(dA, h[n], du * ld(Bb + n * L + t));
+            const float x = dt * a[n];
+            const float dA = expf(x);
+            // input weight: Euler Delta, or the zero-order hold (e^x - 1)/a
+            const float w = !p.zoh ? du : (a[n] != 0.f ? expm1f(x) / a[n] : dt) * ut;
+            h[n] = fmaf(dA, h[n], w * ld(Bb + n * L + t));
             acc = fmaf(ld(Cb + n * L + t), h[n], acc);
         }
         float out = fmaf(Dd, ut, acc);

@@ -62,7 +62,9 @@ __global__ void __launch_bounds__(256) state_update_kernel(StepParams p) {
 #pragma unroll
     for (int i = 0; i < SPT; ++i) {
         const float dA = kFast ? ex2_approx(dt * (a[i] * kLog2e)) : expf(dt * a[i]);
-        h[i] = fmaf(dA, h[i], du * Bv[i]);
+        // input weight: Euler Delta, or the zero-order hold (e^{Delta a} - 1)/a
+        const float w = p.zoh ? zoh_weight(dt, a[i], dt * a[i], dA) * ut : du;
+        h[i] = fmaf(dA, h[i], w * Bv[i]);
         acc = fmaf(Cv[i], h[i], acc);
     }
 #pragma unroll

@@ -113,6 +113,21 @@ def test_decode_argument_errors(lib):
     assert step(y=P + 8) == codes["MSS_ERR_ALIAS"]  # y on the state
     assert step(batch=0) == 0
 
+    def step_ex(flags, **kw):
+        a = dict(state=P, u=P + 0x1000000, delta=P + 0x2000000, A=P + 0x3000000,
+                 B=P + 0x4000000, C=P + 0x5000000, y=P + 0x6000000, batch=4, dim=8, N=16, dtype=1)
+        a.update(kw)
+        w = lambda x: v(x) if x is not None else None
+        return lib.mss_state_update_ex(w(a["state"]), w(a["u"]), w(a["delta"]), w(a["A"]), w(a["B"]),
+                                       w(a["C"]), None, None, None, 1, w(a["y"]), a["batch"],
+                                       a["dim"], a["N"], a["dtype"], ctypes.c_uint(flags), None)
+
+    flag_zoh = int(re.search(r"#define MSS_FLAG_ZOH_INPUT (0x[0-9a-f]+)u", _header()).group(1), 16)
+    assert step_ex(0x1) == codes["MSS_ERR_FLAGS"]        # only the input-rule flag applies to decode
+    assert step_ex(flag_zoh, N=5) == codes["MSS_ERR_UNSUPPORTED_N"]
+    assert step_ex(flag_zoh, state=None) == codes["MSS_ERR_NULL"]
+    assert step_ex(flag_zoh, batch=0) == 0
+
 
 def test_binding_refuses_cpu_tensors():
     import torch
@@ -144,6 +159,7 @@ def test_ex2_and_workspace_argument_errors(lib):
     assert ex2(ws=P + 0x5000000, wsb=256) == codes["MSS_ERR_ALIAS"]              # workspace on y
     assert ex2(ws=P + 0x2000000, wsb=256) == codes["MSS_ERR_ALIAS"]              # workspace on A
     assert ex2(batch=0) == 0
+    assert ex2(flags=0x8, batch=0) == 0      # zero-order-hold input rule: a known flag
 
 
 def test_workspace_size_queries(lib):
@@ -154,6 +170,7 @@ def test_workspace_size_queries(lib):
     assert q(1, 16, 3, 4096, 1, 0) == codes["MSS_ERR_UNSUPPORTED_N"]
     assert q(-1, 16, 16, 4096, 1, 0) == codes["MSS_ERR_SHAPE"]
     assert q(1, 16, 16, 4096, 1, 0x80) == codes["MSS_ERR_FLAGS"]
+    assert q(1, 16, 16, 4096, 1, 0x8) >= 0
     # no split: scalar kernel, split disabled, nothing to do, rows not 16-byte multiples
     assert q(1, 16, 16, 4096, 1, 0x2) == 0
     assert q(1, 16, 16, 4096, 1, 0x4) == 0
