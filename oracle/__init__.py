@@ -63,6 +63,14 @@ def _load():
             lib.mss_oracle_state_update.argtypes = [d, f, f, f, f, f, f, f, f, i, i, d,
                                                     i64, i64, i64, i]
             lib.mss_oracle_state_update.restype = i
+            lib.mss_oracle_scan_fwd_conv.argtypes = [f, f, f, i, d, d, f, f, f, f, f, f, f, i, i, d, d, d,
+                                                     i64, i64, i64, i64, i]
+            lib.mss_oracle_scan_fwd_conv.restype = i
+            lib.mss_oracle_causal_conv.argtypes = [f, f, f, i, d, d, d, i64, i64, i64]
+            lib.mss_oracle_causal_conv.restype = i
+            lib.mss_oracle_state_update_conv.argtypes = [d, d, f, f, f, i, f, f, f, f, f, f, f, i, i, d,
+                                                         i64, i64, i64, i]
+            lib.mss_oracle_state_update_conv.restype = i
             lib.mss_oracle_recurrence.argtypes = [d, d, d, i64, i64, d, d]
             lib.mss_oracle_recurrence.restype = i
             lib.mss_oracle_softplus.argtypes = [ctypes.c_double]
@@ -140,6 +148,112 @@ def scan_fwd(u, delta, A, B, C, D=None, z=None, delta_bias=None, softplus_flag=T
         raise RuntimeError(f"mss_oracle_scan_fwd failed with code {rc}")
     del u_a, d_a, B_a, C_a, D_a, z_a, b_a, A_a  # keep buffers alive until here
     return y, last
+
+
+def _f64_opt(x, shape, name):
+    if x is None:
+        return None
+    a = np.ascontiguousarray(np.asarray(x, dtype=np.float64))
+    if a.shape != tuple(shape):
+        raise ValueError(f"{name}: expected shape {tuple(shape)}, got {a.shape}")
+    return a
+
+
+def causal_conv(x, conv_w, conv_b=None, conv_state=None):
+    """Causal depthwise convolution, pre-activation, in fp64.
+
+    x: [batch, dim, L]; conv_w: [dim, K] (tap k multiplies x_{t-(K-1)+k});
+    conv_b: [dim]; conv_state: [batch, dim, K-1] values before the first
+    token (None: zeros).  Returns (xc [batch, dim, L], conv_state_out
+    [batch, dim, K-1])."""
+    x_a, x_p = _f32(x, name="x")
+    batch, dim, L = x_a.shape
+    w_a, w_p = _f32(conv_w, name="conv_w")
+    K = w_a.shape[1]
+    cb_a, cb_p = _f32(conv_b, (dim,), "conv_b")
+    cs = _f64_opt(conv_state, (batch, dim, K - 1), "conv_state")
+    xc = np.empty((batch, dim, L), dtype=np.float64)
+    cs_out = np.empty((batch, dim, K - 1), dtype=np.float64)
+    rc = _load().mss_oracle_causal_conv(x_p, w_p, cb_p, K, None if cs is None else _dptr(cs), _dptr(xc),
+                                        _dptr(cs_out), batch, dim, L)
+    if rc != 0:
+        raise RuntimeError(f"mss_oracle_causal_conv failed with code {rc}")
+    del x_a, w_a, cb_a
+    return xc, cs_out
+
+
+def scan_fwd_conv(x, conv_w, delta, A, B, C, conv_b=None, conv_state=None, D=None, z=None,
+                  delta_bias=None, softplus_flag=True, initial_state=None, zoh_input=False,
+                  nthreads=None):
+    """Forward pass with the causal convolution and SiLU in front, in fp64:
+    u = silu(causal_conv(x)).  Arguments as scan_fwd and causal_conv.
+    Returns (y, last_state, conv_state_out)."""
+    x_a, x_p = _f32(x, name="x")
+    if x_a.ndim != 3:
+        raise ValueError("x must be [batch, dim, L]")
+    batch, dim, L = x_a.shape
+    w_a, w_p = _f32(conv_w, name="conv_w")
+    if w_a.ndim != 2 or w_a.shape[0] != dim:
+        raise ValueError("conv_w must be [dim, K]")
+    K = w_a.shape[1]
+    A_a, A_p = _f32(A, name="A")
+    N = A_a.shape[1]
+    cb_a, cb_p = _f32(conv_b, (dim,), "conv_b")
+    cs = _f64_opt(conv_state, (batch, dim, K - 1), "conv_state")
+    d_a, d_p = _f32(delta, (batch, dim, L), "delta")
+    B_a, B_p = _f32(B, (batch, N, L), "B")
+    C_a, C_p = _f32(C, (batch, N, L), "C")
+    D_a, D_p = _f32(D, (dim,), "D")
+    z_a, z_p = _f32(z, (batch, dim, L), "z")
+    b_a, b_p = _f32(delta_bias, (dim,), "delta_bias")
+    h0 = _f64_opt(initial_state, (batch, dim, N), "initial_state")
+    y = np.empty((batch, dim, L), dtype=np.float64)
+    last = np.empty((batch, dim, N), dtype=np.float64)
+    cs_out = np.empty((batch, dim, K - 1), dtype=np.float64)
+    rc = _load().mss_oracle_scan_fwd_conv(
+        x_p, w_p, cb_p, K, None if cs is None else _dptr(cs), _dptr(cs_out),
+        d_p, A_p, B_p, C_p, D_p, z_p, b_p, int(bool(softplus_flag)), int(bool(zoh_input)),
+        None if h0 is None else _dptr(h0), _dptr(y), _dptr(last), batch, dim, N, L,
+        default_threads() if nthreads is None else int(nthreads))
+    if rc != 0:
+        raise RuntimeError(f"mss_oracle_scan_fwd_conv failed with code {rc}")
+    del x_a, w_a, cb_a, d_a, B_a, C_a, D_a, z_a, b_a, A_a
+    return y, last, cs_out
+
+
+def state_update_conv(state, conv_state, x, conv_w, delta, A, B, C, conv_b=None, D=None, z=None,
+                      delta_bias=None, softplus_flag=True, zoh_input=False, nthreads=None):
+    """One decode step with the causal convolution in front, in fp64.
+
+    state: [batch, dim, N] and conv_state: [batch, dim, K-1], both fp64 and
+    updated in place; x: [batch, dim]; other arguments as state_update.
+    Returns (y, state, conv_state)."""
+    for name, a in (("state", state), ("conv_state", conv_state)):
+        if not (isinstance(a, np.ndarray) and a.dtype == np.float64 and a.flags.c_contiguous):
+            raise ValueError(f"{name} must be a C-contiguous float64 numpy array")
+    batch, dim, N = state.shape
+    w_a, w_p = _f32(conv_w, name="conv_w")
+    K = w_a.shape[1]
+    if conv_state.shape != (batch, dim, K - 1):
+        raise ValueError("conv_state must be [batch, dim, K-1]")
+    x_a, x_p = _f32(x, (batch, dim), "x")
+    cb_a, cb_p = _f32(conv_b, (dim,), "conv_b")
+    d_a, d_p = _f32(delta, (batch, dim), "delta")
+    A_a, A_p = _f32(A, (dim, N), "A")
+    B_a, B_p = _f32(B, (batch, N), "B")
+    C_a, C_p = _f32(C, (batch, N), "C")
+    D_a, D_p = _f32(D, (dim,), "D")
+    z_a, z_p = _f32(z, (batch, dim), "z")
+    b_a, b_p = _f32(delta_bias, (dim,), "delta_bias")
+    y = np.empty((batch, dim), dtype=np.float64)
+    rc = _load().mss_oracle_state_update_conv(
+        _dptr(state), _dptr(conv_state), x_p, w_p, cb_p, K, d_p, A_p, B_p, C_p, D_p, z_p, b_p,
+        int(bool(softplus_flag)), int(bool(zoh_input)), _dptr(y), batch, dim, N,
+        default_threads() if nthreads is None else int(nthreads))
+    if rc != 0:
+        raise RuntimeError(f"mss_oracle_state_update_conv failed with code {rc}")
+    del x_a, w_a, cb_a, d_a, A_a, B_a, C_a, D_a, z_a, b_a
+    return y, state, conv_state
 
 
 def state_update(state, u, delta, A, B, C, D=None, z=None, delta_bias=None,

@@ -39,6 +39,15 @@
  *     ("Mamba" paper review, section "SSM", block description) but print no
  *     formula for it: this part has no printed value to pin against
  *     (parity unpinned beyond its closed-form definition).
+ *   - Optional causal convolution in front of the scan: the input branch is
+ *     "expanded via a linear layer, followed by a convolution and
+ *     non-linearity" before the bank of SISO systems ("Mamba" paper review,
+ *     section "SSM", block description), and the fused kernel of "NN Lab:
+ *     Mamba" includes the causal 1D convolution.  Read as a depthwise
+ *     (per-channel) causal convolution of width K followed by SiLU:
+ *       u_t = silu(cb + sum_{k=0}^{K-1} w[k] x_{t-(K-1)+k}),
+ *     with the K-1 values before the first token taken from a conv state
+ *     (zero by default), and the conv state after the last token returned.
  *   - Final state: the state after the last token.  Decode: one step of the
  *     same recurrence starting from a caller-supplied state, which the
  *     "Exercises" page describes as the generation-time view (constant-size
@@ -124,10 +133,38 @@ typedef struct {
     int softplus_flag, zoh_input;
     double *y, *last_state;
     int64_t batch, dim, N, L;
+    /* causal convolution in front of the scan (conv_width > 0: u holds x) */
+    const float *conv_w, *conv_b;
+    const double *conv_state_in;
+    double *conv_state_out;
+    int conv_width;
     /* rows [row_begin, row_end) of the flattened (batch, dim) index */
     int64_t row_begin, row_end;
     int status;
 } scan_job;
+
+/* Causal depthwise convolution of one channel.  ext holds the K-1 values
+ * before the first token followed by the L inputs; out[t] is the
+ * pre-activation cb + sum_k w[k] * ext[t + k] (ext[t + k] = x_{t-(K-1)+k}). */
+static void causal_conv_row(const double *ext, int64_t L, const float *w, int K, double cb,
+                            double *out)
+{
+    for (int64_t t = 0; t < L; ++t) {
+        double acc = cb;
+        for (int k = 0; k < K; ++k)
+            acc += (double)w[k] * ext[t + k];
+        out[t] = acc;
+    }
+}
+
+/* The extended input of one channel: history (conv state, or zeros) then x. */
+static void conv_extend(const double *state_in, const float *x, int64_t L, int K, double *ext)
+{
+    for (int k = 0; k < K - 1; ++k)
+        ext[k] = state_in ? state_in[k] : 0.0;
+    for (int64_t t = 0; t < L; ++t)
+        ext[K - 1 + t] = (double)x[t];
+}
 
 /* Discretise one token of one channel: Delta from the raw value, then
  * Abar[n] = exp(Delta*A[n]) and Bbar x[n] = Delta * B[n] * u (Euler input
@@ -153,15 +190,28 @@ static void *scan_rows(void *arg)
 {
     scan_job *j = (scan_job *)arg;
     const int64_t N = j->N, L = j->L;
-    double *work = (double *)malloc((size_t)(4 * N) * sizeof(double));
+    const int K = j->conv_width;
+    /* conv: the extended input (K-1+L) and the activations u (L) of a row */
+    const int64_t conv_len = K > 0 ? (K - 1 + 2 * L) : 0;
+    double *work = (double *)malloc((size_t)(4 * N + conv_len) * sizeof(double));
     if (!work) {
         j->status = ORACLE_ENOMEM;
         return NULL;
     }
     double *h = work, *abar = work + N, *bx = work + 2 * N, *c = work + 3 * N;
+    double *ext = work + 4 * N, *uc = ext + (K > 0 ? K - 1 + L : 0);
     for (int64_t row = j->row_begin; row < j->row_end; ++row) {
         const int64_t b = row / j->dim, d = row % j->dim;
         const float *u = j->u + row * L;
+        if (K > 0) {
+            conv_extend(j->conv_state_in ? j->conv_state_in + row * (K - 1) : NULL, u, L, K, ext);
+            causal_conv_row(ext, L, j->conv_w + d * K, K, j->conv_b ? (double)j->conv_b[d] : 0.0, uc);
+            for (int64_t t = 0; t < L; ++t)
+                uc[t] = mss_oracle_silu(uc[t]);
+            if (j->conv_state_out)
+                for (int k = 0; k < K - 1; ++k)
+                    j->conv_state_out[row * (K - 1) + k] = ext[L + k];
+        }
         const float *dr = j->delta + row * L;
         const float *z = j->z ? j->z + row * L : NULL;
         const float *A_row = j->A + d * N;
@@ -173,7 +223,7 @@ static void *scan_rows(void *arg)
         for (int64_t n = 0; n < N; ++n)
             h[n] = j->initial_state ? j->initial_state[row * N + n] : 0.0;
         for (int64_t t = 0; t < L; ++t) {
-            const double ut = (double)u[t];
+            const double ut = K > 0 ? uc[t] : (double)u[t];
             discretise((double)dr[t], bias, j->softplus_flag, j->zoh_input, A_row, B_b + t, C_b + t,
                        L, N, ut, abar, bx, c);
             double out = recurrence_step(h, abar, bx, c, N) + Dd * ut;
@@ -252,10 +302,70 @@ int mss_oracle_scan_fwd(const float *u, const float *delta, const float *A,
     if (batch < 0 || dim < 0 || dstate <= 0 || seqlen < 0)
         return ORACLE_EINVAL;
     scan_job proto = {u, delta, A, B, C, D, z, delta_bias, initial_state, softplus_flag,
-                      zoh_input, y, last_state, batch, dim, dstate, seqlen, 0, 0, ORACLE_OK};
+                      zoh_input, y, last_state, batch, dim, dstate, seqlen,
+                      NULL, NULL, NULL, NULL, 0, 0, 0, ORACLE_OK};
     if (batch * dim == 0)
         return ORACLE_OK;
     return run_threaded(&proto, batch * dim, nthreads, scan_rows);
+}
+
+/*
+ * Forward pass with the causal convolution in front: x takes the place of
+ * u, and u = silu(conv(x)) feeds both the input term and the skip term.
+ *   x            : [batch][dim][L]
+ *   conv_w       : [dim][K], tap k multiplies x_{t-(K-1)+k}
+ *   conv_b       : [dim] (may be NULL)
+ *   conv_state_in: [batch][dim][K-1] fp64, x before the first token, oldest
+ *                  first (NULL: zeros)
+ *   conv_state_out: [batch][dim][K-1] fp64, the last K-1 values of the
+ *                  history followed by x (may be NULL)
+ * The other arguments are those of mss_oracle_scan_fwd.  K >= 1.
+ */
+int mss_oracle_scan_fwd_conv(const float *x, const float *conv_w, const float *conv_b,
+                             int conv_width, const double *conv_state_in, double *conv_state_out,
+                             const float *delta, const float *A, const float *B, const float *C,
+                             const float *D, const float *z, const float *delta_bias,
+                             int softplus_flag, int zoh_input, const double *initial_state,
+                             double *y, double *last_state, int64_t batch, int64_t dim,
+                             int64_t dstate, int64_t seqlen, int nthreads)
+{
+    if (!x || !conv_w || conv_width < 1 || !delta || !A || !B || !C || !y)
+        return ORACLE_EINVAL;
+    if (batch < 0 || dim < 0 || dstate <= 0 || seqlen < 0)
+        return ORACLE_EINVAL;
+    scan_job proto = {x, delta, A, B, C, D, z, delta_bias, initial_state, softplus_flag,
+                      zoh_input, y, last_state, batch, dim, dstate, seqlen,
+                      conv_w, conv_b, conv_state_in, conv_state_out, conv_width, 0, 0, ORACLE_OK};
+    if (batch * dim == 0)
+        return ORACLE_OK;
+    return run_threaded(&proto, batch * dim, nthreads, scan_rows);
+}
+
+/*
+ * The causal convolution alone (pre-activation, no SiLU), with the layouts of
+ * mss_oracle_scan_fwd_conv; xc: [batch][dim][L] fp64.
+ */
+int mss_oracle_causal_conv(const float *x, const float *conv_w, const float *conv_b,
+                           int conv_width, const double *conv_state_in, double *xc,
+                           double *conv_state_out, int64_t batch, int64_t dim, int64_t seqlen)
+{
+    if (!x || !conv_w || conv_width < 1 || !xc || batch < 0 || dim < 0 || seqlen < 0)
+        return ORACLE_EINVAL;
+    const int K = conv_width;
+    const int64_t L = seqlen;
+    double *ext = (double *)malloc((size_t)(K - 1 + L + 1) * sizeof(double));
+    if (!ext)
+        return ORACLE_ENOMEM;
+    for (int64_t row = 0; row < batch * dim; ++row) {
+        const int64_t d = row % dim;
+        conv_extend(conv_state_in ? conv_state_in + row * (K - 1) : NULL, x + row * L, L, K, ext);
+        causal_conv_row(ext, L, conv_w + d * K, K, conv_b ? (double)conv_b[d] : 0.0, xc + row * L);
+        if (conv_state_out)
+            for (int k = 0; k < K - 1; ++k)
+                conv_state_out[row * (K - 1) + k] = ext[L + k];
+    }
+    free(ext);
+    return ORACLE_OK;
 }
 
 /* ------------------------------------------------------------------------ */
@@ -267,6 +377,11 @@ typedef struct {
     int softplus_flag, zoh_input;
     double *y;
     int64_t dim, N;
+    /* causal convolution in front (conv_width > 0: u holds x, conv_state is
+     * read and shifted in place) */
+    const float *conv_w, *conv_b;
+    double *conv_state;
+    int conv_width;
     int64_t row_begin, row_end;
     int status;
 } step_job;
@@ -283,7 +398,21 @@ static void *step_rows(void *arg)
     double *abar = work, *bx = work + N, *c = work + 2 * N;
     for (int64_t row = j->row_begin; row < j->row_end; ++row) {
         const int64_t b = row / j->dim, d = row % j->dim;
-        const double ut = (double)j->u[row];
+        double ut = (double)j->u[row];
+        if (j->conv_width > 0) {
+            /* the window: the K-1 stored values then this token's x */
+            const int K = j->conv_width;
+            double *cs = j->conv_state + row * (K - 1);
+            double acc = j->conv_b ? (double)j->conv_b[d] : 0.0;
+            for (int k = 0; k < K - 1; ++k)
+                acc += (double)j->conv_w[d * K + k] * cs[k];
+            acc += (double)j->conv_w[d * K + K - 1] * ut;
+            for (int k = 0; k + 1 < K - 1; ++k)
+                cs[k] = cs[k + 1];
+            if (K > 1)
+                cs[K - 2] = ut;
+            ut = mss_oracle_silu(acc);
+        }
         const double bias = j->bias ? (double)j->bias[d] : 0.0;
         /* B, C of a decode step are [batch][N]: stride 1 between states. */
         discretise((double)j->delta[row], bias, j->softplus_flag, j->zoh_input, j->A + d * N,
@@ -355,7 +484,32 @@ int mss_oracle_state_update(double *state, const float *u, const float *delta,
     if (batch < 0 || dim < 0 || dstate <= 0)
         return ORACLE_EINVAL;
     step_job proto = {state, u, delta, A, B, C, D, z, delta_bias, softplus_flag, zoh_input, y,
-                      dim, dstate, 0, 0, ORACLE_OK};
+                      dim, dstate, NULL, NULL, NULL, 0, 0, 0, ORACLE_OK};
+    if (batch * dim == 0)
+        return ORACLE_OK;
+    return run_steps(&proto, batch * dim, nthreads);
+}
+
+/*
+ * One decode step with the causal convolution in front: x takes the place of
+ * u; conv_state [batch][dim][K-1] fp64 (oldest first) is read, shifted by one
+ * and ends with this token's x.  Other arguments as mss_oracle_state_update.
+ */
+int mss_oracle_state_update_conv(double *state, double *conv_state, const float *x,
+                                 const float *conv_w, const float *conv_b, int conv_width,
+                                 const float *delta, const float *A, const float *B,
+                                 const float *C, const float *D, const float *z,
+                                 const float *delta_bias, int softplus_flag, int zoh_input,
+                                 double *y, int64_t batch, int64_t dim, int64_t dstate,
+                                 int nthreads)
+{
+    if (!state || !x || !conv_w || conv_width < 1 || (conv_width > 1 && !conv_state) ||
+        !delta || !A || !B || !C || !y)
+        return ORACLE_EINVAL;
+    if (batch < 0 || dim < 0 || dstate <= 0)
+        return ORACLE_EINVAL;
+    step_job proto = {state, x, delta, A, B, C, D, z, delta_bias, softplus_flag, zoh_input, y,
+                      dim, dstate, conv_w, conv_b, conv_state, conv_width, 0, 0, ORACLE_OK};
     if (batch * dim == 0)
         return ORACLE_OK;
     return run_steps(&proto, batch * dim, nthreads);

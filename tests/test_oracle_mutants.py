@@ -38,6 +38,12 @@ MUTANTS = {
     "initial_state_ignored": ("h[n] = j->initial_state ? j->initial_state[row * N + n] : 0.0;", "h[n] = 0.0;"),
     "decode_B_token_stride": ("j->B + b * N, j->C + b * N, 1, N,", "j->B + b * N, j->C + b * N, N, N,"),
     "B_batch_index": ("const float *B_b = j->B + b * N * L;", "const float *B_b = j->B;"),
+    "conv_taps_reversed": ("acc += (double)w[k] * ext[t + k];", "acc += (double)w[K - 1 - k] * ext[t + k];"),
+    "conv_bias_dropped": ("        double acc = cb;\n", "        double acc = 0.0;\n"),
+    "conv_without_silu": ("uc[t] = mss_oracle_silu(uc[t]);", "uc[t] = uc[t];"),
+    "conv_state_out_offset": ("j->conv_state_out[row * (K - 1) + k] = ext[L + k];",
+                              "j->conv_state_out[row * (K - 1) + k] = ext[L + k - 1];"),
+    "conv_decode_no_shift": ("                cs[k] = cs[k + 1];\n", "                cs[k] = cs[k];\n"),
 }
 
 

@@ -535,3 +535,96 @@ def test_zoh_decode_steps_equal_forward():
                                         zoh_input=True, **step)
         assert np.array_equal(yt, y[..., t])
     assert np.array_equal(state, last)
+
+
+# --------------------------------------------------------------------------
+# Causal convolution in front of the scan ("Mamba" paper review, section
+# "SSM", block description: a convolution and non-linearity before the SSM
+# bank; "NN Lab: Mamba": the fused kernel includes the causal 1D convolution)
+
+def _conv_inputs(seed, batch=2, dim=3, L=17, K=4):
+    rng = np.random.default_rng(seed)
+    return (rng.standard_normal((batch, dim, L)).astype(np.float32),
+            rng.standard_normal((dim, K)).astype(np.float32),
+            rng.standard_normal(dim).astype(np.float32))
+
+
+@pytest.mark.parametrize("K", [1, 2, 3, 4])
+def test_causal_conv_is_numpy_convolution(K):
+    """Tap k multiplies x_{t-(K-1)+k}: the causal convolution equals numpy's
+    full convolution with the reversed taps, truncated to the first L outputs."""
+    x, w, cb = _conv_inputs(70 + K, K=K)
+    xc, _ = oracle.causal_conv(x, w, cb)
+    for b in range(x.shape[0]):
+        for d in range(x.shape[1]):
+            ref = cb[d] + np.convolve(x[b, d].astype(np.float64), w[d, ::-1].astype(np.float64))[:x.shape[2]]
+            np.testing.assert_allclose(xc[b, d], ref, rtol=1e-14, atol=1e-14)
+
+
+def test_causal_conv_impulse_response():
+    """A unit impulse at t = 0 returns the taps in reverse order, then the bias."""
+    K, L = 4, 9
+    w = np.array([[0.5, -1.0, 2.0, 0.25]], dtype=np.float32)
+    x = np.zeros((1, 1, L), dtype=np.float32)
+    x[0, 0, 0] = 1.0
+    xc, _ = oracle.causal_conv(x, w, np.array([0.125], dtype=np.float32))
+    want = [0.125 + 0.25, 0.125 + 2.0, 0.125 - 1.0, 0.125 + 0.5] + [0.125] * (L - K)
+    assert xc[0, 0].tolist() == want
+
+
+def test_causal_conv_state_chains():
+    """The state after a prefix (its last K-1 inputs) continues the prefix
+    exactly; with fewer than K-1 new inputs the old state shifts through."""
+    x, w, cb = _conv_inputs(75, L=20)
+    full, st_full = oracle.causal_conv(x, w, cb)
+    for L0 in (1, 2, 5, 19):
+        a, st = oracle.causal_conv(x[..., :L0], w, cb)
+        b, st2 = oracle.causal_conv(x[..., L0:], w, cb, conv_state=st)
+        assert np.array_equal(np.concatenate([a, b], axis=2), full)
+        assert np.array_equal(st2, st_full)
+    assert np.array_equal(st_full, x[..., -3:].astype(np.float64))
+    h0 = np.random.default_rng(76).standard_normal((2, 3, 3))
+    _, st = oracle.causal_conv(x[..., :1], w, cb, conv_state=h0)
+    assert np.array_equal(st, np.concatenate([h0[..., 1:], x[..., :1].astype(np.float64)], axis=2))
+
+
+def test_scan_fwd_conv_feeds_silu_of_conv_to_the_scan():
+    """With the convolution in front, u = silu(conv(x)) drives both the input
+    term and the skip term: the result equals the plain forward pass fed with
+    that u (rounded to fp32, hence the 1e-6 bound)."""
+    x, w, cb = _conv_inputs(77, batch=2, dim=5, L=40)
+    inp = _random_forward_inputs(78, batch=2, dim=5, N=4, L=40)
+    inp.pop("u")
+    y, last, st = oracle.scan_fwd_conv(x, w, conv_b=cb, **inp)
+    xc, st_ref = oracle.causal_conv(x, w, cb)
+    u = (xc / (1.0 + np.exp(-xc))).astype(np.float32)
+    y_ref, last_ref = oracle.scan_fwd(u=u, **inp)
+    np.testing.assert_allclose(y, y_ref, rtol=1e-6, atol=1e-6)
+    np.testing.assert_allclose(last, last_ref, rtol=1e-6, atol=1e-6)
+    assert np.array_equal(st, st_ref)
+    # K = 1 with a unit tap and no bias is silu(x) itself
+    y1, _, _ = oracle.scan_fwd_conv(x, np.ones((5, 1), dtype=np.float32), **inp)
+    u1 = (x / (1.0 + np.exp(-x.astype(np.float64)))).astype(np.float32)
+    np.testing.assert_allclose(y1, oracle.scan_fwd(u=u1, **inp)[0], rtol=1e-6, atol=1e-6)
+
+
+@pytest.mark.parametrize("zoh", [False, True])
+def test_conv_decode_steps_equal_conv_forward(zoh):
+    """Decode with the convolution (its state shifted one token per step)
+    reproduces the forward pass with the convolution, bitwise."""
+    x, w, cb = _conv_inputs(79, batch=2, dim=5, L=30)
+    inp = _random_forward_inputs(80, batch=2, dim=5, N=4, L=30)
+    inp.pop("u")
+    h0 = np.random.default_rng(81).standard_normal((2, 5, 4))
+    c0 = np.random.default_rng(82).standard_normal((2, 5, 3))
+    y, last, st = oracle.scan_fwd_conv(x, w, conv_b=cb, conv_state=c0, initial_state=h0,
+                                       zoh_input=zoh, **inp)
+    state, cstate = h0.copy(), c0.copy()
+    for t in range(30):
+        step = {k: np.ascontiguousarray(inp[k][..., t]) for k in ("delta", "z", "B", "C")}
+        yt, state, cstate = oracle.state_update_conv(state, cstate, np.ascontiguousarray(x[..., t]), w,
+                                                     A=inp["A"], D=inp["D"], delta_bias=inp["delta_bias"],
+                                                     conv_b=cb, zoh_input=zoh, **step)
+        assert np.array_equal(yt, y[..., t])
+    assert np.array_equal(state, last)
+    assert np.array_equal(cstate, st)
