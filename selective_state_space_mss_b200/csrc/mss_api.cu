@@ -17,6 +17,7 @@
 #include "scan_seq.cuh"
 #include "scan_simple.cuh"
 #include "state_update.cuh"
+#include "state_update_tma.cuh"
 
 namespace {
 
@@ -160,6 +161,29 @@ int64_t seg_len_for(int64_t seqlen, int n_seg) {
     using Ly = mss::SeqLayout<T, N>;
     const int64_t n_chunks = (seqlen + Ly::kChunk - 1) / Ly::kChunk;
     return ((n_chunks + n_seg - 1) / n_seg) * Ly::kChunk;
+}
+
+// Resident CTAs of the bulk-staged decode kernel on the current device
+// (SMs x CTAs per SM), looked up once per device; 0 if the query fails.
+template <typename T, int N>
+int decode_tma_slots() {
+    constexpr int kMaxDev = 64;
+    static std::mutex mu;
+    static int slots[kMaxDev] = {};
+    int dev = -1;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDev) return 0;
+    std::lock_guard<std::mutex> lock(mu);
+    if (slots[dev] == 0) {
+        int sms = 0, occ = 0;
+        if (cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess ||
+            cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, mss::state_update_tma_kernel<T, N>,
+                                                          mss::DecodeTile<T, N>::kThreads,
+                                                          mss::DecodeTile<T, N>::kSmemBytes) != cudaSuccess ||
+            occ < 1)
+            return 0;
+        slots[dev] = sms * occ;
+    }
+    return slots[dev];
 }
 
 constexpr unsigned kScanFlags = MSS_FLAG_GENERAL_A | MSS_FLAG_SIMPLE | MSS_FLAG_NO_SPLIT | MSS_FLAG_ZOH_INPUT;
@@ -390,14 +414,38 @@ int mss_state_update_ex(float* state, const void* u, const void* delta, const fl
         return MSS_ERR_ALIAS;
 
     mss::StepParams p{state, u, delta, A, B, C, D, z, delta_bias, y, batch, dim, softplus_flag ? 1 : 0,
-                      (flags & MSS_FLAG_ZOH_INPUT) ? 1 : 0};
+                      (flags & MSS_FLAG_ZOH_INPUT) ? 1 : 0, 0};
     cudaStream_t s = static_cast<cudaStream_t>(stream);
     const bool vec = aligned(state, 16) && aligned(A, 16);
+    // bulk-staged kernel when every streamed tensor is 16-byte aligned and
+    // dim is a whole number of tiles; otherwise the per-thread kernel
+    const bool bulk_ok = vec && aligned(u, 16) && aligned(delta, 16) && aligned(y, 16) && (!z || aligned(z, 16));
     return with_n(dstate, [&](auto nc) {
         constexpr int N = decltype(nc)::value;
+        if constexpr (N == 4 || N == 8 || N == 16) {
+            if (bulk_ok) {
+                auto go_tma = [&](auto tag) -> int {
+                    using T = decltype(tag);
+                    using Ly = mss::DecodeTile<T, N>;
+                    if (dim % Ly::kRows != 0 || batch > 0x7fffffffLL) return 1;  // not handled here
+                    const int64_t n_cblocks = dim / Ly::kRows;
+                    const int slots = decode_tma_slots<T, N>();
+                    if (slots <= 0) return int(MSS_ERR_CUDA);
+                    // batch rows per channel block served by separate CTAs
+                    const int64_t bsplit = std::max<int64_t>(1, std::min<int64_t>(batch, slots / n_cblocks));
+                    const int64_t grid = n_cblocks * bsplit;
+                    if (grid > 0x7fffffffLL) return 1;
+                    mss::state_update_tma_kernel<T, N><<<dim3(unsigned(grid)), Ly::kThreads, Ly::kSmemBytes, s>>>(
+                        p, int(n_cblocks), int(bsplit));
+                    return launch_status();
+                };
+                const int rc = dtype == MSS_DTYPE_BF16 ? go_tma(bf16_t{}) : go_tma(float{});
+                if (rc <= 0) return rc;  // done (MSS_OK) or failed
+            }
+        }
         constexpr int TPC = N < 4 ? 1 : N / 4;
         const int threads = 256;
-        const int64_t blocks = (rows * TPC + threads - 1) / threads;
+        const int64_t blocks = ((rows - p.row0) * TPC + threads - 1) / threads;
         if (blocks > 0x7fffffffLL) return int(MSS_ERR_SHAPE);
         auto go = [&](auto kern) {
             kern<<<dim3(unsigned(blocks)), threads, 0, s>>>(p);

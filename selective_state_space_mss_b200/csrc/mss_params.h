@@ -41,7 +41,8 @@ struct StepParams {
     void* y;
     int64_t batch, dim;
     int softplus;
-    int zoh;  // as in ScanParams
+    int zoh;       // as in ScanParams
+    int64_t row0;  // first (batch * dim + channel) row this launch serves
 };
 
 }  // namespace mss

@@ -23,12 +23,12 @@ __global__ void __launch_bounds__(256) state_update_kernel(StepParams p) {
 
     const int64_t rows = p.batch * p.dim;
     const int64_t gid = int64_t(blockIdx.x) * blockDim.x + threadIdx.x;
-    const int64_t row = gid / TPC;
+    const int64_t row = p.row0 + gid / TPC;
     const int q = int(gid % TPC);
     const bool active = row < rows;
-    // lanes past the end compute on row 0 (rows > 0 here) so that every lane
+    // lanes past the end compute on row row0 (< rows here) so that every lane
     // of a channel group takes part in the shuffles; they store nothing
-    const int64_t r = active ? row : 0;
+    const int64_t r = active ? row : p.row0;
     const int64_t b = r / p.dim, d = r % p.dim;
 
     float h[SPT], a[SPT], Bv[SPT], Cv[SPT];

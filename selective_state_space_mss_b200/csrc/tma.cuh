@@ -1,6 +1,7 @@
-// tma.cuh -- thin wrappers over the sm_100a instructions the streaming kernel
-// uses to stage tiles: mbarrier init / expect-tx / bounded wait, and tiled
-// bulk tensor copies (cp.async.bulk.tensor) from global to shared memory.
+// tma.cuh -- thin wrappers over the sm_100a instructions the streaming kernels
+// use to stage tiles: mbarrier init / expect-tx / bounded wait, tiled bulk
+// tensor copies (cp.async.bulk.tensor) from global to shared memory, and
+// plain 1-D bulk copies (cp.async.bulk) in both directions.
 //
 // No copy here uses cluster multicast: every CTA fetches its own tiles from
 // this GPU's memory.
@@ -86,6 +87,36 @@ __device__ __forceinline__ void tma_load_3d(void* dst, const CUtensorMap* map, i
         "cp.async.bulk.tensor.3d.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3, %4}], [%5];"
         ::"r"(smem_addr(dst)), "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(z), "r"(smem_addr(bar))
         : "memory");
+}
+
+// 1-D bulk copy global -> shared without a tensor map: both addresses 16-byte
+// aligned, `bytes` a multiple of 16; completion signalled on `bar`.
+__device__ __forceinline__ void bulk_load(void* dst, const void* src, uint32_t bytes, uint64_t* bar) {
+    asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];"
+                 ::"r"(smem_addr(dst)), "l"(reinterpret_cast<uint64_t>(src)), "r"(bytes), "r"(smem_addr(bar))
+                 : "memory");
+}
+
+// 1-D bulk copy shared -> global, in the issuing thread's bulk async-group.
+__device__ __forceinline__ void bulk_store(void* dst, const void* src, uint32_t bytes) {
+    asm volatile("cp.async.bulk.global.shared::cta.bulk_group [%0], [%1], %2;"
+                 ::"l"(reinterpret_cast<uint64_t>(dst)), "r"(smem_addr(src)), "r"(bytes)
+                 : "memory");
+}
+
+__device__ __forceinline__ void bulk_commit() { asm volatile("cp.async.bulk.commit_group;" ::: "memory"); }
+
+// Wait until at most `kPending` of this thread's bulk groups still read
+// their shared-memory source (the source may then be overwritten).
+template <int kPending>
+__device__ __forceinline__ void bulk_wait_read() {
+    asm volatile("cp.async.bulk.wait_group.read %0;" ::"n"(kPending) : "memory");
+}
+
+// Wait until at most `kPending` of this thread's bulk groups are incomplete.
+template <int kPending>
+__device__ __forceinline__ void bulk_wait() {
+    asm volatile("cp.async.bulk.wait_group %0;" ::"n"(kPending) : "memory");
 }
 
 __device__ __forceinline__ void prefetch_tensormap(const CUtensorMap* map) {

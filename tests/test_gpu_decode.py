@@ -96,3 +96,34 @@ def test_decode_workload_sampled_every_step():
     st = to_numpy(state)
     assert_close(st[bi, di], ref_state[:, 0], w.dtype, "final state (sampled)")
     assert np.all(np.isfinite(st))
+
+
+@pytest.mark.parametrize("dtype", ["f32", "bf16"])
+@pytest.mark.parametrize("N", [4, 8, 16])
+@pytest.mark.parametrize("zoh", [False, True])
+@pytest.mark.parametrize("gate", [True, False])
+def test_decode_staged_path_matches_oracle(dtype, N, zoh, gate):
+    """Shapes whose channel count is a whole number of 4 KB state tiles
+    (1024/N channels) take the bulk-staged decode kernel; several batch rows
+    per channel block, several channel blocks, and more steps than stages."""
+    batch, dim, steps = 5, 2 * 1024 // N, 6
+    A, D, bias = gen.channel_params(dim, N, "normal", 90 + N)
+    h0 = gen.initial_state(batch, dim, N, 91, "normal")
+    state = torch.from_numpy(h0.copy()).to(DEV)
+    ref_state = h0.astype(np.float64)
+    Ad, Dd, bd = (torch.from_numpy(x).to(DEV) for x in (A, D, bias))
+    flags = mss.FLAG_ZOH_INPUT if zoh else 0
+    for t in range(steps):
+        s = gen.decode_step_inputs(batch, dim, N, dtype, 92, t)
+        dev = _step_dev(s)
+        if not gate:
+            dev["z"] = None
+        y = mss.state_update(state, A=Ad, D=Dd, delta_bias=bd, flags=flags, **dev)
+        y_ref, ref_state = oracle.state_update(ref_state, s["u"].values, s["delta"].values, A,
+                                               s["B"].values, s["C"].values, D=D,
+                                               z=s["z"].values if gate else None,
+                                               delta_bias=bias, zoh_input=zoh)
+        torch.cuda.synchronize()
+        assert_close(to_numpy(y), y_ref, dtype, f"step {t} y")
+    assert_close(to_numpy(state), ref_state, dtype, "final state")
+    assert mss.get_device_error() == 0
