@@ -71,6 +71,9 @@ def _load():
             lib.mss_oracle_state_update_conv.argtypes = [d, d, f, f, f, i, f, f, f, f, f, f, f, i, i, d,
                                                          i64, i64, i64, i]
             lib.mss_oracle_state_update_conv.restype = i
+            lib.mss_oracle_scan_bwd.argtypes = [f, f, f, f, f, f, f, f, i, i, d, f, d,
+                                                d, d, d, d, d, d, d, d, d, i64, i64, i64, i64, i]
+            lib.mss_oracle_scan_bwd.restype = i
             lib.mss_oracle_recurrence.argtypes = [d, d, d, i64, i64, d, d]
             lib.mss_oracle_recurrence.restype = i
             lib.mss_oracle_softplus.argtypes = [ctypes.c_double]
@@ -254,6 +257,46 @@ def state_update_conv(state, conv_state, x, conv_w, delta, A, B, C, conv_b=None,
         raise RuntimeError(f"mss_oracle_state_update_conv failed with code {rc}")
     del x_a, w_a, cb_a, d_a, A_a, B_a, C_a, D_a, z_a, b_a
     return y, state, conv_state
+
+
+def scan_bwd(u, delta, A, B, C, dy, D=None, z=None, delta_bias=None, softplus_flag=True,
+             initial_state=None, dlast=None, zoh_input=False, nthreads=None):
+    """Backward pass of scan_fwd in fp64 (reverse mode).
+
+    dy: [batch, dim, L] gradient with respect to y; dlast: [batch, dim, N]
+    gradient with respect to last_state (None: 0).  Returns a dict with du,
+    ddelta (with respect to delta_raw), dz (None without z), dA [dim, N],
+    dB, dC [batch, N, L], dD, dbias [dim] and dinit [batch, dim, N]
+    (with respect to initial_state)."""
+    u_a, u_p = _f32(u, name="u")
+    batch, dim, L = u_a.shape
+    A_a, A_p = _f32(A, name="A")
+    N = A_a.shape[1]
+    d_a, d_p = _f32(delta, (batch, dim, L), "delta")
+    B_a, B_p = _f32(B, (batch, N, L), "B")
+    C_a, C_p = _f32(C, (batch, N, L), "C")
+    D_a, D_p = _f32(D, (dim,), "D")
+    z_a, z_p = _f32(z, (batch, dim, L), "z")
+    b_a, b_p = _f32(delta_bias, (dim,), "delta_bias")
+    g_a, g_p = _f32(dy, (batch, dim, L), "dy")
+    h0 = _f64_opt(initial_state, (batch, dim, N), "initial_state")
+    dl = _f64_opt(dlast, (batch, dim, N), "dlast")
+    out = {k: np.zeros(shape, dtype=np.float64) for k, shape in
+           (("du", (batch, dim, L)), ("ddelta", (batch, dim, L)), ("dz", (batch, dim, L)), ("dA", (dim, N)),
+            ("dB", (batch, N, L)), ("dC", (batch, N, L)), ("dD", (dim,)), ("dbias", (dim,)),
+            ("dinit", (batch, dim, N)))}
+    rc = _load().mss_oracle_scan_bwd(
+        u_p, d_p, A_p, B_p, C_p, D_p, z_p, b_p, int(bool(softplus_flag)), int(bool(zoh_input)),
+        None if h0 is None else _dptr(h0), g_p, None if dl is None else _dptr(dl),
+        _dptr(out["du"]), _dptr(out["ddelta"]), _dptr(out["dz"]) if z is not None else None, _dptr(out["dA"]),
+        _dptr(out["dB"]), _dptr(out["dC"]), _dptr(out["dD"]), _dptr(out["dbias"]), _dptr(out["dinit"]),
+        batch, dim, N, L, default_threads() if nthreads is None else int(nthreads))
+    if rc != 0:
+        raise RuntimeError(f"mss_oracle_scan_bwd failed with code {rc}")
+    if z is None:
+        out["dz"] = None
+    del u_a, d_a, B_a, C_a, D_a, z_a, b_a, g_a, A_a
+    return out
 
 
 def state_update(state, u, delta, A, B, C, D=None, z=None, delta_bias=None,

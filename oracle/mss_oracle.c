@@ -514,3 +514,214 @@ int mss_oracle_state_update_conv(double *state, double *conv_state, const float 
         return ORACLE_OK;
     return run_steps(&proto, batch * dim, nthreads);
 }
+
+/* ------------------------------------------------------------------------ */
+/* Backward pass (reverse mode) of the forward pass above.                   */
+/*
+ * The pages train the model end to end ("Mamba" paper review, section
+ * "Selection Mechanism": the kernel recomputes intermediate states in the
+ * backward pass instead of storing them).  They print no gradient formula,
+ * so this is the chain rule applied by hand to the definition above, one
+ * step at a time, with the states of each row recomputed in fp64:
+ *
+ *   y_t = r_t * g_t,  g_t = silu(z_t) (1 without a gate),
+ *   r_t = sum_n C_tn h_tn + D u_t,   h_tn = a_tn h_{t-1,n} + w_tn B_tn u_t,
+ *   a_tn = exp(Delta_t A_n),  w_tn = Delta_t (Euler) or expm1(Delta_t A_n)/A_n,
+ *   Delta_t = softplus(s_t) (or s_t),  s_t = delta_raw_t + bias.
+ *
+ * Walking t from L-1 down to 0 with gh = dLoss/dh_t (starting from the
+ * gradient of last_state), each step adds dr_t C_t to gh, takes the
+ * gradients of a_tn and of the input term, and leaves gh * a_t as
+ * dLoss/dh_{t-1}.  B and C are shared by the channels of a batch row, A, D
+ * and the bias by the rows of a channel: their gradients are summed.
+ */
+
+typedef struct {
+    const float *u, *delta, *A, *B, *C, *D, *z, *bias, *dy;
+    const double *initial_state, *dlast;
+    int softplus_flag, zoh_input;
+    int64_t batch, dim, N, L;
+    /* per-row outputs */
+    double *du, *ddelta, *dz, *dinit;
+    /* summed outputs, private to this job: dA [dim][N], dD [dim], dbias [dim],
+     * dB, dC [batch][N][L] */
+    double *dA, *dD, *dbias, *dB, *dC;
+    int64_t row_begin, row_end;
+    int status;
+} bwd_job;
+
+static double sigmoid(double x) { return 1.0 / (1.0 + exp(-x)); }
+
+static void *bwd_rows(void *arg)
+{
+    bwd_job *j = (bwd_job *)arg;
+    const int64_t N = j->N, L = j->L;
+    /* per row: states h_t (L+1 rows, row 0 = the starting state), a_t, w_t,
+     * Delta_t, s_t, r_t, and the adjoint gh */
+    double *h = (double *)malloc((size_t)((L + 1) * N) * sizeof(double));
+    double *a = (double *)malloc((size_t)(L * N + 1) * sizeof(double));
+    double *w = (double *)malloc((size_t)(L * N + 1) * sizeof(double));
+    double *sc = (double *)malloc((size_t)(3 * L + 1) * sizeof(double));
+    double *gh = (double *)malloc((size_t)N * sizeof(double));
+    if (!h || !a || !w || !sc || !gh) {
+        free(h); free(a); free(w); free(sc); free(gh);
+        j->status = ORACLE_ENOMEM;
+        return NULL;
+    }
+    double *dts = sc, *ss = sc + L, *rs = sc + 2 * L;
+    for (int64_t row = j->row_begin; row < j->row_end; ++row) {
+        const int64_t b = row / j->dim, d = row % j->dim;
+        const float *u = j->u + row * L, *dr_raw = j->delta + row * L;
+        const float *z = j->z ? j->z + row * L : NULL;
+        const float *dy = j->dy + row * L;
+        const float *A_row = j->A + d * N;
+        const float *B_b = j->B + b * N * L, *C_b = j->C + b * N * L;
+        const double Dd = j->D ? (double)j->D[d] : 0.0;
+        const double bias = j->bias ? (double)j->bias[d] : 0.0;
+        /* forward, keeping every intermediate */
+        for (int64_t n = 0; n < N; ++n)
+            h[n] = j->initial_state ? j->initial_state[row * N + n] : 0.0;
+        for (int64_t t = 0; t < L; ++t) {
+            const double s = (double)dr_raw[t] + bias;
+            const double dt = j->softplus_flag ? mss_oracle_softplus(s) : s;
+            const double ut = (double)u[t];
+            double acc = 0.0;
+            ss[t] = s;
+            dts[t] = dt;
+            for (int64_t n = 0; n < N; ++n) {
+                const double An = (double)A_row[n];
+                a[t * N + n] = exp(dt * An);
+                w[t * N + n] = (j->zoh_input && An != 0.0) ? expm1(dt * An) / An : dt;
+                h[(t + 1) * N + n] = a[t * N + n] * h[t * N + n] + w[t * N + n] * (double)B_b[n * L + t] * ut;
+                acc += (double)C_b[n * L + t] * h[(t + 1) * N + n];
+            }
+            rs[t] = acc + Dd * ut;
+        }
+        /* reverse */
+        for (int64_t n = 0; n < N; ++n)
+            gh[n] = j->dlast ? j->dlast[row * N + n] : 0.0;
+        for (int64_t t = L - 1; t >= 0; --t) {
+            const double ut = (double)u[t], dt = dts[t];
+            double dr = (double)dy[t];
+            if (z) {
+                const double zt = (double)z[t], sg = sigmoid(zt);
+                j->dz[row * L + t] = (double)dy[t] * rs[t] * (sg + zt * sg * (1.0 - sg));
+                dr *= mss_oracle_silu(zt);
+            }
+            j->dD[d] += dr * ut;
+            double du = dr * Dd, ddt = 0.0;
+            for (int64_t n = 0; n < N; ++n) {
+                const double An = (double)A_row[n], Bn = (double)B_b[n * L + t], Cn = (double)C_b[n * L + t];
+                const double atn = a[t * N + n], wtn = w[t * N + n];
+                gh[n] += dr * Cn; /* now dLoss/dh_t */
+                j->dC[(b * N + n) * L + t] += dr * h[(t + 1) * N + n];
+                /* input term w B u */
+                j->dB[(b * N + n) * L + t] += gh[n] * wtn * ut;
+                du += gh[n] * wtn * Bn;
+                const double dw = gh[n] * Bn * ut;
+                /* transition a = exp(Delta A) */
+                const double da = gh[n] * h[t * N + n];
+                ddt += da * atn * An;
+                j->dA[d * N + n] += da * atn * dt;
+                /* weight: Euler dw/dDelta = 1; zero-order hold dw/dDelta = a,
+                 * dw/dA = (Delta a - w)/A (Delta^2/2 at A = 0) */
+                if (j->zoh_input) {
+                    ddt += dw * atn;
+                    j->dA[d * N + n] += dw * (An != 0.0 ? (dt * atn - wtn) / An : 0.5 * dt * dt);
+                } else {
+                    ddt += dw;
+                }
+                gh[n] *= atn; /* dLoss/dh_{t-1} */
+            }
+            const double ds = ddt * (j->softplus_flag ? sigmoid(ss[t]) : 1.0);
+            j->du[row * L + t] = du;
+            j->ddelta[row * L + t] = ds;
+            j->dbias[d] += ds;
+        }
+        if (j->dinit)
+            for (int64_t n = 0; n < N; ++n)
+                j->dinit[row * N + n] = gh[n];
+    }
+    free(h); free(a); free(w); free(sc); free(gh);
+    j->status = ORACLE_OK;
+    return NULL;
+}
+
+/*
+ * Backward pass.  Inputs as mss_oracle_scan_fwd, plus
+ *   dy      : [batch][dim][L]  gradient of the loss with respect to y
+ *   dlast   : [batch][dim][N]  fp64 gradient with respect to last_state (NULL: 0)
+ * Outputs (fp64, all written):
+ *   du, ddelta   : [batch][dim][L]  (ddelta is with respect to delta_raw)
+ *   dz           : [batch][dim][L]  (NULL allowed; required when z is given)
+ *   dA           : [dim][N];  dD, dbias: [dim]
+ *   dB, dC       : [batch][N][L]
+ *   dinit        : [batch][dim][N] gradient with respect to initial_state (may be NULL)
+ */
+int mss_oracle_scan_bwd(const float *u, const float *delta, const float *A, const float *B,
+                        const float *C, const float *D, const float *z, const float *delta_bias,
+                        int softplus_flag, int zoh_input, const double *initial_state,
+                        const float *dy, const double *dlast,
+                        double *du, double *ddelta, double *dz, double *dA, double *dB, double *dC,
+                        double *dD, double *dbias, double *dinit,
+                        int64_t batch, int64_t dim, int64_t dstate, int64_t seqlen, int nthreads)
+{
+    if (!u || !delta || !A || !B || !C || !dy || !du || !ddelta || !dA || !dB || !dC || !dD || !dbias ||
+        (z && !dz))
+        return ORACLE_EINVAL;
+    if (batch < 0 || dim < 0 || dstate <= 0 || seqlen < 0)
+        return ORACLE_EINVAL;
+    const int64_t N = dstate, L = seqlen, rows = batch * dim;
+    const size_t nA = (size_t)(dim * N), nBC = (size_t)(batch * N * L);
+    for (size_t i = 0; i < nA; ++i) dA[i] = 0.0;
+    for (int64_t i = 0; i < dim; ++i) dD[i] = dbias[i] = 0.0;
+    for (size_t i = 0; i < nBC; ++i) dB[i] = dC[i] = 0.0;
+    if (rows == 0)
+        return ORACLE_OK;
+    if (nthreads < 1)
+        nthreads = 1;
+    if ((int64_t)nthreads > rows)
+        nthreads = (int)rows;
+    bwd_job *jobs = (bwd_job *)calloc((size_t)nthreads, sizeof(bwd_job));
+    pthread_t *tids = (pthread_t *)calloc((size_t)nthreads, sizeof(pthread_t));
+    /* each job sums into private buffers, added up at the end */
+    const size_t priv = nA + 2 * (size_t)dim + 2 * nBC;
+    double *sums = (double *)calloc((size_t)nthreads * priv, sizeof(double));
+    if (!jobs || !tids || !sums) {
+        free(jobs); free(tids); free(sums);
+        return ORACLE_ENOMEM;
+    }
+    for (int i = 0; i < nthreads; ++i) {
+        bwd_job *jb = &jobs[i];
+        double *p = sums + (size_t)i * priv;
+        *jb = (bwd_job){u, delta, A, B, C, D, z, delta_bias, dy, initial_state, dlast,
+                        softplus_flag, zoh_input, batch, dim, N, L, du, ddelta, dz, dinit,
+                        p, p + nA, p + nA + dim, p + nA + 2 * dim, p + nA + 2 * dim + nBC,
+                        rows * i / nthreads, rows * (i + 1) / nthreads, ORACLE_EINVAL};
+        if (nthreads == 1 || pthread_create(&tids[i], NULL, bwd_rows, jb) != 0) {
+            bwd_rows(jb);
+            tids[i] = 0;
+        }
+    }
+    int rc = ORACLE_OK;
+    for (int i = 0; i < nthreads; ++i) {
+        if (tids[i])
+            pthread_join(tids[i], NULL);
+        if (jobs[i].status != ORACLE_OK)
+            rc = jobs[i].status;
+    }
+    for (int i = 0; rc == ORACLE_OK && i < nthreads; ++i) {
+        const bwd_job *jb = &jobs[i];
+        for (size_t k = 0; k < nA; ++k) dA[k] += jb->dA[k];
+        for (int64_t k = 0; k < dim; ++k) {
+            dD[k] += jb->dD[k];
+            dbias[k] += jb->dbias[k];
+        }
+        for (size_t k = 0; k < nBC; ++k) {
+            dB[k] += jb->dB[k];
+            dC[k] += jb->dC[k];
+        }
+    }
+    free(jobs); free(tids); free(sums);
+    return rc;
+}

@@ -33,9 +33,12 @@ MUTANTS = {
     "skip_dropped": ("double out = recurrence_step(h, abar, bx, c, N) + Dd * ut;",
                      "double out = recurrence_step(h, abar, bx, c, N);"),
     "gate_is_sigmoid": ("return z / (1.0 + exp(-z));", "return 1.0 / (1.0 + exp(-z));"),
-    "state_not_reset_per_row": ("        for (int64_t n = 0; n < N; ++n)\n            h[n] = j->initial_state ? j->initial_state[row * N + n] : 0.0;\n        for (int64_t t = 0; t < L; ++t) {",
-                                "        for (int64_t t = 0; t < L; ++t) {"),
-    "initial_state_ignored": ("h[n] = j->initial_state ? j->initial_state[row * N + n] : 0.0;", "h[n] = 0.0;"),
+    "state_not_reset_per_row": ("        for (int64_t n = 0; n < N; ++n)\n            h[n] = j->initial_state ? j->initial_state[row * N + n] : 0.0;\n        for (int64_t t = 0; t < L; ++t) {\n            const double ut = K",
+                                "        for (int64_t t = 0; t < L; ++t) {\n            const double ut = K"),
+    "initial_state_ignored": ("h[n] = j->initial_state ? j->initial_state[row * N + n] : 0.0;\n        for (int64_t t = 0; t < L; ++t) {\n            const double ut = K",
+                              "h[n] = 0.0;\n        for (int64_t t = 0; t < L; ++t) {\n            const double ut = K"),
+    "bwd_initial_state_ignored": ("h[n] = j->initial_state ? j->initial_state[row * N + n] : 0.0;\n        for (int64_t t = 0; t < L; ++t) {\n            const double s =",
+                                  "h[n] = 0.0;\n        for (int64_t t = 0; t < L; ++t) {\n            const double s ="),
     "decode_B_token_stride": ("j->B + b * N, j->C + b * N, 1, N,", "j->B + b * N, j->C + b * N, N, N,"),
     "B_batch_index": ("const float *B_b = j->B + b * N * L;", "const float *B_b = j->B;"),
     "conv_taps_reversed": ("acc += (double)w[k] * ext[t + k];", "acc += (double)w[K - 1 - k] * ext[t + k];"),
@@ -44,6 +47,14 @@ MUTANTS = {
     "conv_state_out_offset": ("j->conv_state_out[row * (K - 1) + k] = ext[L + k];",
                               "j->conv_state_out[row * (K - 1) + k] = ext[L + k - 1];"),
     "conv_decode_no_shift": ("                cs[k] = cs[k + 1];\n", "                cs[k] = cs[k];\n"),
+    "bwd_no_state_propagation": ("gh[n] *= atn; /* dLoss/dh_{t-1} */", "gh[n] *= 1.0;"),
+    "bwd_softplus_derivative": ("ddt * (j->softplus_flag ? sigmoid(ss[t]) : 1.0)",
+                                "ddt * (j->softplus_flag ? sigmoid(-ss[t]) : 1.0)"),
+    "bwd_dB_without_u": ("j->dB[(b * N + n) * L + t] += gh[n] * wtn * ut;", "j->dB[(b * N + n) * L + t] += gh[n] * wtn;"),
+    "bwd_dC_previous_state": ("j->dC[(b * N + n) * L + t] += dr * h[(t + 1) * N + n];",
+                              "j->dC[(b * N + n) * L + t] += dr * h[t * N + n];"),
+    "bwd_zoh_dA_sign": ("(dt * atn - wtn) / An", "(dt * atn + wtn) / An"),
+    "bwd_gate_derivative": ("(sg + zt * sg * (1.0 - sg))", "(sg + zt * sg * sg)"),
 }
 
 

@@ -628,3 +628,126 @@ def test_conv_decode_steps_equal_conv_forward(zoh):
         assert np.array_equal(yt, y[..., t])
     assert np.array_equal(state, last)
     assert np.array_equal(cstate, st)
+
+
+# --------------------------------------------------------------------------
+# Backward pass: the chain rule by hand, pinned to finite differences of the
+# (already pinned) forward pass and to an independent automatic
+# differentiation of the sequential loop.
+
+def _bwd_case(seed, batch=2, dim=3, N=4, L=7):
+    rng = np.random.default_rng(seed)
+    f32 = lambda x: np.asarray(x, dtype=np.float32)
+    inp = dict(
+        u=f32(rng.standard_normal((batch, dim, L))),
+        delta=f32(0.5 * rng.standard_normal((batch, dim, L))),
+        A=f32(-rng.uniform(0.5, 2.0, (dim, N))),
+        B=f32(rng.standard_normal((batch, N, L))),
+        C=f32(rng.standard_normal((batch, N, L))),
+        D=f32(rng.standard_normal(dim)),
+        z=f32(rng.standard_normal((batch, dim, L))),
+        delta_bias=f32(0.3 * rng.standard_normal(dim)),
+    )
+    G = f32(rng.standard_normal((batch, dim, L)))          # dLoss/dy
+    H = rng.standard_normal((batch, dim, N))               # dLoss/dlast_state
+    h0 = rng.standard_normal((batch, dim, N))
+    return inp, G, H, h0
+
+
+def _loss(inp, G, H, h0, **flags):
+    y, last = oracle.scan_fwd(**inp, initial_state=h0, **flags)
+    return float((y * G.astype(np.float64)).sum() + (last * H).sum())
+
+
+GRAD_OF = {"u": "du", "delta": "ddelta", "A": "dA", "B": "dB", "C": "dC", "D": "dD", "z": "dz",
+           "delta_bias": "dbias"}
+
+
+@pytest.mark.parametrize("flags", [dict(), dict(zoh_input=True), dict(softplus_flag=False)],
+                         ids=["euler", "zoh", "no-softplus"])
+def test_backward_matches_finite_differences(flags):
+    """Central differences of the forward pass, on fp32 inputs: the step is
+    the difference of the two rounded perturbed values, so only the O(eps^2)
+    truncation remains (relative 1e-5 is far below any dropped term)."""
+    inp, G, H, h0 = _bwd_case(90)
+    if not flags.get("softplus_flag", True):
+        inp["delta"] = np.abs(inp["delta"]) + np.float32(0.05)
+    g = oracle.scan_bwd(**inp, dy=G, dlast=H, initial_state=h0, **flags)
+    rng = np.random.default_rng(91)
+    for name, key in GRAD_OF.items():
+        x = inp[name]
+        for _ in range(4):
+            idx = tuple(int(rng.integers(s)) for s in x.shape)
+            eps = 1e-4 * max(1.0, abs(float(x[idx])))
+            xp, xm = x.copy(), x.copy()
+            xp[idx] = np.float32(x[idx] + eps)
+            xm[idx] = np.float32(x[idx] - eps)
+            fd = (_loss({**inp, name: xp}, G, H, h0, **flags) - _loss({**inp, name: xm}, G, H, h0, **flags)) / (
+                float(xp[idx]) - float(xm[idx]))
+            assert abs(g[key][idx] - fd) <= 1e-5 * abs(fd) + 1e-7, (name, idx, g[key][idx], fd)
+    # the starting state is fp64: a small symmetric step
+    for _ in range(4):
+        idx = tuple(int(rng.integers(s)) for s in h0.shape)
+        hp, hm = h0.copy(), h0.copy()
+        hp[idx] += 1e-6
+        hm[idx] -= 1e-6
+        fd = (_loss(inp, G, H, hp, **flags) - _loss(inp, G, H, hm, **flags)) / 2e-6
+        assert abs(g["dinit"][idx] - fd) <= 1e-7 * abs(fd) + 1e-8
+
+
+@pytest.mark.parametrize("zoh", [False, True])
+def test_backward_matches_autograd(zoh):
+    """Reverse-mode automatic differentiation (torch, fp64, CPU) of the
+    sequential loop gives every gradient to 1e-11."""
+    import torch
+
+    inp, G, H, h0 = _bwd_case(92)
+    inp["A"][0, 1] = 0.0  # A = 0: the zero-order hold's limit
+    t64 = {k: torch.tensor(v.astype(np.float64), requires_grad=True) for k, v in inp.items()}
+    th0 = torch.tensor(h0, requires_grad=True)
+    u, dr, A, B, C, D, z, bias = (t64[k] for k in ("u", "delta", "A", "B", "C", "D", "z", "delta_bias"))
+    batch, dim, L = u.shape
+    N = A.shape[1]
+    h = th0
+    ys = []
+    for t in range(L):
+        dt = torch.nn.functional.softplus(dr[..., t] + bias)          # [batch, dim]
+        a = torch.exp(dt[..., None] * A)                                # [batch, dim, N]
+        if zoh:
+            # at A = 0 the Taylor series of expm1(x)/x carries the derivative
+            x = dt[..., None] * A
+            safe = torch.where(A == 0, torch.ones_like(A), A)
+            series = dt[..., None] * (1 + x / 2 + x * x / 6 + x * x * x / 24)
+            wgt = torch.where(A == 0, series, torch.expm1(x) / safe)
+        else:
+            wgt = dt[..., None].expand_as(a)
+        h = a * h + wgt * B[:, None, :, t] * u[..., t, None]
+        r = (C[:, None, :, t] * h).sum(-1) + D * u[..., t]
+        ys.append(r * torch.nn.functional.silu(z[..., t]))
+    y = torch.stack(ys, dim=-1)
+    loss = (y * torch.tensor(G.astype(np.float64))).sum() + (h * torch.tensor(H)).sum()
+    loss.backward()
+    g = oracle.scan_bwd(**inp, dy=G, dlast=H, initial_state=h0, zoh_input=zoh)
+    for name, key in GRAD_OF.items():
+        np.testing.assert_allclose(g[key], t64[name].grad.numpy(), rtol=1e-11, atol=1e-12, err_msg=name)
+    np.testing.assert_allclose(g["dinit"], th0.grad.numpy(), rtol=1e-11, atol=1e-12)
+
+
+def test_backward_single_step_by_hand():
+    """One token, one state, no gate, no softplus: y = C (a h0 + Delta B u) + D u
+    with a = e^{Delta A}: every partial derivative written out."""
+    u, dl, A, B, C, D, h0, G = 0.7, 0.25, -1.5, 0.9, -1.3, 0.4, 0.6, 1.0
+    inp = dict(u=np.array([[[u]]], np.float32), delta=np.array([[[dl]]], np.float32),
+               A=np.array([[A]], np.float32), B=np.array([[[B]]], np.float32), C=np.array([[[C]]], np.float32),
+               D=np.array([D], np.float32))
+    g = oracle.scan_bwd(**inp, dy=np.ones((1, 1, 1), np.float32), softplus_flag=False,
+                        initial_state=np.array([[[h0]]]))
+    u, dl, A, B, C, D = (float(np.float32(v)) for v in (u, dl, A, B, C, D))
+    a = math.exp(dl * A)
+    assert math.isclose(g["du"][0, 0, 0], C * dl * B + D, rel_tol=1e-14)
+    assert math.isclose(g["ddelta"][0, 0, 0], C * (A * a * h0 + B * u), rel_tol=1e-14)
+    assert math.isclose(g["dA"][0, 0], C * dl * a * h0, rel_tol=1e-14)
+    assert math.isclose(g["dB"][0, 0, 0], C * dl * u, rel_tol=1e-14)
+    assert math.isclose(g["dC"][0, 0, 0], a * h0 + dl * B * u, rel_tol=1e-14)
+    assert math.isclose(g["dD"][0], u, rel_tol=1e-14)
+    assert math.isclose(g["dinit"][0, 0, 0], C * a, rel_tol=1e-14)
