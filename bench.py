@@ -372,6 +372,25 @@ def run_mss(args, rank, world, local_rank):
     ms_gen, fwd_ms_gen, _ = timed(mss.FLAG_GENERAL_A, args.steps, args.warmup)
     ms_zoh, fwd_ms_zoh, _ = timed(mss.FLAG_ZOH_INPUT, args.steps, args.warmup)
 
+    # the forward pass with the causal convolution (width 4) in front: u is
+    # read as the convolution's input x
+    cw, cb = (torch.from_numpy(v).to(dev) for v in gen.conv_params(w.dim, 4, rank_seed(w.seed, rank)))
+    cs_in = torch.zeros(w.batch, w.dim, 3, dtype=torch.bfloat16, device=dev)
+    cs_out = torch.empty_like(cs_in)
+    conv_ms = []
+    for i in range(args.warmup + args.steps):
+        a_, b_ = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a_.record(stream)
+        mss.scan_fwd_conv(d["u"], cw, d["delta"], d["A"], d["B"], d["C"], conv_b=cb, conv_state=cs_in,
+                          D=d["D"], z=d["z"], delta_bias=d["delta_bias"], y=y, last_state=state,
+                          conv_state_out=cs_out)
+        b_.record(stream)
+        if i >= args.warmup:
+            conv_ms.append((a_, b_))
+    torch.cuda.synchronize(dev)
+    conv_ms = [a_.elapsed_time(b_) for a_, b_ in conv_ms]
+    assert mss.get_device_error() == 0
+
     # end to end through the public call with host buffers: pinned host inputs,
     # copies in, forward + decode token, results copied out, every step
     host = {k: v.cpu().pin_memory() for k, v in d.items()}
@@ -439,6 +458,8 @@ def run_mss(args, rank, world, local_rank):
     fwd_avg = sum(fwd_ms) / len(fwd_ms)
     fwd_avg_gen = sum(fwd_ms_gen) / len(fwd_ms_gen)
     fwd_avg_zoh = sum(fwd_ms_zoh) / len(fwd_ms_zoh)
+    fwd_avg_conv = sum(conv_ms) / len(conv_ms)
+    bytes_conv = bytes_fwd + 2 * w.batch * w.dim * 3 * 2 + w.dim * 5 * 4  # + conv states and taps
     achieved = bytes_fwd / (fwd_avg * 1e-3) / 1e9
     achieved_gen = bytes_fwd / (fwd_avg_gen * 1e-3) / 1e9
     value = whole_job_rate(ct_per_step, world, args.steps, ms)
@@ -467,6 +488,10 @@ def run_mss(args, rank, world, local_rank):
         "general_A_path": {"fwd_ms_avg": fwd_avg_gen, "achieved_gbs": achieved_gen,
                            "frac": achieved_gen / peak,
                            "channel_tokens_per_s": w.batch * w.dim * w.seqlen / (fwd_avg_gen * 1e-3)},
+        "conv_path": {"fwd_ms_avg": fwd_avg_conv, "conv_width": 4,
+                      "achieved_gbs": bytes_conv / (fwd_avg_conv * 1e-3) / 1e9,
+                      "frac": bytes_conv / (fwd_avg_conv * 1e-3) / 1e9 / peak,
+                      "channel_tokens_per_s": w.batch * w.dim * w.seqlen / (fwd_avg_conv * 1e-3)},
         "zoh_input_path": {"fwd_ms_avg": fwd_avg_zoh,
                            "achieved_gbs": bytes_fwd / (fwd_avg_zoh * 1e-3) / 1e9,
                            "frac": bytes_fwd / (fwd_avg_zoh * 1e-3) / 1e9 / peak,

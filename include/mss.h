@@ -56,7 +56,7 @@
 extern "C" {
 #endif
 
-#define MSS_VERSION 10100 /* major*10000 + minor*100 + patch: 1.1.0 */
+#define MSS_VERSION 10200 /* major*10000 + minor*100 + patch: 1.2.0 */
 
 enum mss_dtype {
     MSS_DTYPE_F32 = 0,
@@ -66,7 +66,7 @@ enum mss_dtype {
 enum mss_status {
     MSS_OK = 0,
     MSS_ERR_NULL = -1,           /* a required pointer is NULL */
-    MSS_ERR_SHAPE = -2,          /* a size is negative, or a size product overflows int64 */
+    MSS_ERR_SHAPE = -2,          /* a size is negative or out of range (conv_width), or a product overflows */
     MSS_ERR_UNSUPPORTED_N = -3,  /* dstate is not 1, 2, 4, 8 or 16 */
     MSS_ERR_DTYPE = -4,          /* dtype is not an mss_dtype */
     MSS_ERR_ALIGN = -5,          /* a pointer is not aligned to its element size */
@@ -165,6 +165,41 @@ MSS_API int64_t mss_scan_fwd_workspace_size(int64_t batch, int64_t dim, int64_t 
                                             int dtype, unsigned flags);
 
 /*
+ * mss_scan_fwd_conv -- the forward pass with a causal convolution and SiLU
+ * in front of the scan.  The pages put "a convolution and non-linearity"
+ * between the input projection and the bank of SSMs ("Mamba" paper review,
+ * section "SSM", block description) and fuse the causal 1D convolution into
+ * the scan kernel ("NN Lab -- Mamba"); read as a per-channel causal
+ * convolution of width K followed by SiLU:
+ *
+ *   u[b,d,t] = silu(conv_b[d] + sum_{k<K} conv_w[d,k] * x[b,d,t-(K-1)+k])
+ *
+ * and u drives the scan exactly as in mss_scan_fwd_ex2 (both the input term
+ * and the skip term D*u).  x is read once; u never goes to memory.
+ *
+ *   x             : [batch][dim][seqlen] dtype  (takes the place of u)
+ *   conv_w        : [dim][K] float; tap k multiplies x_{t-(K-1)+k}
+ *   conv_b        : [dim] float (NULL: no bias)
+ *   conv_width    : K, 1..4 (else MSS_ERR_SHAPE)
+ *   conv_state_in : [batch][dim][K-1] dtype, the K-1 inputs before the first
+ *                   token, oldest first (NULL: zeros)
+ *   conv_state_out: [batch][dim][K-1] dtype, written with the last K-1 inputs
+ *                   of the history followed by x (NULL: not written); pass it
+ *                   to mss_state_update_conv or to the next call
+ *
+ * The other arguments, the sequence split and the errors are those of
+ * mss_scan_fwd_ex2 (the workspace size does not depend on the convolution);
+ * conv_state_out must not overlap any other argument.  seqlen == 0 copies
+ * conv_state_in (or zeros) to conv_state_out.
+ */
+MSS_API int mss_scan_fwd_conv(const void *x, const float *conv_w, const float *conv_b, int conv_width,
+                      const void *conv_state_in, void *conv_state_out,
+                      const void *delta, const float *A, const void *B, const void *C, const float *D,
+                      const void *z, const float *delta_bias, int softplus_flag, const float *initial_state,
+                      void *y, float *last_state, int64_t batch, int64_t dim, int64_t dstate, int64_t seqlen,
+                      int dtype, unsigned flags, void *workspace, int64_t workspace_bytes, void *stream);
+
+/*
  * mss_scan_fwd_noalloc -- mss_scan_fwd_ex2 for callers that cannot allocate
  * device memory.  The pages have no counterpart: this is an interface
  * convenience.
@@ -231,6 +266,27 @@ MSS_API int mss_state_update_ex(float *state, const void *u, const void *delta, 
                         const float *delta_bias, int softplus_flag, void *y,
                         int64_t batch, int64_t dim, int64_t dstate, int dtype,
                         unsigned flags, void *stream);
+
+/*
+ * mss_state_update_conv -- one decode token with the causal convolution of
+ * mss_scan_fwd_conv in front: u = silu(conv_b + sum_k conv_w[d,k] * window_k)
+ * over the window (conv_state[b,d,0..K-2], x[b,d]); then conv_state is
+ * shifted by one token in place (it ends with x) and the state update runs
+ * on u as in mss_state_update_ex.
+ *
+ *   conv_state : [batch][dim][K-1] dtype, read and overwritten in place
+ *                (may be NULL when K == 1); must not overlap anything else
+ *   x          : [batch][dim] dtype (takes the place of u)
+ *   conv_w, conv_b, conv_width: as in mss_scan_fwd_conv
+ *
+ * The other arguments and the errors are those of mss_state_update_ex.
+ */
+MSS_API int mss_state_update_conv(float *state, void *conv_state, const void *x, const float *conv_w,
+                          const float *conv_b, int conv_width, const void *delta, const float *A,
+                          const void *B, const void *C, const float *D, const void *z,
+                          const float *delta_bias, int softplus_flag, void *y,
+                          int64_t batch, int64_t dim, int64_t dstate, int dtype, unsigned flags,
+                          void *stream);
 
 /*
  * mss_get_device_error -- synchronises `stream`, then reports and clears the

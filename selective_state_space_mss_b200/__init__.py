@@ -22,7 +22,8 @@ import threading
 
 import torch
 
-__all__ = ["scan_fwd", "state_update", "get_device_error", "library_path", "workspace_size",
+__all__ = ["scan_fwd", "scan_fwd_conv", "state_update", "state_update_conv", "get_device_error",
+           "library_path", "workspace_size",
            "FLAG_GENERAL_A", "FLAG_SIMPLE", "FLAG_NO_SPLIT", "FLAG_ZOH_INPUT", "MssError", "load_library"]
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
@@ -78,6 +79,12 @@ def load_library():
             lib.mss_state_update_ex.argtypes = [fp, vp, vp, fp, vp, vp, fp, vp, fp, i, vp,
                                                 i64, i64, i64, i, u32, vp]
             lib.mss_state_update_ex.restype = i
+            lib.mss_scan_fwd_conv.argtypes = [vp, fp, fp, i, vp, vp, vp, fp, vp, vp, fp, vp, fp, i, fp, vp, fp,
+                                              i64, i64, i64, i64, i, u32, vp, i64, vp]
+            lib.mss_scan_fwd_conv.restype = i
+            lib.mss_state_update_conv.argtypes = [fp, vp, vp, fp, fp, i, vp, fp, vp, vp, fp, vp, fp, i, vp,
+                                                  i64, i64, i64, i, u32, vp]
+            lib.mss_state_update_conv.restype = i
             lib.mss_get_device_error.argtypes = [vp]
             lib.mss_get_device_error.restype = i
             lib.mss_strerror.argtypes = [i]
@@ -189,6 +196,105 @@ def scan_fwd(u, delta, A, B, C, D=None, z=None, delta_bias=None, softplus=True,
     if rc != 0:
         raise MssError(rc, "mss_scan_fwd")
     return y, last_state
+
+
+def scan_fwd_conv(x, conv_w, delta, A, B, C, conv_b=None, conv_state=None, D=None, z=None,
+                  delta_bias=None, softplus=True, y=None, last_state=None, want_last_state=True,
+                  conv_state_out=None, want_conv_state=True, initial_state=None, workspace="auto",
+                  flags=0, stream=None):
+    """Forward pass with the causal convolution and SiLU in front
+    (mss_scan_fwd_conv): u = silu(conv_b + causal conv of x with conv_w).
+    Returns (y, last_state, conv_state_out); each state is None when not
+    wanted and not given.
+
+    x: [batch, dim, L]; conv_w: [dim, K] float32 (K = 1..4); conv_b: [dim]
+    float32; conv_state: [batch, dim, K-1] in x's dtype (None: zeros).  Other
+    arguments as scan_fwd."""
+    if not isinstance(x, torch.Tensor) or x.device.type != "cuda":
+        raise ValueError("x must be a CUDA tensor (there is no CPU path)")
+    if x.dim() != 3:
+        raise ValueError("x must be [batch, dim, L]")
+    batch, dim, L = x.shape
+    dev, dt = x.device, x.dtype
+    code = _io_dtype(x)
+    if A.dim() != 2 or conv_w.dim() != 2:
+        raise ValueError("A must be [dim, N] and conv_w [dim, K]")
+    N, K = A.shape[1], conv_w.shape[1]
+    _check(x, "x", (batch, dim, L), dt, dev)
+    _check(conv_w, "conv_w", (dim, K), torch.float32, dev)
+    _check(conv_b, "conv_b", (dim,), torch.float32, dev, optional=True)
+    _check(conv_state, "conv_state", (batch, dim, K - 1), dt, dev, optional=True)
+    _check(delta, "delta", (batch, dim, L), dt, dev)
+    _check(A, "A", (dim, N), torch.float32, dev)
+    _check(B, "B", (batch, N, L), dt, dev)
+    _check(C, "C", (batch, N, L), dt, dev)
+    _check(D, "D", (dim,), torch.float32, dev, optional=True)
+    _check(z, "z", (batch, dim, L), dt, dev, optional=True)
+    _check(delta_bias, "delta_bias", (dim,), torch.float32, dev, optional=True)
+    _check(initial_state, "initial_state", (batch, dim, N), torch.float32, dev, optional=True)
+    if y is None:
+        y = torch.empty((batch, dim, L), dtype=dt, device=dev)
+    _check(y, "y", (batch, dim, L), dt, dev)
+    if last_state is None and want_last_state:
+        last_state = torch.empty((batch, dim, N), dtype=torch.float32, device=dev)
+    _check(last_state, "last_state", (batch, dim, N), torch.float32, dev, optional=True)
+    if conv_state_out is None and want_conv_state:
+        conv_state_out = torch.empty((batch, dim, K - 1), dtype=dt, device=dev)
+    _check(conv_state_out, "conv_state_out", (batch, dim, K - 1), dt, dev, optional=True)
+    if isinstance(workspace, str):
+        if workspace != "auto":
+            raise ValueError("workspace must be 'auto', None or a uint8 CUDA tensor")
+        nbytes = workspace_size(batch, dim, N, L, dt, flags, dev)
+        workspace = torch.empty(nbytes, dtype=torch.uint8, device=dev) if nbytes > 0 else None
+    if workspace is not None:
+        _check(workspace, "workspace", (workspace.numel(),), torch.uint8, dev)
+    rc = load_library().mss_scan_fwd_conv(
+        _ptr(x), _ptr(conv_w), _ptr(conv_b), int(K), _ptr(conv_state), _ptr(conv_state_out),
+        _ptr(delta), _ptr(A), _ptr(B), _ptr(C), _ptr(D), _ptr(z), _ptr(delta_bias), int(bool(softplus)),
+        _ptr(initial_state), _ptr(y), _ptr(last_state), batch, dim, N, L, code, int(flags),
+        _ptr(workspace), 0 if workspace is None else workspace.numel(), _stream_handle(stream, dev))
+    if rc != 0:
+        raise MssError(rc, "mss_scan_fwd_conv")
+    return y, last_state, conv_state_out
+
+
+def state_update_conv(state, conv_state, x, conv_w, delta, A, B, C, conv_b=None, D=None, z=None,
+                      delta_bias=None, softplus=True, y=None, flags=0, stream=None):
+    """One decode token with the causal convolution in front
+    (mss_state_update_conv); `state` and `conv_state` ([batch, dim, K-1] in
+    x's dtype, None when K = 1) are updated in place.  Returns y [batch, dim]."""
+    if not isinstance(state, torch.Tensor) or state.device.type != "cuda":
+        raise ValueError("state must be a CUDA tensor (there is no CPU path)")
+    if state.dim() != 3:
+        raise ValueError("state must be [batch, dim, N]")
+    batch, dim, N = state.shape
+    dev, dt = state.device, x.dtype
+    code = _io_dtype(x)
+    if conv_w.dim() != 2:
+        raise ValueError("conv_w must be [dim, K]")
+    K = conv_w.shape[1]
+    _check(state, "state", (batch, dim, N), torch.float32, dev)
+    _check(conv_state, "conv_state", (batch, dim, K - 1), dt, dev, optional=K == 1)
+    _check(x, "x", (batch, dim), dt, dev)
+    _check(conv_w, "conv_w", (dim, K), torch.float32, dev)
+    _check(conv_b, "conv_b", (dim,), torch.float32, dev, optional=True)
+    _check(delta, "delta", (batch, dim), dt, dev)
+    _check(A, "A", (dim, N), torch.float32, dev)
+    _check(B, "B", (batch, N), dt, dev)
+    _check(C, "C", (batch, N), dt, dev)
+    _check(D, "D", (dim,), torch.float32, dev, optional=True)
+    _check(z, "z", (batch, dim), dt, dev, optional=True)
+    _check(delta_bias, "delta_bias", (dim,), torch.float32, dev, optional=True)
+    if y is None:
+        y = torch.empty((batch, dim), dtype=dt, device=dev)
+    _check(y, "y", (batch, dim), dt, dev)
+    rc = load_library().mss_state_update_conv(
+        _ptr(state), _ptr(conv_state), _ptr(x), _ptr(conv_w), _ptr(conv_b), int(K), _ptr(delta), _ptr(A),
+        _ptr(B), _ptr(C), _ptr(D), _ptr(z), _ptr(delta_bias), int(bool(softplus)), _ptr(y), batch, dim, N,
+        code, int(flags), _stream_handle(stream, dev))
+    if rc != 0:
+        raise MssError(rc, "mss_state_update_conv")
+    return y
 
 
 def state_update(state, u, delta, A, B, C, D=None, z=None, delta_bias=None, softplus=True,

@@ -1,0 +1,47 @@
+// launch.h -- the kernel launchers behind the C ABI, one explicit
+// instantiation per (io type, N), compiled in separate translation units
+// (fwd_*.cu, decode.cu) so that the library builds in parallel.
+#pragma once
+
+#include <cstdint>
+
+#include <cuda_runtime.h>
+
+#include "mss_device.cuh"
+#include "mss_params.h"
+
+namespace mss_host {
+
+// Forward pass over validated arguments (p.err set): picks the throughput
+// kernel or the scalar one and, with a workspace, the sequence split.
+template <typename T, int N>
+int launch_forward(mss::ScanParams p, unsigned flags, void* workspace, int64_t workspace_bytes,
+                   cudaStream_t stream);
+
+// Workspace bytes the forward pass would use to split the sequence (0: none).
+template <typename T, int N>
+int64_t forward_workspace_bytes(int64_t batch, int64_t dim, int64_t seqlen);
+
+// Decode update over validated arguments (p.err set).
+template <typename T, int N>
+int launch_decode(mss::StepParams p, cudaStream_t stream);
+
+#define MSS_DECLARE_LAUNCHERS(T, N)                                                                      \
+    extern template int launch_forward<T, N>(mss::ScanParams, unsigned, void*, int64_t, cudaStream_t); \
+    extern template int64_t forward_workspace_bytes<T, N>(int64_t, int64_t, int64_t);                   \
+    extern template int launch_decode<T, N>(mss::StepParams, cudaStream_t);
+
+MSS_DECLARE_LAUNCHERS(mss::bf16_t, 1)
+MSS_DECLARE_LAUNCHERS(mss::bf16_t, 2)
+MSS_DECLARE_LAUNCHERS(mss::bf16_t, 4)
+MSS_DECLARE_LAUNCHERS(mss::bf16_t, 8)
+MSS_DECLARE_LAUNCHERS(mss::bf16_t, 16)
+MSS_DECLARE_LAUNCHERS(float, 1)
+MSS_DECLARE_LAUNCHERS(float, 2)
+MSS_DECLARE_LAUNCHERS(float, 4)
+MSS_DECLARE_LAUNCHERS(float, 8)
+MSS_DECLARE_LAUNCHERS(float, 16)
+
+#undef MSS_DECLARE_LAUNCHERS
+
+}  // namespace mss_host

@@ -118,15 +118,38 @@ __device__ __forceinline__ float zoh_weight(float dt, float a, float x, float e)
 }
 
 // ---------------------------------------------------------------------------
+// Causal convolution in front of the scan ("Mamba" paper review, section
+// "SSM", block description: a convolution and non-linearity before the SSM
+// bank).  The K <= 4 taps of a channel are kept right-aligned in four slots,
+// so that slot j multiplies x_{t-3+j} and slots below 4-K hold zero; the
+// window is the three previous inputs and the current one.
+
+struct ConvTaps {
+    float w[4];
+    float b;
+};
+
+__device__ __forceinline__ ConvTaps load_conv_taps(const float* conv_w, const float* conv_b, int K, int64_t d) {
+    ConvTaps c;
+#pragma unroll
+    for (int j = 0; j < 4; ++j) c.w[j] = j >= 4 - K ? __ldg(conv_w + d * K + (j - (4 - K))) : 0.f;
+    c.b = conv_b ? __ldg(conv_b + d) : 0.f;
+    return c;
+}
+
+// Pre-activation cb + sum_j w[j] x_{t-3+j} for the window (x_{t-3}, x_{t-2}, x_{t-1}, x_t).
+__device__ __forceinline__ float conv_pre(const ConvTaps& c, float xm3, float xm2, float xm1, float x0) {
+    return fmaf(c.w[3], x0, fmaf(c.w[2], xm1, fmaf(c.w[1], xm2, fmaf(c.w[0], xm3, c.b))));
+}
+
+// ---------------------------------------------------------------------------
 // Device error word: set by kernels whose bounded waits give up, read and
-// cleared by mss_get_device_error.  The library is built as a single
-// translation unit (mss_api.cu includes every kernel), so this is its only
-// definition.
-__device__ unsigned int g_mss_device_error = 0u;
+// cleared by mss_get_device_error.  It is one word per device defined in
+// mss_api.cu; every launch receives its address in its parameter block.
 constexpr unsigned int kDeviceErrTimeout = 1u;
 
-__device__ __forceinline__ void raise_device_error(unsigned int code) {
-    atomicOr(&g_mss_device_error, code);
+__device__ __forceinline__ void raise_device_error(unsigned int* err, unsigned int code) {
+    if (err) atomicOr(err, code);
 }
 
 }  // namespace mss

@@ -26,6 +26,14 @@ struct ScanParams {
     int64_t seg_len;
     int n_seg;
     int zoh;  // input matrix: 0 Euler Delta*B, 1 zero-order hold (e^{Delta A} - 1)/A * B
+    unsigned int* err;  // device error word (bounded waits that give up set it)
+    // Causal convolution in front of the scan (conv_width > 0): u holds x and
+    // the scan input is silu(conv_b + sum_k conv_w[d,k] x_{t-(K-1)+k}).
+    const float* conv_w;         // [dim, K]
+    const float* conv_b;         // [dim], may be null
+    const void* conv_state_in;   // [batch, dim, K-1] io type: x before the first token, or null (zeros)
+    void* conv_state_out;        // [batch, dim, K-1] io type: the last K-1 inputs, may be null
+    int conv_width;              // K in 1..4, or 0 without the convolution
 };
 
 struct StepParams {
@@ -43,6 +51,13 @@ struct StepParams {
     int softplus;
     int zoh;       // as in ScanParams
     int64_t row0;  // first (batch * dim + channel) row this launch serves
+    unsigned int* err;  // as in ScanParams
+    // Causal convolution in front (conv_width > 0): u holds this token's x;
+    // conv_state [batch, dim, K-1] (io type, oldest first) is read and shifted.
+    const float* conv_w;  // [dim, K]
+    const float* conv_b;  // [dim], may be null
+    void* conv_state;
+    int conv_width;
 };
 
 }  // namespace mss

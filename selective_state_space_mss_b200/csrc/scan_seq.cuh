@@ -143,6 +143,7 @@ struct LaneConst {
     float2 a2[N / 4];  // this lane's state pairs of A (times log2(e) for bf16 io)
     float ia0;         // 1 / A[d,0]                  (zero-order hold, fast transition)
     float2 ia[N / 4];  // 1 / A of this lane's state pairs (zero-order hold, general path)
+    ConvTaps conv;     // causal convolution taps (kConv)
 };
 
 // Per-token scalars of one channel.
@@ -313,7 +314,7 @@ __device__ __forceinline__ uint2 pack8(const float (&v)[8 / sizeof(T)]) {
 // state without read-out and record its aggregates (exp(A * sum of steps) and
 // the final state); otherwise the full pass, starting from the caller's state
 // carried over the earlier segments' aggregates.
-template <typename T, int N, bool kGeo, bool kGate, bool kSoftplus, bool kFold, bool kZoh>
+template <typename T, int N, bool kGeo, bool kGate, bool kSoftplus, bool kFold, bool kZoh, bool kConv>
 __device__ __forceinline__ void scan_seq_body(const SeqMaps& maps, const ScanParams& p, uint8_t* smem,
                                               uint64_t* bars, const LaneConst<N>& cc, bool valid, int64_t row) {
     using Ly = SeqLayout<T, N>;
@@ -354,21 +355,71 @@ __device__ __forceinline__ void scan_seq_body(const SeqMaps& maps, const ScanPar
     // Bounded wait for chunk c's stage; on timeout give the other copies in
     // flight a bounded chance to land and report failure (warp-uniform).
     auto wait_chunk = [&](int c) -> bool {
-        const bool landed = mbar_wait_bounded(bars + c % S, uint32_t((c / S) & 1));
+        const bool landed = mbar_wait_bounded(bars + c % S, uint32_t((c / S) & 1), p.err);
         if (__all_sync(0xffffffffu, landed)) return true;
         for (int c2 = c + 1; c2 < n_chunks && c2 < c + S; ++c2)
-            mbar_wait_bounded(bars + c2 % S, uint32_t((c2 / S) & 1), 100000000ull);
+            mbar_wait_bounded(bars + c2 % S, uint32_t((c2 / S) & 1), p.err, 100000000ull);
         return false;
     };
     const int swz = ch & 7;  // 128-byte swizzle: 16-byte chunk j of row r sits at j ^ (r & 7)
     // this lane's half of group g's u, delta, z (8 bytes of its channel's row each)
-    auto load_half = [&](int g, float (&uv)[HV], float (&dv)[HV], float (&zv)[HV]) {
+    // causal convolution (kConv): the three inputs before the current group
+    float xl[3] = {0.f, 0.f, 0.f};
+    auto load_half = [&](int g, float (&uv)[HV], float (&dv)[HV], float (&zv)[HV], bool advance) {
         const int c = g / GPC, j = g % GPC;
         const uint8_t* src = smem + (c % S) * Ly::kStageBytes + ch * Ly::kRowBytes + ((j ^ swz) << 4) + 8 * half;
-        unpack8<T>(*reinterpret_cast<const uint2*>(src), uv);
+        if constexpr (kConv) {
+            // the whole group of x (both lanes of the pair read the same 16 bytes)
+            float xa[HV], xb[HV];
+            const uint4 w4 = *reinterpret_cast<const uint4*>(src - 8 * half);
+            unpack8<T>(make_uint2(w4.x, w4.y), xa);
+            unpack8<T>(make_uint2(w4.z, w4.w), xb);
+            float xv[V];
+#pragma unroll
+            for (int i = 0; i < HV; ++i) {
+                xv[i] = xa[i];
+                xv[HV + i] = xb[i];
+            }
+            // this lane's window: inputs half*HV - 3 .. half*HV + HV - 1 of the group
+            // (index e of the extended row xl[0..2], xv[0..V-1] is input e - 3)
+            auto ext = [&](int e) { return e < 3 ? xl[e] : xv[e - 3]; };
+            float win[HV + 3];
+#pragma unroll
+            for (int i = 0; i < HV + 3; ++i) win[i] = half ? ext(HV + i) : ext(i);
+#pragma unroll
+            for (int k = 0; k < HV; ++k) {
+                const float pre = conv_pre(cc.conv, win[k], win[k + 1], win[k + 2], win[k + 3]);
+                uv[k] = kFast ? silu_fast(pre) : silu_precise(pre);
+            }
+            if (advance) {
+                xl[0] = xv[V - 3];
+                xl[1] = xv[V - 2];
+                xl[2] = xv[V - 1];
+            }
+        } else {
+            unpack8<T>(*reinterpret_cast<const uint2*>(src), uv);
+        }
         unpack8<T>(*reinterpret_cast<const uint2*>(src + Ly::kTile), dv);
         if constexpr (kGate) unpack8<T>(*reinterpret_cast<const uint2*>(src + 2 * Ly::kTile), zv);
     };
+    if constexpr (kConv) {
+        const int K = p.conv_width;
+        if (t_begin == 0) {
+            if (p.conv_state_in) {
+                const T* cs = static_cast<const T*>(p.conv_state_in) + row * (K - 1);
+#pragma unroll
+                for (int i = 0; i < 3; ++i) {  // slot i holds stored input i - (4 - K)
+                    const int k = i - (4 - K);
+                    if (k >= 0) xl[i] = ld(cs + k);
+                }
+            }
+        } else {
+            // a later segment: the inputs just before it (t_begin >= one chunk > 3)
+            const T* xr = static_cast<const T*>(p.u) + row * L + t_begin;
+#pragma unroll
+            for (int i = 0; i < 3; ++i) xl[i] = ld(xr - 3 + i);
+        }
+    }
 
     if (lane == 0) {
         for (int c = 0; c < S && c < n_chunks; ++c) issue(c);
@@ -422,7 +473,7 @@ __device__ __forceinline__ void scan_seq_body(const SeqMaps& maps, const ScanPar
     float pdu[HV], prd[HV], pu[HV];
     {
         float uv[HV], dv[HV], zv[HV];
-        load_half(0, uv, dv, zv);
+        load_half(0, uv, dv, zv, true);
 #pragma unroll
         for (int k = 0; k < HV; ++k) {
             own[k] = token_pre<kFast, kGeo, kGate, kSoftplus, kZoh>(uv[k], dv[k], kGate ? zv[k] : 0.f, cc);
@@ -444,7 +495,7 @@ __device__ __forceinline__ void scan_seq_body(const SeqMaps& maps, const ScanPar
         // the next group's u/delta/z, first: its stage must have landed when it opens a new chunk
         if (has_next && j == GPC - 1 && !wait_chunk(c + 1)) return;
         float uv[HV], dv[HV], zv[HV];
-        load_half(has_next ? g + 1 : g, uv, dv, zv);
+        load_half(has_next ? g + 1 : g, uv, dv, zv, has_next);
 
         TokenPre nxt[HV];
         float acc[V];
@@ -561,6 +612,18 @@ __device__ __forceinline__ void scan_seq_body(const SeqMaps& maps, const ScanPar
         for (int k = 0; k < HV; ++k) yv[k] = (pkeep[k] + precv[k] + pskip[k]) * pgate[k];
         if (valid) *reinterpret_cast<uint2*>(yrow + pend_at) = pack8<T>(yv);
     }
+    if constexpr (kConv) {
+        // the conv state after the sequence: its last K-1 inputs
+        const int K = p.conv_width;
+        if (valid && half == 0 && p.conv_state_out && seg == p.n_seg - 1) {
+            T* cs = static_cast<T*>(p.conv_state_out) + row * (K - 1);
+#pragma unroll
+            for (int i = 0; i < 3; ++i) {
+                const int k = i - (4 - K);
+                if (k >= 0) cs[k] = from_f32<T>(xl[i]);
+            }
+        }
+    }
     if (valid && p.last_state && seg == p.n_seg - 1) {
         float* ls = p.last_state + row * N + half;
 #pragma unroll
@@ -577,7 +640,7 @@ __device__ __forceinline__ void scan_seq_body(const SeqMaps& maps, const ScanPar
 // 0 .. n_seg-2, the full pass all n_seg (after the fold has completed).
 // Requirements checked by the host: N in {4, 8, 16}; L * sizeof(T) a multiple
 // of 16; u, delta, z, B, C, y 16-byte aligned; seg_len a multiple of the chunk.
-template <typename T, int N, bool kGate, bool kSoftplus, bool kFold, bool kZoh>
+template <typename T, int N, bool kGate, bool kSoftplus, bool kFold, bool kZoh, bool kConv>
 __global__ void __launch_bounds__(32) scan_fwd_seq_kernel(const __grid_constant__ SeqMaps maps, ScanParams p,
                                                           int allow_geo) {
     using Ly = SeqLayout<T, N>;
@@ -615,6 +678,7 @@ __global__ void __launch_bounds__(32) scan_fwd_seq_kernel(const __grid_constant_
     const float a_first = Arow[0];
     cc.a0 = a_first * kLog2e;
     if constexpr (kZoh) cc.ia0 = 1.f / a_first;  // inf at A = 0, where only the Taylor branch is taken
+    if constexpr (kConv) cc.conv = load_conv_taps(p.conv_w, p.conv_b, p.conv_width, d);
     bool geo = kFast && allow_geo;
 #pragma unroll
     for (int i = 0; i < P; ++i) {
@@ -628,11 +692,11 @@ __global__ void __launch_bounds__(32) scan_fwd_seq_kernel(const __grid_constant_
 
     if constexpr (kFast) {
         if (geo) {
-            scan_seq_body<T, N, true, kGate, kSoftplus, kFold, kZoh>(maps, p, smem, bars, cc, valid, row);
+            scan_seq_body<T, N, true, kGate, kSoftplus, kFold, kZoh, kConv>(maps, p, smem, bars, cc, valid, row);
             return;
         }
     }
-    scan_seq_body<T, N, false, kGate, kSoftplus, kFold, kZoh>(maps, p, smem, bars, cc, valid, row);
+    scan_seq_body<T, N, false, kGate, kSoftplus, kFold, kZoh, kConv>(maps, p, smem, bars, cc, valid, row);
 }
 
 }  // namespace mss

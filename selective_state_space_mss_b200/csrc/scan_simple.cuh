@@ -1,6 +1,9 @@
 // scan_simple.cuh -- reference forward kernel: one thread per (batch, channel),
 // the recurrence run token by token in registers with full-precision math.
 //
+// With the causal convolution in front, each thread keeps its channel's three
+// previous inputs and forms u = silu(conv) token by token.
+//
 // It accepts any element-aligned pointers and any shape, and it is the
 // parity anchor for the throughput kernel (scan_chunked.cuh): both must agree
 // with the oracle, and with each other within the same tolerance.  It is not
@@ -37,9 +40,31 @@ __global__ void __launch_bounds__(128) scan_fwd_simple_kernel(ScanParams p) {
     }
     const float bias = p.delta_bias ? p.delta_bias[d] : 0.f;
     const float Dd = p.D ? p.D[d] : 0.f;
+    // causal convolution: the three previous inputs (zero or the conv state)
+    const int K = p.conv_width;
+    ConvTaps taps{};
+    float xm[3] = {0.f, 0.f, 0.f};
+    if (K > 0) {
+        taps = load_conv_taps(p.conv_w, p.conv_b, K, d);
+        if (p.conv_state_in) {
+            const T* cs = static_cast<const T*>(p.conv_state_in) + row * (K - 1);
+#pragma unroll
+            for (int i = 0; i < 3; ++i) {  // slot i holds stored input i - (4 - K)
+                const int k = i - (4 - K);
+                if (k >= 0) xm[i] = ld(cs + k);
+            }
+        }
+    }
 
     for (int64_t t = 0; t < L; ++t) {
-        const float ut = ld(u + t);
+        float ut = ld(u + t);
+        if (K > 0) {
+            const float x = ut;
+            ut = silu_precise(conv_pre(taps, xm[0], xm[1], xm[2], x));
+            xm[0] = xm[1];
+            xm[1] = xm[2];
+            xm[2] = x;
+        }
         const float s = ld(dr + t) + bias;
         const float dt = p.softplus ? softplus_precise(s) : s;
         const float du = dt * ut;
@@ -60,6 +85,14 @@ __global__ void __launch_bounds__(128) scan_fwd_simple_kernel(ScanParams p) {
     if (p.last_state) {
 #pragma unroll
         for (int n = 0; n < N; ++n) p.last_state[row * N + n] = h[n];
+    }
+    if (K > 1 && p.conv_state_out) {
+        T* cs = static_cast<T*>(p.conv_state_out) + row * (K - 1);
+#pragma unroll
+        for (int i = 0; i < 3; ++i) {
+            const int k = i - (4 - K);
+            if (k >= 0) cs[k] = from_f32<T>(xm[i]);
+        }
     }
 }
 

@@ -54,7 +54,22 @@ __global__ void __launch_bounds__(256) state_update_kernel(StepParams p) {
         Cv[i] = ld(Cp + i);
     }
 
-    const float ut = ld(static_cast<const T*>(p.u) + r);
+    float ut = ld(static_cast<const T*>(p.u) + r);
+    float x_new = 0.f;
+    if (p.conv_width > 0) {
+        // causal convolution over the stored K-1 inputs and this token's x
+        const int K = p.conv_width;
+        const T* cs = static_cast<const T*>(p.conv_state) + r * (K - 1);
+        float xm[3] = {0.f, 0.f, 0.f};
+#pragma unroll
+        for (int i = 0; i < 3; ++i) {  // slot i holds stored input i - (4 - K)
+            const int k = i - (4 - K);
+            if (k >= 0) xm[i] = ld(cs + k);
+        }
+        x_new = ut;
+        const float pre = conv_pre(load_conv_taps(p.conv_w, p.conv_b, K, d), xm[0], xm[1], xm[2], x_new);
+        ut = kFast ? silu_fast(pre) : silu_precise(pre);
+    }
     const float s = ld(static_cast<const T*>(p.delta) + r) + (p.delta_bias ? __ldg(p.delta_bias + d) : 0.f);
     const float dt = p.softplus ? (kFast ? softplus_fast(s) : softplus_precise(s)) : s;
     const float du = dt * ut;
@@ -76,6 +91,14 @@ __global__ void __launch_bounds__(256) state_update_kernel(StepParams p) {
     } else {
 #pragma unroll
         for (int i = 0; i < SPT; ++i) st[i] = h[i];
+    }
+    if (q == 0 && p.conv_width > 1) {
+        // shift the conv state by one token (every lane of the channel has read
+        // it: the shuffles above order those reads before this write)
+        const int K = p.conv_width;
+        T* cs = static_cast<T*>(p.conv_state) + r * (K - 1);
+        for (int k = 0; k + 1 < K - 1; ++k) cs[k] = cs[k + 1];
+        cs[K - 2] = from_f32<T>(x_new);
     }
     if (q == 0) {
         float out = fmaf(p.D ? __ldg(p.D + d) : 0.f, ut, acc);

@@ -13,9 +13,13 @@
 // memory and write y there, and the same thread stores both back with bulk
 // copies, so that neither direction occupies registers while in flight.
 //
+// With the causal convolution in front, the tile's conv state (K-1 inputs per
+// channel) travels with it and is shifted in shared memory.
+//
 // Requirements (checked by the host): N in {4, 8, 16}; dim a multiple of
-// 1024/N; state, A, u, delta, z, y 16-byte aligned (otherwise the host runs
-// state_update_kernel).  Waits on the stage barriers are bounded.
+// 1024/N; state, A, u, delta, z, y and the conv state 16-byte aligned
+// (otherwise the host runs state_update_kernel).  Waits on the stage
+// barriers are bounded.
 #pragma once
 
 #include "mss_device.cuh"
@@ -30,7 +34,8 @@ struct DecodeTile {
     static constexpr int kRows = 1024 / N;                   // channels per tile
     static constexpr int kStateBytes = kRows * N * 4;        // 4 KB
     static constexpr int kIoBytes = kRows * int(sizeof(T));  // one of u, delta, z, y
-    static constexpr int kStageBytes = kStateBytes + 4 * kIoBytes;
+    static constexpr int kConvOffset = kStateBytes + 4 * kIoBytes;  // conv state: up to 3 inputs per channel
+    static constexpr int kStageBytes = kConvOffset + 3 * kIoBytes;
     static constexpr int kStages = 4;
     static constexpr int kThreads = 128;
     static constexpr int kTPC = N / 4;                               // threads per channel
@@ -62,7 +67,9 @@ __global__ void __launch_bounds__(128) state_update_tma_kernel(StepParams p, int
     const int64_t my_tiles = b_first < p.batch ? (p.batch - 1 - b_first) / bsplit + 1 : 0;
     const int64_t d0 = int64_t(cblock) * Ly::kRows;
     const bool gated = p.z != nullptr;
-    const uint32_t tx = uint32_t(Ly::kStateBytes + (gated ? 3 : 2) * Ly::kIoBytes);
+    const int K = p.conv_width;
+    const int conv_bytes = K > 1 ? (K - 1) * Ly::kIoBytes : 0;  // this tile's conv state
+    const uint32_t tx = uint32_t(Ly::kStateBytes + (gated ? 3 : 2) * Ly::kIoBytes + conv_bytes);
 
     if (tid == 0) {
         for (int s = 0; s < S; ++s) mbar_init(bars + s, 1);
@@ -82,13 +89,16 @@ __global__ void __launch_bounds__(128) state_update_tma_kernel(StepParams p, int
         bulk_load(st + Ly::kStateBytes + Ly::kIoBytes, static_cast<const T*>(p.delta) + row0, Ly::kIoBytes, bar);
         if (gated)
             bulk_load(st + Ly::kStateBytes + 2 * Ly::kIoBytes, static_cast<const T*>(p.z) + row0, Ly::kIoBytes, bar);
+        if (conv_bytes)
+            bulk_load(st + Ly::kConvOffset, static_cast<const T*>(p.conv_state) + row0 * (K - 1), conv_bytes, bar);
     };
     if (tid == 0) {
         for (int64_t k = 0; k < S - 1 && k < my_tiles; ++k) issue(k);
     }
 
-    // per-slot channel constants: A (this thread's 4 states), D, bias
+    // per-slot channel constants: A (this thread's 4 states), D, bias, conv taps
     float a[V][4], Dd[V], bias[V];
+    ConvTaps taps[V];
 #pragma unroll
     for (int v = 0; v < V; ++v) {
         const int slot = tid + v * Ly::kThreads;
@@ -97,6 +107,7 @@ __global__ void __launch_bounds__(128) state_update_tma_kernel(StepParams p, int
         a[v][0] = av.x; a[v][1] = av.y; a[v][2] = av.z; a[v][3] = av.w;
         Dd[v] = p.D ? __ldg(p.D + d) : 0.f;
         bias[v] = p.delta_bias ? __ldg(p.delta_bias + d) : 0.f;
+        if (K > 0) taps[v] = load_conv_taps(p.conv_w, p.conv_b, K, d);
     }
     // B and C of a batch row for this thread's states (the same for every slot)
     const int q = tid % Ly::kTPC;  // slot % kTPC == tid % kTPC: kThreads is a multiple of kTPC
@@ -121,13 +132,13 @@ __global__ void __launch_bounds__(128) state_update_tma_kernel(StepParams p, int
             Cv[i] = Cn[i];
         }
         if (k + 1 < my_tiles) load_bc(b_first + (k + 1) * bsplit, Bn, Cn);
-        const bool landed = mbar_wait_bounded(bars + int(k % S), uint32_t((k / S) & 1));
+        const bool landed = mbar_wait_bounded(bars + int(k % S), uint32_t((k / S) & 1), p.err);
         if (!__syncthreads_and(landed)) {
             // give the other loads in flight a bounded chance to land, let the
             // issued stores finish, and stop
             if (tid == 0) {
                 for (int64_t k2 = k + 1; k2 < my_tiles && k2 < k + S - 1; ++k2)
-                    mbar_wait_bounded(bars + int(k2 % S), uint32_t((k2 / S) & 1), 100000000ull);
+                    mbar_wait_bounded(bars + int(k2 % S), uint32_t((k2 / S) & 1), p.err, 100000000ull);
                 bulk_wait<0>();
             }
             return;
@@ -138,13 +149,27 @@ __global__ void __launch_bounds__(128) state_update_tma_kernel(StepParams p, int
         const T* ds = reinterpret_cast<const T*>(st + Ly::kStateBytes + Ly::kIoBytes);
         const T* zs = reinterpret_cast<const T*>(st + Ly::kStateBytes + 2 * Ly::kIoBytes);
         T* ys = reinterpret_cast<T*>(st + Ly::kStateBytes + 3 * Ly::kIoBytes);
+        T* cs_tile = reinterpret_cast<T*>(st + Ly::kConvOffset);
 #pragma unroll
         for (int v = 0; v < V; ++v) {
             const int slot = tid + v * Ly::kThreads;  // float4 slot of the tile's state
             const int ch = slot / Ly::kTPC;
             const float4 hv = hs[slot];
             float h[4] = {hv.x, hv.y, hv.z, hv.w};
-            const float ut = to_f32(us[ch]);
+            float ut = to_f32(us[ch]);
+            const float x_new = ut;
+            if (K > 0) {
+                // causal convolution over the stored K-1 inputs and this token's x
+                const T* cs = cs_tile + ch * (K - 1);
+                float xm[3] = {0.f, 0.f, 0.f};
+#pragma unroll
+                for (int i = 0; i < 3; ++i) {  // slot i holds stored input i - (4 - K)
+                    const int k = i - (4 - K);
+                    if (k >= 0) xm[i] = to_f32(cs[k]);
+                }
+                const float pre = conv_pre(taps[v], xm[0], xm[1], xm[2], x_new);
+                ut = kFast ? silu_fast(pre) : silu_precise(pre);
+            }
             const float s = to_f32(ds[ch]) + bias[v];
             const float dt = p.softplus ? (kFast ? softplus_fast(s) : softplus_precise(s)) : s;
             const float du = dt * ut;
@@ -160,6 +185,12 @@ __global__ void __launch_bounds__(128) state_update_tma_kernel(StepParams p, int
 #pragma unroll
             for (int off = 1; off < Ly::kTPC; off <<= 1) acc += __shfl_xor_sync(0xffffffffu, acc, off);
             hs[slot] = make_float4(h[0], h[1], h[2], h[3]);
+            if (q == 0 && K > 1) {
+                // shift the conv state (the channel's lanes read it before the shuffles)
+                T* cs = cs_tile + ch * (K - 1);
+                for (int k = 0; k + 1 < K - 1; ++k) cs[k] = cs[k + 1];
+                cs[K - 2] = from_f32<T>(x_new);
+            }
             if (q == 0) {
                 float out = fmaf(Dd[v], ut, acc);
                 if (gated) out *= kFast ? silu_fast(to_f32(zs[ch])) : silu_precise(to_f32(zs[ch]));
@@ -172,6 +203,8 @@ __global__ void __launch_bounds__(128) state_update_tma_kernel(StepParams p, int
         if (tid == 0) {
             bulk_store(p.state + row0 * N, st, Ly::kStateBytes);
             bulk_store(static_cast<T*>(p.y) + row0, ys, Ly::kIoBytes);
+            if (conv_bytes)
+                bulk_store(static_cast<T*>(p.conv_state) + row0 * (K - 1), cs_tile, uint32_t(conv_bytes));
             bulk_commit();
             if (k + S - 1 < my_tiles) {
                 // the stage of tile k-1 is reused once its store has read it

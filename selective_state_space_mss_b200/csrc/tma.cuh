@@ -57,16 +57,16 @@ __device__ __forceinline__ uint64_t global_timer_ns() {
 }
 
 // Wait for phase `parity` of `bar` to complete, for at most `limit_ns`
-// nanoseconds.  On timeout it sets the library's device error word and
-// returns false; the caller must then stop using the staged data.
-__device__ __forceinline__ bool mbar_wait_bounded(uint64_t* bar, uint32_t parity,
+// nanoseconds.  On timeout it sets the device error word `err` and returns
+// false; the caller must then stop using the staged data.
+__device__ __forceinline__ bool mbar_wait_bounded(uint64_t* bar, uint32_t parity, unsigned int* err,
                                                   uint64_t limit_ns = 2000000000ull) {
     if (mbar_try_wait(bar, parity)) return true;
     const uint64_t t0 = global_timer_ns();
     for (uint32_t i = 1;; ++i) {
         if (mbar_try_wait(bar, parity)) return true;
         if ((i & 255u) == 0 && global_timer_ns() - t0 > limit_ns) {
-            raise_device_error(kDeviceErrTimeout);
+            raise_device_error(err, kDeviceErrTimeout);
             return false;
         }
     }

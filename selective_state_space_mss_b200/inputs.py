@@ -18,6 +18,11 @@ Recipe (the same for every workload; the seed is fixed per workload):
 * D = 1, or D ~ N(1, 0.1) where the workload says so
 * everything is drawn in fp32, then rounded to bf16 for bf16 workloads;
   A, D and bias stay fp32.
+
+With the causal convolution in front of the scan, u is read as the
+convolution's input x (the same N(0, 1) draws), the taps are
+conv_w ~ N(0, 0.5^2) and conv_b ~ N(0, 0.1^2) (fp32), and a conv state (the
+inputs before the first token) is N(0, 1) in the io type.
 """
 from __future__ import annotations
 
@@ -160,3 +165,16 @@ def initial_state(batch: int, dim: int, dstate: int, seed: int, kind: str = "zer
     if kind == "normal":
         return _rng(seed, 3).standard_normal((batch, dim, dstate), dtype=np.float32)
     raise ValueError(f"unknown initial state {kind!r}")
+
+
+def conv_params(dim: int, width: int, seed: int):
+    """Causal convolution taps [dim, width] and bias [dim], fp32."""
+    rng = _rng(seed, 4)
+    w = (np.float32(0.5) * rng.standard_normal((dim, width), dtype=np.float32)).astype(np.float32)
+    b = (np.float32(0.1) * rng.standard_normal(dim, dtype=np.float32)).astype(np.float32)
+    return w, b
+
+
+def conv_state(batch: int, dim: int, width: int, dtype: str, seed: int) -> Tensor:
+    """The width-1 inputs before the first token, [batch, dim, width-1]."""
+    return _store(_rng(seed, 5).standard_normal((batch, dim, width - 1), dtype=np.float32), dtype)

@@ -177,3 +177,52 @@ def test_workspace_size_queries(lib):
     assert q(1, 16, 16, 0, 1, 0) == 0
     assert q(1, 16, 16, 4097, 1, 0) == 0
     assert q(1, 16, 2, 4096, 1, 0) == 0
+
+
+def test_conv_argument_errors(lib):
+    codes = _enum("mss_status")
+    v = ctypes.c_void_p
+    lib.mss_scan_fwd_conv.restype = ctypes.c_int
+    lib.mss_state_update_conv.restype = ctypes.c_int
+
+    def fwd(**kw):
+        a = dict(x=P, w=P + 0x1000000, b=None, K=4, csi=None, cso=P + 0x2000000, delta=P + 0x3000000,
+                 A=P + 0x4000000, B=P + 0x5000000, C=P + 0x6000000, y=P + 0x7000000, batch=2, dim=8, N=16,
+                 L=32, dtype=1)
+        a.update(kw)
+        w = lambda x: v(x) if x is not None else None
+        return lib.mss_scan_fwd_conv(w(a["x"]), w(a["w"]), w(a["b"]), a["K"], w(a["csi"]), w(a["cso"]),
+                                     w(a["delta"]), w(a["A"]), w(a["B"]), w(a["C"]), None, None, None, 1, None,
+                                     w(a["y"]), None, ctypes.c_int64(a["batch"]), ctypes.c_int64(a["dim"]),
+                                     ctypes.c_int64(a["N"]), ctypes.c_int64(a["L"]), a["dtype"], ctypes.c_uint(0),
+                                     None, ctypes.c_int64(0), None)
+
+    assert fwd(K=0) == codes["MSS_ERR_SHAPE"]
+    assert fwd(K=5) == codes["MSS_ERR_SHAPE"]
+    assert fwd(w=None) == codes["MSS_ERR_NULL"]
+    assert fwd(cso=P + 0x2000001) == codes["MSS_ERR_ALIGN"]          # bf16 conv state: 2-byte elements
+    assert fwd(w=P + 0x1000002) == codes["MSS_ERR_ALIGN"]            # fp32 taps
+    assert fwd(cso=P + 0x7000000) == codes["MSS_ERR_ALIAS"]          # conv state out on y
+    assert fwd(cso=P + 0x1000000) == codes["MSS_ERR_ALIAS"]          # conv state out on the taps
+    assert fwd(batch=0) == 0
+
+    def step(**kw):
+        a = dict(state=P, cs=P + 0x1000000, x=P + 0x2000000, w=P + 0x3000000, K=4, delta=P + 0x4000000,
+                 A=P + 0x5000000, B=P + 0x6000000, C=P + 0x7000000, y=P + 0x8000000, batch=4, dim=8, N=16,
+                 dtype=1, flags=0)
+        a.update(kw)
+        w = lambda x: v(x) if x is not None else None
+        return lib.mss_state_update_conv(w(a["state"]), w(a["cs"]), w(a["x"]), w(a["w"]), None, a["K"],
+                                         w(a["delta"]), w(a["A"]), w(a["B"]), w(a["C"]), None, None, None, 1,
+                                         w(a["y"]), ctypes.c_int64(a["batch"]), ctypes.c_int64(a["dim"]),
+                                         ctypes.c_int64(a["N"]), a["dtype"], ctypes.c_uint(a["flags"]), None)
+
+    assert step(K=0) == codes["MSS_ERR_SHAPE"]
+    assert step(K=5) == codes["MSS_ERR_SHAPE"]
+    assert step(cs=None) == codes["MSS_ERR_NULL"]
+    assert step(w=None) == codes["MSS_ERR_NULL"]
+    assert step(cs=P + 0x1000001) == codes["MSS_ERR_ALIGN"]
+    assert step(cs=P + 0x40) == codes["MSS_ERR_ALIAS"]               # conv state on the state
+    assert step(cs=P + 0x2000000) == codes["MSS_ERR_ALIAS"]          # conv state on x
+    assert step(flags=0x1) == codes["MSS_ERR_FLAGS"]
+    assert step(batch=0) == 0
