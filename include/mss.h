@@ -56,7 +56,7 @@
 extern "C" {
 #endif
 
-#define MSS_VERSION 10200 /* major*10000 + minor*100 + patch: 1.2.0 */
+#define MSS_VERSION 10300 /* major*10000 + minor*100 + patch: 1.3.0 */
 
 enum mss_dtype {
     MSS_DTYPE_F32 = 0,
@@ -74,7 +74,8 @@ enum mss_status {
     MSS_ERR_DEVICE_TIMEOUT = -7, /* a bounded wait inside a kernel gave up */
     MSS_ERR_FLAGS = -8,          /* unknown bits in `flags` */
     MSS_ERR_ALIAS = -9,          /* an output overlaps an input */
-    MSS_ERR_SCRATCH = -10        /* mss_scan_fwd_noalloc: the split needs more than its fixed scratch */
+    MSS_ERR_SCRATCH = -10,       /* mss_scan_fwd_noalloc: the split needs more than its fixed scratch */
+    MSS_ERR_WORKSPACE = -11      /* mss_scan_bwd: no workspace, or smaller than it needs */
 };
 
 /* Flags of mss_scan_fwd_ex / mss_scan_fwd_ex2 / mss_scan_fwd_noalloc
@@ -237,6 +238,54 @@ MSS_API int mss_scan_fwd_noalloc(const void *u, const void *delta, const float *
 
 /* Size in bytes of mss_scan_fwd_noalloc's fixed scratch (per device). */
 MSS_API int64_t mss_scan_fwd_noalloc_scratch_bytes(void);
+
+/*
+ * mss_scan_bwd -- backward pass of mss_scan_fwd_ex2 (without the convolution):
+ * the gradients of a loss with respect to every input, given its gradients
+ * with respect to y and last_state.  The pages train the model end to end
+ * and have the fused kernel recompute the states in the backward pass rather
+ * than store them ("Mamba" paper review, section "Selection Mechanism"); they
+ * print no gradient, so this is the chain rule of the forward definition.
+ * The states are recomputed from checkpoints (one state per channel every
+ * 128 bytes of a row, or every 16 tokens on the scalar path) that the call
+ * writes into the caller's workspace; nothing else is stored.
+ *
+ *   forward inputs: u, delta, A, B, C, D, z, delta_bias, softplus_flag,
+ *                   initial_state, with the layouts of mss_scan_fwd_ex2, and
+ *                   flags (MSS_FLAG_ZOH_INPUT, MSS_FLAG_GENERAL_A,
+ *                   MSS_FLAG_SIMPLE) as used by the forward pass
+ *   dy      : [batch][dim][seqlen] dtype, dLoss/dy
+ *   dlast   : [batch][dim][dstate] float, dLoss/dlast_state (NULL: zero)
+ *   du, ddelta : [batch][dim][seqlen] dtype out (ddelta: with respect to
+ *                the raw delta, i.e. through softplus and the bias)
+ *   dz      : [batch][dim][seqlen] dtype out, required when z is given
+ *   dA      : [dim][dstate] float out
+ *   dB, dC  : [batch][dstate][seqlen] float out (sums over the channels)
+ *   dD, dbias : [dim] float out (NULL: not computed)
+ *   dinit   : [batch][dim][dstate] float out, dLoss/dinitial_state (NULL: not written)
+ *   workspace : at least mss_scan_bwd_workspace_size bytes of device memory,
+ *               16-byte aligned, owned by the caller; its contents on entry
+ *               do not matter
+ *
+ * dA, dB, dC, dD and dbias are zeroed and then accumulated with float atomics
+ * on the stream, so they are not bitwise reproducible between runs.  No
+ * output may overlap an input, another output or the workspace.  Errors as
+ * mss_scan_fwd_ex2, plus MSS_ERR_WORKSPACE.  seqlen == 0: the per-token and
+ * summed gradients are empty or zero and dinit = dlast.
+ */
+MSS_API int mss_scan_bwd(const void *u, const void *delta, const float *A, const void *B, const void *C,
+                 const float *D, const void *z, const float *delta_bias, int softplus_flag,
+                 const float *initial_state, const void *dy, const float *dlast,
+                 void *du, void *ddelta, void *dz, float *dA, float *dB, float *dC, float *dD,
+                 float *dbias, float *dinit, int64_t batch, int64_t dim, int64_t dstate, int64_t seqlen,
+                 int dtype, unsigned flags, void *workspace, int64_t workspace_bytes, void *stream);
+
+/* Workspace bytes mss_scan_bwd needs for these sizes and flags, assuming
+ * 16-byte aligned tensors (with unaligned ones it takes the scalar path: ask
+ * with MSS_FLAG_SIMPLE for that size).  Negative mss_status on bad
+ * arguments; 0 when there is nothing to do. */
+MSS_API int64_t mss_scan_bwd_workspace_size(int64_t batch, int64_t dim, int64_t dstate, int64_t seqlen,
+                                    int dtype, unsigned flags);
 
 /*
  * mss_state_update -- one decode token for every (batch, channel):

@@ -22,7 +22,8 @@ import threading
 
 import torch
 
-__all__ = ["scan_fwd", "scan_fwd_conv", "state_update", "state_update_conv", "get_device_error",
+__all__ = ["scan_fwd", "scan_fwd_conv", "scan_bwd", "bwd_workspace_size", "state_update", "state_update_conv",
+           "get_device_error",
            "library_path", "workspace_size",
            "FLAG_GENERAL_A", "FLAG_SIMPLE", "FLAG_NO_SPLIT", "FLAG_ZOH_INPUT", "MssError", "load_library"]
 
@@ -79,6 +80,11 @@ def load_library():
             lib.mss_state_update_ex.argtypes = [fp, vp, vp, fp, vp, vp, fp, vp, fp, i, vp,
                                                 i64, i64, i64, i, u32, vp]
             lib.mss_state_update_ex.restype = i
+            lib.mss_scan_bwd.argtypes = [vp, vp, fp, vp, vp, fp, vp, fp, i, fp, vp, fp,
+                                         vp, vp, vp, fp, fp, fp, fp, fp, fp, i64, i64, i64, i64, i, u32, vp, i64, vp]
+            lib.mss_scan_bwd.restype = i
+            lib.mss_scan_bwd_workspace_size.argtypes = [i64, i64, i64, i64, i, u32]
+            lib.mss_scan_bwd_workspace_size.restype = i64
             lib.mss_scan_fwd_conv.argtypes = [vp, fp, fp, i, vp, vp, vp, fp, vp, vp, fp, vp, fp, i, fp, vp, fp,
                                               i64, i64, i64, i64, i, u32, vp, i64, vp]
             lib.mss_scan_fwd_conv.restype = i
@@ -256,6 +262,61 @@ def scan_fwd_conv(x, conv_w, delta, A, B, C, conv_b=None, conv_state=None, D=Non
     if rc != 0:
         raise MssError(rc, "mss_scan_fwd_conv")
     return y, last_state, conv_state_out
+
+
+def bwd_workspace_size(batch, dim, dstate, seqlen, dtype=torch.bfloat16, flags=0) -> int:
+    """Bytes of workspace scan_bwd needs (16-byte aligned tensors)."""
+    code = DTYPE_BF16 if dtype == torch.bfloat16 else DTYPE_F32
+    n = int(load_library().mss_scan_bwd_workspace_size(batch, dim, dstate, seqlen, code, int(flags)))
+    if n < 0:
+        raise MssError(n, "mss_scan_bwd_workspace_size")
+    return n
+
+
+def scan_bwd(u, delta, A, B, C, dy, D=None, z=None, delta_bias=None, softplus=True, initial_state=None,
+             dlast=None, flags=0, workspace="auto", want_dinit=True, stream=None):
+    """Backward pass of scan_fwd (mss_scan_bwd).  dy: [batch, dim, L] (the io
+    dtype), dlast: [batch, dim, N] float32 or None.  Returns a dict with du,
+    ddelta, dz (None without z) in the io dtype, dA [dim, N], dB, dC
+    [batch, N, L], dD, dbias [dim] and dinit [batch, dim, N] in float32."""
+    if not isinstance(u, torch.Tensor) or u.device.type != "cuda":
+        raise ValueError("u must be a CUDA tensor (there is no CPU path)")
+    batch, dim, L = u.shape
+    dev, dt = u.device, u.dtype
+    code = _io_dtype(u)
+    N = A.shape[1]
+    for t, name, shape, typ, opt in ((u, "u", (batch, dim, L), dt, False), (delta, "delta", (batch, dim, L), dt, False),
+                                     (A, "A", (dim, N), torch.float32, False), (B, "B", (batch, N, L), dt, False),
+                                     (C, "C", (batch, N, L), dt, False), (dy, "dy", (batch, dim, L), dt, False),
+                                     (D, "D", (dim,), torch.float32, True), (z, "z", (batch, dim, L), dt, True),
+                                     (delta_bias, "delta_bias", (dim,), torch.float32, True),
+                                     (initial_state, "initial_state", (batch, dim, N), torch.float32, True),
+                                     (dlast, "dlast", (batch, dim, N), torch.float32, True)):
+        _check(t, name, shape, typ, dev, optional=opt)
+    f32 = dict(dtype=torch.float32, device=dev)
+    out = dict(du=torch.empty((batch, dim, L), dtype=dt, device=dev),
+               ddelta=torch.empty((batch, dim, L), dtype=dt, device=dev),
+               dz=torch.empty((batch, dim, L), dtype=dt, device=dev) if z is not None else None,
+               dA=torch.empty((dim, N), **f32), dB=torch.empty((batch, N, L), **f32),
+               dC=torch.empty((batch, N, L), **f32), dD=torch.empty((dim,), **f32),
+               dbias=torch.empty((dim,), **f32),
+               dinit=torch.empty((batch, dim, N), **f32) if want_dinit else None)
+    if isinstance(workspace, str):
+        if workspace != "auto":
+            raise ValueError("workspace must be 'auto', None or a uint8 CUDA tensor")
+        nbytes = bwd_workspace_size(batch, dim, N, L, dt, flags)
+        workspace = torch.empty(nbytes, dtype=torch.uint8, device=dev) if nbytes > 0 else None
+    if workspace is not None:
+        _check(workspace, "workspace", (workspace.numel(),), torch.uint8, dev)
+    rc = load_library().mss_scan_bwd(
+        _ptr(u), _ptr(delta), _ptr(A), _ptr(B), _ptr(C), _ptr(D), _ptr(z), _ptr(delta_bias), int(bool(softplus)),
+        _ptr(initial_state), _ptr(dy), _ptr(dlast), _ptr(out["du"]), _ptr(out["ddelta"]), _ptr(out["dz"]),
+        _ptr(out["dA"]), _ptr(out["dB"]), _ptr(out["dC"]), _ptr(out["dD"]), _ptr(out["dbias"]), _ptr(out["dinit"]),
+        batch, dim, N, L, code, int(flags), _ptr(workspace), 0 if workspace is None else workspace.numel(),
+        _stream_handle(stream, dev))
+    if rc != 0:
+        raise MssError(rc, "mss_scan_bwd")
+    return out
 
 
 def state_update_conv(state, conv_state, x, conv_w, delta, A, B, C, conv_b=None, D=None, z=None,

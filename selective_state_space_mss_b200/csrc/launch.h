@@ -22,6 +22,15 @@ int launch_forward(mss::ScanParams p, unsigned flags, void* workspace, int64_t w
 template <typename T, int N>
 int64_t forward_workspace_bytes(int64_t batch, int64_t dim, int64_t seqlen);
 
+// Backward pass over validated arguments: fp holds the forward arguments
+// (with p.err), bp the gradients; the workspace holds the checkpoints.
+template <typename T, int N>
+int launch_backward(mss::ScanParams fp, mss::BwdParams bp, unsigned flags, void* workspace, int64_t workspace_bytes,
+                    cudaStream_t stream);
+
+template <typename T, int N>
+int64_t backward_workspace_bytes(int64_t batch, int64_t dim, int64_t seqlen, unsigned flags);
+
 // Decode update over validated arguments (p.err set).
 template <typename T, int N>
 int launch_decode(mss::StepParams p, cudaStream_t stream);
@@ -29,7 +38,10 @@ int launch_decode(mss::StepParams p, cudaStream_t stream);
 #define MSS_DECLARE_LAUNCHERS(T, N)                                                                      \
     extern template int launch_forward<T, N>(mss::ScanParams, unsigned, void*, int64_t, cudaStream_t); \
     extern template int64_t forward_workspace_bytes<T, N>(int64_t, int64_t, int64_t);                   \
-    extern template int launch_decode<T, N>(mss::StepParams, cudaStream_t);
+    extern template int launch_decode<T, N>(mss::StepParams, cudaStream_t);                              \
+    extern template int launch_backward<T, N>(mss::ScanParams, mss::BwdParams, unsigned, void*, int64_t,   \
+                                              cudaStream_t);                                             \
+    extern template int64_t backward_workspace_bytes<T, N>(int64_t, int64_t, int64_t, unsigned);
 
 MSS_DECLARE_LAUNCHERS(mss::bf16_t, 1)
 MSS_DECLARE_LAUNCHERS(mss::bf16_t, 2)

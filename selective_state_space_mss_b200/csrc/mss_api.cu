@@ -221,6 +221,7 @@ const char* mss_strerror(int code) {
         case MSS_ERR_FLAGS: return "unknown bits in flags";
         case MSS_ERR_ALIAS: return "an output overlaps an input";
         case MSS_ERR_SCRATCH: return "the sequence split needs more than the library's fixed scratch holds";
+        case MSS_ERR_WORKSPACE: return "no workspace, or a workspace smaller than the call needs";
         default: return "unknown status code";
     }
 }
@@ -306,6 +307,96 @@ int mss_state_update_conv(float* state, void* conv_state, const void* x, const f
     if (conv_width < 1) return MSS_ERR_SHAPE;
     return state_update_impl(state, conv_state, conv_w, conv_b, conv_width, x, delta, A, B, C, D, z, delta_bias,
                              softplus_flag, y, batch, dim, dstate, dtype, flags, stream);
+}
+
+int mss_scan_bwd(const void* u, const void* delta, const float* A, const void* B, const void* C,
+                 const float* D, const void* z, const float* delta_bias, int softplus_flag,
+                 const float* initial_state, const void* dy, const float* dlast,
+                 void* du, void* ddelta, void* dz, float* dA, float* dB, float* dC, float* dD,
+                 float* dbias, float* dinit, int64_t batch, int64_t dim, int64_t dstate, int64_t seqlen,
+                 int dtype, unsigned flags, void* workspace, int64_t workspace_bytes, void* stream) {
+    if (dtype != MSS_DTYPE_F32 && dtype != MSS_DTYPE_BF16) return MSS_ERR_DTYPE;
+    if (flags & ~(MSS_FLAG_GENERAL_A | MSS_FLAG_SIMPLE | MSS_FLAG_ZOH_INPUT)) return MSS_ERR_FLAGS;
+    if (batch < 0 || dim < 0 || seqlen < 0 || workspace_bytes < 0) return MSS_ERR_SHAPE;
+    if (!valid_n(dstate)) return MSS_ERR_UNSUPPORTED_N;
+    const int64_t esz = dtype == MSS_DTYPE_BF16 ? 2 : 4;
+    int64_t rows, seq_elems, seq_bytes, bc_elems, bcf_bytes, bc_bytes, st_elems, st_bytes;
+    if (!mul_ok(batch, dim, &rows) || !mul_ok(rows, seqlen, &seq_elems) ||
+        !mul_ok(seq_elems, esz, &seq_bytes) || !mul_ok(batch * dstate, seqlen, &bc_elems) ||
+        !mul_ok(bc_elems, esz, &bc_bytes) || !mul_ok(bc_elems, 4, &bcf_bytes) || !mul_ok(rows, dstate, &st_elems) ||
+        !mul_ok(st_elems, 4, &st_bytes) || rows > (int64_t(1) << 40))
+        return MSS_ERR_SHAPE;
+    if (rows == 0) return MSS_OK;
+    if (!A || !dA || (seqlen > 0 && (!u || !delta || !B || !C || !dy || !du || !ddelta || !dB || !dC)) ||
+        (z && seqlen > 0 && !dz))
+        return MSS_ERR_NULL;
+    const void* io[] = {u, delta, B, C, z, dy, du, ddelta, dz};
+    for (const void* p : io)
+        if (p && !aligned(p, size_t(esz))) return MSS_ERR_ALIGN;
+    const void* fp[] = {A, D, delta_bias, initial_state, dlast, dA, dB, dC, dD, dbias, dinit, workspace};
+    for (const void* p : fp)
+        if (p && !aligned(p, 4)) return MSS_ERR_ALIGN;
+    const int64_t ws = workspace ? workspace_bytes : 0;
+    struct Range { const void* p; int64_t n; };
+    const Range outs[] = {{du, seq_bytes}, {ddelta, seq_bytes}, {z ? dz : nullptr, seq_bytes}, {dA, dim * dstate * 4},
+                          {dB, bcf_bytes}, {dC, bcf_bytes}, {dD, dim * 4}, {dbias, dim * 4}, {dinit, st_bytes},
+                          {workspace, ws}};
+    const Range ins[] = {{u, seq_bytes}, {delta, seq_bytes}, {z, seq_bytes}, {dy, seq_bytes}, {B, bc_bytes},
+                         {C, bc_bytes}, {A, dim * dstate * 4}, {D, dim * 4}, {delta_bias, dim * 4},
+                         {initial_state, st_bytes}, {dlast, st_bytes}};
+    for (const Range& o : outs) {
+        for (const Range& i : ins)
+            if (overlaps(o.p, o.n, i.p, i.n)) return MSS_ERR_ALIAS;
+        for (const Range& o2 : outs)
+            if (&o != &o2 && overlaps(o.p, o.n, o2.p, o2.n)) return MSS_ERR_ALIAS;
+    }
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    if (seqlen == 0) {
+        // no tokens: nothing flows through the recurrence
+        if (cudaMemsetAsync(dA, 0, size_t(dim * dstate * 4), s) != cudaSuccess ||
+            (dD && cudaMemsetAsync(dD, 0, size_t(dim * 4), s) != cudaSuccess) ||
+            (dbias && cudaMemsetAsync(dbias, 0, size_t(dim * 4), s) != cudaSuccess))
+            return MSS_ERR_CUDA;
+        if (dinit) {
+            const cudaError_t e = dlast ? cudaMemcpyAsync(dinit, dlast, size_t(st_bytes), cudaMemcpyDeviceToDevice, s)
+                                        : cudaMemsetAsync(dinit, 0, size_t(st_bytes), s);
+            if (e != cudaSuccess) return MSS_ERR_CUDA;
+        }
+        return MSS_OK;
+    }
+    mss::ScanParams p{};
+    p.u = u; p.delta = delta; p.A = A; p.B = B; p.C = C; p.D = D; p.z = z; p.delta_bias = delta_bias;
+    p.batch = batch; p.dim = dim; p.seqlen = seqlen; p.softplus = softplus_flag ? 1 : 0;
+    p.initial_state = initial_state; p.seg_len = seqlen; p.n_seg = 1;
+    p.zoh = (flags & MSS_FLAG_ZOH_INPUT) ? 1 : 0;
+    if (!(p.err = device_error_word())) return MSS_ERR_CUDA;
+    mss::BwdParams q{};
+    q.u = u; q.delta = delta; q.A = A; q.B = B; q.C = C; q.D = D; q.z = z; q.delta_bias = delta_bias;
+    q.dy = dy; q.dlast = dlast; q.du = du; q.ddelta = ddelta; q.dz = z ? dz : nullptr; q.dA = dA; q.dB = dB;
+    q.dC = dC; q.dD = dD; q.dbias = dbias; q.dinit = dinit; q.batch = batch; q.dim = dim; q.seqlen = seqlen;
+    q.softplus = p.softplus; q.err = p.err;
+    return with_n(dstate, [&](auto nc) {
+        constexpr int N = decltype(nc)::value;
+        return dtype == MSS_DTYPE_BF16 ? launch_backward<bf16_t, N>(p, q, flags, workspace, ws, s)
+                                       : launch_backward<float, N>(p, q, flags, workspace, ws, s);
+    });
+}
+
+int64_t mss_scan_bwd_workspace_size(int64_t batch, int64_t dim, int64_t dstate, int64_t seqlen, int dtype,
+                                    unsigned flags) {
+    if (dtype != MSS_DTYPE_F32 && dtype != MSS_DTYPE_BF16) return MSS_ERR_DTYPE;
+    if (flags & ~(MSS_FLAG_GENERAL_A | MSS_FLAG_SIMPLE | MSS_FLAG_ZOH_INPUT)) return MSS_ERR_FLAGS;
+    if (batch < 0 || dim < 0 || seqlen < 0) return MSS_ERR_SHAPE;
+    if (!valid_n(dstate)) return MSS_ERR_UNSUPPORTED_N;
+    int64_t rows, elems;
+    if (!mul_ok(batch, dim, &rows) || rows > (int64_t(1) << 40) || !mul_ok(rows, seqlen, &elems) ||
+        !mul_ok(elems, dstate * 4, &elems))
+        return MSS_ERR_SHAPE;
+    return with_n(dstate, [&](auto nc) -> int64_t {
+        constexpr int N = decltype(nc)::value;
+        return dtype == MSS_DTYPE_BF16 ? backward_workspace_bytes<bf16_t, N>(batch, dim, seqlen, flags)
+                                       : backward_workspace_bytes<float, N>(batch, dim, seqlen, flags);
+    });
 }
 
 int mss_get_device_error(void* stream) {

@@ -34,6 +34,41 @@ struct ScanParams {
     const void* conv_state_in;   // [batch, dim, K-1] io type: x before the first token, or null (zeros)
     void* conv_state_out;        // [batch, dim, K-1] io type: the last K-1 inputs, may be null
     int conv_width;              // K in 1..4, or 0 without the convolution
+    // Checkpoint pass of the backward pass (fold launches only): the state at
+    // the start of every chunk, [batch * dim, n_chunks, N].
+    float* ckpt;
+};
+
+// Backward pass (scan_bwd.cuh).  Inputs as ScanParams; dy is the gradient
+// with respect to y, dlast with respect to last_state (may be null).  The
+// per-token gradients du, ddelta (with respect to delta_raw) and dz have the
+// io type; dB, dC [batch, N, L], dA [dim, N], dD, dbias [dim] are fp32 sums
+// (zeroed by the host, accumulated with atomics); dinit [batch, dim, N] is
+// the gradient with respect to the starting state (may be null).
+struct BwdParams {
+    const void* u;
+    const void* delta;
+    const float* A;
+    const void* B;
+    const void* C;
+    const float* D;           // may be null
+    const void* z;            // may be null
+    const float* delta_bias;  // may be null
+    const void* dy;
+    const float* dlast;       // may be null
+    const float* ckpt;        // [batch * dim, n_chunks, N] states at chunk starts
+    void* du;
+    void* ddelta;
+    void* dz;                 // null when z is null
+    float* dA;
+    float* dB;
+    float* dC;
+    float* dD;
+    float* dbias;
+    float* dinit;             // may be null
+    int64_t batch, dim, seqlen;
+    int softplus;
+    unsigned int* err;
 };
 
 struct StepParams {

@@ -1,0 +1,466 @@
+// scan_bwd.cuh -- backward pass of the selective scan, with recomputation.
+//
+// The pages train the model end to end and say the fused kernel recomputes
+// the states in the backward pass instead of storing them ("Mamba" paper
+// review, section "Selection Mechanism").  This kernel is the chain rule of
+// the forward definition walked backwards in time:
+//
+//   gh = dLoss/dh_t:  gh += dr_t C_t;  dC_t += dr_t h_t;  dB_t += gh w_t u_t;
+//   du_t += gh w_t B_t;  dDelta_t += gh (h_{t-1} a_t A + B_t u_t dw/dDelta);
+//   dA += gh (h_{t-1} a_t Delta_t + B_t u_t dw/dA);  gh *= a_t,
+//
+// with dr_t = dy_t silu(z_t), dz_t = dy_t r_t silu'(z_t), ddelta_raw =
+// dDelta softplus'(s) and the skip term's du += dr D, dD += dr u.
+//
+// States.  A checkpoint pass (the forward kernel's fold launch with p.ckpt)
+// records the state at the start of every chunk.  This kernel walks the
+// chunks from last to first; for each it recomputes the states forward from
+// the chunk's checkpoint, keeping the state at the start of each group of V
+// tokens in shared memory, then walks the groups from last to first: it
+// recomputes the group's V states into registers and runs the V reverse
+// steps.  Every state is recomputed twice; none is stored in HBM.
+//
+// Work split and reductions.  As in the forward kernel, a CTA is one warp
+// serving 16 channels of a batch row, a lane pair per channel, each lane
+// holding N/2 states.  Per-channel sums (dA, dD, dbias) stay in registers and
+// are added into HBM once per CTA.  dB and dC are sums over the channels of a
+// batch row: each token's 2N per-lane values are reduce-scattered over the
+// 16 channels of the warp with shuffles (15 at N = 16), leaving one (state,
+// B or C) sum per lane, which is kept for the V tokens of a group and added
+// into HBM with one vector reduction (red.global.v4.f32.add) per 4 tokens.
+// The float additions of different CTAs land in an unspecified order, so
+// dB, dC, dA, dD and dbias are not bitwise reproducible from run to run.
+//
+// The transition uses the forward kernel's fast form (Abar_n = r^{n+1}) when
+// A[d,n] = (n+1) A[d,0] across the warp; the zero-order-hold input rule
+// always takes the general form here.  Waits are bounded as in the forward
+// kernel.
+#pragma once
+
+#include "scan_seq.cuh"
+
+namespace mss {
+
+struct BwdMaps {
+    CUtensorMap u, delta, z, dy, B, C;
+};
+
+template <typename T, int N>
+struct BwdLayout {
+    using F = SeqLayout<T, N>;
+    static constexpr int kRows = F::kRows;
+    static constexpr int kRowBytes = F::kRowBytes;
+    static constexpr int kChunk = F::kChunk;
+    static constexpr int kVec = F::kVec;
+    static constexpr int kGroups = kChunk / kVec;          // groups per chunk
+    static constexpr int kPairs = F::kPairs;
+    static constexpr int kTile = F::kTile;
+    static constexpr int kBCTile = F::kBCTile;
+    static constexpr int kStages = 2;
+    static constexpr int kStageBytes = 4 * kTile + 2 * kBCTile;  // u, delta, z, dy, B, C
+    static constexpr int kBCfRow = F::kBCfRow;
+    static constexpr int kBCfBytes = F::kBCfBytes;
+    static constexpr int kBCfOffset = kStages * kStageBytes;
+    static constexpr int kGsOffset = kBCfOffset + kBCfBytes;      // group-start states
+    static constexpr int kGsBytes = kGroups * 32 * (N / 2) * 4;
+    static constexpr int kBarOffset = kGsOffset + kGsBytes;
+    static constexpr int kSmemBytes = kBarOffset + kStages * 8 + 1024;
+    static_assert(kStageBytes % 1024 == 0, "stage tiles must stay 1024-byte aligned");
+};
+
+// Per-token scalars of the backward pass.
+struct BwdTok {
+    float dt;   // Delta
+    float du;   // Delta * u
+    float rdt;  // r = exp(Delta A[d,0]) (fast transition) or Delta
+    float dsp;  // dDelta / ddelta_raw: sigmoid(s) with softplus, else 1
+};
+
+template <bool kFast, bool kGeo, bool kSoftplus, int N>
+__device__ __forceinline__ BwdTok bwd_token(float ut, float dr, const LaneConst<N>& cc) {
+    BwdTok tk;
+    const float s = dr + cc.bias;
+    tk.dt = s;
+    tk.dsp = 1.f;
+    if constexpr (kSoftplus) {
+        tk.dt = kFast ? softplus_fast(s) : softplus_precise(s);
+        tk.dsp = kFast ? rcp_approx(1.f + ex2_approx(-s * kLog2e)) : 1.f / (1.f + expf(-s));
+    }
+    tk.du = tk.dt * ut;
+    tk.rdt = kGeo ? ex2_approx(tk.dt * cc.a0) : tk.dt;
+    return tk;
+}
+
+// The 8 (bf16) or 4 (fp32) tokens of one 16-byte group.
+template <typename T>
+__device__ __forceinline__ void unpack16(const uint4& w, float (&v)[16 / sizeof(T)]) {
+    constexpr int H = 8 / int(sizeof(T));
+    float a[H], b[H];
+    unpack8<T>(make_uint2(w.x, w.y), a);
+    unpack8<T>(make_uint2(w.z, w.w), b);
+#pragma unroll
+    for (int i = 0; i < H; ++i) {
+        v[i] = a[i];
+        v[H + i] = b[i];
+    }
+}
+
+// Sum of the M = 4 * (N/4) values v over the 16 channels of the warp (lane
+// bits 1..4), scattered: the lane keeps one sum; returns it.  `index` is the
+// value it holds, `writer` whether this lane is the one of its group that
+// stores it (for N < 16 the last channel bits are summed by all).
+template <int M>
+__device__ __forceinline__ float reduce_scatter_channels(float (&v)[M], int lane, int& index, bool& writer) {
+    int c = M;
+    index = 0;
+#pragma unroll
+    for (int bit = 1; bit <= 4; ++bit) {
+        const int m = 1 << bit;
+        const bool up = (lane & m) != 0;
+        if (c > 1) {
+            const int hcount = c / 2;
+#pragma unroll
+            for (int j = 0; j < M / 2; ++j) {
+                if (j < hcount) {
+                    const float send = up ? v[j] : v[j + hcount];
+                    const float keep = up ? v[j + hcount] : v[j];
+                    v[j] = keep + __shfl_xor_sync(0xffffffffu, send, m);
+                }
+            }
+            if (up) index += hcount;
+            c = hcount;
+        } else {
+            v[0] += __shfl_xor_sync(0xffffffffu, v[0], m);
+        }
+    }
+    // for M < 16 the bits after the scatter are summed: lanes with those bits
+    // clear store
+    writer = true;
+    int scatter_bits = 0;
+    for (int cc = M; cc > 1; cc >>= 1) ++scatter_bits;
+#pragma unroll
+    for (int bit = 1; bit <= 4; ++bit)
+        if (bit > scatter_bits && (lane & (1 << bit))) writer = false;
+    return v[0];
+}
+
+__device__ __forceinline__ void red_add_v4(float* p, float a, float b, float c, float d) {
+    asm volatile("red.global.v4.f32.add [%0], {%1, %2, %3, %4};" ::"l"(p), "f"(a), "f"(b), "f"(c), "f"(d)
+                 : "memory");
+}
+
+template <typename T, int N, bool kGeo, bool kGate, bool kSoftplus, bool kZoh>
+__device__ __forceinline__ void scan_bwd_body(const BwdMaps& maps, const BwdParams& p, uint8_t* smem,
+                                              uint64_t* bars, const LaneConst<N>& cc, bool valid, int64_t row) {
+    using Ly = BwdLayout<T, N>;
+    constexpr bool kFast = sizeof(T) == 2;
+    constexpr int S = Ly::kStages;
+    constexpr int V = Ly::kVec;
+    constexpr int HV = V / 2;
+    constexpr int P = Ly::kPairs;
+    constexpr int GPC = Ly::kGroups;
+    constexpr int M = 4 * P;  // dB and dC values of a lane per token
+    static_assert(!(kZoh && kGeo), "the zero-order hold takes the general transition here");
+    const int lane = threadIdx.x;
+    const int half = lane & 1;
+    const int ch = lane >> 1;
+    const int b = blockIdx.y;
+    const int row0 = int(int64_t(b) * p.dim + int64_t(blockIdx.x) * Ly::kRows);
+    const int64_t L = p.seqlen;
+    const int n_chunks = int((L + Ly::kChunk - 1) / Ly::kChunk);
+    const int64_t d = row - int64_t(b) * p.dim;
+    float* bcf = reinterpret_cast<float*>(smem + Ly::kBCfOffset);
+    float2* gs = reinterpret_cast<float2*>(smem + Ly::kGsOffset);
+    const uint32_t stage_tx = uint32_t((kGate ? 4 : 3) * Ly::kTile + 2 * Ly::kBCTile);
+
+    // the k-th chunk processed is chunk n_chunks - 1 - k
+    auto issue = [&](int k) {
+        uint8_t* st = smem + (k % S) * Ly::kStageBytes;
+        uint64_t* bar = bars + k % S;
+        const int x = (n_chunks - 1 - k) * Ly::kChunk;
+        mbar_arrive_expect_tx(bar, stage_tx);
+        tma_load_2d(st, &maps.u, x, row0, bar);
+        tma_load_2d(st + Ly::kTile, &maps.delta, x, row0, bar);
+        if constexpr (kGate) tma_load_2d(st + 2 * Ly::kTile, &maps.z, x, row0, bar);
+        tma_load_2d(st + 3 * Ly::kTile, &maps.dy, x, row0, bar);
+        tma_load_3d(st + 4 * Ly::kTile, &maps.B, x, 0, b, bar);
+        tma_load_3d(st + 4 * Ly::kTile + Ly::kBCTile, &maps.C, x, 0, b, bar);
+    };
+    auto wait_chunk = [&](int k) -> bool {
+        const bool landed = mbar_wait_bounded(bars + k % S, uint32_t((k / S) & 1), p.err);
+        if (__all_sync(0xffffffffu, landed)) return true;
+        for (int k2 = k + 1; k2 < n_chunks && k2 < k + S; ++k2)
+            mbar_wait_bounded(bars + k2 % S, uint32_t((k2 / S) & 1), p.err, 100000000ull);
+        return false;
+    };
+    if (lane == 0) {
+        for (int k = 0; k < S && k < n_chunks; ++k) issue(k);
+    }
+
+    const int swz = ch & 7;
+    auto group_word = [&](const uint8_t* st, int tile, int g) -> uint4 {
+        return *reinterpret_cast<const uint4*>(st + tile * Ly::kTile + ch * Ly::kRowBytes + ((g ^ swz) << 4));
+    };
+    const float4* my_bcf = reinterpret_cast<const float4*>(bcf) + half * P;
+    constexpr int kRowF4 = Ly::kBCfRow / 4;
+    // natural A of this lane's state pairs
+    float2 an[P];
+#pragma unroll
+    for (int i = 0; i < P; ++i) an[i] = kFast ? __fmul2_rn(cc.a2[i], make_float2(kLn2, kLn2)) : cc.a2[i];
+
+    // adjoint state, per-channel sums
+    float2 gh[P], dA_acc[P];
+#pragma unroll
+    for (int i = 0; i < P; ++i) {
+        gh[i] = make_float2(0.f, 0.f);
+        dA_acc[i] = make_float2(0.f, 0.f);
+    }
+    if (p.dlast && valid) {
+        const float* dl = p.dlast + row * N + half;
+#pragma unroll
+        for (int i = 0; i < P; ++i) gh[i] = make_float2(dl[4 * i], dl[4 * i + 2]);
+    }
+    float dD_acc = 0.f, dbias_acc = 0.f;
+
+    for (int k = 0; k < n_chunks; ++k) {
+        const int c = n_chunks - 1 - k;
+        if (!wait_chunk(k)) return;
+        const uint8_t* st = smem + (k % S) * Ly::kStageBytes;
+        convert_bc<T, N, false>(st + 4 * Ly::kTile, st + 4 * Ly::kTile + Ly::kBCTile, bcf, lane);
+        __syncwarp();
+        const int64_t t_chunk = int64_t(c) * Ly::kChunk;
+        const int ng = int(min(int64_t(GPC), (L - t_chunk) / V));
+
+        // forward from the chunk's checkpoint, keeping each group's start state
+        float2 h[P];
+        {
+            const float* ck = p.ckpt + (size_t(row) * size_t(n_chunks) + size_t(c)) * N + half;
+#pragma unroll
+            for (int i = 0; i < P; ++i) h[i] = make_float2(ck[4 * i], ck[4 * i + 2]);
+        }
+#pragma unroll 1
+        for (int g = 0; g < ng; ++g) {
+#pragma unroll
+            for (int i = 0; i < P; ++i) gs[(g * 32 + lane) * P + i] = h[i];
+            float uv[V], dv[V];
+            unpack16<T>(group_word(st, 0, g), uv);
+            unpack16<T>(group_word(st, 1, g), dv);
+            const float4* base = my_bcf + (g * V) * kRowF4;
+#pragma unroll
+            for (int t = 0; t < V; ++t) {
+                const BwdTok tk = bwd_token<kFast, kGeo, kSoftplus>(uv[t], dv[t], cc);
+                float4 rowv[P];
+#pragma unroll
+                for (int i = 0; i < P; ++i) rowv[i] = base[t * kRowF4 + i];
+                token_states<N, kFast, kGeo, kZoh, false>(h, rowv, tk.du, tk.rdt, uv[t], half, cc);
+            }
+        }
+        __syncwarp();
+
+        // groups from last to first
+#pragma unroll 1
+        for (int g = ng - 1; g >= 0; --g) {
+            float uv[V], dv[V], zv[V], yv[V];
+            unpack16<T>(group_word(st, 0, g), uv);
+            unpack16<T>(group_word(st, 1, g), dv);
+            if constexpr (kGate) unpack16<T>(group_word(st, 2, g), zv);
+            unpack16<T>(group_word(st, 3, g), yv);
+            if (!valid) {
+                // a lane past the last channel contributes nothing to the sums
+#pragma unroll
+                for (int t = 0; t < V; ++t) yv[t] = 0.f;
+            }
+            const float4* base = my_bcf + (g * V) * kRowF4;
+            // the group's states, recomputed
+            float2 h0[P], hs[V][P];
+#pragma unroll
+            for (int i = 0; i < P; ++i) h0[i] = gs[(g * 32 + lane) * P + i];
+            {
+                float2 hh[P];
+#pragma unroll
+                for (int i = 0; i < P; ++i) hh[i] = h0[i];
+#pragma unroll
+                for (int t = 0; t < V; ++t) {
+                    const BwdTok tk = bwd_token<kFast, kGeo, kSoftplus>(uv[t], dv[t], cc);
+                    float4 rowv[P];
+#pragma unroll
+                    for (int i = 0; i < P; ++i) rowv[i] = base[t * kRowF4 + i];
+                    token_states<N, kFast, kGeo, kZoh, false>(hh, rowv, tk.du, tk.rdt, uv[t], half, cc);
+#pragma unroll
+                    for (int i = 0; i < P; ++i) hs[t][i] = hh[i];
+                }
+            }
+            float red[V];  // this lane's dB or dC sum over the warp's channels, per token
+            int red_index = 0;
+            bool red_writer = true;
+            float du_o[V], ds_o[V], dz_o[V];
+#pragma unroll
+            for (int t = V - 1; t >= 0; --t) {
+                const BwdTok tk = bwd_token<kFast, kGeo, kSoftplus>(uv[t], dv[t], cc);
+                const float ut = uv[t];
+                float4 rowv[P];
+#pragma unroll
+                for (int i = 0; i < P; ++i) rowv[i] = base[t * kRowF4 + i];
+                // read-out and gate
+                float dr = yv[t];
+                if constexpr (kGate) {
+                    float racc = 0.f;
+#pragma unroll
+                    for (int i = 0; i < P; ++i) racc = fmaf(rowv[i].z, hs[t][i].x, fmaf(rowv[i].w, hs[t][i].y, racc));
+                    const float r = racc + __shfl_xor_sync(0xffffffffu, racc, 1) + cc.D * ut;
+                    const float zt = zv[t];
+                    const float sz = kFast ? rcp_approx(1.f + ex2_approx(-zt * kLog2e)) : 1.f / (1.f + expf(-zt));
+                    dz_o[t] = yv[t] * r * (sz * fmaf(zt, 1.f - sz, 1.f));
+                    dr = yv[t] * (zt * sz);
+                }
+                float2 dA[P];
+                transition<N, kFast, kGeo>(dA, tk.rdt, half, cc);
+                float vals[M];
+                float du_acc = 0.f, ddt = 0.f;
+#pragma unroll
+                for (int i = 0; i < P; ++i) {
+                    const float2 hp = t > 0 ? hs[t > 0 ? t - 1 : 0][i] : h0[i];
+                    const float Bx = rowv[i].x, By = rowv[i].y;
+                    float gx = fmaf(dr, rowv[i].z, gh[i].x), gy = fmaf(dr, rowv[i].w, gh[i].y);
+                    vals[P * 2 + 2 * i] = dr * hs[t][i].x;  // dC
+                    vals[P * 2 + 2 * i + 1] = dr * hs[t][i].y;
+                    float wx = tk.dt, wy = tk.dt, dwx = 1.f, dwy = 1.f, dAwx = 0.f, dAwy = 0.f;
+                    if constexpr (kZoh) {
+                        const float xx = tk.dt * an[i].x, xy = tk.dt * an[i].y;
+                        wx = zoh_weight(tk.dt, an[i].x, xx, dA[i].x);
+                        wy = zoh_weight(tk.dt, an[i].y, xy, dA[i].y);
+                        dwx = dA[i].x;
+                        dwy = dA[i].y;
+                        dAwx = zoh_weight_dA(tk.dt, an[i].x, xx, dA[i].x, wx);
+                        dAwy = zoh_weight_dA(tk.dt, an[i].y, xy, dA[i].y, wy);
+                    }
+                    vals[2 * i] = gx * wx * ut;  // dB
+                    vals[2 * i + 1] = gy * wy * ut;
+                    du_acc = fmaf(gx * wx, Bx, fmaf(gy * wy, By, du_acc));
+                    const float dwsx = gx * Bx * ut, dwsy = gy * By * ut;
+                    const float dax = gx * hp.x, day = gy * hp.y;
+                    ddt = fmaf(dax * dA[i].x, an[i].x, fmaf(day * dA[i].y, an[i].y, ddt));
+                    ddt = fmaf(dwsx, dwx, fmaf(dwsy, dwy, ddt));
+                    dA_acc[i].x = fmaf(dax * dA[i].x, tk.dt, fmaf(dwsx, dAwx, dA_acc[i].x));
+                    dA_acc[i].y = fmaf(day * dA[i].y, tk.dt, fmaf(dwsy, dAwy, dA_acc[i].y));
+                    gh[i] = make_float2(gx * dA[i].x, gy * dA[i].y);
+                }
+                const float du_t = du_acc + __shfl_xor_sync(0xffffffffu, du_acc, 1) + dr * cc.D;
+                const float ds_t = (ddt + __shfl_xor_sync(0xffffffffu, ddt, 1)) * tk.dsp;
+                du_o[t] = du_t;
+                ds_o[t] = ds_t;
+                dD_acc = fmaf(dr, ut, dD_acc);
+                dbias_acc += ds_t;
+                red[t] = reduce_scatter_channels<M>(vals, lane, red_index, red_writer);
+            }
+            // per-token gradients: lane half h stores tokens [h*HV, h*HV + HV)
+            if (valid) {
+                const int64_t t0 = t_chunk + int64_t(g) * V + HV * half;
+                float o1[HV], o2[HV], o3[HV];
+#pragma unroll
+                for (int k2 = 0; k2 < HV; ++k2) {
+                    o1[k2] = half ? du_o[HV + k2] : du_o[k2];
+                    o2[k2] = half ? ds_o[HV + k2] : ds_o[k2];
+                    if constexpr (kGate) o3[k2] = half ? dz_o[HV + k2] : dz_o[k2];
+                }
+                *reinterpret_cast<uint2*>(static_cast<T*>(p.du) + row * L + t0) = pack8<T>(o1);
+                *reinterpret_cast<uint2*>(static_cast<T*>(p.ddelta) + row * L + t0) = pack8<T>(o2);
+                if constexpr (kGate) *reinterpret_cast<uint2*>(static_cast<T*>(p.dz) + row * L + t0) = pack8<T>(o3);
+            }
+            // dB / dC of the group's tokens for this lane's (state, B or C)
+            if (red_writer) {
+                const int q = red_index / (2 * P);  // 0: dB, 1: dC
+                const int i = red_index % (2 * P);
+                const int n = half + 4 * (i / 2) + 2 * (i % 2);
+                float* dst = (q ? p.dC : p.dB) + (size_t(b) * N + n) * size_t(L) + size_t(t_chunk + int64_t(g) * V);
+#pragma unroll
+                for (int k2 = 0; k2 < V; k2 += 4) red_add_v4(dst + k2, red[k2], red[k2 + 1], red[k2 + 2], red[k2 + 3]);
+            }
+        }
+
+        // hand the stage to chunk k + S
+        __syncwarp();
+        if (lane == 0 && k + S < n_chunks) {
+            fence_proxy_async_smem();
+            issue(k + S);
+        }
+    }
+
+    if (!valid) return;
+    if (p.dinit) {
+        float* di = p.dinit + row * N + half;
+#pragma unroll
+        for (int i = 0; i < P; ++i) {
+            di[4 * i] = gh[i].x;
+            di[4 * i + 2] = gh[i].y;
+        }
+    }
+    float* dA_row = p.dA + d * N + half;
+#pragma unroll
+    for (int i = 0; i < P; ++i) {
+        atomicAdd(dA_row + 4 * i, dA_acc[i].x);
+        atomicAdd(dA_row + 4 * i + 2, dA_acc[i].y);
+    }
+    if (half == 0) {
+        if (p.dD) atomicAdd(p.dD + d, dD_acc);
+        if (p.dbias) atomicAdd(p.dbias + d, dbias_acc);
+    }
+}
+
+// grid = (ceil(dim / 16), batch), block = 32 threads, dynamic shared memory
+// BwdLayout<T, N>::kSmemBytes.  Requirements as the forward kernel's
+// (checked by the host), plus the checkpoints of the same chunking.
+template <typename T, int N, bool kGate, bool kSoftplus, bool kZoh>
+__global__ void __launch_bounds__(32) scan_bwd_kernel(const __grid_constant__ BwdMaps maps, BwdParams p,
+                                                      int allow_geo) {
+    using Ly = BwdLayout<T, N>;
+    constexpr int P = Ly::kPairs;
+    extern __shared__ __align__(16) uint8_t smem_raw[];
+    uint8_t* smem = smem_raw + ((1024u - (smem_addr(smem_raw) & 1023u)) & 1023u);
+    uint64_t* bars = reinterpret_cast<uint64_t*>(smem + Ly::kBarOffset);
+    const int lane = threadIdx.x;
+    const int half = lane & 1;
+    const int64_t c = int64_t(blockIdx.x) * Ly::kRows + (lane >> 1);
+    const bool valid = c < p.dim;
+    const int64_t d = valid ? c : 0;
+    const int64_t row = int64_t(blockIdx.y) * p.dim + d;
+
+    if (lane == 0) {
+        for (int s = 0; s < Ly::kStages; ++s) mbar_init(bars + s, 1);
+        fence_barrier_init();
+        prefetch_tensormap(&maps.u);
+        prefetch_tensormap(&maps.delta);
+        if (kGate) prefetch_tensormap(&maps.z);
+        prefetch_tensormap(&maps.dy);
+        prefetch_tensormap(&maps.B);
+        prefetch_tensormap(&maps.C);
+    }
+    __syncwarp();
+
+    constexpr bool kFast = sizeof(T) == 2;
+    LaneConst<N> cc;
+    cc.bias = p.delta_bias ? p.delta_bias[d] : 0.f;
+    cc.D = p.D ? p.D[d] : 0.f;
+    const float* Arow = p.A + d * N;
+    const float a_first = Arow[0];
+    cc.a0 = a_first * kLog2e;
+    bool geo = kFast && !kZoh && allow_geo;
+#pragma unroll
+    for (int i = 0; i < P; ++i) {
+        const int n = half + 4 * i;
+        const float x0 = Arow[n], x1 = Arow[n + 2];
+        cc.a2[i] = kFast ? make_float2(x0 * kLog2e, x1 * kLog2e) : make_float2(x0, x1);
+        if constexpr (kZoh) cc.ia[i] = make_float2(1.f / x0, 1.f / x1);
+        geo = geo && x0 == float(n + 1) * a_first && x1 == float(n + 3) * a_first;
+    }
+    geo = __all_sync(0xffffffffu, geo || !valid);
+    if constexpr (kFast && !kZoh) {
+        if (geo) {
+            scan_bwd_body<T, N, true, kGate, kSoftplus, kZoh>(maps, p, smem, bars, cc, valid, row);
+            return;
+        }
+    }
+    scan_bwd_body<T, N, false, kGate, kSoftplus, kZoh>(maps, p, smem, bars, cc, valid, row);
+}
+
+}  // namespace mss

@@ -313,7 +313,9 @@ __device__ __forceinline__ uint2 pack8(const float (&v)[8 / sizeof(T)]) {
 // kFold: the first pass of a split sequence -- run the segment from a zero
 // state without read-out and record its aggregates (exp(A * sum of steps) and
 // the final state); otherwise the full pass, starting from the caller's state
-// carried over the earlier segments' aggregates.
+// carried over the earlier segments' aggregates.  A fold with p.ckpt set is
+// the backward pass's checkpoint pass instead: one segment from the caller's
+// state, recording the state at the start of every chunk.
 template <typename T, int N, bool kGeo, bool kGate, bool kSoftplus, bool kFold, bool kZoh, bool kConv>
 __device__ __forceinline__ void scan_seq_body(const SeqMaps& maps, const ScanParams& p, uint8_t* smem,
                                               uint64_t* bars, const LaneConst<N>& cc, bool valid, int64_t row) {
@@ -424,18 +426,19 @@ __device__ __forceinline__ void scan_seq_body(const SeqMaps& maps, const ScanPar
     if (lane == 0) {
         for (int c = 0; c < S && c < n_chunks; ++c) issue(c);
     }
-    // starting state: zero for a fold; otherwise the caller's state carried
-    // over the aggregates of the earlier segments
+    // starting state: zero for a fold (the caller's state for a checkpoint
+    // pass); otherwise the caller's state carried over the aggregates of the
+    // earlier segments
     float2 h[P];
 #pragma unroll
     for (int i = 0; i < P; ++i) h[i] = make_float2(0.f, 0.f);
-    if constexpr (!kFold) {
+    if (!kFold || p.ckpt) {
         if (p.initial_state) {
             const float* h0 = p.initial_state + row * N + half;
 #pragma unroll
             for (int i = 0; i < P; ++i) h[i] = make_float2(h0[4 * i], h0[4 * i + 2]);
         }
-        for (int s2 = 0; s2 < seg; ++s2) {
+        for (int s2 = 0; s2 < (kFold ? 0 : seg); ++s2) {
             const float* ga = p.agg + ((size_t(s2) * 2) * rows_total + size_t(row)) * N + half;
             const float* gb = ga + rows_total * N;
 #pragma unroll
@@ -455,6 +458,18 @@ __device__ __forceinline__ void scan_seq_body(const SeqMaps& maps, const ScanPar
         else
             return h[i];
     };
+    // checkpoint pass: the state at the start of every chunk, in h_n form
+    auto store_ckpt = [&](int chunk) {
+        if (!valid) return;
+        float* ck = p.ckpt + (size_t(row) * size_t(n_chunks) + size_t(chunk)) * N + half;
+#pragma unroll
+        for (int i = 0; i < P; ++i) {
+            const float2 hs = state_out(i);
+            ck[4 * i] = hs.x;
+            ck[4 * i + 2] = hs.y;
+        }
+    };
+    if (kFold && p.ckpt) store_ckpt(0);
     float dsum = 0.f, dcomp = 0.f;  // fold: compensated sum of this lane's steps
     T* yrow = static_cast<T*>(p.y) + row * L + t_begin + HV * half;
     const float4* my_bcf = reinterpret_cast<const float4*>(bcf) + half * P;  // this lane's chunks of a row
@@ -566,6 +581,7 @@ __device__ __forceinline__ void scan_seq_body(const SeqMaps& maps, const ScanPar
         if (j == GPC - 1 || !has_next) {
             // chunk c is consumed: convert the next chunk's B/C (its stage was
             // waited for above), then hand chunk c's stage to chunk c + S
+            if (kFold && p.ckpt && has_next) store_ckpt(c + 1);
             __syncwarp();
             if (has_next) {
                 const uint8_t* st = smem + ((c + 1) % S) * Ly::kStageBytes;
@@ -586,7 +602,7 @@ __device__ __forceinline__ void scan_seq_body(const SeqMaps& maps, const ScanPar
         // it ends in from zero
         const float tot = (dsum + __shfl_xor_sync(0xffffffffu, dsum, 1)) -
                           (dcomp + __shfl_xor_sync(0xffffffffu, dcomp, 1));
-        if (valid) {
+        if (valid && p.agg) {
             float* ga = p.agg + ((size_t(seg) * 2) * rows_total + size_t(row)) * N + half;
             float* gb = ga + rows_total * N;
 #pragma unroll

@@ -178,3 +178,12 @@ def conv_params(dim: int, width: int, seed: int):
 def conv_state(batch: int, dim: int, width: int, dtype: str, seed: int) -> Tensor:
     """The width-1 inputs before the first token, [batch, dim, width-1]."""
     return _store(_rng(seed, 5).standard_normal((batch, dim, width - 1), dtype=np.float32), dtype)
+
+
+def upstream_gradients(batch: int, dim: int, dstate: int, seqlen: int, dtype: str, seed: int):
+    """Gradients arriving at the backward pass: dy ~ N(0, 1) [batch, dim, L]
+    in the io type, dlast ~ N(0, 1) [batch, dim, N] fp32."""
+    rng = _rng(seed, 6)
+    dy = _store(rng.standard_normal((batch, dim, seqlen), dtype=np.float32), dtype)
+    dlast = rng.standard_normal((batch, dim, dstate), dtype=np.float32)
+    return dy, dlast

@@ -226,3 +226,41 @@ def test_conv_argument_errors(lib):
     assert step(cs=P + 0x2000000) == codes["MSS_ERR_ALIAS"]          # conv state on x
     assert step(flags=0x1) == codes["MSS_ERR_FLAGS"]
     assert step(batch=0) == 0
+
+
+def test_bwd_argument_errors(lib):
+    codes = _enum("mss_status")
+    v = ctypes.c_void_p
+    lib.mss_scan_bwd.restype = ctypes.c_int
+    lib.mss_scan_bwd_workspace_size.restype = ctypes.c_int64
+
+    def bwd(**kw):
+        a = dict(u=P, delta=P + 0x1000000, A=P + 0x2000000, B=P + 0x3000000, C=P + 0x4000000, z=None,
+                 dy=P + 0x5000000, du=P + 0x6000000, ddelta=P + 0x7000000, dz=None, dA=P + 0x8000000,
+                 dB=P + 0x9000000, dC=P + 0xa000000, ws=P + 0xb000000, wsb=1 << 20, batch=2, dim=8, N=16, L=32,
+                 dtype=1, flags=0)
+        a.update(kw)
+        w = lambda x: v(x) if x is not None else None
+        return lib.mss_scan_bwd(w(a["u"]), w(a["delta"]), w(a["A"]), w(a["B"]), w(a["C"]), None, w(a["z"]), None, 1,
+                                None, w(a["dy"]), None, w(a["du"]), w(a["ddelta"]), w(a["dz"]), w(a["dA"]),
+                                w(a["dB"]), w(a["dC"]), None, None, None, ctypes.c_int64(a["batch"]),
+                                ctypes.c_int64(a["dim"]), ctypes.c_int64(a["N"]), ctypes.c_int64(a["L"]), a["dtype"],
+                                ctypes.c_uint(a["flags"]), w(a["ws"]), ctypes.c_int64(a["wsb"]), None)
+
+    assert bwd(dtype=3) == codes["MSS_ERR_DTYPE"]
+    assert bwd(flags=0x4) == codes["MSS_ERR_FLAGS"]      # no sequence split in the backward pass
+    assert bwd(N=3) == codes["MSS_ERR_UNSUPPORTED_N"]
+    assert bwd(L=-1) == codes["MSS_ERR_SHAPE"]
+    assert bwd(dy=None) == codes["MSS_ERR_NULL"]
+    assert bwd(z=P + 0xc000000) == codes["MSS_ERR_NULL"]  # z given without dz
+    assert bwd(dB=P + 0x9000002) == codes["MSS_ERR_ALIGN"]
+    assert bwd(du=P + 0x5000000) == codes["MSS_ERR_ALIAS"]   # du on dy
+    assert bwd(dC=P + 0x9000000) == codes["MSS_ERR_ALIAS"]   # dC on dB
+    assert bwd(ws=P + 0x8000000) == codes["MSS_ERR_ALIAS"]   # workspace on dA
+    assert bwd(batch=0) == 0
+    q = lambda *a: lib.mss_scan_bwd_workspace_size(*a)
+    assert q(1, 16, 16, 4096, 1, 0) == 16 * 64 * 16 * 4            # one state per 64-token chunk
+    assert q(1, 16, 16, 4096, 1, 0x2) == 16 * 256 * 16 * 4         # scalar path: one per 16 tokens
+    assert q(1, 16, 16, 4097, 1, 0) == 16 * 257 * 16 * 4           # odd rows take the scalar path
+    assert q(1, 16, 16, 0, 1, 0) == 0
+    assert q(1, 16, 3, 64, 1, 0) == codes["MSS_ERR_UNSUPPORTED_N"]
