@@ -40,7 +40,10 @@ METRIC = "selective-scan fwd: achieved HBM GB/s (% of B200 peak) and channel-tok
 UNIT = "channel-tokens/s"
 WORKLOAD = gen.BENCH_WORKLOAD
 FALLBACK_HBM_GBS = 6650.0
-KERNEL_SOURCES = ["selective_state_space_mss_b200/csrc"]
+# the files the timed forward kernel (and its launch) is built from: the
+# recorded DRAM traffic is reported only while they are unchanged
+KERNEL_SOURCES = ["selective_state_space_mss_b200/csrc/" + f for f in (
+    "scan_seq.cuh", "tma.cuh", "mss_device.cuh", "mss_params.h", "forward.cuh", "fwd_bf16_n16.cu")]
 
 
 def log(*a):
@@ -94,10 +97,8 @@ def measured_peaks():
 def kernel_source_hash():
     h = hashlib.sha256()
     for rel in KERNEL_SOURCES:
-        base = os.path.join(ROOT, rel)
-        for name in sorted(os.listdir(base)):
-            with open(os.path.join(base, name), "rb") as f:
-                h.update(name.encode() + b"\0" + f.read())
+        with open(os.path.join(ROOT, rel), "rb") as f:
+            h.update(os.path.basename(rel).encode() + b"\0" + f.read())
     return h.hexdigest()[:16]
 
 
@@ -391,6 +392,23 @@ def run_mss(args, rank, world, local_rank):
     conv_ms = [a_.elapsed_time(b_) for a_, b_ in conv_ms]
     assert mss.get_device_error() == 0
 
+    # the backward pass (gradients of every input, states recomputed from
+    # checkpoints) on the same workload
+    dy_h, dlast_h = gen.upstream_gradients(w.batch, w.dim, w.dstate, w.seqlen, w.dtype, rank_seed(w.seed, rank))
+    dy_d, dlast_d = to_dev(dy_h), torch.from_numpy(dlast_h).to(dev)
+    ws_b = torch.empty(mss.bwd_workspace_size(w.batch, w.dim, w.dstate, w.seqlen), dtype=torch.uint8, device=dev)
+    bwd_ev = []
+    for i in range(args.warmup + args.steps):
+        a_, b_ = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a_.record(stream)
+        mss.scan_bwd(**d, dy=dy_d, dlast=dlast_d, workspace=ws_b)
+        b_.record(stream)
+        if i >= args.warmup:
+            bwd_ev.append((a_, b_))
+    torch.cuda.synchronize(dev)
+    bwd_ms = [a_.elapsed_time(b_) for a_, b_ in bwd_ev]
+    assert mss.get_device_error() == 0
+
     # end to end through the public call with host buffers: pinned host inputs,
     # copies in, forward + decode token, results copied out, every step
     host = {k: v.cpu().pin_memory() for k, v in d.items()}
@@ -459,6 +477,14 @@ def run_mss(args, rank, world, local_rank):
     fwd_avg_gen = sum(fwd_ms_gen) / len(fwd_ms_gen)
     fwd_avg_zoh = sum(fwd_ms_zoh) / len(fwd_ms_zoh)
     fwd_avg_conv = sum(conv_ms) / len(conv_ms)
+    bwd_avg = sum(bwd_ms) / len(bwd_ms)
+    # backward traffic: u, delta read by the checkpoint pass; u, delta, z, dy
+    # read and du, ddelta, dz written by the backward kernel (bf16); B, C read
+    # by both passes, dB, dC written (fp32); checkpoints (one fp32 state per
+    # 64-token chunk) written and read
+    n_ck = (w.seqlen + 63) // 64
+    bytes_bwd = (w.batch * w.dim * w.seqlen * 2 * (2 + 4 + 3) + 2 * w.batch * w.dstate * w.seqlen * (2 + 2 + 4)
+                 + 2 * w.batch * w.dim * n_ck * w.dstate * 4)
     bytes_conv = bytes_fwd + 2 * w.batch * w.dim * 3 * 2 + w.dim * 5 * 4  # + conv states and taps
     achieved = bytes_fwd / (fwd_avg * 1e-3) / 1e9
     achieved_gen = bytes_fwd / (fwd_avg_gen * 1e-3) / 1e9
@@ -492,6 +518,10 @@ def run_mss(args, rank, world, local_rank):
                       "achieved_gbs": bytes_conv / (fwd_avg_conv * 1e-3) / 1e9,
                       "frac": bytes_conv / (fwd_avg_conv * 1e-3) / 1e9 / peak,
                       "channel_tokens_per_s": w.batch * w.dim * w.seqlen / (fwd_avg_conv * 1e-3)},
+        "backward": {"ms_avg": bwd_avg, "channel_tokens_per_s": w.batch * w.dim * w.seqlen / (bwd_avg * 1e-3),
+                     "achieved_gbs": bytes_bwd / (bwd_avg * 1e-3) / 1e9,
+                     "frac": bytes_bwd / (bwd_avg * 1e-3) / 1e9 / peak,
+                     "note": "gradients of u, delta, A, B, C, D, z, bias, starting state; checkpoint pass included"},
         "zoh_input_path": {"fwd_ms_avg": fwd_avg_zoh,
                            "achieved_gbs": bytes_fwd / (fwd_avg_zoh * 1e-3) / 1e9,
                            "frac": bytes_fwd / (fwd_avg_zoh * 1e-3) / 1e9 / peak,
