@@ -120,9 +120,12 @@ __device__ __forceinline__ float zoh_weight(float dt, float a, float x, float e)
 // d/da of the weight Delta * phi(Delta a) (the backward pass):
 // Delta^2 phi'(x), phi'(x) = 1/2 + x/3 + x^2/8 + x^3/30 + x^4/144 + ... below
 // |x| = 1/8 (first omitted term under 2e-7 of the sum), else (Delta e - w)/a.
+__device__ __forceinline__ float dphi_taylor(float x) {
+    return fmaf(fmaf(fmaf(fmaf(x, 1.f / 144.f, 1.f / 30.f), x, 1.f / 8.f), x, 1.f / 3.f), x, 0.5f);
+}
+
 __device__ __forceinline__ float zoh_weight_dA(float dt, float a, float x, float e, float w) {
-    const float dphi = fmaf(fmaf(fmaf(fmaf(x, 1.f / 144.f, 1.f / 30.f), x, 1.f / 8.f), x, 1.f / 3.f), x, 0.5f);
-    return fabsf(x) < kZohTaylorMax ? dt * dt * dphi : (dt * e - w) / a;
+    return fabsf(x) < kZohTaylorMax ? dt * dt * dphi_taylor(x) : (dt * e - w) / a;
 }
 
 // ---------------------------------------------------------------------------

@@ -37,6 +37,8 @@
 // kernel.
 #pragma once
 
+#include <type_traits>
+
 #include "scan_seq.cuh"
 
 namespace mss {
@@ -149,6 +151,10 @@ __device__ __forceinline__ void red_add_v4(float* p, float a, float b, float c, 
                  : "memory");
 }
 
+__device__ __forceinline__ void red_add_v2(float* p, float a, float b) {
+    asm volatile("red.global.v2.f32.add [%0], {%1, %2};" ::"l"(p), "f"(a), "f"(b) : "memory");
+}
+
 template <typename T, int N, bool kGeo, bool kGate, bool kSoftplus, bool kZoh>
 __device__ __forceinline__ void scan_bwd_body(const BwdMaps& maps, const BwdParams& p, uint8_t* smem,
                                               uint64_t* bars, const LaneConst<N>& cc, bool valid, int64_t row) {
@@ -257,12 +263,19 @@ __device__ __forceinline__ void scan_bwd_body(const BwdMaps& maps, const BwdPara
         }
         __syncwarp();
 
-        // groups from last to first
+        // groups from last to first; each group in two halves of HV tokens
+        // (second half first), so that only HV recomputed states are live
 #pragma unroll 1
         for (int g = ng - 1; g >= 0; --g) {
-            float uv[V], dv[V], zv[V], yv[V];
-            unpack16<T>(group_word(st, 0, g), uv);
-            unpack16<T>(group_word(st, 1, g), dv);
+            float uv[V], zv[V], yv[V];
+            BwdTok tok[V];
+            {
+                float dv[V];
+                unpack16<T>(group_word(st, 0, g), uv);
+                unpack16<T>(group_word(st, 1, g), dv);
+#pragma unroll
+                for (int t = 0; t < V; ++t) tok[t] = bwd_token<kFast, kGeo, kSoftplus>(uv[t], dv[t], cc);
+            }
             if constexpr (kGate) unpack16<T>(group_word(st, 2, g), zv);
             unpack16<T>(group_word(st, 3, g), yv);
             if (!valid) {
@@ -271,111 +284,123 @@ __device__ __forceinline__ void scan_bwd_body(const BwdMaps& maps, const BwdPara
                 for (int t = 0; t < V; ++t) yv[t] = 0.f;
             }
             const float4* base = my_bcf + (g * V) * kRowF4;
-            // the group's states, recomputed
-            float2 h0[P], hs[V][P];
-#pragma unroll
-            for (int i = 0; i < P; ++i) h0[i] = gs[(g * 32 + lane) * P + i];
-            {
-                float2 hh[P];
-#pragma unroll
-                for (int i = 0; i < P; ++i) hh[i] = h0[i];
-#pragma unroll
-                for (int t = 0; t < V; ++t) {
-                    const BwdTok tk = bwd_token<kFast, kGeo, kSoftplus>(uv[t], dv[t], cc);
-                    float4 rowv[P];
-#pragma unroll
-                    for (int i = 0; i < P; ++i) rowv[i] = base[t * kRowF4 + i];
-                    token_states<N, kFast, kGeo, kZoh, false>(hh, rowv, tk.du, tk.rdt, uv[t], half, cc);
-#pragma unroll
-                    for (int i = 0; i < P; ++i) hs[t][i] = hh[i];
-                }
-            }
-            float red[V];  // this lane's dB or dC sum over the warp's channels, per token
-            int red_index = 0;
-            bool red_writer = true;
-            float du_o[V], ds_o[V], dz_o[V];
-#pragma unroll
-            for (int t = V - 1; t >= 0; --t) {
-                const BwdTok tk = bwd_token<kFast, kGeo, kSoftplus>(uv[t], dv[t], cc);
-                const float ut = uv[t];
-                float4 rowv[P];
+            auto row_of = [&](int t, float4 (&rowv)[P]) {
 #pragma unroll
                 for (int i = 0; i < P; ++i) rowv[i] = base[t * kRowF4 + i];
-                // read-out and gate
-                float dr = yv[t];
-                if constexpr (kGate) {
-                    float racc = 0.f;
+            };
+            float2 h0[P], hmid[P];
 #pragma unroll
-                    for (int i = 0; i < P; ++i) racc = fmaf(rowv[i].z, hs[t][i].x, fmaf(rowv[i].w, hs[t][i].y, racc));
-                    const float r = racc + __shfl_xor_sync(0xffffffffu, racc, 1) + cc.D * ut;
-                    const float zt = zv[t];
-                    const float sz = kFast ? rcp_approx(1.f + ex2_approx(-zt * kLog2e)) : 1.f / (1.f + expf(-zt));
-                    dz_o[t] = yv[t] * r * (sz * fmaf(zt, 1.f - sz, 1.f));
-                    dr = yv[t] * (zt * sz);
-                }
-                float2 dA[P];
-                transition<N, kFast, kGeo>(dA, tk.rdt, half, cc);
-                float vals[M];
-                float du_acc = 0.f, ddt = 0.f;
+            for (int i = 0; i < P; ++i) h0[i] = hmid[i] = gs[(g * 32 + lane) * P + i];
 #pragma unroll
-                for (int i = 0; i < P; ++i) {
-                    const float2 hp = t > 0 ? hs[t > 0 ? t - 1 : 0][i] : h0[i];
-                    const float Bx = rowv[i].x, By = rowv[i].y;
-                    float gx = fmaf(dr, rowv[i].z, gh[i].x), gy = fmaf(dr, rowv[i].w, gh[i].y);
-                    vals[P * 2 + 2 * i] = dr * hs[t][i].x;  // dC
-                    vals[P * 2 + 2 * i + 1] = dr * hs[t][i].y;
-                    float wx = tk.dt, wy = tk.dt, dwx = 1.f, dwy = 1.f, dAwx = 0.f, dAwy = 0.f;
-                    if constexpr (kZoh) {
-                        const float xx = tk.dt * an[i].x, xy = tk.dt * an[i].y;
-                        wx = zoh_weight(tk.dt, an[i].x, xx, dA[i].x);
-                        wy = zoh_weight(tk.dt, an[i].y, xy, dA[i].y);
-                        dwx = dA[i].x;
-                        dwy = dA[i].y;
-                        dAwx = zoh_weight_dA(tk.dt, an[i].x, xx, dA[i].x, wx);
-                        dAwy = zoh_weight_dA(tk.dt, an[i].y, xy, dA[i].y, wy);
+            for (int t = 0; t < HV; ++t) {
+                float4 rowv[P];
+                row_of(t, rowv);
+                token_states<N, kFast, kGeo, kZoh, false>(hmid, rowv, tok[t].du, tok[t].rdt, uv[t], half, cc);
+            }
+            const int64_t tg = t_chunk + int64_t(g) * V;
+            auto run_half = [&](auto span) {
+                constexpr int T0 = decltype(span)::value;  // first token of this half
+                float2 hs[HV][P];
+                {
+                    float2 hh[P];
+#pragma unroll
+                    for (int i = 0; i < P; ++i) hh[i] = T0 == 0 ? h0[i] : hmid[i];
+#pragma unroll
+                    for (int t = 0; t < HV; ++t) {
+                        float4 rowv[P];
+                        row_of(T0 + t, rowv);
+                        token_states<N, kFast, kGeo, kZoh, false>(hh, rowv, tok[T0 + t].du, tok[T0 + t].rdt,
+                                                                   uv[T0 + t], half, cc);
+#pragma unroll
+                        for (int i = 0; i < P; ++i) hs[t][i] = hh[i];
                     }
-                    vals[2 * i] = gx * wx * ut;  // dB
-                    vals[2 * i + 1] = gy * wy * ut;
-                    du_acc = fmaf(gx * wx, Bx, fmaf(gy * wy, By, du_acc));
-                    const float dwsx = gx * Bx * ut, dwsy = gy * By * ut;
-                    const float dax = gx * hp.x, day = gy * hp.y;
-                    ddt = fmaf(dax * dA[i].x, an[i].x, fmaf(day * dA[i].y, an[i].y, ddt));
-                    ddt = fmaf(dwsx, dwx, fmaf(dwsy, dwy, ddt));
-                    dA_acc[i].x = fmaf(dax * dA[i].x, tk.dt, fmaf(dwsx, dAwx, dA_acc[i].x));
-                    dA_acc[i].y = fmaf(day * dA[i].y, tk.dt, fmaf(dwsy, dAwy, dA_acc[i].y));
-                    gh[i] = make_float2(gx * dA[i].x, gy * dA[i].y);
                 }
-                const float du_t = du_acc + __shfl_xor_sync(0xffffffffu, du_acc, 1) + dr * cc.D;
-                const float ds_t = (ddt + __shfl_xor_sync(0xffffffffu, ddt, 1)) * tk.dsp;
-                du_o[t] = du_t;
-                ds_o[t] = ds_t;
-                dD_acc = fmaf(dr, ut, dD_acc);
-                dbias_acc += ds_t;
-                red[t] = reduce_scatter_channels<M>(vals, lane, red_index, red_writer);
-            }
-            // per-token gradients: lane half h stores tokens [h*HV, h*HV + HV)
-            if (valid) {
-                const int64_t t0 = t_chunk + int64_t(g) * V + HV * half;
-                float o1[HV], o2[HV], o3[HV];
+                float red[HV], du_o[HV], ds_o[HV], dz_o[HV];
+                int red_index = 0;
+                bool red_writer = true;
 #pragma unroll
-                for (int k2 = 0; k2 < HV; ++k2) {
-                    o1[k2] = half ? du_o[HV + k2] : du_o[k2];
-                    o2[k2] = half ? ds_o[HV + k2] : ds_o[k2];
-                    if constexpr (kGate) o3[k2] = half ? dz_o[HV + k2] : dz_o[k2];
+                for (int tt = HV - 1; tt >= 0; --tt) {
+                    const int t = T0 + tt;
+                    const BwdTok& tk = tok[t];
+                    const float ut = uv[t];
+                    float4 rowv[P];
+                    row_of(t, rowv);
+                    // read-out and gate
+                    float dr = yv[t];
+                    if constexpr (kGate) {
+                        float racc = 0.f;
+#pragma unroll
+                        for (int i = 0; i < P; ++i)
+                            racc = fmaf(rowv[i].z, hs[tt][i].x, fmaf(rowv[i].w, hs[tt][i].y, racc));
+                        const float r = racc + __shfl_xor_sync(0xffffffffu, racc, 1) + cc.D * ut;
+                        const float zt = zv[t];
+                        const float sz = kFast ? rcp_approx(1.f + ex2_approx(-zt * kLog2e)) : 1.f / (1.f + expf(-zt));
+                        dz_o[tt] = yv[t] * r * (sz * fmaf(zt, 1.f - sz, 1.f));
+                        dr = yv[t] * (zt * sz);
+                    }
+                    float2 dA[P];
+                    transition<N, kFast, kGeo>(dA, tk.rdt, half, cc);
+                    float vals[M];
+                    float du_acc = 0.f, ddt = 0.f;
+#pragma unroll
+                    for (int i = 0; i < P; ++i) {
+                        const float2 hp = tt > 0 ? hs[tt > 0 ? tt - 1 : 0][i] : (T0 == 0 ? h0[i] : hmid[i]);
+                        const float Bx = rowv[i].x, By = rowv[i].y;
+                        const float gx = fmaf(dr, rowv[i].z, gh[i].x), gy = fmaf(dr, rowv[i].w, gh[i].y);
+                        vals[P * 2 + 2 * i] = dr * hs[tt][i].x;  // dC
+                        vals[P * 2 + 2 * i + 1] = dr * hs[tt][i].y;
+                        float wx = tk.dt, wy = tk.dt, dwx = 1.f, dwy = 1.f, dAwx = 0.f, dAwy = 0.f;
+                        if constexpr (kZoh) {
+                            // w = Delta phi(x), dw/dDelta = a, dw/dA = Delta^2 phi'(x)
+                            const float xx = tk.dt * an[i].x, xy = tk.dt * an[i].y;
+                            const bool sx = fabsf(xx) < kZohTaylorMax, sy = fabsf(xy) < kZohTaylorMax;
+                            wx = sx ? tk.dt * phi_taylor(xx) : (dA[i].x - 1.f) * cc.ia[i].x;
+                            wy = sy ? tk.dt * phi_taylor(xy) : (dA[i].y - 1.f) * cc.ia[i].y;
+                            dwx = dA[i].x;
+                            dwy = dA[i].y;
+                            dAwx = sx ? tk.dt * tk.dt * dphi_taylor(xx) : fmaf(tk.dt, dA[i].x, -wx) * cc.ia[i].x;
+                            dAwy = sy ? tk.dt * tk.dt * dphi_taylor(xy) : fmaf(tk.dt, dA[i].y, -wy) * cc.ia[i].y;
+                        }
+                        vals[2 * i] = gx * wx * ut;  // dB
+                        vals[2 * i + 1] = gy * wy * ut;
+                        du_acc = fmaf(gx * wx, Bx, fmaf(gy * wy, By, du_acc));
+                        const float dwsx = gx * Bx * ut, dwsy = gy * By * ut;
+                        const float dax = gx * hp.x * dA[i].x, day = gy * hp.y * dA[i].y;
+                        ddt = fmaf(dax, an[i].x, fmaf(day, an[i].y, ddt));
+                        ddt = fmaf(dwsx, dwx, fmaf(dwsy, dwy, ddt));
+                        dA_acc[i].x = fmaf(dax, tk.dt, fmaf(dwsx, dAwx, dA_acc[i].x));
+                        dA_acc[i].y = fmaf(day, tk.dt, fmaf(dwsy, dAwy, dA_acc[i].y));
+                        gh[i] = make_float2(gx * dA[i].x, gy * dA[i].y);
+                    }
+                    const float du_t = du_acc + __shfl_xor_sync(0xffffffffu, du_acc, 1) + dr * cc.D;
+                    const float ds_t = (ddt + __shfl_xor_sync(0xffffffffu, ddt, 1)) * tk.dsp;
+                    du_o[tt] = du_t;
+                    ds_o[tt] = ds_t;
+                    dD_acc = fmaf(dr, ut, dD_acc);
+                    dbias_acc += ds_t;
+                    red[tt] = reduce_scatter_channels<M>(vals, lane, red_index, red_writer);
                 }
-                *reinterpret_cast<uint2*>(static_cast<T*>(p.du) + row * L + t0) = pack8<T>(o1);
-                *reinterpret_cast<uint2*>(static_cast<T*>(p.ddelta) + row * L + t0) = pack8<T>(o2);
-                if constexpr (kGate) *reinterpret_cast<uint2*>(static_cast<T*>(p.dz) + row * L + t0) = pack8<T>(o3);
-            }
-            // dB / dC of the group's tokens for this lane's (state, B or C)
-            if (red_writer) {
-                const int q = red_index / (2 * P);  // 0: dB, 1: dC
-                const int i = red_index % (2 * P);
-                const int n = half + 4 * (i / 2) + 2 * (i % 2);
-                float* dst = (q ? p.dC : p.dB) + (size_t(b) * N + n) * size_t(L) + size_t(t_chunk + int64_t(g) * V);
-#pragma unroll
-                for (int k2 = 0; k2 < V; k2 += 4) red_add_v4(dst + k2, red[k2], red[k2 + 1], red[k2 + 2], red[k2 + 3]);
-            }
+                // this half's per-token gradients: stored by lane half T0 / HV
+                if (valid && half == T0 / HV) {
+                    const int64_t at = row * L + tg + T0;
+                    *reinterpret_cast<uint2*>(static_cast<T*>(p.du) + at) = pack8<T>(du_o);
+                    *reinterpret_cast<uint2*>(static_cast<T*>(p.ddelta) + at) = pack8<T>(ds_o);
+                    if constexpr (kGate) *reinterpret_cast<uint2*>(static_cast<T*>(p.dz) + at) = pack8<T>(dz_o);
+                }
+                // dB / dC of the half's tokens for this lane's (state, B or C)
+                if (red_writer) {
+                    const int q = red_index / (2 * P);  // 0: dB, 1: dC
+                    const int i = red_index % (2 * P);
+                    const int n = half + 4 * (i / 2) + 2 * (i % 2);
+                    float* dst = (q ? p.dC : p.dB) + (size_t(b) * N + n) * size_t(L) + size_t(tg + T0);
+                    if constexpr (HV == 4)
+                        red_add_v4(dst, red[0], red[1], red[2], red[3]);
+                    else
+                        red_add_v2(dst, red[0], red[1]);
+                }
+            };
+            run_half(std::integral_constant<int, HV>{});
+            run_half(std::integral_constant<int, 0>{});
         }
 
         // hand the stage to chunk k + S
