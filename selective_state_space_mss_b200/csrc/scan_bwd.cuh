@@ -58,7 +58,10 @@ struct BwdLayout {
     static constexpr int kPairs = F::kPairs;
     static constexpr int kTile = F::kTile;
     static constexpr int kBCTile = F::kBCTile;
-    static constexpr int kStages = 2;
+    // one stage: the next chunk's tiles are fetched while the chunk's first
+    // group is reversed, once every tile word has been read (B and C are read
+    // when the chunk starts); a second stage would cost a CTA per SM
+    static constexpr int kStages = 1;
     static constexpr int kStageBytes = 4 * kTile + 2 * kBCTile;  // u, delta, z, dy, B, C
     static constexpr int kBCfRow = F::kBCfRow;
     static constexpr int kBCfBytes = F::kBCfBytes;
@@ -78,7 +81,8 @@ struct BwdTok {
     float dsp;  // dDelta / ddelta_raw: sigmoid(s) with softplus, else 1
 };
 
-template <bool kFast, bool kGeo, bool kSoftplus, int N>
+// kDsp: also the softplus derivative (the recompute-only passes skip it).
+template <bool kFast, bool kGeo, bool kSoftplus, bool kDsp = true, int N>
 __device__ __forceinline__ BwdTok bwd_token(float ut, float dr, const LaneConst<N>& cc) {
     BwdTok tk;
     const float s = dr + cc.bias;
@@ -86,11 +90,23 @@ __device__ __forceinline__ BwdTok bwd_token(float ut, float dr, const LaneConst<
     tk.dsp = 1.f;
     if constexpr (kSoftplus) {
         tk.dt = kFast ? softplus_fast(s) : softplus_precise(s);
-        tk.dsp = kFast ? rcp_approx(1.f + ex2_approx(-s * kLog2e)) : 1.f / (1.f + expf(-s));
+        if constexpr (kDsp) tk.dsp = kFast ? rcp_approx(1.f + ex2_approx(-s * kLog2e)) : 1.f / (1.f + expf(-s));
     }
     tk.du = tk.dt * ut;
     tk.rdt = kGeo ? ex2_approx(tk.dt * cc.a0) : tk.dt;
     return tk;
+}
+
+// Token t of a 16-byte group held as its raw word (t a compile-time index).
+template <typename T>
+__device__ __forceinline__ float elem16(const uint4& w, int t) {
+    constexpr int per = 4 / int(sizeof(T));  // tokens per 32-bit word
+    const int k = t / per;
+    const uint32_t word = k == 0 ? w.x : k == 1 ? w.y : k == 2 ? w.z : w.w;
+    if constexpr (sizeof(T) == 2)
+        return (t & 1) ? bf16_hi(word) : bf16_lo(word);
+    else
+        return __uint_as_float(word);
 }
 
 // The 8 (bf16) or 4 (fp32) tokens of one 16-byte group.
@@ -209,10 +225,8 @@ __device__ __forceinline__ void scan_bwd_body(const BwdMaps& maps, const BwdPara
     };
     const float4* my_bcf = reinterpret_cast<const float4*>(bcf) + half * P;
     constexpr int kRowF4 = Ly::kBCfRow / 4;
-    // natural A of this lane's state pairs
-    float2 an[P];
-#pragma unroll
-    for (int i = 0; i < P; ++i) an[i] = kFast ? __fmul2_rn(cc.a2[i], make_float2(kLn2, kLn2)) : cc.a2[i];
+    // natural A of a state pair
+    auto a_nat = [&](int i) { return kFast ? __fmul2_rn(cc.a2[i], make_float2(kLn2, kLn2)) : cc.a2[i]; };
 
     // adjoint state, per-channel sums
     float2 gh[P], dA_acc[P];
@@ -254,7 +268,7 @@ __device__ __forceinline__ void scan_bwd_body(const BwdMaps& maps, const BwdPara
             const float4* base = my_bcf + (g * V) * kRowF4;
 #pragma unroll
             for (int t = 0; t < V; ++t) {
-                const BwdTok tk = bwd_token<kFast, kGeo, kSoftplus>(uv[t], dv[t], cc);
+                const BwdTok tk = bwd_token<kFast, kGeo, kSoftplus, false>(uv[t], dv[t], cc);
                 float4 rowv[P];
 #pragma unroll
                 for (int i = 0; i < P; ++i) rowv[i] = base[t * kRowF4 + i];
@@ -267,21 +281,36 @@ __device__ __forceinline__ void scan_bwd_body(const BwdMaps& maps, const BwdPara
         // (second half first), so that only HV recomputed states are live
 #pragma unroll 1
         for (int g = ng - 1; g >= 0; --g) {
-            float uv[V], zv[V], yv[V];
             BwdTok tok[V];
+            uint4 zw = make_uint4(0u, 0u, 0u, 0u), yw;
+            const uint4 uw = group_word(st, 0, g);
             {
-                float dv[V];
-                unpack16<T>(group_word(st, 0, g), uv);
+                float uv[V], dv[V];
+                unpack16<T>(uw, uv);
                 unpack16<T>(group_word(st, 1, g), dv);
+                if constexpr (kGate) zw = group_word(st, 2, g);
+                yw = valid ? group_word(st, 3, g) : make_uint4(0u, 0u, 0u, 0u);  // past the last channel: no gradient
+                if (g == 0) {
+                    // every tile word of the chunk has been read: fetch the next chunk
+                    __syncwarp();
+                    if (lane == 0 && k + S < n_chunks) {
+                        fence_proxy_async_smem();
+                        issue(k + S);
+                    }
+                }
 #pragma unroll
-                for (int t = 0; t < V; ++t) tok[t] = bwd_token<kFast, kGeo, kSoftplus>(uv[t], dv[t], cc);
-            }
-            if constexpr (kGate) unpack16<T>(group_word(st, 2, g), zv);
-            unpack16<T>(group_word(st, 3, g), yv);
-            if (!valid) {
-                // a lane past the last channel contributes nothing to the sums
-#pragma unroll
-                for (int t = 0; t < V; ++t) yv[t] = 0.f;
+                for (int k2 = 0; k2 < HV; ++k2) {
+                    // each lane of the pair computes half the tokens and swaps
+                    const float uk = half ? uv[HV + k2] : uv[k2], dk = half ? dv[HV + k2] : dv[k2];
+                    const BwdTok mine = bwd_token<kFast, kGeo, kSoftplus>(uk, dk, cc);
+                    BwdTok other;
+                    other.dt = __shfl_xor_sync(0xffffffffu, mine.dt, 1);
+                    other.du = 0.f;  // formed again from dt where it is used
+                    other.rdt = __shfl_xor_sync(0xffffffffu, mine.rdt, 1);
+                    other.dsp = __shfl_xor_sync(0xffffffffu, mine.dsp, 1);
+                    tok[k2] = half ? other : mine;
+                    tok[HV + k2] = half ? mine : other;
+                }
             }
             const float4* base = my_bcf + (g * V) * kRowF4;
             auto row_of = [&](int t, float4 (&rowv)[P]) {
@@ -295,7 +324,8 @@ __device__ __forceinline__ void scan_bwd_body(const BwdMaps& maps, const BwdPara
             for (int t = 0; t < HV; ++t) {
                 float4 rowv[P];
                 row_of(t, rowv);
-                token_states<N, kFast, kGeo, kZoh, false>(hmid, rowv, tok[t].du, tok[t].rdt, uv[t], half, cc);
+                const float ut = elem16<T>(uw, t);
+                token_states<N, kFast, kGeo, kZoh, false>(hmid, rowv, tok[t].dt * ut, tok[t].rdt, ut, half, cc);
             }
             const int64_t tg = t_chunk + int64_t(g) * V;
             auto run_half = [&](auto span) {
@@ -309,8 +339,9 @@ __device__ __forceinline__ void scan_bwd_body(const BwdMaps& maps, const BwdPara
                     for (int t = 0; t < HV; ++t) {
                         float4 rowv[P];
                         row_of(T0 + t, rowv);
-                        token_states<N, kFast, kGeo, kZoh, false>(hh, rowv, tok[T0 + t].du, tok[T0 + t].rdt,
-                                                                   uv[T0 + t], half, cc);
+                        const float ut = elem16<T>(uw, T0 + t);
+                        token_states<N, kFast, kGeo, kZoh, false>(hh, rowv, tok[T0 + t].dt * ut, tok[T0 + t].rdt,
+                                                                   elem16<T>(uw, T0 + t), half, cc);
 #pragma unroll
                         for (int i = 0; i < P; ++i) hs[t][i] = hh[i];
                     }
@@ -322,21 +353,21 @@ __device__ __forceinline__ void scan_bwd_body(const BwdMaps& maps, const BwdPara
                 for (int tt = HV - 1; tt >= 0; --tt) {
                     const int t = T0 + tt;
                     const BwdTok& tk = tok[t];
-                    const float ut = uv[t];
+                    const float ut = elem16<T>(uw, t);
                     float4 rowv[P];
                     row_of(t, rowv);
                     // read-out and gate
-                    float dr = yv[t];
+                    float dr = elem16<T>(yw, t);
                     if constexpr (kGate) {
                         float racc = 0.f;
 #pragma unroll
                         for (int i = 0; i < P; ++i)
                             racc = fmaf(rowv[i].z, hs[tt][i].x, fmaf(rowv[i].w, hs[tt][i].y, racc));
                         const float r = racc + __shfl_xor_sync(0xffffffffu, racc, 1) + cc.D * ut;
-                        const float zt = zv[t];
+                        const float zt = elem16<T>(zw, t);
                         const float sz = kFast ? rcp_approx(1.f + ex2_approx(-zt * kLog2e)) : 1.f / (1.f + expf(-zt));
-                        dz_o[tt] = yv[t] * r * (sz * fmaf(zt, 1.f - sz, 1.f));
-                        dr = yv[t] * (zt * sz);
+                        dz_o[tt] = elem16<T>(yw, t) * r * (sz * fmaf(zt, 1.f - sz, 1.f));
+                        dr = elem16<T>(yw, t) * (zt * sz);
                     }
                     float2 dA[P];
                     transition<N, kFast, kGeo>(dA, tk.rdt, half, cc);
@@ -352,7 +383,8 @@ __device__ __forceinline__ void scan_bwd_body(const BwdMaps& maps, const BwdPara
                         float wx = tk.dt, wy = tk.dt, dwx = 1.f, dwy = 1.f, dAwx = 0.f, dAwy = 0.f;
                         if constexpr (kZoh) {
                             // w = Delta phi(x), dw/dDelta = a, dw/dA = Delta^2 phi'(x)
-                            const float xx = tk.dt * an[i].x, xy = tk.dt * an[i].y;
+                            const float2 an = a_nat(i);
+                            const float xx = tk.dt * an.x, xy = tk.dt * an.y;
                             const bool sx = fabsf(xx) < kZohTaylorMax, sy = fabsf(xy) < kZohTaylorMax;
                             wx = sx ? tk.dt * phi_taylor(xx) : (dA[i].x - 1.f) * cc.ia[i].x;
                             wy = sy ? tk.dt * phi_taylor(xy) : (dA[i].y - 1.f) * cc.ia[i].y;
@@ -366,7 +398,8 @@ __device__ __forceinline__ void scan_bwd_body(const BwdMaps& maps, const BwdPara
                         du_acc = fmaf(gx * wx, Bx, fmaf(gy * wy, By, du_acc));
                         const float dwsx = gx * Bx * ut, dwsy = gy * By * ut;
                         const float dax = gx * hp.x * dA[i].x, day = gy * hp.y * dA[i].y;
-                        ddt = fmaf(dax, an[i].x, fmaf(day, an[i].y, ddt));
+                        const float2 ani = a_nat(i);
+                        ddt = fmaf(dax, ani.x, fmaf(day, ani.y, ddt));
                         ddt = fmaf(dwsx, dwx, fmaf(dwsy, dwy, ddt));
                         dA_acc[i].x = fmaf(dax, tk.dt, fmaf(dwsx, dAwx, dA_acc[i].x));
                         dA_acc[i].y = fmaf(day, tk.dt, fmaf(dwsy, dAwy, dA_acc[i].y));
@@ -403,12 +436,7 @@ __device__ __forceinline__ void scan_bwd_body(const BwdMaps& maps, const BwdPara
             run_half(std::integral_constant<int, 0>{});
         }
 
-        // hand the stage to chunk k + S
         __syncwarp();
-        if (lane == 0 && k + S < n_chunks) {
-            fence_proxy_async_smem();
-            issue(k + S);
-        }
     }
 
     if (!valid) return;
