@@ -74,6 +74,8 @@ def _load():
             lib.mss_oracle_scan_bwd.argtypes = [f, f, f, f, f, f, f, f, i, i, d, f, d,
                                                 d, d, d, d, d, d, d, d, d, i64, i64, i64, i64, i]
             lib.mss_oracle_scan_bwd.restype = i
+            lib.mss_oracle_ssd_fwd.argtypes = [f, f, f, f, f, f, f, f, i, d, d, d, i64, i64, i64, i64, i64, i64, i]
+            lib.mss_oracle_ssd_fwd.restype = i
             lib.mss_oracle_recurrence.argtypes = [d, d, d, i64, i64, d, d]
             lib.mss_oracle_recurrence.restype = i
             lib.mss_oracle_softplus.argtypes = [ctypes.c_double]
@@ -328,6 +330,39 @@ def state_update(state, u, delta, A, B, C, D=None, z=None, delta_bias=None,
         raise RuntimeError(f"mss_oracle_state_update failed with code {rc}")
     del u_a, d_a, A_a, B_a, C_a, D_a, z_a, b_a
     return y, state
+
+
+def ssd_fwd(x, dt, A, B, C, D=None, z=None, dt_bias=None, softplus_flag=True, initial_state=None,
+            nthreads=None):
+    """Structured state space duality (Mamba-2) forward pass in fp64: A is a
+    scalar per head.  x, z: [batch, L, H, P]; dt: [batch, L, H]; A, D,
+    dt_bias: [H]; B, C: [batch, L, G, N] (head h reads group h // (H // G));
+    initial_state: [batch, H, N, P].  Returns (y [batch, L, H, P],
+    last_state [batch, H, N, P])."""
+    x_a, x_p = _f32(x, name="x")
+    if x_a.ndim != 4:
+        raise ValueError("x must be [batch, L, H, P]")
+    batch, L, H, P = x_a.shape
+    B_a, B_p = _f32(B, name="B")
+    if B_a.ndim != 4 or B_a.shape[:2] != (batch, L):
+        raise ValueError("B must be [batch, L, G, N]")
+    G, N = B_a.shape[2], B_a.shape[3]
+    dt_a, dt_p = _f32(dt, (batch, L, H), "dt")
+    A_a, A_p = _f32(A, (H,), "A")
+    C_a, C_p = _f32(C, (batch, L, G, N), "C")
+    D_a, D_p = _f32(D, (H,), "D")
+    z_a, z_p = _f32(z, (batch, L, H, P), "z")
+    b_a, b_p = _f32(dt_bias, (H,), "dt_bias")
+    h0 = _f64_opt(initial_state, (batch, H, N, P), "initial_state")
+    y = np.empty((batch, L, H, P), dtype=np.float64)
+    last = np.empty((batch, H, N, P), dtype=np.float64)
+    rc = _load().mss_oracle_ssd_fwd(x_p, dt_p, A_p, B_p, C_p, D_p, z_p, b_p, int(bool(softplus_flag)),
+                                    None if h0 is None else _dptr(h0), _dptr(y), _dptr(last),
+                                    batch, L, H, P, G, N, default_threads() if nthreads is None else int(nthreads))
+    if rc != 0:
+        raise RuntimeError(f"mss_oracle_ssd_fwd failed with code {rc}")
+    del x_a, dt_a, A_a, B_a, C_a, D_a, z_a, b_a
+    return y, last
 
 
 def recurrence(abar, bbar_x, c):

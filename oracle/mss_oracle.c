@@ -725,3 +725,118 @@ int mss_oracle_scan_bwd(const float *u, const float *delta, const float *A, cons
     free(jobs); free(tids); free(sums);
     return rc;
 }
+
+/* ------------------------------------------------------------------------ */
+/* Structured state space duality (Mamba-2): scalar-times-identity A.        */
+/*
+ * "NN Lab: Mamba" (Structured State Space Duality) and the "Mamba" paper
+ * review (section "Mamba 2"): A is restricted to a scalar times the identity
+ * per head, which makes the sequence map a 1-semiseparable matrix
+ * M_ji = a_{j:i} (C_j . B_i) and lets heads of P channels share B and C.
+ * The oracle is the recurrence itself, per (batch, head), with an N x P state:
+ *
+ *   Delta_t = softplus(dt_t + bias_h),  a_t = exp(Delta_t A_h),
+ *   S_t[n][p] = a_t S_{t-1}[n][p] + Delta_t B_t[n] x_t[p],
+ *   y_t[p] = sum_n C_t[n] S_t[n][p] + D_h x_t[p],  times silu(z_t[p]).
+ *
+ * Layouts (token-major, as the heads of a token are contiguous):
+ *   x, z, y : [batch][L][H][P];  dt: [batch][L][H];  A, D, bias: [H];
+ *   B, C    : [batch][L][G][N], head h reads group h / (H / G);
+ *   initial_state, last_state: [batch][H][N][P] (fp64).
+ */
+
+typedef struct {
+    const float *x, *dt, *A, *B, *C, *D, *z, *bias;
+    const double *initial_state;
+    int softplus_flag;
+    double *y, *last_state;
+    int64_t batch, L, H, P, G, N;
+    int64_t row_begin, row_end; /* rows = (batch, head) pairs */
+    int status;
+} ssd_job;
+
+static void *ssd_rows(void *arg)
+{
+    ssd_job *j = (ssd_job *)arg;
+    const int64_t L = j->L, H = j->H, P = j->P, G = j->G, N = j->N;
+    double *S = (double *)malloc((size_t)(N * P) * sizeof(double));
+    if (!S) {
+        j->status = ORACLE_ENOMEM;
+        return NULL;
+    }
+    for (int64_t row = j->row_begin; row < j->row_end; ++row) {
+        const int64_t b = row / H, h = row % H, g = h / (H / G);
+        const double Ah = (double)j->A[h];
+        const double bias = j->bias ? (double)j->bias[h] : 0.0;
+        const double Dh = j->D ? (double)j->D[h] : 0.0;
+        for (int64_t k = 0; k < N * P; ++k)
+            S[k] = j->initial_state ? j->initial_state[row * N * P + k] : 0.0;
+        for (int64_t t = 0; t < L; ++t) {
+            const double s = (double)j->dt[(b * L + t) * H + h] + bias;
+            const double delta = j->softplus_flag ? mss_oracle_softplus(s) : s;
+            const double a = exp(delta * Ah);
+            const float *Bt = j->B + ((b * L + t) * G + g) * N;
+            const float *Ct = j->C + ((b * L + t) * G + g) * N;
+            const float *xt = j->x + ((b * L + t) * H + h) * P;
+            for (int64_t p = 0; p < P; ++p) {
+                double acc = 0.0;
+                for (int64_t n = 0; n < N; ++n) {
+                    S[n * P + p] = a * S[n * P + p] + delta * (double)Bt[n] * (double)xt[p];
+                    acc += (double)Ct[n] * S[n * P + p];
+                }
+                double out = acc + Dh * (double)xt[p];
+                if (j->z)
+                    out *= mss_oracle_silu((double)j->z[((b * L + t) * H + h) * P + p]);
+                j->y[((b * L + t) * H + h) * P + p] = out;
+            }
+        }
+        if (j->last_state)
+            for (int64_t k = 0; k < N * P; ++k)
+                j->last_state[row * N * P + k] = S[k];
+    }
+    free(S);
+    j->status = ORACLE_OK;
+    return NULL;
+}
+
+int mss_oracle_ssd_fwd(const float *x, const float *dt, const float *A, const float *B, const float *C,
+                       const float *D, const float *z, const float *dt_bias, int softplus_flag,
+                       const double *initial_state, double *y, double *last_state,
+                       int64_t batch, int64_t L, int64_t H, int64_t P, int64_t G, int64_t N, int nthreads)
+{
+    if (!x || !dt || !A || !B || !C || !y || batch < 0 || L < 0 || H <= 0 || P <= 0 || G <= 0 || N <= 0 ||
+        H % G != 0)
+        return ORACLE_EINVAL;
+    const int64_t rows = batch * H;
+    if (rows == 0)
+        return ORACLE_OK;
+    if (nthreads < 1)
+        nthreads = 1;
+    if ((int64_t)nthreads > rows)
+        nthreads = (int)rows;
+    ssd_job *jobs = (ssd_job *)calloc((size_t)nthreads, sizeof(ssd_job));
+    pthread_t *tids = (pthread_t *)calloc((size_t)nthreads, sizeof(pthread_t));
+    if (!jobs || !tids) {
+        free(jobs);
+        free(tids);
+        return ORACLE_ENOMEM;
+    }
+    for (int i = 0; i < nthreads; ++i) {
+        jobs[i] = (ssd_job){x, dt, A, B, C, D, z, dt_bias, initial_state, softplus_flag, y, last_state,
+                            batch, L, H, P, G, N, rows * i / nthreads, rows * (i + 1) / nthreads, ORACLE_EINVAL};
+        if (nthreads == 1 || pthread_create(&tids[i], NULL, ssd_rows, &jobs[i]) != 0) {
+            ssd_rows(&jobs[i]);
+            tids[i] = 0;
+        }
+    }
+    int rc = ORACLE_OK;
+    for (int i = 0; i < nthreads; ++i) {
+        if (tids[i])
+            pthread_join(tids[i], NULL);
+        if (jobs[i].status != ORACLE_OK)
+            rc = jobs[i].status;
+    }
+    free(jobs);
+    free(tids);
+    return rc;
+}

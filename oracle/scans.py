@@ -147,3 +147,47 @@ def sss_matrix(abar, bbar, c):
                 decay = decay * abar[k]
             M[j, i] = np.sum(c[j] * decay * bbar[i])
     return M
+
+
+# --------------------------------------------------------------------------
+# Structured state space duality (scalar A per head): the matrix view and the
+# chunked algorithm ("NN Lab -- Mamba", Structured State Space Duality;
+# "Mamba" paper review, section "Mamba 2").  One head, fp64, numpy.
+
+def ssd_matrix(a, delta, B, C):
+    """The 1-semiseparable matrix of one head: M[j, i] = a_{i+1} ... a_j
+    (C_j . B_i) delta_i for i <= j, else 0.  a, delta: [L]; B, C: [L, N]."""
+    L = len(a)
+    M = np.zeros((L, L))
+    for j in range(L):
+        prod = 1.0
+        for i in range(j, -1, -1):
+            M[j, i] = prod * float(C[j] @ B[i]) * delta[i]
+            prod *= a[i]
+    return M
+
+
+def ssd_chunked(a, delta, B, C, X, chunk, S0=None):
+    """The chunked form: within each chunk the quadratic (attention-like)
+    product of the masked M block with X; across chunks the state
+    S = (decay of the chunk) S + (the chunk's contribution), carried forward.
+    a, delta: [L]; B, C: [L, N]; X: [L, P]; S0: [N, P].  Returns (Y [L, P], S)."""
+    L, P = X.shape
+    N = B.shape[1]
+    S = np.zeros((N, P)) if S0 is None else np.array(S0, dtype=np.float64)
+    Y = np.zeros((L, P))
+    for c0 in range(0, L, chunk):
+        c1 = min(c0 + chunk, L)
+        ac, dc, Bc, Cc, Xc = a[c0:c1], delta[c0:c1], B[c0:c1], C[c0:c1], X[c0:c1]
+        q = c1 - c0
+        # cumulative decay from the chunk start: cum[t] = a_{c0} ... a_{c0+t}
+        cum = np.cumprod(ac)
+        # intra-chunk: masked quadratic form
+        Mc = ssd_matrix(ac, dc, Bc, Cc)
+        Y[c0:c1] = Mc @ Xc
+        # inter-chunk: the incoming state seen through the decay so far
+        Y[c0:c1] += (Cc * cum[:, None]) @ S
+        # the chunk's contribution to the state at its end
+        tail = np.array([np.prod(ac[t + 1:]) for t in range(q)])
+        S = cum[-1] * S + (Bc * (dc * tail)[:, None]).T @ Xc
+    return Y, S

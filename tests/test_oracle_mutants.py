@@ -55,6 +55,10 @@ MUTANTS = {
                               "j->dC[(b * N + n) * L + t] += dr * h[t * N + n];"),
     "bwd_zoh_dA_sign": ("(dt * atn - wtn) / An", "(dt * atn + wtn) / An"),
     "bwd_gate_derivative": ("(sg + zt * sg * (1.0 - sg))", "(sg + zt * sg * sg)"),
+    "ssd_group_index": ("g = h / (H / G);", "g = h % G;"),
+    "ssd_no_decay": ("S[n * P + p] = a * S[n * P + p] + delta", "S[n * P + p] = S[n * P + p] + delta"),
+    "ssd_input_without_step": ("+ delta * (double)Bt[n] * (double)xt[p];", "+ (double)Bt[n] * (double)xt[p];"),
+    "ssd_state_layout": ("acc += (double)Ct[n] * S[n * P + p];", "acc += (double)Ct[n] * S[p * N + n];"),
 }
 
 
@@ -62,7 +66,7 @@ def _run_pins(lib_path):
     env = dict(os.environ, MSS_ORACLE_LIB=lib_path)
     return subprocess.run(
         [sys.executable, "-m", "pytest", "-q", "-x", "-p", "no:cacheprovider",
-         os.path.join(ROOT, "tests", "test_oracle_pins.py")],
+         os.path.join(ROOT, "tests", "test_oracle_pins.py"), os.path.join(ROOT, "tests", "test_oracle_ssd.py")],
         cwd=ROOT, env=env, capture_output=True, text=True, timeout=600)
 
 
