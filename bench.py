@@ -235,6 +235,18 @@ def calibrate_rows(inp, nthreads, target_s):
     return int(min(inp["dim"], max(nthreads, target_s / max(per_row, 1e-9))))
 
 
+def cpu_model():
+    """The host CPU's model name (Linux), for the baseline's record."""
+    try:
+        with open("/proc/cpuinfo") as f:
+            for line in f:
+                if line.startswith("model name"):
+                    return line.split(":", 1)[1].strip()
+    except OSError:
+        pass
+    return "unknown"
+
+
 def cpu_baseline(inp, target_s=10.0):
     """The oracle on the host cores over the same workload, repeated until
     about target_s seconds of work."""
@@ -246,7 +258,7 @@ def cpu_baseline(inp, target_s=10.0):
     while total_s < target_s or passes == 0:
         ct, sec = oracle_sample_rate(inp, rows, nthreads)
         total_ct, total_s, passes = total_ct + ct, total_s + sec, passes + 1
-    return {"value": total_ct / total_s, "unit": UNIT, "cores": nthreads, "kind": "oracle",
+    return {"value": total_ct / total_s, "unit": UNIT, "cores": nthreads, "kind": "oracle", "cpu": cpu_model(),
             "sample": f"{passes} pass(es) of {inp['batch']}x{rows} channels x {inp['seqlen']} tokens "
                       f"of {WORKLOAD} (fp64, {nthreads} threads, {total_s:.1f} s)"}
 
@@ -469,6 +481,31 @@ def run_mss(args, rank, world, local_rank):
             dec_ms.append(a_.elapsed_time(b_))
     dec_med = statistics.median(dec_ms)
     dec_bytes = decode_bytes(dw.batch, dw.dim, dw.dstate)
+    # the same tokens back to back from a CUDA graph (16 tokens per replay, no
+    # flush: the state stays partly in L2 between tokens, as when serving)
+    graph_tokens = 16
+    side = torch.cuda.Stream(dev)
+    side.wait_stream(stream)
+    with torch.cuda.stream(side):
+        for t in range(graph_tokens):  # the first calls run outside the capture
+            mss.state_update(st5, A=A5, D=D5, delta_bias=b5, y=y5, **steps5[t % 4])
+    stream.wait_stream(side)
+    graph = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(graph, stream=side):
+        for t in range(graph_tokens):
+            mss.state_update(st5, A=A5, D=D5, delta_bias=b5, y=y5, **steps5[t % 4])
+    for _ in range(3):
+        graph.replay()
+    torch.cuda.synchronize(dev)
+    g0, g1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    g0.record(stream)
+    for _ in range(10):
+        graph.replay()
+    g1.record(stream)
+    torch.cuda.synchronize(dev)
+    dec_graph_ms = g0.elapsed_time(g1) / (10 * graph_tokens)
+    del graph
+    assert mss.get_device_error() == 0
 
     peak, peak_kind, sm_max_mhz = measured_peaks()
     alu_ops = fwd_alu_ops(w.batch, w.dim, w.dstate, w.seqlen)
@@ -507,7 +544,9 @@ def run_mss(args, rank, world, local_rank):
                      "kernel": "scan_fwd_seq (forward scan)",
                      "peak_kind": f"derived: {SMS} SMs x {FP32_LANES_PER_SM} fp32 lanes x {sm_max_mhz:.0f} MHz",
                      "algorithmic_ops_per_launch": alu_ops, "algorithmic_bytes_per_launch": bytes_fwd,
-                     "launch_ms_avg": fwd_avg},
+                     "launch_ms_avg": fwd_avg,
+                     "launch_ms_p10_p50_p90": [float(np.percentile(fwd_ms, q)) for q in (10, 50, 90)],
+                     "state_updates_per_s": w.batch * w.dim * w.seqlen * w.dstate / (fwd_avg * 1e-3)},
         "roofline_hbm": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
                          "frac": achieved / peak, "traffic": recorded_traffic(),
                          "peak_kind": peak_kind, "algorithmic_bytes_per_launch": bytes_fwd},
@@ -529,7 +568,9 @@ def run_mss(args, rank, world, local_rank):
         "decode": {"workload": gen.DECODE_WORKLOAD, "ms_per_token_median": dec_med,
                    "achieved_gbs": dec_bytes / (dec_med * 1e-3) / 1e9,
                    "frac": dec_bytes / (dec_med * 1e-3) / 1e9 / peak,
-                   "l2": "flushed before each token (512 MB written, then 256 MB of another buffer read)"},
+                   "l2": "flushed before each token (512 MB written, then 256 MB of another buffer read)",
+                   "graph_ms_per_token": dec_graph_ms,
+                   "graph_note": f"{graph_tokens} tokens per CUDA graph replay, back to back, no flush"},
         "e2e": {"value": whole_job_rate(ct_per_step, world, args.steps, e2e_ms), "unit": UNIT,
                 "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
         "gpu_launches": launches_per_step * args.steps,

@@ -123,6 +123,17 @@ __device__ __forceinline__ void unpack16(const uint4& w, float (&v)[16 / sizeof(
     }
 }
 
+// Token t of a 16-byte group, t known only at run time (selects, no local memory).
+template <typename T>
+__device__ __forceinline__ float elem16rt(const uint4& w, int t) {
+    float v[16 / sizeof(T)];
+    unpack16<T>(w, v);
+    float r = v[0];
+#pragma unroll
+    for (int i = 1; i < int(16 / sizeof(T)); ++i) r = t == i ? v[i] : r;
+    return r;
+}
+
 // Sum of the M = 4 * (N/4) values v over the 16 channels of the warp (lane
 // bits 1..4), scattered: the lane keeps one sum; returns it.  `index` is the
 // value it holds, `writer` whether this lane is the one of its group that
@@ -281,67 +292,80 @@ __device__ __forceinline__ void scan_bwd_body(const BwdMaps& maps, const BwdPara
         // (second half first), so that only HV recomputed states are live
 #pragma unroll 1
         for (int g = ng - 1; g >= 0; --g) {
-            BwdTok tok[V];
             uint4 zw = make_uint4(0u, 0u, 0u, 0u), yw;
             const uint4 uw = group_word(st, 0, g);
-            {
-                float uv[V], dv[V];
-                unpack16<T>(uw, uv);
-                unpack16<T>(group_word(st, 1, g), dv);
-                if constexpr (kGate) zw = group_word(st, 2, g);
-                yw = valid ? group_word(st, 3, g) : make_uint4(0u, 0u, 0u, 0u);  // past the last channel: no gradient
-                if (g == 0) {
-                    // every tile word of the chunk has been read: fetch the next chunk
-                    __syncwarp();
-                    if (lane == 0 && k + S < n_chunks) {
-                        fence_proxy_async_smem();
-                        issue(k + S);
-                    }
+            const uint4 dw = group_word(st, 1, g);
+            if constexpr (kGate) zw = group_word(st, 2, g);
+            yw = valid ? group_word(st, 3, g) : make_uint4(0u, 0u, 0u, 0u);  // past the last channel: no gradient
+            if (g == 0) {
+                // every tile word of the chunk has been read: fetch the next chunk
+                __syncwarp();
+                if (lane == 0 && k + S < n_chunks) {
+                    fence_proxy_async_smem();
+                    issue(k + S);
                 }
+            }
+            // scalars of the HV tokens from `first` on: each lane of the pair
+            // computes half of them and they swap
+            auto half_tokens = [&](int first, BwdTok (&th)[HV]) {
 #pragma unroll
-                for (int k2 = 0; k2 < HV; ++k2) {
-                    // each lane of the pair computes half the tokens and swaps
-                    const float uk = half ? uv[HV + k2] : uv[k2], dk = half ? dv[HV + k2] : dv[k2];
-                    const BwdTok mine = bwd_token<kFast, kGeo, kSoftplus>(uk, dk, cc);
+                for (int k2 = 0; k2 < HV / 2; ++k2) {
+                    const int tm = first + (half ? HV / 2 : 0) + k2;
+                    const BwdTok mine = bwd_token<kFast, kGeo, kSoftplus>(elem16rt<T>(uw, tm), elem16rt<T>(dw, tm), cc);
                     BwdTok other;
                     other.dt = __shfl_xor_sync(0xffffffffu, mine.dt, 1);
                     other.du = 0.f;  // formed again from dt where it is used
                     other.rdt = __shfl_xor_sync(0xffffffffu, mine.rdt, 1);
                     other.dsp = __shfl_xor_sync(0xffffffffu, mine.dsp, 1);
-                    tok[k2] = half ? other : mine;
-                    tok[HV + k2] = half ? mine : other;
+                    th[k2] = half ? other : mine;
+                    th[HV / 2 + k2] = half ? mine : other;
                 }
-            }
-            const float4* base = my_bcf + (g * V) * kRowF4;
-            auto row_of = [&](int t, float4 (&rowv)[P]) {
-#pragma unroll
-                for (int i = 0; i < P; ++i) rowv[i] = base[t * kRowF4 + i];
             };
+            const float4* base = my_bcf + (g * V) * kRowF4;
             float2 h0[P], hmid[P];
 #pragma unroll
             for (int i = 0; i < P; ++i) h0[i] = hmid[i] = gs[(g * 32 + lane) * P + i];
+            {
+                BwdTok th[HV];
+                half_tokens(0, th);
 #pragma unroll
-            for (int t = 0; t < HV; ++t) {
-                float4 rowv[P];
-                row_of(t, rowv);
-                const float ut = elem16<T>(uw, t);
-                token_states<N, kFast, kGeo, kZoh, false>(hmid, rowv, tok[t].dt * ut, tok[t].rdt, ut, half, cc);
+                for (int t = 0; t < HV; ++t) {
+                    float4 rowv[P];
+#pragma unroll
+                    for (int i = 0; i < P; ++i) rowv[i] = base[t * kRowF4 + i];
+                    const float ut = elem16<T>(uw, t);
+                    token_states<N, kFast, kGeo, kZoh, false>(hmid, rowv, th[t].dt * ut, th[t].rdt, ut, half, cc);
+                }
             }
             const int64_t tg = t_chunk + int64_t(g) * V;
-            auto run_half = [&](auto span) {
-                constexpr int T0 = decltype(span)::value;  // first token of this half
+            // the second half, then the first: one copy of the code
+#pragma unroll 1
+            for (int hf = 1; hf >= 0; --hf) {
+                const int T0 = hf * HV;
+                BwdTok th[HV];
+                half_tokens(T0, th);
+                float uh[HV], zh[HV], yh[HV];
+#pragma unroll
+                for (int k2 = 0; k2 < HV; ++k2) {
+                    uh[k2] = hf ? elem16<T>(uw, HV + k2) : elem16<T>(uw, k2);
+                    yh[k2] = hf ? elem16<T>(yw, HV + k2) : elem16<T>(yw, k2);
+                    if constexpr (kGate) zh[k2] = hf ? elem16<T>(zw, HV + k2) : elem16<T>(zw, k2);
+                }
+                const float4* hbase = base + T0 * kRowF4;
+                float2 hst[P];
+#pragma unroll
+                for (int i = 0; i < P; ++i) hst[i] = hf ? hmid[i] : h0[i];
                 float2 hs[HV][P];
                 {
                     float2 hh[P];
 #pragma unroll
-                    for (int i = 0; i < P; ++i) hh[i] = T0 == 0 ? h0[i] : hmid[i];
+                    for (int i = 0; i < P; ++i) hh[i] = hst[i];
 #pragma unroll
                     for (int t = 0; t < HV; ++t) {
                         float4 rowv[P];
-                        row_of(T0 + t, rowv);
-                        const float ut = elem16<T>(uw, T0 + t);
-                        token_states<N, kFast, kGeo, kZoh, false>(hh, rowv, tok[T0 + t].dt * ut, tok[T0 + t].rdt,
-                                                                   elem16<T>(uw, T0 + t), half, cc);
+#pragma unroll
+                        for (int i = 0; i < P; ++i) rowv[i] = hbase[t * kRowF4 + i];
+                        token_states<N, kFast, kGeo, kZoh, false>(hh, rowv, th[t].dt * uh[t], th[t].rdt, uh[t], half, cc);
 #pragma unroll
                         for (int i = 0; i < P; ++i) hs[t][i] = hh[i];
                     }
@@ -351,23 +375,23 @@ __device__ __forceinline__ void scan_bwd_body(const BwdMaps& maps, const BwdPara
                 bool red_writer = true;
 #pragma unroll
                 for (int tt = HV - 1; tt >= 0; --tt) {
-                    const int t = T0 + tt;
-                    const BwdTok& tk = tok[t];
-                    const float ut = elem16<T>(uw, t);
+                    const BwdTok& tk = th[tt];
+                    const float ut = uh[tt];
                     float4 rowv[P];
-                    row_of(t, rowv);
+#pragma unroll
+                    for (int i = 0; i < P; ++i) rowv[i] = hbase[tt * kRowF4 + i];
                     // read-out and gate
-                    float dr = elem16<T>(yw, t);
+                    float dr = yh[tt];
                     if constexpr (kGate) {
                         float racc = 0.f;
 #pragma unroll
                         for (int i = 0; i < P; ++i)
                             racc = fmaf(rowv[i].z, hs[tt][i].x, fmaf(rowv[i].w, hs[tt][i].y, racc));
                         const float r = racc + __shfl_xor_sync(0xffffffffu, racc, 1) + cc.D * ut;
-                        const float zt = elem16<T>(zw, t);
+                        const float zt = zh[tt];
                         const float sz = kFast ? rcp_approx(1.f + ex2_approx(-zt * kLog2e)) : 1.f / (1.f + expf(-zt));
-                        dz_o[tt] = elem16<T>(yw, t) * r * (sz * fmaf(zt, 1.f - sz, 1.f));
-                        dr = elem16<T>(yw, t) * (zt * sz);
+                        dz_o[tt] = yh[tt] * r * (sz * fmaf(zt, 1.f - sz, 1.f));
+                        dr = yh[tt] * (zt * sz);
                     }
                     float2 dA[P];
                     transition<N, kFast, kGeo>(dA, tk.rdt, half, cc);
@@ -375,7 +399,7 @@ __device__ __forceinline__ void scan_bwd_body(const BwdMaps& maps, const BwdPara
                     float du_acc = 0.f, ddt = 0.f;
 #pragma unroll
                     for (int i = 0; i < P; ++i) {
-                        const float2 hp = tt > 0 ? hs[tt > 0 ? tt - 1 : 0][i] : (T0 == 0 ? h0[i] : hmid[i]);
+                        const float2 hp = tt > 0 ? hs[tt > 0 ? tt - 1 : 0][i] : hst[i];
                         const float Bx = rowv[i].x, By = rowv[i].y;
                         const float gx = fmaf(dr, rowv[i].z, gh[i].x), gy = fmaf(dr, rowv[i].w, gh[i].y);
                         vals[P * 2 + 2 * i] = dr * hs[tt][i].x;  // dC
@@ -413,8 +437,8 @@ __device__ __forceinline__ void scan_bwd_body(const BwdMaps& maps, const BwdPara
                     dbias_acc += ds_t;
                     red[tt] = reduce_scatter_channels<M>(vals, lane, red_index, red_writer);
                 }
-                // this half's per-token gradients: stored by lane half T0 / HV
-                if (valid && half == T0 / HV) {
+                // this half's per-token gradients: stored by lane half hf
+                if (valid && half == hf) {
                     const int64_t at = row * L + tg + T0;
                     *reinterpret_cast<uint2*>(static_cast<T*>(p.du) + at) = pack8<T>(du_o);
                     *reinterpret_cast<uint2*>(static_cast<T*>(p.ddelta) + at) = pack8<T>(ds_o);
@@ -431,9 +455,7 @@ __device__ __forceinline__ void scan_bwd_body(const BwdMaps& maps, const BwdPara
                     else
                         red_add_v2(dst, red[0], red[1]);
                 }
-            };
-            run_half(std::integral_constant<int, HV>{});
-            run_half(std::integral_constant<int, 0>{});
+            }
         }
 
         __syncwarp();
