@@ -56,7 +56,7 @@
 extern "C" {
 #endif
 
-#define MSS_VERSION 10300 /* major*10000 + minor*100 + patch: 1.3.0 */
+#define MSS_VERSION 10400 /* major*10000 + minor*100 + patch: 1.4.0 */
 
 enum mss_dtype {
     MSS_DTYPE_F32 = 0,
@@ -286,6 +286,38 @@ MSS_API int mss_scan_bwd(const void *u, const void *delta, const float *A, const
  * arguments; 0 when there is nothing to do. */
 MSS_API int64_t mss_scan_bwd_workspace_size(int64_t batch, int64_t dim, int64_t dstate, int64_t seqlen,
                                     int dtype, unsigned flags);
+
+/*
+ * mss_ssd_fwd -- forward pass of the structured state space duality layer
+ * (Mamba-2): A is a scalar per head, each head carries an N x P state, and
+ * the heads of a group share B and C ("NN Lab -- Mamba", Structured State
+ * Space Duality; "Mamba" paper review, section "Mamba 2").  Per (batch, head):
+ *
+ *   Delta_t = softplus(dt_t + dt_bias_h) (or dt_t + dt_bias_h),
+ *   S_t = exp(Delta_t A_h) S_{t-1} + Delta_t B_t x_t^T,
+ *   y_t = S_t^T C_t + D_h x_t, times silu(z_t) when z is given,
+ *
+ * computed chunk by chunk (64 tokens) with tensor-core matrix products: the
+ * masked quadratic form within a chunk plus the state carried across.
+ *
+ *   x, z, y  : [batch][seqlen][nheads][headdim]  bf16 (z may be NULL)
+ *   dt       : [batch][seqlen][nheads]           bf16
+ *   A, D, dt_bias : [nheads] float (D and dt_bias may be NULL)
+ *   B, C     : [batch][seqlen][ngroups][dstate]   bf16; head h reads group
+ *              h / (nheads / ngroups)
+ *   initial_state, last_state : [batch][nheads][dstate][headdim] float
+ *              (NULL: zero / not written)
+ *
+ * Supported: dtype MSS_DTYPE_BF16 (else MSS_ERR_DTYPE); headdim 64, dstate
+ * 64 or 128, nheads a multiple of ngroups (else MSS_ERR_SHAPE); x, B, C, y,
+ * z 16-byte aligned (else MSS_ERR_ALIGN).  Outputs must not overlap inputs.
+ * The intermediate products round to bf16 (the masked score matrix, the
+ * state as read by the next chunk), as tensor-core operands do.
+ */
+MSS_API int mss_ssd_fwd(const void *x, const void *dt, const float *A, const void *B, const void *C,
+                const float *D, const void *z, const float *dt_bias, int softplus_flag,
+                const float *initial_state, void *y, float *last_state, int64_t batch, int64_t seqlen,
+                int64_t nheads, int64_t headdim, int64_t ngroups, int64_t dstate, int dtype, void *stream);
 
 /*
  * mss_state_update -- one decode token for every (batch, channel):

@@ -22,7 +22,7 @@ import threading
 
 import torch
 
-__all__ = ["scan_fwd", "scan_fwd_conv", "scan_bwd", "bwd_workspace_size", "state_update", "state_update_conv",
+__all__ = ["scan_fwd", "scan_fwd_conv", "scan_bwd", "ssd_fwd", "bwd_workspace_size", "state_update", "state_update_conv",
            "get_device_error",
            "library_path", "workspace_size",
            "FLAG_GENERAL_A", "FLAG_SIMPLE", "FLAG_NO_SPLIT", "FLAG_ZOH_INPUT", "MssError", "load_library"]
@@ -85,6 +85,9 @@ def load_library():
             lib.mss_scan_bwd.restype = i
             lib.mss_scan_bwd_workspace_size.argtypes = [i64, i64, i64, i64, i, u32]
             lib.mss_scan_bwd_workspace_size.restype = i64
+            lib.mss_ssd_fwd.argtypes = [vp, vp, fp, vp, vp, fp, vp, fp, i, fp, vp, fp,
+                                        i64, i64, i64, i64, i64, i64, i, vp]
+            lib.mss_ssd_fwd.restype = i
             lib.mss_scan_fwd_conv.argtypes = [vp, fp, fp, i, vp, vp, vp, fp, vp, vp, fp, vp, fp, i, fp, vp, fp,
                                               i64, i64, i64, i64, i, u32, vp, i64, vp]
             lib.mss_scan_fwd_conv.restype = i
@@ -262,6 +265,41 @@ def scan_fwd_conv(x, conv_w, delta, A, B, C, conv_b=None, conv_state=None, D=Non
     if rc != 0:
         raise MssError(rc, "mss_scan_fwd_conv")
     return y, last_state, conv_state_out
+
+
+def ssd_fwd(x, dt, A, B, C, D=None, z=None, dt_bias=None, softplus=True, initial_state=None, y=None,
+            last_state=None, want_last_state=True, stream=None):
+    """Structured-state-space-duality forward pass (mss_ssd_fwd).  x, z:
+    [batch, L, H, P] bf16; dt: [batch, L, H] bf16; A, D, dt_bias: [H]
+    float32; B, C: [batch, L, G, N] bf16; initial_state: [batch, H, N, P]
+    float32.  Returns (y, last_state)."""
+    if not isinstance(x, torch.Tensor) or x.device.type != "cuda":
+        raise ValueError("x must be a CUDA tensor (there is no CPU path)")
+    if x.dim() != 4 or B.dim() != 4:
+        raise ValueError("x must be [batch, L, H, P] and B [batch, L, G, N]")
+    batch, L, H, P = x.shape
+    G, N = B.shape[2], B.shape[3]
+    dev, dt_ = x.device, x.dtype
+    code = _io_dtype(x)
+    for t, name, shape, typ, opt in ((x, "x", (batch, L, H, P), dt_, False), (dt, "dt", (batch, L, H), dt_, False),
+                                     (A, "A", (H,), torch.float32, False), (B, "B", (batch, L, G, N), dt_, False),
+                                     (C, "C", (batch, L, G, N), dt_, False), (D, "D", (H,), torch.float32, True),
+                                     (z, "z", (batch, L, H, P), dt_, True),
+                                     (dt_bias, "dt_bias", (H,), torch.float32, True),
+                                     (initial_state, "initial_state", (batch, H, N, P), torch.float32, True)):
+        _check(t, name, shape, typ, dev, optional=opt)
+    if y is None:
+        y = torch.empty((batch, L, H, P), dtype=dt_, device=dev)
+    _check(y, "y", (batch, L, H, P), dt_, dev)
+    if last_state is None and want_last_state:
+        last_state = torch.empty((batch, H, N, P), dtype=torch.float32, device=dev)
+    _check(last_state, "last_state", (batch, H, N, P), torch.float32, dev, optional=True)
+    rc = load_library().mss_ssd_fwd(
+        _ptr(x), _ptr(dt), _ptr(A), _ptr(B), _ptr(C), _ptr(D), _ptr(z), _ptr(dt_bias), int(bool(softplus)),
+        _ptr(initial_state), _ptr(y), _ptr(last_state), batch, L, H, P, G, N, code, _stream_handle(stream, dev))
+    if rc != 0:
+        raise MssError(rc, "mss_ssd_fwd")
+    return y, last_state
 
 
 def bwd_workspace_size(batch, dim, dstate, seqlen, dtype=torch.bfloat16, flags=0) -> int:

@@ -35,6 +35,10 @@ int64_t backward_workspace_bytes(int64_t batch, int64_t dim, int64_t seqlen, uns
 template <typename T, int N>
 int launch_decode(mss::StepParams p, cudaStream_t stream);
 
+// Structured-state-space-duality forward pass over validated arguments
+// (bf16 io, P = 64, dstate 64 or 128).
+int launch_ssd(const mss::SsdParams& p, int dstate, cudaStream_t stream);
+
 #define MSS_DECLARE_LAUNCHERS(T, N)                                                                      \
     extern template int launch_forward<T, N>(mss::ScanParams, unsigned, void*, int64_t, cudaStream_t); \
     extern template int64_t forward_workspace_bytes<T, N>(int64_t, int64_t, int64_t);                   \

@@ -399,6 +399,54 @@ int64_t mss_scan_bwd_workspace_size(int64_t batch, int64_t dim, int64_t dstate, 
     });
 }
 
+int mss_ssd_fwd(const void* x, const void* dt, const float* A, const void* B, const void* C, const float* D,
+                const void* z, const float* dt_bias, int softplus_flag, const float* initial_state, void* y,
+                float* last_state, int64_t batch, int64_t seqlen, int64_t nheads, int64_t headdim,
+                int64_t ngroups, int64_t dstate, int dtype, void* stream) {
+    if (dtype != MSS_DTYPE_BF16) return MSS_ERR_DTYPE;  // the tensor-core path takes bf16 io
+    if (batch < 0 || seqlen < 0 || nheads < 1 || ngroups < 1 || nheads % ngroups != 0 || headdim != 64 ||
+        (dstate != 64 && dstate != 128))
+        return MSS_ERR_SHAPE;
+    int64_t tok, xe, xbytes, bce, bcbytes, ste, stbytes, dtbytes;
+    if (!mul_ok(batch, seqlen, &tok) || !mul_ok(tok, nheads * headdim, &xe) || !mul_ok(xe, 2, &xbytes) ||
+        !mul_ok(tok, ngroups * dstate, &bce) || !mul_ok(bce, 2, &bcbytes) ||
+        !mul_ok(batch * nheads, dstate * headdim, &ste) || !mul_ok(ste, 4, &stbytes) ||
+        !mul_ok(tok, nheads * 2, &dtbytes) || tok > (int64_t(1) << 40))
+        return MSS_ERR_SHAPE;
+    if (batch == 0) return MSS_OK;
+    if (!A || (seqlen > 0 && (!x || !dt || !B || !C || !y))) return MSS_ERR_NULL;
+    const void* v16[] = {x, B, C, y, z};
+    for (const void* q : v16)
+        if (q && !aligned(q, 16)) return MSS_ERR_ALIGN;
+    if (dt && !aligned(dt, 2)) return MSS_ERR_ALIGN;
+    const void* fp[] = {A, D, dt_bias, initial_state, last_state};
+    for (const void* q : fp)
+        if (q && !aligned(q, 4)) return MSS_ERR_ALIGN;
+    struct Range { const void* p; int64_t n; };
+    const Range outs[] = {{y, xbytes}, {last_state, stbytes}};
+    const Range ins[] = {{x, xbytes}, {z, xbytes}, {dt, dtbytes}, {B, bcbytes}, {C, bcbytes}, {A, nheads * 4},
+                         {D, nheads * 4}, {dt_bias, nheads * 4}, {initial_state, stbytes}};
+    for (const Range& o : outs) {
+        for (const Range& r : ins)
+            if (overlaps(o.p, o.n, r.p, r.n)) return MSS_ERR_ALIAS;
+        for (const Range& o2 : outs)
+            if (&o != &o2 && overlaps(o.p, o.n, o2.p, o2.n)) return MSS_ERR_ALIAS;
+    }
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    if (seqlen == 0) {
+        if (last_state) {
+            const cudaError_t e = initial_state
+                ? cudaMemcpyAsync(last_state, initial_state, size_t(stbytes), cudaMemcpyDeviceToDevice, s)
+                : cudaMemsetAsync(last_state, 0, size_t(stbytes), s);
+            if (e != cudaSuccess) return MSS_ERR_CUDA;
+        }
+        return MSS_OK;
+    }
+    mss::SsdParams p{x, dt, A, B, C, D, z, dt_bias, initial_state, y, last_state, batch, seqlen, nheads, ngroups,
+                     softplus_flag ? 1 : 0};
+    return launch_ssd(p, int(dstate), s);
+}
+
 int mss_get_device_error(void* stream) {
     cudaStream_t s = static_cast<cudaStream_t>(stream);
     if (cudaStreamSynchronize(s) != cudaSuccess) return MSS_ERR_CUDA;

@@ -71,6 +71,25 @@ struct BwdParams {
     unsigned int* err;
 };
 
+// Structured state space duality (ssd_mma.cuh): x, z, y [batch, L, H, P];
+// dt [batch, L, H]; B, C [batch, L, G, N]; A, D, dt_bias [H] fp32;
+// initial_state, last_state [batch, H, N, P] fp32.
+struct SsdParams {
+    const void* x;
+    const void* dt;
+    const float* A;
+    const void* B;
+    const void* C;
+    const float* D;        // may be null
+    const void* z;         // may be null
+    const float* dt_bias;  // may be null
+    const float* initial_state;  // may be null
+    void* y;
+    float* last_state;     // may be null
+    int64_t batch, seqlen, nheads, ngroups;
+    int softplus;
+};
+
 struct StepParams {
     float* state;
     const void* u;

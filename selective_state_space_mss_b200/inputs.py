@@ -187,3 +187,31 @@ def upstream_gradients(batch: int, dim: int, dstate: int, seqlen: int, dtype: st
     dy = _store(rng.standard_normal((batch, dim, seqlen), dtype=np.float32), dtype)
     dlast = rng.standard_normal((batch, dim, dstate), dtype=np.float32)
     return dy, dlast
+
+
+# The structured-state-space-duality (Mamba-2) layer: token-major tensors,
+# a scalar A per head, heads sharing B and C within a group.
+SSD_WORKLOAD = "mamba2-layer-bf16-b4-l4096-h64-p64-n128-g1"
+SSD_SHAPES = {SSD_WORKLOAD: dict(batch=4, seqlen=4096, nheads=64, headdim=64, ngroups=1, dstate=128, seed=1006)}
+
+
+def ssd_inputs(batch: int, seqlen: int, nheads: int, headdim: int, ngroups: int, dstate: int, seed: int,
+               dtype: str = "bf16") -> dict:
+    """x, z ~ N(0, 1) [batch, L, H, P]; dt_raw = 0.1 N(0, 1) [batch, L, H] with
+    dt_bias = softplus^-1 of a log-uniform step on [1e-3, 1e-1] per head;
+    A_h = -exp(U(0, ln 16)); B, C ~ N(0, 1) / sqrt(N) [batch, L, G, N] (so that
+    C . B stays of order one); D ~ N(1, 0.1).  bf16 storage for x, z, dt, B, C."""
+    rng = _rng(seed, 7)
+    f = lambda *s: rng.standard_normal(s, dtype=np.float32)
+    dt_h = np.exp(rng.uniform(np.log(1e-3), np.log(1e-1), size=nheads))
+    scale = np.float32(1.0 / np.sqrt(dstate))
+    return dict(
+        x=_store(f(batch, seqlen, nheads, headdim), dtype),
+        z=_store(f(batch, seqlen, nheads, headdim), dtype),
+        dt=_store(np.float32(0.1) * f(batch, seqlen, nheads), dtype),
+        dt_bias=np.log(np.expm1(dt_h)).astype(np.float32),
+        A=(-np.exp(rng.uniform(0.0, np.log(16.0), size=nheads))).astype(np.float32),
+        B=_store(scale * f(batch, seqlen, ngroups, dstate), dtype),
+        C=_store(scale * f(batch, seqlen, ngroups, dstate), dtype),
+        D=(1.0 + 0.1 * rng.standard_normal(nheads)).astype(np.float32),
+    )

@@ -264,3 +264,28 @@ def test_bwd_argument_errors(lib):
     assert q(1, 16, 16, 4097, 1, 0) == 16 * 257 * 16 * 4           # odd rows take the scalar path
     assert q(1, 16, 16, 0, 1, 0) == 0
     assert q(1, 16, 3, 64, 1, 0) == codes["MSS_ERR_UNSUPPORTED_N"]
+
+
+def test_ssd_argument_errors(lib):
+    codes = _enum("mss_status")
+    v = ctypes.c_void_p
+    lib.mss_ssd_fwd.restype = ctypes.c_int
+
+    def ssd(**kw):
+        a = dict(x=P, dt=P + 0x1000000, A=P + 0x2000000, B=P + 0x3000000, C=P + 0x4000000, y=P + 0x5000000,
+                 last=None, batch=2, L=64, H=4, Pd=64, G=1, N=128, dtype=1)
+        a.update(kw)
+        w = lambda x: v(x) if x is not None else None
+        return lib.mss_ssd_fwd(w(a["x"]), w(a["dt"]), w(a["A"]), w(a["B"]), w(a["C"]), None, None, None, 1, None,
+                               w(a["y"]), w(a["last"]), ctypes.c_int64(a["batch"]), ctypes.c_int64(a["L"]),
+                               ctypes.c_int64(a["H"]), ctypes.c_int64(a["Pd"]), ctypes.c_int64(a["G"]),
+                               ctypes.c_int64(a["N"]), a["dtype"], None)
+
+    assert ssd(dtype=0) == codes["MSS_ERR_DTYPE"]          # the tensor-core path takes bf16
+    assert ssd(Pd=32) == codes["MSS_ERR_SHAPE"]
+    assert ssd(N=96) == codes["MSS_ERR_SHAPE"]
+    assert ssd(H=3, G=2) == codes["MSS_ERR_SHAPE"]
+    assert ssd(x=None) == codes["MSS_ERR_NULL"]
+    assert ssd(B=P + 0x3000008) == codes["MSS_ERR_ALIGN"]
+    assert ssd(y=P) == codes["MSS_ERR_ALIAS"]
+    assert ssd(batch=0) == 0

@@ -1,0 +1,95 @@
+"""GPU parity of the structured-state-space-duality (Mamba-2) forward pass
+(mss_ssd_fwd) against the fp64 oracle (oracle.ssd_fwd, pinned to the Mamba-1
+oracle, the semiseparable matrix and the chunked algorithm).  bf16 io, so the
+bf16 tolerance of tests/helpers.py applies; the tensor-core operands (masked
+scores, the carried state) round to bf16 inside the kernel as well."""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import selective_state_space_mss_b200 as mss
+from selective_state_space_mss_b200 import inputs as gen
+
+from tests.helpers import assert_close, to_numpy, to_torch
+
+pytestmark = pytest.mark.gpu
+DEV = torch.device("cuda", 0)
+
+
+def _dev(inp, gate=True, with_D=True, with_bias=True):
+    return dict(x=to_torch(inp["x"], DEV), dt=to_torch(inp["dt"], DEV), A=torch.from_numpy(inp["A"]).to(DEV),
+                B=to_torch(inp["B"], DEV), C=to_torch(inp["C"], DEV),
+                D=torch.from_numpy(inp["D"]).to(DEV) if with_D else None,
+                z=to_torch(inp["z"], DEV) if gate else None,
+                dt_bias=torch.from_numpy(inp["dt_bias"]).to(DEV) if with_bias else None)
+
+
+def _ref(inp, gate=True, with_D=True, with_bias=True, h0=None):
+    return oracle.ssd_fwd(inp["x"].values, inp["dt"].values, inp["A"], inp["B"].values, inp["C"].values,
+                          D=inp["D"] if with_D else None, z=inp["z"].values if gate else None,
+                          dt_bias=inp["dt_bias"] if with_bias else None, initial_state=h0)
+
+
+@pytest.mark.parametrize("N", [64, 128])
+@pytest.mark.parametrize("L", [64, 200, 512])
+@pytest.mark.parametrize("G", [1, 2])
+def test_ssd_matches_oracle(N, L, G):
+    """Whole chunks, a ragged last chunk, one or two groups of heads."""
+    inp = gen.ssd_inputs(2, L, 4, 64, G, N, seed=700 + L + N + G)
+    y, last = mss.ssd_fwd(**_dev(inp))
+    torch.cuda.synchronize()
+    assert mss.get_device_error() == 0
+    y_ref, last_ref = _ref(inp)
+    assert_close(to_numpy(y), y_ref, "bf16", f"N={N} L={L} G={G} y")
+    assert_close(to_numpy(last), last_ref, "bf16", f"N={N} L={L} G={G} last_state")
+
+
+def test_ssd_starting_state_and_chaining():
+    inp = gen.ssd_inputs(2, 320, 4, 64, 1, 128, seed=720)
+    h0 = np.random.default_rng(721).standard_normal((2, 4, 128, 64)).astype(np.float32) * 0.1
+    d = _dev(inp)
+    y, last = mss.ssd_fwd(**d, initial_state=torch.from_numpy(h0).to(DEV))
+    torch.cuda.synchronize()
+    y_ref, last_ref = _ref(inp, h0=h0.astype(np.float64))
+    assert_close(to_numpy(y), y_ref, "bf16", "y from a starting state")
+    assert_close(to_numpy(last), last_ref, "bf16", "last_state from a starting state")
+    # two calls chained through last_state equal one call
+    part = lambda t0, t1: {k: (v[:, t0:t1].contiguous() if k in ("x", "dt", "B", "C", "z") else v)
+                           for k, v in d.items()}
+    y0, last0 = mss.ssd_fwd(**part(0, 128))
+    y1, last1 = mss.ssd_fwd(**part(128, 320), initial_state=last0)
+    y_all, last_all = mss.ssd_fwd(**d)
+    torch.cuda.synchronize()
+    assert_close(to_numpy(torch.cat([y0, y1], dim=1)), to_numpy(y_all).astype(np.float64), "bf16", "chained y")
+    assert_close(to_numpy(last1), to_numpy(last_all).astype(np.float64), "bf16", "chained state")
+
+
+def test_ssd_without_optional_inputs():
+    inp = gen.ssd_inputs(1, 256, 2, 64, 1, 64, seed=730)
+    y, last = mss.ssd_fwd(**_dev(inp, gate=False, with_D=False, with_bias=False))
+    torch.cuda.synchronize()
+    y_ref, last_ref = _ref(inp, gate=False, with_D=False, with_bias=False)
+    assert_close(to_numpy(y), y_ref, "bf16", "bare y")
+    assert_close(to_numpy(last), last_ref, "bf16", "bare last_state")
+
+
+def test_ssd_workload_sampled_heads():
+    """The bench workload (4 x 4096 tokens, 64 heads of 64, N = 128): y and
+    the final state of sampled (batch, head) pairs against the oracle."""
+    s = gen.SSD_SHAPES[gen.SSD_WORKLOAD]
+    inp = gen.ssd_inputs(**s)
+    y, last = mss.ssd_fwd(**_dev(inp))
+    torch.cuda.synchronize()
+    assert mss.get_device_error() == 0
+    yn, ln = to_numpy(y), to_numpy(last)
+    rng = np.random.default_rng(740)
+    for _ in range(3):
+        b, h = int(rng.integers(s["batch"])), int(rng.integers(s["nheads"]))
+        sub = {k: (v.values[b:b + 1, :, h:h + 1] if k in ("x", "z", "dt") else v)
+               for k, v in inp.items() if k in ("x", "z", "dt")}
+        y_ref, last_ref = oracle.ssd_fwd(sub["x"], sub["dt"], inp["A"][h:h + 1], inp["B"].values[b:b + 1],
+                                         inp["C"].values[b:b + 1], D=inp["D"][h:h + 1], z=sub["z"],
+                                         dt_bias=inp["dt_bias"][h:h + 1])
+        assert_close(yn[b:b + 1, :, h:h + 1], y_ref, "bf16", f"y of (b={b}, h={h})")
+        assert_close(ln[b:b + 1, h:h + 1], last_ref, "bf16", f"state of (b={b}, h={h})")
