@@ -94,6 +94,16 @@ def measured_peaks():
         return FALLBACK_HBM_GBS, "fallback", 1965.0
 
 
+def measured_bf16_tflops():
+    """The pool's measured dense bf16 GEMM rate (burst), TFLOP/s, or the
+    fallback figure."""
+    try:
+        with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
+            return float(json.load(f)["bf16_tflops"]), "measured"
+    except Exception:
+        return 1590.0, "fallback"
+
+
 def kernel_source_hash():
     h = hashlib.sha256()
     for rel in KERNEL_SOURCES:
@@ -404,6 +414,31 @@ def run_mss(args, rank, world, local_rank):
     conv_ms = [a_.elapsed_time(b_) for a_, b_ in conv_ms]
     assert mss.get_device_error() == 0
 
+    # the structured-state-space-duality (Mamba-2) layer: its own workload
+    ss = gen.SSD_SHAPES[gen.SSD_WORKLOAD]
+    sin = gen.ssd_inputs(**ss)
+    sd = dict(x=to_dev(sin["x"]), dt=to_dev(sin["dt"]), A=torch.from_numpy(sin["A"]).to(dev),
+              B=to_dev(sin["B"]), C=to_dev(sin["C"]), D=torch.from_numpy(sin["D"]).to(dev), z=to_dev(sin["z"]),
+              dt_bias=torch.from_numpy(sin["dt_bias"]).to(dev))
+    ssd_y = torch.empty_like(sd["x"])
+    ssd_last = torch.empty(ss["batch"], ss["nheads"], ss["dstate"], ss["headdim"], device=dev)
+    ssd_ev = []
+    for i in range(args.warmup + args.steps):
+        a_, b_ = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a_.record(stream)
+        mss.ssd_fwd(**sd, y=ssd_y, last_state=ssd_last)
+        b_.record(stream)
+        if i >= args.warmup:
+            ssd_ev.append((a_, b_))
+    torch.cuda.synchronize(dev)
+    ssd_ms = sum(a_.elapsed_time(b_) for a_, b_ in ssd_ev) / len(ssd_ev)
+    assert mss.get_device_error() == 0
+    del sd, ssd_y, sin
+    # matrix-form flops per (token, head): C B^T and M X within the chunk, C S
+    # and the state product B^T X across chunks (chunk of 64, P = 64)
+    ssd_flops = ss["batch"] * ss["seqlen"] * ss["nheads"] * (
+        2 * 64 * ss["dstate"] + 2 * 64 * ss["headdim"] + 2 * ss["dstate"] * ss["headdim"] * 2)
+
     # the backward pass (gradients of every input, states recomputed from
     # checkpoints) on the same workload
     dy_h, dlast_h = gen.upstream_gradients(w.batch, w.dim, w.dstate, w.seqlen, w.dtype, rank_seed(w.seed, rank))
@@ -561,6 +596,13 @@ def run_mss(args, rank, world, local_rank):
                      "achieved_gbs": bytes_bwd / (bwd_avg * 1e-3) / 1e9,
                      "frac": bytes_bwd / (bwd_avg * 1e-3) / 1e9 / peak,
                      "note": "gradients of u, delta, A, B, C, D, z, bias, starting state; checkpoint pass included"},
+        "ssd_path": {"workload": gen.SSD_WORKLOAD, "ms_avg": ssd_ms,
+                     "channel_tokens_per_s": ss["batch"] * ss["seqlen"] * ss["nheads"] * ss["headdim"] / (ssd_ms * 1e-3),
+                     "roofline": {"bound": "tensor", "achieved": ssd_flops / (ssd_ms * 1e-3) / 1e12,
+                                  "peak": measured_bf16_tflops()[0], "unit": "TFLOP/s",
+                                  "frac": ssd_flops / (ssd_ms * 1e-3) / 1e12 / measured_bf16_tflops()[0],
+                                  "peak_kind": measured_bf16_tflops()[1],
+                                  "note": "bf16 mma.sync products, fp32 accumulation"}},
         "zoh_input_path": {"fwd_ms_avg": fwd_avg_zoh,
                            "achieved_gbs": bytes_fwd / (fwd_avg_zoh * 1e-3) / 1e9,
                            "frac": bytes_fwd / (fwd_avg_zoh * 1e-3) / 1e9 / peak,

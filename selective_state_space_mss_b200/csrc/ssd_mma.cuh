@@ -46,11 +46,14 @@ struct SsdLayout {
     static constexpr int kXBytes = kQ * kXStride * 2;
     static constexpr int kBBytes = kQ * kBStride * 2;
     static constexpr int kSBytes = NS * kSStride * 2;
-    static constexpr int kXs = 0;                      // X
-    static constexpr int kXw = kXs + kXBytes;          // X scaled by exp(cs_last - cs_j) Delta_j
-    static constexpr int kBs = kXw + kXBytes;
-    static constexpr int kCs = kBs + kBBytes;
-    static constexpr int kSs = kCs + kBBytes;
+    // two buffers of X, B, C: the next chunk's copies run during this one
+    static constexpr int kBufBytes = kXBytes + 2 * kBBytes;
+    static constexpr int kBuf = 0;                     // [2] x (X, B, C)
+    // the state's bf16 copy, read by C S_prev; then, in the same bytes, X
+    // scaled by exp(cs_last - cs_j) Delta_j for the state product
+    static constexpr int kSs = 2 * kBufBytes;
+    static constexpr int kXw = kSs;
+    static_assert(kXBytes <= kSBytes, "X fits where the state copy was");
     static constexpr int kScal = kSs + kSBytes;        // per token: Delta, cs (fp32)
     static constexpr int kSmemBytes = kScal + 2 * kQ * 4;
 };
@@ -82,6 +85,15 @@ __device__ __forceinline__ void mma_bf16(float (&d)[4], const uint32_t (&a)[4], 
 
 __device__ __forceinline__ uint32_t pack_bf16(float lo, float hi) { return pack_bf16x2(lo, hi); }
 
+// 16-byte asynchronous copy global -> shared; src_bytes = 0 writes zeros.
+__device__ __forceinline__ void cp_async16(void* dst, const void* src, uint32_t src_bytes) {
+    asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(smem_u32(dst)), "l"(src), "r"(src_bytes)
+                 : "memory");
+}
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+template <int kPending>
+__device__ __forceinline__ void cp_async_wait() { asm volatile("cp.async.wait_group %0;" ::"n"(kPending) : "memory"); }
+
 // grid = batch * nheads, block = 128 threads, dynamic shared memory
 // SsdLayout<NS>::kSmemBytes.
 template <int NS, bool kGate, bool kSoftplus>
@@ -90,10 +102,7 @@ __global__ void __launch_bounds__(128) ssd_fwd_kernel(SsdParams p) {
     constexpr int Q = Ly::kQ, P = Ly::kP;
     constexpr int MS = NS / 64;  // 16-row state tiles per warp (the state is NS rows over 4 warps)
     extern __shared__ __align__(16) uint8_t smem[];
-    bf16_t* Xs = reinterpret_cast<bf16_t*>(smem + Ly::kXs);
     bf16_t* Xw = reinterpret_cast<bf16_t*>(smem + Ly::kXw);
-    bf16_t* Bs = reinterpret_cast<bf16_t*>(smem + Ly::kBs);
-    bf16_t* Cs = reinterpret_cast<bf16_t*>(smem + Ly::kCs);
     bf16_t* Ss = reinterpret_cast<bf16_t*>(smem + Ly::kSs);
     float* dts = reinterpret_cast<float*>(smem + Ly::kScal);
     float* css = dts + Q;
@@ -127,28 +136,59 @@ __global__ void __launch_bounds__(128) ssd_fwd_kernel(SsdParams p) {
             }
 
     const int64_t n_chunks = (L + Q - 1) / Q;
+    auto buf_x = [&](int64_t c) { return reinterpret_cast<bf16_t*>(smem + Ly::kBuf + (c & 1) * Ly::kBufBytes); };
+    auto buf_b = [&](int64_t c) { return buf_x(c) + Q * Ly::kXStride; };
+    auto buf_c = [&](int64_t c) { return buf_b(c) + Q * Ly::kBStride; };
+    // X, B, C rows of chunk c (16-byte pieces) into its buffer, zero past the sequence
+    auto issue = [&](int64_t c) {
+        const int64_t t0 = c * Q;
+        const int q = int(min(int64_t(Q), L - t0));
+        bf16_t* X_ = buf_x(c);
+        bf16_t* B_ = buf_b(c);
+        bf16_t* C_ = buf_c(c);
+        for (int i = tid; i < Q * (P / 8); i += Ly::kThreads) {
+            const int r = i / (P / 8), k8 = i % (P / 8);
+            const int rr = r < q ? r : 0;  // a row inside the sequence, copied as zeros
+            cp_async16(X_ + r * Ly::kXStride + k8 * 8, x + ((b * L + t0 + rr) * H + h) * P + k8 * 8, r < q ? 16u : 0u);
+        }
+        for (int i = tid; i < Q * (NS / 8); i += Ly::kThreads) {
+            const int r = i / (NS / 8), k8 = i % (NS / 8);
+            const int rr = r < q ? r : 0;
+            const int64_t off = ((b * L + t0 + rr) * p.ngroups + g) * NS + k8 * 8;
+            cp_async16(B_ + r * Ly::kBStride + k8 * 8, Bg + off, r < q ? 16u : 0u);
+            cp_async16(C_ + r * Ly::kBStride + k8 * 8, Cg + off, r < q ? 16u : 0u);
+        }
+        cp_async_commit();
+    };
+    // step sizes of chunk c's tokens, two a lane of warp 0
+    auto load_dt = [&](int64_t c, float (&dv)[2]) {
+        const int64_t t0 = c * Q;
+        const int q = int(min(int64_t(Q), L - t0));
+#pragma unroll
+        for (int k = 0; k < 2; ++k) {
+            const int r = 2 * lane + k;
+            float d = 0.f;
+            if (r < q) {
+                const float sraw = to_f32(dtp[(b * L + t0 + r) * H + h]) + bias;
+                d = kSoftplus ? softplus_fast(sraw) : sraw;
+            }
+            dv[k] = d;
+        }
+    };
+    float dnext[2] = {0.f, 0.f};
+    if (n_chunks > 0) {
+        issue(0);
+        if (warp == 0) load_dt(0, dnext);
+    }
     for (int64_t c = 0; c < n_chunks; ++c) {
         const int64_t t0 = c * Q;
         const int q = int(min(int64_t(Q), L - t0));
         __syncthreads();  // the previous chunk's reads of shared memory are done
-        // X, B, C rows of the chunk (16-byte pieces), zero past the sequence
-        for (int i = tid; i < Q * (P / 8); i += Ly::kThreads) {
-            const int r = i / (P / 8), k8 = i % (P / 8);
-            uint4 v = make_uint4(0u, 0u, 0u, 0u);
-            if (r < q) v = *reinterpret_cast<const uint4*>(x + ((b * L + t0 + r) * H + h) * P + k8 * 8);
-            *reinterpret_cast<uint4*>(Xs + r * Ly::kXStride + k8 * 8) = v;
-        }
-        for (int i = tid; i < Q * (NS / 8); i += Ly::kThreads) {
-            const int r = i / (NS / 8), k8 = i % (NS / 8);
-            uint4 vb = make_uint4(0u, 0u, 0u, 0u), vc = vb;
-            if (r < q) {
-                const int64_t off = ((b * L + t0 + r) * p.ngroups + g) * NS + k8 * 8;
-                vb = *reinterpret_cast<const uint4*>(Bg + off);
-                vc = *reinterpret_cast<const uint4*>(Cg + off);
-            }
-            *reinterpret_cast<uint4*>(Bs + r * Ly::kBStride + k8 * 8) = vb;
-            *reinterpret_cast<uint4*>(Cs + r * Ly::kBStride + k8 * 8) = vc;
-        }
+        // the next chunk's copies run during this chunk
+        if (c + 1 < n_chunks) issue(c + 1);
+        const bf16_t* Xs = buf_x(c);
+        const bf16_t* Bs = buf_b(c);
+        const bf16_t* Cs = buf_c(c);
         // the incoming state as bf16, [n][p]
 #pragma unroll
         for (int m = 0; m < MS; ++m)
@@ -160,19 +200,11 @@ __global__ void __launch_bounds__(128) ssd_fwd_kernel(SsdParams p) {
                     *reinterpret_cast<uint32_t*>(Ss + n * Ly::kSStride + pc) =
                         pack_bf16(s[m][pt][2 * hr], s[m][pt][2 * hr + 1]);
                 }
-        // step sizes and the running sum of Delta A (warp 0: two tokens a lane)
+        // step sizes and the running sum of Delta A (warp 0: two tokens a lane);
+        // the next chunk's step sizes are read now, used then
         if (warp == 0) {
-            float dv[2], cv[2];
-#pragma unroll
-            for (int k = 0; k < 2; ++k) {
-                const int r = 2 * lane + k;
-                float d = 0.f;
-                if (r < q) {
-                    const float sraw = to_f32(dtp[(b * L + t0 + r) * H + h]) + bias;
-                    d = kSoftplus ? softplus_fast(sraw) : sraw;
-                }
-                dv[k] = d;
-            }
+            float dv[2] = {dnext[0], dnext[1]}, cv[2];
+            if (c + 1 < n_chunks) load_dt(c + 1, dnext);
             cv[0] = dv[0] * Ah;
             cv[1] = cv[0] + dv[1] * Ah;
             float run = cv[1];
@@ -187,6 +219,11 @@ __global__ void __launch_bounds__(128) ssd_fwd_kernel(SsdParams p) {
             css[2 * lane] = before + cv[0];
             css[2 * lane + 1] = before + cv[1];
         }
+        // this chunk's copies have landed (the next chunk's may still run)
+        if (c + 1 < n_chunks)
+            cp_async_wait<1>();
+        else
+            cp_async_wait<0>();
         __syncthreads();
         const float cs_last = css[Q - 1];
 
@@ -280,7 +317,9 @@ __global__ void __launch_bounds__(128) ssd_fwd_kernel(SsdParams p) {
                 }
             }
         }
-        // X scaled by w_j = exp(cs_last - cs_j) Delta_j for the state product
+        // X scaled by w_j = exp(cs_last - cs_j) Delta_j for the state product,
+        // where the state copy was (every warp is done reading it)
+        __syncthreads();
         for (int i = tid; i < Q * (P / 2); i += Ly::kThreads) {
             const int r = i / (P / 2), k2 = i % (P / 2);
             const float w = __expf(cs_last - css[r]) * dts[r];
