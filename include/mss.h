@@ -319,6 +319,30 @@ MSS_API int mss_ssd_fwd(const void *x, const void *dt, const float *A, const voi
                 const float *initial_state, void *y, float *last_state, int64_t batch, int64_t seqlen,
                 int64_t nheads, int64_t headdim, int64_t ngroups, int64_t dstate, int dtype, void *stream);
 
+/* mss_ssd_fwd with a caller-owned workspace (device memory, 16-byte aligned,
+ * at least mss_ssd_fwd_workspace_size bytes, not overlapping any argument).
+ * When batch * nheads leaves the in-order kernel's last wave of CTAs (one
+ * per (batch, head), up to two per SM) short enough, the chunks of every
+ * head then run in parallel in three passes (chunk states, the recurrence of
+ * chunk states, chunk outputs) instead of one CTA walking a head's chunks in
+ * order; otherwise the workspace is not used (the passes' extra state
+ * traffic would cost more than they gain).  On a 148-SM B200 the passes run
+ * for 1-230 pairs and 297-417, for instance, not for 231-296;
+ * mss_ssd_fwd_workspace_size returns 0 where the workspace goes unused.
+ * Same result up to rounding; a NULL workspace is mss_ssd_fwd.
+ * MSS_ERR_WORKSPACE if it is too small. */
+MSS_API int mss_ssd_fwd_ex(const void *x, const void *dt, const float *A, const void *B, const void *C,
+                   const float *D, const void *z, const float *dt_bias, int softplus_flag,
+                   const float *initial_state, void *y, float *last_state, int64_t batch, int64_t seqlen,
+                   int64_t nheads, int64_t headdim, int64_t ngroups, int64_t dstate, int dtype,
+                   void *workspace, int64_t workspace_bytes, void *stream);
+
+/* Workspace bytes mss_ssd_fwd_ex would use for these sizes on the current
+ * device (0: the in-order kernel, or no tokens), or a negative mss_status
+ * (MSS_ERR_SHAPE for unsupported sizes). */
+MSS_API int64_t mss_ssd_fwd_workspace_size(int64_t batch, int64_t seqlen, int64_t nheads, int64_t headdim,
+                                   int64_t ngroups, int64_t dstate);
+
 /*
  * mss_state_update -- one decode token for every (batch, channel):
  * the recurrence above applied once to a caller-held state

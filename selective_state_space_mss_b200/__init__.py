@@ -88,6 +88,11 @@ def load_library():
             lib.mss_ssd_fwd.argtypes = [vp, vp, fp, vp, vp, fp, vp, fp, i, fp, vp, fp,
                                         i64, i64, i64, i64, i64, i64, i, vp]
             lib.mss_ssd_fwd.restype = i
+            lib.mss_ssd_fwd_ex.argtypes = [vp, vp, fp, vp, vp, fp, vp, fp, i, fp, vp, fp,
+                                           i64, i64, i64, i64, i64, i64, i, vp, i64, vp]
+            lib.mss_ssd_fwd_ex.restype = i
+            lib.mss_ssd_fwd_workspace_size.argtypes = [i64, i64, i64, i64, i64, i64]
+            lib.mss_ssd_fwd_workspace_size.restype = i64
             lib.mss_scan_fwd_conv.argtypes = [vp, fp, fp, i, vp, vp, vp, fp, vp, vp, fp, vp, fp, i, fp, vp, fp,
                                               i64, i64, i64, i64, i, u32, vp, i64, vp]
             lib.mss_scan_fwd_conv.restype = i
@@ -268,11 +273,14 @@ def scan_fwd_conv(x, conv_w, delta, A, B, C, conv_b=None, conv_state=None, D=Non
 
 
 def ssd_fwd(x, dt, A, B, C, D=None, z=None, dt_bias=None, softplus=True, initial_state=None, y=None,
-            last_state=None, want_last_state=True, stream=None):
-    """Structured-state-space-duality forward pass (mss_ssd_fwd).  x, z:
+            last_state=None, want_last_state=True, workspace="auto", stream=None):
+    """Structured-state-space-duality forward pass (mss_ssd_fwd_ex).  x, z:
     [batch, L, H, P] bf16; dt: [batch, L, H] bf16; A, D, dt_bias: [H]
     float32; B, C: [batch, L, G, N] bf16; initial_state: [batch, H, N, P]
-    float32.  Returns (y, last_state)."""
+    float32.  workspace: "auto" (what mss_ssd_fwd_workspace_size asks for,
+    from PyTorch's allocator: every chunk in parallel where that beats one CTA
+    per head, else nothing), None (one CTA per head walks its chunks) or a
+    uint8 CUDA tensor.  Returns (y, last_state)."""
     if not isinstance(x, torch.Tensor) or x.device.type != "cuda":
         raise ValueError("x must be a CUDA tensor (there is no CPU path)")
     if x.dim() != 4 or B.dim() != 4:
@@ -294,9 +302,19 @@ def ssd_fwd(x, dt, A, B, C, D=None, z=None, dt_bias=None, softplus=True, initial
     if last_state is None and want_last_state:
         last_state = torch.empty((batch, H, N, P), dtype=torch.float32, device=dev)
     _check(last_state, "last_state", (batch, H, N, P), torch.float32, dev, optional=True)
-    rc = load_library().mss_ssd_fwd(
+    if isinstance(workspace, str):
+        if workspace != "auto":
+            raise ValueError("workspace must be 'auto', None or a uint8 CUDA tensor")
+        nbytes = int(load_library().mss_ssd_fwd_workspace_size(batch, L, H, P, G, N))
+        if nbytes < 0:
+            raise MssError(nbytes, "mss_ssd_fwd_workspace_size")
+        workspace = torch.empty(nbytes, dtype=torch.uint8, device=dev) if nbytes > 0 else None
+    if workspace is not None:
+        _check(workspace, "workspace", (workspace.numel(),), torch.uint8, dev)
+    rc = load_library().mss_ssd_fwd_ex(
         _ptr(x), _ptr(dt), _ptr(A), _ptr(B), _ptr(C), _ptr(D), _ptr(z), _ptr(dt_bias), int(bool(softplus)),
-        _ptr(initial_state), _ptr(y), _ptr(last_state), batch, L, H, P, G, N, code, _stream_handle(stream, dev))
+        _ptr(initial_state), _ptr(y), _ptr(last_state), batch, L, H, P, G, N, code, _ptr(workspace),
+        0 if workspace is None else workspace.numel(), _stream_handle(stream, dev))
     if rc != 0:
         raise MssError(rc, "mss_ssd_fwd")
     return y, last_state

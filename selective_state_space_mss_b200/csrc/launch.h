@@ -39,6 +39,14 @@ int launch_decode(mss::StepParams p, cudaStream_t stream);
 // (bf16 io, P = 64, dstate 64 or 128).
 int launch_ssd(const mss::SsdParams& p, int dstate, cudaStream_t stream);
 
+// The same with every chunk in parallel (three passes) over a workspace of
+// ssd_workspace_bytes (16-byte aligned).
+int launch_ssd_chunked(const mss::SsdParams& p, int dstate, void* workspace, cudaStream_t stream);
+int64_t ssd_workspace_bytes(int64_t batch, int64_t seqlen, int64_t nheads, int64_t dstate);
+// Whether the chunk-parallel passes beat the in-order kernel for this many
+// (batch, head) pairs on the current device.
+bool ssd_chunked_pays(int64_t batch, int64_t nheads);
+
 #define MSS_DECLARE_LAUNCHERS(T, N)                                                                      \
     extern template int launch_forward<T, N>(mss::ScanParams, unsigned, void*, int64_t, cudaStream_t); \
     extern template int64_t forward_workspace_bytes<T, N>(int64_t, int64_t, int64_t);                   \

@@ -403,6 +403,26 @@ int mss_ssd_fwd(const void* x, const void* dt, const float* A, const void* B, co
                 const void* z, const float* dt_bias, int softplus_flag, const float* initial_state, void* y,
                 float* last_state, int64_t batch, int64_t seqlen, int64_t nheads, int64_t headdim,
                 int64_t ngroups, int64_t dstate, int dtype, void* stream) {
+    return mss_ssd_fwd_ex(x, dt, A, B, C, D, z, dt_bias, softplus_flag, initial_state, y, last_state, batch, seqlen,
+                          nheads, headdim, ngroups, dstate, dtype, nullptr, 0, stream);
+}
+
+int64_t mss_ssd_fwd_workspace_size(int64_t batch, int64_t seqlen, int64_t nheads, int64_t headdim, int64_t ngroups,
+                                   int64_t dstate) {
+    if (batch < 0 || seqlen < 0 || nheads < 1 || ngroups < 1 || nheads % ngroups != 0 || headdim != 64 ||
+        (dstate != 64 && dstate != 128))
+        return MSS_ERR_SHAPE;
+    int64_t bh, tok;
+    if (!mul_ok(batch, nheads, &bh) || !mul_ok(bh, seqlen, &tok) || tok > (int64_t(1) << 40)) return MSS_ERR_SHAPE;
+    return seqlen == 0 || !ssd_chunked_pays(batch, nheads) ? 0 : ssd_workspace_bytes(batch, seqlen, nheads, dstate);
+}
+
+int mss_ssd_fwd_ex(const void* x, const void* dt, const float* A, const void* B, const void* C, const float* D,
+                   const void* z, const float* dt_bias, int softplus_flag, const float* initial_state, void* y,
+                   float* last_state, int64_t batch, int64_t seqlen, int64_t nheads, int64_t headdim,
+                   int64_t ngroups, int64_t dstate, int dtype, void* workspace, int64_t workspace_bytes,
+                   void* stream) {
+    if (workspace_bytes < 0) return MSS_ERR_SHAPE;
     if (dtype != MSS_DTYPE_BF16) return MSS_ERR_DTYPE;  // the tensor-core path takes bf16 io
     if (batch < 0 || seqlen < 0 || nheads < 1 || ngroups < 1 || nheads % ngroups != 0 || headdim != 64 ||
         (dstate != 64 && dstate != 128))
@@ -444,6 +464,16 @@ int mss_ssd_fwd(const void* x, const void* dt, const float* A, const void* B, co
     }
     mss::SsdParams p{x, dt, A, B, C, D, z, dt_bias, initial_state, y, last_state, batch, seqlen, nheads, ngroups,
                      softplus_flag ? 1 : 0};
+    if (workspace && ssd_chunked_pays(batch, nheads)) {
+        const int64_t need = ssd_workspace_bytes(batch, seqlen, nheads, dstate);
+        if (need > workspace_bytes || !aligned(workspace, 16)) return MSS_ERR_WORKSPACE;
+        const Range ws{workspace, workspace_bytes};
+        for (const Range& r : ins)
+            if (overlaps(ws.p, ws.n, r.p, r.n)) return MSS_ERR_ALIAS;
+        for (const Range& o : outs)
+            if (overlaps(ws.p, ws.n, o.p, o.n)) return MSS_ERR_ALIAS;
+        return launch_ssd_chunked(p, int(dstate), workspace, s);
+    }
     return launch_ssd(p, int(dstate), s);
 }
 

@@ -1,9 +1,12 @@
 // ssd.cu -- host-side launch of the structured-state-space-duality forward
 // pass (ssd_mma.cuh).
+#include <mutex>
+
 #include <cuda_runtime.h>
 
 #include "host_common.h"
 #include "launch.h"
+#include "ssd_chunked.cuh"
 #include "ssd_mma.cuh"
 
 namespace mss_host {
@@ -29,6 +32,71 @@ int launch_ssd_n(const mss::SsdParams& p, cudaStream_t s) {
 
 int launch_ssd(const mss::SsdParams& p, int dstate, cudaStream_t s) {
     return dstate == 64 ? launch_ssd_n<64>(p, s) : launch_ssd_n<128>(p, s);
+}
+
+// Cost model for choosing between the two forms, from B200 timings at 4096
+// tokens (headdim 64, dstate 128).  The in-order kernel runs one CTA per
+// (batch, head), up to two per SM: a wave in which some SM holds two takes
+// about 1.23 times as long as one in which none does (740 vs 600 us).  The
+// chunk-parallel passes spread every chunk over all SMs and take about
+// 0.79 of that lone-CTA time per SM's worth of heads (3.2 us per head on 148
+// SMs).  Both scale with the sequence length, so the comparison does not.
+bool ssd_chunked_pays(int64_t batch, int64_t nheads) {
+    static std::mutex mu;
+    static int cache[kMaxDevices] = {};
+    const int64_t sms = per_device(cache, mu, [](int dev) {
+        int n = 0;
+        return cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) == cudaSuccess ? n : 0;
+    });
+    const int64_t pairs = batch * nheads;
+    if (sms <= 0 || pairs <= 0) return false;
+    const int64_t full = (pairs - 1) / (2 * sms), rest = pairs - full * 2 * sms;
+    const int64_t in_order = full * 123 + (rest > sms ? 123 : 100);  // hundredths of a lone-CTA pass
+    const int64_t chunked = 79 * pairs / sms;
+    return chunked < in_order;
+}
+
+int64_t ssd_workspace_bytes(int64_t batch, int64_t seqlen, int64_t nheads, int64_t dstate) {
+    const int64_t nc = (seqlen + 63) / 64;
+    const int64_t per_chunk = dstate * 64 * (4 + 2) + 4;  // S_local fp32, S_in bf16, decay
+    return batch * nheads * nc * per_chunk;
+}
+
+template <int NS, bool kGate, bool kSoftplus>
+int launch_ssd_chunked_variant(const mss::SsdParams& p, void* workspace, cudaStream_t s) {
+    using CL = mss::SsdChunkLayout<NS>;
+    const int64_t nc = (p.seqlen + 63) / 64, bh = p.batch * p.nheads;
+    if (nc > 0x7fffffffLL || p.nheads > 65535 || p.batch > 65535 || bh > 0x7fffffffLL) return MSS_ERR_SHAPE;
+    float* Sl = static_cast<float*>(workspace);
+    mss::bf16_t* Sin = reinterpret_cast<mss::bf16_t*>(Sl + bh * nc * NS * 64);
+    float* decay = reinterpret_cast<float*>(Sin + bh * nc * NS * 64);
+    auto k1 = mss::ssd_chunk_state_kernel<NS, kSoftplus>;
+    auto k3 = mss::ssd_chunk_out_kernel<NS, kGate, kSoftplus>;
+    if (cudaFuncSetAttribute(k1, cudaFuncAttributeMaxDynamicSharedMemorySize, CL::kSmemBytes) != cudaSuccess ||
+        cudaFuncSetAttribute(k3, cudaFuncAttributeMaxDynamicSharedMemorySize, CL::kSmemBytes) != cudaSuccess)
+        return MSS_ERR_CUDA;
+    const dim3 grid(unsigned(nc), unsigned(p.nheads), unsigned(p.batch));
+    k1<<<grid, 128, CL::kSmemBytes, s>>>(p, Sl, decay);
+    int rc = launch_status();
+    if (rc != MSS_OK) return rc;
+    mss::ssd_state_pass_kernel<NS><<<dim3(unsigned(bh), unsigned(NS * 64 / 256)), 256, 0, s>>>(p, Sl, decay, Sin, nc);
+    rc = launch_status();
+    if (rc != MSS_OK) return rc;
+    k3<<<grid, 128, CL::kSmemBytes, s>>>(p, Sin);
+    return launch_status();
+}
+
+template <int NS>
+int launch_ssd_chunked_n(const mss::SsdParams& p, void* ws, cudaStream_t s) {
+    if (p.z)
+        return p.softplus ? launch_ssd_chunked_variant<NS, true, true>(p, ws, s)
+                          : launch_ssd_chunked_variant<NS, true, false>(p, ws, s);
+    return p.softplus ? launch_ssd_chunked_variant<NS, false, true>(p, ws, s)
+                      : launch_ssd_chunked_variant<NS, false, false>(p, ws, s);
+}
+
+int launch_ssd_chunked(const mss::SsdParams& p, int dstate, void* workspace, cudaStream_t s) {
+    return dstate == 64 ? launch_ssd_chunked_n<64>(p, workspace, s) : launch_ssd_chunked_n<128>(p, workspace, s);
 }
 
 }  // namespace mss_host

@@ -289,3 +289,21 @@ def test_ssd_argument_errors(lib):
     assert ssd(B=P + 0x3000008) == codes["MSS_ERR_ALIGN"]
     assert ssd(y=P) == codes["MSS_ERR_ALIAS"]
     assert ssd(batch=0) == 0
+
+
+def test_ssd_workspace_queries(lib):
+    codes = _enum("mss_status")
+    lib.mss_ssd_fwd_workspace_size.restype = ctypes.c_int64
+    q = lambda *a: lib.mss_ssd_fwd_workspace_size(*[ctypes.c_int64(x) for x in a])
+    # without a device the in-order kernel is chosen: no workspace
+    assert q(2, 128, 4, 64, 1, 128) == 0
+    assert q(2, 0, 4, 64, 1, 128) == 0
+    assert q(2, 128, 4, 32, 1, 128) == codes["MSS_ERR_SHAPE"]
+    assert q(2, 128, 3, 64, 2, 128) == codes["MSS_ERR_SHAPE"]
+    lib.mss_ssd_fwd_ex.restype = ctypes.c_int
+    v = ctypes.c_void_p
+    rc = lib.mss_ssd_fwd_ex(v(P), v(P + 0x1000000), v(P + 0x2000000), v(P + 0x3000000), v(P + 0x4000000), None,
+                            None, None, 1, None, v(P + 0x5000000), None, ctypes.c_int64(2), ctypes.c_int64(128),
+                            ctypes.c_int64(4), ctypes.c_int64(64), ctypes.c_int64(1), ctypes.c_int64(128), 1,
+                            v(P + 0x6000000), ctypes.c_int64(100), None)
+    assert rc in (codes["MSS_ERR_WORKSPACE"], codes["MSS_ERR_CUDA"])  # too small, or no device to launch on

@@ -34,10 +34,12 @@ def _ref(inp, gate=True, with_D=True, with_bias=True, h0=None):
 @pytest.mark.parametrize("N", [64, 128])
 @pytest.mark.parametrize("L", [64, 200, 512])
 @pytest.mark.parametrize("G", [1, 2])
-def test_ssd_matches_oracle(N, L, G):
-    """Whole chunks, a ragged last chunk, one or two groups of heads."""
+@pytest.mark.parametrize("chunks", ["parallel", "in-order"])
+def test_ssd_matches_oracle(N, L, G, chunks):
+    """Whole chunks, a ragged last chunk, one or two groups of heads; the
+    chunk-parallel passes (with a workspace) and the in-order kernel."""
     inp = gen.ssd_inputs(2, L, 4, 64, G, N, seed=700 + L + N + G)
-    y, last = mss.ssd_fwd(**_dev(inp))
+    y, last = mss.ssd_fwd(**_dev(inp), workspace="auto" if chunks == "parallel" else None)
     torch.cuda.synchronize()
     assert mss.get_device_error() == 0
     y_ref, last_ref = _ref(inp)
@@ -49,11 +51,12 @@ def test_ssd_starting_state_and_chaining():
     inp = gen.ssd_inputs(2, 320, 4, 64, 1, 128, seed=720)
     h0 = np.random.default_rng(721).standard_normal((2, 4, 128, 64)).astype(np.float32) * 0.1
     d = _dev(inp)
-    y, last = mss.ssd_fwd(**d, initial_state=torch.from_numpy(h0).to(DEV))
-    torch.cuda.synchronize()
     y_ref, last_ref = _ref(inp, h0=h0.astype(np.float64))
-    assert_close(to_numpy(y), y_ref, "bf16", "y from a starting state")
-    assert_close(to_numpy(last), last_ref, "bf16", "last_state from a starting state")
+    for ws in ("auto", None):
+        y, last = mss.ssd_fwd(**d, initial_state=torch.from_numpy(h0).to(DEV), workspace=ws)
+        torch.cuda.synchronize()
+        assert_close(to_numpy(y), y_ref, "bf16", f"y from a starting state (workspace {ws})")
+        assert_close(to_numpy(last), last_ref, "bf16", f"last_state from a starting state (workspace {ws})")
     # two calls chained through last_state equal one call
     part = lambda t0, t1: {k: (v[:, t0:t1].contiguous() if k in ("x", "dt", "B", "C", "z") else v)
                            for k, v in d.items()}
@@ -65,6 +68,20 @@ def test_ssd_starting_state_and_chaining():
     assert_close(to_numpy(last1), to_numpy(last_all).astype(np.float64), "bf16", "chained state")
 
 
+def test_ssd_workspace_only_when_it_pays():
+    """Few (batch, head) pairs take the chunk-parallel passes, many the
+    in-order kernel; both give the oracle's result."""
+    sms = torch.cuda.get_device_properties(0).multi_processor_count
+    assert mss.load_library().mss_ssd_fwd_workspace_size(1, 4096, 4, 64, 1, 128) > 0
+    assert mss.load_library().mss_ssd_fwd_workspace_size(4, 4096, sms, 64, 1, 128) == 0
+    inp = gen.ssd_inputs(1, 1024, 2, 64, 1, 128, seed=735)
+    y, last = mss.ssd_fwd(**_dev(inp))
+    torch.cuda.synchronize()
+    y_ref, last_ref = _ref(inp)
+    assert_close(to_numpy(y), y_ref, "bf16", "few heads y")
+    assert_close(to_numpy(last), last_ref, "bf16", "few heads last_state")
+
+
 def test_ssd_without_optional_inputs():
     inp = gen.ssd_inputs(1, 256, 2, 64, 1, 64, seed=730)
     y, last = mss.ssd_fwd(**_dev(inp, gate=False, with_D=False, with_bias=False))
@@ -74,10 +91,15 @@ def test_ssd_without_optional_inputs():
     assert_close(to_numpy(last), last_ref, "bf16", "bare last_state")
 
 
-def test_ssd_workload_sampled_heads():
-    """The bench workload (4 x 4096 tokens, 64 heads of 64, N = 128): y and
+@pytest.mark.parametrize("batch", [4, 1])
+def test_ssd_workload_sampled_heads(batch):
+    """The bench workload (4 x 4096 tokens, 64 heads of 64, N = 128; the
+    in-order kernel) and one sequence of it (the chunk-parallel passes): y and
     the final state of sampled (batch, head) pairs against the oracle."""
-    s = gen.SSD_SHAPES[gen.SSD_WORKLOAD]
+    s = dict(gen.SSD_SHAPES[gen.SSD_WORKLOAD], batch=batch)
+    ws = mss.load_library().mss_ssd_fwd_workspace_size(batch, s["seqlen"], s["nheads"], s["headdim"],
+                                                        s["ngroups"], s["dstate"])
+    assert (ws > 0) == (batch == 1)
     inp = gen.ssd_inputs(**s)
     y, last = mss.ssd_fwd(**_dev(inp))
     torch.cuda.synchronize()
