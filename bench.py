@@ -308,6 +308,50 @@ def run_reference(args, rank):
 # ---------------------------------------------------------------------------
 # The CUDA path.
 
+def kernel_only(args, mss, d, y, state, w, dev, to_dev, rank):
+    """warmup + steps launches of one kernel on its workload, nothing timed
+    and no JSON line: the command that profiler captures run."""
+    import torch
+
+    n = args.warmup + args.steps
+    if args.kernel == "forward":
+        for _ in range(n):
+            mss.scan_fwd(**d, y=y, last_state=state)
+        what = f"{w.batch}x{w.dim}x{w.dstate}x{w.seqlen}"
+    elif args.kernel == "backward":
+        dy_h, dlast_h = gen.upstream_gradients(w.batch, w.dim, w.dstate, w.seqlen, w.dtype, rank_seed(w.seed, rank))
+        dy_d, dlast_d = to_dev(dy_h), torch.from_numpy(dlast_h).to(dev)
+        ws = torch.empty(mss.bwd_workspace_size(w.batch, w.dim, w.dstate, w.seqlen), dtype=torch.uint8, device=dev)
+        for _ in range(n):
+            mss.scan_bwd(**d, dy=dy_d, dlast=dlast_d, workspace=ws)
+        what = f"{w.batch}x{w.dim}x{w.dstate}x{w.seqlen}"
+    elif args.kernel == "decode":
+        dw = gen.WORKLOADS[gen.DECODE_WORKLOAD]
+        A5, D5, b5 = (torch.from_numpy(x).to(dev) for x in gen.channel_params(dw.dim, dw.dstate, dw.d_skip, dw.seed))
+        st5 = torch.zeros(dw.batch, dw.dim, dw.dstate, device=dev)
+        steps5 = [{k: to_dev(v) for k, v in gen.decode_step_inputs(dw.batch, dw.dim, dw.dstate, dw.dtype,
+                                                                  dw.seed, t).items()} for t in range(4)]
+        y5 = torch.empty(dw.batch, dw.dim, dtype=torch.bfloat16, device=dev)
+        for t in range(n):
+            mss.state_update(st5, A=A5, D=D5, delta_bias=b5, y=y5, **steps5[t % 4])
+        what = f"{dw.batch}x{dw.dim}x{dw.dstate}"
+    else:
+        ss = dict(gen.SSD_SHAPES[gen.SSD_WORKLOAD])
+        if args.seqlen:
+            ss["seqlen"] = args.seqlen
+        sin = gen.ssd_inputs(**ss)
+        sd = dict(x=to_dev(sin["x"]), dt=to_dev(sin["dt"]), A=torch.from_numpy(sin["A"]).to(dev),
+                  B=to_dev(sin["B"]), C=to_dev(sin["C"]), D=torch.from_numpy(sin["D"]).to(dev),
+                  z=to_dev(sin["z"]), dt_bias=torch.from_numpy(sin["dt_bias"]).to(dev))
+        for _ in range(n):
+            mss.ssd_fwd(**sd)
+        what = "x".join(str(ss[k]) for k in ("batch", "seqlen", "nheads", "headdim", "dstate"))
+    torch.cuda.synchronize(dev)
+    assert mss.get_device_error() == 0
+    log(f"kernel-only: {n} {args.kernel} launches on {what}")
+    return 0
+
+
 def run_mss(args, rank, world, local_rank):
     import torch
     import torch.distributed as dist
@@ -381,13 +425,7 @@ def run_mss(args, rank, world, local_rank):
 
     assert mss.get_device_error() == 0
     if args.kernel_only:
-        # forward launches only (used for profiling captures): no JSON line
-        for _ in range(args.warmup + args.steps):
-            mss.scan_fwd(**d, y=y, last_state=state)
-        torch.cuda.synchronize(dev)
-        assert mss.get_device_error() == 0
-        log(f"kernel-only: {args.warmup + args.steps} forward launches on {w.batch}x{w.dim}x{w.dstate}x{w.seqlen}")
-        return 0
+        return kernel_only(args, mss, d, y, state, w, dev, to_dev, rank)
     # the timed run keeps the clock sampler busy for at least ~2 s
     k_clock = args.steps
     ms, fwd_ms, clocks = timed(0, k_clock, args.warmup, with_clocks=True)
@@ -636,8 +674,11 @@ def main():
     ap.add_argument("--impl", choices=["mss", "reference"], default="mss")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--kernel-only", action="store_true",
-                    help="only launch the forward kernel (warmup + steps times); for profiler captures")
-    ap.add_argument("--seqlen", type=int, default=0, help="override the workload's sequence length")
+                    help="only launch one kernel (warmup + steps times); for profiler captures")
+    ap.add_argument("--kernel", choices=["forward", "backward", "decode", "ssd"], default="forward",
+                    help="which kernel --kernel-only launches")
+    ap.add_argument("--seqlen", type=int, default=0,
+                    help="override the workload's sequence length (the SSD workload's with --kernel ssd)")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be at least 3")

@@ -327,7 +327,7 @@ MSS_API int mss_ssd_fwd(const void *x, const void *dt, const float *A, const voi
  * chunk states, chunk outputs) instead of one CTA walking a head's chunks in
  * order; otherwise the workspace is not used (the passes' extra state
  * traffic would cost more than they gain).  On a 148-SM B200 the passes run
- * for 1-230 pairs and 297-417, for instance, not for 231-296;
+ * for up to 115 pairs;
  * mss_ssd_fwd_workspace_size returns 0 where the workspace goes unused.
  * Same result up to rounding; a NULL workspace is mss_ssd_fwd.
  * MSS_ERR_WORKSPACE if it is too small. */

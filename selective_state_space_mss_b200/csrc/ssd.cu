@@ -37,9 +37,9 @@ int launch_ssd(const mss::SsdParams& p, int dstate, cudaStream_t s) {
 // Cost model for choosing between the two forms, from B200 timings at 4096
 // tokens (headdim 64, dstate 128).  The in-order kernel runs one CTA per
 // (batch, head), up to two per SM: a wave in which some SM holds two takes
-// about 1.23 times as long as one in which none does (740 vs 600 us).  The
-// chunk-parallel passes spread every chunk over all SMs and take about
-// 0.79 of that lone-CTA time per SM's worth of heads (3.2 us per head on 148
+// about 1.24 times as long as one in which none does (460 vs 370 us).  The
+// chunk-parallel passes spread every chunk over all SMs and take about 1.28
+// of that lone-CTA time per SM's worth of heads (3.2 us per head on 148
 // SMs).  Both scale with the sequence length, so the comparison does not.
 bool ssd_chunked_pays(int64_t batch, int64_t nheads) {
     static std::mutex mu;
@@ -51,8 +51,8 @@ bool ssd_chunked_pays(int64_t batch, int64_t nheads) {
     const int64_t pairs = batch * nheads;
     if (sms <= 0 || pairs <= 0) return false;
     const int64_t full = (pairs - 1) / (2 * sms), rest = pairs - full * 2 * sms;
-    const int64_t in_order = full * 123 + (rest > sms ? 123 : 100);  // hundredths of a lone-CTA pass
-    const int64_t chunked = 79 * pairs / sms;
+    const int64_t in_order = full * 124 + (rest > sms ? 124 : 100);  // hundredths of a lone-CTA pass
+    const int64_t chunked = 128 * pairs / sms;
     return chunked < in_order;
 }
 

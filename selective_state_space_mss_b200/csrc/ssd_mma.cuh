@@ -55,7 +55,11 @@ struct SsdLayout {
     static constexpr int kXw = kSs;
     static_assert(kXBytes <= kSBytes, "X fits where the state copy was");
     static constexpr int kScal = kSs + kSBytes;        // per token: Delta, cs (fp32)
-    static constexpr int kSmemBytes = kScal + 2 * kQ * 4;
+    // z of the current chunk, 128-byte rows with 16-byte pieces swizzled
+    // (piece k of row r at k ^ (r & 7)); each warp copies and reads its own 16 rows
+    static constexpr int kZ = kScal + 2 * kQ * 4;
+    static constexpr int kZBytes = kQ * kP * 2;
+    static constexpr int kSmemBytes = kZ + kZBytes;    // 115,200 B at N = 128: two CTAs per SM
 };
 
 __device__ __forceinline__ uint32_t smem_u32(const void* p) {
@@ -160,22 +164,31 @@ __global__ void __launch_bounds__(128) ssd_fwd_kernel(SsdParams p) {
         }
         cp_async_commit();
     };
-    // step sizes of chunk c's tokens, two a lane of warp 0
-    auto load_dt = [&](int64_t c, float (&dv)[2]) {
+    // raw step inputs of chunk c's tokens, two a lane of warp 0 (read one chunk
+    // ahead; the softplus is taken when they are used)
+    auto load_dt = [&](int64_t c, bf16_t (&dv)[2]) {
         const int64_t t0 = c * Q;
         const int q = int(min(int64_t(Q), L - t0));
 #pragma unroll
         for (int k = 0; k < 2; ++k) {
             const int r = 2 * lane + k;
-            float d = 0.f;
-            if (r < q) {
-                const float sraw = to_f32(dtp[(b * L + t0 + r) * H + h]) + bias;
-                d = kSoftplus ? softplus_fast(sraw) : sraw;
-            }
-            dv[k] = d;
+            dv[k] = r < q ? dtp[(b * L + t0 + r) * H + h] : bf16_t{0};
         }
     };
-    float dnext[2] = {0.f, 0.f};
+    // this warp's 16 rows of z for chunk c: four 16-byte pieces a lane
+    bf16_t* Zs = reinterpret_cast<bf16_t*>(smem + Ly::kZ) + warp * 16 * P;
+    auto issue_z = [&](int64_t c) {
+        const int64_t t0 = c * Q;
+        const int q = int(min(int64_t(Q), L - t0));
+#pragma unroll
+        for (int k = 0; k < 4; ++k) {
+            const int piece = lane + 32 * k, r = piece >> 3, k8 = piece & 7;
+            const int i = warp * 16 + r, ii = i < q ? i : 0;
+            cp_async16(Zs + r * P + ((k8 ^ (r & 7)) << 3), zp + ((b * L + t0 + ii) * H + h) * P + k8 * 8,
+                       i < q ? 16u : 0u);
+        }
+    };
+    bf16_t dnext[2] = {bf16_t{0}, bf16_t{0}};
     if (n_chunks > 0) {
         issue(0);
         if (warp == 0) load_dt(0, dnext);
@@ -184,8 +197,15 @@ __global__ void __launch_bounds__(128) ssd_fwd_kernel(SsdParams p) {
         const int64_t t0 = c * Q;
         const int q = int(min(int64_t(Q), L - t0));
         __syncthreads();  // the previous chunk's reads of shared memory are done
-        // the next chunk's copies run during this chunk
-        if (c + 1 < n_chunks) issue(c + 1);
+        // this chunk's z (read by the output) and the next chunk's X, B, C
+        // run during this chunk; two commit groups every chunk (the second
+        // may be empty), so the waits below count the same way each time
+        if constexpr (kGate) issue_z(c);
+        cp_async_commit();
+        if (c + 1 < n_chunks)
+            issue(c + 1);
+        else
+            cp_async_commit();
         const bf16_t* Xs = buf_x(c);
         const bf16_t* Bs = buf_b(c);
         const bf16_t* Cs = buf_c(c);
@@ -203,7 +223,12 @@ __global__ void __launch_bounds__(128) ssd_fwd_kernel(SsdParams p) {
         // step sizes and the running sum of Delta A (warp 0: two tokens a lane);
         // the next chunk's step sizes are read now, used then
         if (warp == 0) {
-            float dv[2] = {dnext[0], dnext[1]}, cv[2];
+            float dv[2], cv[2];
+#pragma unroll
+            for (int k = 0; k < 2; ++k) {
+                const float sraw = to_f32(dnext[k]) + bias;
+                dv[k] = 2 * lane + k < q ? (kSoftplus ? softplus_fast(sraw) : sraw) : 0.f;
+            }
             if (c + 1 < n_chunks) load_dt(c + 1, dnext);
             cv[0] = dv[0] * Ah;
             cv[1] = cv[0] + dv[1] * Ah;
@@ -219,11 +244,8 @@ __global__ void __launch_bounds__(128) ssd_fwd_kernel(SsdParams p) {
             css[2 * lane] = before + cv[0];
             css[2 * lane + 1] = before + cv[1];
         }
-        // this chunk's copies have landed (the next chunk's may still run)
-        if (c + 1 < n_chunks)
-            cp_async_wait<1>();
-        else
-            cp_async_wait<0>();
+        // this chunk's X, B, C have landed (its z and the next chunk's copies may still run)
+        cp_async_wait<2>();
         __syncthreads();
         const float cs_last = css[Q - 1];
 
@@ -294,6 +316,10 @@ __global__ void __launch_bounds__(128) ssd_fwd_kernel(SsdParams p) {
             }
         }
         // output: y = Y_intra + exp(cs_i) C S_prev + D x, gated
+        if constexpr (kGate) {
+            cp_async_wait<1>();  // this lane's pieces of z
+            __syncwarp();        // and its warp's
+        }
         {
             const float e0 = __expf(csi0), e1 = __expf(csi1);
 #pragma unroll
@@ -309,7 +335,9 @@ __global__ void __launch_bounds__(128) ssd_fwd_kernel(SsdParams p) {
                     float o1 = yi[pt][2 * hr + 1] + ex * ye[pt][2 * hr + 1] + Dh * bf16_hi(xw);
                     const int64_t off = ((b * L + t0 + i) * H + h) * P + pc;
                     if constexpr (kGate) {
-                        const uint32_t zw = *reinterpret_cast<const uint32_t*>(zp + off);
+                        const int r = gq + 8 * hr;  // row in the warp's z rows; r & 7 = gq
+                        const uint32_t zw =
+                            *reinterpret_cast<const uint32_t*>(Zs + r * P + ((pt ^ gq) << 3) + 2 * tq);
                         o0 *= silu_fast(bf16_lo(zw));
                         o1 *= silu_fast(bf16_hi(zw));
                     }
