@@ -494,25 +494,31 @@ def run_mss(args, rank, world, local_rank):
     bwd_ms = [a_.elapsed_time(b_) for a_, b_ in bwd_ev]
     assert mss.get_device_error() == 0
 
-    # end to end through the public call with host buffers: pinned host inputs,
-    # copies in, forward + decode token, results copied out, every step
+    # end to end through the public calls with host buffers, every step: the
+    # forward pass over pinned host inputs and outputs (mss_scan_fwd_host:
+    # the library copies pieces in, runs them and copies y and last_state out,
+    # overlapping the two directions), then the decode token from that state
+    # (state and token inputs copied in, y and the new state copied out)
     host = {k: v.cpu().pin_memory() for k, v in d.items()}
     host1 = {k: v.cpu().pin_memory() for k, v in s1.items()}
     y_host = torch.empty(y.shape, dtype=y.dtype, pin_memory=True)
     st_host = torch.empty(state.shape, dtype=state.dtype, pin_memory=True)
+    st1_host = torch.empty(state.shape, dtype=state.dtype, pin_memory=True)
     y1_host = torch.empty(y1.shape, dtype=y1.dtype, pin_memory=True)
-    h2d = sum(v.numel() * v.element_size() for v in list(host.values()) + list(host1.values()))
-    d2h = y_host.numel() * 2 + st_host.numel() * 4 + y1_host.numel() * 2
+    ws_host = torch.empty(int(mss.load_library().mss_scan_fwd_host_workspace_size(
+        w.batch, w.dim, w.dstate, w.seqlen, mss.DTYPE_BF16, 1, 1, 1, 0, 1)), dtype=torch.uint8, device=dev)
+    h2d = (sum(v.numel() * v.element_size() for v in list(host.values()) + list(host1.values()))
+           + st_host.numel() * 4)
+    d2h = y_host.numel() * 2 + st_host.numel() * 4 + y1_host.numel() * 2 + st1_host.numel() * 4
 
     def e2e_step():
-        for k_, v in host.items():
-            d[k_].copy_(v, non_blocking=True)
+        mss.scan_fwd_host(**host, y=y_host, last_state=st_host, workspace=ws_host, device=dev)
+        state.copy_(st_host, non_blocking=True)
         for k_, v in host1.items():
             s1[k_].copy_(v, non_blocking=True)
-        step(0)
-        y_host.copy_(y, non_blocking=True)
-        st_host.copy_(state, non_blocking=True)
+        mss.state_update(state, A=d["A"], D=d["D"], delta_bias=d["delta_bias"], y=y1, **s1)
         y1_host.copy_(y1, non_blocking=True)
+        st1_host.copy_(state, non_blocking=True)
 
     for _ in range(max(1, args.warmup)):
         e2e_step()

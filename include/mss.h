@@ -56,7 +56,7 @@
 extern "C" {
 #endif
 
-#define MSS_VERSION 10400 /* major*10000 + minor*100 + patch: 1.4.0 */
+#define MSS_VERSION 10500 /* major*10000 + minor*100 + patch: 1.5.0 */
 
 enum mss_dtype {
     MSS_DTYPE_F32 = 0,
@@ -164,6 +164,47 @@ MSS_API int mss_scan_fwd_ex2(const void *u, const void *delta, const float *A, c
  */
 MSS_API int64_t mss_scan_fwd_workspace_size(int64_t batch, int64_t dim, int64_t dstate, int64_t seqlen,
                                             int dtype, unsigned flags);
+
+/*
+ * mss_scan_fwd_host -- mss_scan_fwd_ex2 over inputs and outputs in HOST
+ * memory: u, delta, A, B, C, D, z, delta_bias, initial_state are read from
+ * the host, y and last_state written to the host, with the layouts of
+ * mss_scan_fwd.  The channels are cut into pieces of whole batch rows or
+ * parts of them.  Each piece is staged through a caller-owned device
+ * workspace.  The library's own streams on the current device then overlap
+ * the host-to-device copies of one piece, the kernel of the one before it,
+ * and the device-to-host copies of the one before that.
+ *
+ *   workspace, workspace_bytes : device memory on the current device,
+ *       256-byte aligned, at least mss_scan_fwd_host_workspace_size bytes
+ *       for the same sizes and the same optional arguments (else
+ *       MSS_ERR_NULL / MSS_ERR_ALIGN / MSS_ERR_WORKSPACE).  Its contents on
+ *       return are unspecified.
+ *   stream : the call is asynchronous on it like every other entry point.
+ *       The copies wait for the work already queued on it, and work queued
+ *       on it later waits for the last copy out.  The host buffers must
+ *       stay valid and untouched until then.  Page-locked (pinned) host
+ *       memory is needed for the copies to overlap.  Pageable memory works
+ *       but is copied synchronously.
+ *
+ * The kernels run with MSS_FLAG_NO_SPLIT added to flags (the pieces, not a
+ * sequence split, fill the GPU).  y and last_state must not overlap the host
+ * inputs.  Returns MSS_OK or a negative mss_status; argument errors are
+ * found before anything is queued.
+ */
+MSS_API int mss_scan_fwd_host(const void *u, const void *delta, const float *A, const void *B,
+                              const void *C, const float *D, const void *z, const float *delta_bias,
+                              int softplus_flag, const float *initial_state, void *y, float *last_state,
+                              int64_t batch, int64_t dim, int64_t dstate, int64_t seqlen,
+                              int dtype, unsigned flags, void *workspace, int64_t workspace_bytes,
+                              void *stream);
+
+/* Device workspace bytes mss_scan_fwd_host needs for these sizes, with z, D,
+ * delta_bias, initial_state and last_state present (nonzero) or NULL (0);
+ * 0 when batch * dim == 0, or a negative mss_status. */
+MSS_API int64_t mss_scan_fwd_host_workspace_size(int64_t batch, int64_t dim, int64_t dstate, int64_t seqlen,
+                                                 int dtype, int with_z, int with_D, int with_delta_bias,
+                                                 int with_initial_state, int with_last_state);
 
 /*
  * mss_scan_fwd_conv -- the forward pass with a causal convolution and SiLU

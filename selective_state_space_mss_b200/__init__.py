@@ -22,7 +22,7 @@ import threading
 
 import torch
 
-__all__ = ["scan_fwd", "scan_fwd_conv", "scan_bwd", "ssd_fwd", "bwd_workspace_size", "state_update", "state_update_conv",
+__all__ = ["scan_fwd", "scan_fwd_host", "scan_fwd_conv", "scan_bwd", "ssd_fwd", "bwd_workspace_size", "state_update", "state_update_conv",
            "get_device_error",
            "library_path", "workspace_size",
            "FLAG_GENERAL_A", "FLAG_SIMPLE", "FLAG_NO_SPLIT", "FLAG_ZOH_INPUT", "MssError", "load_library"]
@@ -99,6 +99,11 @@ def load_library():
             lib.mss_state_update_conv.argtypes = [fp, vp, vp, fp, fp, i, vp, fp, vp, vp, fp, vp, fp, i, vp,
                                                   i64, i64, i64, i, u32, vp]
             lib.mss_state_update_conv.restype = i
+            lib.mss_scan_fwd_host.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, i, vp, vp, vp,
+                                              i64, i64, i64, i64, i, u32, vp, i64, vp]
+            lib.mss_scan_fwd_host.restype = i
+            lib.mss_scan_fwd_host_workspace_size.argtypes = [i64, i64, i64, i64, i, i, i, i, i, i]
+            lib.mss_scan_fwd_host_workspace_size.restype = i64
             lib.mss_get_device_error.argtypes = [vp]
             lib.mss_get_device_error.restype = i
             lib.mss_strerror.argtypes = [i]
@@ -209,6 +214,61 @@ def scan_fwd(u, delta, A, B, C, D=None, z=None, delta_bias=None, softplus=True,
         _stream_handle(stream, dev))
     if rc != 0:
         raise MssError(rc, "mss_scan_fwd")
+    return y, last_state
+
+
+def scan_fwd_host(u, delta, A, B, C, D=None, z=None, delta_bias=None, softplus=True,
+                  y=None, last_state=None, want_last_state=True, initial_state=None,
+                  workspace="auto", flags=0, device=None, stream=None):
+    """The forward pass over CPU tensors (mss_scan_fwd_host): the library
+    copies the inputs to `device` piece by piece through a device workspace,
+    runs the kernels and copies y and last_state back, overlapping the copies
+    of different pieces with each other and with the kernels.  Inputs and
+    outputs are CPU tensors in the layouts of scan_fwd.  Pinned memory is
+    needed for the overlap, and outputs created here are pinned.  The call is
+    asynchronous on `stream` (default: the current stream of `device`), so
+    the outputs are complete only after that stream has been synchronised.
+    Returns (y, last_state)."""
+    if not isinstance(u, torch.Tensor) or u.device.type != "cpu":
+        raise ValueError("u must be a CPU tensor (scan_fwd takes CUDA tensors)")
+    if u.dim() != 3 or A.dim() != 2:
+        raise ValueError("u must be [batch, dim, L] and A [dim, N]")
+    batch, dim, L = u.shape
+    N = A.shape[1]
+    cpu, dt = torch.device("cpu"), u.dtype
+    code = _io_dtype(u)
+    dev = torch.device("cuda", torch.cuda.current_device()) if device is None else torch.device(device)
+    for t, name, shape, typ, opt in ((u, "u", (batch, dim, L), dt, False), (delta, "delta", (batch, dim, L), dt, False),
+                                     (A, "A", (dim, N), torch.float32, False), (B, "B", (batch, N, L), dt, False),
+                                     (C, "C", (batch, N, L), dt, False), (D, "D", (dim,), torch.float32, True),
+                                     (z, "z", (batch, dim, L), dt, True),
+                                     (delta_bias, "delta_bias", (dim,), torch.float32, True),
+                                     (initial_state, "initial_state", (batch, dim, N), torch.float32, True)):
+        _check(t, name, shape, typ, cpu, optional=opt)
+    if y is None:
+        y = torch.empty((batch, dim, L), dtype=dt, pin_memory=True)
+    _check(y, "y", (batch, dim, L), dt, cpu)
+    if last_state is None and want_last_state:
+        last_state = torch.empty((batch, dim, N), dtype=torch.float32, pin_memory=True)
+    _check(last_state, "last_state", (batch, dim, N), torch.float32, cpu, optional=True)
+    lib = load_library()
+    with torch.cuda.device(dev):
+        if isinstance(workspace, str):
+            if workspace != "auto":
+                raise ValueError("workspace must be 'auto' or a uint8 CUDA tensor")
+            nbytes = int(lib.mss_scan_fwd_host_workspace_size(
+                batch, dim, N, L, code, int(z is not None), int(D is not None), int(delta_bias is not None),
+                int(initial_state is not None), int(last_state is not None)))
+            if nbytes < 0:
+                raise MssError(nbytes, "mss_scan_fwd_host_workspace_size")
+            workspace = torch.empty(max(nbytes, 1), dtype=torch.uint8, device=dev)
+        _check(workspace, "workspace", (workspace.numel(),), torch.uint8, dev)
+        rc = lib.mss_scan_fwd_host(
+            _ptr(u), _ptr(delta), _ptr(A), _ptr(B), _ptr(C), _ptr(D), _ptr(z), _ptr(delta_bias),
+            int(bool(softplus)), _ptr(initial_state), _ptr(y), _ptr(last_state), batch, dim, N, L, code,
+            int(flags), _ptr(workspace), workspace.numel(), _stream_handle(stream, dev))
+    if rc != 0:
+        raise MssError(rc, "mss_scan_fwd_host")
     return y, last_state
 
 

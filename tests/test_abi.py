@@ -314,3 +314,47 @@ def test_ssd_workspace_queries(lib):
                             v(P + 0x6000000), ctypes.c_int64(100), None)
     # too small (checked before any launch), or no device to launch on
     assert rc == (codes["MSS_ERR_WORKSPACE"] if ws else codes["MSS_ERR_CUDA"])
+
+
+def test_host_call_argument_errors(lib):
+    """mss_scan_fwd_host: every error below is found before anything is
+    queued (the pointers are made up and never dereferenced)."""
+    codes = _enum("mss_status")
+    v = ctypes.c_void_p
+    lib.mss_scan_fwd_host_workspace_size.restype = ctypes.c_int64
+    need = lib.mss_scan_fwd_host_workspace_size(ctypes.c_int64(2), ctypes.c_int64(8), ctypes.c_int64(16),
+                                                ctypes.c_int64(32), 1, 0, 0, 0, 0, 0)
+    # A, B, C once; one slot is u, delta, y (8 channels x 32 tokens of bf16,
+    # each rounded up to 256 bytes); three slots
+    assert need == 512 + 2 * 2048 + 3 * 3 * 512
+
+    def host(**kw):
+        a = dict(u=P, delta=P + 0x1000000, A=P + 0x2000000, B=P + 0x3000000, C=P + 0x4000000,
+                 y=P + 0x5000000, last=None, ws=P + 0x6000000, wsb=need, batch=2, dim=8, N=16, L=32,
+                 dtype=1, flags=0)
+        a.update(kw)
+        w = lambda x: v(x) if x is not None else None
+        return lib.mss_scan_fwd_host(w(a["u"]), w(a["delta"]), w(a["A"]), w(a["B"]), w(a["C"]), None, None,
+                                     None, 1, None, w(a["y"]), w(a["last"]), ctypes.c_int64(a["batch"]),
+                                     ctypes.c_int64(a["dim"]), ctypes.c_int64(a["N"]), ctypes.c_int64(a["L"]),
+                                     a["dtype"], a["flags"], w(a["ws"]), ctypes.c_int64(a["wsb"]), None)
+
+    assert host(dtype=5) == codes["MSS_ERR_DTYPE"]
+    assert host(flags=0x40) == codes["MSS_ERR_FLAGS"]
+    assert host(batch=-1) == codes["MSS_ERR_SHAPE"]
+    assert host(N=3) == codes["MSS_ERR_UNSUPPORTED_N"]
+    assert host(u=None) == codes["MSS_ERR_NULL"]
+    assert host(ws=None) == codes["MSS_ERR_NULL"]
+    assert host(u=P + 1) == codes["MSS_ERR_ALIGN"]
+    assert host(ws=P + 0x6000010) == codes["MSS_ERR_ALIGN"]        # 16 but not 256-byte aligned
+    assert host(y=P + 0x1000000) == codes["MSS_ERR_ALIAS"]         # y on delta
+    assert host(last=P + 0x5000000) == codes["MSS_ERR_ALIAS"]      # last_state on y
+    assert host(wsb=need - 1) == codes["MSS_ERR_WORKSPACE"]
+    assert host(batch=0) == 0
+    q = lambda *a: lib.mss_scan_fwd_host_workspace_size(*[ctypes.c_int64(x) for x in a[:4]], *a[4:])
+    assert q(0, 8, 16, 32, 1, 1, 1, 1, 1, 1) == 0
+    assert q(2, 8, 16, 32, 9, 0, 0, 0, 0, 0) == codes["MSS_ERR_DTYPE"]
+    assert q(2, 8, 5, 32, 1, 0, 0, 0, 0, 0) == codes["MSS_ERR_UNSUPPORTED_N"]
+    # every optional input adds its own piece: z one more [8 x 32] slot tensor,
+    # D and bias [dim] floats, the two states [8 x 16] floats per slot
+    assert q(2, 8, 16, 32, 1, 1, 1, 1, 1, 1) == need + 3 * 512 + 2 * 256 + 3 * 2 * 512
