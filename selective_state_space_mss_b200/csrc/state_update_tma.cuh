@@ -5,19 +5,22 @@
 // (64 B at N = 16) and moves a few bytes of u, delta, z and y.  Plain loads
 // keep one 16-byte vector per thread in flight, which on B200 is not enough
 // to cover the memory latency at full bandwidth.  Here a persistent CTA walks
-// tiles of 1024/N consecutive channels (4 KB of state) of one batch row
-// through a ring of
-// kStages shared-memory stages: one thread issues cp.async.bulk loads of the
-// tile's state, u, delta and z a few tiles ahead (kStages - 1 tiles, 4.5 KB
-// each, in flight per CTA), all threads update the state in place in shared
-// memory and write y there, and the same thread stores both back with bulk
-// copies, so that neither direction occupies registers while in flight.
+// tiles of 2048/N consecutive channels (8 KB of state) of one batch row
+// through a ring of kStages shared-memory stages: one thread issues
+// cp.async.bulk loads of the tile's state, u, delta and z a few tiles ahead
+// (kStages - 1 tiles, about 9 KB each, in flight per CTA), all threads update
+// the state in place in shared memory and write y there, and the same thread
+// stores both back with bulk copies, so that neither direction occupies
+// registers while in flight.  A B200 sweep of the tile and ring sizes on
+// 256 x 5120 x 16 (one token, L2 flushed) picked 8 KB tiles and three stages:
+// 38.9 us, against 43.0 us for 4 KB tiles (three or four stages) and 49 us
+// or more for 16 KB tiles or two stages.
 //
 // With the causal convolution in front, the tile's conv state (K-1 inputs per
 // channel) travels with it and is shifted in shared memory.
 //
 // Requirements (checked by the host): N in {4, 8, 16}; dim a multiple of
-// 1024/N; state, A, u, delta, z, y and the conv state 16-byte aligned
+// 2048/N; state, A, u, delta, z, y and the conv state 16-byte aligned
 // (otherwise the host runs state_update_kernel).  Waits on the stage
 // barriers are bounded.
 #pragma once
@@ -31,12 +34,12 @@ namespace mss {
 template <typename T, int N>
 struct DecodeTile {
     static_assert(N == 4 || N == 8 || N == 16, "bulk-staged decode supports N = 4, 8, 16");
-    static constexpr int kRows = 1024 / N;                   // channels per tile
-    static constexpr int kStateBytes = kRows * N * 4;        // 4 KB
+    static constexpr int kRows = 2048 / N;                   // channels per tile
+    static constexpr int kStateBytes = kRows * N * 4;        // 8 KB
     static constexpr int kIoBytes = kRows * int(sizeof(T));  // one of u, delta, z, y
     static constexpr int kConvOffset = kStateBytes + 4 * kIoBytes;  // conv state: up to 3 inputs per channel
     static constexpr int kStageBytes = kConvOffset + 3 * kIoBytes;
-    static constexpr int kStages = 4;
+    static constexpr int kStages = 3;
     static constexpr int kThreads = 128;
     static constexpr int kTPC = N / 4;                               // threads per channel
     static constexpr int kSlots = kStateBytes / 16 / kThreads;       // float4 slots per thread per tile

@@ -130,10 +130,10 @@ def test_conv_short_and_empty_sequences(dtype):
 @pytest.mark.parametrize("K", [1, 2, 4])
 @pytest.mark.parametrize("dim_kind", ["tiles", "ragged"])
 def test_conv_decode_matches_oracle(dtype, N, K, dim_kind):
-    """Both decode kernels: whole 4 KB state tiles (bulk-staged) and a
+    """Both decode kernels: whole 8 KB state tiles (bulk-staged) and a
     channel count that is not (per-thread)."""
     batch, steps = 3, 6
-    dim = 2 * 1024 // N if dim_kind == "tiles" else 37
+    dim = 2 * 2048 // N if dim_kind == "tiles" else 37
     A, D, bias = gen.channel_params(dim, N, "normal", 450 + N)
     w, b = gen.conv_params(dim, K, 451)
     h0 = gen.initial_state(batch, dim, N, 452, "normal")

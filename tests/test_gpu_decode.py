@@ -103,10 +103,10 @@ def test_decode_workload_sampled_every_step():
 @pytest.mark.parametrize("zoh", [False, True])
 @pytest.mark.parametrize("gate", [True, False])
 def test_decode_staged_path_matches_oracle(dtype, N, zoh, gate):
-    """Shapes whose channel count is a whole number of 4 KB state tiles
-    (1024/N channels) take the bulk-staged decode kernel; several batch rows
+    """Shapes whose channel count is a whole number of 8 KB state tiles
+    (2048/N channels) take the bulk-staged decode kernel; several batch rows
     per channel block, several channel blocks, and more steps than stages."""
-    batch, dim, steps = 5, 2 * 1024 // N, 6
+    batch, dim, steps = 5, 2 * 2048 // N, 6
     A, D, bias = gen.channel_params(dim, N, "normal", 90 + N)
     h0 = gen.initial_state(batch, dim, N, 91, "normal")
     state = torch.from_numpy(h0.copy()).to(DEV)
