@@ -474,6 +474,12 @@ def run_mss(args, rank, world, local_rank):
     del sd, ssd_y, sin
     # matrix-form flops per (token, head): C B^T and M X within the chunk, C S
     # and the state product B^T X across chunks (chunk of 64, P = 64)
+    # algorithmic bytes: x, z read and y written (bf16), dt read, B and C read
+    # once per (batch, token, group), A, D, dt_bias, and last_state written
+    ssd_bytes = (3 * ss["batch"] * ss["seqlen"] * ss["nheads"] * ss["headdim"] * 2
+                 + ss["batch"] * ss["seqlen"] * ss["nheads"] * 2
+                 + 2 * ss["batch"] * ss["seqlen"] * ss["ngroups"] * ss["dstate"] * 2
+                 + 3 * ss["nheads"] * 4 + ss["batch"] * ss["nheads"] * ss["dstate"] * ss["headdim"] * 4)
     ssd_flops = ss["batch"] * ss["seqlen"] * ss["nheads"] * (
         2 * 64 * ss["dstate"] + 2 * 64 * ss["headdim"] + 2 * ss["dstate"] * ss["headdim"] * 2)
 
@@ -642,11 +648,18 @@ def run_mss(args, rank, world, local_rank):
                      "note": "gradients of u, delta, A, B, C, D, z, bias, starting state; checkpoint pass included"},
         "ssd_path": {"workload": gen.SSD_WORKLOAD, "ms_avg": ssd_ms,
                      "channel_tokens_per_s": ss["batch"] * ss["seqlen"] * ss["nheads"] * ss["headdim"] / (ssd_ms * 1e-3),
-                     "roofline": {"bound": "tensor", "achieved": ssd_flops / (ssd_ms * 1e-3) / 1e12,
-                                  "peak": measured_bf16_tflops()[0], "unit": "TFLOP/s",
-                                  "frac": ssd_flops / (ssd_ms * 1e-3) / 1e12 / measured_bf16_tflops()[0],
-                                  "peak_kind": measured_bf16_tflops()[1],
-                                  "note": "bf16 mma.sync products, fp32 accumulation"}},
+                     # the binding roof at the measured peaks: HBM (its bytes take longer
+                     # than its matrix-form flops at the bf16 GEMM rate)
+                     "roofline": {"bound": "hbm", "achieved": ssd_bytes / (ssd_ms * 1e-3) / 1e9, "peak": peak,
+                                  "unit": "GB/s", "frac": ssd_bytes / (ssd_ms * 1e-3) / 1e9 / peak,
+                                  "peak_kind": peak_kind, "algorithmic_bytes_per_launch": ssd_bytes,
+                                  "time_at_peak_us": 1e6 * ssd_bytes / (peak * 1e9)},
+                     "roofline_tensor": {"bound": "tensor", "achieved": ssd_flops / (ssd_ms * 1e-3) / 1e12,
+                                         "peak": measured_bf16_tflops()[0], "unit": "TFLOP/s",
+                                         "frac": ssd_flops / (ssd_ms * 1e-3) / 1e12 / measured_bf16_tflops()[0],
+                                         "peak_kind": measured_bf16_tflops()[1],
+                                         "time_at_peak_us": ssd_flops / (measured_bf16_tflops()[0] * 1e6),
+                                         "note": "bf16 mma.sync products, fp32 accumulation"}},
         "zoh_input_path": {"fwd_ms_avg": fwd_avg_zoh,
                            "achieved_gbs": bytes_fwd / (fwd_avg_zoh * 1e-3) / 1e9,
                            "frac": bytes_fwd / (fwd_avg_zoh * 1e-3) / 1e9 / peak,
