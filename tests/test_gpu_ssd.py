@@ -115,3 +115,28 @@ def test_ssd_workload_sampled_heads(batch):
                                          dt_bias=inp["dt_bias"][h:h + 1])
         assert_close(yn[b:b + 1, :, h:h + 1], y_ref, "bf16", f"y of (b={b}, h={h})")
         assert_close(ln[b:b + 1, h:h + 1], last_ref, "bf16", f"state of (b={b}, h={h})")
+
+
+@pytest.mark.parametrize("L", [1, 63, 65])
+@pytest.mark.parametrize("chunks", ["parallel", "in-order"])
+def test_ssd_short_and_ragged_sequences(L, chunks):
+    """One token, one token short of a chunk, one token past it; every head
+    its own group (G = H)."""
+    inp = gen.ssd_inputs(1, L, 4, 64, 4, 64, seed=750 + L)
+    y, last = mss.ssd_fwd(**_dev(inp), workspace="auto" if chunks == "parallel" else None)
+    torch.cuda.synchronize()
+    assert mss.get_device_error() == 0
+    y_ref, last_ref = _ref(inp)
+    assert_close(to_numpy(y), y_ref, "bf16", f"L={L} y")
+    assert_close(to_numpy(last), last_ref, "bf16", f"L={L} last_state")
+
+
+def test_ssd_empty_sequence_passes_the_state_on():
+    inp = gen.ssd_inputs(2, 1, 4, 64, 1, 128, seed=760)
+    d = {k: (v[:, :0].contiguous() if k in ("x", "dt", "B", "C", "z") else v) for k, v in _dev(inp).items()}
+    h0 = torch.randn(2, 4, 128, 64, device=DEV)
+    _, last = mss.ssd_fwd(**d, initial_state=h0)
+    _, last0 = mss.ssd_fwd(**d)
+    torch.cuda.synchronize()
+    assert torch.equal(last, h0)
+    assert torch.count_nonzero(last0) == 0
