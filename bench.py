@@ -268,9 +268,18 @@ def cpu_baseline(inp, target_s=10.0):
     while total_s < target_s or passes == 0:
         ct, sec = oracle_sample_rate(inp, rows, nthreads)
         total_ct, total_s, passes = total_ct + ct, total_s + sec, passes + 1
+    # the same oracle on one thread, over a few channels per batch row (about 2 s)
+    rows1 = max(1, min(inp["dim"], calibrate_rows(inp, 1, 1.0) // 2))
+    ct1, s1, passes1 = 0, 0.0, 0
+    while s1 < 2.0 or passes1 == 0:
+        ct, sec = oracle_sample_rate(inp, rows1, 1)
+        ct1, s1, passes1 = ct1 + ct, s1 + sec, passes1 + 1
     return {"value": total_ct / total_s, "unit": UNIT, "cores": nthreads, "kind": "oracle", "cpu": cpu_model(),
             "sample": f"{passes} pass(es) of {inp['batch']}x{rows} channels x {inp['seqlen']} tokens "
-                      f"of {WORKLOAD} (fp64, {nthreads} threads, {total_s:.1f} s)"}
+                      f"of {WORKLOAD} (fp64, {nthreads} threads, {total_s:.1f} s)",
+            "single_thread": {"value": ct1 / s1, "unit": UNIT,
+                              "sample": f"{passes1} pass(es) of {inp['batch']}x{rows1} channels x "
+                                        f"{inp['seqlen']} tokens (fp64, 1 thread, {s1:.1f} s)"}}
 
 
 def run_reference(args, rank):
