@@ -1,9 +1,9 @@
 // host_pipeline.cu -- the forward pass over inputs and outputs in host
 // memory (mss_scan_fwd_host).
 //
-// The channels are cut into pieces (a piece stays inside one batch row, so
-// it reads one batch's B and C).  Each piece is staged through one of
-// kSlots slots of a caller-owned device workspace: its inputs are copied in
+// The rows are cut into pieces: parts of one batch row when a row holds more
+// than the piece target, else groups of whole batch rows.  Each piece is
+// staged through one of up to kSlots slots of a caller-owned device workspace: its inputs are copied in
 // on one stream, the forward kernel runs on one of two compute streams, and
 // y and the final state are copied out on a third stream.  Events order the
 // three stages of a piece and hand a slot to the next piece only once its
@@ -30,9 +30,15 @@ constexpr unsigned kHostFlags = MSS_FLAG_GENERAL_A | MSS_FLAG_SIMPLE | MSS_FLAG_
 inline int64_t round_up(int64_t x) { return (x + kAlign - 1) / kAlign * kAlign; }
 
 // Piece size and workspace layout for one call's sizes and optional inputs.
+// A batch row larger than the piece target is cut into pieces of whole
+// 16-channel groups; smaller rows are grouped, several whole batch rows to a
+// piece (their rows are contiguous, so a piece is still one copy per tensor).
 struct Plan {
-    int64_t piece_dim = 0;   // channels per piece (the last piece of a batch row may have fewer)
-    int64_t row_pieces = 0;  // pieces per batch row
+    int64_t piece_batches = 0;  // batch rows per piece (1 when rows are cut)
+    int64_t piece_dim = 0;      // channels per piece and batch row (dim when rows are whole)
+    int64_t row_pieces = 0;     // pieces per batch row (1 when rows are whole)
+    int64_t n_pieces = 0;
+    int slots = 0;              // staging slots in the workspace (at most kSlots)
     // parameter block: A, D, bias, B, C
     int64_t off_A = 0, off_D = 0, off_bias = 0, off_B = 0, off_C = 0;
     // one slot: u, delta, z, y, initial state, last state
@@ -45,11 +51,26 @@ Plan make_plan(int64_t batch, int64_t dim, int64_t dstate, int64_t seqlen, int64
                bool has_bias, bool has_h0, bool has_last) {
     Plan pl;
     const int64_t row_in = seqlen * esz * (gated ? 3 : 2);  // input bytes of one channel
-    int64_t k = row_in > 0 ? (dim * row_in + kPieceInputBytes - 1) / kPieceInputBytes : 1;
-    k = std::max<int64_t>(1, std::min<int64_t>(k, (dim + 15) / 16));
-    // equal pieces of whole 16-channel groups (the forward kernel's CTA)
-    pl.piece_dim = std::min<int64_t>(dim, ((dim + k - 1) / k + 15) / 16 * 16);
-    pl.row_pieces = (dim + pl.piece_dim - 1) / pl.piece_dim;
+    const int64_t batch_row_in = dim * row_in;              // of one batch row
+    if (batch_row_in <= kPieceInputBytes) {
+        int64_t nb = batch_row_in > 0 ? std::max<int64_t>(1, kPieceInputBytes / batch_row_in) : batch;
+        nb = std::min<int64_t>(nb, batch);
+        const int64_t pieces = (batch + nb - 1) / nb;
+        pl.piece_batches = (batch + pieces - 1) / pieces;  // equal pieces
+        pl.piece_dim = dim;
+        pl.row_pieces = 1;
+        pl.n_pieces = (batch + pl.piece_batches - 1) / pl.piece_batches;
+    } else {
+        int64_t k = (batch_row_in + kPieceInputBytes - 1) / kPieceInputBytes;
+        k = std::max<int64_t>(1, std::min<int64_t>(k, (dim + 15) / 16));
+        // equal pieces of whole 16-channel groups (the forward kernel's CTA)
+        pl.piece_batches = 1;
+        pl.piece_dim = std::min<int64_t>(dim, ((dim + k - 1) / k + 15) / 16 * 16);
+        pl.row_pieces = (dim + pl.piece_dim - 1) / pl.piece_dim;
+        pl.n_pieces = batch * pl.row_pieces;
+    }
+    pl.slots = int(std::min<int64_t>(kSlots, pl.n_pieces));
+    const int64_t slot_rows = pl.piece_batches * pl.piece_dim;
     int64_t o = 0;
     pl.off_A = o;    o += round_up(dim * dstate * 4);
     pl.off_D = o;    o += has_D ? round_up(dim * 4) : 0;
@@ -57,7 +78,7 @@ Plan make_plan(int64_t batch, int64_t dim, int64_t dstate, int64_t seqlen, int64
     pl.off_B = o;    o += round_up(batch * dstate * seqlen * esz);
     pl.off_C = o;    o += round_up(batch * dstate * seqlen * esz);
     pl.slot0 = o;
-    const int64_t seq = pl.piece_dim * seqlen * esz, st = pl.piece_dim * dstate * 4;
+    const int64_t seq = slot_rows * seqlen * esz, st = slot_rows * dstate * 4;
     int64_t s = 0;
     pl.off_u = s;     s += round_up(seq);
     pl.off_delta = s; s += round_up(seq);
@@ -66,7 +87,7 @@ Plan make_plan(int64_t batch, int64_t dim, int64_t dstate, int64_t seqlen, int64
     pl.off_h0 = s;    s += has_h0 ? round_up(st) : 0;
     pl.off_last = s;  s += has_last ? round_up(st) : 0;
     pl.slot_bytes = s;
-    pl.total = pl.slot0 + kSlots * s;
+    pl.total = pl.slot0 + pl.slots * s;
     return pl;
 }
 
@@ -207,14 +228,16 @@ int mss_scan_fwd_host(const void* u, const void* delta, const float* A, const vo
         (seqlen > 0 && (!copy(B_d, B, bc_bytes, H2D, ds->h2d) || !copy(C_d, C, bc_bytes, H2D, ds->h2d))))
         return MSS_ERR_CUDA;
 
-    const int64_t n_pieces = batch * pl.row_pieces;
-    for (int64_t i = 0; i < n_pieces; ++i) {
-        const int slot = int(i % kSlots);
-        const int64_t b = i / pl.row_pieces, d0 = (i % pl.row_pieces) * pl.piece_dim;
+    for (int64_t i = 0; i < pl.n_pieces; ++i) {
+        const int slot = int(i % pl.slots);
+        // piece i: batch rows [b, b + nb), channels [d0, d0 + nd) of each
+        const int64_t b = pl.row_pieces > 1 ? i / pl.row_pieces : i * pl.piece_batches;
+        const int64_t nb = std::min<int64_t>(pl.piece_batches, batch - b);
+        const int64_t d0 = pl.row_pieces > 1 ? (i % pl.row_pieces) * pl.piece_dim : 0;
         const int64_t nd = std::min<int64_t>(pl.piece_dim, dim - d0);
-        const int64_t row0 = b * dim + d0;
-        const int64_t seq_off = row0 * seqlen * esz, seq_n = nd * seqlen * esz;
-        const int64_t st_off = row0 * dstate * 4, st_n = nd * dstate * 4;
+        const int64_t row0 = b * dim + d0, rows_n = nb * nd;  // contiguous rows (nb > 1 only with nd = dim)
+        const int64_t seq_off = row0 * seqlen * esz, seq_n = rows_n * seqlen * esz;
+        const int64_t st_off = row0 * dstate * 4, st_n = rows_n * dstate * 4;
         uint8_t* sl = ws + pl.slot0 + slot * pl.slot_bytes;
         uint8_t* u_d = sl + pl.off_u;
         uint8_t* delta_d = sl + pl.off_delta;
@@ -223,7 +246,7 @@ int mss_scan_fwd_host(const void* u, const void* delta, const float* A, const vo
         float* h0_d = initial_state ? reinterpret_cast<float*>(sl + pl.off_h0) : nullptr;
         float* last_d = last_state ? reinterpret_cast<float*>(sl + pl.off_last) : nullptr;
         // in: once the slot's previous piece has left
-        if (i >= kSlots && cudaStreamWaitEvent(ds->h2d, ev.freed[slot], 0) != cudaSuccess) return MSS_ERR_CUDA;
+        if (i >= pl.slots && cudaStreamWaitEvent(ds->h2d, ev.freed[slot], 0) != cudaSuccess) return MSS_ERR_CUDA;
         if (seqlen > 0 &&
             (!copy(u_d, static_cast<const uint8_t*>(u) + seq_off, seq_n, H2D, ds->h2d) ||
              !copy(delta_d, static_cast<const uint8_t*>(delta) + seq_off, seq_n, H2D, ds->h2d) ||
@@ -239,7 +262,7 @@ int mss_scan_fwd_host(const void* u, const void* delta, const float* A, const vo
             seqlen > 0 ? u_d : nullptr, seqlen > 0 ? delta_d : nullptr, A_d + d0 * dstate,
             seqlen > 0 ? B_d + b * dstate * seqlen * esz : nullptr, seqlen > 0 ? C_d + b * dstate * seqlen * esz : nullptr,
             D_d ? D_d + d0 : nullptr, z_d, bias_d ? bias_d + d0 : nullptr, softplus_flag, h0_d,
-            seqlen > 0 ? y_d : nullptr, last_d, 1, nd, dstate, seqlen, dtype, flags | MSS_FLAG_NO_SPLIT, nullptr, 0,
+            seqlen > 0 ? y_d : nullptr, last_d, nb, nd, dstate, seqlen, dtype, flags | MSS_FLAG_NO_SPLIT, nullptr, 0,
             cs);
         if (rc != MSS_OK) return rc;
         if (cudaEventRecord(ev.done[slot], cs) != cudaSuccess) return MSS_ERR_CUDA;

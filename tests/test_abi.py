@@ -324,9 +324,9 @@ def test_host_call_argument_errors(lib):
     lib.mss_scan_fwd_host_workspace_size.restype = ctypes.c_int64
     need = lib.mss_scan_fwd_host_workspace_size(ctypes.c_int64(2), ctypes.c_int64(8), ctypes.c_int64(16),
                                                 ctypes.c_int64(32), 1, 0, 0, 0, 0, 0)
-    # A, B, C once; one slot is u, delta, y (8 channels x 32 tokens of bf16,
-    # each rounded up to 256 bytes); three slots
-    assert need == 512 + 2 * 2048 + 3 * 3 * 512
+    # A, B, C once; both batch rows fit one piece, so one slot of u, delta,
+    # y for 2 x 8 channels x 32 tokens of bf16
+    assert need == 512 + 2 * 2048 + 3 * 1024
 
     def host(**kw):
         a = dict(u=P, delta=P + 0x1000000, A=P + 0x2000000, B=P + 0x3000000, C=P + 0x4000000,
@@ -355,6 +355,11 @@ def test_host_call_argument_errors(lib):
     assert q(0, 8, 16, 32, 1, 1, 1, 1, 1, 1) == 0
     assert q(2, 8, 16, 32, 9, 0, 0, 0, 0, 0) == codes["MSS_ERR_DTYPE"]
     assert q(2, 8, 5, 32, 1, 0, 0, 0, 0, 0) == codes["MSS_ERR_UNSUPPORTED_N"]
-    # every optional input adds its own piece: z one more [8 x 32] slot tensor,
-    # D and bias [dim] floats, the two states [8 x 16] floats per slot
-    assert q(2, 8, 16, 32, 1, 1, 1, 1, 1, 1) == need + 3 * 512 + 2 * 256 + 3 * 2 * 512
+    # every optional input adds its own buffer: z one more [16 x 32] slot
+    # tensor, D and bias [dim] floats, the two states [16 x 16] floats
+    assert q(2, 8, 16, 32, 1, 1, 1, 1, 1, 1) == need + 1024 + 2 * 256 + 2 * 1024
+    # rows beyond 64 MB of inputs are cut: 4144 channels x 4096 bf16 tokens with
+    # z is about 100 MB a row, so two pieces of 2080 channels, three slots
+    big = q(2, 4144, 16, 4096, 1, 1, 0, 0, 0, 0)
+    params = 4144 * 16 * 4 + 2 * (2 * 16 * 4096 * 2)
+    assert big == params + 3 * 4 * (2080 * 4096 * 2)

@@ -3,10 +3,10 @@
 The call stages pieces of the channels through a device workspace and runs
 the same forward kernel on each piece, so its outputs must equal, bit for bit,
 those of the device call on the same inputs, and the oracle within the
-tolerances of tests/helpers.py.  The cases cover one piece per batch row,
-more pieces than workspace slots (slot reuse), several pieces per batch row
-with a ragged last piece, the optional inputs, an empty sequence and
-pageable host memory.
+tolerances of tests/helpers.py.  The cases cover all rows in one piece,
+whole batch rows grouped into more pieces than workspace slots (slot
+reuse), several pieces per batch row with a ragged last piece, the optional
+inputs, an empty sequence, pageable host memory and chaining.
 """
 import numpy as np
 import pytest
@@ -37,7 +37,7 @@ def _device_twin(h):
 @pytest.mark.parametrize("dtype", ["f32", "bf16"])
 @pytest.mark.parametrize("batch", [1, 5])
 def test_host_call_matches_oracle_and_device_call(dtype, batch):
-    # L = 300: a ragged tail; batch 5 > three workspace slots
+    # L = 300: a ragged tail; the rows are small, so one piece holds them all
     inp = gen.scan_inputs(batch, 40, 16, 300, dtype, seed=800 + batch, d_skip="normal")
     h = _host_inputs(inp)
     h0 = torch.randn(batch, 40, 16, generator=torch.Generator().manual_seed(801)).pin_memory()
@@ -68,6 +68,27 @@ def test_host_call_pieces_within_a_batch_row():
     assert torch.equal(y, yd.cpu()) and torch.equal(last, lastd.cpu())
     # and a sampled channel on each side of the piece boundary against the oracle
     for b, d in ((0, 2079), (1, 2080), (1, dim - 1)):
+        y_ref, last_ref = oracle.scan_fwd(inp["u"].values[b:b + 1, d:d + 1], inp["delta"].values[b:b + 1, d:d + 1],
+                                          inp["A"][d:d + 1], inp["B"].values[b:b + 1], inp["C"].values[b:b + 1],
+                                          D=inp["D"][d:d + 1], z=inp["z"].values[b:b + 1, d:d + 1],
+                                          delta_bias=inp["delta_bias"][d:d + 1])
+        assert_close(to_numpy(y[b:b + 1, d:d + 1]), y_ref, "bf16", f"y of ({b}, {d})")
+        assert_close(to_numpy(last[b:b + 1, d:d + 1]), last_ref, "bf16", f"state of ({b}, {d})")
+
+
+def test_host_call_groups_whole_batch_rows():
+    """Rows of 2048 channels x 2048 bf16 tokens (about 25 MB of inputs): two
+    whole batch rows to a piece, nine rows in five pieces (the last one row),
+    so the three workspace slots are reused."""
+    batch, dim, N, L = 9, 2048, 16, 2048
+    inp = gen.scan_inputs(batch, dim, N, L, "bf16", seed=815, d_skip="normal")
+    h = _host_inputs(inp)
+    y, last = mss.scan_fwd_host(**h)
+    yd, lastd = mss.scan_fwd(**_device_twin(h), workspace=None, flags=mss.FLAG_NO_SPLIT)
+    torch.cuda.synchronize()
+    assert mss.get_device_error() == 0
+    assert torch.equal(y, yd.cpu()) and torch.equal(last, lastd.cpu())
+    for b, d in ((1, 0), (2, 2047), (8, 1000)):
         y_ref, last_ref = oracle.scan_fwd(inp["u"].values[b:b + 1, d:d + 1], inp["delta"].values[b:b + 1, d:d + 1],
                                           inp["A"][d:d + 1], inp["B"].values[b:b + 1], inp["C"].values[b:b + 1],
                                           D=inp["D"][d:d + 1], z=inp["z"].values[b:b + 1, d:d + 1],
