@@ -134,6 +134,25 @@ struct CallEvents {
     }
 };
 
+// On a failure after work was queued, the caller's stream still waits for
+// everything already queued on the library's streams, so that the caller
+// does not release the workspace or the host buffers under copies in flight.
+struct JoinOnFailure {
+    DeviceStreams* ds;
+    cudaStream_t caller;
+    bool armed = true;
+    ~JoinOnFailure() {
+        if (!armed) return;
+        cudaStream_t all[] = {ds->h2d, ds->d2h, ds->comp[0], ds->comp[1]};
+        for (cudaStream_t h : all) {
+            cudaEvent_t e;
+            if (cudaEventCreateWithFlags(&e, cudaEventDisableTiming) != cudaSuccess) continue;
+            if (cudaEventRecord(e, h) == cudaSuccess) cudaStreamWaitEvent(caller, e, 0);
+            cudaEventDestroy(e);
+        }
+    }
+};
+
 inline bool copy(void* dst, const void* src, int64_t bytes, cudaMemcpyKind kind, cudaStream_t s) {
     return bytes <= 0 || cudaMemcpyAsync(dst, src, size_t(bytes), kind, s) == cudaSuccess;
 }
@@ -207,6 +226,7 @@ int mss_scan_fwd_host(const void* u, const void* delta, const float* A, const vo
     CallEvents ev;
     if (!ev.ok) return MSS_ERR_CUDA;
     cudaStream_t s = static_cast<cudaStream_t>(stream);
+    JoinOnFailure join{ds, s};
     uint8_t* ws = static_cast<uint8_t*>(workspace);
     const cudaMemcpyKind H2D = cudaMemcpyHostToDevice, D2H = cudaMemcpyDeviceToHost;
 
@@ -277,6 +297,7 @@ int mss_scan_fwd_host(const void* u, const void* delta, const float* A, const vo
     // out run in order on one stream, and each follows its piece's kernel)
     if (cudaEventRecord(ev.end, ds->d2h) != cudaSuccess || cudaStreamWaitEvent(s, ev.end, 0) != cudaSuccess)
         return MSS_ERR_CUDA;
+    join.armed = false;
     return MSS_OK;
 }
 
