@@ -22,8 +22,9 @@
  *
  * Conventions shared by every entry point:
  *   - Every tensor pointer is a DEVICE pointer owned by the caller, C-contiguous
- *     in the layout given below.  The library never allocates memory on the
- *     forward or decode path and never frees caller memory.
+ *     in the layout given below (mss_scan_fwd_host alone takes HOST tensors).
+ *     The library never allocates memory on the forward or decode path and
+ *     never frees caller memory.
  *   - Work is enqueued on `stream` (a cudaStream_t passed as void*; NULL means
  *     the legacy default stream) and is asynchronous: a return of MSS_OK means
  *     the launch was accepted, not that it has finished.
@@ -37,9 +38,10 @@
  *     float.  All arithmetic is fp32.
  *   - dstate (N) must be 1, 2, 4, 8 or 16.
  *   - Outputs must not overlap inputs (the decode state is in/out by design).
- *   - Thread safety: the library keeps no host state besides a per-device,
- *     lazily resolved driver entry point; calls from several host threads are
- *     safe.
+ *   - Thread safety: the library's only host state is looked up or created
+ *     once per device on first use and then kept: a driver entry point,
+ *     occupancy figures, and for mss_scan_fwd_host four streams.  Calls from
+ *     several host threads are safe.
  */
 #ifndef MSS_H
 #define MSS_H

@@ -363,3 +363,24 @@ def test_host_call_argument_errors(lib):
     big = q(2, 4144, 16, 4096, 1, 1, 0, 0, 0, 0)
     params = 4144 * 16 * 4 + 2 * (2 * 16 * 4096 * 2)
     assert big == params + 3 * 4 * (2080 * 4096 * 2)
+
+
+def test_plain_c_client_compiles_links_and_runs(lib):
+    """include/mss.h is a C header and libmss.so a C library: a C99 program
+    (tests/c_client.c) compiles against the header, links the library and
+    makes the calls that need no GPU."""
+    import shutil
+    import subprocess
+
+    if shutil.which("gcc") is None:
+        pytest.skip("no C compiler")
+    out_dir = os.path.join(ROOT, "selective_state_space_mss_b200", "_build")
+    os.makedirs(out_dir, exist_ok=True)
+    exe = os.path.join(out_dir, "c_client")
+    lib_dir = os.path.dirname(mss.library_path())
+    build = subprocess.run(["gcc", "-std=c99", "-Wall", "-Wextra", "-Werror", "-I", os.path.join(ROOT, "include"),
+                            os.path.join(ROOT, "tests", "c_client.c"), "-o", exe, mss.library_path(),
+                            "-Wl,-rpath," + lib_dir], capture_output=True, text=True)
+    assert build.returncode == 0, build.stderr
+    run = subprocess.run([exe], capture_output=True, text=True, timeout=60)
+    assert run.returncode == 0 and run.stdout.strip() == "ok", run.stdout + run.stderr
