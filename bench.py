@@ -183,6 +183,69 @@ class ClockSampler:
                 "reasons": reasons, "samples": len(rows)}
 
 
+class NvmlSampler:
+    """SM clock, power and clock-event reasons read through NVML every ~2 ms
+    by a host thread while the timed region runs (the host waits in
+    synchronize while the GPU works, so the samples fall under load).  Only
+    reads; any NVML failure leaves it with no samples."""
+
+    REASONS = (("sw_power_cap", 0x4), ("hw_slowdown", 0x8), ("sw_thermal_slowdown", 0x20),
+               ("hw_thermal_slowdown", 0x40))
+
+    def __init__(self, gpu_index, period_s=0.002):
+        self.gpu = str(gpu_index)
+        self.period = period_s
+        self.rows = []
+        self.max_mhz = None
+        self._thread = None
+
+    def __enter__(self):
+        import threading
+
+        try:
+            import pynvml
+
+            pynvml.nvmlInit()
+            h = (pynvml.nvmlDeviceGetHandleByUUID(self.gpu) if self.gpu.startswith("GPU-")
+                 else pynvml.nvmlDeviceGetHandleByIndex(int(self.gpu)))
+            self.max_mhz = float(pynvml.nvmlDeviceGetMaxClockInfo(h, pynvml.NVML_CLOCK_SM))
+            reasons = (getattr(pynvml, "nvmlDeviceGetCurrentClocksEventReasons", None)
+                       or pynvml.nvmlDeviceGetCurrentClocksThrottleReasons)
+        except Exception:
+            return self
+        self._stop = threading.Event()
+
+        def run():
+            while not self._stop.is_set():
+                try:
+                    self.rows.append((float(pynvml.nvmlDeviceGetClockInfo(h, pynvml.NVML_CLOCK_SM)),
+                                      int(reasons(h)), pynvml.nvmlDeviceGetPowerUsage(h) / 1000.0))
+                except Exception:
+                    return
+                time.sleep(self.period)
+
+        self._thread = threading.Thread(target=run, daemon=True)
+        self._thread.start()
+        return self
+
+    def __exit__(self, *exc):
+        if self._thread is not None:
+            self._stop.set()
+            self._thread.join(timeout=5)
+        return False
+
+    def summary(self):
+        if not self.rows:
+            return None
+        mask = 0
+        for _, r, _ in self.rows:
+            mask |= r
+        return {"sm_mhz": statistics.median(r[0] for r in self.rows), "sm_max_mhz": self.max_mhz,
+                "power_w_max": max(r[2] for r in self.rows),
+                "reasons": [name for name, bit in self.REASONS if mask & bit], "samples": len(self.rows),
+                "source": "NVML every 2 ms during the timed region"}
+
+
 # ---------------------------------------------------------------------------
 # Multi-rank plumbing: every rank runs its own replica of the workload (the
 # channels are independent, so there is no data-path collective); the only
@@ -416,21 +479,32 @@ def run_mss(args, rank, world, local_rank):
         evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(k)]
         start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         sampler = ClockSampler(physical_gpu_index(local_rank))
+        nvml = NvmlSampler(physical_gpu_index(local_rank))
         if with_clocks:
             sampler.__enter__()
             time.sleep(0.3)
+            nvml.__enter__()
         start.record(stream)
         for i in range(k):
             step(flags, evs[i])
         end.record(stream)
         torch.cuda.synchronize(dev)
         if with_clocks:
+            nvml.__exit__(None, None, None)
             sampler.__exit__(None, None, None)
         if world > 1:
             dist.barrier()
         ms = max_over_ranks(start.elapsed_time(end), world, dev)
         fwd_ms = [a.elapsed_time(b) for a, b in evs]
-        return ms, fwd_ms, (sampler.summary() if with_clocks else None)
+        clocks = None
+        if with_clocks:
+            clocks = nvml.summary()
+            smi = sampler.summary()
+            if clocks is None:
+                clocks = smi
+            else:
+                clocks["nvidia_smi"] = smi
+        return ms, fwd_ms, clocks
 
     assert mss.get_device_error() == 0
     if args.kernel_only:
