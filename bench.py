@@ -183,6 +183,20 @@ class ClockSampler:
                 "reasons": reasons, "samples": len(rows)}
 
 
+def nvml_device_id(dev, local_rank):
+    """The CUDA device's UUID in NVML's form ("GPU-..."), so that NVML reads
+    the same physical GPU whatever the enumeration order; else its index."""
+    try:
+        import torch
+
+        u = str(torch.cuda.get_device_properties(dev).uuid)
+        if u:
+            return u if u.startswith("GPU-") else "GPU-" + u
+    except Exception:
+        pass
+    return physical_gpu_index(local_rank)
+
+
 class NvmlSampler:
     """SM clock, power and clock-event reasons read through NVML every ~2 ms
     by a host thread while the timed region runs (the host waits in
@@ -479,7 +493,7 @@ def run_mss(args, rank, world, local_rank):
         evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(k)]
         start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         sampler = ClockSampler(physical_gpu_index(local_rank))
-        nvml = NvmlSampler(physical_gpu_index(local_rank))
+        nvml = NvmlSampler(nvml_device_id(dev, local_rank))
         if with_clocks:
             sampler.__enter__()
             time.sleep(0.3)
