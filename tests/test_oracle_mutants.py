@@ -59,6 +59,14 @@ MUTANTS = {
     "ssd_no_decay": ("S[n * P + p] = a * S[n * P + p] + delta", "S[n * P + p] = S[n * P + p] + delta"),
     "ssd_input_without_step": ("+ delta * (double)Bt[n] * (double)xt[p];", "+ (double)Bt[n] * (double)xt[p];"),
     "ssd_state_layout": ("acc += (double)Ct[n] * S[n * P + p];", "acc += (double)Ct[n] * S[p * N + n];"),
+    "ssd_bias_dropped": ("const double bias = j->bias ? (double)j->bias[h] : 0.0;", "const double bias = 0.0;"),
+    "ssd_skip_dropped": ("double out = acc + Dh * (double)xt[p];", "double out = acc;"),
+    "ssd_gate_dropped": ("out *= mss_oracle_silu((double)j->z[((b * L + t) * H + h) * P + p]);", "out *= 1.0;"),
+    "ssd_initial_state_ignored": ("S[k] = j->initial_state ? j->initial_state[row * N * P + k] : 0.0;",
+                                  "S[k] = 0.0;"),
+    "ssd_last_state_row": ("j->last_state[row * N * P + k] = S[k];", "j->last_state[k] = S[k];"),
+    "ssd_x_head_index": ("const float *xt = j->x + ((b * L + t) * H + h) * P;",
+                         "const float *xt = j->x + ((b * L + t) * H) * P;"),
 }
 
 
@@ -70,27 +78,43 @@ def _run_pins(lib_path):
         cwd=ROOT, env=env, capture_output=True, text=True, timeout=600)
 
 
-def _build(src_text, tmp_path, name):
-    c = tmp_path / f"{name}.c"
-    so = tmp_path / f"{name}.so"
-    c.write_text(src_text)
+# mutant builds stay inside the repository (a git-ignored build folder)
+BUILD_DIR = os.path.join(ROOT, "oracle", "_build", "mutants")
+
+
+def _build(src_text, name):
+    os.makedirs(BUILD_DIR, exist_ok=True)
+    c = os.path.join(BUILD_DIR, f"{name}.{os.getpid()}.c")
+    so = os.path.join(BUILD_DIR, f"{name}.{os.getpid()}.so")
+    with open(c, "w") as f:
+        f.write(src_text)
     subprocess.check_call(["gcc", "-std=c99", "-O2", "-fno-fast-math", "-ffp-contract=off",
-                           "-fPIC", "-shared", "-o", str(so), str(c), "-lm", "-lpthread"])
-    return str(so)
+                           "-fPIC", "-shared", "-o", so, c, "-lm", "-lpthread"])
+    return so
 
 
-def test_unmodified_source_passes(tmp_path):
+def _pins_on(src_text, name):
+    so = _build(src_text, name)
+    try:
+        return _run_pins(so)
+    finally:
+        for path in (so, so[:-3] + ".c"):
+            if os.path.exists(path):
+                os.remove(path)
+
+
+def test_unmodified_source_passes():
     with open(SRC) as f:
         text = f.read()
-    r = _run_pins(_build(text, tmp_path, "original"))
+    r = _pins_on(text, "original")
     assert r.returncode == 0, r.stdout[-2000:]
 
 
 @pytest.mark.parametrize("name", sorted(MUTANTS))
-def test_pins_catch_mutant(name, tmp_path):
+def test_pins_catch_mutant(name):
     old, new = MUTANTS[name]
     with open(SRC) as f:
         text = f.read()
     assert text.count(old) == 1, f"mutation site for {name} not found exactly once"
-    r = _run_pins(_build(text.replace(old, new), tmp_path, name))
+    r = _pins_on(text.replace(old, new), name)
     assert r.returncode != 0, f"pins did not catch mutant {name}"
