@@ -212,6 +212,9 @@ class NvmlSampler:
         self.rows = []
         self.max_mhz = None
         self._thread = None
+        self._nvml = None
+        self._t0 = self._t1 = None
+        self.stopped_early = False
 
     def __enter__(self):
         import threading
@@ -220,6 +223,7 @@ class NvmlSampler:
             import pynvml
 
             pynvml.nvmlInit()
+            self._nvml = pynvml
             h = (pynvml.nvmlDeviceGetHandleByUUID(self.gpu) if self.gpu.startswith("GPU-")
                  else pynvml.nvmlDeviceGetHandleByIndex(int(self.gpu)))
             self.max_mhz = float(pynvml.nvmlDeviceGetMaxClockInfo(h, pynvml.NVML_CLOCK_SM))
@@ -235,9 +239,11 @@ class NvmlSampler:
                     self.rows.append((float(pynvml.nvmlDeviceGetClockInfo(h, pynvml.NVML_CLOCK_SM)),
                                       int(reasons(h)), pynvml.nvmlDeviceGetPowerUsage(h) / 1000.0))
                 except Exception:
+                    self.stopped_early = True
                     return
                 time.sleep(self.period)
 
+        self._t0 = time.perf_counter()
         self._thread = threading.Thread(target=run, daemon=True)
         self._thread.start()
         return self
@@ -246,6 +252,13 @@ class NvmlSampler:
         if self._thread is not None:
             self._stop.set()
             self._thread.join(timeout=5)
+            self._t1 = time.perf_counter()
+        if self._nvml is not None:
+            try:
+                self._nvml.nvmlShutdown()
+            except Exception:
+                pass
+            self._nvml = None
         return False
 
     def summary(self):
@@ -254,9 +267,13 @@ class NvmlSampler:
         mask = 0
         for _, r, _ in self.rows:
             mask |= r
+        # samples one thread can take in the window (each read also takes time,
+        # so the count comes in below this); far fewer means it stopped early
+        expected = None if self._t1 is None else int((self._t1 - self._t0) / self.period)
         return {"sm_mhz": statistics.median(r[0] for r in self.rows), "sm_max_mhz": self.max_mhz,
                 "power_w_max": max(r[2] for r in self.rows),
                 "reasons": [name for name, bit in self.REASONS if mask & bit], "samples": len(self.rows),
+                "samples_at_most": expected, "sampler_stopped_early": self.stopped_early,
                 "source": "NVML every 2 ms during the timed region"}
 
 

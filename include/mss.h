@@ -91,6 +91,17 @@ enum mss_status {
  * "Paper: Mamba", Objectives).  The transition Abar = exp(Delta A) is the
  * same under both rules. */
 #define MSS_FLAG_ZOH_INPUT 0x8u
+/* Self-test of the kernels' bounded waits (for tests of the failure path):
+ * every CTA of the tiled forward kernel first waits on a barrier that no copy
+ * will ever complete -- none has been issued yet -- with a limit of 1 ms.  The
+ * wait gives up, sets the device error word (mss_get_device_error then
+ * returns MSS_ERR_DEVICE_TIMEOUT, once) and the CTA returns; y, last_state and
+ * the workspace are not written.  The CUDA context stays usable and later
+ * calls are unaffected.  The flag needs a call that takes the tiled kernel
+ * (16-byte-aligned rows, dstate 4, 8 or 16, no MSS_FLAG_SIMPLE); otherwise the
+ * call returns MSS_ERR_FLAGS and launches nothing.  The sequence is not
+ * split. */
+#define MSS_FLAG_SELFTEST_TIMEOUT 0x10u
 
 /*
  * mss_scan_fwd -- selective-scan forward pass over whole sequences.
@@ -325,8 +336,10 @@ MSS_API int mss_scan_bwd(const void *u, const void *delta, const float *A, const
 
 /* Workspace bytes mss_scan_bwd needs for these sizes and flags, assuming
  * 16-byte aligned tensors (with unaligned ones it takes the scalar path: ask
- * with MSS_FLAG_SIMPLE for that size).  Negative mss_status on bad
- * arguments; 0 when there is nothing to do. */
+ * with MSS_FLAG_SIMPLE for that size).  Sizes the tiled kernels cannot take
+ * (batch > 65535, batch * dim >= 2^31, seqlen >= 2^31) get the scalar path's
+ * size here, as they get its kernel.  Negative mss_status on bad arguments;
+ * 0 when there is nothing to do. */
 MSS_API int64_t mss_scan_bwd_workspace_size(int64_t batch, int64_t dim, int64_t dstate, int64_t seqlen,
                                     int dtype, unsigned flags);
 

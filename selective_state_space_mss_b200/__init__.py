@@ -25,7 +25,8 @@ import torch
 __all__ = ["scan_fwd", "scan_fwd_host", "scan_fwd_conv", "scan_bwd", "ssd_fwd", "bwd_workspace_size", "state_update", "state_update_conv",
            "get_device_error",
            "library_path", "workspace_size",
-           "FLAG_GENERAL_A", "FLAG_SIMPLE", "FLAG_NO_SPLIT", "FLAG_ZOH_INPUT", "MssError", "load_library"]
+           "FLAG_GENERAL_A", "FLAG_SIMPLE", "FLAG_NO_SPLIT", "FLAG_ZOH_INPUT", "FLAG_SELFTEST_TIMEOUT",
+           "ERR_DEVICE_TIMEOUT", "ERR_FLAGS", "MssError", "load_library"]
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
 _LIB_PATH = os.path.join(_HERE, "libmss.so")
@@ -36,6 +37,9 @@ FLAG_GENERAL_A = 0x1
 FLAG_SIMPLE = 0x2
 FLAG_NO_SPLIT = 0x4
 FLAG_ZOH_INPUT = 0x8  # zero-order-hold input matrix (e^{Delta A} - 1)/A * B instead of Delta * B
+FLAG_SELFTEST_TIMEOUT = 0x10  # the tiled kernel's bounded wait gives up on purpose (failure-path tests)
+ERR_FLAGS = -8
+ERR_DEVICE_TIMEOUT = -7
 
 _lib = None
 _lock = threading.Lock()
@@ -390,11 +394,13 @@ def bwd_workspace_size(batch, dim, dstate, seqlen, dtype=torch.bfloat16, flags=0
 
 
 def scan_bwd(u, delta, A, B, C, dy, D=None, z=None, delta_bias=None, softplus=True, initial_state=None,
-             dlast=None, flags=0, workspace="auto", want_dinit=True, stream=None):
+             dlast=None, flags=0, workspace="auto", want_dinit=True, out=None, stream=None):
     """Backward pass of scan_fwd (mss_scan_bwd).  dy: [batch, dim, L] (the io
     dtype), dlast: [batch, dim, N] float32 or None.  Returns a dict with du,
     ddelta, dz (None without z) in the io dtype, dA [dim, N], dB, dC
-    [batch, N, L], dD, dbias [dim] and dinit [batch, dim, N] in float32."""
+    [batch, N, L], dD, dbias [dim] and dinit [batch, dim, N] in float32.
+    out: optional dict of caller-owned output tensors under those names (the
+    rest are allocated)."""
     if not isinstance(u, torch.Tensor) or u.device.type != "cuda":
         raise ValueError("u must be a CUDA tensor (there is no CPU path)")
     batch, dim, L = u.shape
@@ -410,13 +416,18 @@ def scan_bwd(u, delta, A, B, C, dy, D=None, z=None, delta_bias=None, softplus=Tr
                                      (dlast, "dlast", (batch, dim, N), torch.float32, True)):
         _check(t, name, shape, typ, dev, optional=opt)
     f32 = dict(dtype=torch.float32, device=dev)
-    out = dict(du=torch.empty((batch, dim, L), dtype=dt, device=dev),
+    ret = dict(du=torch.empty((batch, dim, L), dtype=dt, device=dev),
                ddelta=torch.empty((batch, dim, L), dtype=dt, device=dev),
                dz=torch.empty((batch, dim, L), dtype=dt, device=dev) if z is not None else None,
                dA=torch.empty((dim, N), **f32), dB=torch.empty((batch, N, L), **f32),
                dC=torch.empty((batch, N, L), **f32), dD=torch.empty((dim,), **f32),
                dbias=torch.empty((dim,), **f32),
                dinit=torch.empty((batch, dim, N), **f32) if want_dinit else None)
+    for k, t in (out or {}).items():
+        if k not in ret or ret[k] is None:
+            raise ValueError(f"out[{k!r}]: no such output here")
+        _check(t, k, tuple(ret[k].shape), ret[k].dtype, dev)
+        ret[k] = t
     if isinstance(workspace, str):
         if workspace != "auto":
             raise ValueError("workspace must be 'auto', None or a uint8 CUDA tensor")
@@ -426,13 +437,13 @@ def scan_bwd(u, delta, A, B, C, dy, D=None, z=None, delta_bias=None, softplus=Tr
         _check(workspace, "workspace", (workspace.numel(),), torch.uint8, dev)
     rc = load_library().mss_scan_bwd(
         _ptr(u), _ptr(delta), _ptr(A), _ptr(B), _ptr(C), _ptr(D), _ptr(z), _ptr(delta_bias), int(bool(softplus)),
-        _ptr(initial_state), _ptr(dy), _ptr(dlast), _ptr(out["du"]), _ptr(out["ddelta"]), _ptr(out["dz"]),
-        _ptr(out["dA"]), _ptr(out["dB"]), _ptr(out["dC"]), _ptr(out["dD"]), _ptr(out["dbias"]), _ptr(out["dinit"]),
+        _ptr(initial_state), _ptr(dy), _ptr(dlast), _ptr(ret["du"]), _ptr(ret["ddelta"]), _ptr(ret["dz"]),
+        _ptr(ret["dA"]), _ptr(ret["dB"]), _ptr(ret["dC"]), _ptr(ret["dD"]), _ptr(ret["dbias"]), _ptr(ret["dinit"]),
         batch, dim, N, L, code, int(flags), _ptr(workspace), 0 if workspace is None else workspace.numel(),
         _stream_handle(stream, dev))
     if rc != 0:
         raise MssError(rc, "mss_scan_bwd")
-    return out
+    return ret
 
 
 def state_update_conv(state, conv_state, x, conv_w, delta, A, B, C, conv_b=None, D=None, z=None,

@@ -12,13 +12,14 @@
 namespace mss_host {
 
 // Workspace bytes of the backward pass: the checkpoints of the throughput
-// kernels (one state per chunk of 128 bytes of a row) when the shape can take
-// them, else those of the scalar kernel (one per 16 tokens).
+// kernels (one state per chunk of 128 bytes of a row) when the sizes can take
+// them (the same test as the launch, for 16-byte-aligned tensors), else those
+// of the scalar kernel (one per 16 tokens).
 template <typename T, int N>
 int64_t backward_workspace_bytes(int64_t batch, int64_t dim, int64_t seqlen, unsigned flags) {
     const int64_t rows = batch * dim;
     if (rows == 0 || seqlen == 0) return 0;
-    bool fast = !(flags & MSS_FLAG_SIMPLE) && (N == 4 || N == 8 || N == 16) && (seqlen * int64_t(sizeof(T))) % 16 == 0;
+    const bool fast = seq_shape_ok(batch, dim, seqlen, N, int(sizeof(T)), flags);
     const int64_t chunk = fast ? mss::SeqLayout<T, (N >= 4 ? N : 4)>::kChunk : mss::kBwdSimpleChunk;
     return rows * ((seqlen + chunk - 1) / chunk) * N * 4;
 }

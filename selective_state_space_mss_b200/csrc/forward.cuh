@@ -73,13 +73,20 @@ int launch_simple(const mss::ScanParams& p, cudaStream_t stream) {
     return launch_status();
 }
 
-// The throughput kernel's requirements; otherwise the scalar kernel runs.
-inline bool seq_eligible(const mss::ScanParams& p, int64_t N, int esz, unsigned flags) {
+// The sizes the tiled kernels take (grid limits, 32-bit tensor-map row
+// coordinates); the backward pass's workspace size follows the same test.
+inline bool seq_shape_ok(int64_t batch, int64_t dim, int64_t seqlen, int64_t N, int esz, unsigned flags) {
     if (flags & MSS_FLAG_SIMPLE) return false;
     if (N != 4 && N != 8 && N != 16) return false;
-    if ((p.seqlen * esz) % 16 != 0) return false;
-    if (p.batch * p.dim >= (int64_t(1) << 31) || p.seqlen >= (int64_t(1) << 31)) return false;
-    if ((p.dim + 15) / 16 > 0x7fffffffLL || p.batch > 65535) return false;
+    if ((seqlen * esz) % 16 != 0) return false;
+    if (batch * dim >= (int64_t(1) << 31) || seqlen >= (int64_t(1) << 31)) return false;
+    if ((dim + 15) / 16 > 0x7fffffffLL || batch > 65535) return false;
+    return true;
+}
+
+// The throughput kernel's requirements; otherwise the scalar kernel runs.
+inline bool seq_eligible(const mss::ScanParams& p, int64_t N, int esz, unsigned flags) {
+    if (!seq_shape_ok(p.batch, p.dim, p.seqlen, N, esz, flags)) return false;
     const void* v[] = {p.u, p.delta, p.z, p.B, p.C, p.y};
     for (const void* q : v)
         if (q && !aligned(q, 16)) return false;
@@ -183,7 +190,7 @@ int launch_seq(mss::ScanParams p, unsigned flags, void* workspace, int64_t works
     p.n_seg = 1;
     p.seg_len = p.seqlen;
     p.agg = nullptr;
-    if (!(flags & MSS_FLAG_NO_SPLIT) && workspace) {
+    if (!(flags & (MSS_FLAG_NO_SPLIT | MSS_FLAG_SELFTEST_TIMEOUT)) && workspace) {
         const int n_seg = choose_segments<T, N>(p.batch, p.dim, p.seqlen);
         if (n_seg > 1 && agg_bytes(n_seg, rows, N) <= workspace_bytes) {
             p.n_seg = n_seg;
@@ -199,8 +206,12 @@ template <typename T, int N>
 int launch_forward(mss::ScanParams p, unsigned flags, void* workspace, int64_t workspace_bytes,
                    cudaStream_t stream) {
     if constexpr (N == 4 || N == 8 || N == 16) {
-        if (seq_eligible(p, N, int(sizeof(T)), flags)) return launch_seq<T, N>(p, flags, workspace, workspace_bytes, stream);
+        if (seq_eligible(p, N, int(sizeof(T)), flags)) {
+            p.selftest_wait_ns = (flags & MSS_FLAG_SELFTEST_TIMEOUT) ? 1000000ull : 0ull;
+            return launch_seq<T, N>(p, flags, workspace, workspace_bytes, stream);
+        }
     }
+    if (flags & MSS_FLAG_SELFTEST_TIMEOUT) return MSS_ERR_FLAGS;  // only the tiled kernel has the self-test
     return launch_simple<T, N>(p, stream);
 }
 

@@ -19,7 +19,8 @@ namespace {
 using mss::bf16_t;
 using namespace mss_host;
 
-constexpr unsigned kScanFlags = MSS_FLAG_GENERAL_A | MSS_FLAG_SIMPLE | MSS_FLAG_NO_SPLIT | MSS_FLAG_ZOH_INPUT;
+constexpr unsigned kScanFlags =
+    MSS_FLAG_GENERAL_A | MSS_FLAG_SIMPLE | MSS_FLAG_NO_SPLIT | MSS_FLAG_ZOH_INPUT | MSS_FLAG_SELFTEST_TIMEOUT;
 
 // The device error word (one per device, in the library image): kernels
 // whose bounded waits give up set it through the address in their

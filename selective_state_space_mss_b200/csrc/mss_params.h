@@ -37,6 +37,10 @@ struct ScanParams {
     // Checkpoint pass of the backward pass (fold launches only): the state at
     // the start of every chunk, [batch * dim, n_chunks, N].
     float* ckpt;
+    // Self-test of the bounded waits (MSS_FLAG_SELFTEST_TIMEOUT): nonzero makes
+    // every CTA of the tiled kernel wait this many nanoseconds on a barrier no
+    // copy completes, then return; 0 otherwise.
+    unsigned long long selftest_wait_ns;
 };
 
 // Backward pass (scan_bwd.cuh).  Inputs as ScanParams; dy is the gradient

@@ -86,7 +86,8 @@ struct SeqLayout {
     static constexpr int kBCfRow = 2 * N + 4;                  // floats per token row, +16 B padding
     static constexpr int kBCfBytes = kChunk * kBCfRow * 4;
     static constexpr int kBarOffset = kStages * kStageBytes + kBCfBytes;
-    static constexpr int kSmemBytes = kBarOffset + kStages * 8 + 1024;  // +1024: base alignment slack
+    // one barrier per stage and one for the wait self-test; +1024: base alignment slack
+    static constexpr int kSmemBytes = kBarOffset + (kStages + 1) * 8 + 1024;
     static_assert(kStageBytes % 1024 == 0, "stage tiles must stay 1024-byte aligned");
 };
 
@@ -156,8 +157,9 @@ struct TokenPre {
     float gate;  // silu(z), or 1 without a gate
 };
 
-template <bool kFast, bool kGeo, bool kGate, bool kSoftplus, bool kZoh, int N>
-__device__ __forceinline__ TokenPre token_pre(float ut, float dr, float zt, const LaneConst<N>& cc) {
+// `Consts` carries bias, D, a0 = A[d,0] log2(e) and ia0 = 1 / A[d,0].
+template <bool kFast, bool kGeo, bool kGate, bool kSoftplus, bool kZoh, typename Consts>
+__device__ __forceinline__ TokenPre token_pre(float ut, float dr, float zt, const Consts& cc) {
     TokenPre tp;
     const float s = dr + cc.bias;
     float dt = s;
@@ -676,7 +678,7 @@ __global__ void __launch_bounds__(32) scan_fwd_seq_kernel(const __grid_constant_
     const int64_t row = int64_t(blockIdx.y) * p.dim + d;
 
     if (lane == 0) {
-        for (int s = 0; s < Ly::kStages; ++s) mbar_init(bars + s, 1);
+        for (int s = 0; s <= Ly::kStages; ++s) mbar_init(bars + s, 1);
         fence_barrier_init();
         prefetch_tensormap(&maps.u);
         prefetch_tensormap(&maps.delta);
@@ -685,6 +687,13 @@ __global__ void __launch_bounds__(32) scan_fwd_seq_kernel(const __grid_constant_
         prefetch_tensormap(&maps.C);
     }
     __syncwarp();
+    if (p.selftest_wait_ns) {
+        // wait self-test: barrier kStages never completes (no copy has been
+        // issued and nothing arrives), so the bounded wait gives up and sets
+        // the error word; the CTA returns with nothing in flight
+        mbar_wait_bounded(bars + Ly::kStages, 0u, p.err, p.selftest_wait_ns);
+        return;
+    }
 
     constexpr bool kFast = sizeof(T) == 2;
     LaneConst<N> cc;

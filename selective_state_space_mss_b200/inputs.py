@@ -14,7 +14,13 @@ Recipe (the same for every workload; the seed is fixed per workload):
 * delta_raw = 0.1 * N(0, 1)
 * bias[d] = softplus^-1(dt_d) = log(expm1(dt_d)),  dt_d = exp(U(ln 1e-3, ln 1e-1)),
   so that softplus(delta_raw + bias) is log-uniform on about [1e-3, 1e-1]
-* A[d, n] = -(n + 1)  (the S4D-Real initialisation with negative real poles)
+* A[d, n] = -(n + 1)  (the S4D-Real initialisation with negative real poles);
+  other A recipes (tests only): "scaled" A[d, n] = -(n + 1) * s_d with
+  s_d = exp(U(ln 0.5, ln 2)) per channel (the product rounded in fp32, so the
+  rows stay exactly geometric); "random" A[d, n] = -exp(U(ln 0.1, ln 20)) per
+  channel and state; "mixed" cycles channel by channel through the S4D-Real,
+  random and scaled rows, so that every group of consecutive channels holds
+  all three kinds
 * D = 1, or D ~ N(1, 0.1) where the workload says so
 * everything is drawn in fp32, then rounded to bf16 for bf16 workloads;
   A, D and bias stay fp32.
@@ -105,10 +111,32 @@ def _rng(seed, *stream):
     return np.random.Generator(np.random.PCG64(np.random.SeedSequence([int(seed), *map(int, stream)])))
 
 
-def channel_params(dim: int, dstate: int, d_skip: str, seed: int):
+A_RECIPES = ("s4d-real", "scaled", "random", "mixed")
+
+
+def a_matrix(dim: int, dstate: int, recipe: str, seed: int) -> np.ndarray:
+    """A [dim, N] fp32 (negative values) by recipe; see the module docstring."""
+    s4d = -np.broadcast_to(np.arange(1, dstate + 1, dtype=np.float32), (dim, dstate)).copy()
+    if recipe == "s4d-real":
+        return s4d
+    if recipe not in A_RECIPES:
+        raise ValueError(f"unknown A recipe {recipe!r}")
+    rng = _rng(seed, 8)
+    scale = np.exp(rng.uniform(np.log(0.5), np.log(2.0), size=(dim, 1))).astype(np.float32)
+    scaled = (s4d * scale).astype(np.float32)          # fp32 products: exactly (n+1) * A[d, 0]
+    rand = (-np.exp(rng.uniform(np.log(0.1), np.log(20.0), size=(dim, dstate)))).astype(np.float32)
+    if recipe == "scaled":
+        return scaled
+    if recipe == "random":
+        return rand
+    kind = np.arange(dim) % 3
+    return np.where((kind == 0)[:, None], s4d, np.where((kind == 1)[:, None], rand, scaled)).astype(np.float32)
+
+
+def channel_params(dim: int, dstate: int, d_skip: str, seed: int, a_init: str = "s4d-real"):
     """A [dim, N], D [dim], bias [dim] -- fp32."""
     rng = _rng(seed, 0)
-    A = -np.broadcast_to(np.arange(1, dstate + 1, dtype=np.float32), (dim, dstate)).copy()
+    A = a_matrix(dim, dstate, a_init, seed)
     log_dt = rng.uniform(np.log(1e-3), np.log(1e-1), size=dim)
     dt = np.exp(log_dt)
     bias = np.log(np.expm1(dt)).astype(np.float32)
@@ -122,10 +150,10 @@ def channel_params(dim: int, dstate: int, d_skip: str, seed: int):
 
 
 def scan_inputs(batch: int, dim: int, dstate: int, seqlen: int, dtype: str,
-                seed: int, d_skip: str = "one") -> dict:
+                seed: int, d_skip: str = "one", a_init: str = "s4d-real") -> dict:
     """Inputs of one forward pass.  u, delta, z: [batch, dim, L]; B, C:
     [batch, N, L]; A: [dim, N]; D, delta_bias: [dim]."""
-    A, D, bias = channel_params(dim, dstate, d_skip, seed)
+    A, D, bias = channel_params(dim, dstate, d_skip, seed, a_init)
     rng = _rng(seed, 1)
     shape = (batch, dim, seqlen)
     u = _store(rng.standard_normal(shape, dtype=np.float32), dtype)

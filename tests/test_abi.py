@@ -265,6 +265,9 @@ def test_bwd_argument_errors(lib):
     assert q(1, 16, 16, 4097, 1, 0) == 16 * 257 * 16 * 4           # odd rows take the scalar path
     assert q(1, 16, 16, 0, 1, 0) == 0
     assert q(1, 16, 3, 64, 1, 0) == codes["MSS_ERR_UNSUPPORTED_N"]
+    # more batch rows than the tiled kernels' grid takes: the scalar path's size
+    assert q(70000, 16, 16, 64, 1, 0) == 70000 * 16 * 4 * 16 * 4
+    assert q(65535, 16, 16, 64, 1, 0) == 65535 * 16 * 1 * 16 * 4
 
 
 def test_ssd_argument_errors(lib):

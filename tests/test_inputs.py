@@ -40,3 +40,28 @@ def test_workload_table():
     assert small["u"].stored.dtype == np.float32 and small["u"].values.shape == (1, 16, 256)
     s = inputs.decode_step_inputs(4, 8, 16, "bf16", 1005, 3)
     assert s["B"].values.shape == (4, 16) and s["u"].values.shape == (4, 8)
+
+
+def test_a_recipes():
+    n = np.arange(1, 17, dtype=np.float32)
+    for recipe in inputs.A_RECIPES:
+        A = inputs.a_matrix(40, 16, recipe, 77)
+        assert A.shape == (40, 16) and A.dtype == np.float32 and np.all(A < 0)
+        geo = np.array([np.array_equal(A[d], (n * A[d, 0]).astype(np.float32)) for d in range(40)])
+        if recipe in ("s4d-real", "scaled"):
+            assert geo.all()
+        elif recipe == "random":
+            assert not geo.any() and A.min() >= -20.0 and A.max() <= -0.1
+            assert len(np.unique(A[:, 0])) == 40
+        else:
+            # every 16 consecutive channels hold S4D-Real, random and scaled rows
+            for d0 in range(0, 40 - 16 + 1):
+                kinds = {0 if np.array_equal(A[d], -n) else (2 if geo[d] else 1) for d in range(d0, d0 + 16)}
+                assert kinds == {0, 1, 2}
+        if recipe == "scaled":
+            assert len(np.unique(A[:, 0])) == 40
+    # the A recipe leaves the other draws unchanged
+    a = inputs.scan_inputs(2, 8, 16, 32, "bf16", 5, "normal")
+    b = inputs.scan_inputs(2, 8, 16, 32, "bf16", 5, "normal", a_init="random")
+    assert np.array_equal(a["D"], b["D"]) and np.array_equal(a["delta_bias"], b["delta_bias"])
+    assert np.array_equal(a["u"].stored, b["u"].stored) and not np.array_equal(a["A"], b["A"])

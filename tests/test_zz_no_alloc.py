@@ -34,13 +34,14 @@ def _lib():
     return lib
 
 
-def _call_noalloc(lib, d, y, last, h0=None):
+def _call_noalloc(lib, d, y, last, h0=None, flags=0):
     ptr = lambda t: None if t is None else ctypes.c_void_p(t.data_ptr())
     batch, dim, L = d["u"].shape
     N = d["A"].shape[1]
+    dtype = 1 if d["u"].dtype == torch.bfloat16 else 0
     return lib.mss_scan_fwd_noalloc(
         ptr(d["u"]), ptr(d["delta"]), ptr(d["A"]), ptr(d["B"]), ptr(d["C"]), ptr(d["D"]), ptr(d["z"]),
-        ptr(d["delta_bias"]), 1, ptr(h0), ptr(y), ptr(last), batch, dim, N, L, 1, 0,
+        ptr(d["delta_bias"]), 1, ptr(h0), ptr(y), ptr(last), batch, dim, N, L, dtype, flags,
         ctypes.c_void_p(torch.cuda.current_stream(DEV).cuda_stream))
 
 
@@ -65,3 +66,34 @@ def test_noalloc_matches_the_workspace_path_on_two_calls_in_a_row():
         assert_close(to_numpy(y), to_numpy(y_ref).astype("float64"), "bf16", f"{(batch, dim, N, L)} y")
         assert_close(to_numpy(last), to_numpy(last_ref).astype("float64"), "bf16",
                      f"{(batch, dim, N, L)} last_state")
+
+
+def test_noalloc_without_a_split_and_in_fp32():
+    """Calls that need no scratch (no split asked for, a short sequence: the
+    array is not touched) and an fp32 call that does, each against the
+    workspace entry point; the fp32 one also against the fp64 oracle."""
+    import oracle
+
+    lib = _lib()
+    cases = [("bf16", (1, 32, 16, 8192), mss.FLAG_NO_SPLIT, 0),
+             ("bf16", (2, 64, 16, 256), 0, 0),
+             ("f32", (1, 16, 16, 4096), 0, 1)]
+    for dtype, (batch, dim, N, L), flags, splits in cases:
+        tdt = torch.bfloat16 if dtype == "bf16" else torch.float32
+        need = mss.workspace_size(batch, dim, N, L, tdt, flags=flags, device=DEV)
+        assert (need > 0) == bool(splits)
+        inp = gen.scan_inputs(batch, dim, N, L, dtype, seed=70 + L, d_skip="normal")
+        d = device_inputs(inp, DEV)
+        y_ref, last_ref = mss.scan_fwd(**d, flags=flags)
+        y, last = torch.empty_like(y_ref), torch.empty_like(last_ref)
+        assert _call_noalloc(lib, d, y, last, flags=flags) == 0
+        torch.cuda.synchronize()
+        assert mss.get_device_error() == 0
+        what = f"{dtype} {(batch, dim, N, L)} flags={flags}"
+        assert_close(to_numpy(y), to_numpy(y_ref).astype("float64"), dtype, f"{what} y")
+        assert_close(to_numpy(last), to_numpy(last_ref).astype("float64"), dtype, f"{what} last_state")
+        if dtype == "f32":
+            yo, lo = oracle.scan_fwd(inp["u"].values, inp["delta"].values, inp["A"], inp["B"].values,
+                                     inp["C"].values, D=inp["D"], z=inp["z"].values, delta_bias=inp["delta_bias"])
+            assert_close(to_numpy(y), yo, dtype, f"{what} y vs oracle")
+            assert_close(to_numpy(last), lo, dtype, f"{what} last_state vs oracle")
