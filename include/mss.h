@@ -353,8 +353,10 @@ MSS_API int64_t mss_scan_bwd_workspace_size(int64_t batch, int64_t dim, int64_t 
  *   S_t = exp(Delta_t A_h) S_{t-1} + Delta_t B_t x_t^T,
  *   y_t = S_t^T C_t + D_h x_t, times silu(z_t) when z is given,
  *
- * computed chunk by chunk (64 tokens) with tensor-core matrix products: the
- * masked quadratic form within a chunk plus the state carried across.
+ * computed chunk by chunk with tensor-core matrix products: the masked
+ * quadratic form within a chunk plus the state carried across (chunks of 128
+ * tokens on the tcgen05 kernel for dstate 128, 64 on the warp-level kernels;
+ * see mss_ssd_fwd_ex2).
  *
  *   x, z, y  : [batch][seqlen][nheads][headdim]  bf16 (z may be NULL)
  *   dt       : [batch][seqlen][nheads]           bf16
@@ -395,9 +397,38 @@ MSS_API int mss_ssd_fwd_ex(const void *x, const void *dt, const float *A, const 
 
 /* Workspace bytes mss_ssd_fwd_ex would use for these sizes on the current
  * device (0: the in-order kernel, or no tokens), or a negative mss_status
- * (MSS_ERR_SHAPE for unsupported sizes). */
+ * (MSS_ERR_SHAPE for unsupported sizes).  dstate 128 runs the tcgen05 kernel
+ * in order: 0. */
 MSS_API int64_t mss_ssd_fwd_workspace_size(int64_t batch, int64_t seqlen, int64_t nheads, int64_t headdim,
                                    int64_t ngroups, int64_t dstate);
+
+/* Flags of mss_ssd_fwd_ex2. */
+#define MSS_SSD_FLAG_WARP_MMA 0x1u /* the warp-level (mma.sync) kernels instead of the tcgen05 one */
+
+/*
+ * mss_ssd_fwd_ex2 -- mss_ssd_fwd_ex with `flags`, for testing and measurement.
+ *
+ * With flags == 0 (this is then mss_ssd_fwd_ex): dstate 128 runs the tcgen05
+ * kernel -- one CTA per (batch, head) walking chunks of 128 tokens in order,
+ * operands staged by TMA in shared memory, the four chunk products
+ * (C B^T, B^T diag(w) X, C S_prev, M X) on the fifth-generation tensor cores
+ * with fp32 accumulators in tensor memory -- and ignores the workspace;
+ * dstate 64 runs the warp-level kernels as described at mss_ssd_fwd_ex.
+ * MSS_SSD_FLAG_WARP_MMA: the warp-level kernels for both dstate (in order,
+ * or the chunk-parallel passes with a workspace where they pay).  Other
+ * bits: MSS_ERR_FLAGS.  Same results up to rounding; the tcgen05 kernel's
+ * bounded waits report through mss_get_device_error.
+ */
+MSS_API int mss_ssd_fwd_ex2(const void *x, const void *dt, const float *A, const void *B, const void *C,
+                    const float *D, const void *z, const float *dt_bias, int softplus_flag,
+                    const float *initial_state, void *y, float *last_state, int64_t batch, int64_t seqlen,
+                    int64_t nheads, int64_t headdim, int64_t ngroups, int64_t dstate, int dtype,
+                    unsigned flags, void *workspace, int64_t workspace_bytes, void *stream);
+
+/* Workspace bytes mss_ssd_fwd_ex2 would use with these flags (as
+ * mss_ssd_fwd_workspace_size, which is flags == 0). */
+MSS_API int64_t mss_ssd_fwd_workspace_size_ex(int64_t batch, int64_t seqlen, int64_t nheads, int64_t headdim,
+                                      int64_t ngroups, int64_t dstate, unsigned flags);
 
 /*
  * mss_state_update -- one decode token for every (batch, channel):

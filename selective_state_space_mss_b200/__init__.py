@@ -26,7 +26,7 @@ __all__ = ["scan_fwd", "scan_fwd_host", "scan_fwd_conv", "scan_bwd", "ssd_fwd", 
            "get_device_error",
            "library_path", "workspace_size",
            "FLAG_GENERAL_A", "FLAG_SIMPLE", "FLAG_NO_SPLIT", "FLAG_ZOH_INPUT", "FLAG_SELFTEST_TIMEOUT",
-           "ERR_DEVICE_TIMEOUT", "ERR_FLAGS", "MssError", "load_library"]
+           "ERR_DEVICE_TIMEOUT", "ERR_FLAGS", "SSD_FLAG_WARP_MMA", "MssError", "load_library"]
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
 _LIB_PATH = os.path.join(_HERE, "libmss.so")
@@ -39,6 +39,7 @@ FLAG_NO_SPLIT = 0x4
 FLAG_ZOH_INPUT = 0x8  # zero-order-hold input matrix (e^{Delta A} - 1)/A * B instead of Delta * B
 FLAG_SELFTEST_TIMEOUT = 0x10  # the tiled kernel's bounded wait gives up on purpose (failure-path tests)
 ERR_FLAGS = -8
+SSD_FLAG_WARP_MMA = 0x1  # ssd_fwd: the warp-level (mma.sync) kernels instead of the tcgen05 one
 ERR_DEVICE_TIMEOUT = -7
 
 _lib = None
@@ -97,6 +98,11 @@ def load_library():
             lib.mss_ssd_fwd_ex.restype = i
             lib.mss_ssd_fwd_workspace_size.argtypes = [i64, i64, i64, i64, i64, i64]
             lib.mss_ssd_fwd_workspace_size.restype = i64
+            lib.mss_ssd_fwd_ex2.argtypes = [vp, vp, fp, vp, vp, fp, vp, fp, i, fp, vp, fp,
+                                            i64, i64, i64, i64, i64, i64, i, u32, vp, i64, vp]
+            lib.mss_ssd_fwd_ex2.restype = i
+            lib.mss_ssd_fwd_workspace_size_ex.argtypes = [i64, i64, i64, i64, i64, i64, u32]
+            lib.mss_ssd_fwd_workspace_size_ex.restype = i64
             lib.mss_scan_fwd_conv.argtypes = [vp, fp, fp, i, vp, vp, vp, fp, vp, vp, fp, vp, fp, i, fp, vp, fp,
                                               i64, i64, i64, i64, i, u32, vp, i64, vp]
             lib.mss_scan_fwd_conv.restype = i
@@ -337,14 +343,15 @@ def scan_fwd_conv(x, conv_w, delta, A, B, C, conv_b=None, conv_state=None, D=Non
 
 
 def ssd_fwd(x, dt, A, B, C, D=None, z=None, dt_bias=None, softplus=True, initial_state=None, y=None,
-            last_state=None, want_last_state=True, workspace="auto", stream=None):
-    """Structured-state-space-duality forward pass (mss_ssd_fwd_ex).  x, z:
+            last_state=None, want_last_state=True, workspace="auto", flags=0, stream=None):
+    """Structured-state-space-duality forward pass (mss_ssd_fwd_ex2).  x, z:
     [batch, L, H, P] bf16; dt: [batch, L, H] bf16; A, D, dt_bias: [H]
     float32; B, C: [batch, L, G, N] bf16; initial_state: [batch, H, N, P]
-    float32.  workspace: "auto" (what mss_ssd_fwd_workspace_size asks for,
+    float32.  workspace: "auto" (what mss_ssd_fwd_workspace_size_ex asks for,
     from PyTorch's allocator: every chunk in parallel where that beats one CTA
     per head, else nothing), None (one CTA per head walks its chunks) or a
-    uint8 CUDA tensor.  Returns (y, last_state)."""
+    uint8 CUDA tensor.  flags: 0 (the tcgen05 kernel for N = 128) or
+    SSD_FLAG_WARP_MMA (the warp-level kernels).  Returns (y, last_state)."""
     if not isinstance(x, torch.Tensor) or x.device.type != "cuda":
         raise ValueError("x must be a CUDA tensor (there is no CPU path)")
     if x.dim() != 4 or B.dim() != 4:
@@ -369,15 +376,15 @@ def ssd_fwd(x, dt, A, B, C, D=None, z=None, dt_bias=None, softplus=True, initial
     if isinstance(workspace, str):
         if workspace != "auto":
             raise ValueError("workspace must be 'auto', None or a uint8 CUDA tensor")
-        nbytes = int(load_library().mss_ssd_fwd_workspace_size(batch, L, H, P, G, N))
+        nbytes = int(load_library().mss_ssd_fwd_workspace_size_ex(batch, L, H, P, G, N, int(flags)))
         if nbytes < 0:
-            raise MssError(nbytes, "mss_ssd_fwd_workspace_size")
+            raise MssError(nbytes, "mss_ssd_fwd_workspace_size_ex")
         workspace = torch.empty(nbytes, dtype=torch.uint8, device=dev) if nbytes > 0 else None
     if workspace is not None:
         _check(workspace, "workspace", (workspace.numel(),), torch.uint8, dev)
-    rc = load_library().mss_ssd_fwd_ex(
+    rc = load_library().mss_ssd_fwd_ex2(
         _ptr(x), _ptr(dt), _ptr(A), _ptr(B), _ptr(C), _ptr(D), _ptr(z), _ptr(dt_bias), int(bool(softplus)),
-        _ptr(initial_state), _ptr(y), _ptr(last_state), batch, L, H, P, G, N, code, _ptr(workspace),
+        _ptr(initial_state), _ptr(y), _ptr(last_state), batch, L, H, P, G, N, code, int(flags), _ptr(workspace),
         0 if workspace is None else workspace.numel(), _stream_handle(stream, dev))
     if rc != 0:
         raise MssError(rc, "mss_ssd_fwd")

@@ -36,8 +36,12 @@ template <typename T, int N>
 int launch_decode(mss::StepParams p, cudaStream_t stream);
 
 // Structured-state-space-duality forward pass over validated arguments
-// (bf16 io, P = 64, dstate 64 or 128).
+// (bf16 io, P = 64, dstate 64 or 128): the warp-level (mma.sync) kernel.
 int launch_ssd(const mss::SsdParams& p, int dstate, cudaStream_t stream);
+
+// The same on the tcgen05 tensor cores (dstate 128; x, z, y, B, C 16-byte
+// aligned).
+int launch_ssd_tc(const mss::SsdParams& p, cudaStream_t stream);
 
 // The same with every chunk in parallel (three passes) over a workspace of
 // ssd_workspace_bytes (16-byte aligned).

@@ -410,11 +410,19 @@ int mss_ssd_fwd(const void* x, const void* dt, const float* A, const void* B, co
 
 int64_t mss_ssd_fwd_workspace_size(int64_t batch, int64_t seqlen, int64_t nheads, int64_t headdim, int64_t ngroups,
                                    int64_t dstate) {
+    return mss_ssd_fwd_workspace_size_ex(batch, seqlen, nheads, headdim, ngroups, dstate, 0u);
+}
+
+int64_t mss_ssd_fwd_workspace_size_ex(int64_t batch, int64_t seqlen, int64_t nheads, int64_t headdim,
+                                      int64_t ngroups, int64_t dstate, unsigned flags) {
+    if (flags & ~unsigned(MSS_SSD_FLAG_WARP_MMA)) return MSS_ERR_FLAGS;
     if (batch < 0 || seqlen < 0 || nheads < 1 || ngroups < 1 || nheads % ngroups != 0 || headdim != 64 ||
         (dstate != 64 && dstate != 128))
         return MSS_ERR_SHAPE;
     int64_t bh, tok;
     if (!mul_ok(batch, nheads, &bh) || !mul_ok(bh, seqlen, &tok) || tok > (int64_t(1) << 40)) return MSS_ERR_SHAPE;
+    // dstate 128 runs the tcgen05 kernel in order unless the warp-level kernels are asked for
+    if (dstate == 128 && !(flags & MSS_SSD_FLAG_WARP_MMA)) return 0;
     return seqlen == 0 || !ssd_chunked_pays(batch, nheads) ? 0 : ssd_workspace_bytes(batch, seqlen, nheads, dstate);
 }
 
@@ -423,6 +431,16 @@ int mss_ssd_fwd_ex(const void* x, const void* dt, const float* A, const void* B,
                    float* last_state, int64_t batch, int64_t seqlen, int64_t nheads, int64_t headdim,
                    int64_t ngroups, int64_t dstate, int dtype, void* workspace, int64_t workspace_bytes,
                    void* stream) {
+    return mss_ssd_fwd_ex2(x, dt, A, B, C, D, z, dt_bias, softplus_flag, initial_state, y, last_state, batch, seqlen,
+                           nheads, headdim, ngroups, dstate, dtype, 0u, workspace, workspace_bytes, stream);
+}
+
+int mss_ssd_fwd_ex2(const void* x, const void* dt, const float* A, const void* B, const void* C, const float* D,
+                    const void* z, const float* dt_bias, int softplus_flag, const float* initial_state, void* y,
+                    float* last_state, int64_t batch, int64_t seqlen, int64_t nheads, int64_t headdim,
+                    int64_t ngroups, int64_t dstate, int dtype, unsigned flags, void* workspace,
+                    int64_t workspace_bytes, void* stream) {
+    if (flags & ~unsigned(MSS_SSD_FLAG_WARP_MMA)) return MSS_ERR_FLAGS;
     if (workspace_bytes < 0) return MSS_ERR_SHAPE;
     if (dtype != MSS_DTYPE_BF16) return MSS_ERR_DTYPE;  // the tensor-core path takes bf16 io
     if (batch < 0 || seqlen < 0 || nheads < 1 || ngroups < 1 || nheads % ngroups != 0 || headdim != 64 ||
@@ -465,6 +483,8 @@ int mss_ssd_fwd_ex(const void* x, const void* dt, const float* A, const void* B,
     }
     mss::SsdParams p{x, dt, A, B, C, D, z, dt_bias, initial_state, y, last_state, batch, seqlen, nheads, ngroups,
                      softplus_flag ? 1 : 0};
+    if (!(p.err = device_error_word())) return MSS_ERR_CUDA;
+    if (dstate == 128 && !(flags & MSS_SSD_FLAG_WARP_MMA)) return launch_ssd_tc(p, s);
     if (workspace && ssd_chunked_pays(batch, nheads)) {
         const int64_t need = ssd_workspace_bytes(batch, seqlen, nheads, dstate);
         if (need > workspace_bytes || !aligned(workspace, 16)) return MSS_ERR_WORKSPACE;

@@ -92,6 +92,7 @@ struct SsdParams {
     float* last_state;     // may be null
     int64_t batch, seqlen, nheads, ngroups;
     int softplus;
+    unsigned int* err;     // device error word (the tcgen05 kernel's bounded waits)
 };
 
 struct StepParams {

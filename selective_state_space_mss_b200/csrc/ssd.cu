@@ -1,15 +1,79 @@
 // ssd.cu -- host-side launch of the structured-state-space-duality forward
 // pass (ssd_mma.cuh).
+#include <cstring>
 #include <mutex>
 
+#include <cuda.h>
+#include <cudaTypedefs.h>
 #include <cuda_runtime.h>
 
 #include "host_common.h"
 #include "launch.h"
 #include "ssd_chunked.cuh"
 #include "ssd_mma.cuh"
+#include "ssd_tc.cuh"
 
 namespace mss_host {
+
+namespace {
+
+PFN_cuTensorMapEncodeTiled_v12000 ssd_encode_fn() {
+    static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+    static std::once_flag once;
+    std::call_once(once, [] {
+        void* f = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &f, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(f);
+    });
+    return fn;
+}
+
+// [batch][L][n1][n0] bf16 as a 4-D view (n0 innermost); box = 64 x 1 x 128 x 1
+// (128 tokens of 64 elements), 128-byte swizzle.  Tokens past L read as zero
+// and are not written by stores.
+bool encode_token_major(CUtensorMap* m, const void* base, int64_t batch, int64_t L, int64_t n1, int64_t n0) {
+    auto enc = ssd_encode_fn();
+    if (!enc) return false;
+    const cuuint64_t dims[4] = {cuuint64_t(n0), cuuint64_t(n1), cuuint64_t(L), cuuint64_t(batch)};
+    const cuuint64_t strides[3] = {cuuint64_t(n0 * 2), cuuint64_t(n1 * n0 * 2), cuuint64_t(L * n1 * n0 * 2)};
+    const cuuint32_t box[4] = {64u, 1u, 128u, 1u};
+    const cuuint32_t estr[4] = {1u, 1u, 1u, 1u};
+    return enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void*>(base), dims, strides, box, estr,
+               CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+template <bool kGate, bool kSoftplus>
+int launch_ssd_tc_variant(const mss::SsdTcMaps& maps, const mss::SsdParams& p, cudaStream_t s) {
+    using Ly = mss::SsdTcLayout;
+    auto kern = mss::ssd_tc_kernel<kGate, kSoftplus>;
+    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, Ly::kSmemBytes) != cudaSuccess)
+        return MSS_ERR_CUDA;
+    const int64_t blocks = p.batch * p.nheads;
+    if (blocks > 0x7fffffffLL) return MSS_ERR_SHAPE;
+    kern<<<dim3(unsigned(blocks)), Ly::kThreads, Ly::kSmemBytes, s>>>(maps, p);
+    return launch_status();
+}
+
+}  // namespace
+
+// The tcgen05 kernel (dstate 128, headdim 64).
+int launch_ssd_tc(const mss::SsdParams& p, cudaStream_t s) {
+    if (p.batch > 0x7fffffffLL || p.seqlen > 0x7fffffffLL || p.nheads > 0x7fffffffLL) return MSS_ERR_SHAPE;
+    mss::SsdTcMaps maps;
+    std::memset(&maps, 0, sizeof(maps));
+    if (!encode_token_major(&maps.x, p.x, p.batch, p.seqlen, p.nheads, 64) ||
+        !encode_token_major(&maps.y, p.y, p.batch, p.seqlen, p.nheads, 64) ||
+        (p.z && !encode_token_major(&maps.z, p.z, p.batch, p.seqlen, p.nheads, 64)) ||
+        !encode_token_major(&maps.B, p.B, p.batch, p.seqlen, p.ngroups, 128) ||
+        !encode_token_major(&maps.C, p.C, p.batch, p.seqlen, p.ngroups, 128))
+        return MSS_ERR_CUDA;
+    if (p.z)
+        return p.softplus ? launch_ssd_tc_variant<true, true>(maps, p, s) : launch_ssd_tc_variant<true, false>(maps, p, s);
+    return p.softplus ? launch_ssd_tc_variant<false, true>(maps, p, s) : launch_ssd_tc_variant<false, false>(maps, p, s);
+}
 
 template <int NS, bool kGate, bool kSoftplus>
 int launch_ssd_variant(const mss::SsdParams& p, cudaStream_t s) {

@@ -31,15 +31,21 @@ def _ref(inp, gate=True, with_D=True, with_bias=True, h0=None):
                           dt_bias=inp["dt_bias"] if with_bias else None, initial_state=h0)
 
 
+# the tcgen05 kernel (N = 128; N = 64 runs the warp-level kernels either way)
+# and the warp-level (mma.sync) kernels
+KERNELS = {"tcgen05": 0, "warp": mss.SSD_FLAG_WARP_MMA}
+
+
+@pytest.mark.parametrize("kernel", sorted(KERNELS))
 @pytest.mark.parametrize("N", [64, 128])
 @pytest.mark.parametrize("L", [64, 200, 512])
 @pytest.mark.parametrize("G", [1, 2])
 @pytest.mark.parametrize("chunks", ["parallel", "in-order"])
-def test_ssd_matches_oracle(N, L, G, chunks):
+def test_ssd_matches_oracle(N, L, G, chunks, kernel):
     """Whole chunks, a ragged last chunk, one or two groups of heads; the
-    chunk-parallel passes (with a workspace) and the in-order kernel."""
+    chunk-parallel passes (with a workspace) and the in-order kernels."""
     inp = gen.ssd_inputs(2, L, 4, 64, G, N, seed=700 + L + N + G)
-    y, last = mss.ssd_fwd(**_dev(inp), workspace="auto" if chunks == "parallel" else None)
+    y, last = mss.ssd_fwd(**_dev(inp), workspace="auto" if chunks == "parallel" else None, flags=KERNELS[kernel])
     torch.cuda.synchronize()
     assert mss.get_device_error() == 0
     y_ref, last_ref = _ref(inp)
@@ -47,43 +53,52 @@ def test_ssd_matches_oracle(N, L, G, chunks):
     assert_close(to_numpy(last), last_ref, "bf16", f"N={N} L={L} G={G} last_state")
 
 
-def test_ssd_starting_state_and_chaining():
+@pytest.mark.parametrize("kernel", sorted(KERNELS))
+def test_ssd_starting_state_and_chaining(kernel):
+    f = KERNELS[kernel]
     inp = gen.ssd_inputs(2, 320, 4, 64, 1, 128, seed=720)
     h0 = np.random.default_rng(721).standard_normal((2, 4, 128, 64)).astype(np.float32) * 0.1
     d = _dev(inp)
     y_ref, last_ref = _ref(inp, h0=h0.astype(np.float64))
     for ws in ("auto", None):
-        y, last = mss.ssd_fwd(**d, initial_state=torch.from_numpy(h0).to(DEV), workspace=ws)
+        y, last = mss.ssd_fwd(**d, initial_state=torch.from_numpy(h0).to(DEV), workspace=ws, flags=f)
         torch.cuda.synchronize()
         assert_close(to_numpy(y), y_ref, "bf16", f"y from a starting state (workspace {ws})")
         assert_close(to_numpy(last), last_ref, "bf16", f"last_state from a starting state (workspace {ws})")
     # two calls chained through last_state equal one call
     part = lambda t0, t1: {k: (v[:, t0:t1].contiguous() if k in ("x", "dt", "B", "C", "z") else v)
                            for k, v in d.items()}
-    y0, last0 = mss.ssd_fwd(**part(0, 128))
-    y1, last1 = mss.ssd_fwd(**part(128, 320), initial_state=last0)
-    y_all, last_all = mss.ssd_fwd(**d)
+    y0, last0 = mss.ssd_fwd(**part(0, 128), flags=f)
+    y1, last1 = mss.ssd_fwd(**part(128, 320), initial_state=last0, flags=f)
+    y_all, last_all = mss.ssd_fwd(**d, flags=f)
     torch.cuda.synchronize()
     assert_close(to_numpy(torch.cat([y0, y1], dim=1)), to_numpy(y_all).astype(np.float64), "bf16", "chained y")
     assert_close(to_numpy(last1), to_numpy(last_all).astype(np.float64), "bf16", "chained state")
 
 
 def test_ssd_workspace_only_when_it_pays():
-    """Few (batch, head) pairs take the chunk-parallel passes, many the
-    in-order kernel; both give the oracle's result."""
+    """The warp-level kernels: few (batch, head) pairs take the chunk-parallel
+    passes, many the in-order kernel.  N = 128 runs the tcgen05 kernel in
+    order and asks for no workspace.  Each gives the oracle's result."""
+    lib = mss.load_library()
     sms = torch.cuda.get_device_properties(0).multi_processor_count
-    assert mss.load_library().mss_ssd_fwd_workspace_size(1, 4096, 4, 64, 1, 128) > 0
-    assert mss.load_library().mss_ssd_fwd_workspace_size(4, 4096, sms, 64, 1, 128) == 0
+    w = mss.SSD_FLAG_WARP_MMA
+    assert lib.mss_ssd_fwd_workspace_size_ex(1, 4096, 4, 64, 1, 128, w) > 0
+    assert lib.mss_ssd_fwd_workspace_size_ex(4, 4096, sms, 64, 1, 128, w) == 0
+    assert lib.mss_ssd_fwd_workspace_size(1, 4096, 4, 64, 1, 128) == 0
+    assert lib.mss_ssd_fwd_workspace_size(1, 4096, 4, 64, 1, 64) > 0
     inp = gen.ssd_inputs(1, 1024, 2, 64, 1, 128, seed=735)
-    y, last = mss.ssd_fwd(**_dev(inp))
-    torch.cuda.synchronize()
     y_ref, last_ref = _ref(inp)
-    assert_close(to_numpy(y), y_ref, "bf16", "few heads y")
-    assert_close(to_numpy(last), last_ref, "bf16", "few heads last_state")
+    for f in (0, w):
+        y, last = mss.ssd_fwd(**_dev(inp), flags=f)
+        torch.cuda.synchronize()
+        assert_close(to_numpy(y), y_ref, "bf16", f"few heads y (flags {f})")
+        assert_close(to_numpy(last), last_ref, "bf16", f"few heads last_state (flags {f})")
 
 
-def test_ssd_without_optional_inputs():
-    inp = gen.ssd_inputs(1, 256, 2, 64, 1, 64, seed=730)
+@pytest.mark.parametrize("N", [64, 128])
+def test_ssd_without_optional_inputs(N):
+    inp = gen.ssd_inputs(1, 256, 2, 64, 1, N, seed=730)
     y, last = mss.ssd_fwd(**_dev(inp, gate=False, with_D=False, with_bias=False))
     torch.cuda.synchronize()
     y_ref, last_ref = _ref(inp, gate=False, with_D=False, with_bias=False)
@@ -91,22 +106,25 @@ def test_ssd_without_optional_inputs():
     assert_close(to_numpy(last), last_ref, "bf16", "bare last_state")
 
 
+@pytest.mark.parametrize("kernel", sorted(KERNELS))
 @pytest.mark.parametrize("batch", [4, 1])
-def test_ssd_workload_sampled_heads(batch):
-    """The bench workload (4 x 4096 tokens, 64 heads of 64, N = 128; the
-    in-order kernel) and one sequence of it (the chunk-parallel passes): y and
-    the final state of sampled (batch, head) pairs against the oracle."""
+def test_ssd_workload_sampled_heads(batch, kernel):
+    """The bench workload (4 x 4096 tokens, 64 heads of 64, N = 128) and one
+    sequence of it, on each kernel (the warp-level kernels take the
+    chunk-parallel passes for the single sequence): y and the final state of
+    sampled (batch, head) pairs against the oracle."""
+    f = KERNELS[kernel]
     s = dict(gen.SSD_SHAPES[gen.SSD_WORKLOAD], batch=batch)
-    ws = mss.load_library().mss_ssd_fwd_workspace_size(batch, s["seqlen"], s["nheads"], s["headdim"],
-                                                        s["ngroups"], s["dstate"])
-    assert (ws > 0) == (batch == 1)
+    ws = mss.load_library().mss_ssd_fwd_workspace_size_ex(batch, s["seqlen"], s["nheads"], s["headdim"],
+                                                           s["ngroups"], s["dstate"], f)
+    assert (ws > 0) == (batch == 1 and f != 0)
     inp = gen.ssd_inputs(**s)
-    y, last = mss.ssd_fwd(**_dev(inp))
+    y, last = mss.ssd_fwd(**_dev(inp), flags=f)
     torch.cuda.synchronize()
     assert mss.get_device_error() == 0
     yn, ln = to_numpy(y), to_numpy(last)
     rng = np.random.default_rng(740)
-    for _ in range(3):
+    for _ in range(6):
         b, h = int(rng.integers(s["batch"])), int(rng.integers(s["nheads"]))
         sub = {k: (v.values[b:b + 1, :, h:h + 1] if k in ("x", "z", "dt") else v)
                for k, v in inp.items() if k in ("x", "z", "dt")}
@@ -117,13 +135,15 @@ def test_ssd_workload_sampled_heads(batch):
         assert_close(ln[b:b + 1, h:h + 1], last_ref, "bf16", f"state of (b={b}, h={h})")
 
 
-@pytest.mark.parametrize("L", [1, 63, 65])
+@pytest.mark.parametrize("kernel", sorted(KERNELS))
+@pytest.mark.parametrize("N", [64, 128])
+@pytest.mark.parametrize("L", [1, 63, 65, 127, 129])
 @pytest.mark.parametrize("chunks", ["parallel", "in-order"])
-def test_ssd_short_and_ragged_sequences(L, chunks):
-    """One token, one token short of a chunk, one token past it; every head
-    its own group (G = H)."""
-    inp = gen.ssd_inputs(1, L, 4, 64, 4, 64, seed=750 + L)
-    y, last = mss.ssd_fwd(**_dev(inp), workspace="auto" if chunks == "parallel" else None)
+def test_ssd_short_and_ragged_sequences(L, chunks, N, kernel):
+    """One token, one token short of a chunk, one token past it (chunks of 64
+    and of 128 tokens); every head its own group (G = H)."""
+    inp = gen.ssd_inputs(1, L, 4, 64, 4, N, seed=750 + L)
+    y, last = mss.ssd_fwd(**_dev(inp), workspace="auto" if chunks == "parallel" else None, flags=KERNELS[kernel])
     torch.cuda.synchronize()
     assert mss.get_device_error() == 0
     y_ref, last_ref = _ref(inp)

@@ -69,14 +69,15 @@ def test_noalloc_matches_the_workspace_path_on_two_calls_in_a_row():
 
 
 def test_noalloc_without_a_split_and_in_fp32():
-    """Calls that need no scratch (no split asked for, a short sequence: the
-    array is not touched) and an fp32 call that does, each against the
-    workspace entry point; the fp32 one also against the fp64 oracle."""
+    """Calls that need no scratch (no split asked for; enough channels to
+    fill the GPU: the array is not touched) and an fp32 call that does, each
+    against the workspace entry point; the fp32 one also against the fp64
+    oracle."""
     import oracle
 
     lib = _lib()
     cases = [("bf16", (1, 32, 16, 8192), mss.FLAG_NO_SPLIT, 0),
-             ("bf16", (2, 64, 16, 256), 0, 0),
+             ("bf16", (8, 2048, 16, 256), 0, 0),   # enough channels to fill the GPU: no split
              ("f32", (1, 16, 16, 4096), 0, 1)]
     for dtype, (batch, dim, N, L), flags, splits in cases:
         tdt = torch.bfloat16 if dtype == "bf16" else torch.float32
