@@ -23,6 +23,7 @@ from __future__ import annotations
 import argparse
 import hashlib
 import json
+import math
 import os
 import statistics
 import subprocess
@@ -455,6 +456,71 @@ def kernel_only(args, mss, d, y, state, w, dev, to_dev, rank):
     return 0
 
 
+def forward_record(w, ms_avg, ms_list, launches, segments=None, note=None):
+    """Throughput of one forward workload: CUDA-event time per call, channel-
+    tokens/s, algorithmic HBM GB/s and its fraction of the peak, and the
+    fraction of the fp32 lane-operation peak."""
+    peak, peak_kind, sm_max_mhz = measured_peaks()
+    esz = 2 if w.dtype == "bf16" else 4
+    nbytes = fwd_bytes(w.batch, w.dim, w.dstate, w.seqlen, esz=esz)
+    ops = fwd_alu_ops(w.batch, w.dim, w.dstate, w.seqlen)
+    ct = w.batch * w.dim * w.seqlen
+    rec = {"batch": w.batch, "d_inner": w.dim, "dstate": w.dstate, "seqlen": w.seqlen, "io_dtype": w.dtype,
+           "ms_avg": ms_avg, "ms_p10_p50_p90": [float(np.percentile(ms_list, q)) for q in (10, 50, 90)],
+           "launches_per_call": launches,
+           "channel_tokens_per_s": ct / (ms_avg * 1e-3),
+           "algorithmic_bytes": nbytes, "achieved_gbs": nbytes / (ms_avg * 1e-3) / 1e9,
+           "hbm_frac": nbytes / (ms_avg * 1e-3) / 1e9 / peak, "hbm_peak_kind": peak_kind,
+           "alu_frac": ops / (ms_avg * 1e-3) / alu_peak_ops(sm_max_mhz)}
+    if segments is not None:
+        rec["sequence_segments"] = segments
+    if note:
+        rec["note"] = note
+    return rec
+
+
+def time_workload(mss, name, args, dev, stream, rank):
+    """One forward workload timed alone: warm-up, then `steps` calls with CUDA
+    events around each (the call's launches: the fold pass and the full pass
+    where the sequence is split)."""
+    import torch
+
+    w = gen.WORKLOADS[name]
+    inp = gen.scan_inputs(w.batch, w.dim, w.dstate, w.seqlen, w.dtype, rank_seed(w.seed, rank), w.d_skip)
+    tdt = torch.bfloat16 if w.dtype == "bf16" else torch.float32
+
+    def to_dev(t):
+        if w.dtype == "f32":
+            return torch.from_numpy(np.ascontiguousarray(t.stored)).to(dev)
+        return torch.from_numpy(np.ascontiguousarray(t.stored).view(np.int16)).view(torch.bfloat16).to(dev)
+
+    d = dict(u=to_dev(inp["u"]), delta=to_dev(inp["delta"]), z=to_dev(inp["z"]), B=to_dev(inp["B"]),
+             C=to_dev(inp["C"]), A=torch.from_numpy(inp["A"]).to(dev), D=torch.from_numpy(inp["D"]).to(dev),
+             delta_bias=torch.from_numpy(inp["delta_bias"]).to(dev))
+    del inp
+    y = torch.empty_like(d["u"])
+    last = torch.empty(w.batch, w.dim, w.dstate, dtype=torch.float32, device=dev)
+    nbytes = mss.workspace_size(w.batch, w.dim, w.dstate, w.seqlen, tdt, device=dev)
+    ws = torch.empty(nbytes, dtype=torch.uint8, device=dev) if nbytes > 0 else None
+    evs = []
+    for i in range(args.warmup + args.steps):
+        a_, b_ = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a_.record(stream)
+        mss.scan_fwd(**d, y=y, last_state=last, workspace=ws)
+        b_.record(stream)
+        if i >= args.warmup:
+            evs.append((a_, b_))
+    torch.cuda.synchronize(dev)
+    ms_list = [a_.elapsed_time(b_) for a_, b_ in evs]
+    segs = None
+    if nbytes > 0:
+        # the split's aggregates take (segments - 1) * 2 * rows * N fp32 values
+        segs = 1 + nbytes // (2 * w.batch * w.dim * w.dstate * 4)
+    note = "launch-bound parity workload; its throughput says little" if w.seqlen * w.dim * w.batch < 1e6 else None
+    return forward_record(w, sum(ms_list) / len(ms_list), ms_list, launches=2 if segs else 1, segments=segs,
+                          note=note)
+
+
 def run_mss(args, rank, world, local_rank):
     import torch
     import torch.distributed as dist
@@ -540,9 +606,18 @@ def run_mss(args, rank, world, local_rank):
     assert mss.get_device_error() == 0
     if args.kernel_only:
         return kernel_only(args, mss, d, y, state, w, dev, to_dev, rank)
-    # the timed run keeps the clock sampler busy for at least ~2 s
-    k_clock = args.steps
-    ms, fwd_ms, clocks = timed(0, k_clock, args.warmup, with_clocks=True)
+    ms, fwd_ms, clocks = timed(0, args.steps, args.warmup, with_clocks=True)
+    assert mss.get_device_error() == 0
+
+    # the same step in a loop of at least 1.5 s with the clocks sampled
+    # throughout, so that the clock record of the step is long enough to read
+    reps = max(args.steps, int(math.ceil(1.5 / max(ms / args.steps * 1e-3, 1e-6))))
+    ms_loop, _, clocks_loop = timed(0, reps, args.warmup, with_clocks=True)
+    loop_step_ms = ms_loop / reps
+    clock_loop = {"steps": reps, "seconds": ms_loop * 1e-3, "ms_per_step": loop_step_ms,
+                  "clocks": clocks_loop,
+                  "ms_x_median_sm_mhz": (loop_step_ms * clocks_loop["sm_mhz"]
+                                         if clocks_loop and clocks_loop.get("sm_mhz") else None)}
     assert mss.get_device_error() == 0
     ms_gen, fwd_ms_gen, _ = timed(mss.FLAG_GENERAL_A, args.steps, args.warmup)
     ms_zoh, fwd_ms_zoh, _ = timed(mss.FLAG_ZOH_INPUT, args.steps, args.warmup)
@@ -566,6 +641,14 @@ def run_mss(args, rank, world, local_rank):
     conv_ms = [a_.elapsed_time(b_) for a_, b_ in conv_ms]
     assert mss.get_device_error() == 0
 
+    # the other forward workloads, each in the launch configuration the
+    # library picks (sequence split with its workspace where it applies)
+    workloads = {WORKLOAD: forward_record(w, sum(fwd_ms) / len(fwd_ms), fwd_ms, launches=1)}
+    for name in ("mamba130m-layer-bf16-b8-d1536-n16-l2048", "long-seq-bf16-b1-d2048-n16-l131072",
+                 "s6-fwd-fp32-b1-d16-n4-l256"):
+        workloads[name] = time_workload(mss, name, args, dev, stream, rank)
+        assert mss.get_device_error() == 0
+
     # the structured-state-space-duality (Mamba-2) layer: its own workload
     ss = gen.SSD_SHAPES[gen.SSD_WORKLOAD]
     sin = gen.ssd_inputs(**ss)
@@ -574,20 +657,26 @@ def run_mss(args, rank, world, local_rank):
               dt_bias=torch.from_numpy(sin["dt_bias"]).to(dev))
     ssd_y = torch.empty_like(sd["x"])
     ssd_last = torch.empty(ss["batch"], ss["nheads"], ss["dstate"], ss["headdim"], device=dev)
-    ssd_ev = []
-    for i in range(args.warmup + args.steps):
-        a_, b_ = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        a_.record(stream)
-        mss.ssd_fwd(**sd, y=ssd_y, last_state=ssd_last)
-        b_.record(stream)
-        if i >= args.warmup:
-            ssd_ev.append((a_, b_))
-    torch.cuda.synchronize(dev)
-    ssd_ms = sum(a_.elapsed_time(b_) for a_, b_ in ssd_ev) / len(ssd_ev)
-    assert mss.get_device_error() == 0
+
+    def time_ssd(flags):
+        ev = []
+        for i in range(args.warmup + args.steps):
+            a_, b_ = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            a_.record(stream)
+            mss.ssd_fwd(**sd, y=ssd_y, last_state=ssd_last, flags=flags)
+            b_.record(stream)
+            if i >= args.warmup:
+                ev.append((a_, b_))
+        torch.cuda.synchronize(dev)
+        assert mss.get_device_error() == 0
+        return sum(a_.elapsed_time(b_) for a_, b_ in ev) / len(ev)
+
+    ssd_ms = time_ssd(0)  # the tcgen05 kernel
+    ssd_ms_warp = time_ssd(mss.SSD_FLAG_WARP_MMA)  # the warp-level (mma.sync) kernel, for comparison
     del sd, ssd_y, sin
-    # matrix-form flops per (token, head): C B^T and M X within the chunk, C S
-    # and the state product B^T X across chunks (chunk of 64, P = 64)
+    # matrix-form flops per (token, head) of the tcgen05 kernel's chunks of
+    # 128 tokens: C B^T and M X within the chunk, C S and the state product
+    # B^T X across chunks (P = 64)
     # algorithmic bytes: x, z read and y written (bf16), dt read, B and C read
     # once per (batch, token, group), A, D, dt_bias, and last_state written
     ssd_bytes = (3 * ss["batch"] * ss["seqlen"] * ss["nheads"] * ss["headdim"] * 2
@@ -595,7 +684,7 @@ def run_mss(args, rank, world, local_rank):
                  + 2 * ss["batch"] * ss["seqlen"] * ss["ngroups"] * ss["dstate"] * 2
                  + 3 * ss["nheads"] * 4 + ss["batch"] * ss["nheads"] * ss["dstate"] * ss["headdim"] * 4)
     ssd_flops = ss["batch"] * ss["seqlen"] * ss["nheads"] * (
-        2 * 64 * ss["dstate"] + 2 * 64 * ss["headdim"] + 2 * ss["dstate"] * ss["headdim"] * 2)
+        2 * 128 * ss["dstate"] + 2 * 128 * ss["headdim"] + 2 * ss["dstate"] * ss["headdim"] * 2)
 
     # the backward pass (gradients of every input, states recomputed from
     # checkpoints) on the same workload
@@ -773,7 +862,12 @@ def run_mss(args, rank, world, local_rank):
                                          "frac": ssd_flops / (ssd_ms * 1e-3) / 1e12 / measured_bf16_tflops()[0],
                                          "peak_kind": measured_bf16_tflops()[1],
                                          "time_at_peak_us": ssd_flops / (measured_bf16_tflops()[0] * 1e6),
-                                         "note": "bf16 mma.sync products, fp32 accumulation"}},
+                                         "note": "tcgen05.mma bf16 products, fp32 accumulators in TMEM, "
+                                                 "chunks of 128 tokens"},
+                     "warp_mma_kernel": {"ms_avg": ssd_ms_warp,
+                                         "achieved_gbs": ssd_bytes / (ssd_ms_warp * 1e-3) / 1e9,
+                                         "note": "the warp-level mma.sync kernel (chunks of 64), "
+                                                 "MSS_SSD_FLAG_WARP_MMA"}},
         "zoh_input_path": {"fwd_ms_avg": fwd_avg_zoh,
                            "achieved_gbs": bytes_fwd / (fwd_avg_zoh * 1e-3) / 1e9,
                            "frac": bytes_fwd / (fwd_avg_zoh * 1e-3) / 1e9 / peak,
@@ -788,6 +882,8 @@ def run_mss(args, rank, world, local_rank):
                 "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
         "gpu_launches": launches_per_step * args.steps,
         "clocks": clocks,
+        "clock_loop": clock_loop,
+        "workloads": workloads,
         "kernel_source_sha": kernel_source_hash(),
     }
     if rank == 0 and world == 1 and not args.no_cpu_baseline:

@@ -6,8 +6,8 @@
 // 1-semiseparable matrix M_ij = exp(cs_i - cs_j) (C_i . B_j) Delta_j (j <= i,
 // cs the running sum of Delta A over the chunk) plus the state carried in
 // from earlier chunks ("NN Lab -- Mamba", Structured State Space Duality;
-// "Mamba" paper review, section "Mamba 2").  One CTA of eight warps serves one
-// (batch, head) and walks its chunks of Q = 128 tokens in order.  Per chunk:
+// "Mamba" paper review, section "Mamba 2").  One CTA of sixteen warps serves
+// one (batch, head) and walks its chunks of Q = 128 tokens in order.  Per chunk:
 //
 //   G   = C B^T                   (128 x 128, K = N)     TMEM columns   0..127
 //   dS  = B^T diag(w) X,  w_j = exp(cs_last - cs_j) Delta_j
@@ -18,10 +18,12 @@
 //   S   = exp(cs_last) S_prev + dS        (fp32, registers)
 //   y   = (Ym + exp(cs_i) Yx + D x) silu(z)  -> smem -> TMA store
 //
-// Thread t of the CTA owns TMEM lane (and row) t % 128 and half t / 128 of the
-// columns of each product it reads.  The fp32 state S (N x P) lives in
-// registers (thread t: row n = t % 128, columns 32 (t / 128) ..), its bf16
-// copy in shared memory is the B operand of the next chunk's C S_prev.
+// Thread t of the CTA owns TMEM lane (and row) t % 128 and quarter t / 128 of
+// the columns of each product it reads (four warps share each 32-lane TMEM
+// quarter).  The fp32 state S (N x P) lives in registers (thread t: row
+// n = t % 128, columns 16 (t / 128) ..), its bf16 copy in shared memory is the
+// B operand of the next chunk's C S_prev.  Sixteen warps (four per scheduler)
+// hide the latencies of the TMEM loads, the exponentials and the barriers.
 // Operands: C and B tiles [128 tokens][64 state] x 2 and X [128 tokens][64]
 // in the 128-byte swizzle TMA writes, double buffered (the next chunk's
 // loads run during this one); M, X_w and the state copy are written by the
@@ -50,37 +52,43 @@ struct SsdTcMaps {
 
 struct SsdTcLayout {
     static constexpr int kQ = 128, kP = 64, kN = 128;
-    static constexpr int kThreads = 256;
+    static constexpr int kThreads = 512;
     static constexpr int kBox = 16384;  // one [128][64] bf16 tile
     // stage: C (two boxes along N), B (two boxes), X
     static constexpr int kC = 0, kB = 2 * kBox, kX = 4 * kBox;
     static constexpr int kStageBytes = 5 * kBox;
-    static constexpr int kM = 2 * kStageBytes;    // masked scores, bf16, two boxes along K
-    static constexpr int kXw = kM + 2 * kBox;     // w-scaled X; then the y tile of the same chunk
+    static constexpr int kM = 2 * kStageBytes;    // masked scores, bf16, two boxes along K; then y's tile
+    static constexpr int kXw = kM + 2 * kBox;     // w-scaled X
     static constexpr int kS = kXw + kBox;         // bf16 copy of the state [128 n][64 p]
-    static constexpr int kScal = kS + kBox;       // per token: Delta, cs (log2 units); warp sums
-    static constexpr int kBars = kScal + 2 * kQ * 4 + 64;
-    static constexpr int kTmemSlot = kBars + 4 * 8;
+    // per token of the chunk: Delta, cs in log2 units, and the column factor
+    // f_j = exp2(cs_L - cs_j) Delta_j of the masked scores (L the last token of
+    // j's 32-token block); read up to the masked scores, then rewritten for the
+    // next chunk (each thread keeps the values its output step needs)
+    static constexpr int kScal = kS + kBox;
+    static constexpr int kBars = kScal + 3 * kQ * 4;
+    static constexpr int kTmemSlot = kBars + 5 * 8;
     static constexpr int kSmemBytes = kTmemSlot + 16 + 1024;  // + base alignment slack
     static constexpr uint32_t kTmemCols = 512;
     static constexpr uint32_t kColG = 0, kColYm = 128, kColYx = 192, kColS = 256;
 };
 
 template <bool kGate, bool kSoftplus>
-__global__ void __launch_bounds__(256, 1) ssd_tc_kernel(const __grid_constant__ SsdTcMaps maps, SsdParams p) {
+__global__ void __launch_bounds__(512, 1) ssd_tc_kernel(const __grid_constant__ SsdTcMaps maps, SsdParams p) {
     using Ly = SsdTcLayout;
     constexpr int Q = Ly::kQ, P = Ly::kP, NS = Ly::kN;
     extern __shared__ __align__(16) uint8_t smem_raw[];
     uint8_t* smem = smem_raw + ((1024u - (smem_addr(smem_raw) & 1023u)) & 1023u);
-    float* dts = reinterpret_cast<float*>(smem + Ly::kScal);  // Delta (0 past the sequence)
-    float* css = dts + Q;                                     // cs * log2(e)
-    float* wsum = css + Q;                                    // warp totals of the scan
+    float* dts = reinterpret_cast<float*>(smem + Ly::kScal);  // [Q] Delta (0 past the sequence)
+    float* css = dts + Q;                                     // [Q] cs * log2(e)
+    float* fss = css + Q;                                     // [Q] column factors of the scores
     uint64_t* full = reinterpret_cast<uint64_t*>(smem + Ly::kBars);  // [2] TMA stages
-    uint64_t* mbar = full + 2;                                       // MMA completion
+    uint64_t* gbar = full + 2;  // C B^T complete
+    uint64_t* mbar = full + 3;  // B^T X_w and C S_prev complete
+    uint64_t* ybar = full + 4;  // M X complete
     uint32_t* tslot = reinterpret_cast<uint32_t*>(smem + Ly::kTmemSlot);
 
     const int tid = threadIdx.x, warp = tid >> 5;
-    const int row = tid & 127, half = tid >> 7;
+    const int row = tid & 127, qd = tid >> 7;  // TMEM lane / row, column quarter
     const int64_t H = p.nheads, L = p.seqlen;
     const int64_t b = blockIdx.x / H, h = blockIdx.x % H;
     const int g = int(h / (H / p.ngroups));
@@ -90,9 +98,7 @@ __global__ void __launch_bounds__(256, 1) ssd_tc_kernel(const __grid_constant__ 
     const int n_chunks = int((L + Q - 1) / Q);
 
     if (tid == 0) {
-        mbar_init(full, 1);
-        mbar_init(full + 1, 1);
-        mbar_init(mbar, 1);
+        for (int k = 0; k < 5; ++k) mbar_init(full + k, 1);
         fence_barrier_init();
         prefetch_tensormap(&maps.x);
         prefetch_tensormap(&maps.B);
@@ -126,74 +132,128 @@ __global__ void __launch_bounds__(256, 1) ssd_tc_kernel(const __grid_constant__ 
         if (n_chunks > 1) issue_chunk(1);
     }
 
-    // the state: row n = `row`, columns 32 * half .. + 31
-    float S[32];
+    // the state: row n = `row`, columns 16 * qd .. + 15
+    float S[16];
     {
-        const float* s0 = p.initial_state ? p.initial_state + ((b * H + h) * NS + row) * P + 32 * half : nullptr;
+        const float* s0 = p.initial_state ? p.initial_state + ((b * H + h) * NS + row) * P + 16 * qd : nullptr;
 #pragma unroll
-        for (int k = 0; k < 32; ++k) S[k] = s0 ? s0[k] : 0.f;
+        for (int k = 0; k < 16; ++k) S[k] = s0 ? s0[k] : 0.f;
     }
     auto write_state_copy = [&]() {
         uint8_t* Ss = smem + Ly::kS;
 #pragma unroll
-        for (int q = 0; q < 4; ++q) {
+        for (int q = 0; q < 2; ++q) {
             uint4 v = make_uint4(pack_bf16x2(S[8 * q], S[8 * q + 1]), pack_bf16x2(S[8 * q + 2], S[8 * q + 3]),
                                  pack_bf16x2(S[8 * q + 4], S[8 * q + 5]), pack_bf16x2(S[8 * q + 6], S[8 * q + 7]));
-            *reinterpret_cast<uint4*>(Ss + sw128(row, 4 * half + q)) = v;
+            *reinterpret_cast<uint4*>(Ss + sw128(row, 2 * qd + q)) = v;
         }
     };
     write_state_copy();
     fence_proxy_async_smem();
 
     bool ok = true;
-    uint32_t mphase = 0;
     constexpr uint32_t idG = idesc_bf16_f32(128, 128, 0, 0);
     constexpr uint32_t idK = idesc_bf16_f32(128, 64, 0, 1);   // K-major A, N-major B
     constexpr uint32_t idMN = idesc_bf16_f32(128, 64, 1, 1);  // M-major A, N-major B
     const uint32_t sbase = smem_addr(smem);
+    const bf16_t* dtp = static_cast<const bf16_t*>(p.dt) + b * L * H + h;
+    const int lane = tid & 31;
 
+    // Warp 0 prepares each chunk's step sizes and their running sum ahead of
+    // it: lane l takes tokens 4l .. 4l+3 (raw steps loaded one chunk earlier
+    // still), a warp scan adds the lanes' totals.  Results go to the scalar
+    // buffer of the chunk's parity.
+    float raw[4];
+    auto load_raw = [&](int c) {
+#pragma unroll
+        for (int k = 0; k < 4; ++k) {
+            const int64_t t = int64_t(c) * Q + 4 * lane + k;
+            raw[k] = t < L ? ld(dtp + t * H) : 0.f;
+        }
+    };
+    auto scan_chunk = [&](int c) {
+        float d[4], a[4], run = 0.f;
+#pragma unroll
+        for (int k = 0; k < 4; ++k) {
+            const bool valid = int64_t(c) * Q + 4 * lane + k < L;
+            const float s0 = raw[k] + bias;
+            d[k] = valid ? (kSoftplus ? softplus_fast(s0) : s0) : 0.f;
+            run += d[k] * A2;
+            a[k] = run;
+        }
+        float incl = run;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+            const float v = __shfl_up_sync(0xffffffffu, incl, o);
+            if (lane >= o) incl += v;
+        }
+        const float excl = incl - run;
+#pragma unroll
+        for (int k = 0; k < 4; ++k) a[k] += excl;
+        // the last token of this lane's 32-token block is token 3 of lane 8 (l / 8) + 7
+        const float cL = __shfl_sync(0xffffffffu, a[3], (lane & ~7) | 7);
+        reinterpret_cast<float4*>(dts)[lane] = make_float4(d[0], d[1], d[2], d[3]);
+        reinterpret_cast<float4*>(css)[lane] = make_float4(a[0], a[1], a[2], a[3]);
+        reinterpret_cast<float4*>(fss)[lane] =
+            make_float4(ex2_approx(cL - a[0]) * d[0], ex2_approx(cL - a[1]) * d[1], ex2_approx(cL - a[2]) * d[2],
+                        ex2_approx(cL - a[3]) * d[3]);
+    };
+    if (warp == 0) {
+        load_raw(0);
+        scan_chunk(0);
+        if (n_chunks > 1) load_raw(1);
+    }
+    __syncthreads();
+
+    // issue C B^T of chunk c once its tiles have landed (thread 0)
+    auto issue_scores = [&](int c) -> bool {
+        const uint32_t st = sbase + uint32_t((c & 1) * Ly::kStageBytes);
+        if (!mbar_wait_bounded(full + (c & 1), uint32_t((c >> 1) & 1), p.err)) return false;
+        tc_fence_after_sync();
+#pragma unroll
+        for (int k = 0; k < NS / 16; ++k) {
+            const uint32_t off = uint32_t((k >> 2) * Ly::kBox + (k & 3) * 32);
+            umma_bf16(tmem + Ly::kColG, smem_desc_sw128(st + Ly::kC + off, 16, 1024),
+                      smem_desc_sw128(st + Ly::kB + off, 16, 1024), idG, k > 0);
+        }
+        umma_commit(gbar);
+        return true;
+    };
+
+    bool abort = false;  // a bounded wait of this thread gave up (folded into the next CTA barrier)
     for (int c = 0; c < n_chunks && ok; ++c) {
         const int t0 = c * Q;
+        const uint32_t ph = uint32_t(c & 1);  // each completion barrier completes once per chunk
         const uint32_t st = sbase + uint32_t((c & 1) * Ly::kStageBytes);
-        // the previous chunk's y store must have read its tile (the X_w bytes)
-        if (tid == 0) bulk_wait_read<0>();
-        // step sizes and their running sum over the chunk (log2 units)
-        if (tid < Q) {
-            float d = 0.f;
-            if (t0 + tid < L) {
-                const float raw = ld(static_cast<const bf16_t*>(p.dt) + ((b * L + t0 + tid) * H + h)) + bias;
-                d = kSoftplus ? softplus_fast(raw) : raw;
-            }
-            float a = d * A2;
+        const float* dtc = dts;
+        const float* csc = css;
+        // thread 0: the chunk's scores start on the tensor cores at once; the
+        // previous chunk's y store must have read its tile (the first box of
+        // the score tile, rewritten after the next barrier)
+        if (tid == 0) {
+            abort |= !issue_scores(c);
+            bulk_wait_read<0>();
+        }
+        // z of this chunk's rows, in registers until the output step
+        uint4 zr[2];
+        if constexpr (kGate) {
+            const int64_t tok = t0 + row;
+            const bf16_t* zp = static_cast<const bf16_t*>(p.z) + ((b * L + tok) * H + h) * P + 16 * qd;
 #pragma unroll
-            for (int o = 1; o < 32; o <<= 1) {
-                const float v = __shfl_up_sync(0xffffffffu, a, o);
-                if ((tid & 31) >= o) a += v;
-            }
-            dts[tid] = d;
-            css[tid] = a;
-            if ((tid & 31) == 31) wsum[warp] = a;
+            for (int q = 0; q < 2; ++q)
+                zr[q] = tok < L ? *reinterpret_cast<const uint4*>(zp + 8 * q) : make_uint4(0u, 0u, 0u, 0u);
         }
-        const bool landed = mbar_wait_bounded(full + (c & 1), uint32_t((c >> 1) & 1), p.err);
-        if (__syncthreads_or(!landed)) {
-            ok = false;
-            break;
-        }
-        if (tid < Q) {
-            float off = 0.f;
-            for (int w = 0; w < (tid >> 5); ++w) off += wsum[w];
-            css[tid] += off;
-        }
-        __syncthreads();
-        const float cl = css[Q - 1];
-        // X_w = w_j x_j (row j = `row`, this thread's half of the 64 columns)
+        abort |= !mbar_wait_bounded(full + (c & 1), uint32_t((c >> 1) & 1), p.err);
+        const float cl = csc[Q - 1];
+        const float ci = csc[row];  // kept for the output step (the next chunk's scan rewrites css)
+        // X_w = w_j x_j (row j = `row`, this thread's quarter of the 64 columns)
         {
-            const float wj = ex2_approx(cl - css[row]) * dts[row];
+            const float wj = ex2_approx(cl - ci) * dtc[row];
             const uint8_t* xs = smem + (c & 1) * Ly::kStageBytes + Ly::kX;
             uint8_t* xw = smem + Ly::kXw;
 #pragma unroll
-            for (int q = 0; q < 4; ++q) {
-                const uint32_t off = sw128(row, 4 * half + q);
+            for (int q = 0; q < 2; ++q) {
+                const uint32_t off = sw128(row, 2 * qd + q);
                 const uint4 v = *reinterpret_cast<const uint4*>(xs + off);
                 const uint32_t w4[4] = {v.x, v.y, v.z, v.w};
                 uint32_t o4[4];
@@ -203,16 +263,13 @@ __global__ void __launch_bounds__(256, 1) ssd_tc_kernel(const __grid_constant__ 
             }
         }
         fence_proxy_async_smem();
-        __syncthreads();
-        // G = C B^T, dS = B^T X_w, Yx = C S_prev
+        if (__syncthreads_or(abort)) {
+            ok = false;
+            break;
+        }
+        // dS = B^T X_w and Yx = C S_prev, while the scores are masked
         if (tid == 0) {
             tc_fence_after_sync();
-#pragma unroll
-            for (int k = 0; k < NS / 16; ++k) {
-                const uint32_t off = uint32_t((k >> 2) * Ly::kBox + (k & 3) * 32);
-                umma_bf16(tmem + Ly::kColG, smem_desc_sw128(st + Ly::kC + off, 16, 1024),
-                          smem_desc_sw128(st + Ly::kB + off, 16, 1024), idG, k > 0);
-            }
 #pragma unroll
             for (int k = 0; k < Q / 16; ++k) {
                 const uint32_t off = uint32_t(k * 2048);
@@ -227,43 +284,69 @@ __global__ void __launch_bounds__(256, 1) ssd_tc_kernel(const __grid_constant__ 
             }
             umma_commit(mbar);
         }
-        if (__syncthreads_or(!mbar_wait_bounded(mbar, mphase, p.err))) {
-            ok = false;
-            break;
-        }
-        mphase ^= 1u;
+        abort |= !mbar_wait_bounded(gbar, ph, p.err);
         tc_fence_after_sync();
-        // M_ij = G_ij exp(cs_i - cs_j) Delta_j for j <= i, this thread's 64 columns j
+        // M_ij = G_ij exp(cs_i - cs_j) Delta_j for j <= i, this thread's 32 columns j
+        // (box qd / 2 of the two 64-wide K boxes, pieces 4 (qd % 2) ..).  A
+        // warp's 32 rows against a quarter of 32 columns to their right are all
+        // masked (rows 32 (warp % 4) .. < columns 32 qd ..): zeros, with no TMEM
+        // load and no exponential (a warp-uniform branch).
         {
-            const float ci = css[row];
-            uint8_t* Ms = smem + Ly::kM + half * Ly::kBox;
+            uint8_t* Ms = smem + Ly::kM + (qd >> 1) * Ly::kBox;
+            if ((warp & 3) < qd) {
 #pragma unroll
-            for (int part = 0; part < 2; ++part) {
+                for (int q = 0; q < 4; ++q)
+                    *reinterpret_cast<uint4*>(Ms + sw128(row, 4 * (qd & 1) + q)) = make_uint4(0u, 0u, 0u, 0u);
+            } else {
                 float gv[32];
-                tmem_ld32(tlane + Ly::kColG + uint32_t(64 * half + 32 * part), gv);
+                tmem_ld32(tlane + Ly::kColG + uint32_t(32 * qd), gv);
                 tmem_wait_ld();
+                // A block wholly below the diagonal (every j <= i): exp2(cs_i - cs_j)
+                // = exp2(cs_i - cs_L) exp2(cs_L - cs_j) with L = 32 qd + 31 <= i;
+                // both exponents are <= 0 for A <= 0, so neither factor overflows,
+                // and the column factor (times Delta_j) is shared by every row.
+                if ((warp & 3) > qd) {
+                    const float ri = ex2_approx(ci - csc[32 * qd + 31]);
+                    const float4* f4 = reinterpret_cast<const float4*>(fss + 32 * qd);
 #pragma unroll
-                for (int q = 0; q < 4; ++q) {
-                    uint32_t o4[4];
+                    for (int q = 0; q < 4; ++q) {
+                        const float4 fa = f4[2 * q], fb = f4[2 * q + 1];
+                        const float f[8] = {fa.x, fa.y, fa.z, fa.w, fb.x, fb.y, fb.z, fb.w};
+                        uint32_t o4[4];
 #pragma unroll
-                    for (int k = 0; k < 4; ++k) {
-                        float m2[2];
-#pragma unroll
-                        for (int e = 0; e < 2; ++e) {
-                            const int jj = 8 * q + 2 * k + e;          // 0..31 within this part
-                            const int j = 64 * half + 32 * part + jj;  // token index in the chunk
-                            m2[e] = j <= row ? gv[jj] * ex2_approx(ci - css[j]) * dts[j] : 0.f;
-                        }
-                        o4[k] = pack_bf16x2(m2[0], m2[1]);
+                        for (int k = 0; k < 4; ++k)
+                            o4[k] = pack_bf16x2(gv[8 * q + 2 * k] * ri * f[2 * k], gv[8 * q + 2 * k + 1] * ri * f[2 * k + 1]);
+                        *reinterpret_cast<uint4*>(Ms + sw128(row, 4 * (qd & 1) + q)) =
+                            make_uint4(o4[0], o4[1], o4[2], o4[3]);
                     }
-                    *reinterpret_cast<uint4*>(Ms + sw128(row, 4 * part + q)) = make_uint4(o4[0], o4[1], o4[2], o4[3]);
+                } else {
+#pragma unroll
+                    for (int q = 0; q < 4; ++q) {
+                        uint32_t o4[4];
+#pragma unroll
+                        for (int k = 0; k < 4; ++k) {
+                            float m2[2];
+#pragma unroll
+                            for (int e = 0; e < 2; ++e) {
+                                const int jj = 8 * q + 2 * k + e;  // 0..31 within this quarter
+                                const int j = 32 * qd + jj;        // token index in the chunk
+                                m2[e] = j <= row ? gv[jj] * ex2_approx(ci - csc[j]) * dtc[j] : 0.f;
+                            }
+                            o4[k] = pack_bf16x2(m2[0], m2[1]);
+                        }
+                        *reinterpret_cast<uint4*>(Ms + sw128(row, 4 * (qd & 1) + q)) =
+                            make_uint4(o4[0], o4[1], o4[2], o4[3]);
+                    }
                 }
             }
         }
         tc_fence_before_sync();
         fence_proxy_async_smem();
-        __syncthreads();
-        // Ym = M X
+        if (__syncthreads_or(abort)) {
+            ok = false;
+            break;
+        }
+        // Ym = M X; meanwhile warp 0 prepares the next chunk's step sizes
         if (tid == 0) {
             tc_fence_after_sync();
 #pragma unroll
@@ -272,45 +355,51 @@ __global__ void __launch_bounds__(256, 1) ssd_tc_kernel(const __grid_constant__ 
                 umma_bf16(tmem + Ly::kColYm, smem_desc_sw128(sbase + Ly::kM + offa, 16, 1024),
                           smem_desc_sw128(st + Ly::kX + uint32_t(k * 2048), 0, 1024), idK, k > 0);
             }
-            umma_commit(mbar);
+            umma_commit(ybar);
         }
-        if (__syncthreads_or(!mbar_wait_bounded(mbar, mphase, p.err))) {
-            ok = false;
-            break;
+        if (warp == 0 && c + 1 < n_chunks) {
+            __syncwarp();
+            scan_chunk(c + 1);
+            if (c + 2 < n_chunks) load_raw(c + 2);
         }
-        mphase ^= 1u;
+        // the state: S = exp(cs_last) S + dS, and its bf16 copy for the next
+        // chunk (C S_prev has read the old copy: it completed with dS)
+        abort |= !mbar_wait_bounded(mbar, ph, p.err);
         tc_fence_after_sync();
-        // the state: S = exp(cs_last) S + dS, and its bf16 copy for the next chunk
         {
-            float ds[32];
-            tmem_ld32(tlane + Ly::kColS + uint32_t(32 * half), ds);
+            float ds[16];
+            tmem_ld16(tlane + Ly::kColS + uint32_t(16 * qd), ds);
             tmem_wait_ld();
             const float dec = ex2_approx(cl);
 #pragma unroll
-            for (int k = 0; k < 32; ++k) S[k] = fmaf(dec, S[k], ds[k]);
+            for (int k = 0; k < 16; ++k) S[k] = fmaf(dec, S[k], ds[k]);
             write_state_copy();
         }
-        // y = (Ym + exp(cs_i) Yx + D x) silu(z) for row i = `row`, this half's 32 columns
+        abort |= !mbar_wait_bounded(ybar, ph, p.err);
+        tc_fence_after_sync();
+        // y = (Ym + exp(cs_i) Yx + D x) silu(z) for row i = `row`, this
+        // quarter's 16 columns, staged in the score tile's first box (M X has
+        // read it) for the store
         {
-            float ym[32], yx[32];
-            tmem_ld32(tlane + Ly::kColYm + uint32_t(32 * half), ym);
-            tmem_ld32(tlane + Ly::kColYx + uint32_t(32 * half), yx);
+            float ym[16], yx[16];
+            tmem_ld16(tlane + Ly::kColYm + uint32_t(16 * qd), ym);
+            tmem_ld16(tlane + Ly::kColYx + uint32_t(16 * qd), yx);
             tmem_wait_ld();
-            const float ei = ex2_approx(css[row]);
-            const int64_t tok = t0 + row;
-            const bool valid = tok < L;
+            const float ei = ex2_approx(ci);
             const uint8_t* xs = smem + (c & 1) * Ly::kStageBytes + Ly::kX;
-            uint8_t* ys = smem + Ly::kXw;
-            const bf16_t* zr = kGate && valid ? static_cast<const bf16_t*>(p.z) + ((b * L + tok) * H + h) * P + 32 * half
-                                              : nullptr;
+            uint8_t* ys = smem + Ly::kM;
 #pragma unroll
-            for (int q = 0; q < 4; ++q) {
-                const uint32_t off = sw128(row, 4 * half + q);
+            for (int q = 0; q < 2; ++q) {
+                const uint32_t off = sw128(row, 2 * qd + q);
                 const uint4 xv = *reinterpret_cast<const uint4*>(xs + off);
                 const uint32_t x4[4] = {xv.x, xv.y, xv.z, xv.w};
-                uint4 zv = make_uint4(0u, 0u, 0u, 0u);
-                if (kGate && valid) zv = *reinterpret_cast<const uint4*>(zr + 8 * q);
-                const uint32_t z4[4] = {zv.x, zv.y, zv.z, zv.w};
+                uint32_t z4[4] = {0u, 0u, 0u, 0u};
+                if constexpr (kGate) {
+                    z4[0] = zr[q].x;
+                    z4[1] = zr[q].y;
+                    z4[2] = zr[q].z;
+                    z4[3] = zr[q].w;
+                }
                 uint32_t o4[4];
 #pragma unroll
                 for (int k = 0; k < 4; ++k) {
@@ -328,23 +417,28 @@ __global__ void __launch_bounds__(256, 1) ssd_tc_kernel(const __grid_constant__ 
         }
         tc_fence_before_sync();
         fence_proxy_async_smem();
-        __syncthreads();
+        if (__syncthreads_or(abort)) {
+            ok = false;
+            break;
+        }
         if (tid == 0) {
-            tma_store_4d(&maps.y, smem + Ly::kXw, 0, int(h), t0, int(b));
+            tma_store_4d(&maps.y, smem + Ly::kM, 0, int(h), t0, int(b));
             bulk_commit();
             if (c + 2 < n_chunks) issue_chunk(c + 2);
         }
     }
     if (!ok && tid == 0) {
         // give the copies and products still in flight a bounded chance to land
-        for (int s = 0; s < 2; ++s) mbar_wait_bounded(full + s, 0u, nullptr, 100000000ull);
-        mbar_wait_bounded(mbar, mphase, nullptr, 100000000ull);
+        for (int k = 0; k < 5; ++k) {
+            mbar_wait_bounded(full + k, 0u, nullptr, 50000000ull);
+            mbar_wait_bounded(full + k, 1u, nullptr, 50000000ull);
+        }
     }
     if (tid == 0) bulk_wait<0>();
     if (ok && p.last_state) {
-        float* ls = p.last_state + ((b * H + h) * NS + row) * P + 32 * half;
+        float* ls = p.last_state + ((b * H + h) * NS + row) * P + 16 * qd;
 #pragma unroll
-        for (int k = 0; k < 32; k += 4) *reinterpret_cast<float4*>(ls + k) = make_float4(S[k], S[k + 1], S[k + 2], S[k + 3]);
+        for (int k = 0; k < 16; k += 4) *reinterpret_cast<float4*>(ls + k) = make_float4(S[k], S[k + 1], S[k + 2], S[k + 3]);
     }
     tc_fence_before_sync();
     __syncthreads();
