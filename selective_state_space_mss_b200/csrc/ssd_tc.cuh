@@ -29,6 +29,20 @@
 // loads run during this one); M, X_w and the state copy are written by the
 // threads in the same layout.  One thread issues the MMAs and the TMA copies.
 //
+// Order within a chunk, with three CTA barriers: C B^T starts as soon as the
+// chunk's tiles land; the threads scale X (barrier); B^T X_w and C S_prev
+// start, and the threads mask and decay the scores as soon as C B^T is done
+// (barrier); M X starts while warp 0 prepares the next chunk's step sizes and
+// decay sums (their raw steps and this chunk's z were loaded a chunk ahead);
+// the state update waits only for B^T X_w, the output only for M X
+// (barrier); then the y store and the loads of chunk c + 2.  Each thread
+// waits on the MMA completion barriers itself; a wait that gives up is
+// folded into the next CTA barrier.  Score blocks of 32 x 32 wholly above
+// the diagonal are skipped by the warp; blocks wholly below it use
+// exp2(cs_i - cs_j) = exp2(cs_i - cs_L) exp2(cs_L - cs_j) (L the block's last
+// column), both factors at most one for A <= 0, with the column factor
+// shared by every row, so they need no exponential per score.
+//
 // Waits are bounded (~2 s): on a timeout the CTA sets the device error word,
 // gives its copies and products in flight a bounded chance to finish, frees
 // its TMEM and returns.

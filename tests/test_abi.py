@@ -298,25 +298,47 @@ def test_ssd_argument_errors(lib):
 def test_ssd_workspace_queries(lib):
     codes = _enum("mss_status")
     lib.mss_ssd_fwd_workspace_size.restype = ctypes.c_int64
+    lib.mss_ssd_fwd_workspace_size_ex.restype = ctypes.c_int64
     q = lambda *a: lib.mss_ssd_fwd_workspace_size(*[ctypes.c_int64(x) for x in a])
-    # 8 (batch, head) pairs: the chunk-parallel passes on a device (per chunk of
-    # 64 tokens the fp32 chunk state, its bf16 copy and the decay); without a
-    # device the in-order kernel, which takes no workspace
-    ws = q(2, 128, 4, 64, 1, 128)
-    assert ws == (2 * 4 * 2 * (128 * 64 * 6 + 4) if torch.cuda.is_available() else 0)
+    qx = lambda *a, flags=0: lib.mss_ssd_fwd_workspace_size_ex(*[ctypes.c_int64(x) for x in a], ctypes.c_uint(flags))
+    warp = 0x1  # MSS_SSD_FLAG_WARP_MMA
+    chunked = 2 * 4 * 2 * (128 * 64 * 6 + 4)  # per chunk of 64 tokens: fp32 chunk state, its bf16 copy, decay
+    # 8 (batch, head) pairs take the warp-level chunk-parallel passes on a
+    # device; without a device the in-order kernel, which takes no workspace
+    ws = q(2, 128, 4, 64, 1, 64)
+    assert ws == (2 * 4 * 2 * (64 * 64 * 6 + 4) if torch.cuda.is_available() else 0)
+    assert qx(2, 128, 4, 64, 1, 128, flags=warp) == (chunked if torch.cuda.is_available() else 0)
+    # dstate 128 runs the tcgen05 kernel in order: no workspace
+    assert q(2, 128, 4, 64, 1, 128) == 0 and qx(2, 128, 4, 64, 1, 128) == 0
     assert q(2, 0, 4, 64, 1, 128) == 0
     assert q(2, 128, 4, 32, 1, 128) == codes["MSS_ERR_SHAPE"]
     assert q(2, 128, 3, 64, 2, 128) == codes["MSS_ERR_SHAPE"]
+    assert qx(2, 128, 4, 64, 1, 128, flags=0x2) == codes["MSS_ERR_FLAGS"]
     if ws == 0 and torch.cuda.is_available():
         return  # the call below would launch on the made-up pointers
     lib.mss_ssd_fwd_ex.restype = ctypes.c_int
     v = ctypes.c_void_p
     rc = lib.mss_ssd_fwd_ex(v(P), v(P + 0x1000000), v(P + 0x2000000), v(P + 0x3000000), v(P + 0x4000000), None,
                             None, None, 1, None, v(P + 0x5000000), None, ctypes.c_int64(2), ctypes.c_int64(128),
-                            ctypes.c_int64(4), ctypes.c_int64(64), ctypes.c_int64(1), ctypes.c_int64(128), 1,
+                            ctypes.c_int64(4), ctypes.c_int64(64), ctypes.c_int64(1), ctypes.c_int64(64), 1,
                             v(P + 0x6000000), ctypes.c_int64(100), None)
     # too small (checked before any launch), or no device to launch on
     assert rc == (codes["MSS_ERR_WORKSPACE"] if ws else codes["MSS_ERR_CUDA"])
+
+
+def test_ssd_ex2_flag_errors(lib):
+    codes = _enum("mss_status")
+    lib.mss_ssd_fwd_ex2.restype = ctypes.c_int
+    v = ctypes.c_void_p
+
+    def call(flags, dtype=1):
+        return lib.mss_ssd_fwd_ex2(v(P), v(P + 0x1000000), v(P + 0x2000000), v(P + 0x3000000), v(P + 0x4000000),
+                                   None, None, None, 1, None, v(P + 0x5000000), None, ctypes.c_int64(2),
+                                   ctypes.c_int64(128), ctypes.c_int64(4), ctypes.c_int64(64), ctypes.c_int64(1),
+                                   ctypes.c_int64(128), dtype, ctypes.c_uint(flags), None, ctypes.c_int64(0), None)
+
+    assert call(0x2) == codes["MSS_ERR_FLAGS"]          # unknown bit, refused before anything else
+    assert call(0x1, dtype=0) == codes["MSS_ERR_DTYPE"]  # bf16 io only, on either kernel
 
 
 def test_host_call_argument_errors(lib):
