@@ -81,17 +81,22 @@ struct BwdTok {
     float dsp;  // dDelta / ddelta_raw: sigmoid(s) with softplus, else 1
 };
 
-// kDsp: also the softplus derivative (the recompute-only passes skip it).
-template <bool kFast, bool kGeo, bool kSoftplus, bool kDsp = true, int N>
+// dDelta / ddelta_raw: the slope of the softplus, sigmoid(s), else 1.
+template <bool kFast, bool kSoftplus>
+__device__ __forceinline__ float softplus_slope(float s) {
+    if constexpr (!kSoftplus) return 1.f;
+    return kFast ? rcp_approx(1.f + ex2_approx(-s * kLog2e)) : 1.f / (1.f + expf(-s));
+}
+
+// Delta, Delta * u and r of one token (dsp is left at 1: the slope is formed
+// only for the tokens whose gradient a lane stores).
+template <bool kFast, bool kGeo, bool kSoftplus, int N>
 __device__ __forceinline__ BwdTok bwd_token(float ut, float dr, const LaneConst<N>& cc) {
     BwdTok tk;
     const float s = dr + cc.bias;
     tk.dt = s;
     tk.dsp = 1.f;
-    if constexpr (kSoftplus) {
-        tk.dt = kFast ? softplus_fast(s) : softplus_precise(s);
-        if constexpr (kDsp) tk.dsp = kFast ? rcp_approx(1.f + ex2_approx(-s * kLog2e)) : 1.f / (1.f + expf(-s));
-    }
+    if constexpr (kSoftplus) tk.dt = kFast ? softplus_fast(s) : softplus_precise(s);
     tk.du = tk.dt * ut;
     tk.rdt = kGeo ? ex2_approx(tk.dt * cc.a0) : tk.dt;
     return tk;
@@ -121,17 +126,6 @@ __device__ __forceinline__ void unpack16(const uint4& w, float (&v)[16 / sizeof(
         v[i] = a[i];
         v[H + i] = b[i];
     }
-}
-
-// Token t of a 16-byte group, t known only at run time (selects, no local memory).
-template <typename T>
-__device__ __forceinline__ float elem16rt(const uint4& w, int t) {
-    float v[16 / sizeof(T)];
-    unpack16<T>(w, v);
-    float r = v[0];
-#pragma unroll
-    for (int i = 1; i < int(16 / sizeof(T)); ++i) r = t == i ? v[i] : r;
-    return r;
 }
 
 // Sum of the M = 4 * (N/4) values v over the 16 channels of the warp (lane
@@ -279,7 +273,7 @@ __device__ __forceinline__ void scan_bwd_body(const BwdMaps& maps, const BwdPara
             const float4* base = my_bcf + (g * V) * kRowF4;
 #pragma unroll
             for (int t = 0; t < V; ++t) {
-                const BwdTok tk = bwd_token<kFast, kGeo, kSoftplus, false>(uv[t], dv[t], cc);
+                const BwdTok tk = bwd_token<kFast, kGeo, kSoftplus>(uv[t], dv[t], cc);
                 float4 rowv[P];
 #pragma unroll
                 for (int i = 0; i < P; ++i) rowv[i] = base[t * kRowF4 + i];
@@ -305,37 +299,36 @@ __device__ __forceinline__ void scan_bwd_body(const BwdMaps& maps, const BwdPara
                     issue(k + S);
                 }
             }
-            // scalars of the HV tokens from `first` on: each lane of the pair
-            // computes half of them and they swap
-            auto half_tokens = [&](int first, BwdTok (&th)[HV]) {
+            // the group's per-token scalars: Delta and r for all V tokens (each
+            // lane of the pair forms them all, which costs less than swapping
+            // them), the softplus slope for the HV tokens this lane stores
+            // (tokens half * HV ..)
+            float dtv[V], rv[V], dspv[HV];
+            {
+                float uv[V], dv[V];
+                unpack16<T>(uw, uv);
+                unpack16<T>(dw, dv);
 #pragma unroll
-                for (int k2 = 0; k2 < HV / 2; ++k2) {
-                    const int tm = first + (half ? HV / 2 : 0) + k2;
-                    const BwdTok mine = bwd_token<kFast, kGeo, kSoftplus>(elem16rt<T>(uw, tm), elem16rt<T>(dw, tm), cc);
-                    BwdTok other;
-                    other.dt = __shfl_xor_sync(0xffffffffu, mine.dt, 1);
-                    other.du = 0.f;  // formed again from dt where it is used
-                    other.rdt = __shfl_xor_sync(0xffffffffu, mine.rdt, 1);
-                    other.dsp = __shfl_xor_sync(0xffffffffu, mine.dsp, 1);
-                    th[k2] = half ? other : mine;
-                    th[HV / 2 + k2] = half ? mine : other;
+                for (int t = 0; t < V; ++t) {
+                    const BwdTok tk = bwd_token<kFast, kGeo, kSoftplus>(uv[t], dv[t], cc);
+                    dtv[t] = tk.dt;
+                    rv[t] = tk.rdt;
                 }
-            };
+#pragma unroll
+                for (int k2 = 0; k2 < HV; ++k2)
+                    dspv[k2] = softplus_slope<kFast, kSoftplus>((half ? dv[HV + k2] : dv[k2]) + cc.bias);
+            }
             const float4* base = my_bcf + (g * V) * kRowF4;
             float2 h0[P], hmid[P];
 #pragma unroll
             for (int i = 0; i < P; ++i) h0[i] = hmid[i] = gs[(g * 32 + lane) * P + i];
-            {
-                BwdTok th[HV];
-                half_tokens(0, th);
 #pragma unroll
-                for (int t = 0; t < HV; ++t) {
-                    float4 rowv[P];
+            for (int t = 0; t < HV; ++t) {
+                float4 rowv[P];
 #pragma unroll
-                    for (int i = 0; i < P; ++i) rowv[i] = base[t * kRowF4 + i];
-                    const float ut = elem16<T>(uw, t);
-                    token_states<N, kFast, kGeo, kZoh, false>(hmid, rowv, th[t].dt * ut, th[t].rdt, ut, half, cc);
-                }
+                for (int i = 0; i < P; ++i) rowv[i] = base[t * kRowF4 + i];
+                const float ut = elem16<T>(uw, t);
+                token_states<N, kFast, kGeo, kZoh, false>(hmid, rowv, dtv[t] * ut, rv[t], ut, half, cc);
             }
             const int64_t tg = t_chunk + int64_t(g) * V;
             // the second half, then the first: one copy of the code
@@ -343,10 +336,12 @@ __device__ __forceinline__ void scan_bwd_body(const BwdMaps& maps, const BwdPara
             for (int hf = 1; hf >= 0; --hf) {
                 const int T0 = hf * HV;
                 BwdTok th[HV];
-                half_tokens(T0, th);
                 float uh[HV], zh[HV], yh[HV];
 #pragma unroll
                 for (int k2 = 0; k2 < HV; ++k2) {
+                    th[k2].dt = hf ? dtv[HV + k2] : dtv[k2];
+                    th[k2].rdt = hf ? rv[HV + k2] : rv[k2];
+                    th[k2].dsp = dspv[k2];  // the right token's on the lane that stores this half
                     uh[k2] = hf ? elem16<T>(uw, HV + k2) : elem16<T>(uw, k2);
                     yh[k2] = hf ? elem16<T>(yw, HV + k2) : elem16<T>(yw, k2);
                     if constexpr (kGate) zh[k2] = hf ? elem16<T>(zw, HV + k2) : elem16<T>(zw, k2);
@@ -383,10 +378,10 @@ __device__ __forceinline__ void scan_bwd_body(const BwdMaps& maps, const BwdPara
                     // read-out and gate
                     float dr = yh[tt];
                     if constexpr (kGate) {
-                        float racc = 0.f;
+                        float2 racc2 = make_float2(0.f, 0.f);
 #pragma unroll
-                        for (int i = 0; i < P; ++i)
-                            racc = fmaf(rowv[i].z, hs[tt][i].x, fmaf(rowv[i].w, hs[tt][i].y, racc));
+                        for (int i = 0; i < P; ++i) racc2 = __ffma2_rn(make_float2(rowv[i].z, rowv[i].w), hs[tt][i], racc2);
+                        const float racc = racc2.x + racc2.y;
                         const float r = racc + __shfl_xor_sync(0xffffffffu, racc, 1) + cc.D * ut;
                         const float zt = zh[tt];
                         const float sz = kFast ? rcp_approx(1.f + ex2_approx(-zt * kLog2e)) : 1.f / (1.f + expf(-zt));
@@ -396,45 +391,74 @@ __device__ __forceinline__ void scan_bwd_body(const BwdMaps& maps, const BwdPara
                     float2 dA[P];
                     transition<N, kFast, kGeo>(dA, tk.rdt, half, cc);
                     float vals[M];
-                    float du_acc = 0.f, ddt = 0.f;
+                    float du_t, ds_t;
+                    if constexpr (!kZoh) {
+                        // Euler: w_n = Delta for every state, so
+                        //   du    = Delta * S1 + dr D,       S1 = sum_n g_n B_n,
+                        //   dDelta = u * S1 + S2,            S2 = sum_n q_n A_n,
+                        //   dA_n += Delta q_n,  dB_n = Delta u g_n,  dC_n = dr h_n,
+                        // with g_n = gh_n + dr C_n and q_n = g_n Abar_n h_{t-1,n} = gh'_n h_{t-1,n}
+                        const float2 dr2 = make_float2(dr, dr), dt2 = make_float2(tk.dt, tk.dt);
+                        const float2 du2 = make_float2(tk.dt * ut, tk.dt * ut);
+                        float2 s1 = make_float2(0.f, 0.f), s2 = make_float2(0.f, 0.f);
 #pragma unroll
-                    for (int i = 0; i < P; ++i) {
-                        const float2 hp = tt > 0 ? hs[tt > 0 ? tt - 1 : 0][i] : hst[i];
-                        const float Bx = rowv[i].x, By = rowv[i].y;
-                        const float gx = fmaf(dr, rowv[i].z, gh[i].x), gy = fmaf(dr, rowv[i].w, gh[i].y);
-                        vals[P * 2 + 2 * i] = dr * hs[tt][i].x;  // dC
-                        vals[P * 2 + 2 * i + 1] = dr * hs[tt][i].y;
-                        float wx = tk.dt, wy = tk.dt, dwx = 1.f, dwy = 1.f, dAwx = 0.f, dAwy = 0.f;
-                        if constexpr (kZoh) {
+                        for (int i = 0; i < P; ++i) {
+                            const float2 hp = tt > 0 ? hs[tt > 0 ? tt - 1 : 0][i] : hst[i];
+                            const float2 g = __ffma2_rn(dr2, make_float2(rowv[i].z, rowv[i].w), gh[i]);
+                            const float2 dc = __fmul2_rn(dr2, hs[tt][i]);
+                            const float2 db = __fmul2_rn(du2, g);
+                            s1 = __ffma2_rn(g, make_float2(rowv[i].x, rowv[i].y), s1);
+                            gh[i] = __fmul2_rn(g, dA[i]);
+                            const float2 q = __fmul2_rn(gh[i], hp);
+                            s2 = __ffma2_rn(q, cc.a2[i], s2);  // A in log2 units for bf16 io
+                            dA_acc[i] = __ffma2_rn(q, dt2, dA_acc[i]);
+                            vals[2 * i] = db.x;
+                            vals[2 * i + 1] = db.y;
+                            vals[P * 2 + 2 * i] = dc.x;
+                            vals[P * 2 + 2 * i + 1] = dc.y;
+                        }
+                        float S1 = s1.x + s1.y, S2 = s2.x + s2.y;
+                        S1 += __shfl_xor_sync(0xffffffffu, S1, 1);
+                        S2 += __shfl_xor_sync(0xffffffffu, S2, 1);
+                        if constexpr (kFast) S2 *= kLn2;
+                        du_t = fmaf(tk.dt, S1, dr * cc.D);
+                        ds_t = fmaf(ut, S1, S2) * tk.dsp;
+                    } else {
+                        float du_acc = 0.f, ddt = 0.f;
+#pragma unroll
+                        for (int i = 0; i < P; ++i) {
+                            const float2 hp = tt > 0 ? hs[tt > 0 ? tt - 1 : 0][i] : hst[i];
+                            const float Bx = rowv[i].x, By = rowv[i].y;
+                            const float gx = fmaf(dr, rowv[i].z, gh[i].x), gy = fmaf(dr, rowv[i].w, gh[i].y);
+                            vals[P * 2 + 2 * i] = dr * hs[tt][i].x;  // dC
+                            vals[P * 2 + 2 * i + 1] = dr * hs[tt][i].y;
                             // w = Delta phi(x), dw/dDelta = a, dw/dA = Delta^2 phi'(x)
                             const float2 an = a_nat(i);
                             const float xx = tk.dt * an.x, xy = tk.dt * an.y;
                             const bool sx = fabsf(xx) < kZohTaylorMax, sy = fabsf(xy) < kZohTaylorMax;
-                            wx = sx ? tk.dt * phi_taylor(xx) : (dA[i].x - 1.f) * cc.ia[i].x;
-                            wy = sy ? tk.dt * phi_taylor(xy) : (dA[i].y - 1.f) * cc.ia[i].y;
-                            dwx = dA[i].x;
-                            dwy = dA[i].y;
-                            dAwx = sx ? tk.dt * tk.dt * dphi_taylor(xx) : fmaf(tk.dt, dA[i].x, -wx) * cc.ia[i].x;
-                            dAwy = sy ? tk.dt * tk.dt * dphi_taylor(xy) : fmaf(tk.dt, dA[i].y, -wy) * cc.ia[i].y;
+                            const float wx = sx ? tk.dt * phi_taylor(xx) : (dA[i].x - 1.f) * cc.ia[i].x;
+                            const float wy = sy ? tk.dt * phi_taylor(xy) : (dA[i].y - 1.f) * cc.ia[i].y;
+                            const float dwx = dA[i].x, dwy = dA[i].y;
+                            const float dAwx = sx ? tk.dt * tk.dt * dphi_taylor(xx) : fmaf(tk.dt, dA[i].x, -wx) * cc.ia[i].x;
+                            const float dAwy = sy ? tk.dt * tk.dt * dphi_taylor(xy) : fmaf(tk.dt, dA[i].y, -wy) * cc.ia[i].y;
+                            vals[2 * i] = gx * wx * ut;  // dB
+                            vals[2 * i + 1] = gy * wy * ut;
+                            du_acc = fmaf(gx * wx, Bx, fmaf(gy * wy, By, du_acc));
+                            const float dwsx = gx * Bx * ut, dwsy = gy * By * ut;
+                            const float dax = gx * hp.x * dA[i].x, day = gy * hp.y * dA[i].y;
+                            ddt = fmaf(dax, an.x, fmaf(day, an.y, ddt));
+                            ddt = fmaf(dwsx, dwx, fmaf(dwsy, dwy, ddt));
+                            dA_acc[i].x = fmaf(dax, tk.dt, fmaf(dwsx, dAwx, dA_acc[i].x));
+                            dA_acc[i].y = fmaf(day, tk.dt, fmaf(dwsy, dAwy, dA_acc[i].y));
+                            gh[i] = make_float2(gx * dA[i].x, gy * dA[i].y);
                         }
-                        vals[2 * i] = gx * wx * ut;  // dB
-                        vals[2 * i + 1] = gy * wy * ut;
-                        du_acc = fmaf(gx * wx, Bx, fmaf(gy * wy, By, du_acc));
-                        const float dwsx = gx * Bx * ut, dwsy = gy * By * ut;
-                        const float dax = gx * hp.x * dA[i].x, day = gy * hp.y * dA[i].y;
-                        const float2 ani = a_nat(i);
-                        ddt = fmaf(dax, ani.x, fmaf(day, ani.y, ddt));
-                        ddt = fmaf(dwsx, dwx, fmaf(dwsy, dwy, ddt));
-                        dA_acc[i].x = fmaf(dax, tk.dt, fmaf(dwsx, dAwx, dA_acc[i].x));
-                        dA_acc[i].y = fmaf(day, tk.dt, fmaf(dwsy, dAwy, dA_acc[i].y));
-                        gh[i] = make_float2(gx * dA[i].x, gy * dA[i].y);
+                        du_t = du_acc + __shfl_xor_sync(0xffffffffu, du_acc, 1) + dr * cc.D;
+                        ds_t = (ddt + __shfl_xor_sync(0xffffffffu, ddt, 1)) * tk.dsp;
                     }
-                    const float du_t = du_acc + __shfl_xor_sync(0xffffffffu, du_acc, 1) + dr * cc.D;
-                    const float ds_t = (ddt + __shfl_xor_sync(0xffffffffu, ddt, 1)) * tk.dsp;
                     du_o[tt] = du_t;
                     ds_o[tt] = ds_t;
                     dD_acc = fmaf(dr, ut, dD_acc);
-                    dbias_acc += ds_t;
+                    if (half == hf) dbias_acc += ds_t;
                     red[tt] = reduce_scatter_channels<M>(vals, lane, red_index, red_writer);
                 }
                 // this half's per-token gradients: stored by lane half hf
@@ -461,6 +485,8 @@ __device__ __forceinline__ void scan_bwd_body(const BwdMaps& maps, const BwdPara
         __syncwarp();
     }
 
+    // each lane summed the slopes of the tokens it stored
+    dbias_acc += __shfl_xor_sync(0xffffffffu, dbias_acc, 1);
     if (!valid) return;
     if (p.dinit) {
         float* di = p.dinit + row * N + half;
