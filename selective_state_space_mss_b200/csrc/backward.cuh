@@ -1,7 +1,7 @@
 // backward.cuh -- host-side launch of the backward pass (included by the
 // bwd_*.cu translation units): zeroing of the summed gradients, the
 // checkpoint pass (the forward kernel's fold launch recording the state at
-// every chunk start), then the backward kernel; or the scalar reference
+// every group start), then the backward kernel; or the scalar reference
 // kernel for the shapes the throughput kernels do not take.
 #pragma once
 
@@ -12,16 +12,34 @@
 namespace mss_host {
 
 // Workspace bytes of the backward pass: the checkpoints of the throughput
-// kernels (one state per chunk of 128 bytes of a row) when the sizes can take
-// them (the same test as the launch, for 16-byte-aligned tensors), else those
-// of the scalar kernel (one per 16 tokens).
+// kernels (one state per group of 16 bytes of a row: 8 bf16 or 4 fp32 tokens)
+// when the sizes can take them (the same test as the launch, for
+// 16-byte-aligned tensors), else those of the scalar kernel (one per 16
+// tokens).
 template <typename T, int N>
 int64_t backward_workspace_bytes(int64_t batch, int64_t dim, int64_t seqlen, unsigned flags) {
     const int64_t rows = batch * dim;
     if (rows == 0 || seqlen == 0) return 0;
     const bool fast = seq_shape_ok(batch, dim, seqlen, N, int(sizeof(T)), flags);
-    const int64_t chunk = fast ? mss::SeqLayout<T, (N >= 4 ? N : 4)>::kChunk : mss::kBwdSimpleChunk;
-    return rows * ((seqlen + chunk - 1) / chunk) * N * 4;
+    const int64_t every = fast ? mss::SeqLayout<T, (N >= 4 ? N : 4)>::kVec : mss::kBwdSimpleChunk;
+    return rows * ((seqlen + every - 1) / every) * N * 4;
+}
+
+// [rows, seqlen / V * N] fp32 view of the group-start states, box = 16 rows x
+// the chunk's groups.
+template <typename T, int N>
+bool encode_ckpt(CUtensorMap* m, const void* base, int64_t rows, int64_t seqlen) {
+    using Ly = mss::BwdLayout<T, N>;
+    auto enc = encode_tiled_fn();
+    if (!enc) return false;
+    const int64_t width = seqlen / Ly::kVec * N;
+    const cuuint64_t dims[2] = {cuuint64_t(width), cuuint64_t(rows)};
+    const cuuint64_t strides[1] = {cuuint64_t(width * 4)};
+    const cuuint32_t box[2] = {cuuint32_t(Ly::kGroups * N), cuuint32_t(Ly::kRows)};
+    const cuuint32_t estr[2] = {1u, 1u};
+    return enc(m, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 2, const_cast<void*>(base), dims, strides, box, estr,
+               CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
 template <typename T, int N, bool kGate, bool kSoftplus, bool kZoh>
@@ -62,7 +80,8 @@ int launch_bwd_fast(mss::ScanParams fp, const mss::BwdParams& bp, unsigned flags
     if (!encode_rows(&bm.u, bp.u, rows, bp.seqlen, esz, br) || !encode_rows(&bm.delta, bp.delta, rows, bp.seqlen, esz, br) ||
         (bp.z && !encode_rows(&bm.z, bp.z, rows, bp.seqlen, esz, br)) ||
         !encode_rows(&bm.dy, bp.dy, rows, bp.seqlen, esz, br) ||
-        !encode_bc(&bm.B, bp.B, bp.batch, N, bp.seqlen, esz) || !encode_bc(&bm.C, bp.C, bp.batch, N, bp.seqlen, esz))
+        !encode_bc(&bm.B, bp.B, bp.batch, N, bp.seqlen, esz) || !encode_bc(&bm.C, bp.C, bp.batch, N, bp.seqlen, esz) ||
+        !encode_ckpt<T, N>(&bm.ck, bp.ckpt, rows, bp.seqlen))
         return MSS_ERR_CUDA;
     if (bp.z)
         return bp.softplus ? launch_bwd_variant<T, N, true, true, kZoh>(bm, bp, flags, s)

@@ -35,7 +35,8 @@ struct ScanParams {
     void* conv_state_out;        // [batch, dim, K-1] io type: the last K-1 inputs, may be null
     int conv_width;              // K in 1..4, or 0 without the convolution
     // Checkpoint pass of the backward pass (fold launches only): the state at
-    // the start of every chunk, [batch * dim, n_chunks, N].
+    // the start of every group of V tokens, [batch * dim, seqlen / V, N], each
+    // group's N floats in lane order (lane half h: pairs (h_n, h_n+2), n = h + 4i).
     float* ckpt;
     // Self-test of the bounded waits (MSS_FLAG_SELFTEST_TIMEOUT): nonzero makes
     // every CTA of the tiled kernel wait this many nanoseconds on a barrier no
@@ -60,7 +61,7 @@ struct BwdParams {
     const float* delta_bias;  // may be null
     const void* dy;
     const float* dlast;       // may be null
-    const float* ckpt;        // [batch * dim, n_chunks, N] states at chunk starts
+    const float* ckpt;        // [batch * dim, seqlen / V, N] states at the start of each group of V tokens
     void* du;
     void* ddelta;
     void* dz;                 // null when z is null

@@ -13,12 +13,14 @@
 // dDelta softplus'(s) and the skip term's du += dr D, dD += dr u.
 //
 // States.  A checkpoint pass (the forward kernel's fold launch with p.ckpt)
-// records the state at the start of every chunk.  This kernel walks the
-// chunks from last to first; for each it recomputes the states forward from
-// the chunk's checkpoint, keeping the state at the start of each group of V
-// tokens in shared memory, then walks the groups from last to first: it
-// recomputes the group's V states into registers and runs the V reverse
-// steps.  Every state is recomputed twice; none is stored in HBM.
+// records the state at the start of every group of V tokens (8 bytes per
+// channel and token at N = 16, against the 14 bytes of inputs and gradients
+// the pass moves anyway).  This kernel walks the chunks from last to first,
+// the group-start states arriving by TMA with the chunk's other tiles, and
+// the groups of a chunk from last to first: it recomputes the state in the
+// middle of the group, then each half's HV states into registers, and runs
+// the HV reverse steps of the half.  A state is recomputed 1.5 times on
+// average; none is stored in HBM besides the checkpoints.
 //
 // Work split and reductions.  As in the forward kernel, a CTA is one warp
 // serving 16 channels of a batch row, a lane pair per channel, each lane
@@ -44,7 +46,7 @@
 namespace mss {
 
 struct BwdMaps {
-    CUtensorMap u, delta, z, dy, B, C;
+    CUtensorMap u, delta, z, dy, B, C, ck;
 };
 
 template <typename T, int N>
@@ -58,17 +60,18 @@ struct BwdLayout {
     static constexpr int kPairs = F::kPairs;
     static constexpr int kTile = F::kTile;
     static constexpr int kBCTile = F::kBCTile;
+    // the group-start states of the chunk: [16 rows][kGroups][N] floats
+    static constexpr int kCkTile = kRows * kGroups * N * 4;
     // one stage: the next chunk's tiles are fetched while the chunk's first
     // group is reversed, once every tile word has been read (B and C are read
     // when the chunk starts); a second stage would cost a CTA per SM
     static constexpr int kStages = 1;
-    static constexpr int kStageBytes = 4 * kTile + 2 * kBCTile;  // u, delta, z, dy, B, C
+    static constexpr int kCkOffset = 4 * kTile + 2 * kBCTile;
+    static constexpr int kStageBytes = kCkOffset + kCkTile;  // u, delta, z, dy, B, C, states
     static constexpr int kBCfRow = F::kBCfRow;
     static constexpr int kBCfBytes = F::kBCfBytes;
     static constexpr int kBCfOffset = kStages * kStageBytes;
-    static constexpr int kGsOffset = kBCfOffset + kBCfBytes;      // group-start states
-    static constexpr int kGsBytes = kGroups * 32 * (N / 2) * 4;
-    static constexpr int kBarOffset = kGsOffset + kGsBytes;
+    static constexpr int kBarOffset = kBCfOffset + kBCfBytes;
     static constexpr int kSmemBytes = kBarOffset + kStages * 8 + 1024;
     static_assert(kStageBytes % 1024 == 0, "stage tiles must stay 1024-byte aligned");
 };
@@ -197,8 +200,7 @@ __device__ __forceinline__ void scan_bwd_body(const BwdMaps& maps, const BwdPara
     const int n_chunks = int((L + Ly::kChunk - 1) / Ly::kChunk);
     const int64_t d = row - int64_t(b) * p.dim;
     float* bcf = reinterpret_cast<float*>(smem + Ly::kBCfOffset);
-    float2* gs = reinterpret_cast<float2*>(smem + Ly::kGsOffset);
-    const uint32_t stage_tx = uint32_t((kGate ? 4 : 3) * Ly::kTile + 2 * Ly::kBCTile);
+    const uint32_t stage_tx = uint32_t((kGate ? 4 : 3) * Ly::kTile + 2 * Ly::kBCTile + Ly::kCkTile);
 
     // the k-th chunk processed is chunk n_chunks - 1 - k
     auto issue = [&](int k) {
@@ -212,6 +214,7 @@ __device__ __forceinline__ void scan_bwd_body(const BwdMaps& maps, const BwdPara
         tma_load_2d(st + 3 * Ly::kTile, &maps.dy, x, row0, bar);
         tma_load_3d(st + 4 * Ly::kTile, &maps.B, x, 0, b, bar);
         tma_load_3d(st + 4 * Ly::kTile + Ly::kBCTile, &maps.C, x, 0, b, bar);
+        tma_load_2d(st + Ly::kCkOffset, &maps.ck, (n_chunks - 1 - k) * GPC * N, row0, bar);
     };
     auto wait_chunk = [&](int k) -> bool {
         const bool landed = mbar_wait_bounded(bars + k % S, uint32_t((k / S) & 1), p.err);
@@ -256,32 +259,6 @@ __device__ __forceinline__ void scan_bwd_body(const BwdMaps& maps, const BwdPara
         const int64_t t_chunk = int64_t(c) * Ly::kChunk;
         const int ng = int(min(int64_t(GPC), (L - t_chunk) / V));
 
-        // forward from the chunk's checkpoint, keeping each group's start state
-        float2 h[P];
-        {
-            const float* ck = p.ckpt + (size_t(row) * size_t(n_chunks) + size_t(c)) * N + half;
-#pragma unroll
-            for (int i = 0; i < P; ++i) h[i] = make_float2(ck[4 * i], ck[4 * i + 2]);
-        }
-#pragma unroll 1
-        for (int g = 0; g < ng; ++g) {
-#pragma unroll
-            for (int i = 0; i < P; ++i) gs[(g * 32 + lane) * P + i] = h[i];
-            float uv[V], dv[V];
-            unpack16<T>(group_word(st, 0, g), uv);
-            unpack16<T>(group_word(st, 1, g), dv);
-            const float4* base = my_bcf + (g * V) * kRowF4;
-#pragma unroll
-            for (int t = 0; t < V; ++t) {
-                const BwdTok tk = bwd_token<kFast, kGeo, kSoftplus>(uv[t], dv[t], cc);
-                float4 rowv[P];
-#pragma unroll
-                for (int i = 0; i < P; ++i) rowv[i] = base[t * kRowF4 + i];
-                token_states<N, kFast, kGeo, kZoh, false>(h, rowv, tk.du, tk.rdt, uv[t], half, cc);
-            }
-        }
-        __syncwarp();
-
         // groups from last to first; each group in two halves of HV tokens
         // (second half first), so that only HV recomputed states are live
 #pragma unroll 1
@@ -291,6 +268,13 @@ __device__ __forceinline__ void scan_bwd_body(const BwdMaps& maps, const BwdPara
             const uint4 dw = group_word(st, 1, g);
             if constexpr (kGate) zw = group_word(st, 2, g);
             yw = valid ? group_word(st, 3, g) : make_uint4(0u, 0u, 0u, 0u);  // past the last channel: no gradient
+            // the group's start state, from the checkpoint pass
+            float2 h0[P], hmid[P];
+            {
+                const float2* ck = reinterpret_cast<const float2*>(st + Ly::kCkOffset) + (ch * GPC + g) * (N / 2) + half * P;
+#pragma unroll
+                for (int i = 0; i < P; ++i) h0[i] = hmid[i] = ck[i];
+            }
             if (g == 0) {
                 // every tile word of the chunk has been read: fetch the next chunk
                 __syncwarp();
@@ -319,9 +303,6 @@ __device__ __forceinline__ void scan_bwd_body(const BwdMaps& maps, const BwdPara
                     dspv[k2] = softplus_slope<kFast, kSoftplus>((half ? dv[HV + k2] : dv[k2]) + cc.bias);
             }
             const float4* base = my_bcf + (g * V) * kRowF4;
-            float2 h0[P], hmid[P];
-#pragma unroll
-            for (int i = 0; i < P; ++i) h0[i] = hmid[i] = gs[(g * 32 + lane) * P + i];
 #pragma unroll
             for (int t = 0; t < HV; ++t) {
                 float4 rowv[P];
@@ -535,6 +516,7 @@ __global__ void __launch_bounds__(32) scan_bwd_kernel(const __grid_constant__ Bw
         prefetch_tensormap(&maps.dy);
         prefetch_tensormap(&maps.B);
         prefetch_tensormap(&maps.C);
+        prefetch_tensormap(&maps.ck);
     }
     __syncwarp();
 

@@ -317,7 +317,7 @@ __device__ __forceinline__ uint2 pack8(const float (&v)[8 / sizeof(T)]) {
 // the final state); otherwise the full pass, starting from the caller's state
 // carried over the earlier segments' aggregates.  A fold with p.ckpt set is
 // the backward pass's checkpoint pass instead: one segment from the caller's
-// state, recording the state at the start of every chunk.
+// state, recording the state at the start of every group of V tokens.
 template <typename T, int N, bool kGeo, bool kGate, bool kSoftplus, bool kFold, bool kZoh, bool kConv>
 __device__ __forceinline__ void scan_seq_body(const SeqMaps& maps, const ScanParams& p, uint8_t* smem,
                                               uint64_t* bars, const LaneConst<N>& cc, bool valid, int64_t row) {
@@ -460,18 +460,23 @@ __device__ __forceinline__ void scan_seq_body(const SeqMaps& maps, const ScanPar
         else
             return h[i];
     };
-    // checkpoint pass: the state at the start of every chunk, in h_n form
-    auto store_ckpt = [&](int chunk) {
+    // checkpoint pass: the state at the start of every group of V tokens, in
+    // h_n form, as [row][group][N] floats in lane order (lane half h's N/2
+    // floats at h * N/2: its pairs (h_n, h_n+2), n = h + 4i)
+    auto store_ckpt = [&](int group) {
         if (!valid) return;
-        float* ck = p.ckpt + (size_t(row) * size_t(n_chunks) + size_t(chunk)) * N + half;
+        float2* ck = reinterpret_cast<float2*>(p.ckpt + (size_t(row) * size_t(n_groups) + size_t(group)) * N) +
+                     half * P;
 #pragma unroll
-        for (int i = 0; i < P; ++i) {
-            const float2 hs = state_out(i);
-            ck[4 * i] = hs.x;
-            ck[4 * i + 2] = hs.y;
+        for (int i = 0; i < P; i += 2) {
+            if (i + 1 < P) {
+                const float2 a = state_out(i), b2 = state_out(i + 1);
+                *reinterpret_cast<float4*>(ck + i) = make_float4(a.x, a.y, b2.x, b2.y);
+            } else {
+                ck[i] = state_out(i);
+            }
         }
     };
-    if (kFold && p.ckpt) store_ckpt(0);
     float dsum = 0.f, dcomp = 0.f;  // fold: compensated sum of this lane's steps
     T* yrow = static_cast<T*>(p.y) + row * L + t_begin + HV * half;
     const float4* my_bcf = reinterpret_cast<const float4*>(bcf) + half * P;  // this lane's chunks of a row
@@ -509,6 +514,7 @@ __device__ __forceinline__ void scan_seq_body(const SeqMaps& maps, const ScanPar
     for (int g = 0; g < n_groups; ++g) {
         const int c = g / GPC, j = g % GPC;
         const bool has_next = g + 1 < n_groups;
+        if (kFold && p.ckpt) store_ckpt(g);
         // the next group's u/delta/z, first: its stage must have landed when it opens a new chunk
         if (has_next && j == GPC - 1 && !wait_chunk(c + 1)) return;
         float uv[HV], dv[HV], zv[HV];
@@ -583,7 +589,6 @@ __device__ __forceinline__ void scan_seq_body(const SeqMaps& maps, const ScanPar
         if (j == GPC - 1 || !has_next) {
             // chunk c is consumed: convert the next chunk's B/C (its stage was
             // waited for above), then hand chunk c's stage to chunk c + S
-            if (kFold && p.ckpt && has_next) store_ckpt(c + 1);
             __syncwarp();
             if (has_next) {
                 const uint8_t* st = smem + ((c + 1) % S) * Ly::kStageBytes;

@@ -260,14 +260,15 @@ def test_bwd_argument_errors(lib):
     assert bwd(ws=P + 0x8000000) == codes["MSS_ERR_ALIAS"]   # workspace on dA
     assert bwd(batch=0) == 0
     q = lambda *a: lib.mss_scan_bwd_workspace_size(*a)
-    assert q(1, 16, 16, 4096, 1, 0) == 16 * 64 * 16 * 4            # one state per 64-token chunk
+    assert q(1, 16, 16, 4096, 1, 0) == 16 * 512 * 16 * 4           # one state per 8-token group
     assert q(1, 16, 16, 4096, 1, 0x2) == 16 * 256 * 16 * 4         # scalar path: one per 16 tokens
     assert q(1, 16, 16, 4097, 1, 0) == 16 * 257 * 16 * 4           # odd rows take the scalar path
     assert q(1, 16, 16, 0, 1, 0) == 0
     assert q(1, 16, 3, 64, 1, 0) == codes["MSS_ERR_UNSUPPORTED_N"]
     # more batch rows than the tiled kernels' grid takes: the scalar path's size
     assert q(70000, 16, 16, 64, 1, 0) == 70000 * 16 * 4 * 16 * 4
-    assert q(65535, 16, 16, 64, 1, 0) == 65535 * 16 * 1 * 16 * 4
+    assert q(65535, 16, 16, 64, 1, 0) == 65535 * 16 * 8 * 16 * 4
+    assert q(1, 16, 16, 4096, 0, 0) == 16 * 1024 * 16 * 4          # fp32: one per 4-token group
 
 
 def test_ssd_argument_errors(lib):
