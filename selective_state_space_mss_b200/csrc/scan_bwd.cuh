@@ -318,14 +318,15 @@ __device__ __forceinline__ void scan_bwd_body(const BwdMaps& maps, const BwdPara
                 const int T0 = hf * HV;
                 BwdTok th[HV];
                 float uh[HV], zh[HV], yh[HV];
+                // the half's 8 bytes of each group word
+                unpack8<T>(hf ? make_uint2(uw.z, uw.w) : make_uint2(uw.x, uw.y), uh);
+                unpack8<T>(hf ? make_uint2(yw.z, yw.w) : make_uint2(yw.x, yw.y), yh);
+                if constexpr (kGate) unpack8<T>(hf ? make_uint2(zw.z, zw.w) : make_uint2(zw.x, zw.y), zh);
 #pragma unroll
                 for (int k2 = 0; k2 < HV; ++k2) {
                     th[k2].dt = hf ? dtv[HV + k2] : dtv[k2];
                     th[k2].rdt = hf ? rv[HV + k2] : rv[k2];
                     th[k2].dsp = dspv[k2];  // the right token's on the lane that stores this half
-                    uh[k2] = hf ? elem16<T>(uw, HV + k2) : elem16<T>(uw, k2);
-                    yh[k2] = hf ? elem16<T>(yw, HV + k2) : elem16<T>(yw, k2);
-                    if constexpr (kGate) zh[k2] = hf ? elem16<T>(zw, HV + k2) : elem16<T>(zw, k2);
                 }
                 const float4* hbase = base + T0 * kRowF4;
                 float2 hst[P];

@@ -27,12 +27,13 @@
 // Operands: C and B tiles [128 tokens][64 state] x 2 and X [128 tokens][64]
 // in the 128-byte swizzle TMA writes, double buffered (the next chunk's
 // loads run during this one); M, X_w and the state copy are written by the
-// threads in the same layout.  One thread issues the MMAs and the TMA copies.
+// threads in the same layout.  One thread issues the MMAs and the TMA copies,
+// from a warp whose scores are all masked (it has the least work).
 //
 // Order within a chunk, with three CTA barriers: C B^T starts as soon as the
 // chunk's tiles land; the threads scale X (barrier); B^T X_w and C S_prev
 // start, and the threads mask and decay the scores as soon as C B^T is done
-// (barrier); M X starts while warp 0 prepares the next chunk's step sizes and
+// (barrier); M X starts while another such warp prepares the next chunk's step sizes and
 // decay sums (their raw steps and this chunk's z were loaded a chunk ahead);
 // the state update waits only for B^T X_w, the output only for M X
 // (barrier); then the y store and the loads of chunk c + 2.  Each thread
@@ -103,6 +104,12 @@ __global__ void __launch_bounds__(512, 1) ssd_tc_kernel(const __grid_constant__ 
 
     const int tid = threadIdx.x, warp = tid >> 5;
     const int row = tid & 127, qd = tid >> 7;  // TMEM lane / row, column quarter
+    // The thread that issues the MMAs and the TMA copies, and the warp that
+    // prepares the step sizes, sit in warps whose score blocks are all masked
+    // (rows 0..31 against columns 96..127, rows 32..63 against 96..127), so
+    // that their extra work does not hold up the CTA barriers.
+    constexpr int kCtlWarp = 12, kScanWarp = 13;
+    const bool ctl = tid == kCtlWarp * 32;
     const int64_t H = p.nheads, L = p.seqlen;
     const int64_t b = blockIdx.x / H, h = blockIdx.x % H;
     const int g = int(h / (H / p.ngroups));
@@ -141,7 +148,7 @@ __global__ void __launch_bounds__(512, 1) ssd_tc_kernel(const __grid_constant__ 
         tma_load_4d(st + Ly::kB + Ly::kBox, &maps.B, 64, g, t0, int(b), bar);
         tma_load_4d(st + Ly::kX, &maps.x, 0, int(h), t0, int(b), bar);
     };
-    if (tid == 0) {
+    if (ctl) {
         issue_chunk(0);
         if (n_chunks > 1) issue_chunk(1);
     }
@@ -173,7 +180,7 @@ __global__ void __launch_bounds__(512, 1) ssd_tc_kernel(const __grid_constant__ 
     const bf16_t* dtp = static_cast<const bf16_t*>(p.dt) + b * L * H + h;
     const int lane = tid & 31;
 
-    // Warp 0 prepares each chunk's step sizes and their running sum ahead of
+    // The scan warp prepares each chunk's step sizes and their running sum ahead of
     // it: lane l takes tokens 4l .. 4l+3 (raw steps loaded one chunk earlier
     // still), a warp scan adds the lanes' totals.  Results go to the scalar
     // buffer of the chunk's parity.
@@ -212,7 +219,7 @@ __global__ void __launch_bounds__(512, 1) ssd_tc_kernel(const __grid_constant__ 
             make_float4(ex2_approx(cL - a[0]) * d[0], ex2_approx(cL - a[1]) * d[1], ex2_approx(cL - a[2]) * d[2],
                         ex2_approx(cL - a[3]) * d[3]);
     };
-    if (warp == 0) {
+    if (warp == kScanWarp) {
         load_raw(0);
         scan_chunk(0);
         if (n_chunks > 1) load_raw(1);
@@ -241,13 +248,8 @@ __global__ void __launch_bounds__(512, 1) ssd_tc_kernel(const __grid_constant__ 
         const uint32_t st = sbase + uint32_t((c & 1) * Ly::kStageBytes);
         const float* dtc = dts;
         const float* csc = css;
-        // thread 0: the chunk's scores start on the tensor cores at once; the
-        // previous chunk's y store must have read its tile (the first box of
-        // the score tile, rewritten after the next barrier)
-        if (tid == 0) {
-            abort |= !issue_scores(c);
-            bulk_wait_read<0>();
-        }
+        // the chunk's scores start on the tensor cores at once
+        if (ctl) abort |= !issue_scores(c);
         // z of this chunk's rows, in registers until the output step
         uint4 zr[2];
         if constexpr (kGate) {
@@ -277,12 +279,15 @@ __global__ void __launch_bounds__(512, 1) ssd_tc_kernel(const __grid_constant__ 
             }
         }
         fence_proxy_async_smem();
+        // the previous chunk's y store must have read its tile (the first box
+        // of the score tile, rewritten after this barrier)
+        if (ctl) bulk_wait_read<0>();
         if (__syncthreads_or(abort)) {
             ok = false;
             break;
         }
         // dS = B^T X_w and Yx = C S_prev, while the scores are masked
-        if (tid == 0) {
+        if (ctl) {
             tc_fence_after_sync();
 #pragma unroll
             for (int k = 0; k < Q / 16; ++k) {
@@ -360,8 +365,8 @@ __global__ void __launch_bounds__(512, 1) ssd_tc_kernel(const __grid_constant__ 
             ok = false;
             break;
         }
-        // Ym = M X; meanwhile warp 0 prepares the next chunk's step sizes
-        if (tid == 0) {
+        // Ym = M X; meanwhile the scan warp prepares the next chunk's step sizes
+        if (ctl) {
             tc_fence_after_sync();
 #pragma unroll
             for (int k = 0; k < Q / 16; ++k) {
@@ -371,7 +376,7 @@ __global__ void __launch_bounds__(512, 1) ssd_tc_kernel(const __grid_constant__ 
             }
             umma_commit(ybar);
         }
-        if (warp == 0 && c + 1 < n_chunks) {
+        if (warp == kScanWarp && c + 1 < n_chunks) {
             __syncwarp();
             scan_chunk(c + 1);
             if (c + 2 < n_chunks) load_raw(c + 2);
@@ -435,20 +440,20 @@ __global__ void __launch_bounds__(512, 1) ssd_tc_kernel(const __grid_constant__ 
             ok = false;
             break;
         }
-        if (tid == 0) {
+        if (ctl) {
             tma_store_4d(&maps.y, smem + Ly::kM, 0, int(h), t0, int(b));
             bulk_commit();
             if (c + 2 < n_chunks) issue_chunk(c + 2);
         }
     }
-    if (!ok && tid == 0) {
+    if (!ok && ctl) {
         // give the copies and products still in flight a bounded chance to land
         for (int k = 0; k < 5; ++k) {
             mbar_wait_bounded(full + k, 0u, nullptr, 50000000ull);
             mbar_wait_bounded(full + k, 1u, nullptr, 50000000ull);
         }
     }
-    if (tid == 0) bulk_wait<0>();
+    if (ctl) bulk_wait<0>();
     if (ok && p.last_state) {
         float* ls = p.last_state + ((b * H + h) * NS + row) * P + 16 * qd;
 #pragma unroll
