@@ -10,6 +10,7 @@
 // one (batch, head) and walks its chunks of Q = 128 tokens in order.  Per chunk:
 //
 //   G   = C B^T                   (128 x 128, K = N)     TMEM columns   0..127
+//                                                        (384..511 for odd chunks)
 //   dS  = B^T diag(w) X,  w_j = exp(cs_last - cs_j) Delta_j
 //                                  (N x P = 128 x 64, K = Q) columns 256..319
 //   Yx  = C S_prev                (128 x 64, K = N)      columns 192..255
@@ -30,13 +31,13 @@
 // threads in the same layout.  One thread issues the MMAs and the TMA copies,
 // from a warp whose scores are all masked (it has the least work).
 //
-// Order within a chunk, with three CTA barriers: C B^T starts as soon as the
-// chunk's tiles land; the threads scale X (barrier); B^T X_w and C S_prev
-// start, and the threads mask and decay the scores as soon as C B^T is done
-// (barrier); M X starts while another such warp prepares the next chunk's step sizes and
-// decay sums (their raw steps and this chunk's z were loaded a chunk ahead);
-// the state update waits only for B^T X_w, the output only for M X
-// (barrier); then the y store and the loads of chunk c + 2.  Each thread
+// Order within a chunk, with three CTA barriers: the threads scale X
+// (barrier); B^T X_w and C S_prev start, and the threads mask and decay the
+// scores, whose C B^T ran during the previous chunk's output step (barrier);
+// M X starts, then the next chunk's C B^T, while another lightly loaded warp
+// prepares the next chunk's step sizes and decay sums (their raw steps were
+// loaded a chunk ahead); the state update waits only for B^T X_w, the output
+// only for M X (barrier); then the y store and the loads of chunk c + 2.  Each thread
 // waits on the MMA completion barriers itself; a wait that gives up is
 // folded into the next CTA barrier.  Score blocks of 32 x 32 wholly above
 // the diagonal are skipped by the warp; blocks wholly below it use
@@ -84,7 +85,9 @@ struct SsdTcLayout {
     static constexpr int kTmemSlot = kBars + 5 * 8;
     static constexpr int kSmemBytes = kTmemSlot + 16 + 1024;  // + base alignment slack
     static constexpr uint32_t kTmemCols = 512;
-    static constexpr uint32_t kColG = 0, kColYm = 128, kColYx = 192, kColS = 256;
+    // scores of even and odd chunks (the next chunk's are computed during this
+    // one's output step), M X, C S_prev, B^T X_w
+    static constexpr uint32_t kColG = 0, kColYm = 128, kColYx = 192, kColS = 256, kColG2 = 384;
 };
 
 template <bool kGate, bool kSoftplus>
@@ -234,7 +237,7 @@ __global__ void __launch_bounds__(512, 1) ssd_tc_kernel(const __grid_constant__ 
 #pragma unroll
         for (int k = 0; k < NS / 16; ++k) {
             const uint32_t off = uint32_t((k >> 2) * Ly::kBox + (k & 3) * 32);
-            umma_bf16(tmem + Ly::kColG, smem_desc_sw128(st + Ly::kC + off, 16, 1024),
+            umma_bf16(tmem + ((c & 1) ? Ly::kColG2 : Ly::kColG), smem_desc_sw128(st + Ly::kC + off, 16, 1024),
                       smem_desc_sw128(st + Ly::kB + off, 16, 1024), idG, k > 0);
         }
         umma_commit(gbar);
@@ -242,14 +245,15 @@ __global__ void __launch_bounds__(512, 1) ssd_tc_kernel(const __grid_constant__ 
     };
 
     bool abort = false;  // a bounded wait of this thread gave up (folded into the next CTA barrier)
+    // the first chunk's scores; each later chunk's start during the previous
+    // chunk's output step
+    if (ctl && n_chunks > 0) abort |= !issue_scores(0);
     for (int c = 0; c < n_chunks && ok; ++c) {
         const int t0 = c * Q;
         const uint32_t ph = uint32_t(c & 1);  // each completion barrier completes once per chunk
         const uint32_t st = sbase + uint32_t((c & 1) * Ly::kStageBytes);
         const float* dtc = dts;
         const float* csc = css;
-        // the chunk's scores start on the tensor cores at once
-        if (ctl) abort |= !issue_scores(c);
         // z of this chunk's rows, in registers until the output step
         uint4 zr[2];
         if constexpr (kGate) {
@@ -318,7 +322,7 @@ __global__ void __launch_bounds__(512, 1) ssd_tc_kernel(const __grid_constant__ 
                     *reinterpret_cast<uint4*>(Ms + sw128(row, 4 * (qd & 1) + q)) = make_uint4(0u, 0u, 0u, 0u);
             } else {
                 float gv[32];
-                tmem_ld32(tlane + Ly::kColG + uint32_t(32 * qd), gv);
+                tmem_ld32(tlane + ((c & 1) ? Ly::kColG2 : Ly::kColG) + uint32_t(32 * qd), gv);
                 tmem_wait_ld();
                 // A block wholly below the diagonal (every j <= i): exp2(cs_i - cs_j)
                 // = exp2(cs_i - cs_L) exp2(cs_L - cs_j) with L = 32 qd + 31 <= i;
@@ -375,6 +379,10 @@ __global__ void __launch_bounds__(512, 1) ssd_tc_kernel(const __grid_constant__ 
                           smem_desc_sw128(st + Ly::kX + uint32_t(k * 2048), 0, 1024), idK, k > 0);
             }
             umma_commit(ybar);
+            // the next chunk's scores, into the other score buffer (its last
+            // reader, the masking of chunk c - 1, finished before this chunk's
+            // first barrier)
+            if (c + 1 < n_chunks) abort |= !issue_scores(c + 1);
         }
         if (warp == kScanWarp && c + 1 < n_chunks) {
             __syncwarp();
