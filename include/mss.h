@@ -301,8 +301,9 @@ MSS_API int64_t mss_scan_fwd_noalloc_scratch_bytes(void);
  * than store them ("Mamba" paper review, section "Selection Mechanism"); they
  * print no gradient, so this is the chain rule of the forward definition.
  * The states are recomputed from checkpoints (one state per channel every
- * 128 bytes of a row, or every 16 tokens on the scalar path) that the call
- * writes into the caller's workspace; nothing else is stored.
+ * 16 bytes of a row, i.e. 8 bf16 or 4 fp32 tokens, or every 16 tokens on the
+ * scalar path) that the call writes into the caller's workspace; nothing
+ * else is stored.
  *
  *   forward inputs: u, delta, A, B, C, D, z, delta_bias, softplus_flag,
  *                   initial_state, with the layouts of mss_scan_fwd_ex2, and
