@@ -701,6 +701,25 @@ def run_mss(args, rank, world, local_rank):
             bwd_ev.append((a_, b_))
     torch.cuda.synchronize(dev)
     bwd_ms = [a_.elapsed_time(b_) for a_, b_ in bwd_ev]
+
+    # a training step: the forward pass that stores the states, then the
+    # backward pass from them (no checkpoint pass)
+    y_t = torch.empty_like(y)
+    st_t = torch.empty_like(state)
+    tr_ev = []
+    for i in range(args.warmup + args.steps):
+        e = [torch.cuda.Event(enable_timing=True) for _ in range(3)]
+        e[0].record(stream)
+        mss.scan_fwd_save(**d, y=y_t, last_state=st_t, states=ws_b)
+        e[1].record(stream)
+        mss.scan_bwd(**d, dy=dy_d, dlast=dlast_d, saved_states=ws_b)
+        e[2].record(stream)
+        if i >= args.warmup:
+            tr_ev.append(e)
+    torch.cuda.synchronize(dev)
+    fwd_save_ms = [e[0].elapsed_time(e[1]) for e in tr_ev]
+    bwd_saved_ms = [e[1].elapsed_time(e[2]) for e in tr_ev]
+    assert mss.get_device_error() == 0
     assert mss.get_device_error() == 0
 
     # end to end through the public calls with host buffers, every step: the
@@ -806,8 +825,8 @@ def run_mss(args, rank, world, local_rank):
     # backward traffic: u, delta read by the checkpoint pass; u, delta, z, dy
     # read and du, ddelta, dz written by the backward kernel (bf16); B, C read
     # by both passes, dB, dC written (fp32); checkpoints (one fp32 state per
-    # 64-token chunk) written and read
-    n_ck = (w.seqlen + 63) // 64
+    # 8-token group) written and read
+    n_ck = (w.seqlen + 7) // 8
     bytes_bwd = (w.batch * w.dim * w.seqlen * 2 * (2 + 4 + 3) + 2 * w.batch * w.dstate * w.seqlen * (2 + 2 + 4)
                  + 2 * w.batch * w.dim * n_ck * w.dstate * 4)
     bytes_conv = bytes_fwd + 2 * w.batch * w.dim * 3 * 2 + w.dim * 5 * 4  # + conv states and taps
@@ -849,6 +868,14 @@ def run_mss(args, rank, world, local_rank):
                      "achieved_gbs": bytes_bwd / (bwd_avg * 1e-3) / 1e9,
                      "frac": bytes_bwd / (bwd_avg * 1e-3) / 1e9 / peak,
                      "note": "gradients of u, delta, A, B, C, D, z, bias, starting state; checkpoint pass included"},
+        "training_step": {"fwd_save_ms_avg": sum(fwd_save_ms) / len(fwd_save_ms),
+                          "bwd_saved_ms_avg": sum(bwd_saved_ms) / len(bwd_saved_ms),
+                          "step_ms": sum(fwd_save_ms) / len(fwd_save_ms) + sum(bwd_saved_ms) / len(bwd_saved_ms),
+                          "recompute_step_ms": fwd_avg + bwd_avg,
+                          "states_bytes": int(ws_b.numel()),
+                          "note": "mss_scan_fwd_save (the forward pass also storing the state at every 8-token "
+                                  "group) then mss_scan_bwd with MSS_FLAG_SAVED_STATES; recompute_step_ms: "
+                                  "mss_scan_fwd_ex2 then mss_scan_bwd with its checkpoint pass"},
         "ssd_path": {"workload": gen.SSD_WORKLOAD, "ms_avg": ssd_ms,
                      "channel_tokens_per_s": ss["batch"] * ss["seqlen"] * ss["nheads"] * ss["headdim"] / (ssd_ms * 1e-3),
                      # the binding roof at the measured peaks: HBM (its bytes take longer

@@ -77,7 +77,8 @@ enum mss_status {
     MSS_ERR_FLAGS = -8,          /* unknown bits in `flags` */
     MSS_ERR_ALIAS = -9,          /* an output overlaps an input */
     MSS_ERR_SCRATCH = -10,       /* mss_scan_fwd_noalloc: the split needs more than its fixed scratch */
-    MSS_ERR_WORKSPACE = -11      /* mss_scan_bwd: no workspace, or smaller than it needs */
+    MSS_ERR_WORKSPACE = -11,     /* mss_scan_bwd: no workspace, or smaller than it needs */
+    MSS_ERR_PATH = -12           /* saved states: the sizes, flags or alignments take the scalar kernels */
 };
 
 /* Flags of mss_scan_fwd_ex / mss_scan_fwd_ex2 / mss_scan_fwd_noalloc
@@ -102,6 +103,10 @@ enum mss_status {
  * call returns MSS_ERR_FLAGS and launches nothing.  The sequence is not
  * split. */
 #define MSS_FLAG_SELFTEST_TIMEOUT 0x10u
+/* mss_scan_bwd (and mss_scan_bwd_workspace_size): the workspace already holds
+ * the states that mss_scan_fwd_save wrote for the same inputs, so the call
+ * skips its checkpoint pass.  See mss_scan_fwd_save. */
+#define MSS_FLAG_SAVED_STATES 0x20u
 
 /*
  * mss_scan_fwd -- selective-scan forward pass over whole sequences.
@@ -169,6 +174,39 @@ MSS_API int mss_scan_fwd_ex2(const void *u, const void *delta, const float *A, c
                              int64_t batch, int64_t dim, int64_t dstate, int64_t seqlen,
                              int dtype, unsigned flags, void *workspace, int64_t workspace_bytes,
                              void *stream);
+
+/*
+ * mss_scan_fwd_save -- mss_scan_fwd_ex2 for a training step: the forward pass
+ * that also stores the states mss_scan_bwd would otherwise recompute in its
+ * checkpoint pass.  The pages train the model end to end and have the fused
+ * kernel keep the states out of HBM except where the backward pass needs them
+ * ("Mamba" paper review, section "Selection Mechanism"); the forward pass is
+ * where those states are formed anyway, so storing them costs writes only.
+ *
+ *   every argument of mss_scan_fwd_ex2, with the same meaning, then
+ *   states       : device memory of at least states_bytes =
+ *                  mss_scan_bwd_workspace_size(batch, dim, dstate, seqlen,
+ *                  dtype, flags) bytes, 16-byte aligned, owned by the caller:
+ *                  the state at the start of every group of 16 bytes of a row
+ *                  (8 bf16 or 4 fp32 tokens), written in full by the call and
+ *                  read by mss_scan_bwd with MSS_FLAG_SAVED_STATES.  Its layout
+ *                  is private to the library.
+ *
+ * Then call mss_scan_bwd with the same forward inputs, the same flags plus
+ * MSS_FLAG_SAVED_STATES, and `states` as its workspace (not modified between
+ * the two calls).  The call needs the tiled kernels: dstate 4, 8 or 16,
+ * 16-byte-aligned rows and tensors, no MSS_FLAG_SIMPLE; otherwise it returns
+ * MSS_ERR_PATH and launches nothing (use mss_scan_fwd_ex2 and mss_scan_bwd
+ * without the flag).  y and last_state are those of mss_scan_fwd_ex2, bit for
+ * bit.  MSS_ERR_WORKSPACE when states is NULL or too small; MSS_ERR_ALIAS when
+ * it overlaps another argument; otherwise the errors of mss_scan_fwd_ex2.
+ */
+MSS_API int mss_scan_fwd_save(const void *u, const void *delta, const float *A, const void *B,
+                              const void *C, const float *D, const void *z, const float *delta_bias,
+                              int softplus_flag, const float *initial_state, void *y, float *last_state,
+                              int64_t batch, int64_t dim, int64_t dstate, int64_t seqlen,
+                              int dtype, unsigned flags, void *workspace, int64_t workspace_bytes,
+                              void *states, int64_t states_bytes, void *stream);
 
 /*
  * mss_scan_fwd_workspace_size -- bytes of workspace mss_scan_fwd_ex2 would use
@@ -308,7 +346,10 @@ MSS_API int64_t mss_scan_fwd_noalloc_scratch_bytes(void);
  *   forward inputs: u, delta, A, B, C, D, z, delta_bias, softplus_flag,
  *                   initial_state, with the layouts of mss_scan_fwd_ex2, and
  *                   flags (MSS_FLAG_ZOH_INPUT, MSS_FLAG_GENERAL_A,
- *                   MSS_FLAG_SIMPLE) as used by the forward pass
+ *                   MSS_FLAG_SIMPLE) as used by the forward pass, plus
+ *                   MSS_FLAG_SAVED_STATES when the workspace holds the states
+ *                   of mss_scan_fwd_save (the checkpoint pass is skipped; the
+ *                   call then needs the tiled kernels, else MSS_ERR_PATH)
  *   dy      : [batch][dim][seqlen] dtype, dLoss/dy
  *   dlast   : [batch][dim][dstate] float, dLoss/dlast_state (NULL: zero)
  *   du, ddelta : [batch][dim][seqlen] dtype out (ddelta: with respect to
@@ -320,7 +361,8 @@ MSS_API int64_t mss_scan_fwd_noalloc_scratch_bytes(void);
  *   dinit   : [batch][dim][dstate] float out, dLoss/dinitial_state (NULL: not written)
  *   workspace : at least mss_scan_bwd_workspace_size bytes of device memory,
  *               16-byte aligned, owned by the caller; its contents on entry
- *               do not matter
+ *               do not matter, except with MSS_FLAG_SAVED_STATES, where they
+ *               are read and not written
  *
  * dA, dB, dC, dD and dbias are zeroed and then accumulated with float atomics
  * on the stream, so they are not bitwise reproducible between runs.  No

@@ -38,6 +38,8 @@ FLAG_SIMPLE = 0x2
 FLAG_NO_SPLIT = 0x4
 FLAG_ZOH_INPUT = 0x8  # zero-order-hold input matrix (e^{Delta A} - 1)/A * B instead of Delta * B
 FLAG_SELFTEST_TIMEOUT = 0x10  # the tiled kernel's bounded wait gives up on purpose (failure-path tests)
+FLAG_SAVED_STATES = 0x20  # scan_bwd: the workspace holds the states scan_fwd_save stored
+ERR_PATH = -12
 ERR_FLAGS = -8
 SSD_FLAG_WARP_MMA = 0x1  # ssd_fwd: the warp-level (mma.sync) kernels instead of the tcgen05 one
 ERR_DEVICE_TIMEOUT = -7
@@ -77,6 +79,9 @@ def load_library():
             lib.mss_scan_fwd_ex2.argtypes = [vp, vp, fp, vp, vp, fp, vp, fp, i, fp, vp, fp,
                                              i64, i64, i64, i64, i, u32, vp, i64, vp]
             lib.mss_scan_fwd_ex2.restype = i
+            lib.mss_scan_fwd_save.argtypes = [vp, vp, fp, vp, vp, fp, vp, fp, i, fp, vp, fp,
+                                              i64, i64, i64, i64, i, u32, vp, i64, vp, i64, vp]
+            lib.mss_scan_fwd_save.restype = i
             lib.mss_scan_fwd_workspace_size.argtypes = [i64, i64, i64, i64, i, u32]
             lib.mss_scan_fwd_workspace_size.restype = i64
             lib.mss_state_update.argtypes = [fp, vp, vp, fp, vp, vp, fp, vp, fp, i, vp,
@@ -185,6 +190,26 @@ def scan_fwd(u, delta, A, B, C, D=None, z=None, delta_bias=None, softplus=True,
     input matrix.  workspace: "auto" (the size the library asks for, allocated from
     PyTorch's caching allocator), None (no sequence split), or a uint8 CUDA
     tensor the call may use."""
+    y, last_state, _ = _scan_fwd(u, delta, A, B, C, D, z, delta_bias, softplus, y, last_state, want_last_state,
+                                 initial_state, workspace, flags, stream, None)
+    return y, last_state
+
+
+def scan_fwd_save(u, delta, A, B, C, D=None, z=None, delta_bias=None, softplus=True,
+                  y=None, last_state=None, want_last_state=True, initial_state=None,
+                  workspace="auto", states="auto", flags=0, stream=None):
+    """The forward pass of a training step (mss_scan_fwd_save): scan_fwd that
+    also stores the states scan_bwd needs.  Returns (y, last_state, states);
+    pass `states` to scan_bwd(saved_states=...) with the same inputs and flags.
+    states: "auto" (allocated here) or a uint8 CUDA tensor of at least
+    bwd_workspace_size(...) bytes.  Raises MssError(ERR_PATH) for calls the
+    tiled kernels do not take (then use scan_fwd and scan_bwd without it)."""
+    return _scan_fwd(u, delta, A, B, C, D, z, delta_bias, softplus, y, last_state, want_last_state,
+                     initial_state, workspace, flags, stream, states)
+
+
+def _scan_fwd(u, delta, A, B, C, D, z, delta_bias, softplus, y, last_state, want_last_state, initial_state,
+              workspace, flags, stream, states):
     if not isinstance(u, torch.Tensor) or u.device.type != "cuda":
         raise ValueError("u must be a CUDA tensor (there is no CPU path)")
     if u.dim() != 3:
@@ -217,14 +242,29 @@ def scan_fwd(u, delta, A, B, C, D=None, z=None, delta_bias=None, softplus=True,
         workspace = torch.empty(nbytes, dtype=torch.uint8, device=dev) if nbytes > 0 else None
     if workspace is not None:
         _check(workspace, "workspace", (workspace.numel(),), torch.uint8, dev)
-    rc = load_library().mss_scan_fwd_ex2(
+    if states is None:
+        rc = load_library().mss_scan_fwd_ex2(
+            _ptr(u), _ptr(delta), _ptr(A), _ptr(B), _ptr(C), _ptr(D), _ptr(z), _ptr(delta_bias),
+            int(bool(softplus)), _ptr(initial_state), _ptr(y), _ptr(last_state), batch, dim, N, L, code,
+            int(flags), _ptr(workspace), 0 if workspace is None else workspace.numel(),
+            _stream_handle(stream, dev))
+        if rc != 0:
+            raise MssError(rc, "mss_scan_fwd")
+        return y, last_state, None
+    if isinstance(states, str):
+        if states != "auto":
+            raise ValueError("states must be 'auto' or a uint8 CUDA tensor")
+        states = torch.empty(max(bwd_workspace_size(batch, dim, N, L, dt, flags), 16), dtype=torch.uint8,
+                             device=dev)
+    _check(states, "states", (states.numel(),), torch.uint8, dev)
+    rc = load_library().mss_scan_fwd_save(
         _ptr(u), _ptr(delta), _ptr(A), _ptr(B), _ptr(C), _ptr(D), _ptr(z), _ptr(delta_bias),
         int(bool(softplus)), _ptr(initial_state), _ptr(y), _ptr(last_state), batch, dim, N, L, code,
-        int(flags), _ptr(workspace), 0 if workspace is None else workspace.numel(),
-        _stream_handle(stream, dev))
+        int(flags), _ptr(workspace), 0 if workspace is None else workspace.numel(), _ptr(states),
+        states.numel(), _stream_handle(stream, dev))
     if rc != 0:
-        raise MssError(rc, "mss_scan_fwd")
-    return y, last_state
+        raise MssError(rc, "mss_scan_fwd_save")
+    return y, last_state, states
 
 
 def scan_fwd_host(u, delta, A, B, C, D=None, z=None, delta_bias=None, softplus=True,
@@ -401,13 +441,18 @@ def bwd_workspace_size(batch, dim, dstate, seqlen, dtype=torch.bfloat16, flags=0
 
 
 def scan_bwd(u, delta, A, B, C, dy, D=None, z=None, delta_bias=None, softplus=True, initial_state=None,
-             dlast=None, flags=0, workspace="auto", want_dinit=True, out=None, stream=None):
+             dlast=None, flags=0, workspace="auto", want_dinit=True, out=None, stream=None, saved_states=None):
     """Backward pass of scan_fwd (mss_scan_bwd).  dy: [batch, dim, L] (the io
     dtype), dlast: [batch, dim, N] float32 or None.  Returns a dict with du,
     ddelta, dz (None without z) in the io dtype, dA [dim, N], dB, dC
     [batch, N, L], dD, dbias [dim] and dinit [batch, dim, N] in float32.
     out: optional dict of caller-owned output tensors under those names (the
-    rest are allocated)."""
+    rest are allocated).  saved_states: the states scan_fwd_save returned for
+    these inputs and flags; the call then skips its checkpoint pass (the
+    tensor is its workspace)."""
+    if saved_states is not None:
+        flags = int(flags) | FLAG_SAVED_STATES
+        workspace = saved_states
     if not isinstance(u, torch.Tensor) or u.device.type != "cuda":
         raise ValueError("u must be a CUDA tensor (there is no CPU path)")
     batch, dim, L = u.shape

@@ -56,24 +56,28 @@ int launch_bwd_variant(const mss::BwdMaps& maps, const mss::BwdParams& p, unsign
 
 template <typename T, int N, bool kZoh>
 int launch_bwd_fast(mss::ScanParams fp, const mss::BwdParams& bp, unsigned flags, cudaStream_t s) {
+    const bool saved = (flags & MSS_FLAG_SAVED_STATES) != 0;
     constexpr int esz = int(sizeof(T));
     const int64_t rows = fp.batch * fp.dim;
     constexpr int br = mss::SeqLayout<T, N>::kRows;
-    // checkpoint pass
-    mss::SeqMaps fm;
-    std::memset(&fm, 0, sizeof(fm));
-    if (!encode_rows(&fm.u, fp.u, rows, fp.seqlen, esz, br) || !encode_rows(&fm.delta, fp.delta, rows, fp.seqlen, esz, br) ||
-        !encode_bc(&fm.B, fp.B, fp.batch, N, fp.seqlen, esz) || !encode_bc(&fm.C, fp.C, fp.batch, N, fp.seqlen, esz))
-        return MSS_ERR_CUDA;
-    fp.n_seg = 1;
-    fp.seg_len = fp.seqlen;
-    fp.agg = nullptr;
-    fp.y = nullptr;
-    fp.last_state = nullptr;
-    fp.z = nullptr;
-    int rc = fp.softplus ? launch_seq_variant<T, N, false, true, true, kZoh, false>(fm, fp, flags, 1, s)
-                         : launch_seq_variant<T, N, false, false, true, kZoh, false>(fm, fp, flags, 1, s);
-    if (rc != MSS_OK) return rc;
+    // checkpoint pass, unless the forward pass saved the states
+    if (!saved) {
+        mss::SeqMaps fm;
+        std::memset(&fm, 0, sizeof(fm));
+        if (!encode_rows(&fm.u, fp.u, rows, fp.seqlen, esz, br) ||
+            !encode_rows(&fm.delta, fp.delta, rows, fp.seqlen, esz, br) ||
+            !encode_bc(&fm.B, fp.B, fp.batch, N, fp.seqlen, esz) || !encode_bc(&fm.C, fp.C, fp.batch, N, fp.seqlen, esz))
+            return MSS_ERR_CUDA;
+        fp.n_seg = 1;
+        fp.seg_len = fp.seqlen;
+        fp.agg = nullptr;
+        fp.y = nullptr;
+        fp.last_state = nullptr;
+        fp.z = nullptr;
+        const int rc = fp.softplus ? launch_seq_variant<T, N, false, true, true, kZoh, false>(fm, fp, flags, 1, s)
+                                   : launch_seq_variant<T, N, false, false, true, kZoh, false>(fm, fp, flags, 1, s);
+        if (rc != MSS_OK) return rc;
+    }
     // backward
     mss::BwdMaps bm;
     std::memset(&bm, 0, sizeof(bm));
@@ -116,6 +120,8 @@ int launch_backward(mss::ScanParams fp, mss::BwdParams bp, unsigned flags, void*
             return fp.zoh ? launch_bwd_fast<T, N, true>(fp, bp, flags, s) : launch_bwd_fast<T, N, false>(fp, bp, flags, s);
         }
     }
+    // saved states are in the tiled kernels' layout
+    if (flags & MSS_FLAG_SAVED_STATES) return MSS_ERR_PATH;
     const int64_t need = rows * ((L + mss::kBwdSimpleChunk - 1) / mss::kBwdSimpleChunk) * N * 4;
     if (!workspace || need > workspace_bytes || !aligned(workspace, 4)) return MSS_ERR_WORKSPACE;
     const int64_t blocks = (rows + 127) / 128;

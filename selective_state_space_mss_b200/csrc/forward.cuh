@@ -73,26 +73,6 @@ int launch_simple(const mss::ScanParams& p, cudaStream_t stream) {
     return launch_status();
 }
 
-// The sizes the tiled kernels take (grid limits, 32-bit tensor-map row
-// coordinates); the backward pass's workspace size follows the same test.
-inline bool seq_shape_ok(int64_t batch, int64_t dim, int64_t seqlen, int64_t N, int esz, unsigned flags) {
-    if (flags & MSS_FLAG_SIMPLE) return false;
-    if (N != 4 && N != 8 && N != 16) return false;
-    if ((seqlen * esz) % 16 != 0) return false;
-    if (batch * dim >= (int64_t(1) << 31) || seqlen >= (int64_t(1) << 31)) return false;
-    if ((dim + 15) / 16 > 0x7fffffffLL || batch > 65535) return false;
-    return true;
-}
-
-// The throughput kernel's requirements; otherwise the scalar kernel runs.
-inline bool seq_eligible(const mss::ScanParams& p, int64_t N, int esz, unsigned flags) {
-    if (!seq_shape_ok(p.batch, p.dim, p.seqlen, N, esz, flags)) return false;
-    const void* v[] = {p.u, p.delta, p.z, p.B, p.C, p.y};
-    for (const void* q : v)
-        if (q && !aligned(q, 16)) return false;
-    return true;
-}
-
 template <typename T, int N, bool kGate, bool kSoftplus, bool kFold, bool kZoh, bool kConv>
 int launch_seq_variant(const mss::SeqMaps& maps, const mss::ScanParams& p, unsigned flags, int segs,
                        cudaStream_t stream) {
@@ -154,10 +134,13 @@ inline int64_t agg_bytes(int n_seg, int64_t rows, int64_t N) { return n_seg > 1 
 template <typename T, int N, bool kZoh, bool kConv>
 int launch_seq_passes(const mss::SeqMaps& maps, const mss::ScanParams& p, unsigned flags, cudaStream_t stream) {
     if (p.n_seg > 1) {
-        // first pass: each segment but the last folds to its aggregates
+        // first pass: each segment but the last folds to its aggregates (from
+        // a zero state: its states are not the sequence's, so it stores none)
+        mss::ScanParams pf = p;
+        pf.ckpt = nullptr;
         const int rc = p.softplus
-                           ? launch_seq_variant<T, N, false, true, true, kZoh, kConv>(maps, p, flags, p.n_seg - 1, stream)
-                           : launch_seq_variant<T, N, false, false, true, kZoh, kConv>(maps, p, flags, p.n_seg - 1, stream);
+                           ? launch_seq_variant<T, N, false, true, true, kZoh, kConv>(maps, pf, flags, p.n_seg - 1, stream)
+                           : launch_seq_variant<T, N, false, false, true, kZoh, kConv>(maps, pf, flags, p.n_seg - 1, stream);
         if (rc != MSS_OK) return rc;
     }
     if (p.z)
@@ -215,6 +198,21 @@ int launch_forward(mss::ScanParams p, unsigned flags, void* workspace, int64_t w
     return launch_simple<T, N>(p, stream);
 }
 
+// The forward pass that also stores the backward pass's group-start states
+// (mss_scan_fwd_save): the tiled kernel only, whose full pass writes them.
+template <typename T, int N>
+int launch_forward_save(mss::ScanParams p, unsigned flags, void* workspace, int64_t workspace_bytes, float* states,
+                        cudaStream_t stream) {
+    if constexpr (N == 4 || N == 8 || N == 16) {
+        if (seq_eligible(p, N, int(sizeof(T)), flags)) {
+            p.selftest_wait_ns = (flags & MSS_FLAG_SELFTEST_TIMEOUT) ? 1000000ull : 0ull;
+            p.ckpt = states;
+            return launch_seq<T, N>(p, flags, workspace, workspace_bytes, stream);
+        }
+    }
+    return MSS_ERR_PATH;
+}
+
 template <typename T, int N>
 int64_t forward_workspace_bytes(int64_t batch, int64_t dim, int64_t seqlen) {
     if constexpr (N == 4 || N == 8 || N == 16)
@@ -224,6 +222,7 @@ int64_t forward_workspace_bytes(int64_t batch, int64_t dim, int64_t seqlen) {
 
 #define MSS_INSTANTIATE_FORWARD(T, N)                                                                     \
     template int launch_forward<T, N>(mss::ScanParams, unsigned, void*, int64_t, cudaStream_t);          \
+    template int launch_forward_save<T, N>(mss::ScanParams, unsigned, void*, int64_t, float*, cudaStream_t); \
     template int64_t forward_workspace_bytes<T, N>(int64_t, int64_t, int64_t);
 
 // The convolution variants of (T, N) live in another translation unit.

@@ -10,6 +10,7 @@
 #include <cuda_runtime.h>
 
 #include "../../include/mss.h"
+#include "mss_params.h"
 
 namespace mss_host {
 
@@ -37,6 +38,26 @@ auto with_n(int64_t n, F&& f) -> decltype(f(std::integral_constant<int, 1>{})) {
         case 16: return f(std::integral_constant<int, 16>{});
         default: return MSS_ERR_UNSUPPORTED_N;
     }
+}
+
+// The sizes the tiled kernels take (grid limits, 32-bit tensor-map row
+// coordinates); the backward pass's workspace size follows the same test.
+inline bool seq_shape_ok(int64_t batch, int64_t dim, int64_t seqlen, int64_t N, int esz, unsigned flags) {
+    if (flags & MSS_FLAG_SIMPLE) return false;
+    if (N != 4 && N != 8 && N != 16) return false;
+    if ((seqlen * esz) % 16 != 0) return false;
+    if (batch * dim >= (int64_t(1) << 31) || seqlen >= (int64_t(1) << 31)) return false;
+    if ((dim + 15) / 16 > 0x7fffffffLL || batch > 65535) return false;
+    return true;
+}
+
+// The throughput kernel's requirements; otherwise the scalar kernel runs.
+inline bool seq_eligible(const mss::ScanParams& p, int64_t N, int esz, unsigned flags) {
+    if (!seq_shape_ok(p.batch, p.dim, p.seqlen, N, esz, flags)) return false;
+    const void* v[] = {p.u, p.delta, p.z, p.B, p.C, p.y};
+    for (const void* q : v)
+        if (q && !aligned(q, 16)) return false;
+    return true;
 }
 
 inline int launch_status() { return cudaGetLastError() == cudaSuccess ? MSS_OK : MSS_ERR_CUDA; }

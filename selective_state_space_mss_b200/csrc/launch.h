@@ -18,12 +18,19 @@ template <typename T, int N>
 int launch_forward(mss::ScanParams p, unsigned flags, void* workspace, int64_t workspace_bytes,
                    cudaStream_t stream);
 
+// The same through the tiled kernel only, also storing the backward pass's
+// group-start states; MSS_ERR_PATH when the tiled kernel does not take it.
+template <typename T, int N>
+int launch_forward_save(mss::ScanParams p, unsigned flags, void* workspace, int64_t workspace_bytes, float* states,
+                        cudaStream_t stream);
+
 // Workspace bytes the forward pass would use to split the sequence (0: none).
 template <typename T, int N>
 int64_t forward_workspace_bytes(int64_t batch, int64_t dim, int64_t seqlen);
 
 // Backward pass over validated arguments: fp holds the forward arguments
-// (with p.err), bp the gradients; the workspace holds the checkpoints.
+// (with p.err), bp the gradients; the workspace holds the checkpoints (with
+// MSS_FLAG_SAVED_STATES already written by the saving forward pass).
 template <typename T, int N>
 int launch_backward(mss::ScanParams fp, mss::BwdParams bp, unsigned flags, void* workspace, int64_t workspace_bytes,
                     cudaStream_t stream);
@@ -53,6 +60,8 @@ bool ssd_chunked_pays(int64_t batch, int64_t nheads);
 
 #define MSS_DECLARE_LAUNCHERS(T, N)                                                                      \
     extern template int launch_forward<T, N>(mss::ScanParams, unsigned, void*, int64_t, cudaStream_t); \
+    extern template int launch_forward_save<T, N>(mss::ScanParams, unsigned, void*, int64_t, float*,    \
+                                                  cudaStream_t);                                         \
     extern template int64_t forward_workspace_bytes<T, N>(int64_t, int64_t, int64_t);                   \
     extern template int launch_decode<T, N>(mss::StepParams, cudaStream_t);                              \
     extern template int launch_backward<T, N>(mss::ScanParams, mss::BwdParams, unsigned, void*, int64_t,   \

@@ -21,6 +21,7 @@ using namespace mss_host;
 
 constexpr unsigned kScanFlags =
     MSS_FLAG_GENERAL_A | MSS_FLAG_SIMPLE | MSS_FLAG_NO_SPLIT | MSS_FLAG_ZOH_INPUT | MSS_FLAG_SELFTEST_TIMEOUT;
+constexpr unsigned kBwdFlags = MSS_FLAG_GENERAL_A | MSS_FLAG_SIMPLE | MSS_FLAG_ZOH_INPUT | MSS_FLAG_SAVED_STATES;
 
 // The device error word (one per device, in the library image): kernels
 // whose bounded waits give up set it through the address in their
@@ -57,15 +58,17 @@ struct ConvArgs {
 };
 
 // The forward pass behind every mss_scan_fwd* entry point; cv = nullptr
-// without the convolution.
+// without the convolution; save: also store the backward pass's states
+// (mss_scan_fwd_save).
 int scan_fwd_impl(const ConvArgs* cv, const void* u, const void* delta, const float* A, const void* B,
                   const void* C, const float* D, const void* z, const float* delta_bias,
                   int softplus_flag, const float* initial_state, void* y, float* last_state,
                   int64_t batch, int64_t dim, int64_t dstate, int64_t seqlen,
-                  int dtype, unsigned flags, void* workspace, int64_t workspace_bytes, void* stream) {
+                  int dtype, unsigned flags, void* workspace, int64_t workspace_bytes, bool save, void* states,
+                  int64_t states_bytes, void* stream) {
     if (dtype != MSS_DTYPE_F32 && dtype != MSS_DTYPE_BF16) return MSS_ERR_DTYPE;
     if (flags & ~kScanFlags) return MSS_ERR_FLAGS;
-    if (batch < 0 || dim < 0 || seqlen < 0 || workspace_bytes < 0) return MSS_ERR_SHAPE;
+    if (batch < 0 || dim < 0 || seqlen < 0 || workspace_bytes < 0 || states_bytes < 0) return MSS_ERR_SHAPE;
     if (!valid_n(dstate)) return MSS_ERR_UNSUPPORTED_N;
     const int64_t esz = dtype == MSS_DTYPE_BF16 ? 2 : 4;
     int64_t rows, seq_elems, seq_bytes, bc_elems, bc_bytes, st_elems, st_bytes;
@@ -88,11 +91,24 @@ int scan_fwd_impl(const ConvArgs* cv, const void* u, const void* delta, const fl
                         cv ? cv->b : nullptr};
     for (const void* p : fp)
         if (p && !aligned(p, 4)) return MSS_ERR_ALIGN;
-    // outputs (y, last_state, workspace) must not overlap inputs or each other
+    // the saved states: the backward pass's workspace size for these arguments
+    int64_t need_states = 0;
+    if (save) {
+        if (cv) return MSS_ERR_PATH;
+        need_states = with_n(dstate, [&](auto nc) -> int64_t {
+            constexpr int N = decltype(nc)::value;
+            return dtype == MSS_DTYPE_BF16 ? backward_workspace_bytes<bf16_t, N>(batch, dim, seqlen, flags)
+                                           : backward_workspace_bytes<float, N>(batch, dim, seqlen, flags);
+        });
+        if (need_states > 0 && (!states || states_bytes < need_states)) return MSS_ERR_WORKSPACE;
+        if (states && !aligned(states, 16)) return MSS_ERR_ALIGN;
+    }
+    // outputs (y, last_state, workspace, states) must not overlap inputs or each other
     const int64_t ws = workspace ? workspace_bytes : 0;
+    const int64_t ss = save && states ? states_bytes : 0;
     struct Range { const void* p; int64_t n; };
     const Range outs[] = {{y, seq_bytes}, {last_state, st_bytes}, {workspace, ws},
-                          {cv ? cv->state_out : nullptr, cs_bytes}};
+                          {cv ? cv->state_out : nullptr, cs_bytes}, {save ? states : nullptr, ss}};
     const Range ins[] = {{u, seq_bytes}, {delta, seq_bytes}, {z, seq_bytes}, {B, bc_bytes}, {C, bc_bytes},
                          {A, dim * dstate * 4}, {D, dim * 4}, {delta_bias, dim * 4},
                          {initial_state, st_bytes}, {cv ? cv->w : nullptr, dim * K * 4},
@@ -132,9 +148,15 @@ int scan_fwd_impl(const ConvArgs* cv, const void* u, const void* delta, const fl
         p.conv_w = cv->w; p.conv_b = cv->b; p.conv_state_in = cv->state_in; p.conv_state_out = cv->state_out;
         p.conv_width = K;
     }
+    // saved states are written by the tiled kernel only
+    if (save && !seq_eligible(p, dstate, int(esz), flags)) return MSS_ERR_PATH;
     if (!(p.err = device_error_word())) return MSS_ERR_CUDA;
     return with_n(dstate, [&](auto nc) {
         constexpr int N = decltype(nc)::value;
+        float* st = static_cast<float*>(states);
+        if (save)
+            return dtype == MSS_DTYPE_BF16 ? launch_forward_save<bf16_t, N>(p, flags, workspace, ws, st, s)
+                                           : launch_forward_save<float, N>(p, flags, workspace, ws, st, s);
         return dtype == MSS_DTYPE_BF16 ? launch_forward<bf16_t, N>(p, flags, workspace, ws, s)
                                        : launch_forward<float, N>(p, flags, workspace, ws, s);
     });
@@ -223,6 +245,7 @@ const char* mss_strerror(int code) {
         case MSS_ERR_ALIAS: return "an output overlaps an input";
         case MSS_ERR_SCRATCH: return "the sequence split needs more than the library's fixed scratch holds";
         case MSS_ERR_WORKSPACE: return "no workspace, or a workspace smaller than the call needs";
+        case MSS_ERR_PATH: return "saved states need the tiled kernels, which these sizes, flags or alignments do not take";
         default: return "unknown status code";
     }
 }
@@ -233,7 +256,19 @@ int mss_scan_fwd_ex2(const void* u, const void* delta, const float* A, const voi
                      int64_t batch, int64_t dim, int64_t dstate, int64_t seqlen,
                      int dtype, unsigned flags, void* workspace, int64_t workspace_bytes, void* stream) {
     return scan_fwd_impl(nullptr, u, delta, A, B, C, D, z, delta_bias, softplus_flag, initial_state, y, last_state,
-                         batch, dim, dstate, seqlen, dtype, flags, workspace, workspace_bytes, stream);
+                         batch, dim, dstate, seqlen, dtype, flags, workspace, workspace_bytes, false, nullptr, 0,
+                         stream);
+}
+
+int mss_scan_fwd_save(const void* u, const void* delta, const float* A, const void* B,
+                      const void* C, const float* D, const void* z, const float* delta_bias,
+                      int softplus_flag, const float* initial_state, void* y, float* last_state,
+                      int64_t batch, int64_t dim, int64_t dstate, int64_t seqlen,
+                      int dtype, unsigned flags, void* workspace, int64_t workspace_bytes,
+                      void* states, int64_t states_bytes, void* stream) {
+    return scan_fwd_impl(nullptr, u, delta, A, B, C, D, z, delta_bias, softplus_flag, initial_state, y, last_state,
+                         batch, dim, dstate, seqlen, dtype, flags, workspace, workspace_bytes, true, states,
+                         states_bytes, stream);
 }
 
 int mss_scan_fwd_conv(const void* x, const float* conv_w, const float* conv_b, int conv_width,
@@ -244,7 +279,8 @@ int mss_scan_fwd_conv(const void* x, const float* conv_w, const float* conv_b, i
                       int dtype, unsigned flags, void* workspace, int64_t workspace_bytes, void* stream) {
     const ConvArgs cv{conv_w, conv_b, conv_width, conv_state_in, conv_state_out};
     return scan_fwd_impl(&cv, x, delta, A, B, C, D, z, delta_bias, softplus_flag, initial_state, y, last_state,
-                         batch, dim, dstate, seqlen, dtype, flags, workspace, workspace_bytes, stream);
+                         batch, dim, dstate, seqlen, dtype, flags, workspace, workspace_bytes, false, nullptr, 0,
+                         stream);
 }
 
 int64_t mss_scan_fwd_workspace_size(int64_t batch, int64_t dim, int64_t dstate, int64_t seqlen, int dtype,
@@ -317,7 +353,7 @@ int mss_scan_bwd(const void* u, const void* delta, const float* A, const void* B
                  float* dbias, float* dinit, int64_t batch, int64_t dim, int64_t dstate, int64_t seqlen,
                  int dtype, unsigned flags, void* workspace, int64_t workspace_bytes, void* stream) {
     if (dtype != MSS_DTYPE_F32 && dtype != MSS_DTYPE_BF16) return MSS_ERR_DTYPE;
-    if (flags & ~(MSS_FLAG_GENERAL_A | MSS_FLAG_SIMPLE | MSS_FLAG_ZOH_INPUT)) return MSS_ERR_FLAGS;
+    if (flags & ~kBwdFlags) return MSS_ERR_FLAGS;
     if (batch < 0 || dim < 0 || seqlen < 0 || workspace_bytes < 0) return MSS_ERR_SHAPE;
     if (!valid_n(dstate)) return MSS_ERR_UNSUPPORTED_N;
     const int64_t esz = dtype == MSS_DTYPE_BF16 ? 2 : 4;
@@ -370,6 +406,14 @@ int mss_scan_bwd(const void* u, const void* delta, const float* A, const void* B
     p.batch = batch; p.dim = dim; p.seqlen = seqlen; p.softplus = softplus_flag ? 1 : 0;
     p.initial_state = initial_state; p.seg_len = seqlen; p.n_seg = 1;
     p.zoh = (flags & MSS_FLAG_ZOH_INPUT) ? 1 : 0;
+    if (flags & MSS_FLAG_SAVED_STATES) {
+        // the saved states are in the tiled kernels' layout: the call must take them
+        bool tiled = seq_eligible(p, dstate, int(esz), flags);
+        const void* g16[] = {dy, du, ddelta, z ? dz : nullptr, dB, dC};
+        for (const void* g : g16)
+            if (g && !aligned(g, 16)) tiled = false;
+        if (!tiled) return MSS_ERR_PATH;
+    }
     if (!(p.err = device_error_word())) return MSS_ERR_CUDA;
     mss::BwdParams q{};
     q.u = u; q.delta = delta; q.A = A; q.B = B; q.C = C; q.D = D; q.z = z; q.delta_bias = delta_bias;
@@ -386,7 +430,7 @@ int mss_scan_bwd(const void* u, const void* delta, const float* A, const void* B
 int64_t mss_scan_bwd_workspace_size(int64_t batch, int64_t dim, int64_t dstate, int64_t seqlen, int dtype,
                                     unsigned flags) {
     if (dtype != MSS_DTYPE_F32 && dtype != MSS_DTYPE_BF16) return MSS_ERR_DTYPE;
-    if (flags & ~(MSS_FLAG_GENERAL_A | MSS_FLAG_SIMPLE | MSS_FLAG_ZOH_INPUT)) return MSS_ERR_FLAGS;
+    if (flags & ~kBwdFlags) return MSS_ERR_FLAGS;
     if (batch < 0 || dim < 0 || seqlen < 0) return MSS_ERR_SHAPE;
     if (!valid_n(dstate)) return MSS_ERR_UNSUPPORTED_N;
     int64_t rows, elems;

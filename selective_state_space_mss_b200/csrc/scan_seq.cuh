@@ -460,13 +460,14 @@ __device__ __forceinline__ void scan_seq_body(const SeqMaps& maps, const ScanPar
         else
             return h[i];
     };
-    // checkpoint pass: the state at the start of every group of V tokens, in
-    // h_n form, as [row][group][N] floats in lane order (lane half h's N/2
-    // floats at h * N/2: its pairs (h_n, h_n+2), n = h + 4i)
+    // checkpoint pass, or a forward pass that saves the states: the state at
+    // the start of every group of V tokens, in h_n form, as [row][group][N]
+    // floats over the whole sequence in lane order (lane half h's N/2 floats
+    // at h * N/2: its pairs (h_n, h_n+2), n = h + 4i)
     auto store_ckpt = [&](int group) {
         if (!valid) return;
-        float2* ck = reinterpret_cast<float2*>(p.ckpt + (size_t(row) * size_t(n_groups) + size_t(group)) * N) +
-                     half * P;
+        const size_t g_all = size_t(t_begin / V) + size_t(group);
+        float2* ck = reinterpret_cast<float2*>(p.ckpt + (size_t(row) * size_t(L / V) + g_all) * N) + half * P;
 #pragma unroll
         for (int i = 0; i < P; i += 2) {
             if (i + 1 < P) {
@@ -514,7 +515,7 @@ __device__ __forceinline__ void scan_seq_body(const SeqMaps& maps, const ScanPar
     for (int g = 0; g < n_groups; ++g) {
         const int c = g / GPC, j = g % GPC;
         const bool has_next = g + 1 < n_groups;
-        if (kFold && p.ckpt) store_ckpt(g);
+        if (p.ckpt) store_ckpt(g);
         // the next group's u/delta/z, first: its stage must have landed when it opens a new chunk
         if (has_next && j == GPC - 1 && !wait_chunk(c + 1)) return;
         float uv[HV], dv[HV], zv[HV];

@@ -271,6 +271,63 @@ def test_bwd_argument_errors(lib):
     assert q(1, 16, 16, 4096, 0, 0) == 16 * 1024 * 16 * 4          # fp32: one per 4-token group
 
 
+def test_saved_states_argument_errors(lib):
+    """mss_scan_fwd_save and MSS_FLAG_SAVED_STATES: the checks that need no
+    device (sizes, alignment, overlap, the tiled-path test)."""
+    codes = _enum("mss_status")
+    flag = int(re.search(r"#define MSS_FLAG_SAVED_STATES (0x[0-9a-f]+)u", _header()).group(1), 16)
+    v = ctypes.c_void_p
+    lib.mss_scan_fwd_save.restype = ctypes.c_int
+    lib.mss_scan_bwd.restype = ctypes.c_int
+    lib.mss_scan_bwd_workspace_size.restype = ctypes.c_int64
+    need = lib.mss_scan_bwd_workspace_size(ctypes.c_int64(2), ctypes.c_int64(8), ctypes.c_int64(16),
+                                           ctypes.c_int64(32), 1, ctypes.c_uint(0))
+    assert need == 2 * 8 * 4 * 16 * 4  # one state per 8-token group
+    assert lib.mss_scan_bwd_workspace_size(ctypes.c_int64(2), ctypes.c_int64(8), ctypes.c_int64(16),
+                                           ctypes.c_int64(32), 1, ctypes.c_uint(flag)) == need
+
+    def save(**kw):
+        a = dict(u=P, delta=P + 0x1000000, B=P + 0x3000000, C=P + 0x4000000, y=P + 0x5000000,
+                 st=P + 0x6000000, stb=need, batch=2, dim=8, N=16, L=32, dtype=1, flags=0)
+        a.update(kw)
+        w = lambda x: v(x) if x is not None else None
+        return lib.mss_scan_fwd_save(w(a["u"]), w(a["delta"]), v(P + 0x2000000), w(a["B"]), w(a["C"]), None, None,
+                                     None, 1, None, w(a["y"]), None, ctypes.c_int64(a["batch"]),
+                                     ctypes.c_int64(a["dim"]), ctypes.c_int64(a["N"]), ctypes.c_int64(a["L"]),
+                                     a["dtype"], ctypes.c_uint(a["flags"]), None, ctypes.c_int64(0), w(a["st"]),
+                                     ctypes.c_int64(a["stb"]), None)
+
+    assert save(st=None) == codes["MSS_ERR_WORKSPACE"]
+    assert save(stb=need - 1) == codes["MSS_ERR_WORKSPACE"]
+    assert save(stb=-1) == codes["MSS_ERR_SHAPE"]
+    assert save(st=P + 0x6000008) == codes["MSS_ERR_ALIGN"]          # states need 16-byte alignment
+    assert save(st=P + 0x5000000) == codes["MSS_ERR_ALIAS"]          # states on y
+    assert save(st=P + 0x1000000) == codes["MSS_ERR_ALIAS"]          # states on delta
+    assert save(flags=0x2, stb=1 << 20) == codes["MSS_ERR_PATH"]     # the scalar kernel stores none
+    assert save(N=2, stb=1 << 20) == codes["MSS_ERR_PATH"]
+    assert save(u=P + 2) == codes["MSS_ERR_PATH"]                   # rows not 16-byte aligned
+    assert save(L=33, stb=1 << 20) == codes["MSS_ERR_PATH"]          # odd rows
+    assert save(flags=0x40) == codes["MSS_ERR_FLAGS"]
+    assert save(batch=0) == 0
+    assert save(L=0, st=None, stb=0) == 0
+
+    def bwd(**kw):
+        a = dict(du=P + 0x6000000, dB=P + 0x9000000, N=16, L=32, flags=flag)
+        a.update(kw)
+        return lib.mss_scan_bwd(v(P), v(P + 0x1000000), v(P + 0x2000000), v(P + 0x3000000), v(P + 0x4000000), None,
+                                None, None, 1, None, v(P + 0x5000000), None, v(a["du"]), v(P + 0x7000000), None,
+                                v(P + 0x8000000), v(a["dB"]), v(P + 0xa000000), None, None, None, ctypes.c_int64(2),
+                                ctypes.c_int64(8), ctypes.c_int64(a["N"]), ctypes.c_int64(a["L"]), 1,
+                                ctypes.c_uint(a["flags"]), v(P + 0xb000000), ctypes.c_int64(1 << 20), None)
+
+    assert bwd(flags=flag | 0x2) == codes["MSS_ERR_PATH"]
+    assert bwd(N=2) == codes["MSS_ERR_PATH"]
+    assert bwd(du=P + 0x6000002) == codes["MSS_ERR_PATH"]   # a gradient row not 16-byte aligned
+    assert bwd(dB=P + 0x9000004) == codes["MSS_ERR_PATH"]
+    assert bwd(flags=0x40) == codes["MSS_ERR_FLAGS"]
+    assert "tiled" in lib.mss_strerror(codes["MSS_ERR_PATH"]).decode()
+
+
 def test_ssd_argument_errors(lib):
     codes = _enum("mss_status")
     v = ctypes.c_void_p

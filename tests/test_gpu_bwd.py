@@ -106,3 +106,54 @@ def test_bwd_zero_length():
     torch.cuda.synchronize()
     assert torch.equal(g["dinit"], dl)
     assert torch.count_nonzero(g["dA"]) == 0 and torch.count_nonzero(g["dD"]) == 0
+
+
+@pytest.mark.parametrize("dtype", ["f32", "bf16"])
+@pytest.mark.parametrize("N", [4, 8, 16])
+@pytest.mark.parametrize("zoh", [False, True], ids=["euler", "zoh"])
+@pytest.mark.parametrize("split", [False, True], ids=["one-pass", "split"])
+def test_saved_states_training_step(dtype, N, zoh, split):
+    """scan_fwd_save + scan_bwd(saved_states=...): y and last_state bit for bit
+    those of scan_fwd, every gradient within the oracle's bound; without a
+    sequence split the stored states are the checkpoint pass's, so the
+    per-token gradients and dinit also equal those of scan_bwd bit for bit."""
+    # few channels: with a workspace the forward pass takes its two-pass
+    # sequence split, without one it runs in one pass
+    batch, dim, L = (1, 48, 4096) if split else (2, 40, 1000)
+    flags = mss.FLAG_ZOH_INPUT if zoh else 0
+    io = torch.bfloat16 if dtype == "bf16" else torch.float32
+    ws = "auto" if split else None
+    assert mss.workspace_size(batch, dim, N, L, io) > 0
+    inp = gen.scan_inputs(batch, dim, N, L, dtype, seed=700 + N, d_skip="normal")
+    d = device_inputs(inp, DEV)
+    dy, dl = gen.upstream_gradients(batch, dim, N, L, dtype, 701)
+    h0 = np.random.default_rng(702).standard_normal((batch, dim, N)).astype(np.float32)
+    h0_d, dy_d, dl_d = torch.from_numpy(h0).to(DEV), to_torch(dy, DEV), torch.from_numpy(dl).to(DEV)
+    y_s, last_s, states = mss.scan_fwd_save(**d, initial_state=h0_d, flags=flags, workspace=ws)
+    y, last = mss.scan_fwd(**d, initial_state=h0_d, flags=flags, workspace=ws)
+    g_s = mss.scan_bwd(**d, dy=dy_d, dlast=dl_d, initial_state=h0_d, flags=flags, saved_states=states)
+    g = mss.scan_bwd(**d, dy=dy_d, dlast=dl_d, initial_state=h0_d, flags=flags)
+    torch.cuda.synchronize()
+    assert mss.get_device_error() == 0
+    assert states.numel() == mss.bwd_workspace_size(batch, dim, N, L, io, flags)
+    assert torch.equal(y_s, y) and torch.equal(last_s, last)
+    ref = oracle.scan_bwd(inp["u"].values, inp["delta"].values, inp["A"], inp["B"].values, inp["C"].values,
+                          dy.values, D=inp["D"], z=inp["z"].values, delta_bias=inp["delta_bias"],
+                          initial_state=h0.astype(np.float64), dlast=dl.astype(np.float64), zoh_input=zoh)
+    _compare(g_s, ref, dtype, f"saved N={N}")
+    if not split:
+        for k in ("du", "ddelta", "dz", "dinit"):
+            assert torch.equal(g_s[k], g[k]), k
+
+
+def test_saved_states_refused_off_the_tiled_path():
+    inp = gen.scan_inputs(2, 40, 2, 64, "bf16", seed=710)
+    d = device_inputs(inp, DEV)
+    with pytest.raises(mss.MssError) as e:
+        mss.scan_fwd_save(**d)
+    assert e.value.code == mss.ERR_PATH
+    inp = gen.scan_inputs(2, 40, 16, 64, "bf16", seed=711)
+    d = device_inputs(inp, DEV)
+    with pytest.raises(mss.MssError) as e:
+        mss.scan_fwd_save(**d, flags=mss.FLAG_SIMPLE)
+    assert e.value.code == mss.ERR_PATH
