@@ -107,6 +107,11 @@ enum mss_status {
  * the states that mss_scan_fwd_save wrote for the same inputs, so the call
  * skips its checkpoint pass.  See mss_scan_fwd_save. */
 #define MSS_FLAG_SAVED_STATES 0x20u
+/* Forward passes: run the two-lanes-per-channel kernel where the four-lane
+ * one would (fp32 io, N = 8 or 16, one pass over the sequence, Euler input
+ * rule, no convolution); for testing and measurement, the results agree
+ * within the io type's rounding. */
+#define MSS_FLAG_PAIR_LANES 0x40u
 
 /*
  * mss_scan_fwd -- selective-scan forward pass over whole sequences.

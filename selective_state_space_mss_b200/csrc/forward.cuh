@@ -16,6 +16,7 @@
 #include "host_common.h"
 #include "launch.h"
 #include "scan_seq.cuh"
+#include "scan_seq4.cuh"
 #include "scan_simple.cuh"
 
 namespace mss_host {
@@ -158,6 +159,28 @@ int launch_seq_conv(const mss::SeqMaps& maps, const mss::ScanParams& p, unsigned
                  : launch_seq_passes<T, N, false, kConv>(maps, p, flags, stream);
 }
 
+// The four-lane kernel (one pass, Euler input rule, no convolution, no
+// checkpoints).
+template <typename T, int N, bool kGate, bool kSoftplus>
+int launch_seq4_variant(const mss::SeqMaps& maps, const mss::ScanParams& p, unsigned flags, cudaStream_t stream) {
+    using Ly = mss::Seq4Layout<T, N>;
+    auto kern = mss::scan_fwd_seq4_kernel<T, N, kGate, kSoftplus>;
+    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, Ly::kSmemBytes) != cudaSuccess)
+        return MSS_ERR_CUDA;
+    const dim3 grid(unsigned((p.dim + Ly::kRows - 1) / Ly::kRows), unsigned(p.batch), 1u);
+    kern<<<grid, Ly::kThreads, Ly::kSmemBytes, stream>>>(maps, p, (flags & MSS_FLAG_GENERAL_A) ? 0 : 1);
+    return launch_status();
+}
+
+template <typename T, int N>
+int launch_seq4(const mss::SeqMaps& maps, const mss::ScanParams& p, unsigned flags, cudaStream_t stream) {
+    if (p.z)
+        return p.softplus ? launch_seq4_variant<T, N, true, true>(maps, p, flags, stream)
+                          : launch_seq4_variant<T, N, true, false>(maps, p, flags, stream);
+    return p.softplus ? launch_seq4_variant<T, N, false, true>(maps, p, flags, stream)
+                      : launch_seq4_variant<T, N, false, false>(maps, p, flags, stream);
+}
+
 template <typename T, int N>
 int launch_seq(mss::ScanParams p, unsigned flags, void* workspace, int64_t workspace_bytes, cudaStream_t stream) {
     constexpr int esz = int(sizeof(T));
@@ -180,6 +203,15 @@ int launch_seq(mss::ScanParams p, unsigned flags, void* workspace, int64_t works
             p.seg_len = seg_len_for<T, N>(p.seqlen, n_seg);
             p.agg = static_cast<float*>(workspace);
         }
+    }
+    if constexpr (sizeof(T) == 4 && (N == 8 || N == 16)) {
+        // fp32 io, one pass without the convolution, the zero-order hold or
+        // stored states: four lanes per channel, twice the warps of the pair
+        // kernel (for bf16 io its extra shuffles and selects cost more than
+        // the warps recover, so bf16 keeps the pair kernel)
+        if (p.n_seg == 1 && p.conv_width == 0 && !p.zoh && !p.ckpt && !p.selftest_wait_ns &&
+            !(flags & MSS_FLAG_PAIR_LANES))
+            return launch_seq4<T, N>(maps, p, flags, stream);
     }
     return p.conv_width > 0 ? launch_seq_conv<T, N, true>(maps, p, flags, stream)
                             : launch_seq_conv<T, N, false>(maps, p, flags, stream);

@@ -20,7 +20,8 @@ using mss::bf16_t;
 using namespace mss_host;
 
 constexpr unsigned kScanFlags =
-    MSS_FLAG_GENERAL_A | MSS_FLAG_SIMPLE | MSS_FLAG_NO_SPLIT | MSS_FLAG_ZOH_INPUT | MSS_FLAG_SELFTEST_TIMEOUT;
+    MSS_FLAG_GENERAL_A | MSS_FLAG_SIMPLE | MSS_FLAG_NO_SPLIT | MSS_FLAG_ZOH_INPUT | MSS_FLAG_SELFTEST_TIMEOUT |
+    MSS_FLAG_PAIR_LANES;
 constexpr unsigned kBwdFlags = MSS_FLAG_GENERAL_A | MSS_FLAG_SIMPLE | MSS_FLAG_ZOH_INPUT | MSS_FLAG_SAVED_STATES;
 
 // The device error word (one per device, in the library image): kernels

@@ -152,7 +152,7 @@ def test_ex2_and_workspace_argument_errors(lib):
                                     None, 1, w(a["h0"]), w(a["y"]), w(a["last"]), a["batch"], a["dim"],
                                     a["N"], a["L"], a["dtype"], a["flags"], w(a["ws"]), a["wsb"], None)
 
-    assert ex2(flags=0x40) == codes["MSS_ERR_FLAGS"]
+    assert ex2(flags=0x80) == codes["MSS_ERR_FLAGS"]
     assert ex2(wsb=-1) == codes["MSS_ERR_SHAPE"]
     assert ex2(h0=P + 0x6000002) == codes["MSS_ERR_ALIGN"]
     assert ex2(ws=P + 0x6000001, wsb=64) == codes["MSS_ERR_ALIGN"]
@@ -307,7 +307,7 @@ def test_saved_states_argument_errors(lib):
     assert save(N=2, stb=1 << 20) == codes["MSS_ERR_PATH"]
     assert save(u=P + 2) == codes["MSS_ERR_PATH"]                   # rows not 16-byte aligned
     assert save(L=33, stb=1 << 20) == codes["MSS_ERR_PATH"]          # odd rows
-    assert save(flags=0x40) == codes["MSS_ERR_FLAGS"]
+    assert save(flags=0x80) == codes["MSS_ERR_FLAGS"]
     assert save(batch=0) == 0
     assert save(L=0, st=None, stb=0) == 0
 
