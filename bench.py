@@ -44,7 +44,8 @@ FALLBACK_HBM_GBS = 6650.0
 # the files the timed forward kernel (and its launch) is built from: the
 # recorded DRAM traffic is reported only while they are unchanged
 KERNEL_SOURCES = ["selective_state_space_mss_b200/csrc/" + f for f in (
-    "scan_seq.cuh", "tma.cuh", "mss_device.cuh", "mss_params.h", "forward.cuh", "fwd_bf16_n16.cu")]
+    "scan_seq.cuh", "scan_seq4.cuh", "tma.cuh", "mss_device.cuh", "mss_params.h", "host_common.h", "forward.cuh",
+    "fwd_bf16_n16.cu")]
 
 
 def log(*a):
@@ -75,6 +76,17 @@ def fwd_alu_ops(batch, dim, N, L):
     term, update, read-out), per token ten more (bias add, softplus, Delta*u,
     Delta*A_0, skip, read-out sum, gate)."""
     return batch * dim * L * (4 * N + 10)
+
+
+def bwd_alu_ops(batch, dim, N, L, checkpoint_pass=True):
+    """Algorithmic fp32 lane operations of one backward call (Euler rule): per
+    token and state, three to form the state again (transition, input term,
+    update) and nine for the reverse step (g = gh + dr C, gh' = g Abar,
+    q = gh' h_prev, dA += Delta q, the sums of q A and g B, the dB and dC terms,
+    the read-out C h for dz); three more per token and state when the call
+    also runs its checkpoint pass (the forward fold); per token twenty (the
+    step, its slope, the gate and its slope, the per-token gradients)."""
+    return batch * dim * L * ((15 if checkpoint_pass else 12) * N + 20)
 
 
 # B200: 148 SMs x 128 fp32 lanes per SM and clock, at the maximum SM clock.
@@ -867,11 +879,15 @@ def run_mss(args, rank, world, local_rank):
         "backward": {"ms_avg": bwd_avg, "channel_tokens_per_s": w.batch * w.dim * w.seqlen / (bwd_avg * 1e-3),
                      "achieved_gbs": bytes_bwd / (bwd_avg * 1e-3) / 1e9,
                      "frac": bytes_bwd / (bwd_avg * 1e-3) / 1e9 / peak,
+                     "alu_ops": bwd_alu_ops(w.batch, w.dim, w.dstate, w.seqlen),
+                     "alu_frac": bwd_alu_ops(w.batch, w.dim, w.dstate, w.seqlen) / (bwd_avg * 1e-3) / alu_peak,
                      "note": "gradients of u, delta, A, B, C, D, z, bias, starting state; checkpoint pass included"},
         "training_step": {"fwd_save_ms_avg": sum(fwd_save_ms) / len(fwd_save_ms),
                           "bwd_saved_ms_avg": sum(bwd_saved_ms) / len(bwd_saved_ms),
                           "step_ms": sum(fwd_save_ms) / len(fwd_save_ms) + sum(bwd_saved_ms) / len(bwd_saved_ms),
                           "recompute_step_ms": fwd_avg + bwd_avg,
+                          "bwd_saved_alu_frac": bwd_alu_ops(w.batch, w.dim, w.dstate, w.seqlen, False)
+                          / (sum(bwd_saved_ms) / len(bwd_saved_ms) * 1e-3) / alu_peak,
                           "states_bytes": int(ws_b.numel()),
                           "note": "mss_scan_fwd_save (the forward pass also storing the state at every 8-token "
                                   "group) then mss_scan_bwd with MSS_FLAG_SAVED_STATES; recompute_step_ms: "
