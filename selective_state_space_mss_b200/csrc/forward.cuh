@@ -74,10 +74,10 @@ int launch_simple(const mss::ScanParams& p, cudaStream_t stream) {
     return launch_status();
 }
 
-template <typename T, int N, bool kGate, bool kSoftplus, bool kFold, bool kZoh, bool kConv>
+template <typename T, int N, bool kGate, bool kSoftplus, bool kFold, bool kZoh, bool kConv, bool kSave = false>
 int launch_seq_variant(const mss::SeqMaps& maps, const mss::ScanParams& p, unsigned flags, int segs,
                        cudaStream_t stream) {
-    auto kern = mss::scan_fwd_seq_kernel<T, N, kGate, kSoftplus, kFold, kZoh, kConv>;
+    auto kern = mss::scan_fwd_seq_kernel<T, N, kGate, kSoftplus, kFold, kZoh, kConv, kSave>;
     const int smem = mss::SeqLayout<T, N>::kSmemBytes;
     if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess)
         return MSS_ERR_CUDA;
@@ -143,6 +143,18 @@ int launch_seq_passes(const mss::SeqMaps& maps, const mss::ScanParams& p, unsign
                            ? launch_seq_variant<T, N, false, true, true, kZoh, kConv>(maps, pf, flags, p.n_seg - 1, stream)
                            : launch_seq_variant<T, N, false, false, true, kZoh, kConv>(maps, pf, flags, p.n_seg - 1, stream);
         if (rc != MSS_OK) return rc;
+    }
+    if constexpr (!kConv) {
+        // the full pass that also stores the states (mss_scan_fwd_save)
+        if (p.ckpt) {
+            if (p.z)
+                return p.softplus
+                           ? launch_seq_variant<T, N, true, true, false, kZoh, false, true>(maps, p, flags, p.n_seg, stream)
+                           : launch_seq_variant<T, N, true, false, false, kZoh, false, true>(maps, p, flags, p.n_seg, stream);
+            return p.softplus
+                       ? launch_seq_variant<T, N, false, true, false, kZoh, false, true>(maps, p, flags, p.n_seg, stream)
+                       : launch_seq_variant<T, N, false, false, false, kZoh, false, true>(maps, p, flags, p.n_seg, stream);
+        }
     }
     if (p.z)
         return p.softplus ? launch_seq_variant<T, N, true, true, false, kZoh, kConv>(maps, p, flags, p.n_seg, stream)

@@ -317,8 +317,11 @@ __device__ __forceinline__ uint2 pack8(const float (&v)[8 / sizeof(T)]) {
 // the final state); otherwise the full pass, starting from the caller's state
 // carried over the earlier segments' aggregates.  A fold with p.ckpt set is
 // the backward pass's checkpoint pass instead: one segment from the caller's
-// state, recording the state at the start of every group of V tokens.
-template <typename T, int N, bool kGeo, bool kGate, bool kSoftplus, bool kFold, bool kZoh, bool kConv>
+// state, recording the state at the start of every group of V tokens.  kSave:
+// a full pass that records those states as well (mss_scan_fwd_save); a
+// separate variant, so that the plain full pass carries no code for it.
+template <typename T, int N, bool kGeo, bool kGate, bool kSoftplus, bool kFold, bool kZoh, bool kConv,
+          bool kSave = false>
 __device__ __forceinline__ void scan_seq_body(const SeqMaps& maps, const ScanParams& p, uint8_t* smem,
                                               uint64_t* bars, const LaneConst<N>& cc, bool valid, int64_t row) {
     using Ly = SeqLayout<T, N>;
@@ -515,7 +518,9 @@ __device__ __forceinline__ void scan_seq_body(const SeqMaps& maps, const ScanPar
     for (int g = 0; g < n_groups; ++g) {
         const int c = g / GPC, j = g % GPC;
         const bool has_next = g + 1 < n_groups;
-        if (p.ckpt) store_ckpt(g);
+        if constexpr (kFold || kSave) {
+            if (p.ckpt) store_ckpt(g);
+        }
         // the next group's u/delta/z, first: its stage must have landed when it opens a new chunk
         if (has_next && j == GPC - 1 && !wait_chunk(c + 1)) return;
         float uv[HV], dv[HV], zv[HV];
@@ -664,7 +669,7 @@ __device__ __forceinline__ void scan_seq_body(const SeqMaps& maps, const ScanPar
 // 0 .. n_seg-2, the full pass all n_seg (after the fold has completed).
 // Requirements checked by the host: N in {4, 8, 16}; L * sizeof(T) a multiple
 // of 16; u, delta, z, B, C, y 16-byte aligned; seg_len a multiple of the chunk.
-template <typename T, int N, bool kGate, bool kSoftplus, bool kFold, bool kZoh, bool kConv>
+template <typename T, int N, bool kGate, bool kSoftplus, bool kFold, bool kZoh, bool kConv, bool kSave = false>
 __global__ void __launch_bounds__(32) scan_fwd_seq_kernel(const __grid_constant__ SeqMaps maps, ScanParams p,
                                                           int allow_geo) {
     using Ly = SeqLayout<T, N>;
@@ -723,11 +728,11 @@ __global__ void __launch_bounds__(32) scan_fwd_seq_kernel(const __grid_constant_
 
     if constexpr (kFast) {
         if (geo) {
-            scan_seq_body<T, N, true, kGate, kSoftplus, kFold, kZoh, kConv>(maps, p, smem, bars, cc, valid, row);
+            scan_seq_body<T, N, true, kGate, kSoftplus, kFold, kZoh, kConv, kSave>(maps, p, smem, bars, cc, valid, row);
             return;
         }
     }
-    scan_seq_body<T, N, false, kGate, kSoftplus, kFold, kZoh, kConv>(maps, p, smem, bars, cc, valid, row);
+    scan_seq_body<T, N, false, kGate, kSoftplus, kFold, kZoh, kConv, kSave>(maps, p, smem, bars, cc, valid, row);
 }
 
 }  // namespace mss

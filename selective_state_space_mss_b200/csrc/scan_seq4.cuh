@@ -32,11 +32,13 @@
 //
 // Scope: fp32 io, the Euler input rule, no sequence split, no convolution,
 // no checkpoints, no wait self-test; the host sends everything else to the
-// two-lane kernel.  Measured on the 4 x 4096-channel layer: fp32 io at
-// L = 2048 takes 480 us against 517 us for the pair kernel; bf16 io at
-// L = 4096 took 466 us against 375 us, its per-token shuffles of Delta*u and
-// r, the lane-dependent power selects and the second reduce stage adding 38%
-// instructions that the doubled warps (3.3 per scheduler) do not recover.
+// two-lane kernel.  Measured with fp32 io: 340 us against 371 us for the
+// pair kernel on 4 x 4096 channels at N = 8 (L = 2048), 199 us against 246 us
+// on 8 x 1536 channels at N = 16 (L = 1024), about even on 4 x 4096 at N = 16.
+// With bf16 io it took 466 us against 375 us (L = 4096): its per-token
+// shuffles of Delta*u and r, the lane-dependent power selects and the second
+// reduce stage add 38% instructions that the doubled warps (3.3 per
+// scheduler) do not recover.
 #pragma once
 
 #include <cstdint>
