@@ -65,8 +65,6 @@ int launch_ssd_tc(const mss::SsdParams& p, cudaStream_t s) {
     mss::SsdTcMaps maps;
     std::memset(&maps, 0, sizeof(maps));
     if (!encode_token_major(&maps.x, p.x, p.batch, p.seqlen, p.nheads, 64) ||
-        !encode_token_major(&maps.y, p.y, p.batch, p.seqlen, p.nheads, 64) ||
-        (p.z && !encode_token_major(&maps.z, p.z, p.batch, p.seqlen, p.nheads, 64)) ||
         !encode_token_major(&maps.B, p.B, p.batch, p.seqlen, p.ngroups, 128) ||
         !encode_token_major(&maps.C, p.C, p.batch, p.seqlen, p.ngroups, 128))
         return MSS_ERR_CUDA;

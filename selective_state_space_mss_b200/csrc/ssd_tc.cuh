@@ -17,7 +17,7 @@
 //   M   = mask(G) . exp(cs_i - cs_j) Delta_j on the CUDA cores, bf16 in smem
 //   Ym  = M X                     (128 x 64, K = Q)      columns 128..191
 //   S   = exp(cs_last) S_prev + dS        (fp32, registers)
-//   y   = (Ym + exp(cs_i) Yx + D x) silu(z)  -> smem -> TMA store
+//   y   = (Ym + exp(cs_i) Yx + D x) silu(z)  -> stored from registers
 //
 // Thread t of the CTA owns TMEM lane (and row) t % 128 and quarter t / 128 of
 // the columns of each product it reads (four warps share each 32-lane TMEM
@@ -37,7 +37,10 @@
 // M X starts, then the next chunk's C B^T, while another lightly loaded warp
 // prepares the next chunk's step sizes and decay sums (their raw steps were
 // loaded a chunk ahead); the state update waits only for B^T X_w, the output
-// only for M X (barrier); then the y store and the loads of chunk c + 2.  Each thread
+// only for M X, and y goes straight from registers to memory (barrier); then
+// the loads of chunk c + 2.  z is loaded after the first barrier: a proxy
+// fence waits for a thread's loads in flight, so z loaded before the scaling
+// of X held that fence for the loads' whole latency.  Each thread
 // waits on the MMA completion barriers itself; a wait that gives up is
 // folded into the next CTA barrier.  Score blocks of 32 x 32 wholly above
 // the diagonal are skipped by the warp; blocks wholly below it use
@@ -63,7 +66,7 @@
 namespace mss {
 
 struct SsdTcMaps {
-    CUtensorMap x, z, y, B, C;  // x, y: [batch][L][H][64]; B, C: [batch][L][G][128] (4-D views)
+    CUtensorMap x, B, C;  // x: [batch][L][H][64]; B, C: [batch][L][G][128] (4-D views)
 };
 
 struct SsdTcLayout {
@@ -73,7 +76,7 @@ struct SsdTcLayout {
     // stage: C (two boxes along N), B (two boxes), X
     static constexpr int kC = 0, kB = 2 * kBox, kX = 4 * kBox;
     static constexpr int kStageBytes = 5 * kBox;
-    static constexpr int kM = 2 * kStageBytes;    // masked scores, bf16, two boxes along K; then y's tile
+    static constexpr int kM = 2 * kStageBytes;    // masked scores, bf16, two boxes along K
     static constexpr int kXw = kM + 2 * kBox;     // w-scaled X
     static constexpr int kS = kXw + kBox;         // bf16 copy of the state [128 n][64 p]
     // per token of the chunk: Delta, cs in log2 units, and the column factor
@@ -127,8 +130,6 @@ __global__ void __launch_bounds__(512, 1) ssd_tc_kernel(const __grid_constant__ 
         prefetch_tensormap(&maps.x);
         prefetch_tensormap(&maps.B);
         prefetch_tensormap(&maps.C);
-        prefetch_tensormap(&maps.y);
-        if (kGate) prefetch_tensormap(&maps.z);
     }
     if (warp == 0) {
         tmem_alloc(tslot, Ly::kTmemCols);
@@ -254,15 +255,6 @@ __global__ void __launch_bounds__(512, 1) ssd_tc_kernel(const __grid_constant__ 
         const uint32_t st = sbase + uint32_t((c & 1) * Ly::kStageBytes);
         const float* dtc = dts;
         const float* csc = css;
-        // z of this chunk's rows, in registers until the output step
-        uint4 zr[2];
-        if constexpr (kGate) {
-            const int64_t tok = t0 + row;
-            const bf16_t* zp = static_cast<const bf16_t*>(p.z) + ((b * L + tok) * H + h) * P + 16 * qd;
-#pragma unroll
-            for (int q = 0; q < 2; ++q)
-                zr[q] = tok < L ? *reinterpret_cast<const uint4*>(zp + 8 * q) : make_uint4(0u, 0u, 0u, 0u);
-        }
         abort |= !mbar_wait_bounded(full + (c & 1), uint32_t((c >> 1) & 1), p.err);
         const float cl = csc[Q - 1];
         const float ci = csc[row];  // kept for the output step (the next chunk's scan rewrites css)
@@ -283,12 +275,20 @@ __global__ void __launch_bounds__(512, 1) ssd_tc_kernel(const __grid_constant__ 
             }
         }
         fence_proxy_async_smem();
-        // the previous chunk's y store must have read its tile (the first box
-        // of the score tile, rewritten after this barrier)
-        if (ctl) bulk_wait_read<0>();
         if (__syncthreads_or(abort)) {
             ok = false;
             break;
+        }
+        // z of this chunk's rows, in registers until the output step; loaded
+        // only now, after the proxy fence above, which would otherwise wait
+        // for these loads to land
+        uint4 zr[2] = {make_uint4(0u, 0u, 0u, 0u), make_uint4(0u, 0u, 0u, 0u)};
+        const int64_t tok = int64_t(t0) + row;
+        if constexpr (kGate) {
+            const bf16_t* zp = static_cast<const bf16_t*>(p.z) + ((b * L + tok) * H + h) * P + 16 * qd;
+#pragma unroll
+            for (int q = 0; q < 2; ++q)
+                if (tok < L) zr[q] = *reinterpret_cast<const uint4*>(zp + 8 * q);
         }
         // dS = B^T X_w and Yx = C S_prev, while the scores are masked
         if (ctl) {
@@ -405,8 +405,8 @@ __global__ void __launch_bounds__(512, 1) ssd_tc_kernel(const __grid_constant__ 
         abort |= !mbar_wait_bounded(ybar, ph, p.err);
         tc_fence_after_sync();
         // y = (Ym + exp(cs_i) Yx + D x) silu(z) for row i = `row`, this
-        // quarter's 16 columns, staged in the score tile's first box (M X has
-        // read it) for the store
+        // quarter's 16 columns: 32 contiguous bytes of the token's row, stored
+        // from registers
         {
             float ym[16], yx[16];
             tmem_ld16(tlane + Ly::kColYm + uint32_t(16 * qd), ym);
@@ -414,7 +414,7 @@ __global__ void __launch_bounds__(512, 1) ssd_tc_kernel(const __grid_constant__ 
             tmem_wait_ld();
             const float ei = ex2_approx(ci);
             const uint8_t* xs = smem + (c & 1) * Ly::kStageBytes + Ly::kX;
-            uint8_t* ys = smem + Ly::kM;
+            bf16_t* yp = static_cast<bf16_t*>(p.y) + ((b * L + tok) * H + h) * P + 16 * qd;
 #pragma unroll
             for (int q = 0; q < 2; ++q) {
                 const uint32_t off = sw128(row, 2 * qd + q);
@@ -439,19 +439,18 @@ __global__ void __launch_bounds__(512, 1) ssd_tc_kernel(const __grid_constant__ 
                     }
                     o4[k] = pack_bf16x2(y0, y1);
                 }
-                *reinterpret_cast<uint4*>(ys + off) = make_uint4(o4[0], o4[1], o4[2], o4[3]);
+                if (tok < L) *reinterpret_cast<uint4*>(yp + 8 * q) = make_uint4(o4[0], o4[1], o4[2], o4[3]);
             }
         }
         tc_fence_before_sync();
-        fence_proxy_async_smem();
         if (__syncthreads_or(abort)) {
             ok = false;
             break;
         }
-        if (ctl) {
-            tma_store_4d(&maps.y, smem + Ly::kM, 0, int(h), t0, int(b));
-            bulk_commit();
-            if (c + 2 < n_chunks) issue_chunk(c + 2);
+        // every read of chunk c's stage is done: its tiles give way to chunk c + 2
+        if (ctl && c + 2 < n_chunks) {
+            fence_proxy_async_smem();
+            issue_chunk(c + 2);
         }
     }
     if (!ok && ctl) {
@@ -461,7 +460,6 @@ __global__ void __launch_bounds__(512, 1) ssd_tc_kernel(const __grid_constant__ 
             mbar_wait_bounded(full + k, 1u, nullptr, 50000000ull);
         }
     }
-    if (ctl) bulk_wait<0>();
     if (ok && p.last_state) {
         float* ls = p.last_state + ((b * H + h) * NS + row) * P + 16 * qd;
 #pragma unroll
