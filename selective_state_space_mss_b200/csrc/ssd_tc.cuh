@@ -35,9 +35,10 @@
 // (barrier); B^T X_w and C S_prev start, and the threads mask and decay the
 // scores, whose C B^T ran during the previous chunk's output step (barrier);
 // M X starts, then the next chunk's C B^T, while another lightly loaded warp
-// prepares the next chunk's step sizes and decay sums (their raw steps were
-// loaded a chunk ahead); the state update waits only for B^T X_w, the output
-// only for M X, and y goes straight from registers to memory (barrier); then
+// stores the next chunk's step sizes and decay sums (formed during the
+// masking, in which its scores are all masked; their raw steps were loaded a
+// chunk ahead); the state update waits only for B^T X_w, the output only for
+// M X, and y goes straight from registers to memory (barrier); then
 // the loads of chunk c + 2.  z is loaded after the first barrier: a proxy
 // fence waits for a thread's loads in flight, so z loaded before the scaling
 // of X held that fence for the loads' whole latency.  Each thread
@@ -196,8 +197,12 @@ __global__ void __launch_bounds__(512, 1) ssd_tc_kernel(const __grid_constant__ 
             raw[k] = t < L ? ld(dtp + t * H) : 0.f;
         }
     };
-    auto scan_chunk = [&](int c) {
-        float d[4], a[4], run = 0.f;
+    // scan_compute forms the values into registers, scan_store writes them
+    float sd[4], sa[4], sf[4];
+    auto scan_compute = [&](int c) {
+        float* d = sd;
+        float* a = sa;
+        float run = 0.f;
 #pragma unroll
         for (int k = 0; k < 4; ++k) {
             const bool valid = int64_t(c) * Q + 4 * lane + k < L;
@@ -217,15 +222,18 @@ __global__ void __launch_bounds__(512, 1) ssd_tc_kernel(const __grid_constant__ 
         for (int k = 0; k < 4; ++k) a[k] += excl;
         // the last token of this lane's 32-token block is token 3 of lane 8 (l / 8) + 7
         const float cL = __shfl_sync(0xffffffffu, a[3], (lane & ~7) | 7);
-        reinterpret_cast<float4*>(dts)[lane] = make_float4(d[0], d[1], d[2], d[3]);
-        reinterpret_cast<float4*>(css)[lane] = make_float4(a[0], a[1], a[2], a[3]);
-        reinterpret_cast<float4*>(fss)[lane] =
-            make_float4(ex2_approx(cL - a[0]) * d[0], ex2_approx(cL - a[1]) * d[1], ex2_approx(cL - a[2]) * d[2],
-                        ex2_approx(cL - a[3]) * d[3]);
+#pragma unroll
+        for (int k = 0; k < 4; ++k) sf[k] = ex2_approx(cL - a[k]) * d[k];
+    };
+    auto scan_store = [&]() {
+        reinterpret_cast<float4*>(dts)[lane] = make_float4(sd[0], sd[1], sd[2], sd[3]);
+        reinterpret_cast<float4*>(css)[lane] = make_float4(sa[0], sa[1], sa[2], sa[3]);
+        reinterpret_cast<float4*>(fss)[lane] = make_float4(sf[0], sf[1], sf[2], sf[3]);
     };
     if (warp == kScanWarp) {
         load_raw(0);
-        scan_chunk(0);
+        scan_compute(0);
+        scan_store();
         if (n_chunks > 1) load_raw(1);
     }
     __syncthreads();
@@ -363,13 +371,17 @@ __global__ void __launch_bounds__(512, 1) ssd_tc_kernel(const __grid_constant__ 
                 }
             }
         }
+        // the scan warp, whose scores are all masked, forms the next chunk's
+        // step sizes and decay sums now (stored once every warp has read
+        // this chunk's, after the barrier)
+        if (warp == kScanWarp && c + 1 < n_chunks) scan_compute(c + 1);
         tc_fence_before_sync();
         fence_proxy_async_smem();
         if (__syncthreads_or(abort)) {
             ok = false;
             break;
         }
-        // Ym = M X; meanwhile the scan warp prepares the next chunk's step sizes
+        // Ym = M X; meanwhile the scan warp stores the next chunk's step sizes
         if (ctl) {
             tc_fence_after_sync();
 #pragma unroll
@@ -385,8 +397,7 @@ __global__ void __launch_bounds__(512, 1) ssd_tc_kernel(const __grid_constant__ 
             if (c + 1 < n_chunks) abort |= !issue_scores(c + 1);
         }
         if (warp == kScanWarp && c + 1 < n_chunks) {
-            __syncwarp();
-            scan_chunk(c + 1);
+            scan_store();
             if (c + 2 < n_chunks) load_raw(c + 2);
         }
         // the state: S = exp(cs_last) S + dS, and its bf16 copy for the next
