@@ -661,42 +661,47 @@ def run_mss(args, rank, world, local_rank):
         workloads[name] = time_workload(mss, name, args, dev, stream, rank)
         assert mss.get_device_error() == 0
 
-    # the structured-state-space-duality (Mamba-2) layer: its own workload
-    ss = gen.SSD_SHAPES[gen.SSD_WORKLOAD]
-    sin = gen.ssd_inputs(**ss)
-    sd = dict(x=to_dev(sin["x"]), dt=to_dev(sin["dt"]), A=torch.from_numpy(sin["A"]).to(dev),
-              B=to_dev(sin["B"]), C=to_dev(sin["C"]), D=torch.from_numpy(sin["D"]).to(dev), z=to_dev(sin["z"]),
-              dt_bias=torch.from_numpy(sin["dt_bias"]).to(dev))
-    ssd_y = torch.empty_like(sd["x"])
-    ssd_last = torch.empty(ss["batch"], ss["nheads"], ss["dstate"], ss["headdim"], device=dev)
+    # the structured-state-space-duality (Mamba-2) layer: its own workloads,
+    # each on the tcgen05 kernel and, for comparison, the warp-level one
+    def time_ssd(name):
+        ss = gen.SSD_SHAPES[name]
+        sin = gen.ssd_inputs(**ss)
+        sd = dict(x=to_dev(sin["x"]), dt=to_dev(sin["dt"]), A=torch.from_numpy(sin["A"]).to(dev),
+                  B=to_dev(sin["B"]), C=to_dev(sin["C"]), D=torch.from_numpy(sin["D"]).to(dev),
+                  z=to_dev(sin["z"]), dt_bias=torch.from_numpy(sin["dt_bias"]).to(dev))
+        ssd_y = torch.empty_like(sd["x"])
+        ssd_last = torch.empty(ss["batch"], ss["nheads"], ss["dstate"], ss["headdim"], device=dev)
 
-    def time_ssd(flags):
-        ev = []
-        for i in range(args.warmup + args.steps):
-            a_, b_ = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-            a_.record(stream)
-            mss.ssd_fwd(**sd, y=ssd_y, last_state=ssd_last, flags=flags)
-            b_.record(stream)
-            if i >= args.warmup:
-                ev.append((a_, b_))
-        torch.cuda.synchronize(dev)
-        assert mss.get_device_error() == 0
-        return sum(a_.elapsed_time(b_) for a_, b_ in ev) / len(ev)
+        def one(flags):
+            ev = []
+            for i in range(args.warmup + args.steps):
+                a_, b_ = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+                a_.record(stream)
+                mss.ssd_fwd(**sd, y=ssd_y, last_state=ssd_last, flags=flags)
+                b_.record(stream)
+                if i >= args.warmup:
+                    ev.append((a_, b_))
+            torch.cuda.synchronize(dev)
+            assert mss.get_device_error() == 0
+            return sum(a_.elapsed_time(b_) for a_, b_ in ev) / len(ev)
 
-    ssd_ms = time_ssd(0)  # the tcgen05 kernel
-    ssd_ms_warp = time_ssd(mss.SSD_FLAG_WARP_MMA)  # the warp-level (mma.sync) kernel, for comparison
-    del sd, ssd_y, sin
-    # matrix-form flops per (token, head) of the tcgen05 kernel's chunks of
-    # 128 tokens: C B^T and M X within the chunk, C S and the state product
-    # B^T X across chunks (P = 64)
-    # algorithmic bytes: x, z read and y written (bf16), dt read, B and C read
-    # once per (batch, token, group), A, D, dt_bias, and last_state written
-    ssd_bytes = (3 * ss["batch"] * ss["seqlen"] * ss["nheads"] * ss["headdim"] * 2
-                 + ss["batch"] * ss["seqlen"] * ss["nheads"] * 2
-                 + 2 * ss["batch"] * ss["seqlen"] * ss["ngroups"] * ss["dstate"] * 2
-                 + 3 * ss["nheads"] * 4 + ss["batch"] * ss["nheads"] * ss["dstate"] * ss["headdim"] * 4)
-    ssd_flops = ss["batch"] * ss["seqlen"] * ss["nheads"] * (
-        2 * 128 * ss["dstate"] + 2 * 128 * ss["headdim"] + 2 * ss["dstate"] * ss["headdim"] * 2)
+        ms_tc = one(0)  # the tcgen05 kernel
+        ms_warp = one(mss.SSD_FLAG_WARP_MMA)  # the warp-level (mma.sync) kernel
+        # algorithmic bytes: x, z read and y written (bf16), dt read, B and C
+        # read once per (batch, token, group), A, D, dt_bias, and last_state
+        # written; matrix-form flops per (token, head) of chunks of 128
+        # tokens: C B^T and M X within the chunk, C S and the state product
+        # B^T X across chunks
+        nbytes = (3 * ss["batch"] * ss["seqlen"] * ss["nheads"] * ss["headdim"] * 2
+                  + ss["batch"] * ss["seqlen"] * ss["nheads"] * 2
+                  + 2 * ss["batch"] * ss["seqlen"] * ss["ngroups"] * ss["dstate"] * 2
+                  + 3 * ss["nheads"] * 4 + ss["batch"] * ss["nheads"] * ss["dstate"] * ss["headdim"] * 4)
+        flops = ss["batch"] * ss["seqlen"] * ss["nheads"] * (
+            2 * 128 * ss["dstate"] + 2 * 128 * ss["headdim"] + 2 * ss["dstate"] * ss["headdim"] * 2)
+        return ss, ms_tc, ms_warp, nbytes, flops
+
+    ss, ssd_ms, ssd_ms_warp, ssd_bytes, ssd_flops = time_ssd(gen.SSD_WORKLOAD)
+    ss2, ssd2_ms, ssd2_ms_warp, ssd2_bytes, ssd2_flops = time_ssd(gen.SSD_WORKLOAD_2)
 
     # the backward pass (gradients of every input, states recomputed from
     # checkpoints) on the same workload
@@ -910,7 +915,15 @@ def run_mss(args, rank, world, local_rank):
                      "warp_mma_kernel": {"ms_avg": ssd_ms_warp,
                                          "achieved_gbs": ssd_bytes / (ssd_ms_warp * 1e-3) / 1e9,
                                          "note": "the warp-level mma.sync kernel (chunks of 64), "
-                                                 "MSS_SSD_FLAG_WARP_MMA"}},
+                                                 "MSS_SSD_FLAG_WARP_MMA"},
+                     "second_workload": {
+                         "workload": gen.SSD_WORKLOAD_2, "ms_avg": ssd2_ms, "warp_mma_ms_avg": ssd2_ms_warp,
+                         "channel_tokens_per_s": ss2["batch"] * ss2["seqlen"] * ss2["nheads"] * ss2["headdim"]
+                         / (ssd2_ms * 1e-3),
+                         "hbm_frac": ssd2_bytes / (ssd2_ms * 1e-3) / 1e9 / peak,
+                         "tensor_frac": ssd2_flops / (ssd2_ms * 1e-3) / 1e12 / measured_bf16_tflops()[0],
+                         "algorithmic_bytes_per_launch": ssd2_bytes,
+                         "note": "160 (batch, head) CTAs: 1.08 waves of 148 SMs"}},
         "zoh_input_path": {"fwd_ms_avg": fwd_avg_zoh,
                            "achieved_gbs": bytes_fwd / (fwd_avg_zoh * 1e-3) / 1e9,
                            "frac": bytes_fwd / (fwd_avg_zoh * 1e-3) / 1e9 / peak,

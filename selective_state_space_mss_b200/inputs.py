@@ -220,7 +220,10 @@ def upstream_gradients(batch: int, dim: int, dstate: int, seqlen: int, dtype: st
 # The structured-state-space-duality (Mamba-2) layer: token-major tensors,
 # a scalar A per head, heads sharing B and C within a group.
 SSD_WORKLOAD = "mamba2-layer-bf16-b4-l4096-h64-p64-n128-g1"
-SSD_SHAPES = {SSD_WORKLOAD: dict(batch=4, seqlen=4096, nheads=64, headdim=64, ngroups=1, dstate=128, seed=1006)}
+# a second layer shape: 80 heads of 64 (d_inner 5120), two sequences
+SSD_WORKLOAD_2 = "mamba2-layer-bf16-b2-l4096-h80-p64-n128-g1"
+SSD_SHAPES = {SSD_WORKLOAD: dict(batch=4, seqlen=4096, nheads=64, headdim=64, ngroups=1, dstate=128, seed=1006),
+              SSD_WORKLOAD_2: dict(batch=2, seqlen=4096, nheads=80, headdim=64, ngroups=1, dstate=128, seed=1007)}
 
 
 def ssd_inputs(batch: int, seqlen: int, nheads: int, headdim: int, ngroups: int, dstate: int, seed: int,

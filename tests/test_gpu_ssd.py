@@ -160,3 +160,25 @@ def test_ssd_empty_sequence_passes_the_state_on():
     torch.cuda.synchronize()
     assert torch.equal(last, h0)
     assert torch.count_nonzero(last0) == 0
+
+
+@pytest.mark.parametrize("kernel", sorted(KERNELS))
+def test_ssd_second_workload_sampled_heads(kernel):
+    """The second bench workload (2 x 4096 tokens, 80 heads of 64, N = 128) on
+    each kernel: y and the final state of sampled (batch, head) pairs against
+    the oracle."""
+    s = dict(gen.SSD_SHAPES[gen.SSD_WORKLOAD_2])
+    inp = gen.ssd_inputs(**s)
+    y, last = mss.ssd_fwd(**_dev(inp), flags=KERNELS[kernel])
+    torch.cuda.synchronize()
+    assert mss.get_device_error() == 0
+    yn, ln = to_numpy(y), to_numpy(last)
+    rng = np.random.default_rng(741)
+    for _ in range(4):
+        b, h = int(rng.integers(s["batch"])), int(rng.integers(s["nheads"]))
+        sub = {k: inp[k].values[b:b + 1, :, h:h + 1] for k in ("x", "z", "dt")}
+        y_ref, last_ref = oracle.ssd_fwd(sub["x"], sub["dt"], inp["A"][h:h + 1], inp["B"].values[b:b + 1],
+                                         inp["C"].values[b:b + 1], D=inp["D"][h:h + 1], z=sub["z"],
+                                         dt_bias=inp["dt_bias"][h:h + 1])
+        assert_close(yn[b:b + 1, :, h:h + 1], y_ref, "bf16", f"y of (b={b}, h={h})")
+        assert_close(ln[b:b + 1, h:h + 1], last_ref, "bf16", f"state of (b={b}, h={h})")
