@@ -73,7 +73,7 @@ def test_four_lane_outputs_stay_in_bounds(shape):
 
 def _kernels_launched(fn):
     from torch.profiler import ProfilerActivity, profile
-    with profile(activities=[ProfilerActivity.CUDA]) as prof:
+    with profile(activities=[ProfilerActivity.CUDA], acc_events=True) as prof:
         fn()
         torch.cuda.synchronize()
     return [e.name for e in prof.events() if e.device_type.name == "CUDA"]
