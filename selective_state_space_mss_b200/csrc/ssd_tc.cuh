@@ -80,10 +80,11 @@ struct SsdTcLayout {
     static constexpr int kM = 2 * kStageBytes;    // masked scores, bf16, two boxes along K
     static constexpr int kXw = kM + 2 * kBox;     // w-scaled X
     static constexpr int kS = kXw + kBox;         // bf16 copy of the state [128 n][64 p]
-    // per token of the chunk: Delta, cs in log2 units, and the column factor
-    // f_j = exp2(cs_L - cs_j) Delta_j of the masked scores (L the last token of
-    // j's 32-token block); read up to the masked scores, then rewritten for the
-    // next chunk (each thread keeps the values its output step needs)
+    // per token of the chunk: Delta (with softplus cs - log2(Delta)), cs in
+    // log2 units, and the column factor f_j = exp2(cs_L - cs_j) Delta_j of the
+    // masked scores (L the last token of j's 32-token block); read up to the
+    // masked scores, then rewritten for the next chunk (each thread keeps the
+    // values its output step needs)
     static constexpr int kScal = kS + kBox;
     static constexpr int kBars = kScal + 3 * kQ * 4;
     static constexpr int kTmemSlot = kBars + 5 * 8;
@@ -100,7 +101,8 @@ __global__ void __launch_bounds__(512, 1) ssd_tc_kernel(const __grid_constant__ 
     constexpr int Q = Ly::kQ, P = Ly::kP, NS = Ly::kN;
     extern __shared__ __align__(16) uint8_t smem_raw[];
     uint8_t* smem = smem_raw + ((1024u - (smem_addr(smem_raw) & 1023u)) & 1023u);
-    float* dts = reinterpret_cast<float*>(smem + Ly::kScal);  // [Q] Delta (0 past the sequence)
+    float* dts = reinterpret_cast<float*>(smem + Ly::kScal);  // [Q] Delta (0 past the sequence), or with
+                                                              // softplus cs - log2(Delta)
     float* css = dts + Q;                                     // [Q] cs * log2(e)
     float* fss = css + Q;                                     // [Q] column factors of the scores
     uint64_t* full = reinterpret_cast<uint64_t*>(smem + Ly::kBars);  // [2] TMA stages
@@ -226,6 +228,13 @@ __global__ void __launch_bounds__(512, 1) ssd_tc_kernel(const __grid_constant__ 
         for (int k = 0; k < 4; ++k) sf[k] = ex2_approx(cL - a[k]) * d[k];
     };
     auto scan_store = [&]() {
+        if constexpr (kSoftplus) {
+            // Delta > 0: the array holds cs_j - log2(Delta_j) instead (+inf
+            // where Delta_j is zero), so that exp2(x - it) = exp2(x - cs_j) Delta_j
+            // costs one exponential and no multiply
+#pragma unroll
+            for (int k = 0; k < 4; ++k) sd[k] = sa[k] - lg2_approx(sd[k]);
+        }
         reinterpret_cast<float4*>(dts)[lane] = make_float4(sd[0], sd[1], sd[2], sd[3]);
         reinterpret_cast<float4*>(css)[lane] = make_float4(sa[0], sa[1], sa[2], sa[3]);
         reinterpret_cast<float4*>(fss)[lane] = make_float4(sf[0], sf[1], sf[2], sf[3]);
@@ -268,7 +277,7 @@ __global__ void __launch_bounds__(512, 1) ssd_tc_kernel(const __grid_constant__ 
         const float ci = csc[row];  // kept for the output step (the next chunk's scan rewrites css)
         // X_w = w_j x_j (row j = `row`, this thread's quarter of the 64 columns)
         {
-            const float wj = ex2_approx(cl - ci) * dtc[row];
+            const float wj = kSoftplus ? ex2_approx(cl - dtc[row]) : ex2_approx(cl - ci) * dtc[row];
             const uint8_t* xs = smem + (c & 1) * Ly::kStageBytes + Ly::kX;
             uint8_t* xw = smem + Ly::kXw;
 #pragma unroll
@@ -361,7 +370,9 @@ __global__ void __launch_bounds__(512, 1) ssd_tc_kernel(const __grid_constant__ 
                             for (int e = 0; e < 2; ++e) {
                                 const int jj = 8 * q + 2 * k + e;  // 0..31 within this quarter
                                 const int j = 32 * qd + jj;        // token index in the chunk
-                                m2[e] = j <= row ? gv[jj] * ex2_approx(ci - csc[j]) * dtc[j] : 0.f;
+                                const float dec = kSoftplus ? ex2_approx(ci - dtc[j])
+                                                            : ex2_approx(ci - csc[j]) * dtc[j];
+                                m2[e] = j <= row ? gv[jj] * dec : 0.f;
                             }
                             o4[k] = pack_bf16x2(m2[0], m2[1]);
                         }
