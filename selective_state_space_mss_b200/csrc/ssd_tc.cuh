@@ -29,13 +29,15 @@
 // in the 128-byte swizzle TMA writes, double buffered (the next chunk's
 // loads run during this one); M, X_w and the state copy are written by the
 // threads in the same layout.  One thread issues the MMAs and the TMA copies,
-// from a warp whose scores are all masked (it has the least work).
+// from a warp whose scores are all masked (it has the least work); the score
+// products come from a thread of another such warp.
 //
 // Order within a chunk, with three CTA barriers: the threads scale X
 // (barrier); B^T X_w and C S_prev start, and the threads mask and decay the
 // scores, whose C B^T ran during the previous chunk's output step (barrier);
-// M X starts, then the next chunk's C B^T, while another lightly loaded warp
-// stores the next chunk's step sizes and decay sums (formed during the
+// M X starts (the next chunk's C B^T follows it, issued by a third lightly
+// loaded warp once M X is done), while another such warp stores the next
+// chunk's step sizes and decay sums (formed during the
 // masking, in which its scores are all masked; their raw steps were loaded a
 // chunk ahead); the state update waits only for B^T X_w, the output only for
 // M X, and y goes straight from registers to memory (barrier); then
@@ -117,8 +119,13 @@ __global__ void __launch_bounds__(512, 1) ssd_tc_kernel(const __grid_constant__ 
     // prepares the step sizes, sit in warps whose score blocks are all masked
     // (rows 0..31 against columns 96..127, rows 32..63 against 96..127), so
     // that their extra work does not hold up the CTA barriers.
-    constexpr int kCtlWarp = 12, kScanWarp = 13;
+    constexpr int kCtlWarp = 12, kScanWarp = 13, kScoreWarp = 8;
     const bool ctl = tid == kCtlWarp * 32;
+    // the thread that issues the score products C B^T (and commits their
+    // barrier), in a third all-masked warp: the next chunk's product waits
+    // for this chunk's M X to complete, and the waiting thread must not be the
+    // one that issues everything else
+    const bool scorer = tid == kScoreWarp * 32;
     const int64_t H = p.nheads, L = p.seqlen;
     const int64_t b = blockIdx.x / H, h = blockIdx.x % H;
     const int g = int(h / (H / p.ngroups));
@@ -265,7 +272,7 @@ __global__ void __launch_bounds__(512, 1) ssd_tc_kernel(const __grid_constant__ 
     bool abort = false;  // a bounded wait of this thread gave up (folded into the next CTA barrier)
     // the first chunk's scores; each later chunk's start during the previous
     // chunk's output step
-    if (ctl && n_chunks > 0) abort |= !issue_scores(0);
+    if (scorer && n_chunks > 0) abort |= !issue_scores(0);
     for (int c = 0; c < n_chunks && ok; ++c) {
         const int t0 = c * Q;
         const uint32_t ph = uint32_t(c & 1);  // each completion barrier completes once per chunk
@@ -402,10 +409,6 @@ __global__ void __launch_bounds__(512, 1) ssd_tc_kernel(const __grid_constant__ 
                           smem_desc_sw128(st + Ly::kX + uint32_t(k * 2048), 0, 1024), idK, k > 0);
             }
             umma_commit(ybar);
-            // the next chunk's scores, into the other score buffer (its last
-            // reader, the masking of chunk c - 1, finished before this chunk's
-            // first barrier)
-            if (c + 1 < n_chunks) abort |= !issue_scores(c + 1);
         }
         if (warp == kScanWarp && c + 1 < n_chunks) {
             scan_store();
@@ -426,6 +429,10 @@ __global__ void __launch_bounds__(512, 1) ssd_tc_kernel(const __grid_constant__ 
         }
         abort |= !mbar_wait_bounded(ybar, ph, p.err);
         tc_fence_after_sync();
+        // the next chunk's scores, into the other score buffer (its last
+        // reader, the masking of chunk c - 1, finished before this chunk's
+        // first barrier), once M X has left the tensor pipe
+        if (scorer && c + 1 < n_chunks) abort |= !issue_scores(c + 1);
         // y = (Ym + exp(cs_i) Yx + D x) silu(z) for row i = `row`, this
         // quarter's 16 columns: 32 contiguous bytes of the token's row, stored
         // from registers
