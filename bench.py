@@ -850,6 +850,9 @@ def run_mss(args, rank, world, local_rank):
     achieved = bytes_fwd / (fwd_avg * 1e-3) / 1e9
     achieved_gen = bytes_fwd / (fwd_avg_gen * 1e-3) / 1e9
     value = whole_job_rate(ct_per_step, world, args.steps, ms)
+    # what the fp32, multi-function and shuffle units deliver per SM and clock
+    # (outside every timed region)
+    pipe_rates = mss.probe_pipe_rates()
     line = {
         "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": ms / args.steps, "higher_is_better": True,
@@ -867,6 +870,8 @@ def run_mss(args, rank, world, local_rank):
                      "frac": alu_ops / (fwd_avg * 1e-3) / alu_peak, "traffic": recorded_traffic(),
                      "kernel": "scan_fwd_seq (forward scan)",
                      "peak_kind": f"derived: {SMS} SMs x {FP32_LANES_PER_SM} fp32 lanes x {sm_max_mhz:.0f} MHz",
+                     "probe_per_sm_per_clk": pipe_rates,
+                     "peak_probe_ffma2": pipe_rates["ffma2"] * SMS * sm_max_mhz * 1e6 / 1e12,
                      "algorithmic_ops_per_launch": alu_ops, "algorithmic_bytes_per_launch": bytes_fwd,
                      "launch_ms_avg": fwd_avg,
                      "launch_ms_p10_p50_p90": [float(np.percentile(fwd_ms, q)) for q in (10, 50, 90)],
@@ -951,6 +956,25 @@ def run_mss(args, rank, world, local_rank):
     return 0
 
 
+def pipe_rates_only(args):
+    """Print one JSON line: the pipe rates (operations per SM and clock) of
+    `args.steps` calls of mss_probe_pipe_rates, each key's median and range."""
+    import torch
+
+    import selective_state_space_mss_b200 as mss
+
+    torch.cuda.set_device(0)
+    runs = [mss.probe_pipe_rates() for _ in range(max(1, args.steps))]
+    out = {}
+    for k in mss.PIPE_RATE_NAMES:
+        v = sorted(r[k] for r in runs)
+        out[k] = {"median": v[len(v) // 2], "min": v[0], "max": v[-1]}
+    print(json.dumps({"pipe_rates_per_sm_per_clk": out, "calls": len(runs),
+                      "device": torch.cuda.get_device_name(0),
+                      "sms": torch.cuda.get_device_properties(0).multi_processor_count}), flush=True)
+    return 0
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -962,6 +986,8 @@ def main():
                     help="only launch one kernel (warmup + steps times); for profiler captures")
     ap.add_argument("--kernel", choices=["forward", "backward", "decode", "ssd"], default="forward",
                     help="which kernel --kernel-only launches")
+    ap.add_argument("--pipe-rates", action="store_true",
+                    help="only measure the fp32 fma, packed fma, ex2 and shuffle rates per SM and clock")
     ap.add_argument("--seqlen", type=int, default=0,
                     help="override the workload's sequence length (the SSD workload's with --kernel ssd)")
     args = ap.parse_args()
@@ -973,6 +999,8 @@ def main():
     local_rank = int(os.environ.get("LOCAL_RANK", "0"))
     if args.impl == "reference":
         return run_reference(args, rank)
+    if args.pipe_rates:
+        return pipe_rates_only(args)
 
     if world > 1:
         import datetime

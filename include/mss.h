@@ -538,6 +538,32 @@ MSS_API int mss_state_update_conv(float *state, void *conv_state, const void *x,
  */
 MSS_API int mss_get_device_error(void *stream);
 
+/*
+ * mss_probe_pipe_rates -- a measurement aid, not part of the scan: the
+ * throughput of the pipes the scan kernels are bound by, on the current
+ * device, in operations per SM and SM clock cycle.  The scan's arithmetic
+ * roof is stated from unit counts (128 fp32 lanes per SM); this call
+ * measures what those units deliver.
+ *
+ *   rates   HOST array of n_rates doubles, written:
+ *             [0] fp32 fma lane operations (scalar fma)
+ *             [1] fp32 fma lane operations with the packed two-wide fma
+ *             [2] ex2.approx results (multi-function unit)
+ *             [3] warp-shuffle results (one per lane)
+ *           entries past [3] are set to 0
+ *   stream  the stream the four loops run on; the call synchronises it
+ *
+ * Each loop runs 8 CTAs of 256 threads per SM, every thread 8 independent
+ * chains of one instruction; a rate is the operations an SM's CTAs executed
+ * over the SM clock cycles from their first start to their last end (the
+ * per-SM cycle counter), averaged over the SMs.  Uses four fixed device
+ * arrays in the library image; allocates nothing.  Not safe to call
+ * concurrently from several host threads on one device.
+ * Errors: MSS_ERR_NULL (rates NULL), MSS_ERR_SHAPE (n_rates < 0),
+ * MSS_ERR_CUDA (launch, copy or synchronisation failed).
+ */
+MSS_API int mss_probe_pipe_rates(double *rates, int n_rates, void *stream);
+
 /* Human-readable text for a status code (static storage, never NULL). */
 MSS_API const char *mss_strerror(int code);
 

@@ -23,7 +23,7 @@ import threading
 import torch
 
 __all__ = ["scan_fwd", "scan_fwd_host", "scan_fwd_conv", "scan_bwd", "ssd_fwd", "bwd_workspace_size", "state_update", "state_update_conv",
-           "get_device_error",
+           "get_device_error", "probe_pipe_rates",
            "library_path", "workspace_size",
            "FLAG_GENERAL_A", "FLAG_SIMPLE", "FLAG_NO_SPLIT", "FLAG_ZOH_INPUT", "FLAG_SELFTEST_TIMEOUT",
            "ERR_DEVICE_TIMEOUT", "ERR_FLAGS", "SSD_FLAG_WARP_MMA", "MssError", "load_library"]
@@ -126,6 +126,8 @@ def load_library():
             lib.mss_strerror.restype = ctypes.c_char_p
             lib.mss_version.argtypes = []
             lib.mss_version.restype = i
+            lib.mss_probe_pipe_rates.argtypes = [ctypes.POINTER(ctypes.c_double), i, vp]
+            lib.mss_probe_pipe_rates.restype = i
             _lib = lib
     return _lib
 
@@ -568,6 +570,22 @@ def state_update(state, u, delta, A, B, C, D=None, z=None, delta_bias=None, soft
     if rc != 0:
         raise MssError(rc, "mss_state_update")
     return y
+
+
+PIPE_RATE_NAMES = ("ffma", "ffma2", "mufu_ex2", "shfl")
+
+
+def probe_pipe_rates(stream=None, device=None) -> dict:
+    """Measured throughput of the fp32 fma pipe (scalar and packed, lane
+    operations), the multi-function unit (ex2 results) and warp shuffles
+    (results), per SM and SM clock cycle, on the current device
+    (mss_probe_pipe_rates)."""
+    dev = torch.device("cuda", torch.cuda.current_device()) if device is None else device
+    out = (ctypes.c_double * len(PIPE_RATE_NAMES))()
+    rc = load_library().mss_probe_pipe_rates(out, len(PIPE_RATE_NAMES), _stream_handle(stream, dev))
+    if rc != 0:
+        raise MssError(rc, "mss_probe_pipe_rates")
+    return {k: float(v) for k, v in zip(PIPE_RATE_NAMES, out)}
 
 
 def get_device_error(stream=None, device=None) -> int:

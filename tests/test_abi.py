@@ -467,3 +467,10 @@ def test_plain_c_client_compiles_links_and_runs(lib):
     assert build.returncode == 0, build.stderr
     run = subprocess.run([exe], capture_output=True, text=True, timeout=60)
     assert run.returncode == 0 and run.stdout.strip() == "ok", run.stdout + run.stderr
+
+
+def test_probe_argument_errors(lib):
+    codes = _enum("mss_status")
+    buf = (ctypes.c_double * 4)()
+    assert lib.mss_probe_pipe_rates(None, 4, None) == codes["MSS_ERR_NULL"]
+    assert lib.mss_probe_pipe_rates(buf, -1, None) == codes["MSS_ERR_SHAPE"]
