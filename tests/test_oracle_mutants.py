@@ -6,6 +6,7 @@ runs the pin tests against it in a subprocess.  The pins must fail for every
 mutant and pass for the unmodified source.  CPU only; nothing here touches
 the CUDA path.
 """
+import concurrent.futures
 import os
 import subprocess
 import sys
@@ -103,18 +104,31 @@ def _pins_on(src_text, name):
                 os.remove(path)
 
 
-def test_unmodified_source_passes():
+@pytest.fixture(scope="module")
+def pin_runs():
+    """The pin run of the unmodified source and of every mutant whose site is
+    found exactly once, run side by side (one subprocess per core)."""
     with open(SRC) as f:
         text = f.read()
-    r = _pins_on(text, "original")
+    jobs = {"original": text}
+    for name, (old, new) in MUTANTS.items():
+        if text.count(old) == 1:
+            jobs[name] = text.replace(old, new)
+    with concurrent.futures.ThreadPoolExecutor(max_workers=max(1, min(len(jobs), os.cpu_count() or 1))) as ex:
+        futures = {name: ex.submit(_pins_on, src, name) for name, src in jobs.items()}
+        return {name: fut.result() for name, fut in futures.items()}
+
+
+def test_unmodified_source_passes(pin_runs):
+    r = pin_runs["original"]
     assert r.returncode == 0, r.stdout[-2000:]
 
 
 @pytest.mark.parametrize("name", sorted(MUTANTS))
-def test_pins_catch_mutant(name):
-    old, new = MUTANTS[name]
+def test_pins_catch_mutant(name, pin_runs):
+    old, _ = MUTANTS[name]
     with open(SRC) as f:
         text = f.read()
     assert text.count(old) == 1, f"mutation site for {name} not found exactly once"
-    r = _pins_on(text.replace(old, new), name)
+    r = pin_runs[name]
     assert r.returncode != 0, f"pins did not catch mutant {name}"
