@@ -227,7 +227,14 @@ class NvmlSampler:
         self._thread = None
         self._nvml = None
         self._t0 = self._t1 = None
+        self._first = 0
         self.stopped_early = False
+
+    def mark(self):
+        """Start of the window the summary covers (the samples before it, taken
+        while the sampler started up and the warm-up ran, are left out)."""
+        self._first = len(self.rows)
+        self._t0 = time.perf_counter()
 
     def __enter__(self):
         import threading
@@ -275,17 +282,18 @@ class NvmlSampler:
         return False
 
     def summary(self):
-        if not self.rows:
+        rows = self.rows[self._first:]
+        if not rows:
             return None
         mask = 0
-        for _, r, _ in self.rows:
+        for _, r, _ in rows:
             mask |= r
         # samples one thread can take in the window (each read also takes time,
         # so the count comes in below this); far fewer means it stopped early
         expected = None if self._t1 is None else int((self._t1 - self._t0) / self.period)
-        return {"sm_mhz": statistics.median(r[0] for r in self.rows), "sm_max_mhz": self.max_mhz,
-                "power_w_max": max(r[2] for r in self.rows),
-                "reasons": [name for name, bit in self.REASONS if mask & bit], "samples": len(self.rows),
+        return {"sm_mhz": statistics.median(r[0] for r in rows), "sm_max_mhz": self.max_mhz,
+                "power_w_max": max(r[2] for r in rows),
+                "reasons": [name for name, bit in self.REASONS if mask & bit], "samples": len(rows),
                 "samples_at_most": expected, "sampler_stopped_early": self.stopped_early,
                 "source": "NVML every 2 ms during the timed region"}
 
@@ -580,19 +588,24 @@ def run_mss(args, rank, world, local_rank):
     bytes_step = bytes_fwd + decode_bytes(w.batch, w.dim, w.dstate)
 
     def timed(flags, k, warm, with_clocks=False):
-        for _ in range(warm):
-            step(flags)
-        if world > 1:
-            dist.barrier()
-        torch.cuda.synchronize(dev)
         evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(k)]
         start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         sampler = ClockSampler(physical_gpu_index(local_rank))
         nvml = NvmlSampler(nvml_device_id(dev, local_rank))
         if with_clocks:
+            # the samplers start (and nvidia-smi gets its first reading) before
+            # the warm-up, so that the GPU does not idle between the warm-up
+            # and the timed steps
             sampler.__enter__()
-            time.sleep(0.3)
             nvml.__enter__()
+            time.sleep(0.3)
+        for _ in range(warm):
+            step(flags)
+        if world > 1:
+            dist.barrier()
+        torch.cuda.synchronize(dev)
+        if with_clocks:
+            nvml.mark()
         start.record(stream)
         for i in range(k):
             step(flags, evs[i])
