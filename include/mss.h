@@ -108,9 +108,10 @@ enum mss_status {
  * skips its checkpoint pass.  See mss_scan_fwd_save. */
 #define MSS_FLAG_SAVED_STATES 0x20u
 /* Forward passes: run the two-lanes-per-channel kernel where the four-lane
- * one would (fp32 io, N = 8 or 16, one pass over the sequence, Euler input
- * rule, no convolution); for testing and measurement, the results agree
- * within the io type's rounding. */
+ * one would (N = 8 or 16, one pass over the sequence, Euler input rule, no
+ * convolution; fp32 io on any grid, bf16 io when batch * ceil(dim / 16) is
+ * at most 384); for testing and measurement, the results agree within the
+ * io type's rounding. */
 #define MSS_FLAG_PAIR_LANES 0x40u
 
 /*

@@ -172,7 +172,10 @@ int launch_seq_conv(const mss::SeqMaps& maps, const mss::ScanParams& p, unsigned
 }
 
 // The four-lane kernel (one pass, Euler input rule, no convolution, no
-// checkpoints).
+// checkpoints).  With bf16 io it is taken for grids of at most this many
+// 16-channel units (2.6 per SM on 148 SMs).
+constexpr int64_t kFourLaneBf16MaxUnits = 384;
+
 template <typename T, int N, bool kGate, bool kSoftplus>
 int launch_seq4_variant(const mss::SeqMaps& maps, const mss::ScanParams& p, unsigned flags, cudaStream_t stream) {
     using Ly = mss::Seq4Layout<T, N>;
@@ -216,13 +219,16 @@ int launch_seq(mss::ScanParams p, unsigned flags, void* workspace, int64_t works
             p.agg = static_cast<float*>(workspace);
         }
     }
-    if constexpr (sizeof(T) == 4 && (N == 8 || N == 16)) {
-        // fp32 io, one pass without the convolution, the zero-order hold or
-        // stored states: four lanes per channel, twice the warps of the pair
-        // kernel (for bf16 io its extra shuffles and selects cost more than
-        // the warps recover, so bf16 keeps the pair kernel)
+    if constexpr (N == 8 || N == 16) {
+        // one pass without the convolution, the zero-order hold or stored
+        // states: four lanes per channel, twice the warps of the pair kernel.
+        // fp32 io always; bf16 io only on small grids, where the doubled warps
+        // outweigh its extra shuffles and selects (measured on B200: 0.78x the
+        // pair kernel's time at 128 and 256 units of 16 channels, 1.05x at
+        // 512, 1.27x at 1024)
+        const int64_t units = p.batch * ((p.dim + br - 1) / br);
         if (p.n_seg == 1 && p.conv_width == 0 && !p.zoh && !p.ckpt && !p.selftest_wait_ns &&
-            !(flags & MSS_FLAG_PAIR_LANES))
+            !(flags & MSS_FLAG_PAIR_LANES) && (sizeof(T) == 4 || units <= kFourLaneBf16MaxUnits))
             return launch_seq4<T, N>(maps, p, flags, stream);
     }
     return p.conv_width > 0 ? launch_seq_conv<T, N, true>(maps, p, flags, stream)

@@ -30,15 +30,18 @@
 // then a CTA-wide vote, so that no warp leaves while the other waits at a
 // barrier).
 //
-// Scope: fp32 io, the Euler input rule, no sequence split, no convolution,
-// no checkpoints, no wait self-test; the host sends everything else to the
-// two-lane kernel.  Measured with fp32 io: 340 us against 371 us for the
-// pair kernel on 4 x 4096 channels at N = 8 (L = 2048), 199 us against 246 us
-// on 8 x 1536 channels at N = 16 (L = 1024), about even on 4 x 4096 at N = 16.
-// With bf16 io it took 466 us against 375 us (L = 4096): its per-token
-// shuffles of Delta*u and r, the lane-dependent power selects and the second
-// reduce stage add 38% instructions that the doubled warps (3.3 per
-// scheduler) do not recover.
+// Scope: the Euler input rule, no sequence split, no convolution, no
+// checkpoints, no wait self-test; fp32 io on any grid, bf16 io on small
+// grids; the host sends everything else to the two-lane kernel.  Measured
+// with fp32 io: 340 us against 371 us for the pair kernel on 4 x 4096
+// channels at N = 8 (L = 2048), 199 us against 246 us on 8 x 1536 channels
+// at N = 16 (L = 1024), about even on 4 x 4096 at N = 16.  With bf16 io at
+// N = 16 its per-token shuffles of Delta*u and r, the lane-dependent power
+// selects and the second reduce stage add 38% instructions: on 4 x 4096
+// channels (1024 CTAs, L = 4096) it took 465 us against 367 us, on 512 CTAs
+// 279 against 267 us, but on 256 CTAs (2 x 2048, L = 4096) 209 against
+// 258 us and on 128 CTAs (1 x 2048, L = 8192) 396 against 506 us, where the
+// pair kernel has under half a warp per scheduler.
 #pragma once
 
 #include <cstdint>
