@@ -1,9 +1,13 @@
 """GPU tests of the forward pass over host buffers (mss_scan_fwd_host).
 
 The call stages pieces of the channels through a device workspace and runs
-the same forward kernel on each piece, so its outputs must equal, bit for bit,
-those of the device call on the same inputs, and the oracle within the
-tolerances of tests/helpers.py.  The cases cover all rows in one piece,
+the forward pass on each piece.  A piece may take the four-lane kernel where
+the whole call takes the pair kernel (small grids of bf16 channels); the two
+sum in the same order and agree bit for bit wherever they take the same
+transition path, which these inputs' A rows (uniform within each group of 16
+channels) guarantee.  So the outputs must equal, bit for bit, those of the
+device call on the same inputs, and the oracle within the tolerances of
+tests/helpers.py.  The cases cover all rows in one piece,
 whole batch rows grouped into more pieces than workspace slots (slot
 reuse), several pieces per batch row with a ragged last piece, the optional
 inputs, an empty sequence, pageable host memory and chaining.
