@@ -39,7 +39,7 @@ FLAG_NO_SPLIT = 0x4
 FLAG_ZOH_INPUT = 0x8  # zero-order-hold input matrix (e^{Delta A} - 1)/A * B instead of Delta * B
 FLAG_SELFTEST_TIMEOUT = 0x10  # the tiled kernel's bounded wait gives up on purpose (failure-path tests)
 FLAG_SAVED_STATES = 0x20  # scan_bwd: the workspace holds the states scan_fwd_save stored
-FLAG_PAIR_LANES = 0x40  # forward: the two-lanes-per-channel kernel where the four-lane one would run (fp32 io)
+FLAG_PAIR_LANES = 0x40  # forward: the two-lanes-per-channel kernel where the four-lane one would run (fp32 io; bf16 io on grids of at most 384 units of 16 channels)
 ERR_PATH = -12
 ERR_FLAGS = -8
 SSD_FLAG_WARP_MMA = 0x1  # ssd_fwd: the warp-level (mma.sync) kernels instead of the tcgen05 one
