@@ -1,6 +1,7 @@
 """A seeded random sweep of the forward pass (plain and with the causal
-convolution in front), the backward pass and the decode step against the
-fp64 oracle.
+convolution in front), the backward pass, the decode step and the
+structured-state-space-duality (Mamba-2) forward pass against the fp64
+oracle.
 
 Each case draws its sizes (odd channel counts; sequence lengths that are
 multiples of the 16-byte row unit, which the tiled kernels take, or ragged,
@@ -22,7 +23,7 @@ from tests.helpers import assert_close, device_inputs, to_numpy, to_torch
 
 pytestmark = pytest.mark.gpu
 DEV = torch.device("cuda", 0)
-N_FWD, N_BWD, N_CONV, N_DEC = 160, 48, 40, 40
+N_FWD, N_BWD, N_CONV, N_DEC, N_SSD = 160, 48, 40, 40, 32
 KEYS = ("du", "ddelta", "dz", "dA", "dB", "dC", "dD", "dbias", "dinit")
 
 
@@ -205,3 +206,63 @@ def test_decode_random_case(i):
         assert_close(to_numpy(y), y_ref, dtype, f"case {i} step {t} y")
     assert_close(to_numpy(state), ref_state, dtype, f"case {i} state")
     assert mss.get_device_error() == 0
+
+
+@pytest.mark.parametrize("i", range(N_SSD))
+def test_ssd_random_case(i):
+    rng = np.random.default_rng([2026, 15, i])
+    batch = int(rng.integers(1, 3))
+    L = int(rng.integers(1, 5)) * 128 if rng.random() < 0.4 else int(rng.integers(1, 600))
+    G = int(rng.choice([1, 2]))
+    H = G * int(rng.integers(1, 4))
+    N = int(rng.choice([64, 128]))
+    flags = mss.SSD_FLAG_WARP_MMA if rng.random() < 0.3 else 0
+    gate, with_D, with_bias = (bool(rng.random() < 0.8) for _ in range(3))
+    workspace = "auto" if rng.random() < 0.5 else None
+    inp = gen.ssd_inputs(batch, L, H, 64, G, N, seed=5000 + i)
+    h0 = (np.random.default_rng(5100 + i).standard_normal((batch, H, N, 64)).astype(np.float32) * 0.1
+          if rng.random() < 0.5 else None)
+    y, last = mss.ssd_fwd(to_torch(inp["x"], DEV), to_torch(inp["dt"], DEV), torch.from_numpy(inp["A"]).to(DEV),
+                          to_torch(inp["B"], DEV), to_torch(inp["C"], DEV),
+                          D=torch.from_numpy(inp["D"]).to(DEV) if with_D else None,
+                          z=to_torch(inp["z"], DEV) if gate else None,
+                          dt_bias=torch.from_numpy(inp["dt_bias"]).to(DEV) if with_bias else None,
+                          initial_state=None if h0 is None else torch.from_numpy(h0).to(DEV),
+                          workspace=workspace, flags=flags)
+    torch.cuda.synchronize()
+    assert mss.get_device_error() == 0
+    y_ref, last_ref = oracle.ssd_fwd(inp["x"].values, inp["dt"].values, inp["A"], inp["B"].values, inp["C"].values,
+                                     D=inp["D"] if with_D else None, z=inp["z"].values if gate else None,
+                                     dt_bias=inp["dt_bias"] if with_bias else None,
+                                     initial_state=None if h0 is None else h0.astype(np.float64))
+    what = f"case {i} b{batch} L{L} H{H} G{G} N{N} flags {flags}"
+    # The products run on bf16 operands (the masked scores, the w-scaled x,
+    # the state read by the next chunk), so an output's rounding error scales
+    # with the sum of the absolute values of its products, not with the
+    # output, which can cancel: without the skip term and with small steps
+    # y is a small difference of larger terms.  That sum is the same pass
+    # with every input in absolute value (the decays are positive) and the
+    # gate's magnitude applied afterwards.
+    y_abs, last_abs = oracle.ssd_fwd(np.abs(inp["x"].values), inp["dt"].values, inp["A"], np.abs(inp["B"].values),
+                                     np.abs(inp["C"].values), D=np.abs(inp["D"]) if with_D else None,
+                                     dt_bias=inp["dt_bias"] if with_bias else None,
+                                     initial_state=None if h0 is None else np.abs(h0).astype(np.float64))
+    if gate:
+        zz = inp["z"].values.astype(np.float64)
+        y_abs = y_abs * np.abs(zz / (1.0 + np.exp(-zz)))
+    _assert_within_products(to_numpy(y), y_ref, y_abs, what + " y")
+    _assert_within_products(to_numpy(last), last_ref, last_abs, what + " last_state")
+
+
+def _assert_within_products(got, ref, scale, what):
+    """|got - ref| <= 2^-7 (sum of |products|) + 2^-8 |ref|: a few bf16
+    operand roundings (2^-9 each) of every product, plus the bf16 output."""
+    got, ref, scale = (np.asarray(a, dtype=np.float64) for a in (got, ref, scale))
+    assert got.shape == ref.shape
+    assert np.all(np.isfinite(got)), f"{what}: non-finite values"
+    bound = 2.0 ** -7 * scale + 2.0 ** -8 * np.abs(ref)
+    bad = np.abs(got - ref) > bound
+    if np.any(bad):
+        k = np.unravel_index(np.argmax(np.abs(got - ref) / np.maximum(bound, 1e-300)), got.shape)
+        raise AssertionError(f"{what}: {int(bad.sum())} of {got.size} elements out of bound; worst at {k}: "
+                             f"got {got[k]!r}, ref {ref[k]!r}, bound {bound[k]!r}")
