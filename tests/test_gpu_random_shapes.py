@@ -1,5 +1,6 @@
-"""A seeded random sweep of the forward pass (plain and with the causal
-convolution in front), the backward pass, the decode step and the
+"""A seeded random sweep of the forward pass (on device buffers, on host
+buffers, and with the causal convolution in front), the backward pass, the
+decode step (plain and with the convolution) and the
 structured-state-space-duality (Mamba-2) forward pass against the fp64
 oracle.
 
@@ -23,7 +24,7 @@ from tests.helpers import assert_close, device_inputs, to_numpy, to_torch
 
 pytestmark = pytest.mark.gpu
 DEV = torch.device("cuda", 0)
-N_FWD, N_BWD, N_CONV, N_DEC, N_SSD = 160, 48, 40, 40, 32
+N_FWD, N_BWD, N_CONV, N_DEC, N_SSD, N_HOST, N_DEC_CONV = 160, 48, 40, 40, 32, 16, 16
 KEYS = ("du", "ddelta", "dz", "dA", "dB", "dC", "dD", "dbias", "dinit")
 
 
@@ -252,6 +253,77 @@ def test_ssd_random_case(i):
         y_abs = y_abs * np.abs(zz / (1.0 + np.exp(-zz)))
     _assert_within_products(to_numpy(y), y_ref, y_abs, what + " y")
     _assert_within_products(to_numpy(last), last_ref, last_abs, what + " last_state")
+
+
+@pytest.mark.parametrize("i", range(N_HOST), ids=lambda i: _id(300 + i, 600))
+def test_host_forward_random_case(i):
+    c = _draw(300 + i, 600)
+    flags = c["flags"] & (mss.FLAG_ZOH_INPUT | mss.FLAG_GENERAL_A | mss.FLAG_SIMPLE | mss.FLAG_NO_SPLIT)
+    inp, h0 = _inputs(c)
+    cpu = torch.device("cpu")
+    pin = c["workspace"]  # pinned or pageable host memory
+
+    def host(t):
+        t = to_torch(t, cpu) if not isinstance(t, np.ndarray) else torch.from_numpy(t)
+        return t.pin_memory() if pin else t
+
+    y, last = mss.scan_fwd_host(host(inp["u"]), host(inp["delta"]), host(inp["A"]), host(inp["B"]), host(inp["C"]),
+                                D=host(inp["D"]) if c["with_D"] else None,
+                                z=host(inp["z"]) if c["gate"] else None,
+                                delta_bias=host(inp["delta_bias"]) if c["with_bias"] else None,
+                                softplus=c["softplus"], initial_state=None if h0 is None else host(h0),
+                                flags=flags, device=DEV)
+    torch.cuda.synchronize()
+    assert mss.get_device_error() == 0
+    y_ref, last_ref = oracle.scan_fwd(inp["u"].values, inp["delta"].values, inp["A"], inp["B"].values,
+                                      inp["C"].values, D=inp["D"] if c["with_D"] else None,
+                                      z=inp["z"].values if c["gate"] else None,
+                                      delta_bias=inp["delta_bias"] if c["with_bias"] else None,
+                                      softplus_flag=c["softplus"],
+                                      initial_state=None if h0 is None else h0.astype(np.float64),
+                                      zoh_input=bool(flags & mss.FLAG_ZOH_INPUT))
+    assert_close(to_numpy(y), y_ref, c["dtype"], f"case {i} y")
+    assert_close(to_numpy(last), last_ref, c["dtype"], f"case {i} last_state")
+
+
+@pytest.mark.parametrize("i", range(N_DEC_CONV))
+def test_decode_conv_random_case(i):
+    rng = np.random.default_rng([2026, 16, i])
+    dtype = str(rng.choice(["f32", "bf16"]))
+    N = int(rng.choice([1, 2, 4, 8, 16]))
+    batch = int(rng.integers(1, 4))
+    dim = int(rng.integers(1, 3)) * (2048 // N) if rng.random() < 0.5 else int(rng.integers(1, 200))
+    K = int(rng.integers(1, 5))
+    zoh = bool(rng.random() < 0.3)
+    gate, with_D = bool(rng.random() < 0.8), bool(rng.random() < 0.8)
+    seed = 6000 + i
+    A, D, bias = gen.channel_params(dim, N, "normal", seed, str(rng.choice(list(gen.A_RECIPES))))
+    cw, cb = gen.conv_params(dim, K, seed + 1)
+    h0 = gen.initial_state(batch, dim, N, seed + 2, "normal")
+    state = torch.from_numpy(h0.copy()).to(DEV)
+    ref_state = h0.astype(np.float64)
+    cs_ref = np.zeros((batch, dim, 0))
+    cs = None
+    if K > 1:
+        cs0 = gen.conv_state(batch, dim, K, dtype, seed + 3)
+        cs = to_torch(cs0, DEV).clone()
+        cs_ref = cs0.values.astype(np.float64).copy()
+    Ad, Dd, bd, cwd, cbd = (torch.from_numpy(x).to(DEV) for x in (A, D, bias, cw, cb))
+    for t in range(3):
+        s = gen.decode_step_inputs(batch, dim, N, dtype, seed + 4, t)
+        y = mss.state_update_conv(state, cs, to_torch(s["u"], DEV), cwd, to_torch(s["delta"], DEV), Ad,
+                                  to_torch(s["B"], DEV), to_torch(s["C"], DEV), conv_b=cbd,
+                                  D=Dd if with_D else None, z=to_torch(s["z"], DEV) if gate else None,
+                                  delta_bias=bd, flags=mss.FLAG_ZOH_INPUT if zoh else 0)
+        y_ref, ref_state, cs_ref = oracle.state_update_conv(
+            ref_state, cs_ref, s["u"].values, cw, s["delta"].values, A, s["B"].values, s["C"].values, conv_b=cb,
+            D=D if with_D else None, z=s["z"].values if gate else None, delta_bias=bias, zoh_input=zoh)
+        torch.cuda.synchronize()
+        assert_close(to_numpy(y), y_ref, dtype, f"case {i} K={K} step {t} y")
+    assert_close(to_numpy(state), ref_state, dtype, f"case {i} K={K} state")
+    if K > 1:
+        assert_close(to_numpy(cs), cs_ref, dtype, f"case {i} K={K} conv_state")
+    assert mss.get_device_error() == 0
 
 
 def _assert_within_products(got, ref, scale, what):
