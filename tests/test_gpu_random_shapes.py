@@ -24,7 +24,7 @@ from tests.helpers import assert_close, device_inputs, to_numpy, to_torch
 
 pytestmark = pytest.mark.gpu
 DEV = torch.device("cuda", 0)
-N_FWD, N_BWD, N_CONV, N_DEC, N_SSD, N_HOST, N_DEC_CONV = 160, 48, 40, 40, 32, 16, 16
+N_FWD, N_BWD, N_CONV, N_DEC, N_SSD, N_HOST, N_DEC_CONV = 320, 96, 64, 64, 64, 24, 32
 KEYS = ("du", "ddelta", "dz", "dA", "dB", "dC", "dD", "dbias", "dinit")
 
 
@@ -101,9 +101,9 @@ def test_forward_random_case(i):
     assert_close(to_numpy(last), last_ref, c["dtype"], f"case {i} last_state")
 
 
-@pytest.mark.parametrize("i", range(N_BWD), ids=lambda i: _id(100 + i, 400))
+@pytest.mark.parametrize("i", range(N_BWD), ids=lambda i: _id(1000 + i, 400))
 def test_backward_random_case(i):
-    c = _draw(100 + i, 400)
+    c = _draw(1000 + i, 400)
     flags = c["flags"] & (mss.FLAG_ZOH_INPUT | mss.FLAG_GENERAL_A | mss.FLAG_SIMPLE)
     inp, h0 = _inputs(c)
     d = device_inputs(inp, DEV, with_z=c["gate"], with_D=c["with_D"], with_bias=c["with_bias"])
@@ -141,9 +141,9 @@ def test_backward_random_case(i):
         assert_close(to_numpy(g2[k]), ref[k], c["dtype"], f"case {i} saved-states {k}")
 
 
-@pytest.mark.parametrize("i", range(N_CONV), ids=lambda i: _id(200 + i, 600))
+@pytest.mark.parametrize("i", range(N_CONV), ids=lambda i: _id(2000 + i, 600))
 def test_conv_forward_random_case(i):
-    c = _draw(200 + i, 600)
+    c = _draw(2000 + i, 600)
     rng = np.random.default_rng([2026, 13, i])
     K = int(rng.integers(1, 5))
     flags = c["flags"] & (mss.FLAG_ZOH_INPUT | mss.FLAG_GENERAL_A | mss.FLAG_SIMPLE | mss.FLAG_NO_SPLIT)
@@ -255,9 +255,9 @@ def test_ssd_random_case(i):
     _assert_within_products(to_numpy(last), last_ref, last_abs, what + " last_state")
 
 
-@pytest.mark.parametrize("i", range(N_HOST), ids=lambda i: _id(300 + i, 600))
+@pytest.mark.parametrize("i", range(N_HOST), ids=lambda i: _id(3000 + i, 600))
 def test_host_forward_random_case(i):
-    c = _draw(300 + i, 600)
+    c = _draw(3000 + i, 600)
     flags = c["flags"] & (mss.FLAG_ZOH_INPUT | mss.FLAG_GENERAL_A | mss.FLAG_SIMPLE | mss.FLAG_NO_SPLIT)
     inp, h0 = _inputs(c)
     cpu = torch.device("cpu")
