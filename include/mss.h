@@ -93,7 +93,8 @@ enum mss_status {
  * same under both rules. */
 #define MSS_FLAG_ZOH_INPUT 0x8u
 /* Self-test of the kernels' bounded waits (for tests of the failure path):
- * every CTA of the tiled forward kernel first waits on a barrier that no copy
+ * every CTA of the tiled forward kernel (two or four lanes per channel,
+ * whichever the call takes) first waits on a barrier that no copy
  * will ever complete -- none has been issued yet -- with a limit of 1 ms.  The
  * wait gives up, sets the device error word (mss_get_device_error then
  * returns MSS_ERR_DEVICE_TIMEOUT, once) and the CTA returns; y, last_state and

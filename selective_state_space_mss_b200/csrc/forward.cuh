@@ -227,8 +227,8 @@ int launch_seq(mss::ScanParams p, unsigned flags, void* workspace, int64_t works
         // pair kernel's time at 128 and 256 units of 16 channels, 1.05x at
         // 512, 1.27x at 1024)
         const int64_t units = p.batch * ((p.dim + br - 1) / br);
-        if (p.n_seg == 1 && p.conv_width == 0 && !p.zoh && !p.ckpt && !p.selftest_wait_ns &&
-            !(flags & MSS_FLAG_PAIR_LANES) && (sizeof(T) == 4 || units <= kFourLaneBf16MaxUnits))
+        if (p.n_seg == 1 && p.conv_width == 0 && !p.zoh && !p.ckpt && !(flags & MSS_FLAG_PAIR_LANES) &&
+            (sizeof(T) == 4 || units <= kFourLaneBf16MaxUnits))
             return launch_seq4<T, N>(maps, p, flags, stream);
     }
     return p.conv_width > 0 ? launch_seq_conv<T, N, true>(maps, p, flags, stream)

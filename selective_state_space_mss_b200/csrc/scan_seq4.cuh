@@ -31,8 +31,8 @@
 // barrier).
 //
 // Scope: the Euler input rule, no sequence split, no convolution, no
-// checkpoints, no wait self-test; fp32 io on any grid, bf16 io on small
-// grids; the host sends everything else to the two-lane kernel.  Measured
+// checkpoints; fp32 io on any grid, bf16 io on small grids; the host sends
+// everything else to the two-lane kernel.  Measured
 // with fp32 io: 340 us against 371 us for the pair kernel on 4 x 4096
 // channels at N = 8 (L = 2048), 199 us against 246 us on 8 x 1536 channels
 // at N = 16 (L = 1024), about even on 4 x 4096 at N = 16.  With bf16 io at
@@ -403,7 +403,7 @@ __global__ void __launch_bounds__(64) scan_fwd_seq4_kernel(const __grid_constant
     const int64_t row = int64_t(blockIdx.y) * p.dim + d;
 
     if (tid == 0) {
-        for (int s = 0; s < F::kStages; ++s) mbar_init(bars + s, 1);
+        for (int s = 0; s <= F::kStages; ++s) mbar_init(bars + s, 1);
         fence_barrier_init();
         prefetch_tensormap(&maps.u);
         prefetch_tensormap(&maps.delta);
@@ -412,6 +412,14 @@ __global__ void __launch_bounds__(64) scan_fwd_seq4_kernel(const __grid_constant
         prefetch_tensormap(&maps.C);
     }
     __syncthreads();
+    if (p.selftest_wait_ns) {
+        // wait self-test, as in the two-lane kernel: barrier kStages never
+        // completes (no copy has been issued and nothing arrives), so every
+        // thread's bounded wait gives up and sets the error word; the CTA
+        // returns with nothing in flight
+        mbar_wait_bounded(bars + F::kStages, 0u, p.err, p.selftest_wait_ns);
+        return;
+    }
 
     constexpr bool kFast = sizeof(T) == 2;
     Lane4Const<N> cc;

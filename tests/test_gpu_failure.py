@@ -31,18 +31,21 @@ PAD = 64  # elements of margin on each side: keeps 16-byte alignment for every d
 # ---------------------------------------------------------------------------
 # Bounded waits
 
-def test_bounded_wait_gives_up_and_the_next_call_is_clean():
+@pytest.mark.parametrize("lanes", [0, mss.FLAG_PAIR_LANES], ids=["four-lane", "pair"])
+def test_bounded_wait_gives_up_and_the_next_call_is_clean(lanes):
+    # 8 units of 16 bf16 channels: the four-lane kernel unless the flag asks
+    # for the pair kernel
     assert mss.get_device_error() == 0
     inp = gen.scan_inputs(2, 64, 16, 512, "bf16", seed=700, d_skip="normal")
     d = device_inputs(inp, DEV)
     y = torch.full((2, 64, 512), 3.0, dtype=torch.bfloat16, device=DEV)
     last = torch.full((2, 64, 16), 5.0, device=DEV)
-    mss.scan_fwd(**d, y=y, last_state=last, flags=mss.FLAG_SELFTEST_TIMEOUT)
+    mss.scan_fwd(**d, y=y, last_state=last, flags=mss.FLAG_SELFTEST_TIMEOUT | lanes)
     assert mss.get_device_error() == mss.ERR_DEVICE_TIMEOUT
     assert mss.get_device_error() == 0  # reported once, then cleared
     assert torch.all(y == 3.0) and torch.all(last == 5.0)  # nothing was written
     # the context is usable and the same call without the flag is right
-    y2, last2 = mss.scan_fwd(**d)
+    y2, last2 = mss.scan_fwd(**d, flags=lanes)
     assert mss.get_device_error() == 0
     y_ref, last_ref = oracle.scan_fwd(inp["u"].values, inp["delta"].values, inp["A"], inp["B"].values,
                                       inp["C"].values, D=inp["D"], z=inp["z"].values, delta_bias=inp["delta_bias"])
