@@ -246,3 +246,28 @@ def ssd_inputs(batch: int, seqlen: int, nheads: int, headdim: int, ngroups: int,
         C=_store(scale * f(batch, seqlen, ngroups, dstate), dtype),
         D=(1.0 + 0.1 * rng.standard_normal(nheads)).astype(np.float32),
     )
+
+
+def device_scan_inputs(batch: int, dim: int, dstate: int, seqlen: int, seed: int, device):
+    """bf16 inputs of one forward pass drawn directly on `device` (for sizes
+    whose host-side draw would not fit in host memory): u, z, B, C ~ N(0, 1)
+    and delta_raw = 0.1 N(0, 1) from torch's seeded generator on the device,
+    rounded to bf16 by torch; A, D (N(1, 0.1)) and the step bias as in
+    channel_params.  Returns a dict of device tensors (A, D, delta_bias fp32);
+    the oracle reads the rows it checks back from the device."""
+    import torch
+
+    g = torch.Generator(device=device)
+    g.manual_seed(int(seed))
+
+    def draw(shape, scale=1.0):
+        t = torch.randn(shape, generator=g, device=device, dtype=torch.float32)
+        if scale != 1.0:
+            t.mul_(scale)
+        return t.to(torch.bfloat16)
+
+    A, D, bias = channel_params(dim, dstate, "normal", seed)
+    return dict(u=draw((batch, dim, seqlen)), delta=draw((batch, dim, seqlen), 0.1),
+                z=draw((batch, dim, seqlen)), B=draw((batch, dstate, seqlen)), C=draw((batch, dstate, seqlen)),
+                A=torch.from_numpy(A).to(device), D=torch.from_numpy(D).to(device),
+                delta_bias=torch.from_numpy(bias).to(device))
