@@ -26,6 +26,7 @@ SAMPLE = (0, DIM // 2, DIM - 17, DIM - 2, DIM - 1)
 @pytest.fixture(scope="module")
 def big():
     assert BATCH * DIM * L > 2 ** 31
+    torch.cuda.empty_cache()  # blocks other tests left in torch's cache
     free, _ = torch.cuda.mem_get_info(DEV)
     if free < 60 * 2 ** 30:
         pytest.skip(f"needs about 60 GB of free device memory, {free / 2**30:.0f} GB free")
@@ -75,6 +76,7 @@ def test_backward_beyond_2_to_31_elements(big):
 def test_decode_state_beyond_2_to_31_elements():
     # state [4096, 32768, 16] fp32: 2^31 elements (8.6 GB), one token
     batch, dim, n = 4096, 32768, 16
+    torch.cuda.empty_cache()  # blocks other tests left in torch's cache
     free, _ = torch.cuda.mem_get_info(DEV)
     if free < 24 * 2 ** 30:
         pytest.skip(f"needs about 24 GB of free device memory, {free / 2**30:.0f} GB free")
@@ -107,6 +109,7 @@ def test_decode_state_beyond_2_to_31_elements():
 def test_ssd_beyond_2_to_31_elements():
     # x, z, y [1, 131072, 256, 64] bf16: 2^31 elements each
     batch, L, H, P, G, NS = 1, 131072, 256, 64, 1, 128
+    torch.cuda.empty_cache()  # blocks other tests left in torch's cache
     free, _ = torch.cuda.mem_get_info(DEV)
     if free < 40 * 2 ** 30:
         pytest.skip(f"needs about 40 GB of free device memory, {free / 2**30:.0f} GB free")
