@@ -430,12 +430,13 @@ MSS_API int mss_ssd_fwd(const void *x, const void *dt, const float *A, const voi
 /* mss_ssd_fwd with a caller-owned workspace (device memory, 16-byte aligned,
  * at least mss_ssd_fwd_workspace_size bytes, not overlapping any argument).
  * When batch * nheads leaves the in-order kernel's last wave of CTAs (one
- * per (batch, head), up to two per SM) short enough, the chunks of every
- * head then run in parallel in three passes (chunk states, the recurrence of
- * chunk states, chunk outputs) instead of one CTA walking a head's chunks in
- * order; otherwise the workspace is not used (the passes' extra state
- * traffic would cost more than they gain).  On a 148-SM B200 the passes run
- * for up to 115 pairs;
+ * per (batch, head): up to two per SM for dstate 64, one for the tcgen05
+ * kernel of dstate 128) short enough, the chunks of every head then run in
+ * parallel in three passes (chunk states, the recurrence of chunk states,
+ * chunk outputs; warp-level kernels) instead of one CTA walking a head's
+ * chunks in order; otherwise the workspace is not used (the passes' extra
+ * state traffic would cost more than they gain).  On a 148-SM B200 the
+ * passes run for up to 115 pairs at dstate 64 and up to 28 at dstate 128;
  * mss_ssd_fwd_workspace_size returns 0 where the workspace goes unused.
  * Same result up to rounding; a NULL workspace is mss_ssd_fwd.
  * MSS_ERR_WORKSPACE if it is too small. */
@@ -447,8 +448,7 @@ MSS_API int mss_ssd_fwd_ex(const void *x, const void *dt, const float *A, const 
 
 /* Workspace bytes mss_ssd_fwd_ex would use for these sizes on the current
  * device (0: the in-order kernel, or no tokens), or a negative mss_status
- * (MSS_ERR_SHAPE for unsupported sizes).  dstate 128 runs the tcgen05 kernel
- * in order: 0. */
+ * (MSS_ERR_SHAPE for unsupported sizes). */
 MSS_API int64_t mss_ssd_fwd_workspace_size(int64_t batch, int64_t seqlen, int64_t nheads, int64_t headdim,
                                    int64_t ngroups, int64_t dstate);
 
@@ -462,8 +462,10 @@ MSS_API int64_t mss_ssd_fwd_workspace_size(int64_t batch, int64_t seqlen, int64_
  * kernel -- one CTA per (batch, head) walking chunks of 128 tokens in order,
  * operands staged by TMA in shared memory, the four chunk products
  * (C B^T, B^T diag(w) X, C S_prev, M X) on the fifth-generation tensor cores
- * with fp32 accumulators in tensor memory -- and ignores the workspace;
- * dstate 64 runs the warp-level kernels as described at mss_ssd_fwd_ex.
+ * with fp32 accumulators in tensor memory -- unless a workspace is given
+ * and there are so few (batch, head) pairs that the chunk-parallel passes
+ * are faster (see mss_ssd_fwd_ex); dstate 64 runs the warp-level kernels as
+ * described at mss_ssd_fwd_ex.
  * MSS_SSD_FLAG_WARP_MMA: the warp-level kernels for both dstate (in order,
  * or the chunk-parallel passes with a workspace where they pay).  Other
  * bits: MSS_ERR_FLAGS.  Same results up to rounding; the tcgen05 kernel's

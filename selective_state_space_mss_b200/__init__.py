@@ -393,8 +393,10 @@ def ssd_fwd(x, dt, A, B, C, D=None, z=None, dt_bias=None, softplus=True, initial
     float32.  workspace: "auto" (what mss_ssd_fwd_workspace_size_ex asks for,
     from PyTorch's allocator: every chunk in parallel where that beats one CTA
     per head, else nothing), None (one CTA per head walks its chunks) or a
-    uint8 CUDA tensor.  flags: 0 (the tcgen05 kernel for N = 128) or
-    SSD_FLAG_WARP_MMA (the warp-level kernels).  Returns (y, last_state)."""
+    uint8 CUDA tensor.  flags: 0 (the tcgen05 kernel for N = 128, unless a
+    workspace is given and the chunk-parallel passes are faster for so few
+    (batch, head) pairs) or SSD_FLAG_WARP_MMA (the warp-level kernels).
+    Returns (y, last_state)."""
     if not isinstance(x, torch.Tensor) or x.device.type != "cuda":
         raise ValueError("x must be a CUDA tensor (there is no CPU path)")
     if x.dim() != 4 or B.dim() != 4:

@@ -57,6 +57,8 @@ int64_t ssd_workspace_bytes(int64_t batch, int64_t seqlen, int64_t nheads, int64
 // Whether the chunk-parallel passes beat the in-order kernel for this many
 // (batch, head) pairs on the current device.
 bool ssd_chunked_pays(int64_t batch, int64_t nheads);
+// The same against the tcgen05 kernel (dstate 128).
+bool ssd_chunked_pays_tc(int64_t batch, int64_t nheads);
 
 #define MSS_DECLARE_LAUNCHERS(T, N)                                                                      \
     extern template int launch_forward<T, N>(mss::ScanParams, unsigned, void*, int64_t, cudaStream_t); \

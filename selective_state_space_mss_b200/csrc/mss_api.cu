@@ -466,9 +466,12 @@ int64_t mss_ssd_fwd_workspace_size_ex(int64_t batch, int64_t seqlen, int64_t nhe
         return MSS_ERR_SHAPE;
     int64_t bh, tok;
     if (!mul_ok(batch, nheads, &bh) || !mul_ok(bh, seqlen, &tok) || tok > (int64_t(1) << 40)) return MSS_ERR_SHAPE;
-    // dstate 128 runs the tcgen05 kernel in order unless the warp-level kernels are asked for
-    if (dstate == 128 && !(flags & MSS_SSD_FLAG_WARP_MMA)) return 0;
-    return seqlen == 0 || !ssd_chunked_pays(batch, nheads) ? 0 : ssd_workspace_bytes(batch, seqlen, nheads, dstate);
+    // dstate 128 runs the tcgen05 kernel in order unless the warp-level kernels
+    // are asked for, or so few (batch, head) pairs leave most SMs idle that
+    // the chunk-parallel passes are faster
+    const bool pays = (dstate == 128 && !(flags & MSS_SSD_FLAG_WARP_MMA)) ? ssd_chunked_pays_tc(batch, nheads)
+                                                                          : ssd_chunked_pays(batch, nheads);
+    return seqlen == 0 || !pays ? 0 : ssd_workspace_bytes(batch, seqlen, nheads, dstate);
 }
 
 int mss_ssd_fwd_ex(const void* x, const void* dt, const float* A, const void* B, const void* C, const float* D,
@@ -529,8 +532,8 @@ int mss_ssd_fwd_ex2(const void* x, const void* dt, const float* A, const void* B
     mss::SsdParams p{x, dt, A, B, C, D, z, dt_bias, initial_state, y, last_state, batch, seqlen, nheads, ngroups,
                      softplus_flag ? 1 : 0};
     if (!(p.err = device_error_word())) return MSS_ERR_CUDA;
-    if (dstate == 128 && !(flags & MSS_SSD_FLAG_WARP_MMA)) return launch_ssd_tc(p, s);
-    if (workspace && ssd_chunked_pays(batch, nheads)) {
+    const bool tc = dstate == 128 && !(flags & MSS_SSD_FLAG_WARP_MMA);
+    if (workspace && (tc ? ssd_chunked_pays_tc(batch, nheads) : ssd_chunked_pays(batch, nheads))) {
         const int64_t need = ssd_workspace_bytes(batch, seqlen, nheads, dstate);
         if (need > workspace_bytes || !aligned(workspace, 16)) return MSS_ERR_WORKSPACE;
         const Range ws{workspace, workspace_bytes};
@@ -540,6 +543,7 @@ int mss_ssd_fwd_ex2(const void* x, const void* dt, const float* A, const void* B
             if (overlaps(ws.p, ws.n, o.p, o.n)) return MSS_ERR_ALIAS;
         return launch_ssd_chunked(p, int(dstate), workspace, s);
     }
+    if (tc) return launch_ssd_tc(p, s);
     return launch_ssd(p, int(dstate), s);
 }
 

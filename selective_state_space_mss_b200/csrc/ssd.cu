@@ -118,6 +118,25 @@ bool ssd_chunked_pays(int64_t batch, int64_t nheads) {
     return chunked < in_order;
 }
 
+// The same choice against the tcgen05 kernel (dstate 128): one CTA per SM,
+// about 0.32 of the warp-level kernel's lone-CTA time per wave of 148
+// (118-126 us at 4096 tokens), while the passes take about 25 us plus
+// 3.2 us per (batch, head) pair; the passes win up to about 28 pairs on 148
+// SMs (B200, 4096 tokens: 61 against 117 us at 4 pairs, 72 against 119 at
+// 16, 101 against 126 at 24, 121 against 119 at 32).
+bool ssd_chunked_pays_tc(int64_t batch, int64_t nheads) {
+    static std::mutex mu;
+    static int cache[kMaxDevices] = {};
+    const int64_t sms = per_device(cache, mu, [](int dev) {
+        int n = 0;
+        return cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) == cudaSuccess ? n : 0;
+    });
+    const int64_t pairs = batch * nheads;
+    if (sms <= 0 || pairs <= 0) return false;
+    const int64_t waves = (pairs + sms - 1) / sms;
+    return 128 * pairs / sms + 7 < 32 * waves;  // hundredths of a lone warp-level pass
+}
+
 int64_t ssd_workspace_bytes(int64_t batch, int64_t seqlen, int64_t nheads, int64_t dstate) {
     const int64_t nc = (seqlen + 63) / 64;
     const int64_t per_chunk = dstate * 64 * (4 + 2) + 4;  // S_local fp32, S_in bf16, decay

@@ -77,23 +77,27 @@ def test_ssd_starting_state_and_chaining(kernel):
 
 
 def test_ssd_workspace_only_when_it_pays():
-    """The warp-level kernels: few (batch, head) pairs take the chunk-parallel
-    passes, many the in-order kernel.  N = 128 runs the tcgen05 kernel in
-    order and asks for no workspace.  Each gives the oracle's result."""
+    """Few (batch, head) pairs take the chunk-parallel passes, many the
+    in-order kernel: up to about 115 pairs on 148 SMs for the warp-level
+    in-order kernel, up to about 28 for the tcgen05 one (N = 128, one CTA
+    per SM).  Each gives the oracle's result."""
     lib = mss.load_library()
     sms = torch.cuda.get_device_properties(0).multi_processor_count
     w = mss.SSD_FLAG_WARP_MMA
     assert lib.mss_ssd_fwd_workspace_size_ex(1, 4096, 4, 64, 1, 128, w) > 0
     assert lib.mss_ssd_fwd_workspace_size_ex(4, 4096, sms, 64, 1, 128, w) == 0
-    assert lib.mss_ssd_fwd_workspace_size(1, 4096, 4, 64, 1, 128) == 0
+    assert lib.mss_ssd_fwd_workspace_size(1, 4096, 4, 64, 1, 128) > 0
+    assert lib.mss_ssd_fwd_workspace_size(1, 4096, 64, 64, 1, 128) == 0
+    assert lib.mss_ssd_fwd_workspace_size(1, 4096, 64, 64, 1, 64) > 0
     assert lib.mss_ssd_fwd_workspace_size(1, 4096, 4, 64, 1, 64) > 0
     inp = gen.ssd_inputs(1, 1024, 2, 64, 1, 128, seed=735)
     y_ref, last_ref = _ref(inp)
     for f in (0, w):
-        y, last = mss.ssd_fwd(**_dev(inp), flags=f)
-        torch.cuda.synchronize()
-        assert_close(to_numpy(y), y_ref, "bf16", f"few heads y (flags {f})")
-        assert_close(to_numpy(last), last_ref, "bf16", f"few heads last_state (flags {f})")
+        for ws in ("auto", None):
+            y, last = mss.ssd_fwd(**_dev(inp), flags=f, workspace=ws)
+            torch.cuda.synchronize()
+            assert_close(to_numpy(y), y_ref, "bf16", f"few heads y (flags {f}, workspace {ws})")
+            assert_close(to_numpy(last), last_ref, "bf16", f"few heads last_state (flags {f}, workspace {ws})")
 
 
 @pytest.mark.parametrize("N", [64, 128])
