@@ -117,6 +117,19 @@ int choose_segments(int64_t batch, int64_t dim, int64_t seqlen) {
     int64_t n = std::min<int64_t>(slots / ctas, (target + ctas - 1) / ctas);
     n = std::min<int64_t>(std::min<int64_t>(n, n_chunks), 64);
     if (n < 2) return 1;
+    // Measured against one pass (L = 4096, B200), where one pass wins: bf16
+    // at N = 16 with two segments (263-267 against 285-291 us at 384-512
+    // units of 16 channels: the fold re-runs half the sequence to double the
+    // warps), fp32 at N = 8 or 16 above 384 units, where the one pass runs
+    // four lanes per channel (646 against 797 us at N = 16, 461 against 483 at
+    // N = 8).  bf16 at N = 8 keeps the split up to 512 units (226 against
+    // 240 us), fp32 up to 384 (607 against 646, 370 against 461 us).
+    if constexpr (sizeof(T) == 2 && N == 16) {
+        if (n == 2) return 1;
+    }
+    if constexpr (sizeof(T) == 4 && N >= 8) {
+        if (ctas > 384) return 1;
+    }
     // equal segments of whole chunks
     const int64_t seg_chunks = (n_chunks + n - 1) / n;
     return int((n_chunks + seg_chunks - 1) / seg_chunks);
