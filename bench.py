@@ -941,7 +941,8 @@ def run_mss(args, rank, world, local_rank):
                          "hbm_frac": ssd2_bytes / (ssd2_ms * 1e-3) / 1e9 / peak,
                          "tensor_frac": ssd2_flops / (ssd2_ms * 1e-3) / 1e12 / measured_bf16_tflops()[0],
                          "algorithmic_bytes_per_launch": ssd2_bytes,
-                         "note": "160 (batch, head) CTAs: 1.08 waves of 148 SMs"}},
+                         "note": "160 (batch, head) pairs: a wave of 148 on the tcgen05 kernel, the 12 past it "
+                                 "on the chunk-parallel passes (the library's workspace)"}},
         "zoh_input_path": {"fwd_ms_avg": fwd_avg_zoh,
                            "achieved_gbs": bytes_fwd / (fwd_avg_zoh * 1e-3) / 1e9,
                            "frac": bytes_fwd / (fwd_avg_zoh * 1e-3) / 1e9 / peak,

@@ -436,7 +436,11 @@ MSS_API int mss_ssd_fwd(const void *x, const void *dt, const float *A, const voi
  * chunk outputs; warp-level kernels) instead of one CTA walking a head's
  * chunks in order; otherwise the workspace is not used (the passes' extra
  * state traffic would cost more than they gain).  On a 148-SM B200 the
- * passes run for up to 115 pairs at dstate 64 and up to 28 at dstate 128;
+ * passes run for up to 115 pairs at dstate 64 and up to 28 at dstate 128.
+ * At dstate 128 they also take the pairs past the tcgen05 kernel's last full
+ * wave (one CTA per SM) when those are at most one in nine SMs' worth (16 on
+ * 148 SMs), the whole waves staying on the tcgen05 kernel, and the
+ * workspace then holds only those pairs' chunk states;
  * mss_ssd_fwd_workspace_size returns 0 where the workspace goes unused.
  * Same result up to rounding; a NULL workspace is mss_ssd_fwd.
  * MSS_ERR_WORKSPACE if it is too small. */

@@ -392,8 +392,9 @@ def ssd_fwd(x, dt, A, B, C, D=None, z=None, dt_bias=None, softplus=True, initial
     float32; B, C: [batch, L, G, N] bf16; initial_state: [batch, H, N, P]
     float32.  workspace: "auto" (what mss_ssd_fwd_workspace_size_ex asks for,
     from PyTorch's allocator: every chunk in parallel where that beats one CTA
-    per head, else nothing), None (one CTA per head walks its chunks) or a
-    uint8 CUDA tensor.  flags: 0 (the tcgen05 kernel for N = 128, unless a
+    per head -- for N = 128 also only the few pairs past the tcgen05 kernel's
+    last full wave -- else nothing), None (one CTA per head walks its chunks)
+    or a uint8 CUDA tensor.  flags: 0 (the tcgen05 kernel for N = 128, unless a
     workspace is given and the chunk-parallel passes are faster for so few
     (batch, head) pairs) or SSD_FLAG_WARP_MMA (the warp-level kernels).
     Returns (y, last_state)."""

@@ -48,17 +48,21 @@ int launch_ssd(const mss::SsdParams& p, int dstate, cudaStream_t stream);
 
 // The same on the tcgen05 tensor cores (dstate 128; x, z, y, B, C 16-byte
 // aligned).
-int launch_ssd_tc(const mss::SsdParams& p, cudaStream_t stream);
+int launch_ssd_tc(const mss::SsdParams& p, int64_t unit0, int64_t units, cudaStream_t stream);
 
 // The same with every chunk in parallel (three passes) over a workspace of
 // ssd_workspace_bytes (16-byte aligned).
-int launch_ssd_chunked(const mss::SsdParams& p, int dstate, void* workspace, cudaStream_t stream);
+int launch_ssd_chunked(const mss::SsdParams& p, int dstate, void* workspace, int64_t unit0, int64_t units,
+                       cudaStream_t stream);
 int64_t ssd_workspace_bytes(int64_t batch, int64_t seqlen, int64_t nheads, int64_t dstate);
 // Whether the chunk-parallel passes beat the in-order kernel for this many
 // (batch, head) pairs on the current device.
 bool ssd_chunked_pays(int64_t batch, int64_t nheads);
 // The same against the tcgen05 kernel (dstate 128).
 bool ssd_chunked_pays_tc(int64_t batch, int64_t nheads);
+// The pairs past the tcgen05 kernel's last full wave that the chunk-parallel
+// passes should take (0: none).
+int64_t ssd_tc_tail_units(int64_t batch, int64_t nheads);
 
 #define MSS_DECLARE_LAUNCHERS(T, N)                                                                      \
     extern template int launch_forward<T, N>(mss::ScanParams, unsigned, void*, int64_t, cudaStream_t); \

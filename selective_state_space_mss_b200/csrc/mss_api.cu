@@ -469,9 +469,13 @@ int64_t mss_ssd_fwd_workspace_size_ex(int64_t batch, int64_t seqlen, int64_t nhe
     // dstate 128 runs the tcgen05 kernel in order unless the warp-level kernels
     // are asked for, or so few (batch, head) pairs leave most SMs idle that
     // the chunk-parallel passes are faster
-    const bool pays = (dstate == 128 && !(flags & MSS_SSD_FLAG_WARP_MMA)) ? ssd_chunked_pays_tc(batch, nheads)
-                                                                          : ssd_chunked_pays(batch, nheads);
-    return seqlen == 0 || !pays ? 0 : ssd_workspace_bytes(batch, seqlen, nheads, dstate);
+    const bool tc = dstate == 128 && !(flags & MSS_SSD_FLAG_WARP_MMA);
+    if (seqlen == 0) return 0;
+    if (tc ? ssd_chunked_pays_tc(batch, nheads) : ssd_chunked_pays(batch, nheads))
+        return ssd_workspace_bytes(batch, seqlen, nheads, dstate);
+    // or only the pairs past the tcgen05 kernel's last full wave
+    const int64_t tail = tc ? ssd_tc_tail_units(batch, nheads) : 0;
+    return tail > 0 ? ssd_workspace_bytes(1, seqlen, tail, dstate) : 0;
 }
 
 int mss_ssd_fwd_ex(const void* x, const void* dt, const float* A, const void* B, const void* C, const float* D,
@@ -533,18 +537,30 @@ int mss_ssd_fwd_ex2(const void* x, const void* dt, const float* A, const void* B
                      softplus_flag ? 1 : 0};
     if (!(p.err = device_error_word())) return MSS_ERR_CUDA;
     const bool tc = dstate == 128 && !(flags & MSS_SSD_FLAG_WARP_MMA);
-    if (workspace && (tc ? ssd_chunked_pays_tc(batch, nheads) : ssd_chunked_pays(batch, nheads))) {
-        const int64_t need = ssd_workspace_bytes(batch, seqlen, nheads, dstate);
+    const int64_t pairs = batch * nheads;
+    // with a workspace: every pair on the chunk-parallel passes where they
+    // pay, or (tcgen05 kernel) only the pairs past its last full wave
+    int64_t chunked0 = pairs;  // the first pair the passes take
+    if (workspace) {
+        if (tc ? ssd_chunked_pays_tc(batch, nheads) : ssd_chunked_pays(batch, nheads))
+            chunked0 = 0;
+        else if (tc)
+            chunked0 = pairs - ssd_tc_tail_units(batch, nheads);
+    }
+    if (chunked0 < pairs) {
+        const int64_t need = ssd_workspace_bytes(1, seqlen, pairs - chunked0, dstate);
         if (need > workspace_bytes || !aligned(workspace, 16)) return MSS_ERR_WORKSPACE;
         const Range ws{workspace, workspace_bytes};
         for (const Range& r : ins)
             if (overlaps(ws.p, ws.n, r.p, r.n)) return MSS_ERR_ALIAS;
         for (const Range& o : outs)
             if (overlaps(ws.p, ws.n, o.p, o.n)) return MSS_ERR_ALIAS;
-        return launch_ssd_chunked(p, int(dstate), workspace, s);
     }
-    if (tc) return launch_ssd_tc(p, s);
-    return launch_ssd(p, int(dstate), s);
+    if (chunked0 > 0) {
+        const int rc = tc ? launch_ssd_tc(p, 0, chunked0, s) : launch_ssd(p, int(dstate), s);
+        if (rc != MSS_OK || chunked0 == pairs) return rc;
+    }
+    return launch_ssd_chunked(p, int(dstate), workspace, chunked0, pairs - chunked0, s);
 }
 
 int mss_get_device_error(void* stream) {

@@ -46,21 +46,23 @@ bool encode_token_major(CUtensorMap* m, const void* base, int64_t batch, int64_t
 }
 
 template <bool kGate, bool kSoftplus>
-int launch_ssd_tc_variant(const mss::SsdTcMaps& maps, const mss::SsdParams& p, cudaStream_t s) {
+int launch_ssd_tc_variant(const mss::SsdTcMaps& maps, const mss::SsdParams& p, int64_t unit0, int64_t units,
+                          cudaStream_t s) {
     using Ly = mss::SsdTcLayout;
     auto kern = mss::ssd_tc_kernel<kGate, kSoftplus>;
     if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, Ly::kSmemBytes) != cudaSuccess)
         return MSS_ERR_CUDA;
-    const int64_t blocks = p.batch * p.nheads;
-    if (blocks > 0x7fffffffLL) return MSS_ERR_SHAPE;
-    kern<<<dim3(unsigned(blocks)), Ly::kThreads, Ly::kSmemBytes, s>>>(maps, p);
+    if (units <= 0) return MSS_OK;
+    if (units > 0x7fffffffLL) return MSS_ERR_SHAPE;
+    kern<<<dim3(unsigned(units)), Ly::kThreads, Ly::kSmemBytes, s>>>(maps, p, unit0);
     return launch_status();
 }
 
 }  // namespace
 
-// The tcgen05 kernel (dstate 128, headdim 64).
-int launch_ssd_tc(const mss::SsdParams& p, cudaStream_t s) {
+// The tcgen05 kernel (dstate 128, headdim 64) on (batch, head) pairs
+// unit0 .. unit0 + units - 1.
+int launch_ssd_tc(const mss::SsdParams& p, int64_t unit0, int64_t units, cudaStream_t s) {
     if (p.batch > 0x7fffffffLL || p.seqlen > 0x7fffffffLL || p.nheads > 0x7fffffffLL) return MSS_ERR_SHAPE;
     mss::SsdTcMaps maps;
     std::memset(&maps, 0, sizeof(maps));
@@ -69,8 +71,10 @@ int launch_ssd_tc(const mss::SsdParams& p, cudaStream_t s) {
         !encode_token_major(&maps.C, p.C, p.batch, p.seqlen, p.ngroups, 128))
         return MSS_ERR_CUDA;
     if (p.z)
-        return p.softplus ? launch_ssd_tc_variant<true, true>(maps, p, s) : launch_ssd_tc_variant<true, false>(maps, p, s);
-    return p.softplus ? launch_ssd_tc_variant<false, true>(maps, p, s) : launch_ssd_tc_variant<false, false>(maps, p, s);
+        return p.softplus ? launch_ssd_tc_variant<true, true>(maps, p, unit0, units, s)
+                          : launch_ssd_tc_variant<true, false>(maps, p, unit0, units, s);
+    return p.softplus ? launch_ssd_tc_variant<false, true>(maps, p, unit0, units, s)
+                      : launch_ssd_tc_variant<false, false>(maps, p, unit0, units, s);
 }
 
 template <int NS, bool kGate, bool kSoftplus>
@@ -144,10 +148,12 @@ int64_t ssd_workspace_bytes(int64_t batch, int64_t seqlen, int64_t nheads, int64
 }
 
 template <int NS, bool kGate, bool kSoftplus>
-int launch_ssd_chunked_variant(const mss::SsdParams& p, void* workspace, cudaStream_t s) {
+int launch_ssd_chunked_variant(const mss::SsdParams& p, void* workspace, int64_t unit0, int64_t units,
+                               cudaStream_t s) {
     using CL = mss::SsdChunkLayout<NS>;
-    const int64_t nc = (p.seqlen + 63) / 64, bh = p.batch * p.nheads;
-    if (nc > 0x7fffffffLL || p.nheads > 65535 || p.batch > 65535 || bh > 0x7fffffffLL) return MSS_ERR_SHAPE;
+    const int64_t nc = (p.seqlen + 63) / 64, bh = units;
+    if (units <= 0) return MSS_OK;
+    if (nc > 0x7fffffffLL || units > 65535) return MSS_ERR_SHAPE;
     float* Sl = static_cast<float*>(workspace);
     mss::bf16_t* Sin = reinterpret_cast<mss::bf16_t*>(Sl + bh * nc * NS * 64);
     float* decay = reinterpret_cast<float*>(Sin + bh * nc * NS * 64);
@@ -156,28 +162,52 @@ int launch_ssd_chunked_variant(const mss::SsdParams& p, void* workspace, cudaStr
     if (cudaFuncSetAttribute(k1, cudaFuncAttributeMaxDynamicSharedMemorySize, CL::kSmemBytes) != cudaSuccess ||
         cudaFuncSetAttribute(k3, cudaFuncAttributeMaxDynamicSharedMemorySize, CL::kSmemBytes) != cudaSuccess)
         return MSS_ERR_CUDA;
-    const dim3 grid(unsigned(nc), unsigned(p.nheads), unsigned(p.batch));
-    k1<<<grid, 128, CL::kSmemBytes, s>>>(p, Sl, decay);
+    const dim3 grid{unsigned(nc), unsigned(units), 1u};
+    k1<<<grid, 128, CL::kSmemBytes, s>>>(p, Sl, decay, unit0);
     int rc = launch_status();
     if (rc != MSS_OK) return rc;
-    mss::ssd_state_pass_kernel<NS><<<dim3(unsigned(bh), unsigned(NS * 64 / 256)), 256, 0, s>>>(p, Sl, decay, Sin, nc);
+    mss::ssd_state_pass_kernel<NS><<<dim3(unsigned(bh), unsigned(NS * 64 / 256)), 256, 0, s>>>(p, Sl, decay, Sin, nc,
+                                                                                             unit0);
     rc = launch_status();
     if (rc != MSS_OK) return rc;
-    k3<<<grid, 128, CL::kSmemBytes, s>>>(p, Sin);
+    k3<<<grid, 128, CL::kSmemBytes, s>>>(p, Sin, unit0);
     return launch_status();
 }
 
 template <int NS>
-int launch_ssd_chunked_n(const mss::SsdParams& p, void* ws, cudaStream_t s) {
+int launch_ssd_chunked_n(const mss::SsdParams& p, void* ws, int64_t unit0, int64_t units, cudaStream_t s) {
     if (p.z)
-        return p.softplus ? launch_ssd_chunked_variant<NS, true, true>(p, ws, s)
-                          : launch_ssd_chunked_variant<NS, true, false>(p, ws, s);
-    return p.softplus ? launch_ssd_chunked_variant<NS, false, true>(p, ws, s)
-                      : launch_ssd_chunked_variant<NS, false, false>(p, ws, s);
+        return p.softplus ? launch_ssd_chunked_variant<NS, true, true>(p, ws, unit0, units, s)
+                          : launch_ssd_chunked_variant<NS, true, false>(p, ws, unit0, units, s);
+    return p.softplus ? launch_ssd_chunked_variant<NS, false, true>(p, ws, unit0, units, s)
+                      : launch_ssd_chunked_variant<NS, false, false>(p, ws, unit0, units, s);
 }
 
-int launch_ssd_chunked(const mss::SsdParams& p, int dstate, void* workspace, cudaStream_t s) {
-    return dstate == 64 ? launch_ssd_chunked_n<64>(p, workspace, s) : launch_ssd_chunked_n<128>(p, workspace, s);
+// The chunk-parallel passes on (batch, head) pairs unit0 .. unit0 + units - 1;
+// the workspace holds those units' chunk states only.
+int launch_ssd_chunked(const mss::SsdParams& p, int dstate, void* workspace, int64_t unit0, int64_t units,
+                       cudaStream_t s) {
+    return dstate == 64 ? launch_ssd_chunked_n<64>(p, workspace, unit0, units, s)
+                        : launch_ssd_chunked_n<128>(p, workspace, unit0, units, s);
+}
+
+// For the tcgen05 kernel (one CTA per SM): the (batch, head) pairs past the
+// last full wave of CTAs when they are few enough that the chunk-parallel
+// passes finish them clearly sooner than a wave of their own (B200, 4096
+// tokens: 4 past a wave, 160 against 226 us; 12 past, 201-205 against
+// 255 us; 28 past, 238 against 226 us): at most one in nine SMs' worth,
+// 16 pairs on 148 SMs; 0 otherwise.
+int64_t ssd_tc_tail_units(int64_t batch, int64_t nheads) {
+    static std::mutex mu;
+    static int cache[kMaxDevices] = {};
+    const int64_t sms = per_device(cache, mu, [](int dev) {
+        int n = 0;
+        return cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) == cudaSuccess ? n : 0;
+    });
+    const int64_t pairs = batch * nheads;
+    if (sms <= 0 || pairs <= sms) return 0;
+    const int64_t tail = pairs % sms;
+    return tail > 0 && tail * 9 <= sms ? tail : 0;
 }
 
 }  // namespace mss_host

@@ -93,10 +93,11 @@ __device__ __forceinline__ void ssd_load_rows(const SsdParams& p, int64_t b, int
     cp_async_commit();
 }
 
-// Pass 1.  grid = (n_chunks, nheads, batch), block = 128.
-// Sl: [batch][nheads][n_chunks][NS][P] fp32; decay: [batch][nheads][n_chunks].
+// Pass 1.  grid = (n_chunks, units), block = 128: (batch, head) pairs
+// unit0 .. unit0 + units - 1 (pair u = batch index * nheads + head).
+// Sl: [units][n_chunks][NS][P] fp32; decay: [units][n_chunks].
 template <int NS, bool kSoftplus>
-__global__ void __launch_bounds__(128) ssd_chunk_state_kernel(SsdParams p, float* Sl, float* decay) {
+__global__ void __launch_bounds__(128) ssd_chunk_state_kernel(SsdParams p, float* Sl, float* decay, int64_t unit0) {
     using Ly = SsdLayout<NS>;
     using CL = SsdChunkLayout<NS>;
     constexpr int Q = Ly::kQ, P = Ly::kP, MS = NS / 64;
@@ -107,8 +108,9 @@ __global__ void __launch_bounds__(128) ssd_chunk_state_kernel(SsdParams p, float
     float* dts = reinterpret_cast<float*>(smem + CL::kScal);
     float* css = dts + Q;
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31, gq = lane >> 2, tq = lane & 3;
-    const int64_t c = blockIdx.x, h = blockIdx.y, b = blockIdx.z;
-    const int64_t H = p.nheads, L = p.seqlen, n_chunks = gridDim.x;
+    // (batch, head) unit unit0 + blockIdx.y; the workspace holds this launch's units only
+    const int64_t c = blockIdx.x, ul = blockIdx.y, H = p.nheads, L = p.seqlen, n_chunks = gridDim.x;
+    const int64_t h = (unit0 + ul) % H, b = (unit0 + ul) / H;
     const int64_t g = h / (H / p.ngroups);
     const int64_t t0 = c * Q;
     const int q = int(min(int64_t(Q), L - t0));
@@ -148,7 +150,7 @@ __global__ void __launch_bounds__(128) ssd_chunk_state_kernel(SsdParams p, float
             }
         }
     }
-    float* out = Sl + (((b * H + h) * n_chunks + c) * NS) * P;
+    float* out = Sl + ((ul * n_chunks + c) * NS) * P;
 #pragma unroll
     for (int m = 0; m < MS; ++m)
 #pragma unroll
@@ -158,21 +160,21 @@ __global__ void __launch_bounds__(128) ssd_chunk_state_kernel(SsdParams p, float
                 const int n = (warp * MS + m) * 16 + gq + hr * 8, pc = pt * 8 + 2 * tq;
                 *reinterpret_cast<float2*>(out + n * P + pc) = make_float2(s[m][pt][2 * hr], s[m][pt][2 * hr + 1]);
             }
-    if (tid == 0) decay[(b * H + h) * n_chunks + c] = __expf(cs_last);
+    if (tid == 0) decay[ul * n_chunks + c] = __expf(cs_last);
 }
 
-// Pass 2.  grid = (batch * nheads, NS * P / 256), block = 256: one state
-// element per thread, the chunks in order.  Sin: [batch][nheads][n_chunks][NS][P] bf16.
+// Pass 2.  grid = (units, NS * P / 256), block = 256: one state element per
+// thread, the chunks in order.  Sin: [units][n_chunks][NS][P] bf16.
 template <int NS>
 __global__ void __launch_bounds__(256) ssd_state_pass_kernel(SsdParams p, const float* Sl, const float* decay,
-                                                             bf16_t* Sin, int64_t n_chunks) {
+                                                             bf16_t* Sin, int64_t n_chunks, int64_t unit0) {
     constexpr int P = SsdLayout<NS>::kP;
-    const int64_t bh = blockIdx.x;
+    const int64_t ul = blockIdx.x, bh = unit0 + ul;  // the launch's unit, the (batch, head) pair
     const int e = blockIdx.y * 256 + threadIdx.x;  // n * P + p
     float S = p.initial_state ? p.initial_state[bh * NS * P + e] : 0.f;
-    const float* sl = Sl + bh * n_chunks * NS * P + e;
-    const float* dc = decay + bh * n_chunks;
-    bf16_t* si = Sin + bh * n_chunks * NS * P + e;
+    const float* sl = Sl + ul * n_chunks * NS * P + e;
+    const float* dc = decay + ul * n_chunks;
+    bf16_t* si = Sin + ul * n_chunks * NS * P + e;
     for (int64_t c = 0; c < n_chunks; ++c) {
         si[c * NS * P] = from_f32<bf16_t>(S);
         S = fmaf(dc[c], S, sl[c * NS * P]);
@@ -180,9 +182,9 @@ __global__ void __launch_bounds__(256) ssd_state_pass_kernel(SsdParams p, const 
     if (p.last_state) p.last_state[bh * NS * P + e] = S;
 }
 
-// Pass 3.  grid = (n_chunks, nheads, batch), block = 128.
+// Pass 3.  grid = (n_chunks, units), block = 128.
 template <int NS, bool kGate, bool kSoftplus>
-__global__ void __launch_bounds__(128) ssd_chunk_out_kernel(SsdParams p, const bf16_t* Sin) {
+__global__ void __launch_bounds__(128) ssd_chunk_out_kernel(SsdParams p, const bf16_t* Sin, int64_t unit0) {
     using Ly = SsdLayout<NS>;
     using CL = SsdChunkLayout<NS>;
     constexpr int Q = Ly::kQ, P = Ly::kP;
@@ -194,8 +196,9 @@ __global__ void __launch_bounds__(128) ssd_chunk_out_kernel(SsdParams p, const b
     float* dts = reinterpret_cast<float*>(smem + CL::kScal);
     float* css = dts + Q;
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31, gq = lane >> 2, tq = lane & 3;
-    const int64_t c = blockIdx.x, h = blockIdx.y, b = blockIdx.z;
-    const int64_t H = p.nheads, L = p.seqlen, n_chunks = gridDim.x;
+    // (batch, head) unit unit0 + blockIdx.y; the workspace holds this launch's units only
+    const int64_t c = blockIdx.x, ul = blockIdx.y, H = p.nheads, L = p.seqlen, n_chunks = gridDim.x;
+    const int64_t h = (unit0 + ul) % H, b = (unit0 + ul) / H;
     const int64_t g = h / (H / p.ngroups);
     const int64_t t0 = c * Q;
     const int q = int(min(int64_t(Q), L - t0));
@@ -203,7 +206,7 @@ __global__ void __launch_bounds__(128) ssd_chunk_out_kernel(SsdParams p, const b
     ssd_load_rows<NS>(p, b, h, g, t0, q, Xs, Bs, Cs, tid);
     {
         // the state entering the chunk, [n][p] bf16 into padded rows
-        const bf16_t* si = Sin + (((b * H + h) * n_chunks + c) * NS) * P;
+        const bf16_t* si = Sin + ((ul * n_chunks + c) * NS) * P;
         for (int i = tid; i < NS * (P / 8); i += 128) {
             const int r = i / (P / 8), k8 = i % (P / 8);
             cp_async16(Ss + r * Ly::kSStride + k8 * 8, si + r * P + k8 * 8, 16u);

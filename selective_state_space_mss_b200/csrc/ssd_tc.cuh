@@ -98,7 +98,8 @@ struct SsdTcLayout {
 };
 
 template <bool kGate, bool kSoftplus>
-__global__ void __launch_bounds__(512, 1) ssd_tc_kernel(const __grid_constant__ SsdTcMaps maps, SsdParams p) {
+__global__ void __launch_bounds__(512, 1) ssd_tc_kernel(const __grid_constant__ SsdTcMaps maps, SsdParams p,
+                                                        int64_t unit0) {
     using Ly = SsdTcLayout;
     constexpr int Q = Ly::kQ, P = Ly::kP, NS = Ly::kN;
     extern __shared__ __align__(16) uint8_t smem_raw[];
@@ -127,7 +128,8 @@ __global__ void __launch_bounds__(512, 1) ssd_tc_kernel(const __grid_constant__ 
     // one that issues everything else
     const bool scorer = tid == kScoreWarp * 32;
     const int64_t H = p.nheads, L = p.seqlen;
-    const int64_t b = blockIdx.x / H, h = blockIdx.x % H;
+    // (batch, head) pair unit0 + blockIdx.x
+    const int64_t b = (unit0 + blockIdx.x) / H, h = (unit0 + blockIdx.x) % H;
     const int g = int(h / (H / p.ngroups));
     const float A2 = p.A[h] * kLog2e;
     const float bias = p.dt_bias ? p.dt_bias[h] : 0.f;

@@ -186,3 +186,28 @@ def test_ssd_second_workload_sampled_heads(kernel):
                                          dt_bias=inp["dt_bias"][h:h + 1])
         assert_close(yn[b:b + 1, :, h:h + 1], y_ref, "bf16", f"y of (b={b}, h={h})")
         assert_close(ln[b:b + 1, h:h + 1], last_ref, "bf16", f"state of (b={b}, h={h})")
+
+
+@pytest.mark.parametrize("extra", [0, 5, 30], ids=["whole-waves", "short-tail", "long-tail"])
+def test_ssd_tail_past_the_last_wave(extra):
+    """N = 128 with a workspace: (batch, head) pairs past the tcgen05
+    kernel's last full wave of CTAs (one per SM) go to the chunk-parallel
+    passes when they are few; whole waves, or a long tail, stay on the
+    tcgen05 kernel.  Each against the oracle, with a starting state."""
+    sms = torch.cuda.get_device_properties(0).multi_processor_count
+    H = sms + extra
+    lib = mss.load_library()
+    ws = lib.mss_ssd_fwd_workspace_size(1, 256, H, 64, 1, 128)
+    if extra == 5:
+        # the chunk states of the 5 tail pairs only
+        assert ws == lib.mss_ssd_fwd_workspace_size_ex(1, 256, 5, 64, 1, 128, mss.SSD_FLAG_WARP_MMA) > 0
+    else:
+        assert ws == 0
+    inp = gen.ssd_inputs(1, 256, H, 64, 1, 128, seed=740 + extra)
+    h0 = np.random.default_rng(741).standard_normal((1, H, 128, 64)).astype(np.float32) * 0.1
+    y, last = mss.ssd_fwd(**_dev(inp), initial_state=torch.from_numpy(h0).to(DEV), workspace="auto")
+    torch.cuda.synchronize()
+    assert mss.get_device_error() == 0
+    y_ref, last_ref = _ref(inp, h0=h0.astype(np.float64))
+    assert_close(to_numpy(y), y_ref, "bf16", f"{extra} past the wave: y")
+    assert_close(to_numpy(last), last_ref, "bf16", f"{extra} past the wave: last_state")
