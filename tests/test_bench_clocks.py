@@ -56,3 +56,19 @@ def test_nvml_sampler_no_reasons_and_uuid_devices(monkeypatch):
 
 def test_nvml_sampler_without_nvml_has_no_samples(monkeypatch):
     assert _sample(monkeypatch, _fake_nvml([1965], 0, fail_init=True)) is None
+
+
+def test_nvml_sampler_summary_starts_at_the_mark(monkeypatch):
+    # idle clocks while the sampler starts and the warm-up runs, load clocks
+    # after the mark: only the latter count
+    clocks = [300] * 20 + [1965] * 10000
+    monkeypatch.setitem(sys.modules, "pynvml", _fake_nvml(clocks, 0))
+    s = bench.NvmlSampler("0", period_s=0.001)
+    with s:
+        while len(s.rows) < 25:
+            time.sleep(0.001)
+        s.mark()
+        time.sleep(0.03)
+    out = s.summary()
+    assert out["sm_mhz"] == 1965 and out["samples"] >= 1
+    assert all(r[0] == 1965 for r in s.rows[s._first:])
